@@ -1,0 +1,439 @@
+"""Benchmark of the e-means hot path on B200 (one JSON line on stdout).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload emb768] [--impl ours|reference]
+
+A step is one mini-batch step of training: gather in the per-pass order, fused
+nearest-centroid search, grouping by label with segmented sums and the EMA
+update, and every 5th step the revival check (runs restart with a fresh begin
+when they end, finalize included). `value` is points assigned per second over the
+K timed steps with the training matrix resident in HBM (fp32, cast to the bf16
+search copy inside each begin). Under torchrun every rank trains its own replica
+on its own GPU (no data-path collective); the time is the max over ranks.
+
+Extra keys: roofline (the assignment kernel against the measured bf16 peak, from
+CUDA events around every assignment launch inside the timed region), e2e (the same
+metric through em_train with a pinned host matrix: host->device copy, training,
+centroid read-back), cpu_baseline (the fp64 oracle on a bounded sample, rank 0 at
+N = 1), lloyd25 (wall-clock and epochs to the test MSE of 25 Lloyd iterations).
+--impl reference times the fp64 oracle on the host cores instead.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "pts assigned/s & wall-clock to Lloyd-25 test MSE, 1M×768 k=4096, 1×B200"
+UNIT = "pts/s"
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def workload_desc(w):
+    return (f"{w.name}: n={w.n_train:,} train + {w.n_test:,} test, d={w.d}, k={w.k:,}, {w.epochs:g} epochs, "
+            f"{w.storage} storage / bf16 search; {w.recipe}")
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if not self.proc:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        time.sleep(0.2)
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- the fp64 oracle on the host
+
+def oracle_sample_rate(w, xt_dev, seconds, rows_per_step=None, log_prefix="cpu"):
+    """Times oracle mini-batch steps (search + statistics + EMA update) on the
+    first batches of pass 0, copied to the host. Returns (pts/s, sample text, threads)."""
+    import numpy as np
+    from threadpoolctl import threadpool_info
+
+    from oracle import emeans_oracle as O
+
+    rec = O.recipe(w.n_train, w.k, w.epochs)
+    B = rec["batch_size"] if rows_per_step is None else int(rows_per_step)
+    order = O.pass_order(w.n_train, 1234, 0)
+    start_rows = O.starting_rows(w.n_train, w.k, 1234)
+    import torch
+
+    idx = torch.from_numpy(start_rows).to(xt_dev.device)
+    c = O.search_copy_of_data(xt_dev.index_select(0, idx).float().cpu().numpy())
+    N = np.zeros(w.k)
+    S = np.zeros((w.k, w.d))
+    t_total, rows_total, steps = 0.0, 0, 0
+    while t_total < seconds and steps < rec["total_steps"]:
+        ids = torch.from_numpy(order[steps * B:(steps + 1) * B]).to(xt_dev.device)
+        xb = O.search_copy_of_data(xt_dev.index_select(0, ids).float().cpu().numpy())
+        t0 = time.perf_counter()
+        labels, _, _ = O.assign(xb, O.search_copy_of_centroids(c))
+        n_j, s_j = O.batch_stats(xb, labels, w.k)
+        N, S, c = O.ema_update(N, S, c, n_j, s_j, O.alpha_at(steps, rec["total_steps"], rec["alpha0"]))
+        t_total += time.perf_counter() - t0
+        rows_total += len(xb)
+        steps += 1
+        log(f"[{log_prefix}] oracle step {steps}: {len(xb)} rows, {t_total:.1f} s so far")
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    sample = (f"{steps} oracle steps of {B} rows each (search against all {w.k} centroids, per-cluster sums, "
+              f"EMA update) from pass 0 of {w.name}; {t_total:.1f} s of host time")
+    return rows_total / t_total, sample, threads
+
+
+# ---------------------------------------------------------------- our arm
+
+def run_ours(args, rank, world):
+    import torch
+
+    import datagen
+    import mini_ema_means_b200 as em
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    peaks = measured_peaks()
+    t0 = time.time()
+    w, xt, xs = datagen.make(args.workload, device=dev, seed=0)
+    torch.cuda.synchronize()
+    log(f"[rank {rank}] data {w.name} ready in {time.time() - t0:.1f} s")
+    stream = torch.cuda.current_stream(dev)
+    m = em.Model(w.d, w.k, seed=1234)
+    m.set_stream(stream.cuda_stream)
+    m.set_option("input_dtype", 1 if w.storage == "bf16" else 0)
+    rec = m.begin(xt, epochs=w.epochs)
+    total = rec["total_steps"]
+
+    # bookkeeping without synchronising: steps left in the current run on the host side
+    state = {"in_run": 0}
+
+    def steps_loop(K):
+        done = 0
+        rows = 0
+        B = rec["batch_size"]
+        full = rec["steps_full_pass"]
+        while done < K:
+            left = total - state["in_run"]
+            take = min(left, K - done)
+            m.step(take)
+            for s in range(state["in_run"], state["in_run"] + take):
+                p = s // full
+                in_pass = s - p * full
+                rows_pass = rec["rows_last_pass"] if p == rec["passes"] - 1 else w.n_train
+                rows += min(B, rows_pass - in_pass * B)
+            state["in_run"] += take
+            done += take
+            if state["in_run"] >= total:
+                m.finalize()
+                m.begin(xt, epochs=w.epochs)
+                state["in_run"] = 0
+        return rows
+
+    # warm-up (untimed)
+    steps_loop(args.warmup)
+    torch.cuda.synchronize()
+    m.finalize()
+    m.begin(xt, epochs=w.epochs)
+    state["in_run"] = 0
+    m.set_option("profile", 1)
+    m.profile(reset=True)
+    sampler = ClockSampler(dev.index)
+    sampler.start()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    rows = steps_loop(args.steps)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    clocks = sampler.stop()
+    ms = e0.elapsed_time(e1)
+    prof = m.profile(reset=True)
+    m.set_option("profile", 0)
+    ms_max = ms
+    rows_all = rows
+    if world > 1:
+        t = torch.tensor([ms], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms_max = float(t.item())
+        r = torch.tensor([rows], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(r)
+        rows_all = int(r.item())
+    value = rows_all / (ms_max / 1e3)
+    out = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": workload_desc(w), "batch_size": rec["batch_size"], "alpha0": round(rec["alpha0"], 6),
+                   "steps_per_run": total,
+                   "l2": "inputs larger than L2: the fp32 training matrix (%.2f GB) and its bf16 copy are re-read "
+                         "in a fresh random order every pass" % (w.n_train * w.d * 4 / 1e9),
+                   "parallelism": "replicas" if world > 1 else "single GPU"},
+    }
+    # roofline of the dominant kernel: the fused assignment (tensor-core bound)
+    a_ms = prof["ms"]["assign"]
+    a_n = max(prof["spans"]["assign"], 1)
+    achieved = prof["assign_flops"] / (a_ms / 1e3) / 1e12 if a_ms > 0 else 0.0
+    peak = peaks["bf16_tflops"]
+    out["roofline"] = {
+        "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+        "frac": achieved / peak, "traffic": args.traffic,
+        "kernel": "k_assign_tc (tcgen05 bf16 x bf16 -> fp32, fused |c|^2 add + row argmin)",
+        "peak_source": f"{peaks['source']} bf16 burst",
+        "frac_of_sustained": achieved / peaks["bf16_tflops_sustained"] if peaks.get("bf16_tflops_sustained") else None,
+        "avg_launch_ms": a_ms / a_n,
+        "launches": prof["spans"]["assign"],
+    }
+    u_ms = prof["ms"]["update"]
+    out["phases_ms"] = {k: round(v, 4) for k, v in prof["ms"].items()}
+    out["update_roofline"] = {
+        "bound": "hbm", "achieved": prof["update_bytes"] / (u_ms / 1e3) / 1e9 if u_ms > 0 else 0.0,
+        "peak": peaks["hbm_gbs"], "unit": "GB/s",
+        "frac": (prof["update_bytes"] / (u_ms / 1e3) / 1e9) / peaks["hbm_gbs"] if u_ms > 0 else 0.0,
+    }
+    out["gpu_launches"] = prof["launches"]
+    out["clocks"] = clocks
+
+    if rank == 0 and not args.no_extras:
+        out["lloyd25"] = lloyd25(m, w, xt, xs, rec)
+    if not args.no_e2e:
+        out["e2e"] = e2e(em, w, xt, stream, world, dev)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, sample, threads = oracle_sample_rate(w, xt, args.cpu_seconds)
+        out["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample}
+    m.close()
+    return out
+
+
+def lloyd25(m, w, xt, xs, rec):
+    """Test MSE of 25 Lloyd iterations from the same starting rows, then the first
+    e-means checkpoint (every ceil(S/20) steps and at pass ends; evaluation time
+    excluded) whose test MSE is at or below it."""
+    import torch
+
+    t0 = time.time()
+    m.lloyd(xt, 25)
+    target = m.mse(xs)
+    lloyd_s = time.time() - t0
+    total = rec["total_steps"]
+    every = math.ceil(total / 20)
+    full = rec["steps_full_pass"]
+    m.begin(xt, epochs=w.epochs)
+    stream = torch.cuda.current_stream()
+    train_ms, steps, hit = 0.0, 0, None
+    history = []
+    while steps < total:
+        nxt = min(total, (steps // every + 1) * every, (steps // full + 1) * full)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        m.step(nxt - steps)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        train_ms += e0.elapsed_time(e1)
+        steps = nxt
+        mse = m.mse(xs)
+        epochs = steps / full
+        history.append((round(epochs, 4), mse))
+        if hit is None and mse <= target:
+            hit = {"seconds": train_ms / 1e3, "epochs": epochs, "test_mse": mse}
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    m.finalize()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    train_ms += e0.elapsed_time(e1)
+    final = m.mse(xs)
+    if hit is None and final <= target:
+        hit = {"seconds": train_ms / 1e3, "epochs": w.epochs, "test_mse": final}
+    return {"lloyd25_test_mse": target, "lloyd25_wall_s": lloyd_s, "emeans_final_test_mse": final,
+            "emeans_train_s": train_ms / 1e3, "reached": hit is not None,
+            "time_to_target_s": hit["seconds"] if hit else None, "epochs_to_target": hit["epochs"] if hit else None,
+            "final_ratio": final / target, "checkpoints": history}
+
+
+def e2e(em, w, xt, stream, world, dev):
+    """em_train through the C ABI with a pinned host matrix: H2D copy, training and
+    the centroid read-back inside the timed region."""
+    import torch
+
+    xh = xt.cpu().pin_memory()
+    m = em.Model(w.d, w.k, seed=1234)
+    m.set_stream(stream.cuda_stream)
+    cent = torch.empty(w.k, w.d).pin_memory()
+    m.train(xh, epochs=w.epochs)  # warm-up run
+    m.centroids(cent)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    m.train(xh, epochs=w.epochs)
+    m.centroids(cent)
+    torch.cuda.synchronize()
+    sec = time.perf_counter() - t0
+    r = m.recipe()
+    rows = w.n_train * w.epochs
+    if world > 1:
+        t = torch.tensor([sec], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        sec = float(t.item())
+        rows *= world
+    m.close()
+    steps = r["total_steps"]
+    return {"value": rows / sec, "unit": UNIT,
+            "h2d_bytes_per_step": xh.numel() * xh.element_size() / steps,
+            "d2h_bytes_per_step": (w.k * w.d * 4) / steps,
+            "what": "em_train on a pinned host fp32 matrix (copied to the device inside the call) + centroid "
+                    "read-back, one whole 5-epoch run, host wall clock"}
+
+
+# ---------------------------------------------------------------- reference arm (the oracle)
+
+def run_reference(args):
+    import torch
+
+    import datagen
+
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    w, xt, _ = datagen.make(args.workload, device=dev, seed=0)
+    budget = args.ref_seconds
+    # calibrate the rows of one step so that warm-up + timed steps fit the budget
+    v0, _, _ = oracle_sample_rate(w, xt, 0.1, rows_per_step=512, log_prefix="ref-calibrate")
+    rows = int(max(64, min(65536, v0 * budget / max(args.steps + args.warmup, 1))))
+    import numpy as np
+    from threadpoolctl import threadpool_info
+
+    from oracle import emeans_oracle as O
+
+    rec = O.recipe(w.n_train, w.k, w.epochs)
+    order = O.pass_order(w.n_train, 1234, 0)
+    start = O.starting_rows(w.n_train, w.k, 1234)
+    c = O.search_copy_of_data(xt.index_select(0, torch.from_numpy(start).to(xt.device)).float().cpu().numpy())
+    N, S = np.zeros(w.k), np.zeros((w.k, w.d))
+
+    def one(t):
+        nonlocal N, S, c
+        ids = order[(t * rows) % (w.n_train - rows):][:rows]
+        xb = O.search_copy_of_data(xt.index_select(0, torch.from_numpy(ids).to(xt.device)).float().cpu().numpy())
+        t0 = time.perf_counter()
+        labels, _, _ = O.assign(xb, O.search_copy_of_centroids(c))
+        n_j, s_j = O.batch_stats(xb, labels, w.k)
+        N, S, c = O.ema_update(N, S, c, n_j, s_j, O.alpha_at(t, rec["total_steps"], rec["alpha0"]))
+        return time.perf_counter() - t0
+
+    for t in range(args.warmup):
+        one(t)
+    sec = sum(one(args.warmup + t) for t in range(args.steps))
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    value = args.steps * rows / sec
+    sample = (f"{args.steps} oracle steps of {rows} rows each from pass 0 of {w.name} (search against all "
+              f"{w.k} centroids, per-cluster sums, EMA update)")
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": sec * 1e3 / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": workload_desc(w), "parallelism": "host cores"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2400)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="emb768")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--ref-seconds", type=float, default=120.0)
+    ap.add_argument("--traffic", type=float, default=None,
+                    help="dram bytes per assignment launch from an ncu capture of the current kernel")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        print(json.dumps(run_reference(args)), flush=True)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
+    try:
+        out = run_ours(args, rank, world)
+        if rank == 0:
+            print(json.dumps(out), flush=True)
+    finally:
+        if world > 1:
+            import torch
+
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

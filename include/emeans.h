@@ -1,0 +1,255 @@
+/*
+ * emeans.h -- C ABI of the B200 e-means library (mini-batch EMA k-means).
+ *
+ * The method and its interface are those of the faiss e-means README
+ * ("e-means: outperforming k-means in one-tenth the epochs"): the model is
+ * built from (d, k, seed) as in its section "Settings and results"
+ * (`Emeans(d, k, nepochs=5, seed=1234)`), trained with `train(x)` and queried
+ * with `assign(x)`; the manual loop of its section "Data too big for memory"
+ * (begin / accumulate+update / end_epoch / finalize) is exposed as
+ * em_begin / em_step / em_finalize.
+ *
+ * Conventions shared by every entry point
+ *  - Return value: EM_OK (0) on success, a negative EM_E_* code on failure.
+ *    em_last_error() then returns a message for the calling thread.
+ *  - Matrices are row-major, rows contiguous: X is n x d, centroids k x d.
+ *  - Pointers may be host or device memory (CUDA unified addressing is used
+ *    to tell them apart). Host input is copied to the device inside the call;
+ *    host output is written after the device work of the call has finished.
+ *    Device pointers must belong to the model's device. Pointers are never
+ *    retained after a call returns, except the X given to em_begin (see there).
+ *  - All device work is ordered on the model's stream (em_set_stream; by
+ *    default a stream the model creates). Calls that return data to a host
+ *    pointer synchronise that stream; the others do not.
+ *  - Nothing is checked for NaN or infinity unless EM_OPT_CHECK_FINITE is set
+ *    (the README, section "Data and centroids fit on 1 GPU", documents the GPU
+ *    path as unchecked).
+ *  - There is no CPU fallback: without a CUDA device every compute entry point
+ *    fails with EM_E_NODEVICE.
+ */
+#ifndef EMEANS_H
+#define EMEANS_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes ---- */
+#define EM_OK 0
+#define EM_E_INVAL (-1)     /* bad argument (sizes, pointers, option values)          */
+#define EM_E_NOMEM (-2)     /* device or pinned-host allocation failed                */
+#define EM_E_CUDA (-3)      /* a CUDA runtime call failed                             */
+#define EM_E_BOUNDS (-4)    /* a kernel's own index check caught an out-of-range index */
+#define EM_E_TIMEOUT (-5)   /* a bounded device-side wait gave up                     */
+#define EM_E_NONFINITE (-6) /* EM_OPT_CHECK_FINITE found NaN or infinity in the input */
+#define EM_E_STATE (-7)     /* call out of order (e.g. em_step before em_begin)       */
+#define EM_E_NODEVICE (-8)  /* no CUDA device is present                              */
+
+/* ---- options (em_set_option / em_get_option; values are doubles) ---- */
+enum em_option {
+    EM_OPT_BATCH_SIZE = 1,       /* 0 (default): from the scaling law; else the batch size,
+                                    and alpha0 follows equation (3) (README "Manual overrides") */
+    EM_OPT_ALPHA0 = 2,           /* 0 (default): from equation (3); else the starting step    */
+    EM_OPT_UNUSED_THRESHOLD = 3, /* tau: revive clusters whose running count is below tau x the
+                                    mean count (README `unused_threshold`). Default 0.1; 0 = off */
+    EM_OPT_REVIVAL = 4,          /* 0 none, 1 split a size-proportional donor (default),
+                                    2 resample from the current batch                          */
+    EM_OPT_FINALIZE = 5,         /* 1 (default): closing mean at the end of the last pass; 0 off */
+    EM_OPT_LAW = 6,              /* 0 "throughput" law (1), default; 1 "quality" law (2)       */
+    EM_OPT_INPUT_DTYPE = 7,      /* dtype of X: 0 fp32 (default), 1 bf16                       */
+    EM_OPT_CHECK_FINITE = 8,     /* 1: scan X for NaN/Inf in em_begin/em_train (EM_E_NONFINITE) */
+    EM_OPT_WAIT_LIMIT_MS = 9,    /* limit of every device-side spin wait, ms (default 2000)    */
+    EM_OPT_AUTO_REVIVE = 10,     /* 1 (default): em_step runs the revival check after every 5th
+                                    step; 0: only em_revive does (step-by-step inspection)      */
+    EM_OPT_CAPTURE_LABELS = 11,  /* 1 (default): keep each row's last-pass label (em_labels)   */
+    EM_OPT_GRAPHS = 12,          /* 1 (default): em_step replays CUDA graphs of whole steps     */
+    EM_OPT_ASSIGN_KERNEL = 13,   /* 0 (default): tcgen05 tensor-core assignment; 1: a plain
+                                    SIMT kernel kept only to localise faults in tests           */
+    EM_OPT_PROFILE = 14          /* 1: bracket every phase of every step with CUDA events on the
+                                    model's stream (read with em_profile); 0 (default): off     */
+};
+
+/* Phases timed by EM_OPT_PROFILE (em_profile_t.ms / spans index). */
+#define EM_PHASE_PREPARE 0   /* input copy / cast, starting centroids                        */
+#define EM_PHASE_GATHER 1    /* batch gather in the per-pass order                            */
+#define EM_PHASE_ASSIGN 2    /* fused nearest-centroid search                                 */
+#define EM_PHASE_UPDATE 3    /* labels, grouping by label, segmented sums + EMA update        */
+#define EM_PHASE_REVIVE 4    /* dead-cluster revival                                           */
+#define EM_PHASE_FINALIZE 5  /* closing mean                                                   */
+#define EM_NPHASES 6
+
+/* revival modes for EM_OPT_REVIVAL */
+#define EM_REVIVE_NONE 0
+#define EM_REVIVE_SPLIT 1
+#define EM_REVIVE_RESAMPLE 2
+
+/* Training recipe (README "Scaling laws" and "Settings and results": batch_size,
+ * alpha0, steps_per_pass, epoch_rows). Every pass but a fractional last one has n rows. */
+typedef struct em_recipe_t {
+    int64_t n, k, d;
+    double epochs;
+    double batch_raw;        /* equation (1)/(2) before rounding (or the manual size)        */
+    int64_t batch_size;      /* nearest power of two in log2, capped at the largest <= n/2  */
+    double alpha0;           /* equation (3), clamped to [1e-4, 1] (or the manual value)    */
+    int64_t passes;          /* ceil(epochs)                                                  */
+    int64_t rows_last_pass;  /* n, or round(frac(epochs) * n) for a fractional last pass      */
+    int64_t steps_full_pass; /* ceil(n / batch_size)                                          */
+    int64_t steps_last_pass; /* ceil(rows_last_pass / batch_size)                             */
+    int64_t total_steps;     /* sum over passes                                               */
+} em_recipe_t;
+
+/* Counters kept on the model (README "Settings and results": iteration_stats, n_splits). */
+typedef struct em_stats_t {
+    int64_t steps_done;      /* mini-batch steps run since em_begin                          */
+    int64_t passes_done;     /* completed passes                                              */
+    int64_t rows_assigned;   /* rows assigned by training steps since em_begin                */
+    int64_t n_splits;        /* dead clusters revived since em_begin                         */
+    int64_t last_dead;       /* clusters found dead at the most recent revival check          */
+    double imbalance;        /* max(N) / mean(N) after the most recent step                   */
+    double last_alpha;       /* step size of the most recent step                             */
+} em_stats_t;
+
+/* Device time per phase and launch counts (EM_OPT_PROFILE). */
+typedef struct em_profile_t {
+    double ms[EM_NPHASES];      /* summed span durations, CUDA events on the model's stream      */
+    int64_t spans[EM_NPHASES];  /* number of spans timed per phase                               */
+    int64_t launches;           /* kernels launched by the library (counted with or without
+                                   EM_OPT_PROFILE)                                               */
+    double assign_flops;        /* 2 * rows * k * d summed over the timed assignment spans      */
+    double update_bytes;        /* algorithmic bytes of the timed update spans:
+                                   2*rows*d (batch rows) + 16*rows (keys, labels, order)
+                                   + 14*k*d (S read + write, c fp32 and bf16 writes)            */
+    double gather_bytes;        /* 4*rows*d: batch rows read and written (bf16)                  */
+} em_profile_t;
+
+/* ---- library ---- */
+
+/* Message of the last failing call on this thread ("" if none). Never NULL. */
+const char* em_last_error(void);
+
+/* Number of CUDA devices visible to the library (0 without a GPU). Host-only. */
+int em_device_count(void);
+
+/* Host-only helpers that run the library's own host code, for checking it
+ * without a GPU. em_compute_recipe evaluates equations (1)-(3) and the rounding
+ * rules (README "Scaling laws", "Manual overrides"); law 0 = throughput,
+ * 1 = quality; batch_override <= 0 and alpha_override <= 0 mean "from the law". */
+int em_compute_recipe(int64_t n, int64_t k, double epochs, int law, int64_t batch_override,
+                      double alpha_override, em_recipe_t* out);
+
+/* The library's per-pass order: out[i] = pi(idx[i]) for the keyed bijection on
+ * [0, n) selected by (seed, stream, which): stream 1 = starting rows (which = 0),
+ * stream 2 = pass order (which = pass index). Same code as the device kernels. */
+int em_permutation(int64_t n, uint64_t seed, int stream, int64_t which, const int64_t* idx,
+                   int64_t count, int64_t* out);
+
+/* ---- model ---- */
+
+/* New model for k clusters of d-dimensional vectors on the current CUDA device
+ * (README "Settings and results": only d and k are required; seed seeds the
+ * starting centroids, the per-pass order and the revivals; the README default is
+ * 1234). Returns NULL on failure (em_last_error). d in [1, 8192], k >= 1. */
+struct em_model;
+typedef struct em_model em_model;
+em_model* em_create(int64_t d, int64_t k, uint64_t seed);
+
+/* Frees every device and host buffer of the model. NULL is ignored. */
+void em_destroy(em_model* m);
+
+int em_set_option(em_model* m, int opt, double value);
+int em_get_option(const em_model* m, int opt, double* value);
+
+/* Orders all later work of the model on `stream` (a cudaStream_t; NULL = the
+ * legacy default stream). The model does not take ownership. */
+int em_set_stream(em_model* m, void* stream);
+
+/* ---- training (README "Quick start", "Data and centroids fit on 1 GPU") ---- */
+
+/* Trains on X (n x d rows, dtype per EM_OPT_INPUT_DTYPE) for `epochs` passes
+ * (fractional allowed): em_begin + em_step until done + em_finalize. Needs
+ * n >= k. Afterwards em_centroids / em_labels / em_stats / em_obj hold the
+ * results. Synchronises the stream and reports device-side errors. */
+int em_train(em_model* m, const void* X, int64_t n, double epochs);
+
+/* Starts a run: computes the recipe, makes the bf16 search copy of X (fp32 input
+ * is rounded to nearest-even; README "Data precision"), picks k distinct rows as
+ * starting centroids (README: random data points, no k-means++) and zeroes the
+ * running counts and sums. A device bf16 X whose rows are 16-byte aligned
+ * (d % 8 == 0) is used in place and must stay valid and unchanged until the
+ * run ends (em_finalize or the next em_begin); any other X is copied. */
+int em_begin(em_model* m, const void* X, int64_t n, double epochs);
+
+/* Runs up to `nsteps` further mini-batch steps of the run (assignment of the
+ * batch, per-cluster count and sum, EMA update with the cosine step size and,
+ * every 5th step, the revival check; README "How the centroid updates work").
+ * *done (may be NULL) receives the number of steps run. Does not synchronise. */
+int em_step(em_model* m, int64_t nsteps, int64_t* done);
+
+/* Ends the run: applies the closing mean if EM_OPT_FINALIZE is on (each
+ * centroid becomes the exact mean of the rows the last pass assigned to it;
+ * clusters without such rows keep their EMA centroid). Synchronises. */
+int em_finalize(em_model* m);
+
+/* Runs the revival check for the most recent step now (for EM_OPT_AUTO_REVIVE
+ * = 0). The batch of that step is the one resampling draws from. */
+int em_revive(em_model* m);
+
+/* Lloyd's k-means (README "How the centroid updates work": the whole dataset as
+ * one batch with a step of 1) for `iters` iterations, from the same starting
+ * rows em_begin would pick for this seed. Natural row order, no revival. The
+ * centroids are left on the model. */
+int em_lloyd(em_model* m, const void* X, int64_t n, int64_t iters);
+
+/* ---- queries ---- */
+
+/* Nearest centroid of every row of X (README "Settings and results":
+ * `assign` returns each vector's nearest centroid and its squared distance).
+ * labels: n int64 (may be NULL); dists: n fp32 squared distances computed with
+ * the bf16 search copies and clamped at 0 (may be NULL). Ties go to the lowest
+ * centroid index. */
+int em_assign(em_model* m, const void* X, int64_t n, int64_t* labels, float* dists);
+
+/* Mean over the rows of X of the squared distance to the nearest centroid
+ * (fp64 accumulation), as em_assign measures it. Synchronises. */
+int em_mse(em_model* m, const void* X, int64_t n, double* out);
+
+/* Copies the k x d fp32 centroids into out. */
+int em_centroids(const em_model* m, float* out);
+
+/* Copies each training row's label from the last pass (int64; -1 for rows a
+ * fractional last pass did not visit) into out (n entries of the last run). */
+int em_labels(const em_model* m, int64_t* out);
+
+int em_recipe(const em_model* m, em_recipe_t* out);
+int em_stats(const em_model* m, em_stats_t* out);
+
+/* Error of each completed pass, measured while the centroids move (README
+ * `obj`): mean squared distance of the pass's rows at the time they were
+ * assigned. Writes up to cap values; *count receives the number available. */
+int em_obj(const em_model* m, double* out, int64_t cap, int64_t* count);
+
+/* Model state: running counts N (k fp32), running sums S (k x d fp32),
+ * centroids c (k x d fp32) and the global step counter. Any pointer may be
+ * NULL. em_set_state replaces the state of the current run (checkpoint resume,
+ * step-by-step comparison); the bf16 search copy is refreshed from c. */
+int em_get_state(const em_model* m, float* N, float* S, float* c, int64_t* step);
+int em_set_state(em_model* m, const float* N, const float* S, const float* c, int64_t step);
+
+/* The most recent training batch: its row ids (int64), labels (int64), squared
+ * distances (fp32) and row count. Any pointer may be NULL. */
+int em_last_batch(const em_model* m, int64_t* ids, int64_t* labels, float* dists, int64_t* rows);
+
+/* Synchronises the model's stream, adds the pending event spans to the totals and
+ * copies the totals to *out; reset != 0 clears them (and the launch count). */
+int em_profile(em_model* m, em_profile_t* out, int reset);
+
+/* Waits for the model's stream and reports device-side errors (EM_E_BOUNDS,
+ * EM_E_TIMEOUT) raised since the last check. */
+int em_sync(em_model* m);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* EMEANS_H */

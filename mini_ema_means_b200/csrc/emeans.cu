@@ -1,0 +1,1111 @@
+// emeans.cu -- host orchestration and the C ABI of the B200 e-means library.
+//
+// One training step (faiss e-means README, "Data too big for memory": accumulate
+// then update, run by `train` internally) is this kernel sequence on the model's
+// stream:
+//   k_gather        batch rows pi_pass(pos..pos+B) -> contiguous bf16 batch, |x|^2
+//   k_assign_tc     nearest centroid of every batch row (tcgen05 + TMA)
+//   k_labels        labels, distances, per-cluster counts and ranks
+//   k_offsets       segment starts, batch error sum
+//   k_scatter       rows in label order
+//   k_segsum        per-cluster sums (fp64) fused with the EMA update
+//   k_fixup         clusters cut by tile edges, clusters without rows
+//   k_revive_*      every 5th step: dead-cluster revival
+// No host synchronisation happens inside a run; the step size of step t is
+// computed on the host (cosine schedule) and passed by value.
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "common.cuh"
+#include "k_assign.cuh"
+#include "k_data.cuh"
+#include "k_reduce.cuh"
+#include "k_revive.cuh"
+
+using namespace em;
+
+// ------------------------------------------------------------------ errors
+
+static thread_local char g_err[1024] = "";
+
+static int fail(int code, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof(g_err), fmt, ap);
+    va_end(ap);
+    return code;
+}
+
+#define CK(call)                                                                                 \
+    do {                                                                                         \
+        cudaError_t e_ = (call);                                                                 \
+        if (e_ != cudaSuccess) return fail(EM_E_CUDA, "%s: %s", #call, cudaGetErrorString(e_)); \
+    } while (0)
+
+#define CKR(expr)              \
+    do {                       \
+        int r_ = (expr);       \
+        if (r_ != EM_OK) return r_; \
+    } while (0)
+
+// ------------------------------------------------------------------ recipe (host)
+
+static const double kLawConst[2] = {0.035134, 0.00439175};
+
+static int compute_recipe(int64_t n, int64_t k, int64_t d, double epochs, int law, int64_t batch_override,
+                          double alpha_override, em_recipe_t* r) {
+    if (n < 1 || k < 1 || !(epochs > 0.0) || law < 0 || law > 1) return fail(EM_E_INVAL, "bad recipe arguments");
+    memset(r, 0, sizeof(*r));
+    r->n = n;
+    r->k = k;
+    r->d = d;
+    r->epochs = epochs;
+    // equations (1)/(2), nearest power of two in log2, capped at the largest power of two <= n/2
+    int64_t b;
+    if (batch_override > 0) {
+        b = batch_override;
+        r->batch_raw = (double)b;
+    } else {
+        r->batch_raw = kLawConst[law] * pow((double)k, 0.134749) * pow((double)n, 0.876473) * pow(epochs, 0.813344);
+        const double lb = log2(std::max(r->batch_raw, 1.0));
+        const long e = lround(lb);  // halves round away from zero, as Python's round never sees them here
+        b = (int64_t)1 << std::min<long>(e, 62);
+        const double half = std::max((double)n / 2.0, 1.0);
+        const int64_t cap = (int64_t)1 << (int)floor(log2(half));
+        b = std::max<int64_t>(1, std::min(b, cap));
+    }
+    r->batch_size = b;
+    // equation (3), clamped to [1e-4, 1]
+    if (alpha_override > 0.0) {
+        r->alpha0 = alpha_override;
+    } else {
+        double a = 0.8244 * pow((double)k, -0.4617) * pow((double)b, 0.9003) * pow((double)n, -0.4498) *
+                   pow(epochs, -0.1057);
+        r->alpha0 = std::min(1.0, std::max(1e-4, a));
+    }
+    const double whole = floor(epochs);
+    const double frac = epochs - whole;
+    r->passes = (int64_t)whole + (frac > 0 ? 1 : 0);
+    r->rows_last_pass = frac > 0 ? std::max<int64_t>(1, (int64_t)floor(frac * (double)n + 0.5)) : n;
+    r->steps_full_pass = (n + b - 1) / b;
+    r->steps_last_pass = (r->rows_last_pass + b - 1) / b;
+    r->total_steps = (r->passes - 1) * r->steps_full_pass + r->steps_last_pass;
+    return EM_OK;
+}
+
+// cosine step size from alpha0 down to alpha0 / 10 over all steps
+static double alpha_at(int64_t t, int64_t total, double alpha0) {
+    const double amin = 0.1 * alpha0;
+    const double frac = total <= 1 ? 0.0 : (double)t / (double)(total - 1);
+    return amin + (alpha0 - amin) * 0.5 * (1.0 + cos(M_PI * frac));
+}
+
+// ------------------------------------------------------------------ tensor maps
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+        else
+            cudaGetLastError();
+    });
+    return fn;
+}
+
+// 2-D bf16 tensor map over `rows` rows of d values (row pitch ld elements), boxes
+// of kc x box_rows with the swizzle the UMMA descriptors expect.
+static int make_tmap(CUtensorMap* tm, const void* base, int64_t rows, int d, int ld, int box_rows, int kc) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return fail(EM_E_CUDA, "cuTensorMapEncodeTiled is not available");
+    if ((reinterpret_cast<uintptr_t>(base) & 15) != 0) return fail(EM_E_INVAL, "tensor base not 16-byte aligned");
+    cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)std::max<int64_t>(rows, 1)};
+    cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
+    cuuint32_t box[2] = {(cuuint32_t)kc, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, kc == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(EM_E_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return EM_OK;
+}
+
+// ------------------------------------------------------------------ model
+
+template <class T>
+struct DBuf {
+    T* p = nullptr;
+    size_t cap = 0;  // elements
+    int ensure(size_t count) {
+        if (count <= cap && p) return EM_OK;
+        if (p) cudaFree(p);
+        p = nullptr;
+        cap = 0;
+        if (cudaMalloc(&p, std::max<size_t>(count, 1) * sizeof(T)) != cudaSuccess) {
+            cudaGetLastError();
+            p = nullptr;
+            return fail(EM_E_NOMEM, "cudaMalloc of %zu bytes failed", count * sizeof(T));
+        }
+        cap = count;
+        return EM_OK;
+    }
+    void release() {
+        if (p) cudaFree(p);
+        p = nullptr;
+        cap = 0;
+    }
+};
+
+struct em_model {
+    int dev = 0, sms = 148;
+    long long wait_cycles = 0;
+    cudaStream_t stream = nullptr;
+    bool own_stream = false;
+    int64_t d = 0, k = 0;
+    int ld = 0, nv = 0, kc = 64;
+    uint64_t seed = 1234;
+    // options
+    int64_t opt_batch = 0;
+    double opt_alpha0 = 0.0, tau = 0.1, wait_ms = 2000.0;
+    int revival = EM_REVIVE_SPLIT, finalize = 1, law = 0, in_dtype = 0, check_finite = 0;
+    int auto_revive = 1, capture = 1, graphs = 1, assign_kernel = 0;
+    // state
+    DBuf<float> N, S, c, cn;
+    DBuf<__nv_bfloat16> cq;
+    DBuf<double> close_sum, close_cnt;
+    DBuf<int> err, flag;
+    // data of the current run
+    const __nv_bfloat16* X = nullptr;
+    int64_t n = 0;
+    DBuf<__nv_bfloat16> Xown;
+    DBuf<uint8_t> stage;  // host-input staging
+    // batch buffers
+    int64_t bcap = 0;
+    int R = 32;
+    DBuf<__nv_bfloat16> Xb;
+    DBuf<float> xn, dists;
+    DBuf<int32_t> ids, labels, cnt, rank, off, perm, slab;
+    DBuf<unsigned long long> keys;
+    DBuf<double> block_err, pfirst, plast, step_err, scalar;
+    DBuf<int64_t> labels_last, labels64;
+    // revival scratch
+    DBuf<int32_t> rv_dead, rv_donor, rv_order, rv_times, rv_ndead;
+    DBuf<double> rv_tree;
+    DBuf<int64_t> rv_splits;
+    // run progress
+    em_recipe_t rec{};
+    bool running = false, have_run = false;
+    int64_t t = 0, pass = 0, pos = 0, rows_assigned = 0;
+    int64_t last_rows = 0;
+    double last_alpha = 0.0;
+    int last_was_lloyd = 0;
+    CUtensorMap tm_cq, tm_xb;
+    // profiling (EM_OPT_PROFILE) and launch counting
+    int profile = 0;
+    int64_t launches = 0;
+    struct Span {
+        int phase;
+        cudaEvent_t a, b;
+        double flops, bytes;
+    };
+    std::vector<Span> pending;
+    std::vector<cudaEvent_t> pool;
+    em_profile_t totals{};
+};
+
+// Opens an event span of `phase` on the model's stream (-1 when profiling is off).
+static int span_begin(em_model* m, int phase) {
+    if (!m->profile) return -1;
+    cudaEvent_t ev[2];
+    for (int i = 0; i < 2; ++i) {
+        if (!m->pool.empty()) {
+            ev[i] = m->pool.back();
+            m->pool.pop_back();
+        } else if (cudaEventCreate(&ev[i]) != cudaSuccess) {
+            cudaGetLastError();
+            return -1;
+        }
+    }
+    cudaEventRecord(ev[0], m->stream);
+    m->pending.push_back({phase, ev[0], ev[1], 0.0, 0.0});
+    return (int)m->pending.size() - 1;
+}
+
+static void span_end(em_model* m, int idx, double flops = 0.0, double bytes = 0.0) {
+    if (idx < 0) return;
+    em_model::Span& sp = m->pending[idx];
+    sp.flops = flops;
+    sp.bytes = bytes;
+    cudaEventRecord(sp.b, m->stream);
+}
+
+#define EM_LAUNCHED(m, count) ((m)->launches += (count))
+
+static int set_device(const em_model* m) {
+    CK(cudaSetDevice(m->dev));
+    return EM_OK;
+}
+
+static int check_device_errors(em_model* m) {
+    int h = 0;
+    CK(cudaMemcpyAsync(&h, m->err.p, sizeof(int), cudaMemcpyDeviceToHost, m->stream));
+    CK(cudaStreamSynchronize(m->stream));
+    if (h != 0) {
+        CK(cudaMemsetAsync(m->err.p, 0, sizeof(int), m->stream));
+        CK(cudaStreamSynchronize(m->stream));
+        return fail(h, h == EM_E_TIMEOUT ? "a device-side wait exceeded its limit"
+                                         : "a kernel's index check failed (device error %d)",
+                    h);
+    }
+    return EM_OK;
+}
+
+static bool is_device_ptr(const void* p) {
+    cudaPointerAttributes a;
+    if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    return a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged;
+}
+
+static int grid_for(int64_t work, int block, int sms, int per_sm = 8) {
+    int64_t g = (work + block - 1) / block;
+    g = std::min<int64_t>(g, (int64_t)sms * per_sm);
+    return (int)std::max<int64_t>(g, 1);
+}
+
+// Makes a bf16 n x ld device copy of X (or uses X in place). *out receives the
+// row source the kernels read.
+static int prepare_input(em_model* m, const void* X, int64_t n, DBuf<__nv_bfloat16>& own,
+                         const __nv_bfloat16** out) {
+    if (!X || n < 1) return fail(EM_E_INVAL, "X is NULL or n < 1");
+    const bool dev = is_device_ptr(X);
+    const size_t esz = m->in_dtype == 1 ? 2 : 4;
+    const size_t raw_bytes = (size_t)n * (size_t)m->d * esz;
+    const void* src = X;
+    if (!dev) {  // host input: copy to the device first
+        CKR(m->stage.ensure(raw_bytes));
+        CK(cudaMemcpyAsync(m->stage.p, X, raw_bytes, cudaMemcpyHostToDevice, m->stream));
+        src = m->stage.p;
+    }
+    if (m->check_finite) {
+        CK(cudaMemsetAsync(m->flag.p, 0, sizeof(int), m->stream));
+        k_check_finite<<<grid_for(n * m->d, 256, m->sms), 256, 0, m->stream>>>(src, n * m->d, m->in_dtype == 1,
+                                                                                m->flag.p);
+        CK(cudaGetLastError());
+        int h = 0;
+        CK(cudaMemcpyAsync(&h, m->flag.p, sizeof(int), cudaMemcpyDeviceToHost, m->stream));
+        CK(cudaStreamSynchronize(m->stream));
+        if (h) return fail(EM_E_NONFINITE, "input holds NaN or infinite values");
+    }
+    if (m->in_dtype == 1 && m->ld == m->d && (reinterpret_cast<uintptr_t>(src) & 15) == 0) {
+        *out = reinterpret_cast<const __nv_bfloat16*>(src);
+        return EM_OK;
+    }
+    CKR(own.ensure((size_t)n * m->ld));
+    if (m->in_dtype == 1) {
+        k_pad_bf16<<<grid_for(n * m->ld, 256, m->sms), 256, 0, m->stream>>>(
+            reinterpret_cast<const __nv_bfloat16*>(src), n, (int)m->d, m->ld, own.p);
+    } else {
+        const int vec_ok = (m->d % 4 == 0) && ((reinterpret_cast<uintptr_t>(src) & 15) == 0);
+        k_cast_f32_bf16<<<grid_for(n * m->nv, 256, m->sms), 256, 0, m->stream>>>(
+            reinterpret_cast<const float*>(src), n, (int)m->d, m->ld, own.p, vec_ok);
+    }
+    CK(cudaGetLastError());
+    EM_LAUNCHED(m, 1);
+    *out = own.p;
+    return EM_OK;
+}
+
+static ClusterState cluster_state(em_model* m) {
+    ClusterState st;
+    st.N = m->N.p;
+    st.S = m->S.p;
+    st.c = m->c.p;
+    st.cq = m->cq.p;
+    st.cn = m->cn.p;
+    st.close_sum = m->close_sum.p;
+    st.close_cnt = m->close_cnt.p;
+    st.ld = m->ld;
+    return st;
+}
+
+static int ensure_batch_buffers(em_model* m, int64_t cap) {
+    m->R = 32;
+    {
+        // tiles of R label-sorted rows per warp: about 16 tiles per SM
+        int64_t want = cap / ((int64_t)m->sms * 16);
+        int r = 8;
+        while (r < 256 && r < want) r <<= 1;
+        m->R = r;
+    }
+    const int64_t ntiles = (cap + m->R - 1) / m->R;
+    CKR(m->xn.ensure(cap));
+    CKR(m->dists.ensure(cap));
+    CKR(m->ids.ensure(cap));
+    CKR(m->labels.ensure(cap));
+    CKR(m->rank.ensure(cap));
+    CKR(m->perm.ensure(cap));
+    CKR(m->slab.ensure(cap));
+    CKR(m->keys.ensure(cap));
+    CKR(m->cnt.ensure(m->k));
+    CKR(m->off.ensure(m->k + 1));
+    CKR(m->block_err.ensure((cap + 255) / 256 + 1));
+    CKR(m->pfirst.ensure((size_t)ntiles * m->ld));
+    CKR(m->plast.ensure((size_t)ntiles * m->ld));
+    m->bcap = cap;
+    return EM_OK;
+}
+
+static int choose_split(int64_t m_tiles, int64_t n_tiles, int sms) {
+    int best = 1;
+    double best_cost = 1e300;
+    for (int s = 1; s <= 8; s <<= 1) {
+        if (s > n_tiles) break;
+        const int64_t units = m_tiles * s;
+        const int64_t waves = (units + sms - 1) / sms;
+        const double cost = (double)waves * (double)((n_tiles + s - 1) / s);
+        if (cost < best_cost * 0.985) {
+            best_cost = cost;
+            best = s;
+        }
+    }
+    return best;
+}
+
+// Nearest-centroid search of `rows` rows described by tmA (row source A for the
+// SIMT path) into m->keys (which the caller has reset to the empty key).
+static int launch_assign(em_model* m, const CUtensorMap& tmA, const __nv_bfloat16* A, int64_t rows) {
+    if (rows <= 0) return EM_OK;
+    if (m->assign_kernel == 1) {
+        k_assign_simt<<<(int)((rows + 127) / 128), 128, 0, m->stream>>>(A, m->ld, (int)rows, m->cq.p, m->cn.p,
+                                                                         (int)m->k, (int)m->d, m->keys.p);
+        CK(cudaGetLastError());
+        EM_LAUNCHED(m, 1);
+        return EM_OK;
+    }
+    const int64_t m_tiles = (rows + tc::BM - 1) / tc::BM;
+    const int64_t n_tiles = (m->k + tc::BN - 1) / tc::BN;
+    const int nkc = (int)((m->d + m->kc - 1) / m->kc);
+    const int split = choose_split(m_tiles, n_tiles, m->sms);
+    const int64_t units = m_tiles * split;
+    const int grid = (int)std::min<int64_t>(units, m->sms);
+    if (m->kc == 64) {
+        tc::k_assign_tc<64><<<grid, tc::kThreads, tc::Cfg<64>::kSmemBytes, m->stream>>>(
+            tmA, m->tm_cq, m->cn.p, (int)m->k, (int)rows, nkc, (int)n_tiles, split, m->keys.p, m->wait_cycles,
+            m->err.p);
+    } else {
+        tc::k_assign_tc<32><<<grid, tc::kThreads, tc::Cfg<32>::kSmemBytes, m->stream>>>(
+            tmA, m->tm_cq, m->cn.p, (int)m->k, (int)rows, nkc, (int)n_tiles, split, m->keys.p, m->wait_cycles,
+            m->err.p);
+    }
+    CK(cudaGetLastError());
+    EM_LAUNCHED(m, 1);
+    return EM_OK;
+}
+
+// Group rows by label and apply the EMA update (k_offsets .. k_fixup); labels,
+// ranks and counts are already in place. `src` holds the rows (batch or data).
+static int launch_reduce(em_model* m, const __nv_bfloat16* src, int64_t rows, int nblocks_labels, double alpha,
+                         int last_pass, double* err_sum_out) {
+    const StepParams sp{alpha, last_pass, 0};
+    k_offsets<<<1, 1024, 0, m->stream>>>(m->cnt.p, (int)m->k, (int)rows, m->off.p, m->block_err.p, nblocks_labels,
+                                         err_sum_out, m->err.p);
+    CK(cudaGetLastError());
+    k_scatter<<<(int)((rows + 255) / 256), 256, 0, m->stream>>>(m->labels.p, m->rank.p, m->off.p, (int)rows,
+                                                                 m->perm.p, m->slab.p, m->err.p);
+    CK(cudaGetLastError());
+    const int64_t ntiles = (rows + m->R - 1) / m->R;
+    const int seg_blocks = (int)((ntiles * 32 + 255) / 256);
+    const ClusterState st = cluster_state(m);
+    const int fix_blocks = grid_for(std::max<int64_t>(ntiles, m->k) * 32, 256, m->sms);
+#define EM_REDUCE(V)                                                                                            \
+    k_segsum<V><<<seg_blocks, 256, 0, m->stream>>>(src, m->perm.p, m->slab.p, m->off.p, (int)rows, m->R, m->nv, \
+                                                   st, sp, m->pfirst.p, m->plast.p);                           \
+    k_fixup<V><<<fix_blocks, 256, 0, m->stream>>>(m->slab.p, m->off.p, m->cnt.p, (int)rows, m->R, (int)ntiles,  \
+                                                  (int)m->k, m->nv, st, sp, m->pfirst.p, m->plast.p)
+    if (m->nv <= 32) {
+        EM_REDUCE(1);
+    } else if (m->nv <= 64) {
+        EM_REDUCE(2);
+    } else if (m->nv <= 96) {
+        EM_REDUCE(3);
+    } else if (m->nv <= 128) {
+        EM_REDUCE(4);
+    } else {
+        EM_REDUCE(8);
+    }
+#undef EM_REDUCE
+    CK(cudaGetLastError());
+    EM_LAUNCHED(m, 4);
+    return EM_OK;
+}
+
+static ReviveScratch revive_scratch(em_model* m) {
+    ReviveScratch sc;
+    sc.dead = m->rv_dead.p;
+    sc.donor = m->rv_donor.p;
+    sc.order = m->rv_order.p;
+    sc.times = m->rv_times.p;
+    sc.tree = m->rv_tree.p;
+    sc.ndead = m->rv_ndead.p;
+    sc.n_splits = m->rv_splits.p;
+    return sc;
+}
+
+static int launch_revive(em_model* m, int64_t t, int64_t rows) {
+    if (m->revival == EM_REVIVE_NONE || !(m->tau > 0.0)) return EM_OK;
+    const ReviveScratch sc = revive_scratch(m);
+    const TreeLayout L = tree_layout((int)m->k);
+    const int smem = (int)tree_smem_bytes(L);
+    k_revive_select<<<1, 1024, smem, m->stream>>>(m->N.p, (int)m->k, m->tau, m->seed, t, m->revival, sc, m->err.p);
+    CK(cudaGetLastError());
+    const ClusterState st = cluster_state(m);
+    const int blocks = grid_for(m->k * 32, 256, m->sms);
+    if (m->revival == EM_REVIVE_SPLIT) {
+        k_revive_dead<<<blocks, 256, 0, m->stream>>>(st, m->nv, sc);
+        k_revive_donors<<<blocks, 256, 0, m->stream>>>(st, m->nv, sc);
+        EM_LAUNCHED(m, 3);
+    } else {
+        k_revive_resample<<<blocks, 256, 0, m->stream>>>(st, m->nv, sc, m->Xb.p, (int)rows, m->seed, t);
+        EM_LAUNCHED(m, 2);
+    }
+    CK(cudaGetLastError());
+    return EM_OK;
+}
+
+// One training step of the current run.
+static int run_step(em_model* m) {
+    const int64_t rows_pass = (m->pass == m->rec.passes - 1) ? m->rec.rows_last_pass : m->n;
+    const int64_t rows = std::min<int64_t>(m->rec.batch_size, rows_pass - m->pos);
+    const int last_pass = (m->pass == m->rec.passes - 1) ? 1 : 0;
+    const double alpha = alpha_at(m->t, m->rec.total_steps, m->rec.alpha0);
+    const double rd = (double)rows, dd = (double)m->d, kd = (double)m->k;
+    int sp = span_begin(m, EM_PHASE_GATHER);
+    k_gather<<<grid_for(rows, 256, m->sms), 256, 0, m->stream>>>(m->X, m->n, m->ld, m->seed, m->pass, m->pos,
+                                                                 (int)rows, 0, m->Xb.p, m->xn.p, m->ids.p,
+                                                                 m->keys.p, m->err.p);
+    CK(cudaGetLastError());
+    EM_LAUNCHED(m, 1);
+    span_end(m, sp, 0.0, 4.0 * rd * dd);
+    sp = span_begin(m, EM_PHASE_ASSIGN);
+    CKR(launch_assign(m, m->tm_xb, m->Xb.p, rows));
+    span_end(m, sp, 2.0 * rd * kd * dd, 0.0);
+    sp = span_begin(m, EM_PHASE_UPDATE);
+    const int nbl = (int)((rows + 255) / 256);
+    const int capture = (m->capture && last_pass) ? 1 : 0;
+    k_labels<<<nbl, 256, 0, m->stream>>>(m->keys.p, m->xn.p, (int)rows, (int)m->k, m->ids.p, m->labels.p,
+                                         m->dists.p, m->cnt.p, m->rank.p, m->block_err.p, m->labels_last.p, capture,
+                                         m->err.p);
+    CK(cudaGetLastError());
+    EM_LAUNCHED(m, 1);
+    CKR(launch_reduce(m, m->Xb.p, rows, nbl, alpha, m->finalize ? last_pass : 0, m->step_err.p + m->t));
+    span_end(m, sp, 0.0, 2.0 * rd * dd + 16.0 * rd + 14.0 * kd * dd);
+    if (m->auto_revive && (m->t + 1) % kReviveEvery == 0) {
+        sp = span_begin(m, EM_PHASE_REVIVE);
+        CKR(launch_revive(m, m->t, rows));
+        span_end(m, sp);
+    }
+    m->last_rows = rows;
+    m->last_alpha = alpha;
+    m->rows_assigned += rows;
+    m->t += 1;
+    m->pos += rows;
+    if (m->pos >= rows_pass) {
+        m->pass += 1;
+        m->pos = 0;
+    }
+    return EM_OK;
+}
+
+static int start_centroids(em_model* m) {
+    k_init_centroids<<<grid_for(m->k * 32, 256, m->sms), 256, 0, m->stream>>>(
+        m->X, m->n, m->ld, (int)m->k, m->seed, m->c.p, m->S.p, m->N.p, m->cq.p, m->cn.p, m->err.p);
+    CK(cudaGetLastError());
+    EM_LAUNCHED(m, 1);
+    return EM_OK;
+}
+
+// ------------------------------------------------------------------ ABI
+
+extern "C" {
+
+const char* em_last_error(void) { return g_err; }
+
+int em_device_count(void) {
+    int n = 0;
+    if (cudaGetDeviceCount(&n) != cudaSuccess) {
+        cudaGetLastError();
+        return 0;
+    }
+    return n;
+}
+
+int em_compute_recipe(int64_t n, int64_t k, double epochs, int law, int64_t batch_override, double alpha_override,
+                      em_recipe_t* out) {
+    if (!out) return fail(EM_E_INVAL, "out is NULL");
+    return compute_recipe(n, k, 0, epochs, law, batch_override, alpha_override, out);
+}
+
+int em_permutation(int64_t n, uint64_t seed, int stream, int64_t which, const int64_t* idx, int64_t count,
+                   int64_t* out) {
+    if (n < 1 || count < 0 || (count > 0 && (!idx || !out))) return fail(EM_E_INVAL, "bad permutation arguments");
+    const Feistel f(n, seed, stream, which);
+    for (int64_t i = 0; i < count; ++i) {
+        if (idx[i] < 0 || idx[i] >= n) return fail(EM_E_INVAL, "index out of range");
+        bool ok = true;
+        out[i] = f((uint64_t)idx[i], &ok);
+        if (!ok) return fail(EM_E_BOUNDS, "cycle walk did not end");
+    }
+    return EM_OK;
+}
+
+em_model* em_create(int64_t d, int64_t k, uint64_t seed) {
+    if (d < 1 || d > 8192 || k < 1 || k > (1ll << 30)) {
+        fail(EM_E_INVAL, "need 1 <= d <= 8192 and 1 <= k <= 2^30");
+        return nullptr;
+    }
+    if (em_device_count() < 1) {
+        fail(EM_E_NODEVICE, "no CUDA device");
+        return nullptr;
+    }
+    em_model* m = new em_model();
+    m->d = d;
+    m->k = k;
+    m->seed = seed;
+    m->ld = (int)((d + 7) / 8 * 8);
+    m->nv = m->ld / 8;
+    m->kc = (d % 64 == 0) ? 64 : 32;
+    auto bail = [&](int code, const char* what) -> em_model* {
+        fail(code, "%s", what);
+        em_destroy(m);
+        return nullptr;
+    };
+    if (cudaGetDevice(&m->dev) != cudaSuccess) return bail(EM_E_CUDA, "cudaGetDevice failed");
+    int clock_khz = 1965000;
+    cudaDeviceGetAttribute(&m->sms, cudaDevAttrMultiProcessorCount, m->dev);
+    cudaDeviceGetAttribute(&clock_khz, cudaDevAttrClockRate, m->dev);
+    m->wait_cycles = (long long)(m->wait_ms * (double)clock_khz);
+    int cc_major = 0, cc_minor = 0;
+    cudaDeviceGetAttribute(&cc_major, cudaDevAttrComputeCapabilityMajor, m->dev);
+    cudaDeviceGetAttribute(&cc_minor, cudaDevAttrComputeCapabilityMinor, m->dev);
+    if (cc_major != 10 || cc_minor != 0) return bail(EM_E_NODEVICE, "this library is built for sm_100a (B200)");
+    if (cudaStreamCreateWithFlags(&m->stream, cudaStreamNonBlocking) != cudaSuccess)
+        return bail(EM_E_CUDA, "cudaStreamCreate failed");
+    m->own_stream = true;
+    const size_t kd = (size_t)k * m->ld;
+    if (m->N.ensure(k) || m->S.ensure(kd) || m->c.ensure(kd) || m->cn.ensure(k) || m->cq.ensure(kd) ||
+        m->close_sum.ensure(kd) || m->close_cnt.ensure(k) || m->err.ensure(1) || m->flag.ensure(1) ||
+        m->scalar.ensure(4) || m->rv_dead.ensure(k) || m->rv_donor.ensure(k) || m->rv_order.ensure(k) ||
+        m->rv_times.ensure(k) || m->rv_ndead.ensure(1) || m->rv_splits.ensure(1) ||
+        m->rv_tree.ensure((size_t)tree_layout((int)k).total))
+        return bail(EM_E_NOMEM, "device allocation failed");
+    cudaMemset(m->err.p, 0, sizeof(int));
+    cudaMemset(m->rv_splits.p, 0, sizeof(int64_t));
+    cudaMemset(m->rv_ndead.p, 0, sizeof(int32_t));
+    cudaMemset(m->N.p, 0, k * sizeof(float));
+    cudaMemset(m->S.p, 0, kd * sizeof(float));
+    cudaMemset(m->c.p, 0, kd * sizeof(float));
+    cudaMemset(m->cq.p, 0, kd * sizeof(__nv_bfloat16));
+    cudaMemset(m->cn.p, 0, k * sizeof(float));
+    if (cudaFuncSetAttribute(tc::k_assign_tc<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             tc::Cfg<64>::kSmemBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(tc::k_assign_tc<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             tc::Cfg<32>::kSmemBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(k_revive_select, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kReviveSmemDoubles * 8) != cudaSuccess)
+        return bail(EM_E_CUDA, "cudaFuncSetAttribute failed");
+    if (make_tmap(&m->tm_cq, m->cq.p, k, (int)d, m->ld, tc::BN, m->kc) != EM_OK) {
+        em_destroy(m);
+        return nullptr;
+    }
+    if (cudaDeviceSynchronize() != cudaSuccess) return bail(EM_E_CUDA, "device initialisation failed");
+    return m;
+}
+
+void em_destroy(em_model* m) {
+    if (!m) return;
+    cudaSetDevice(m->dev);
+    if (m->stream) cudaStreamSynchronize(m->stream);
+    m->N.release(); m->S.release(); m->c.release(); m->cn.release(); m->cq.release();
+    m->close_sum.release(); m->close_cnt.release(); m->err.release(); m->flag.release();
+    m->Xown.release(); m->stage.release(); m->Xb.release(); m->xn.release(); m->dists.release();
+    m->ids.release(); m->labels.release(); m->cnt.release(); m->rank.release(); m->off.release();
+    m->perm.release(); m->slab.release(); m->keys.release(); m->block_err.release(); m->pfirst.release();
+    m->plast.release(); m->step_err.release(); m->scalar.release(); m->labels_last.release();
+    m->labels64.release(); m->rv_dead.release(); m->rv_donor.release(); m->rv_order.release();
+    m->rv_times.release(); m->rv_ndead.release(); m->rv_tree.release(); m->rv_splits.release();
+    for (auto& sp : m->pending) {
+        cudaEventDestroy(sp.a);
+        cudaEventDestroy(sp.b);
+    }
+    for (auto ev : m->pool) cudaEventDestroy(ev);
+    if (m->own_stream && m->stream) cudaStreamDestroy(m->stream);
+    delete m;
+}
+
+int em_set_option(em_model* m, int opt, double v) {
+    if (!m) return fail(EM_E_INVAL, "model is NULL");
+    switch (opt) {
+        case EM_OPT_BATCH_SIZE:
+            if (v < 0 || v != floor(v)) return fail(EM_E_INVAL, "batch size must be a non-negative integer");
+            m->opt_batch = (int64_t)v;
+            break;
+        case EM_OPT_ALPHA0:
+            if (v < 0 || v > 1) return fail(EM_E_INVAL, "alpha0 must be in [0, 1]");
+            m->opt_alpha0 = v;
+            break;
+        case EM_OPT_UNUSED_THRESHOLD:
+            if (!(v >= 0) || v > 1) return fail(EM_E_INVAL, "threshold must be in [0, 1]");
+            m->tau = v;
+            break;
+        case EM_OPT_REVIVAL:
+            if (v != 0 && v != 1 && v != 2) return fail(EM_E_INVAL, "revival mode is 0, 1 or 2");
+            m->revival = (int)v;
+            break;
+        case EM_OPT_FINALIZE: m->finalize = v != 0; break;
+        case EM_OPT_LAW:
+            if (v != 0 && v != 1) return fail(EM_E_INVAL, "law is 0 or 1");
+            m->law = (int)v;
+            break;
+        case EM_OPT_INPUT_DTYPE:
+            if (v != 0 && v != 1) return fail(EM_E_INVAL, "input dtype is 0 (fp32) or 1 (bf16)");
+            m->in_dtype = (int)v;
+            break;
+        case EM_OPT_CHECK_FINITE: m->check_finite = v != 0; break;
+        case EM_OPT_WAIT_LIMIT_MS: {
+            if (!(v > 0)) return fail(EM_E_INVAL, "wait limit must be positive");
+            int clock_khz = 1965000;
+            cudaDeviceGetAttribute(&clock_khz, cudaDevAttrClockRate, m->dev);
+            m->wait_ms = v;
+            m->wait_cycles = (long long)(v * (double)clock_khz);
+            break;
+        }
+        case EM_OPT_AUTO_REVIVE: m->auto_revive = v != 0; break;
+        case EM_OPT_CAPTURE_LABELS: m->capture = v != 0; break;
+        case EM_OPT_GRAPHS: m->graphs = v != 0; break;
+        case EM_OPT_ASSIGN_KERNEL:
+            if (v != 0 && v != 1) return fail(EM_E_INVAL, "assign kernel is 0 or 1");
+            m->assign_kernel = (int)v;
+            break;
+        case EM_OPT_PROFILE: m->profile = v != 0; break;
+        default: return fail(EM_E_INVAL, "unknown option %d", opt);
+    }
+    return EM_OK;
+}
+
+int em_get_option(const em_model* m, int opt, double* v) {
+    if (!m || !v) return fail(EM_E_INVAL, "NULL argument");
+    switch (opt) {
+        case EM_OPT_BATCH_SIZE: *v = (double)m->opt_batch; break;
+        case EM_OPT_ALPHA0: *v = m->opt_alpha0; break;
+        case EM_OPT_UNUSED_THRESHOLD: *v = m->tau; break;
+        case EM_OPT_REVIVAL: *v = m->revival; break;
+        case EM_OPT_FINALIZE: *v = m->finalize; break;
+        case EM_OPT_LAW: *v = m->law; break;
+        case EM_OPT_INPUT_DTYPE: *v = m->in_dtype; break;
+        case EM_OPT_CHECK_FINITE: *v = m->check_finite; break;
+        case EM_OPT_WAIT_LIMIT_MS: *v = m->wait_ms; break;
+        case EM_OPT_AUTO_REVIVE: *v = m->auto_revive; break;
+        case EM_OPT_CAPTURE_LABELS: *v = m->capture; break;
+        case EM_OPT_GRAPHS: *v = m->graphs; break;
+        case EM_OPT_ASSIGN_KERNEL: *v = m->assign_kernel; break;
+        case EM_OPT_PROFILE: *v = m->profile; break;
+        default: return fail(EM_E_INVAL, "unknown option %d", opt);
+    }
+    return EM_OK;
+}
+
+int em_set_stream(em_model* m, void* stream) {
+    if (!m) return fail(EM_E_INVAL, "model is NULL");
+    CKR(set_device(m));
+    CK(cudaStreamSynchronize(m->stream));
+    if (m->own_stream) cudaStreamDestroy(m->stream);
+    m->stream = reinterpret_cast<cudaStream_t>(stream);
+    m->own_stream = false;
+    return EM_OK;
+}
+
+int em_begin(em_model* m, const void* X, int64_t n, double epochs) {
+    if (!m) return fail(EM_E_INVAL, "model is NULL");
+    if (n < m->k) return fail(EM_E_INVAL, "need at least k rows (n = %lld, k = %lld)", (long long)n, (long long)m->k);
+    if (n >= (1ll << 31)) return fail(EM_E_INVAL, "n must be below 2^31");
+    if (!(epochs > 0.0)) return fail(EM_E_INVAL, "epochs must be positive");
+    CKR(set_device(m));
+    CKR(compute_recipe(n, m->k, m->d, epochs, m->law, m->opt_batch, m->opt_alpha0, &m->rec));
+    if (m->rec.batch_size > n) return fail(EM_E_INVAL, "batch size larger than n");
+    m->running = false;
+    m->n = n;
+    const int sp = span_begin(m, EM_PHASE_PREPARE);
+    CKR(prepare_input(m, X, n, m->Xown, &m->X));
+    const int64_t b = m->rec.batch_size;
+    CKR(m->Xb.ensure((size_t)b * m->ld));
+    CKR(ensure_batch_buffers(m, b));
+    CKR(m->step_err.ensure(m->rec.total_steps));
+    CK(cudaMemsetAsync(m->step_err.p, 0, m->rec.total_steps * sizeof(double), m->stream));
+    CK(cudaMemsetAsync(m->cnt.p, 0, m->k * sizeof(int32_t), m->stream));
+    CK(cudaMemsetAsync(m->close_sum.p, 0, (size_t)m->k * m->ld * sizeof(double), m->stream));
+    CK(cudaMemsetAsync(m->close_cnt.p, 0, m->k * sizeof(double), m->stream));
+    CK(cudaMemsetAsync(m->rv_splits.p, 0, sizeof(int64_t), m->stream));
+    CK(cudaMemsetAsync(m->rv_ndead.p, 0, sizeof(int32_t), m->stream));
+    if (m->capture) {
+        CKR(m->labels_last.ensure(n));
+        CK(cudaMemsetAsync(m->labels_last.p, 0xFF, n * sizeof(int64_t), m->stream));
+    }
+    CKR(make_tmap(&m->tm_xb, m->Xb.p, b, (int)m->d, m->ld, tc::BM, m->kc));
+    CKR(start_centroids(m));
+    span_end(m, sp);
+    m->t = m->pass = m->pos = m->rows_assigned = 0;
+    m->last_rows = 0;
+    m->last_alpha = 0.0;
+    m->running = true;
+    m->have_run = true;
+    m->last_was_lloyd = 0;
+    return EM_OK;
+}
+
+int em_step(em_model* m, int64_t nsteps, int64_t* done) {
+    if (done) *done = 0;
+    if (!m) return fail(EM_E_INVAL, "model is NULL");
+    if (!m->running) return fail(EM_E_STATE, "no run in progress (call em_begin)");
+    CKR(set_device(m));
+    int64_t ran = 0;
+    while (ran < nsteps && m->t < m->rec.total_steps) {
+        CKR(run_step(m));
+        ++ran;
+    }
+    if (done) *done = ran;
+    return EM_OK;
+}
+
+int em_revive(em_model* m) {
+    if (!m) return fail(EM_E_INVAL, "model is NULL");
+    if (!m->running || m->t == 0) return fail(EM_E_STATE, "no step has run");
+    CKR(set_device(m));
+    return launch_revive(m, m->t - 1, m->last_rows);
+}
+
+int em_finalize(em_model* m) {
+    if (!m) return fail(EM_E_INVAL, "model is NULL");
+    if (!m->running) return fail(EM_E_STATE, "no run in progress");
+    CKR(set_device(m));
+    if (m->finalize && m->t >= m->rec.total_steps) {
+        const int sp = span_begin(m, EM_PHASE_FINALIZE);
+        k_closing_mean<<<grid_for(m->k * 32, 256, m->sms), 256, 0, m->stream>>>(cluster_state(m), (int)m->k,
+                                                                                  m->nv);
+        CK(cudaGetLastError());
+        EM_LAUNCHED(m, 1);
+        span_end(m, sp);
+    }
+    m->running = false;
+    return check_device_errors(m);
+}
+
+int em_train(em_model* m, const void* X, int64_t n, double epochs) {
+    CKR(em_begin(m, X, n, epochs));
+    CKR(em_step(m, m->rec.total_steps, nullptr));
+    return em_finalize(m);
+}
+
+int em_lloyd(em_model* m, const void* X, int64_t n, int64_t iters) {
+    if (!m) return fail(EM_E_INVAL, "model is NULL");
+    if (n < m->k || n >= (1ll << 31) || iters < 0) return fail(EM_E_INVAL, "bad Lloyd arguments");
+    CKR(set_device(m));
+    m->running = false;
+    m->n = n;
+    CKR(prepare_input(m, X, n, m->Xown, &m->X));
+    CKR(ensure_batch_buffers(m, n));
+    CK(cudaMemsetAsync(m->cnt.p, 0, m->k * sizeof(int32_t), m->stream));
+    CKR(start_centroids(m));
+    CUtensorMap tmx;
+    CKR(make_tmap(&tmx, m->X, n, (int)m->d, m->ld, tc::BM, m->kc));
+    const int nbl = (int)((n + 255) / 256);
+    for (int64_t it = 0; it < iters; ++it) {
+        k_rownorm_keys<<<grid_for(n * 32, 256, m->sms), 256, 0, m->stream>>>(m->X, n, m->ld, m->xn.p, m->keys.p);
+        CK(cudaGetLastError());
+        EM_LAUNCHED(m, 1);
+        CKR(launch_assign(m, tmx, m->X, n));
+        k_labels<<<nbl, 256, 0, m->stream>>>(m->keys.p, m->xn.p, (int)n, (int)m->k, nullptr, m->labels.p,
+                                             m->dists.p, m->cnt.p, m->rank.p, m->block_err.p, nullptr, 0, m->err.p);
+        CK(cudaGetLastError());
+        EM_LAUNCHED(m, 1);
+        CKR(launch_reduce(m, m->X, n, nbl, 1.0, 0, m->scalar.p));
+    }
+    m->have_run = false;
+    m->last_was_lloyd = 1;
+    return check_device_errors(m);
+}
+
+static int assign_pass(em_model* m, const void* X, int64_t n, int64_t* labels_dev, float* dists_dev,
+                       double* sum_dev, DBuf<__nv_bfloat16>& tmp) {
+    const __nv_bfloat16* A = nullptr;
+    CKR(prepare_input(m, X, n, tmp, &A));
+    CKR(m->xn.ensure(n));
+    CKR(m->keys.ensure(n));
+    CKR(m->block_err.ensure((n + 255) / 256 + 1));
+    k_rownorm_keys<<<grid_for(n * 32, 256, m->sms), 256, 0, m->stream>>>(A, n, m->ld, m->xn.p, m->keys.p);
+    CK(cudaGetLastError());
+    EM_LAUNCHED(m, 1);
+    CUtensorMap tmx;
+    CKR(make_tmap(&tmx, A, n, (int)m->d, m->ld, tc::BM, m->kc));
+    CKR(launch_assign(m, tmx, A, n));
+    const int blocks = grid_for(n, 256, m->sms);
+    k_assign_out<<<blocks, 256, 0, m->stream>>>(m->keys.p, m->xn.p, n, (int)m->k, labels_dev, dists_dev, nullptr,
+                                                m->block_err.p, m->err.p);
+    CK(cudaGetLastError());
+    k_sum_blocks<<<1, 32, 0, m->stream>>>(m->block_err.p, blocks, sum_dev);
+    CK(cudaGetLastError());
+    EM_LAUNCHED(m, 2);
+    return EM_OK;
+}
+
+int em_assign(em_model* m, const void* X, int64_t n, int64_t* labels, float* dists) {
+    if (!m) return fail(EM_E_INVAL, "model is NULL");
+    if (n < 1 || n >= (1ll << 31)) return fail(EM_E_INVAL, "need 1 <= n < 2^31");
+    CKR(set_device(m));
+    const bool lab_dev = labels && is_device_ptr(labels);
+    const bool dist_dev = dists && is_device_ptr(dists);
+    int64_t* lab_p = nullptr;
+    float* dist_p = nullptr;
+    DBuf<float> dtmp;
+    if (labels) {
+        if (lab_dev) {
+            lab_p = labels;
+        } else {
+            CKR(m->labels64.ensure(n));
+            lab_p = m->labels64.p;
+        }
+    }
+    if (dists) {
+        if (dist_dev) {
+            dist_p = dists;
+        } else {
+            CKR(dtmp.ensure(n));
+            dist_p = dtmp.p;
+        }
+    }
+    DBuf<__nv_bfloat16> tmp;
+    int rc = assign_pass(m, X, n, lab_p, dist_p, m->scalar.p, tmp);
+    if (rc == EM_OK && labels && !lab_dev)
+        rc = cudaMemcpyAsync(labels, lab_p, n * sizeof(int64_t), cudaMemcpyDeviceToHost, m->stream) == cudaSuccess
+                 ? EM_OK
+                 : fail(EM_E_CUDA, "copy of labels failed");
+    if (rc == EM_OK && dists && !dist_dev)
+        rc = cudaMemcpyAsync(dists, dist_p, n * sizeof(float), cudaMemcpyDeviceToHost, m->stream) == cudaSuccess
+                 ? EM_OK
+                 : fail(EM_E_CUDA, "copy of distances failed");
+    if (rc == EM_OK) rc = check_device_errors(m);
+    cudaStreamSynchronize(m->stream);
+    tmp.release();
+    dtmp.release();
+    return rc;
+}
+
+int em_mse(em_model* m, const void* X, int64_t n, double* out) {
+    if (!m || !out) return fail(EM_E_INVAL, "NULL argument");
+    if (n < 1 || n >= (1ll << 31)) return fail(EM_E_INVAL, "need 1 <= n < 2^31");
+    CKR(set_device(m));
+    DBuf<__nv_bfloat16> tmp;
+    int rc = assign_pass(m, X, n, nullptr, nullptr, m->scalar.p, tmp);
+    double s = 0.0;
+    if (rc == EM_OK)
+        rc = cudaMemcpyAsync(&s, m->scalar.p, sizeof(double), cudaMemcpyDeviceToHost, m->stream) == cudaSuccess
+                 ? EM_OK
+                 : fail(EM_E_CUDA, "copy failed");
+    if (rc == EM_OK) rc = check_device_errors(m);
+    cudaStreamSynchronize(m->stream);
+    tmp.release();
+    if (rc == EM_OK) *out = s / (double)n;
+    return rc;
+}
+
+int em_centroids(const em_model* m, float* out) {
+    if (!m || !out) return fail(EM_E_INVAL, "NULL argument");
+    CKR(set_device(m));
+    CK(cudaMemcpy2DAsync(out, m->d * sizeof(float), m->c.p, m->ld * sizeof(float), m->d * sizeof(float), m->k,
+                         cudaMemcpyDefault, m->stream));
+    CK(cudaStreamSynchronize(m->stream));
+    return EM_OK;
+}
+
+int em_labels(const em_model* m, int64_t* out) {
+    if (!m || !out) return fail(EM_E_INVAL, "NULL argument");
+    if (!m->capture || !m->labels_last.p || m->last_was_lloyd) return fail(EM_E_STATE, "no captured labels");
+    CKR(set_device(m));
+    CK(cudaMemcpyAsync(out, m->labels_last.p, m->n * sizeof(int64_t), cudaMemcpyDefault, m->stream));
+    CK(cudaStreamSynchronize(m->stream));
+    return EM_OK;
+}
+
+int em_recipe(const em_model* m, em_recipe_t* out) {
+    if (!m || !out) return fail(EM_E_INVAL, "NULL argument");
+    if (!m->have_run) return fail(EM_E_STATE, "no run started");
+    *out = m->rec;
+    return EM_OK;
+}
+
+int em_stats(const em_model* m, em_stats_t* out) {
+    if (!m || !out) return fail(EM_E_INVAL, "NULL argument");
+    CKR(set_device(m));
+    memset(out, 0, sizeof(*out));
+    out->steps_done = m->t;
+    out->passes_done = m->pass;
+    out->rows_assigned = m->rows_assigned;
+    out->last_alpha = m->last_alpha;
+    int64_t splits = 0;
+    int32_t nd = 0;
+    std::vector<float> N(m->k);
+    CK(cudaMemcpyAsync(&splits, m->rv_splits.p, sizeof(int64_t), cudaMemcpyDeviceToHost, m->stream));
+    CK(cudaMemcpyAsync(&nd, m->rv_ndead.p, sizeof(int32_t), cudaMemcpyDeviceToHost, m->stream));
+    CK(cudaMemcpyAsync(N.data(), m->N.p, m->k * sizeof(float), cudaMemcpyDeviceToHost, m->stream));
+    CK(cudaStreamSynchronize(m->stream));
+    out->n_splits = splits;
+    out->last_dead = nd;
+    double sum = 0.0, mx = 0.0;
+    for (float v : N) {
+        sum += v;
+        mx = std::max(mx, (double)v);
+    }
+    out->imbalance = sum > 0 ? mx / (sum / (double)m->k) : 0.0;
+    return EM_OK;
+}
+
+int em_obj(const em_model* m, double* out, int64_t cap, int64_t* count) {
+    if (!m || (cap > 0 && !out)) return fail(EM_E_INVAL, "NULL argument");
+    if (!m->have_run) return fail(EM_E_STATE, "no run started");
+    CKR(set_device(m));
+    std::vector<double> se(std::max<int64_t>(m->t, 1));
+    if (m->t > 0) {
+        CK(cudaMemcpyAsync(se.data(), m->step_err.p, m->t * sizeof(double), cudaMemcpyDeviceToHost, m->stream));
+        CK(cudaStreamSynchronize(m->stream));
+    }
+    int64_t avail = 0, s = 0;
+    for (int64_t p = 0; p < m->pass; ++p) {
+        const int64_t steps = (p == m->rec.passes - 1) ? m->rec.steps_last_pass : m->rec.steps_full_pass;
+        const int64_t rows = (p == m->rec.passes - 1) ? m->rec.rows_last_pass : m->n;
+        double tot = 0.0;
+        for (int64_t q = 0; q < steps; ++q) tot += se[s + q];
+        s += steps;
+        if (avail < cap) out[avail] = tot / (double)rows;
+        ++avail;
+    }
+    if (count) *count = avail;
+    return EM_OK;
+}
+
+int em_get_state(const em_model* m, float* N, float* S, float* c, int64_t* step) {
+    if (!m) return fail(EM_E_INVAL, "model is NULL");
+    CKR(set_device(m));
+    if (N) CK(cudaMemcpyAsync(N, m->N.p, m->k * sizeof(float), cudaMemcpyDefault, m->stream));
+    if (S)
+        CK(cudaMemcpy2DAsync(S, m->d * sizeof(float), m->S.p, m->ld * sizeof(float), m->d * sizeof(float), m->k,
+                             cudaMemcpyDefault, m->stream));
+    if (c)
+        CK(cudaMemcpy2DAsync(c, m->d * sizeof(float), m->c.p, m->ld * sizeof(float), m->d * sizeof(float), m->k,
+                             cudaMemcpyDefault, m->stream));
+    if (step) *step = m->t;
+    CK(cudaStreamSynchronize(m->stream));
+    return EM_OK;
+}
+
+int em_set_state(em_model* m, const float* N, const float* S, const float* c, int64_t step) {
+    if (!m) return fail(EM_E_INVAL, "model is NULL");
+    if (m->running && (step < 0 || step > m->rec.total_steps)) return fail(EM_E_INVAL, "step out of range");
+    CKR(set_device(m));
+    if (N) CK(cudaMemcpyAsync(m->N.p, N, m->k * sizeof(float), cudaMemcpyDefault, m->stream));
+    if (S)
+        CK(cudaMemcpy2DAsync(m->S.p, m->ld * sizeof(float), S, m->d * sizeof(float), m->d * sizeof(float), m->k,
+                             cudaMemcpyDefault, m->stream));
+    if (c)
+        CK(cudaMemcpy2DAsync(m->c.p, m->ld * sizeof(float), c, m->d * sizeof(float), m->d * sizeof(float), m->k,
+                             cudaMemcpyDefault, m->stream));
+    k_refresh_operand<<<grid_for(m->k * 32, 256, m->sms), 256, 0, m->stream>>>(cluster_state(m), (int)m->k, m->nv);
+    CK(cudaGetLastError());
+    if (m->running) {
+        // move the run's position to `step` (passes are n rows except a fractional last one)
+        m->t = step;
+        m->pass = std::min<int64_t>(step / m->rec.steps_full_pass, m->rec.passes - 1);
+        const int64_t in_pass = step - m->pass * m->rec.steps_full_pass;
+        m->pos = in_pass * m->rec.batch_size;
+    }
+    CK(cudaStreamSynchronize(m->stream));
+    return EM_OK;
+}
+
+int em_last_batch(const em_model* m, int64_t* ids, int64_t* labels, float* dists, int64_t* rows) {
+    if (!m) return fail(EM_E_INVAL, "model is NULL");
+    CKR(set_device(m));
+    const int64_t r = m->last_rows;
+    if (rows) *rows = r;
+    if (r == 0) return EM_OK;
+    std::vector<int32_t> tmp(r);
+    std::vector<int64_t> wide(r);
+    if (ids) {
+        CK(cudaMemcpyAsync(tmp.data(), m->ids.p, r * sizeof(int32_t), cudaMemcpyDeviceToHost, m->stream));
+        CK(cudaStreamSynchronize(m->stream));
+        for (int64_t i = 0; i < r; ++i) wide[i] = tmp[i];
+        CK(cudaMemcpy(ids, wide.data(), r * sizeof(int64_t), cudaMemcpyDefault));
+    }
+    if (labels) {
+        CK(cudaMemcpyAsync(tmp.data(), m->labels.p, r * sizeof(int32_t), cudaMemcpyDeviceToHost, m->stream));
+        CK(cudaStreamSynchronize(m->stream));
+        for (int64_t i = 0; i < r; ++i) wide[i] = tmp[i];
+        CK(cudaMemcpy(labels, wide.data(), r * sizeof(int64_t), cudaMemcpyDefault));
+    }
+    if (dists) {
+        CK(cudaMemcpyAsync(dists, m->dists.p, r * sizeof(float), cudaMemcpyDefault, m->stream));
+        CK(cudaStreamSynchronize(m->stream));
+    }
+    return EM_OK;
+}
+
+int em_profile(em_model* m, em_profile_t* out, int reset) {
+    if (!m) return fail(EM_E_INVAL, "model is NULL");
+    CKR(set_device(m));
+    CK(cudaStreamSynchronize(m->stream));
+    for (auto& sp : m->pending) {
+        float ms = 0.0f;
+        if (cudaEventElapsedTime(&ms, sp.a, sp.b) == cudaSuccess) {
+            m->totals.ms[sp.phase] += ms;
+            m->totals.spans[sp.phase] += 1;
+            if (sp.phase == EM_PHASE_ASSIGN) m->totals.assign_flops += sp.flops;
+            if (sp.phase == EM_PHASE_UPDATE) m->totals.update_bytes += sp.bytes;
+            if (sp.phase == EM_PHASE_GATHER) m->totals.gather_bytes += sp.bytes;
+        } else {
+            cudaGetLastError();
+        }
+        m->pool.push_back(sp.a);
+        m->pool.push_back(sp.b);
+    }
+    m->pending.clear();
+    m->totals.launches = m->launches;
+    if (out) *out = m->totals;
+    if (reset) {
+        m->totals = em_profile_t{};
+        m->launches = 0;
+    }
+    return EM_OK;
+}
+
+int em_sync(em_model* m) {
+    if (!m) return fail(EM_E_INVAL, "model is NULL");
+    CKR(set_device(m));
+    CK(cudaStreamSynchronize(m->stream));
+    return check_device_errors(m);
+}
+
+}  // extern "C"

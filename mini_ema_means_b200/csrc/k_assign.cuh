@@ -1,0 +1,429 @@
+// k_assign.cuh -- fused nearest-centroid search on the sm_100a tensor cores.
+//
+// For each row x of A (bf16) and each centroid operand q_j = -2 bf16(c_j):
+//     score_ij = |bf16(c_j)|^2 + x_i . q_j   (= |x - c_j|^2 - |x|^2)
+// and the row keeps the smallest score with the lowest j (faiss e-means README,
+// "Kernels": the distance computation is fused with the selection of the nearest
+// centroid, so no n x k distance matrix is ever written).
+//
+// Structure of one CTA (192 threads, one CTA per SM, persistent over work units):
+//   warp 0      TMA producer: 128 x KC tiles of A and 256 x KC tiles of the
+//               centroid operand into a STAGES-deep shared-memory ring
+//   warp 1      allocates 512 TMEM columns; one thread issues tcgen05.mma
+//               (M=128, N=256, K=16, bf16 x bf16 -> fp32) into one of two
+//               TMEM accumulators and commits to mbarriers
+//   warps 2..5  epilogue: tcgen05.ld of the 128 x 256 fp32 tile (thread = row),
+//               add |c|^2, running argmin; frees the accumulator for the next tile
+// A work unit is (128-row tile, group of 256-wide centroid tiles). When k is
+// split over several units, the per-row results are merged with a 64-bit
+// atomicMin on (order-preserving score, index) keys.
+#pragma once
+
+#include "common.cuh"
+
+namespace em {
+namespace tc {
+
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int kThreads = 192;
+constexpr int kEpiThreads = 128;
+
+template <int KC>
+struct Cfg {
+    static constexpr int kStages = KC == 64 ? 4 : 8;
+    static constexpr int kABytes = BM * KC * 2;
+    static constexpr int kBBytes = BN * KC * 2;
+    static constexpr int kStageBytes = kABytes + kBBytes;
+    static constexpr uint64_t kLayout = KC == 64 ? 2ull : 4ull;  // UMMA 128B / 64B swizzle
+    static constexpr uint32_t kSBO = 8u * KC * 2u;                // bytes between 8-row groups
+    static constexpr int kBarBytes = 256;
+    static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kBarBytes + 2 * BN * 4;
+};
+
+// Instruction descriptor of tcgen05.mma kind::f16: fp32 accumulate (bits 4-5 = 1),
+// A and B bf16 (bits 7-9 = 1, 10-12 = 1), both K-major (bits 15, 16 = 0),
+// N >> 3 in bits 17-22, M >> 4 in bits 24-28.
+constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
+                            ((uint32_t)(BM >> 4) << 24);
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Waits for the phase of `bar` with the given parity to complete. Gives up after
+// `limit` clock cycles (raising EM_E_TIMEOUT and the CTA-wide abort flag) or as
+// soon as another thread or CTA has raised an error.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, long long limit, int* err,
+                                          volatile int* abort_flag) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const long long t0 = clock64();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 63u) == 0) {
+            if (*abort_flag || error_raised(err)) {
+                *abort_flag = 1;
+                return false;
+            }
+            if (clock64() - t0 > limit) {
+                raise_error(err, EM_E_TIMEOUT);
+                *abort_flag = 1;
+                return false;
+            }
+        }
+    }
+}
+
+// Time-bounded wait used on the error path to let in-flight copies and MMAs land
+// before the CTA releases its shared memory and tensor memory.
+__device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity, long long limit) {
+    const long long t0 = clock64();
+    while (!mbar_try_wait(bar, parity)) {
+        if (clock64() - t0 > limit) return;
+    }
+}
+
+// AND of `ok` over the 128 epilogue threads; doubles as their named barrier 1.
+__device__ __forceinline__ bool epi_all(bool ok) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.and.pred q, 1, 128, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}\n"
+        : "=r"(r)
+        : "r"((uint32_t)ok)
+        : "memory");
+    return r != 0;
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* tm, int x, int y, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+            dst),
+        "l"((uint64_t)tm), "r"(x), "r"(y), "r"(bar)
+        : "memory");
+}
+
+// Shared-memory matrix descriptor (K-major, swizzled): start address >> 4 in bits
+// 0-13, leading byte offset (unused for swizzled K-major, 16 B) in 16-29, stride
+// byte offset between 8-row groups >> 4 in 32-45, descriptor version 1 in bit 46,
+// layout (swizzle mode) in bits 61-63.
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint64_t layout, uint32_t sbo) {
+    return (uint64_t)((addr & 0x3FFFFu) >> 4) | (1ull << 16) | ((uint64_t)(sbo >> 4) << 32) | (1ull << 46) |
+           (layout << 61);
+}
+
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(a), "l"(b), "r"(kIdesc), "r"(accumulate)
+        : "memory");
+}
+
+__device__ __forceinline__ void umma_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+template <int KC>
+__global__ void __launch_bounds__(kThreads, 1)
+    k_assign_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                const float* __restrict__ cn, int k, int rows, int nkc, int n_tiles, int n_split,
+                unsigned long long* __restrict__ keys, long long wait_limit, int* err) {
+    using C = Cfg<KC>;
+    constexpr int S = C::kStages;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sA = smem;
+    uint8_t* sB = smem + S * C::kABytes;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::kStageBytes);
+    uint64_t* full = bars;
+    uint64_t* empty = bars + S;
+    uint64_t* tfull = bars + 2 * S;
+    uint64_t* tempty = bars + 2 * S + 2;
+    uint64_t* drain = bars + 2 * S + 4;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 5);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    float* cn_s = reinterpret_cast<float*>(smem + S * C::kStageBytes + C::kBarBytes);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    // the error-path drains get at least ~2 s whatever limit the caller chose
+    const long long drain_limit = wait_limit > 4000000000ll ? wait_limit : 4000000000ll;
+    const int m_tiles = (rows + BM - 1) / BM;
+    const int tpg = (n_tiles + n_split - 1) / n_split;
+    const int units = m_tiles * n_split;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(smem_u32(&full[s]), 1);
+            mbar_init(smem_u32(&empty[s]), 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(smem_u32(&tfull[a]), 1);
+            mbar_init(smem_u32(&tempty[a]), kEpiThreads);
+        }
+        mbar_init(smem_u32(drain), 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                     "r"(512u)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    if (warp == 0 && lane == 0) {
+        asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&tmA) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&tmB) : "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        // ---------------- TMA producer
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            uint32_t armed = 0, armed_parity = 0;  // per-stage bit masks
+            for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+                const int m = u / n_split, g = u - m * n_split;
+                const int nt0 = g * tpg, nt1 = min(nt0 + tpg, n_tiles);
+                for (int nt = nt0; nt < nt1 && ok; ++nt) {
+                    for (int kc = 0; kc < nkc; ++kc) {
+                        if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, wait_limit, err, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        const uint32_t fb = smem_u32(&full[stage]);
+                        armed |= 1u << stage;
+                        armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+                        mbar_expect_tx(fb, C::kStageBytes);
+                        tma_load_2d(smem_u32(sA + stage * C::kABytes), &tmA, kc * KC, m * BM, fb);
+                        tma_load_2d(smem_u32(sB + stage * C::kBBytes), &tmB, kc * KC, nt * BN, fb);
+                        if (++stage == S) {
+                            stage = 0;
+                            phase ^= 1u;
+                        }
+                    }
+                }
+            }
+            if (!ok) {  // let every copy this thread started land before shared memory is released
+                for (int s2 = 0; s2 < S; ++s2)
+                    if (armed & (1u << s2)) mbar_drain(smem_u32(&full[s2]), (armed_parity >> s2) & 1u, drain_limit);
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issuer (one thread)
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int acc = 0;
+            uint32_t acc_phase = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+                const int m = u / n_split, g = u - m * n_split;
+                (void)m;
+                const int nt0 = g * tpg, nt1 = min(nt0 + tpg, n_tiles);
+                for (int nt = nt0; nt < nt1 && ok; ++nt) {
+                    if (!mbar_wait(smem_u32(&tempty[acc]), acc_phase ^ 1u, wait_limit, err, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+                    for (int kc = 0; kc < nkc; ++kc) {
+                        if (!mbar_wait(smem_u32(&full[stage]), phase, wait_limit, err, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint32_t a0 = smem_u32(sA + stage * C::kABytes);
+                        const uint32_t b0 = smem_u32(sB + stage * C::kBBytes);
+#pragma unroll
+                        for (int kk = 0; kk < KC / 16; ++kk) {
+                            const uint64_t ad = smem_desc(a0 + kk * 32, C::kLayout, C::kSBO);
+                            const uint64_t bd = smem_desc(b0 + kk * 32, C::kLayout, C::kSBO);
+                            umma_bf16(d_tmem, ad, bd, (kc | kk) != 0);
+                        }
+                        umma_commit(smem_u32(&empty[stage]));
+                        if (++stage == S) {
+                            stage = 0;
+                            phase ^= 1u;
+                        }
+                    }
+                    if (!ok) break;
+                    umma_commit(smem_u32(&tfull[acc]));
+                    acc ^= 1;
+                    if (acc == 0) acc_phase ^= 1u;
+                }
+            }
+            if (!ok) {  // wait for every MMA this thread issued before TMEM is freed
+                umma_commit(smem_u32(drain));
+                mbar_drain(smem_u32(drain), 0u, drain_limit);
+            }
+        }
+    } else {
+        // ---------------- epilogue: 4 warps, thread = accumulator row
+        const int et = threadIdx.x - 64;
+        const int q = warp & 3;
+        const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        int cnbuf = 0;
+        bool ok = true;
+        for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+            const int m = u / n_split, g = u - m * n_split;
+            const int nt0 = g * tpg, nt1 = min(nt0 + tpg, n_tiles);
+            float best = __int_as_float(0x7f800000);  // +inf
+            int bidx = 0;
+            for (int nt = nt0; nt < nt1; ++nt) {
+                float* cnb = cn_s + cnbuf * BN;
+                const int j0 = nt * BN;
+                cnb[et] = (j0 + et < k) ? cn[j0 + et] : __int_as_float(0x7f800000);
+                cnb[et + 128] = (j0 + et + 128 < k) ? cn[j0 + et + 128] : __int_as_float(0x7f800000);
+                const bool got = mbar_wait(smem_u32(&tfull[acc]), acc_phase, wait_limit, err, abort_flag);
+                // one decision for all 128 threads (so none is left at a barrier), and the
+                // barrier that publishes this tile's |c|^2 values
+                if (!epi_all(got)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                __syncwarp();
+                const uint32_t tbase = tmem_base + lane_base + (uint32_t)(acc * BN);
+#pragma unroll 1
+                for (int ch = 0; ch < BN / 32; ch += 2) {
+                    uint32_t v0[32], v1[32];
+                    tmem_ld32(tbase + ch * 32, v0);
+                    tmem_ld32(tbase + ch * 32 + 32, v1);
+                    tmem_wait_ld();
+                    const float4* c4 = reinterpret_cast<const float4*>(cnb + ch * 32);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const float4 cc = c4[i];
+                        const float s0 = cc.x + __uint_as_float(v0[4 * i + 0]);
+                        const float s1 = cc.y + __uint_as_float(v0[4 * i + 1]);
+                        const float s2 = cc.z + __uint_as_float(v0[4 * i + 2]);
+                        const float s3 = cc.w + __uint_as_float(v0[4 * i + 3]);
+                        const int jb = j0 + ch * 32 + 4 * i;
+                        if (s0 < best) { best = s0; bidx = jb; }
+                        if (s1 < best) { best = s1; bidx = jb + 1; }
+                        if (s2 < best) { best = s2; bidx = jb + 2; }
+                        if (s3 < best) { best = s3; bidx = jb + 3; }
+                    }
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const float4 cc = c4[8 + i];
+                        const float s0 = cc.x + __uint_as_float(v1[4 * i + 0]);
+                        const float s1 = cc.y + __uint_as_float(v1[4 * i + 1]);
+                        const float s2 = cc.z + __uint_as_float(v1[4 * i + 2]);
+                        const float s3 = cc.w + __uint_as_float(v1[4 * i + 3]);
+                        const int jb = j0 + ch * 32 + 32 + 4 * i;
+                        if (s0 < best) { best = s0; bidx = jb; }
+                        if (s1 < best) { best = s1; bidx = jb + 1; }
+                        if (s2 < best) { best = s2; bidx = jb + 2; }
+                        if (s3 < best) { best = s3; bidx = jb + 3; }
+                    }
+                }
+                tc_fence_before();
+                mbar_arrive(smem_u32(&tempty[acc]));
+                acc ^= 1;
+                if (acc == 0) acc_phase ^= 1u;
+                cnbuf ^= 1;
+            }
+            if (!ok) break;
+            const int row = m * BM + 32 * q + lane;
+            if (row < rows) {
+                const unsigned long long key = pack_key(best, (uint32_t)bidx);
+                if (n_split > 1)
+                    atomicMin(&keys[row], key);
+                else
+                    keys[row] = key;
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(512u) : "memory");
+    }
+}
+
+}  // namespace tc
+
+// Plain SIMT search (one thread per row, fp32 FMA over bf16 operands). Not used
+// by training unless selected explicitly; it exists to tell a tensor-core fault
+// apart from a fault elsewhere in the step when a parity test fails.
+__global__ void k_assign_simt(const __nv_bfloat16* __restrict__ A, int ld, int rows, const __nv_bfloat16* __restrict__ cq,
+                              const float* __restrict__ cn, int k, int d, unsigned long long* __restrict__ keys) {
+    const int row = blockIdx.x * blockDim.x + threadIdx.x;
+    if (row >= rows) return;
+    const __nv_bfloat16* x = A + (int64_t)row * ld;
+    float best = __int_as_float(0x7f800000);
+    int bidx = 0;
+    for (int j = 0; j < k; ++j) {
+        const __nv_bfloat16* q = cq + (int64_t)j * ld;
+        float acc = 0.0f;
+        for (int e = 0; e < d; ++e) acc = fmaf(__bfloat162float(x[e]), __bfloat162float(q[e]), acc);
+        const float s = cn[j] + acc;
+        if (s < best) {
+            best = s;
+            bidx = j;
+        }
+    }
+    keys[row] = pack_key(best, (uint32_t)bidx);
+}
+
+}  // namespace em

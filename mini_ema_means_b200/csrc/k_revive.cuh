@@ -1,0 +1,348 @@
+// k_revive.cuh -- dead-cluster revival, run after every 5th step.
+//
+// faiss e-means README (`unused_threshold`, "How the centroid updates work") and
+// the jecision.com essay ("Three: dead clusters must be revived"): a cluster
+// whose running count N_j falls below tau times the mean count is revived by
+// splitting a busy cluster in two, the busy cluster being drawn with probability
+// proportional to its size. Readings fixed here:
+//   * the dead set D is fixed before any split; dead clusters are served in
+//     increasing index; each draws its donor among the clusters outside D with
+//     probability proportional to their CURRENT N (a donor halved earlier in the
+//     same check is lighter), with u = Philox(seed, stream 3, t, j);
+//   * split: N_j = N_d / 2, N_d <- N_d / 2, c_j = c_d (1 - eps s),
+//     c_d <- c_d (1 + eps s) with s_i = +1 (even i), -1 (odd i), eps = 2^-10,
+//     and S = N c for both;
+//   * resample (the EnCodec-style arm of the ablation): c_j <- a row of the
+//     current batch drawn with Philox(seed, stream 4, t, j), N_j = S_j = 0.
+//
+// The draws are inherently sequential, so one warp makes them on an fp64 tree
+// of prefix sums (32 children per node: one coalesced load, one ballot per
+// level, and a halving updates one suffix of each level with one lane-parallel
+// subtraction). The vector work is then done in parallel from the closed form:
+// the o-th split taken from donor d (0-based) sees c_d (1 + eps s)^o and N_d / 2^o.
+#pragma once
+
+#include "k_reduce.cuh"
+
+namespace em {
+
+struct ReviveScratch {
+    int32_t* dead;    // k: dead clusters in increasing order
+    int32_t* donor;   // k: donor of each dead cluster (-1 if none)
+    int32_t* order;   // k: how many earlier splits took this donor in this check
+    int32_t* times;   // k: splits taken from each donor in this check
+    double* tree;     // prefix-sum levels that do not fit in shared memory (tree_layout(k).total)
+    int32_t* ndead;   // 1: |D| of the most recent check
+    int64_t* n_splits;  // 1: cumulative number of revived clusters
+};
+
+struct TreeLayout {
+    int levels;
+    int size[8];
+    int64_t offset[8];
+    int64_t total;
+};
+
+// Shared memory the selection kernel may use for the tree (doubles).
+constexpr int kReviveSmemDoubles = 24 * 1024;
+
+EM_HD TreeLayout tree_layout(int k) {
+    TreeLayout L{};
+    int s = k;
+    int64_t off = 0;
+    L.levels = 0;
+    while (true) {
+        L.size[L.levels] = s;
+        L.offset[L.levels] = off;
+        off += ((s + 31) / 32) * 32;
+        ++L.levels;
+        if (s <= 32 || L.levels == 8) break;
+        s = (s + 31) / 32;
+    }
+    L.total = off;
+    return L;
+}
+
+// 0: every level in shared memory; 1: leaves in global memory, the rest shared;
+// 2: every level in global memory.
+EM_HD int tree_placement(const TreeLayout& L) {
+    if (L.total <= kReviveSmemDoubles) return 0;
+    if (L.levels > 1 && L.total - L.offset[1] <= kReviveSmemDoubles) return 1;
+    return 2;
+}
+
+EM_HD int64_t tree_smem_bytes(const TreeLayout& L) {
+    const int p = tree_placement(L);
+    return p == 0 ? L.total * 8 : p == 1 ? (L.total - L.offset[1]) * 8 : 0;
+}
+
+__device__ __forceinline__ double warp_incl_scan(double v, int lane) {
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const double t = __shfl_up_sync(0xFFFFFFFFu, v, o);
+        if (lane >= o) v += t;
+    }
+    return v;
+}
+
+// One CTA of 1024 threads: dead set, tree, sequential donor draws.
+__global__ void __launch_bounds__(1024) k_revive_select(const float* __restrict__ N, int k, double tau, uint64_t seed,
+                                                        int64_t t, int mode, ReviveScratch sc, int* err) {
+    __shared__ double red[32];
+    __shared__ int32_t wcount[32];
+    __shared__ int32_t base_s;
+    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+
+    // total count in a fixed order
+    double part = 0.0;
+    for (int j = tid; j < k; j += 1024) part += (double)N[j];
+    part = warp_sum(part);
+    if (lane == 0) red[w] = part;
+    __syncthreads();
+    if (w == 0) {
+        double v = warp_sum(red[lane]);
+        if (lane == 0) red[0] = v;
+    }
+    __syncthreads();
+    const double total = red[0];
+    const double mean = total / (double)k;
+    const double thr = tau * mean;
+
+    // dead set, compacted in increasing index
+    if (tid == 0) base_s = 0;
+    __syncthreads();
+    for (int b = 0; b < k; b += 1024) {
+        const int j = b + tid;
+        const bool dead = j < k && (double)N[j] < thr;
+        if (j < k) sc.times[j] = 0;
+        const unsigned m = __ballot_sync(0xFFFFFFFFu, dead);
+        if (lane == 0) wcount[w] = __popc(m);
+        __syncthreads();
+        if (w == 0) {
+            const int c = wcount[lane];
+            int incl = c;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int tt = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+                if (lane >= o) incl += tt;
+            }
+            wcount[lane] = incl - c;
+        }
+        __syncthreads();
+        if (dead) sc.dead[base_s + wcount[w] + __popc(m & ((1u << lane) - 1u))] = j;
+        __syncthreads();
+        if (tid == 1023) base_s += wcount[31] + __popc(m);
+        __syncthreads();
+    }
+    const int nd = base_s;
+    if (tid == 0) *sc.ndead = nd;
+    if (mode != EM_REVIVE_SPLIT || nd == 0 || !(total > 0.0)) {
+        for (int i = tid; i < nd; i += 1024) sc.donor[i] = -1;
+        return;
+    }
+
+    // prefix tree over the weights of the eligible clusters (dead ones weigh 0);
+    // all levels in shared memory when they fit, else level 0 in global memory
+    extern __shared__ double stree[];
+    const TreeLayout L = tree_layout(k);
+    double* levp[8];
+    const int placement = tree_placement(L);
+    for (int l = 0; l < L.levels; ++l) {
+        if (placement == 0 || (placement == 1 && l > 0))
+            levp[l] = stree + (L.offset[l] - (placement == 0 ? 0 : L.offset[1]));
+        else
+            levp[l] = sc.tree + L.offset[l];
+    }
+    for (int l = 0; l < L.levels; ++l) {
+        const int sz = L.size[l];
+        double* lev = levp[l];
+        const int ngroups = (sz + 31) / 32;
+        for (int gidx = w; gidx < ngroups; gidx += 32) {
+            const int i = gidx * 32 + lane;
+            double v = 0.0;
+            if (i < sz) {
+                if (l == 0) {
+                    const float nj = N[i];
+                    v = ((double)nj < thr) ? 0.0 : (double)nj;
+                } else {
+                    v = levp[l - 1][i * 32 + 31];  // total of child group i (its last prefix)
+                }
+            }
+            lev[gidx * 32 + lane] = warp_incl_scan(v, lane);
+        }
+        __syncthreads();
+    }
+
+    // sequential draws by warp 0
+    if (w == 0) {
+        const int top = L.levels - 1;
+        double W = levp[top][31];
+        bool exhausted = false;
+        for (int i = 0; i < nd; ++i) {
+            const int j = sc.dead[i];
+            if (exhausted || !(W > 0.0)) {
+                exhausted = true;
+                if (lane == 0) sc.donor[i] = -1;
+                continue;
+            }
+            double target = draw_uniform(seed, kStreamRevive, t, j) * W;
+            int node = 0;
+            for (int l = top; l >= 0; --l) {
+                const int base = node * 32;
+                const double* lev = levp[l];
+                const bool valid = base + lane < L.size[l];
+                const double P = valid ? lev[base + lane] : 0.0;
+                const double Pprev = __shfl_up_sync(0xFFFFFFFFu, P, 1);
+                const double prev_incl = lane == 0 ? 0.0 : Pprev;
+                const unsigned above = __ballot_sync(0xFFFFFFFFu, valid && P > target);
+                int c;
+                if (above) {
+                    c = __ffs(above) - 1;
+                } else {  // target rounded onto the total: take the last child with weight
+                    const unsigned pos = __ballot_sync(0xFFFFFFFFu, valid && P > prev_incl);
+                    c = pos ? 31 - __clz(pos) : 0;
+                }
+                const double before = __shfl_sync(0xFFFFFFFFu, prev_incl, c);
+                target -= before;
+                node = base + c;
+            }
+            const int dn = node;
+            int old = 0;
+            if (lane == 0) {
+                old = sc.times[dn];
+                sc.times[dn] = old + 1;
+                sc.donor[i] = dn;
+                sc.order[i] = old;
+            }
+            old = __shfl_sync(0xFFFFFFFFu, old, 0);
+            if (dn < 0 || dn >= k) raise_error(err, EM_E_BOUNDS);
+            const double delta = ldexp((double)N[dn], -(old + 1));  // half of its current weight
+            int idx = dn;
+            for (int l = 0; l < L.levels; ++l) {
+                const int gb = (idx >> 5) << 5;
+                double* lev = levp[l];
+                if (gb + lane >= idx && gb + lane < L.size[l]) lev[gb + lane] -= delta;
+                idx >>= 5;
+            }
+            W -= delta;
+            __syncwarp();
+        }
+        if (lane == 0) {
+            int done = 0;
+            for (int i = 0; i < nd; ++i) done += sc.donor[i] >= 0;
+            *sc.n_splits += done;
+        }
+    }
+}
+
+// Dead clusters take their half of the donor (reads the donors' state before
+// k_revive_donors changes it).
+__global__ void k_revive_dead(ClusterState st, int nv, ReviveScratch sc) {
+    const int lane = threadIdx.x & 31;
+    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int nwarps = (gridDim.x * blockDim.x) >> 5;
+    const int nd = *sc.ndead;
+    for (int i = warp; i < nd; i += nwarps) {
+        const int dn = sc.donor[i];
+        if (dn < 0) continue;
+        const int j = sc.dead[i];
+        const int o = sc.order[i];
+        const float Nj = ldexpf(st.N[dn], -(o + 1));
+        float cn_part = 0.0f;
+        for (int v = lane; v < nv; v += 32) {
+            const float4* cr = reinterpret_cast<const float4*>(st.c + (int64_t)dn * st.ld) + 2 * v;
+            const float4 a = cr[0], b = cr[1];
+            float cv[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+            float sv[8];
+#pragma unroll
+            for (int tt = 0; tt < 8; ++tt) {
+                const float sg = ((8 * v + tt) & 1) ? -1.0f : 1.0f;
+                float x = cv[tt];
+                for (int r = 0; r < o; ++r) x *= (1.0f + kSplitEps * sg);
+                x *= (1.0f - kSplitEps * sg);
+                cv[tt] = x;
+                sv[tt] = Nj * x;
+            }
+            store_centroid_vec(st.c + (int64_t)j * st.ld, st.cq + (int64_t)j * st.ld, v, cv, cn_part);
+            float4* sr = reinterpret_cast<float4*>(st.S + (int64_t)j * st.ld) + 2 * v;
+            sr[0] = make_float4(sv[0], sv[1], sv[2], sv[3]);
+            sr[1] = make_float4(sv[4], sv[5], sv[6], sv[7]);
+        }
+        cn_part = warp_sum(cn_part);
+        if (lane == 0) {
+            st.N[j] = Nj;
+            st.cn[j] = cn_part;
+        }
+    }
+}
+
+// Each donor, once, after all its splits: c_d (1 + eps s)^m, N_d / 2^m, S = N c.
+__global__ void k_revive_donors(ClusterState st, int nv, ReviveScratch sc) {
+    const int lane = threadIdx.x & 31;
+    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int nwarps = (gridDim.x * blockDim.x) >> 5;
+    const int nd = *sc.ndead;
+    for (int i = warp; i < nd; i += nwarps) {
+        const int dn = sc.donor[i];
+        if (dn < 0) continue;
+        const int m = sc.times[dn];
+        if (sc.order[i] != m - 1) continue;  // only the last split of this donor acts
+        const float Nd = ldexpf(st.N[dn], -m);
+        float cn_part = 0.0f;
+        for (int v = lane; v < nv; v += 32) {
+            float4* cr = reinterpret_cast<float4*>(st.c + (int64_t)dn * st.ld) + 2 * v;
+            const float4 a = cr[0], b = cr[1];
+            float cv[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+            float sv[8];
+#pragma unroll
+            for (int tt = 0; tt < 8; ++tt) {
+                const float sg = ((8 * v + tt) & 1) ? -1.0f : 1.0f;
+                float x = cv[tt];
+                for (int r = 0; r < m; ++r) x *= (1.0f + kSplitEps * sg);
+                cv[tt] = x;
+                sv[tt] = Nd * x;
+            }
+            store_centroid_vec(st.c + (int64_t)dn * st.ld, st.cq + (int64_t)dn * st.ld, v, cv, cn_part);
+            float4* sr = reinterpret_cast<float4*>(st.S + (int64_t)dn * st.ld) + 2 * v;
+            sr[0] = make_float4(sv[0], sv[1], sv[2], sv[3]);
+            sr[1] = make_float4(sv[4], sv[5], sv[6], sv[7]);
+        }
+        cn_part = warp_sum(cn_part);
+        if (lane == 0) {
+            st.N[dn] = Nd;
+            st.cn[dn] = cn_part;
+        }
+    }
+}
+
+// Resample arm: each dead cluster restarts from a row of the current batch.
+__global__ void k_revive_resample(ClusterState st, int nv, ReviveScratch sc, const __nv_bfloat16* __restrict__ Xb,
+                                  int rows, uint64_t seed, int64_t t) {
+    const int lane = threadIdx.x & 31;
+    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int nwarps = (gridDim.x * blockDim.x) >> 5;
+    const int nd = *sc.ndead;
+    for (int i = warp; i < nd; i += nwarps) {
+        const int j = sc.dead[i];
+        const double u = draw_uniform(seed, kStreamResample, t, j);
+        int r = (int)floor(u * (double)rows);
+        if (r > rows - 1) r = rows - 1;
+        float cn_part = 0.0f;
+        for (int v = lane; v < nv; v += 32) {
+            float x[8];
+            unpack8_bf16(reinterpret_cast<const uint4*>(Xb + (int64_t)r * st.ld)[v], x);
+            store_centroid_vec(st.c + (int64_t)j * st.ld, st.cq + (int64_t)j * st.ld, v, x, cn_part);
+            float4* sr = reinterpret_cast<float4*>(st.S + (int64_t)j * st.ld) + 2 * v;
+            sr[0] = make_float4(0, 0, 0, 0);
+            sr[1] = make_float4(0, 0, 0, 0);
+        }
+        cn_part = warp_sum(cn_part);
+        if (lane == 0) {
+            st.N[j] = 0.0f;
+            st.cn[j] = cn_part;
+        }
+    }
+    if (blockIdx.x == 0 && threadIdx.x == 0) *sc.n_splits += nd;
+}
+
+}  // namespace em

@@ -1,0 +1,139 @@
+"""Comparison helpers for the GPU parity tests (CUDA path through the C ABI vs the oracle).
+
+Tolerances (stated once, used by every parity test):
+* labels: bit-exact, except rows whose best-vs-second squared-distance gap is
+  below 1e-3 of the best distance (a near tie under the fp32 accumulation of the
+  tensor cores vs the fp64 oracle); such rows may hold the other near-tied label
+  and may number at most max(1, 1e-4 x rows compared);
+* centroids: relative L2 error per centroid <= 1e-3;
+* MSE: relative error <= 1e-3 (0.1 %).
+"""
+
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from oracle import emeans_oracle as O
+
+LABEL_GAP_REL = 1e-3
+LABEL_MISMATCH_FRACTION = 1e-4
+CENTROID_REL = 1e-3
+MSE_REL = 1e-3
+
+
+class LabelBook:
+    """Accumulates label comparisons over several batches."""
+
+    def __init__(self):
+        self.rows = 0
+        self.mismatch = 0
+
+    def compare(self, gpu_labels, xq_rows, cq):
+        """Checks GPU labels against the oracle's search with search copies cq.
+
+        Returns the accepted labels: the oracle's, except where the GPU picked
+        another label of a near tie (both are correct there)."""
+        gpu_labels = np.asarray(gpu_labels, dtype=np.int64)
+        lab, best, second = O.assign(xq_rows, cq)
+        diff = np.flatnonzero(gpu_labels != lab)
+        if len(diff):
+            d_gpu = ((xq_rows[diff] - cq[gpu_labels[diff]]) ** 2).sum(axis=1)
+            ok = (d_gpu - best[diff]) <= LABEL_GAP_REL * np.maximum(best[diff], 1e-30)
+            ok &= (second[diff] - best[diff]) < LABEL_GAP_REL * np.maximum(best[diff], 1e-30)
+            assert ok.all(), f"{(~ok).sum()} labels differ from the oracle outside near ties"
+        self.rows += len(lab)
+        self.mismatch += len(diff)
+        accepted = lab.copy()
+        accepted[diff] = gpu_labels[diff]
+        return accepted, best
+
+    def finish(self):
+        allowed = max(1, int(LABEL_MISMATCH_FRACTION * self.rows))
+        assert self.mismatch <= allowed, f"{self.mismatch} near-tie label flips in {self.rows} rows (max {allowed})"
+
+
+def centroid_rel_err(c_gpu, c_ref):
+    c_gpu = np.asarray(c_gpu, dtype=np.float64)
+    num = np.linalg.norm(c_gpu - c_ref, axis=1)
+    den = np.maximum(np.linalg.norm(c_ref, axis=1), 1e-30)
+    return num / den
+
+
+def assert_centroids_close(c_gpu, c_ref, what="centroids"):
+    rel = centroid_rel_err(c_gpu, c_ref)
+    assert rel.max() <= CENTROID_REL, f"{what}: max relative L2 error {rel.max():.3e} at {int(rel.argmax())}"
+    return rel.max()
+
+
+def gpu_state(m, k, d):
+    N = torch.empty(k)
+    S = torch.empty(k, d)
+    c = torch.empty(k, d)
+    step = m.get_state(N=N, S=S, c=c)
+    return N.numpy().astype(np.float64), S.numpy().astype(np.float64), c.numpy().astype(np.float64), step
+
+
+def gpu_last_batch(m, rows):
+    ids = torch.empty(rows, dtype=torch.int64)
+    labels = torch.empty(rows, dtype=torch.int64)
+    dists = torch.empty(rows, dtype=torch.float32)
+    r = m.last_batch(ids=ids, labels=labels, dists=dists)
+    return ids.numpy()[:r], labels.numpy()[:r], dists.numpy()[:r].astype(np.float64)
+
+
+def teacher_forced_run(m, orc, x_dev, xq, epochs, revival, check_every=1, max_steps=None):
+    """Runs the GPU model step by step; before each checked step the oracle is
+    given the GPU's state, takes the same step and both results are compared.
+    Returns a summary dict."""
+    import mini_ema_means_b200 as em  # noqa: F401
+
+    k, d = orc.k, orc.d
+    rec = m.begin(x_dev, epochs=epochs)
+    r_or = orc.begin(xq, epochs)
+    assert rec["batch_size"] == r_or["batch_size"] and rec["total_steps"] == r_or["total_steps"]
+    assert abs(rec["alpha0"] - r_or["alpha0"]) <= 1e-12 * r_or["alpha0"]
+    N, S, c, _ = gpu_state(m, k, d)
+    assert np.array_equal(c, orc.c), "starting centroids differ from the oracle's rows"
+    book = LabelBook()
+    worst = {"N": 0.0, "c": 0.0, "dist": 0.0, "revive_c": 0.0}
+    total = rec["total_steps"] if max_steps is None else min(max_steps, rec["total_steps"])
+    revivals = 0
+    for t in range(total):
+        check = (t % check_every == 0) or t == total - 1 or (t + 1) % 5 == 0
+        if check:
+            N0, S0, c0, step = gpu_state(m, k, d)
+            assert step == t
+            orc.N, orc.S, orc.c = N0, S0, c0
+        ids_expected = orc.next_batch_ids()
+        assert m.step(1) == 1
+        ids, labels, dists = gpu_last_batch(m, rec["batch_size"])
+        assert np.array_equal(ids, ids_expected), f"step {t}: batch rows differ from the oracle's order"
+        if check:
+            accepted, best = book.compare(labels, xq[ids], O.search_copy_of_centroids(orc.c))
+            tol = 1e-5 * (np.einsum("ij,ij->i", xq[ids], xq[ids]) + best) + 1e-6
+            worst["dist"] = max(worst["dist"], float(np.max(np.abs(dists - best) / tol)))
+            assert np.all(np.abs(dists - best) <= tol), f"step {t}: distances differ"
+            orc.step(forced_labels=accepted, auto_revive=False)
+            N1, S1, c1, _ = gpu_state(m, k, d)
+            np.testing.assert_allclose(N1, orc.N, rtol=2e-6, atol=1e-30)
+            worst["c"] = max(worst["c"], assert_centroids_close(c1, orc.c, f"step {t} centroids"))
+            rel_s = centroid_rel_err(S1, orc.S)
+            assert rel_s[orc.N > 0].max(initial=0) <= CENTROID_REL
+        else:
+            orc.step(forced_labels=labels, auto_revive=False)
+        if (t + 1) % 5 == 0 and revival != "none":
+            N1, S1, c1, _ = gpu_state(m, k, d)
+            m.revive()
+            N2, S2, c2, _ = gpu_state(m, k, d)
+            orc.N, orc.S, orc.c = N1, S1, c1
+            res = orc.maybe_revive(xq[ids], t=t)
+            if res is not None and len(res[0]):
+                revivals += len(res[0])
+            # counts after a revival are exact halvings (or zero): equal to the bit
+            np.testing.assert_array_equal(N2, orc.N)
+            worst["revive_c"] = max(worst["revive_c"], assert_centroids_close(c2, orc.c, f"step {t} revival"))
+            st = m.stats()
+            assert st["last_dead"] == (0 if res is None else len(res[0]))
+    book.finish()
+    return dict(worst=worst, mismatches=book.mismatch, rows=book.rows, revived=revivals)

@@ -1,0 +1,209 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle.
+
+Teacher-forced runs give the oracle the GPU's state before every step and compare
+the batch order (bit-exact), labels (near-tie rule), distances, running counts,
+sums, centroids, revivals and the closing mean. Tolerances: tests/helpers.py.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from datagen import synth
+import datagen
+from oracle import emeans_oracle as O
+from tests.helpers import (CENTROID_REL, MSE_REL, LabelBook, assert_centroids_close, centroid_rel_err, gpu_state,
+                           teacher_forced_run)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def em():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    import mini_ema_means_b200
+
+    return mini_ema_means_b200
+
+
+def _finish_and_compare(m, orc, n, xq):
+    m.finalize()
+    orc.finalize()
+    _, _, c, _ = gpu_state(m, orc.k, orc.d)
+    assert_centroids_close(c, orc.c, "closing mean")
+    if m.get_option("capture_labels"):
+        lab = torch.empty(n, dtype=torch.int64)
+        m.labels(lab)
+        assert np.array_equal(lab.numpy(), orc.labels_last)
+    return c
+
+
+def test_smoke_entry_point():
+    import __graft_entry__
+
+    __graft_entry__.smoke()
+
+
+@pytest.mark.parametrize("revival", ["split", "resample", "none"])
+def test_tiny_teacher_forced_every_step(em, revival):
+    w, xt, _ = datagen.make("tiny")
+    xq = O.search_copy_of_data(xt.numpy())
+    m = em.Model(w.d, w.k, seed=1234, auto_revive=0, revival=revival)
+    orc = O.EmeansOracle(w.d, w.k, seed=1234, revival=revival)
+    res = teacher_forced_run(m, orc, xt.cuda(), xq, w.epochs, revival)
+    assert res["rows"] == 5 * w.n_train
+    if revival != "none":
+        assert res["revived"] > 0
+    _finish_and_compare(m, orc, w.n_train, xq)
+    obj = m.obj()
+    assert len(obj) == 5
+
+
+@pytest.mark.parametrize("n,d,k,epochs,batch,revival", [
+    (3000, 16, 40, 2.0, None, "split"),
+    (5000, 96, 300, 1.5, 512, "split"),
+    (2000, 128, 513, 2.0, 256, "split"),
+    (1500, 768, 64, 1.0, 256, "split"),
+    (4097, 40, 100, 1.25, 300, "resample"),
+    (1000, 8, 1, 1.0, 100, "split"),
+    (2600, 264, 257, 1.5, None, "split"),
+    (3333, 100, 77, 1.0, 1000, "none"),
+])
+def test_hand_shapes_teacher_forced(em, n, d, k, epochs, batch, revival):
+    x = synth.hand_shape(n, d, max(2, k // 2), seed=n + d)
+    xq = O.search_copy_of_data(x.numpy())
+    opts = dict(auto_revive=0, revival=revival)
+    if batch:
+        opts["batch_size"] = batch
+    m = em.Model(d, k, seed=7, **opts)
+    orc = O.EmeansOracle(d, k, seed=7, revival=revival, batch_size=batch)
+    teacher_forced_run(m, orc, x.cuda(), xq, epochs, revival)
+    _finish_and_compare(m, orc, n, xq)
+
+
+def test_bf16_input_in_place_and_padded(em):
+    for d in (64, 36):  # 16-byte rows are used in place; others are copied with padding
+        x = synth.hand_shape(2500, d, 20, seed=d, storage="bf16")
+        xq = x.to(torch.float64).numpy()
+        m = em.Model(d, 30, seed=3, auto_revive=0)
+        orc = O.EmeansOracle(d, 30, seed=3)
+        teacher_forced_run(m, orc, x.cuda(), xq, 1.0, "split")
+        _finish_and_compare(m, orc, 2500, xq)
+
+
+def test_host_input_goes_through_the_same_path(em):
+    x = synth.hand_shape(3000, 32, 16, seed=11)
+    m1 = em.Model(32, 24, seed=5)
+    m1.train(x.cuda(), epochs=2.0)
+    m2 = em.Model(32, 24, seed=5)
+    m2.train(x.contiguous(), epochs=2.0)  # host tensor: copied to the device inside the call
+    c1, c2 = torch.empty(24, 32), torch.empty(24, 32)
+    m1.centroids(c1)
+    m2.centroids(c2)
+    assert torch.equal(c1, c2)
+
+
+@pytest.mark.parametrize("n,d,k", [(1, 32, 1), (127, 64, 5), (129, 96, 257), (5000, 768, 4096),
+                                   (3000, 128, 600), (777, 100, 300), (20000, 32, 64), (4100, 256, 2048)])
+def test_assign_and_mse_match_oracle(em, n, d, k):
+    g = torch.Generator().manual_seed(n * 31 + k)
+    x = synth.hand_shape(n, d, 16, seed=n + k)
+    c = (x[torch.randint(0, n, (k,), generator=g)] + 0.3 * torch.randn(k, d, generator=g)).float()
+    m = em.Model(d, k, seed=1)
+    m.set_state(c=c)
+    labels = torch.empty(n, dtype=torch.int64, device="cuda")
+    dists = torch.empty(n, dtype=torch.float32, device="cuda")
+    m.assign(x.cuda(), labels=labels, dists=dists)
+    xq = O.search_copy_of_data(x.numpy())
+    cq = O.search_copy_of_centroids(c.numpy().astype(np.float64))
+    book = LabelBook()
+    _, best = book.compare(labels.cpu().numpy(), xq, cq)
+    book.finish()
+    xn = np.einsum("ij,ij->i", xq, xq)
+    np.testing.assert_allclose(dists.cpu().numpy(), best, rtol=1e-4, atol=1e-5 * (xn.mean() + 1))
+    mse = m.mse(x.cuda())
+    assert abs(mse - best.mean()) <= MSE_REL * best.mean() + 1e-12
+    # host outputs take the same path
+    lab_h = torch.empty(n, dtype=torch.int64)
+    m.assign(x, labels=lab_h)
+    assert torch.equal(lab_h, labels.cpu())
+
+
+def test_simt_and_tensor_core_search_agree(em):
+    x = synth.hand_shape(3000, 96, 30, seed=2)
+    k = 700
+    c = x[:k].clone() + 0.01
+    out = []
+    for kernel in (0, 1):
+        m = em.Model(96, k, seed=1, assign_kernel=kernel)
+        m.set_state(c=c)
+        lab = torch.empty(3000, dtype=torch.int64, device="cuda")
+        m.assign(x.cuda(), labels=lab)
+        out.append(lab.cpu().numpy())
+    assert np.mean(out[0] != out[1]) <= 1e-3
+
+
+def test_lloyd_mode_matches_oracle(em):
+    w, xt, xs = datagen.make("tiny")
+    xq, xsq = O.search_copy_of_data(xt.numpy()), O.search_copy_of_data(xs.numpy())
+    m = em.Model(w.d, w.k, seed=1234)
+    m.lloyd(xt.cuda(), 25)
+    _, _, c, _ = gpu_state(m, w.k, w.d)
+    c0 = xq[O.starting_rows(len(xq), w.k, 1234)]
+    c_ref, _ = O.lloyd(xq, c0, 25)
+    rel = centroid_rel_err(c, c_ref)
+    assert np.mean(rel <= CENTROID_REL) >= 0.95
+    mse_gpu = m.mse(xs.cuda())
+    assert abs(mse_gpu - O.mse(xsq, c_ref)) <= MSE_REL * mse_gpu
+
+
+def test_tiny_independent_run_final_mse(em):
+    w, xt, xs = datagen.make("tiny")
+    xq, xsq = O.search_copy_of_data(xt.numpy()), O.search_copy_of_data(xs.numpy())
+    m = em.Model(w.d, w.k, seed=1234)
+    m.train(xt.cuda(), epochs=w.epochs)
+    orc = O.EmeansOracle(w.d, w.k, seed=1234)
+    c_ref, lab_ref = orc.train(xq, w.epochs)
+    mse_gpu, mse_ref = m.mse(xs.cuda()), O.mse(xsq, c_ref)
+    assert abs(mse_gpu - mse_ref) <= MSE_REL * mse_ref
+    obj = m.obj()
+    np.testing.assert_allclose(obj, orc.obj, rtol=1e-3)
+    st = m.stats()
+    assert st["steps_done"] == 50 and st["rows_assigned"] == 5 * w.n_train
+    assert st["n_splits"] == orc.n_splits
+
+
+def test_fractional_epochs_and_labels(em):
+    x = synth.hand_shape(2000, 32, 10, seed=4)
+    m = em.Model(32, 20, seed=9, batch_size=256)
+    m.train(x.cuda(), epochs=1.5)
+    lab = torch.empty(2000, dtype=torch.int64)
+    m.labels(lab)
+    assert int((lab >= 0).sum()) == 1000 and int((lab == -1).sum()) == 1000
+    r = m.recipe()
+    assert r["passes"] == 2 and r["rows_last_pass"] == 1000 and r["total_steps"] == 8 + 4
+
+
+def test_state_roundtrip_and_errors(em):
+    m = em.Model(16, 8, seed=1)
+    with pytest.raises(em.EmeansError) as e:
+        m.step(1)
+    assert e.value.code == em.EM_E_STATE
+    x = synth.hand_shape(100, 16, 4, seed=1)
+    with pytest.raises(em.EmeansError) as e:
+        m.train(x[:5].cuda(), epochs=1.0)  # fewer rows than clusters
+    assert e.value.code == em.EM_E_INVAL
+    N = torch.rand(8)
+    S = torch.randn(8, 16)
+    c = torch.randn(8, 16)
+    m.set_state(N=N, S=S, c=c)
+    N2, S2, c2 = torch.empty(8), torch.empty(8, 16), torch.empty(8, 16)
+    m.get_state(N=N2, S=S2, c=c2)
+    assert torch.equal(N, N2) and torch.equal(S, S2) and torch.equal(c, c2)
+    bad = x.clone()
+    bad[3, 2] = float("nan")
+    m.set_option("check_finite", 1)
+    with pytest.raises(em.EmeansError) as e:
+        m.train(bad.cuda(), epochs=1.0)
+    assert e.value.code == em.EM_E_NONFINITE
