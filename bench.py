@@ -393,6 +393,42 @@ def run_reference(args):
     }
 
 
+def run_kernel_case(args):
+    """A small standalone case for profiler captures: `--kernel-case assign` runs the
+    fused assignment twice on `--case-rows` rows of the workload (bf16, larger than
+    L2) against k starting centroids; `--kernel-case step` runs `--steps` training
+    steps of the full workload."""
+    import torch
+
+    import datagen
+    import mini_ema_means_b200 as em
+
+    torch.cuda.set_device(0)
+    if args.kernel_case == "assign":
+        w, xt, _ = datagen.make(args.workload, device="cuda", seed=0, n_train=args.case_rows, n_test=1)
+        xb = xt.to(torch.bfloat16).contiguous()
+        m = em.Model(w.d, w.k, seed=1234, input_dtype=1)
+        m.set_state(c=xt[: w.k].float().contiguous())
+        lab = torch.empty(w.n_train, dtype=torch.int64, device="cuda")
+        for _ in range(2):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            m.assign(xb, labels=lab)
+            e1.record()
+            torch.cuda.synchronize()
+            ms = e0.elapsed_time(e1)
+            log(f"assign pass {w.n_train} x {w.k} x {w.d}: {ms:.3f} ms, "
+                f"{2.0 * w.n_train * w.k * w.d / ms / 1e9:.1f} TFLOP/s (whole call)")
+    else:
+        w, xt, _ = datagen.make(args.workload, device="cuda", seed=0)
+        m = em.Model(w.d, w.k, seed=1234)
+        m.begin(xt, epochs=w.epochs)
+        m.step(args.steps)
+        m.sync()
+    m.close()
+    print(json.dumps({"kernel_case": args.kernel_case, "workload": args.workload, "ok": True}))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -407,7 +443,12 @@ def main():
     ap.add_argument("--ref-seconds", type=float, default=120.0)
     ap.add_argument("--traffic", type=float, default=None,
                     help="dram bytes per assignment launch from an ncu capture of the current kernel")
+    ap.add_argument("--kernel-case", choices=["assign", "step"], default=None)
+    ap.add_argument("--case-rows", type=int, default=262144)
     args = ap.parse_args()
+    if args.kernel_case:
+        run_kernel_case(args)
+        return
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -203,7 +203,7 @@ struct em_model {
     DBuf<int64_t> labels_last, labels64;
     // revival scratch
     DBuf<int32_t> rv_dead, rv_donor, rv_order, rv_times, rv_ndead;
-    DBuf<double> rv_tree;
+    DBuf<double> rv_tree, rv_target;
     DBuf<int64_t> rv_splits;
     // run progress
     em_recipe_t rec{};
@@ -462,6 +462,7 @@ static ReviveScratch revive_scratch(em_model* m) {
     sc.order = m->rv_order.p;
     sc.times = m->rv_times.p;
     sc.tree = m->rv_tree.p;
+    sc.target = m->rv_target.p;
     sc.ndead = m->rv_ndead.p;
     sc.n_splits = m->rv_splits.p;
     return sc;
@@ -471,7 +472,7 @@ static int launch_revive(em_model* m, int64_t t, int64_t rows) {
     if (m->revival == EM_REVIVE_NONE || !(m->tau > 0.0)) return EM_OK;
     const ReviveScratch sc = revive_scratch(m);
     const TreeLayout L = tree_layout((int)m->k);
-    const int smem = (int)tree_smem_bytes(L);
+    const int smem = (int)tree_smem_bytes(L, (int)m->k);
     k_revive_select<<<1, 1024, smem, m->stream>>>(m->N.p, (int)m->k, m->tau, m->seed, t, m->revival, sc, m->err.p);
     CK(cudaGetLastError());
     const ClusterState st = cluster_state(m);
@@ -611,7 +612,7 @@ em_model* em_create(int64_t d, int64_t k, uint64_t seed) {
     if (m->N.ensure(k) || m->S.ensure(kd) || m->c.ensure(kd) || m->cn.ensure(k) || m->cq.ensure(kd) ||
         m->close_sum.ensure(kd) || m->close_cnt.ensure(k) || m->err.ensure(1) || m->flag.ensure(1) ||
         m->scalar.ensure(4) || m->rv_dead.ensure(k) || m->rv_donor.ensure(k) || m->rv_order.ensure(k) ||
-        m->rv_times.ensure(k) || m->rv_ndead.ensure(1) || m->rv_splits.ensure(1) ||
+        m->rv_times.ensure(k) || m->rv_ndead.ensure(1) || m->rv_splits.ensure(1) || m->rv_target.ensure(k) ||
         m->rv_tree.ensure((size_t)tree_layout((int)k).total))
         return bail(EM_E_NOMEM, "device allocation failed");
     cudaMemset(m->err.p, 0, sizeof(int));
@@ -627,7 +628,7 @@ em_model* em_create(int64_t d, int64_t k, uint64_t seed) {
         cudaFuncSetAttribute(tc::k_assign_tc<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              tc::Cfg<32>::kSmemBytes) != cudaSuccess ||
         cudaFuncSetAttribute(k_revive_select, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kReviveSmemDoubles * 8) != cudaSuccess)
+                             kReviveSmemBytes) != cudaSuccess)
         return bail(EM_E_CUDA, "cudaFuncSetAttribute failed");
     if (make_tmap(&m->tm_cq, m->cq.p, k, (int)d, m->ld, tc::BN, m->kc) != EM_OK) {
         em_destroy(m);
@@ -649,6 +650,7 @@ void em_destroy(em_model* m) {
     m->plast.release(); m->step_err.release(); m->scalar.release(); m->labels_last.release();
     m->labels64.release(); m->rv_dead.release(); m->rv_donor.release(); m->rv_order.release();
     m->rv_times.release(); m->rv_ndead.release(); m->rv_tree.release(); m->rv_splits.release();
+    m->rv_target.release();
     for (auto& sp : m->pending) {
         cudaEventDestroy(sp.a);
         cudaEventDestroy(sp.b);

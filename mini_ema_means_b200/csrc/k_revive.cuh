@@ -15,10 +15,11 @@
 //   * resample (the EnCodec-style arm of the ablation): c_j <- a row of the
 //     current batch drawn with Philox(seed, stream 4, t, j), N_j = S_j = 0.
 //
-// The draws are inherently sequential, so one warp makes them on an fp64 tree
-// of prefix sums (32 children per node: one coalesced load, one ballot per
-// level, and a halving updates one suffix of each level with one lane-parallel
-// subtraction). The vector work is then done in parallel from the closed form:
+// The draws are inherently sequential, so one warp makes them on an fp64 tree in
+// shared memory (32 children per node: one load and one ballot per prefix level,
+// one warp scan of the 32 current leaf weights, and a halving updates one suffix
+// of each level with one lane-parallel subtraction); the uniform draws are made
+// in parallel beforehand. The vector work is then done in parallel from the closed form:
 // the o-th split taken from donor d (0-based) sees c_d (1 + eps s)^o and N_d / 2^o.
 #pragma once
 
@@ -31,20 +32,24 @@ struct ReviveScratch {
     int32_t* donor;   // k: donor of each dead cluster (-1 if none)
     int32_t* order;   // k: how many earlier splits took this donor in this check
     int32_t* times;   // k: splits taken from each donor in this check
-    double* tree;     // prefix-sum levels that do not fit in shared memory (tree_layout(k).total)
+    double* target;   // k: u of each dead cluster (precomputed in parallel)
+    double* tree;     // leaf weights and prefix levels that do not fit in shared memory
     int32_t* ndead;   // 1: |D| of the most recent check
     int64_t* n_splits;  // 1: cumulative number of revived clusters
 };
 
+// Donor tree: level 0 holds the current weight of every cluster (N_j, or 0 for a
+// dead one); level l >= 1 holds, for each group of 32 entries of level l-1, the
+// inclusive prefix of the group totals within its own group of 32.
 struct TreeLayout {
     int levels;
     int size[8];
     int64_t offset[8];
-    int64_t total;
+    int64_t total;   // doubles
 };
 
-// Shared memory the selection kernel may use for the tree (doubles).
-constexpr int kReviveSmemDoubles = 24 * 1024;
+// Shared memory the selection kernel may use (bytes).
+constexpr int kReviveSmemBytes = 200 * 1024;
 
 EM_HD TreeLayout tree_layout(int k) {
     TreeLayout L{};
@@ -63,17 +68,20 @@ EM_HD TreeLayout tree_layout(int k) {
     return L;
 }
 
-// 0: every level in shared memory; 1: leaves in global memory, the rest shared;
-// 2: every level in global memory.
-EM_HD int tree_placement(const TreeLayout& L) {
-    if (L.total <= kReviveSmemDoubles) return 0;
-    if (L.levels > 1 && L.total - L.offset[1] <= kReviveSmemDoubles) return 1;
+// 0: leaves, split counts and upper levels in shared memory; 1: leaves and split
+// counts in global memory, upper levels shared; 2: everything in global memory.
+EM_HD int tree_placement(const TreeLayout& L, int k) {
+    const int64_t upper = (L.total - L.offset[L.levels > 1 ? 1 : 0]) * 8;
+    if (L.total * 8 + (int64_t)k * 4 <= kReviveSmemBytes) return 0;
+    if (L.levels > 1 && upper <= kReviveSmemBytes) return 1;
     return 2;
 }
 
-EM_HD int64_t tree_smem_bytes(const TreeLayout& L) {
-    const int p = tree_placement(L);
-    return p == 0 ? L.total * 8 : p == 1 ? (L.total - L.offset[1]) * 8 : 0;
+EM_HD int64_t tree_smem_bytes(const TreeLayout& L, int k) {
+    const int p = tree_placement(L, k);
+    if (p == 0) return L.total * 8 + (int64_t)k * 4;
+    if (p == 1) return (L.total - L.offset[1]) * 8;
+    return 0;
 }
 
 __device__ __forceinline__ double warp_incl_scan(double v, int lane) {
@@ -85,7 +93,7 @@ __device__ __forceinline__ double warp_incl_scan(double v, int lane) {
     return v;
 }
 
-// One CTA of 1024 threads: dead set, tree, sequential donor draws.
+// One CTA of 1024 threads: dead set, donor tree, sequential donor draws.
 __global__ void __launch_bounds__(1024) k_revive_select(const float* __restrict__ N, int k, double tau, uint64_t seed,
                                                         int64_t t, int mode, ReviveScratch sc, int* err) {
     __shared__ double red[32];
@@ -114,7 +122,6 @@ __global__ void __launch_bounds__(1024) k_revive_select(const float* __restrict_
     for (int b = 0; b < k; b += 1024) {
         const int j = b + tid;
         const bool dead = j < k && (double)N[j] < thr;
-        if (j < k) sc.times[j] = 0;
         const unsigned m = __ballot_sync(0xFFFFFFFFu, dead);
         if (lane == 0) wcount[w] = __popc(m);
         __syncthreads();
@@ -138,37 +145,53 @@ __global__ void __launch_bounds__(1024) k_revive_select(const float* __restrict_
     if (tid == 0) *sc.ndead = nd;
     if (mode != EM_REVIVE_SPLIT || nd == 0 || !(total > 0.0)) {
         for (int i = tid; i < nd; i += 1024) sc.donor[i] = -1;
+        for (int j = tid; j < k; j += 1024) sc.times[j] = 0;
         return;
     }
 
-    // prefix tree over the weights of the eligible clusters (dead ones weigh 0);
-    // all levels in shared memory when they fit, else level 0 in global memory
-    extern __shared__ double stree[];
+    // draws of every dead cluster, in parallel (they do not depend on each other)
+    for (int i = tid; i < nd; i += 1024) sc.target[i] = draw_uniform(seed, kStreamRevive, t, sc.dead[i]);
+
+    // donor tree
+    extern __shared__ double smem_d[];
     const TreeLayout L = tree_layout(k);
+    const int placement = tree_placement(L, k);
     double* levp[8];
-    const int placement = tree_placement(L);
+    int32_t* times;
     for (int l = 0; l < L.levels; ++l) {
-        if (placement == 0 || (placement == 1 && l > 0))
-            levp[l] = stree + (L.offset[l] - (placement == 0 ? 0 : L.offset[1]));
+        if (placement == 0)
+            levp[l] = smem_d + L.offset[l];
+        else if (placement == 1 && l > 0)
+            levp[l] = smem_d + (L.offset[l] - L.offset[1]);
         else
             levp[l] = sc.tree + L.offset[l];
     }
-    for (int l = 0; l < L.levels; ++l) {
+    times = placement == 0 ? reinterpret_cast<int32_t*>(smem_d + L.total) : sc.times;
+    for (int j = tid; j < k; j += 1024) {
+        const float nj = N[j];
+        levp[0][j] = ((double)nj < thr) ? 0.0 : (double)nj;
+        times[j] = 0;
+    }
+    __syncthreads();
+    for (int l = 1; l < L.levels; ++l) {
         const int sz = L.size[l];
-        double* lev = levp[l];
         const int ngroups = (sz + 31) / 32;
         for (int gidx = w; gidx < ngroups; gidx += 32) {
-            const int i = gidx * 32 + lane;
+            const int i = gidx * 32 + lane;  // entry of level l = group i of level l-1
             double v = 0.0;
             if (i < sz) {
-                if (l == 0) {
-                    const float nj = N[i];
-                    v = ((double)nj < thr) ? 0.0 : (double)nj;
+                if (l == 1) {  // total of 32 leaves
+                    double acc = 0.0;
+                    for (int q = 0; q < 32; ++q) {
+                        const int leaf = i * 32 + q;
+                        if (leaf < L.size[0]) acc += levp[0][leaf];
+                    }
+                    v = acc;
                 } else {
-                    v = levp[l - 1][i * 32 + 31];  // total of child group i (its last prefix)
+                    v = levp[l - 1][i * 32 + 31];  // inclusive prefix at the end of child group i
                 }
             }
-            lev[gidx * 32 + lane] = warp_incl_scan(v, lane);
+            levp[l][gidx * 32 + lane] = warp_incl_scan(v, lane);
         }
         __syncthreads();
     }
@@ -176,56 +199,74 @@ __global__ void __launch_bounds__(1024) k_revive_select(const float* __restrict_
     // sequential draws by warp 0
     if (w == 0) {
         const int top = L.levels - 1;
-        double W = levp[top][31];
+        double W;
+        if (L.levels == 1) {
+            const double v = lane < L.size[0] ? levp[0][lane] : 0.0;
+            W = __shfl_sync(0xFFFFFFFFu, warp_incl_scan(v, lane), 31);
+        } else {
+            W = levp[top][31];
+        }
         bool exhausted = false;
-        for (int i = 0; i < nd; ++i) {
-            const int j = sc.dead[i];
-            if (exhausted || !(W > 0.0)) {
-                exhausted = true;
-                if (lane == 0) sc.donor[i] = -1;
-                continue;
-            }
-            double target = draw_uniform(seed, kStreamRevive, t, j) * W;
-            int node = 0;
-            for (int l = top; l >= 0; --l) {
+        for (int i0 = 0; i0 < nd; i0 += 32) {
+            const int cnt = min(32, nd - i0);
+            const double my_u = lane < cnt ? sc.target[i0 + lane] : 0.0;
+            for (int q = 0; q < cnt; ++q) {
+                const int i = i0 + q;
+                if (exhausted || !(W > 0.0)) {
+                    exhausted = true;
+                    if (lane == 0) sc.donor[i] = -1;
+                    continue;
+                }
+                double target = __shfl_sync(0xFFFFFFFFu, my_u, q) * W;
+                int node = 0;
+                for (int l = top; l >= 1; --l) {  // prefix levels: one load and one ballot each
+                    const int base = node * 32;
+                    const bool valid = base + lane < L.size[l];
+                    const double P = valid ? levp[l][base + lane] : 0.0;
+                    const double Pprev = __shfl_up_sync(0xFFFFFFFFu, P, 1);
+                    const double prev_incl = lane == 0 ? 0.0 : Pprev;
+                    const unsigned above = __ballot_sync(0xFFFFFFFFu, valid && P > target);
+                    int c;
+                    if (above) {
+                        c = __ffs(above) - 1;
+                    } else {  // target rounded onto the total: the last child with weight
+                        const unsigned pos = __ballot_sync(0xFFFFFFFFu, valid && P > prev_incl);
+                        c = pos ? 31 - __clz(pos) : 0;
+                    }
+                    target -= __shfl_sync(0xFFFFFFFFu, prev_incl, c);
+                    node = base + c;
+                }
+                // leaves: current weights, scanned by the warp
                 const int base = node * 32;
-                const double* lev = levp[l];
-                const bool valid = base + lane < L.size[l];
-                const double P = valid ? lev[base + lane] : 0.0;
-                const double Pprev = __shfl_up_sync(0xFFFFFFFFu, P, 1);
-                const double prev_incl = lane == 0 ? 0.0 : Pprev;
+                const bool valid = base + lane < L.size[0];
+                const double wv = valid ? levp[0][base + lane] : 0.0;
+                const double P = warp_incl_scan(wv, lane);
                 const unsigned above = __ballot_sync(0xFFFFFFFFu, valid && P > target);
                 int c;
                 if (above) {
                     c = __ffs(above) - 1;
-                } else {  // target rounded onto the total: take the last child with weight
-                    const unsigned pos = __ballot_sync(0xFFFFFFFFu, valid && P > prev_incl);
+                } else {
+                    const unsigned pos = __ballot_sync(0xFFFFFFFFu, valid && wv > 0.0);
                     c = pos ? 31 - __clz(pos) : 0;
                 }
-                const double before = __shfl_sync(0xFFFFFFFFu, prev_incl, c);
-                target -= before;
-                node = base + c;
+                const int dn = base + c;
+                const double delta = 0.5 * __shfl_sync(0xFFFFFFFFu, wv, c);  // half its current weight
+                if (lane == c) levp[0][dn] = wv - delta;
+                if (lane == 0) {
+                    const int old = times[dn];
+                    times[dn] = old + 1;
+                    sc.donor[i] = dn;
+                    sc.order[i] = old;
+                }
+                int idx = dn >> 5;
+                for (int l = 1; l < L.levels; ++l) {
+                    const int gb = (idx >> 5) << 5;
+                    if (gb + lane >= idx && gb + lane < L.size[l]) levp[l][gb + lane] -= delta;
+                    idx >>= 5;
+                }
+                W -= delta;
+                __syncwarp();
             }
-            const int dn = node;
-            int old = 0;
-            if (lane == 0) {
-                old = sc.times[dn];
-                sc.times[dn] = old + 1;
-                sc.donor[i] = dn;
-                sc.order[i] = old;
-            }
-            old = __shfl_sync(0xFFFFFFFFu, old, 0);
-            if (dn < 0 || dn >= k) raise_error(err, EM_E_BOUNDS);
-            const double delta = ldexp((double)N[dn], -(old + 1));  // half of its current weight
-            int idx = dn;
-            for (int l = 0; l < L.levels; ++l) {
-                const int gb = (idx >> 5) << 5;
-                double* lev = levp[l];
-                if (gb + lane >= idx && gb + lane < L.size[l]) lev[gb + lane] -= delta;
-                idx >>= 5;
-            }
-            W -= delta;
-            __syncwarp();
         }
         if (lane == 0) {
             int done = 0;
@@ -233,6 +274,9 @@ __global__ void __launch_bounds__(1024) k_revive_select(const float* __restrict_
             *sc.n_splits += done;
         }
     }
+    __syncthreads();
+    if (placement == 0)
+        for (int j = tid; j < k; j += 1024) sc.times[j] = times[j];
 }
 
 // Dead clusters take their half of the donor (reads the donors' state before
