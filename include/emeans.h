@@ -245,6 +245,36 @@ int em_last_batch(const em_model* m, int64_t* ids, int64_t* labels, float* dists
  * copies the totals to *out; reset != 0 clears them (and the launch count). */
 int em_profile(em_model* m, em_profile_t* out, int reset);
 
+/* ---- assignment without any allocation ----
+ *
+ * The paper has no counterpart to this entry point. It serves callers that cannot
+ * call cudaMalloc: code whose device memory is owned by another allocator or fixed
+ * up front (a serving process that forbids allocation after start-up, a library
+ * running inside a framework's memory pool), or that runs where an allocation would
+ * be an error. It computes the same labels and squared distances as em_assign, with
+ * the same kernels, but needs no model and allocates nothing: its scratch (search
+ * operand, norms, per-row keys, error word) is one file-scope __device__ array of
+ * EM_NOALLOC_SCRATCH_BYTES that every GPU which loads the library holds until exit.
+ *
+ * X: device bf16, n x d row-major, 16-byte aligned, d a multiple of 8 (read in
+ * place). centroids: device fp32, k x d, 16-byte aligned. labels (int64, n) and
+ * dists (fp32, n) are device outputs; either may be NULL. stream: a cudaStream_t
+ * (NULL = legacy default stream). Sizes beyond the limits below return EM_E_INVAL;
+ * host pointers return EM_E_INVAL.
+ *
+ * The first call on a device looks up the array's device address (and sets the
+ * kernels' shared-memory limits); make that first call before any stream capture.
+ * Every call shares the one array, which keeps the previous call's contents: calls
+ * that overlap on the GPU (other threads, other streams) race and must be ordered
+ * by the caller. The call waits for `stream` before it returns, to report
+ * device-side errors. */
+#define EM_NOALLOC_MAX_ROWS 524288
+#define EM_NOALLOC_MAX_K 65536
+#define EM_NOALLOC_MAX_KD 4194304 /* k * d */
+#define EM_NOALLOC_SCRATCH_BYTES 15728640
+int em_assign_noalloc(const void* X, int64_t n, int64_t d, const float* centroids, int64_t k, int64_t* labels,
+                      float* dists, void* stream);
+
 /* Waits for the model's stream and reports device-side errors (EM_E_BOUNDS,
  * EM_E_TIMEOUT) raised since the last check. */
 int em_sync(em_model* m);

@@ -56,6 +56,10 @@ EM_PHASE_FINALIZE = 5
 EM_NPHASES = 6
 PHASE_NAMES = ("prepare", "gather", "assign", "update", "revive", "finalize")
 
+EM_NOALLOC_MAX_ROWS = 524288
+EM_NOALLOC_MAX_K = 65536
+EM_NOALLOC_MAX_KD = 4194304
+
 EM_REVIVE_NONE = 0
 EM_REVIVE_SPLIT = 1
 EM_REVIVE_RESAMPLE = 2
@@ -135,6 +139,7 @@ _SIGS = {
     "em_set_state": (ctypes.c_int, [_P, _P, _P, _P, _I64]),
     "em_last_batch": (ctypes.c_int, [_P, _P, _P, _P, ctypes.POINTER(_I64)]),
     "em_profile": (ctypes.c_int, [_P, ctypes.POINTER(em_profile_t), ctypes.c_int]),
+    "em_assign_noalloc": (ctypes.c_int, [_P, _I64, _I64, _P, _I64, _P, _P, _P]),
     "em_sync": (ctypes.c_int, [_P]),
 }
 

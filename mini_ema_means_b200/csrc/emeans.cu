@@ -1111,3 +1111,137 @@ int em_sync(em_model* m) {
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------ assignment without allocation
+//
+// em_assign_noalloc keeps all of its scratch in this file-scope array. In host
+// code `g_noalloc_scratch` names a host-side stand-in, not device memory: the
+// device address is looked up once per device with cudaGetSymbolAddress.
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[EM_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+constexpr size_t kNaErr = 0;                                                   // int error word
+constexpr size_t kNaCn = 256;                                                  // fp32 [MAX_K]
+constexpr size_t kNaOperand = kNaCn + (size_t)EM_NOALLOC_MAX_K * 4;            // bf16 [MAX_KD]
+constexpr size_t kNaXn = kNaOperand + (size_t)EM_NOALLOC_MAX_KD * 2;           // fp32 [MAX_ROWS]
+constexpr size_t kNaKeys = kNaXn + (size_t)EM_NOALLOC_MAX_ROWS * 4;            // u64 [MAX_ROWS]
+constexpr size_t kNaBlocks = kNaKeys + (size_t)EM_NOALLOC_MAX_ROWS * 8;        // fp64 [kNaMaxBlocks]
+constexpr int kNaMaxBlocks = 4096;
+constexpr size_t kNaEnd = kNaBlocks + (size_t)kNaMaxBlocks * 8;
+static_assert(kNaEnd <= EM_NOALLOC_SCRATCH_BYTES, "scratch layout exceeds the array");
+static_assert(kNaOperand % 256 == 0 && kNaXn % 256 == 0 && kNaKeys % 256 == 0 && kNaBlocks % 256 == 0,
+              "scratch regions must stay 256-byte aligned");
+
+constexpr int kNaMaxDevices = 64;
+std::mutex g_na_mu;
+unsigned char* g_na_base[kNaMaxDevices] = {};
+
+// Search operand -2 bf16(c) and |bf16(c)|^2 from caller centroids (k x d, d % 8 == 0).
+__global__ void k_operand_from_centroids(const float* __restrict__ c, int k, int d, __nv_bfloat16* __restrict__ cq,
+                                         float* __restrict__ cn) {
+    const int lane = threadIdx.x & 31;
+    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int nwarps = (gridDim.x * blockDim.x) >> 5;
+    const int nv = d / 8;
+    for (int j = warp; j < k; j += nwarps) {
+        float part = 0.0f;
+        for (int v = lane; v < nv; v += 32) {
+            const float4* cr = reinterpret_cast<const float4*>(c + (int64_t)j * d) + 2 * v;
+            const float4 a = cr[0], b = cr[1];
+            const float cv[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+            float q[8];
+#pragma unroll
+            for (int t = 0; t < 8; ++t) {
+                const float bv = __bfloat162float(__float2bfloat16_rn(cv[t]));
+                part = fmaf(bv, bv, part);
+                q[t] = -2.0f * bv;
+            }
+            reinterpret_cast<uint4*>(cq + (int64_t)j * d)[v] = pack8_bf16(q);
+        }
+        part = warp_sum(part);
+        if (lane == 0) cn[j] = part;
+    }
+}
+
+// Device address of the scratch array on the current device (looked up once).
+int noalloc_scratch(int dev, unsigned char** out) {
+    if (dev < 0 || dev >= kNaMaxDevices) return fail(EM_E_INVAL, "device index out of range");
+    std::lock_guard<std::mutex> lock(g_na_mu);
+    if (!g_na_base[dev]) {
+        void* p = nullptr;
+        cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess || !p) {
+            cudaGetLastError();
+            return fail(EM_E_CUDA, "cudaGetSymbolAddress of the scratch array failed: %s", cudaGetErrorString(e));
+        }
+        if (cudaFuncSetAttribute(tc::k_assign_tc<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 tc::Cfg<64>::kSmemBytes) != cudaSuccess ||
+            cudaFuncSetAttribute(tc::k_assign_tc<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 tc::Cfg<32>::kSmemBytes) != cudaSuccess)
+            return fail(EM_E_CUDA, "cudaFuncSetAttribute failed");
+        g_na_base[dev] = static_cast<unsigned char*>(p);
+    }
+    *out = g_na_base[dev];
+    return EM_OK;
+}
+
+}  // namespace
+
+extern "C" int em_assign_noalloc(const void* X, int64_t n, int64_t d, const float* centroids, int64_t k,
+                                 int64_t* labels, float* dists, void* stream_) {
+    if (!X || !centroids) return fail(EM_E_INVAL, "X and centroids are required");
+    if (n < 1 || n > EM_NOALLOC_MAX_ROWS)
+        return fail(EM_E_INVAL, "n = %lld is outside [1, %d] rows", (long long)n, EM_NOALLOC_MAX_ROWS);
+    if (k < 1 || k > EM_NOALLOC_MAX_K) return fail(EM_E_INVAL, "k = %lld is outside [1, %d]", (long long)k, EM_NOALLOC_MAX_K);
+    if (d < 8 || d > 8192 || d % 8 != 0) return fail(EM_E_INVAL, "d must be a multiple of 8 in [8, 8192]");
+    if (k * d > EM_NOALLOC_MAX_KD) return fail(EM_E_INVAL, "k * d = %lld exceeds %d", (long long)(k * d), EM_NOALLOC_MAX_KD);
+    if ((reinterpret_cast<uintptr_t>(X) & 15) || (reinterpret_cast<uintptr_t>(centroids) & 15))
+        return fail(EM_E_INVAL, "X and centroids must be 16-byte aligned");
+    if (!is_device_ptr(X) || !is_device_ptr(centroids) || (labels && !is_device_ptr(labels)) ||
+        (dists && !is_device_ptr(dists)))
+        return fail(EM_E_INVAL, "em_assign_noalloc takes device pointers only");
+    int dev = 0;
+    CK(cudaGetDevice(&dev));
+    unsigned char* base = nullptr;
+    CKR(noalloc_scratch(dev, &base));
+    cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+    int sms = 148, clock_khz = 1965000;
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    cudaDeviceGetAttribute(&clock_khz, cudaDevAttrClockRate, dev);
+    int* err = reinterpret_cast<int*>(base + kNaErr);
+    float* cn = reinterpret_cast<float*>(base + kNaCn);
+    __nv_bfloat16* cq = reinterpret_cast<__nv_bfloat16*>(base + kNaOperand);
+    float* xn = reinterpret_cast<float*>(base + kNaXn);
+    unsigned long long* keys = reinterpret_cast<unsigned long long*>(base + kNaKeys);
+    double* blocks = reinterpret_cast<double*>(base + kNaBlocks);
+    const int kc = (d % 64 == 0) ? 64 : 32;
+    CUtensorMap tmA, tmB;
+    CKR(make_tmap(&tmA, X, n, (int)d, (int)d, tc::BM, kc));
+    CKR(make_tmap(&tmB, cq, k, (int)d, (int)d, tc::BN, kc));
+    const auto X16 = reinterpret_cast<const __nv_bfloat16*>(X);
+    CK(cudaMemsetAsync(err, 0, sizeof(int), stream));  // the previous call's error word is stale
+    k_operand_from_centroids<<<grid_for(k * 32, 256, sms), 256, 0, stream>>>(centroids, (int)k, (int)d, cq, cn);
+    k_rownorm_keys<<<grid_for(n * 32, 256, sms), 256, 0, stream>>>(X16, n, (int)d, xn, keys);
+    const int64_t m_tiles = (n + tc::BM - 1) / tc::BM;
+    const int64_t n_tiles = (k + tc::BN - 1) / tc::BN;
+    const int nkc = (int)((d + kc - 1) / kc);
+    const int split = choose_split(m_tiles, n_tiles, sms);
+    const int grid = (int)std::min<int64_t>(m_tiles * split, sms);
+    const long long wait_cycles = (long long)(2000.0 * (double)clock_khz);
+    if (kc == 64)
+        tc::k_assign_tc<64><<<grid, tc::kThreads, tc::Cfg<64>::kSmemBytes, stream>>>(
+            tmA, tmB, cn, (int)k, (int)n, nkc, (int)n_tiles, split, keys, wait_cycles, err);
+    else
+        tc::k_assign_tc<32><<<grid, tc::kThreads, tc::Cfg<32>::kSmemBytes, stream>>>(
+            tmA, tmB, cn, (int)k, (int)n, nkc, (int)n_tiles, split, keys, wait_cycles, err);
+    const int oblocks = std::min(grid_for(n, 256, sms), kNaMaxBlocks);
+    k_assign_out<<<oblocks, 256, 0, stream>>>(keys, xn, n, (int)k, labels, dists, nullptr, blocks, err);
+    CK(cudaGetLastError());
+    int h = 0;
+    CK(cudaMemcpyAsync(&h, err, sizeof(int), cudaMemcpyDeviceToHost, stream));
+    CK(cudaStreamSynchronize(stream));
+    if (h != 0) return fail(h, "device-side error %d in the assignment", h);
+    return EM_OK;
+}
