@@ -187,25 +187,35 @@ def run_ours(args, rank, world):
     # warm-up (untimed)
     steps_loop(args.warmup)
     torch.cuda.synchronize()
-    m.finalize()
-    m.begin(xt, epochs=w.epochs)
-    state["in_run"] = 0
-    m.set_option("profile", 1)
-    m.profile(reset=True)
+
+    def timed_pass(profile):
+        """K steps from a fresh begin between barriers and device syncs; returns (ms, rows)."""
+        m.finalize()
+        m.begin(xt, epochs=w.epochs)
+        state["in_run"] = 0
+        m.set_option("profile", 1 if profile else 0)
+        m.profile(reset=True)
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        rows = steps_loop(args.steps)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+        return e0.elapsed_time(e1), rows
+
+    # pass 1: the headline number (step graphs replayed, no per-launch events)
     sampler = ClockSampler(dev.index)
     sampler.start()
-    if world > 1:
-        torch.distributed.barrier()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    rows = steps_loop(args.steps)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    if world > 1:
-        torch.distributed.barrier()
+    ms, rows = timed_pass(profile=False)
     clocks = sampler.stop()
-    ms = e0.elapsed_time(e1)
+    launches = m.profile(reset=True)["launches"]
+    # pass 2: the same K steps with CUDA events around every phase of every step
+    # (graphs are bypassed while profiling): per-kernel durations for the roofline
+    ms_prof, _ = timed_pass(profile=True)
     prof = m.profile(reset=True)
     m.set_option("profile", 0)
     ms_max = ms
@@ -241,15 +251,17 @@ def run_ours(args, rank, world):
         "frac_of_sustained": achieved / peaks["bf16_tflops_sustained"] if peaks.get("bf16_tflops_sustained") else None,
         "avg_launch_ms": a_ms / a_n,
         "launches": prof["spans"]["assign"],
+        "measured_in": "second timed pass of the same K steps with CUDA events around every launch",
     }
     u_ms = prof["ms"]["update"]
     out["phases_ms"] = {k: round(v, 4) for k, v in prof["ms"].items()}
+    out["profiled_pass_ms_per_step"] = ms_prof / args.steps
     out["update_roofline"] = {
         "bound": "hbm", "achieved": prof["update_bytes"] / (u_ms / 1e3) / 1e9 if u_ms > 0 else 0.0,
         "peak": peaks["hbm_gbs"], "unit": "GB/s",
         "frac": (prof["update_bytes"] / (u_ms / 1e3) / 1e9) / peaks["hbm_gbs"] if u_ms > 0 else 0.0,
     }
-    out["gpu_launches"] = prof["launches"]
+    out["gpu_launches"] = launches
     out["clocks"] = clocks
 
     if rank == 0 and not args.no_extras:
@@ -276,10 +288,20 @@ def lloyd25(m, w, xt, xs, rec):
     total = rec["total_steps"]
     every = math.ceil(total / 20)
     full = rec["steps_full_pass"]
-    m.begin(xt, epochs=w.epochs)
     stream = torch.cuda.current_stream()
-    train_ms, steps, hit = 0.0, 0, None
-    history = []
+    # one untimed pass over the same checkpoint schedule first, so that the timed
+    # pass replays step graphs instead of capturing them
+    for timed in (False, True):
+        m.begin(xt, epochs=w.epochs)
+        train_ms, steps, hit = 0.0, 0, None
+        history = []
+        if timed:
+            break
+        while steps < total:
+            nxt = min(total, (steps // every + 1) * every, (steps // full + 1) * full)
+            m.step(nxt - steps)
+            steps = nxt
+        m.finalize()
     while steps < total:
         nxt = min(total, (steps // every + 1) * every, (steps // full + 1) * full)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -420,7 +442,8 @@ def run_kernel_case(args):
             log(f"assign pass {w.n_train} x {w.k} x {w.d}: {ms:.3f} ms, "
                 f"{2.0 * w.n_train * w.k * w.d / ms / 1e9:.1f} TFLOP/s (whole call)")
     else:
-        w, xt, _ = datagen.make(args.workload, device="cuda", seed=0)
+        rows = args.case_rows if args.case_rows_step else None
+        w, xt, _ = datagen.make(args.workload, device="cuda", seed=0, n_train=rows, n_test=1 if rows else None)
         m = em.Model(w.d, w.k, seed=1234)
         m.begin(xt, epochs=w.epochs)
         m.step(args.steps)
@@ -433,7 +456,7 @@ def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2400)
-    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=100)
     ap.add_argument("--workload", default="emb768")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
@@ -445,6 +468,7 @@ def main():
                     help="dram bytes per assignment launch from an ncu capture of the current kernel")
     ap.add_argument("--kernel-case", choices=["assign", "step"], default=None)
     ap.add_argument("--case-rows", type=int, default=262144)
+    ap.add_argument("--case-rows-step", action="store_true", help="train the step case on --case-rows rows")
     args = ap.parse_args()
     if args.kernel_case:
         run_kernel_case(args)

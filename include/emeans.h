@@ -67,8 +67,12 @@ enum em_option {
     EM_OPT_GRAPHS = 12,          /* 1 (default): em_step replays CUDA graphs of whole steps     */
     EM_OPT_ASSIGN_KERNEL = 13,   /* 0 (default): tcgen05 tensor-core assignment; 1: a plain
                                     SIMT kernel kept only to localise faults in tests           */
-    EM_OPT_PROFILE = 14          /* 1: bracket every phase of every step with CUDA events on the
+    EM_OPT_PROFILE = 14,         /* 1: bracket every phase of every step with CUDA events on the
                                     model's stream (read with em_profile); 0 (default): off     */
+    EM_OPT_EXACT_TIES = 15       /* 1: the search also keeps each row's second best centroid and
+                                    rows whose two best fp32 scores are within the accumulation
+                                    error are settled with exact fp64 distances; 0: plain fp32
+                                    argmin; -1 (default): on when d >= 256                       */
 };
 
 /* Phases timed by EM_OPT_PROFILE (em_profile_t.ms / spans index). */
@@ -271,7 +275,7 @@ int em_profile(em_model* m, em_profile_t* out, int reset);
 #define EM_NOALLOC_MAX_ROWS 524288
 #define EM_NOALLOC_MAX_K 65536
 #define EM_NOALLOC_MAX_KD 4194304 /* k * d */
-#define EM_NOALLOC_SCRATCH_BYTES 15728640
+#define EM_NOALLOC_SCRATCH_BYTES 19922944
 int em_assign_noalloc(const void* X, int64_t n, int64_t d, const float* centroids, int64_t k, int64_t* labels,
                       float* dists, void* stream);
 

@@ -6,10 +6,10 @@
 //   k_gather        batch rows pi_pass(pos..pos+B) -> contiguous bf16 batch, |x|^2
 //   k_assign_tc     nearest centroid of every batch row (tcgen05 + TMA)
 //   k_labels        labels, distances, per-cluster counts and ranks
-//   k_offsets       segment starts, batch error sum
-//   k_scatter       rows in label order
-//   k_segsum        per-cluster sums (fp64) fused with the EMA update
-//   k_fixup         clusters cut by tile edges, clusters without rows
+//   k_offsets       segment starts and work-item starts, batch error sum
+//   k_scatter       rows in label order, one work item per chunk of a cluster
+//   k_segsum        per-chunk sums (fp64) fused with the EMA update of small clusters
+//   k_clusters      large clusters (chunk sums in order), clusters without rows
 //   k_revive_*      every 5th step: dead-cluster revival
 // No host synchronisation happens inside a run; the step size of step t is
 // computed on the host (cosine schedule) and passed by value.
@@ -181,9 +181,10 @@ struct em_model {
     int64_t opt_batch = 0;
     double opt_alpha0 = 0.0, tau = 0.1, wait_ms = 2000.0;
     int revival = EM_REVIVE_SPLIT, finalize = 1, law = 0, in_dtype = 0, check_finite = 0;
-    int auto_revive = 1, capture = 1, graphs = 1, assign_kernel = 0;
+    int auto_revive = 1, capture = 1, graphs = 1, assign_kernel = 0, exact_ties = -1;
+    int last_split = 1;  // centroid-tile groups of the most recent search (keys per row)
     // state
-    DBuf<float> N, S, c, cn;
+    DBuf<float> N, N_prev, S, c, cn, cnp;
     DBuf<__nv_bfloat16> cq;
     DBuf<double> close_sum, close_cnt;
     DBuf<int> err, flag;
@@ -197,9 +198,10 @@ struct em_model {
     int R = 32;
     DBuf<__nv_bfloat16> Xb;
     DBuf<float> xn, dists;
-    DBuf<int32_t> ids, labels, cnt, rank, off, perm, slab;
+    DBuf<int32_t> ids, labels, cnt, rank, off, poff, perm;
+    DBuf<int2> items;
     DBuf<unsigned long long> keys;
-    DBuf<double> block_err, pfirst, plast, step_err, scalar;
+    DBuf<double> block_err, part, step_err, scalar;
     DBuf<int64_t> labels_last, labels64;
     // revival scratch
     DBuf<int32_t> rv_dead, rv_donor, rv_order, rv_times, rv_ndead;
@@ -224,6 +226,14 @@ struct em_model {
     std::vector<Span> pending;
     std::vector<cudaEvent_t> pool;
     em_profile_t totals{};
+    // CUDA graphs of step ranges (EM_OPT_GRAPHS), keyed by everything they bake in
+    struct GraphEntry {
+        std::vector<uint64_t> sig;
+        int64_t t0, count, launches;
+        cudaGraphExec_t exec;
+    };
+    std::vector<GraphEntry> graph_cache;
+    cudaStream_t cap_stream = nullptr;
 };
 
 // Opens an event span of `phase` on the model's stream (-1 when profiling is off).
@@ -334,6 +344,9 @@ static int prepare_input(em_model* m, const void* X, int64_t n, DBuf<__nv_bfloat
 static ClusterState cluster_state(em_model* m) {
     ClusterState st;
     st.N = m->N.p;
+    st.N_prev = m->N_prev.p;
+    st.cnp = m->cnp.p;
+    st.k = (int)m->k;
     st.S = m->S.p;
     st.c = m->c.p;
     st.cq = m->cq.p;
@@ -344,38 +357,35 @@ static ClusterState cluster_state(em_model* m) {
     return st;
 }
 
+// Rows per work item of the grouped update (a cluster's sorted rows are cut into
+// chunks of at most this many rows).
+constexpr int kChunkRows = 64;
+
 static int ensure_batch_buffers(em_model* m, int64_t cap) {
-    m->R = 32;
-    {
-        // tiles of R label-sorted rows per warp: about 16 tiles per SM
-        int64_t want = cap / ((int64_t)m->sms * 16);
-        int r = 8;
-        while (r < 256 && r < want) r <<= 1;
-        m->R = r;
-    }
-    const int64_t ntiles = (cap + m->R - 1) / m->R;
+    m->R = kChunkRows;
+    const int64_t max_items = m->k + (cap + m->R - 1) / m->R;
     CKR(m->xn.ensure(cap));
     CKR(m->dists.ensure(cap));
     CKR(m->ids.ensure(cap));
     CKR(m->labels.ensure(cap));
     CKR(m->rank.ensure(cap));
     CKR(m->perm.ensure(cap));
-    CKR(m->slab.ensure(cap));
     CKR(m->keys.ensure(cap));
     CKR(m->cnt.ensure(m->k));
     CKR(m->off.ensure(m->k + 1));
+    CKR(m->poff.ensure(m->k + 1));
+    CKR(m->items.ensure(max_items));
     CKR(m->block_err.ensure((cap + 255) / 256 + 1));
-    CKR(m->pfirst.ensure((size_t)ntiles * m->ld));
-    CKR(m->plast.ensure((size_t)ntiles * m->ld));
+    CKR(m->part.ensure((size_t)max_items * m->ld));
     m->bcap = cap;
     return EM_OK;
 }
 
-static int choose_split(int64_t m_tiles, int64_t n_tiles, int sms) {
+static int choose_split(int64_t m_tiles, int64_t n_tiles, int sms, int max_split = 8) {
     int best = 1;
     double best_cost = 1e300;
     for (int s = 1; s <= 8; s <<= 1) {
-        if (s > n_tiles) break;
+        if (s > n_tiles || s > max_split) break;
         const int64_t units = m_tiles * s;
         const int64_t waves = (units + sms - 1) / sms;
         const double cost = (double)waves * (double)((n_tiles + s - 1) / s);
@@ -389,67 +399,78 @@ static int choose_split(int64_t m_tiles, int64_t n_tiles, int sms) {
 
 // Nearest-centroid search of `rows` rows described by tmA (row source A for the
 // SIMT path) into m->keys (which the caller has reset to the empty key).
+static bool use_top2(const em_model* m) {
+    return m->exact_ties == 1 || (m->exact_ties < 0 && m->d >= 256);
+}
+
+static int split_for(const em_model* m, int64_t rows) {
+    const int64_t m_tiles = (rows + tc::BM - 1) / tc::BM;
+    const int64_t n_tiles = (m->k + tc::BN - 1) / tc::BN;
+    return choose_split(m_tiles, n_tiles, m->sms);
+}
+
+// Keys the search writes for `rows` rows: two per row per centroid-tile group.
+static size_t keys_needed(const em_model* m, int64_t rows) {
+    return rows > 0 ? (size_t)split_for(m, rows) * (size_t)rows * 2 : 0;
+}
+
 static int launch_assign(em_model* m, const CUtensorMap& tmA, const __nv_bfloat16* A, int64_t rows) {
     if (rows <= 0) return EM_OK;
+    if (m->keys.cap < keys_needed(m, rows)) return fail(EM_E_STATE, "search key buffer too small");
     if (m->assign_kernel == 1) {
         k_assign_simt<<<(int)((rows + 127) / 128), 128, 0, m->stream>>>(A, m->ld, (int)rows, m->cq.p, m->cn.p,
                                                                          (int)m->k, (int)m->d, m->keys.p);
         CK(cudaGetLastError());
         EM_LAUNCHED(m, 1);
+        m->last_split = 1;
         return EM_OK;
     }
     const int64_t m_tiles = (rows + tc::BM - 1) / tc::BM;
     const int64_t n_tiles = (m->k + tc::BN - 1) / tc::BN;
     const int nkc = (int)((m->d + m->kc - 1) / m->kc);
-    const int split = choose_split(m_tiles, n_tiles, m->sms);
+    const int split = split_for(m, rows);
     const int64_t units = m_tiles * split;
     const int grid = (int)std::min<int64_t>(units, m->sms);
+    const bool top2 = use_top2(m);
+#define EM_ASSIGN(KC, T2)                                                                                           \
+    tc::k_assign_tc<KC, T2><<<grid, tc::kThreads, tc::Cfg<KC>::kSmemBytes, m->stream>>>(                           \
+        tmA, m->tm_cq, m->cn.p, (int)m->k, (int)rows, nkc, (int)n_tiles, split, m->keys.p, m->wait_cycles, m->err.p)
     if (m->kc == 64) {
-        tc::k_assign_tc<64><<<grid, tc::kThreads, tc::Cfg<64>::kSmemBytes, m->stream>>>(
-            tmA, m->tm_cq, m->cn.p, (int)m->k, (int)rows, nkc, (int)n_tiles, split, m->keys.p, m->wait_cycles,
-            m->err.p);
+        if (top2)
+            EM_ASSIGN(64, true);
+        else
+            EM_ASSIGN(64, false);
     } else {
-        tc::k_assign_tc<32><<<grid, tc::kThreads, tc::Cfg<32>::kSmemBytes, m->stream>>>(
-            tmA, m->tm_cq, m->cn.p, (int)m->k, (int)rows, nkc, (int)n_tiles, split, m->keys.p, m->wait_cycles,
-            m->err.p);
+        if (top2)
+            EM_ASSIGN(32, true);
+        else
+            EM_ASSIGN(32, false);
     }
+#undef EM_ASSIGN
     CK(cudaGetLastError());
     EM_LAUNCHED(m, 1);
+    m->last_split = split;
     return EM_OK;
 }
 
-// Group rows by label and apply the EMA update (k_offsets .. k_fixup); labels,
+// Group rows by label and apply the EMA update (k_offsets .. k_clusters); labels,
 // ranks and counts are already in place. `src` holds the rows (batch or data).
 static int launch_reduce(em_model* m, const __nv_bfloat16* src, int64_t rows, int nblocks_labels, double alpha,
                          int last_pass, double* err_sum_out) {
     const StepParams sp{alpha, last_pass, 0};
-    k_offsets<<<1, 1024, 0, m->stream>>>(m->cnt.p, (int)m->k, (int)rows, m->off.p, m->block_err.p, nblocks_labels,
-                                         err_sum_out, m->err.p);
+    k_offsets<<<1, 1024, 0, m->stream>>>(m->cnt.p, (int)m->k, (int)rows, m->R, m->off.p, m->poff.p, m->block_err.p,
+                                         nblocks_labels, err_sum_out, m->N.p, m->N_prev.p, m->err.p);
     CK(cudaGetLastError());
-    k_scatter<<<(int)((rows + 255) / 256), 256, 0, m->stream>>>(m->labels.p, m->rank.p, m->off.p, (int)rows,
-                                                                 m->perm.p, m->slab.p, m->err.p);
+    k_scatter<<<(int)((rows + 255) / 256), 256, 0, m->stream>>>(m->labels.p, m->rank.p, m->off.p, m->poff.p,
+                                                                 (int)rows, m->R, m->perm.p, m->items.p, m->err.p);
     CK(cudaGetLastError());
-    const int64_t ntiles = (rows + m->R - 1) / m->R;
-    const int seg_blocks = (int)((ntiles * 32 + 255) / 256);
+    const int64_t max_items = m->k + (rows + m->R - 1) / m->R;
+    const int nslices = (m->nv + 31) / 32;
     const ClusterState st = cluster_state(m);
-    const int fix_blocks = grid_for(std::max<int64_t>(ntiles, m->k) * 32, 256, m->sms);
-#define EM_REDUCE(V)                                                                                            \
-    k_segsum<V><<<seg_blocks, 256, 0, m->stream>>>(src, m->perm.p, m->slab.p, m->off.p, (int)rows, m->R, m->nv, \
-                                                   st, sp, m->pfirst.p, m->plast.p);                           \
-    k_fixup<V><<<fix_blocks, 256, 0, m->stream>>>(m->slab.p, m->off.p, m->cnt.p, (int)rows, m->R, (int)ntiles,  \
-                                                  (int)m->k, m->nv, st, sp, m->pfirst.p, m->plast.p)
-    if (m->nv <= 32) {
-        EM_REDUCE(1);
-    } else if (m->nv <= 64) {
-        EM_REDUCE(2);
-    } else if (m->nv <= 96) {
-        EM_REDUCE(3);
-    } else if (m->nv <= 128) {
-        EM_REDUCE(4);
-    } else {
-        EM_REDUCE(8);
-    }
-#undef EM_REDUCE
+    k_segsum<<<(int)((max_items * nslices * 32 + 255) / 256), 256, 0, m->stream>>>(
+        src, m->perm.p, m->items.p, m->off.p, m->poff.p, m->R, nslices, m->nv, st, sp, m->part.p);
+    k_clusters<<<grid_for(m->k * 32, 256, m->sms), 256, 0, m->stream>>>(m->off.p, m->poff.p, m->cnt.p, m->R, nslices,
+                                                                         m->nv, st, sp, m->part.p);
     CK(cudaGetLastError());
     EM_LAUNCHED(m, 4);
     return EM_OK;
@@ -489,17 +510,46 @@ static int launch_revive(em_model* m, int64_t t, int64_t rows) {
     return EM_OK;
 }
 
-// One training step of the current run.
-static int run_step(em_model* m) {
+// One training step of the current run: what it does (host-side plan), the
+// kernels it launches, and the host bookkeeping after it.
+struct StepPlan {
+    int64_t t, pass, pos, rows;
+    int last_pass, revive;
+    double alpha;
+};
+
+static StepPlan plan_step(const em_model* m) {
+    StepPlan p;
     const int64_t rows_pass = (m->pass == m->rec.passes - 1) ? m->rec.rows_last_pass : m->n;
-    const int64_t rows = std::min<int64_t>(m->rec.batch_size, rows_pass - m->pos);
-    const int last_pass = (m->pass == m->rec.passes - 1) ? 1 : 0;
-    const double alpha = alpha_at(m->t, m->rec.total_steps, m->rec.alpha0);
+    p.t = m->t;
+    p.pass = m->pass;
+    p.pos = m->pos;
+    p.rows = std::min<int64_t>(m->rec.batch_size, rows_pass - m->pos);
+    p.last_pass = (m->pass == m->rec.passes - 1) ? 1 : 0;
+    p.alpha = alpha_at(m->t, m->rec.total_steps, m->rec.alpha0);
+    p.revive = (m->auto_revive && (m->t + 1) % kReviveEvery == 0) ? 1 : 0;
+    return p;
+}
+
+static void advance_step(em_model* m, const StepPlan& p) {
+    const int64_t rows_pass = (m->pass == m->rec.passes - 1) ? m->rec.rows_last_pass : m->n;
+    m->last_rows = p.rows;
+    m->last_alpha = p.alpha;
+    m->rows_assigned += p.rows;
+    m->t += 1;
+    m->pos += p.rows;
+    if (m->pos >= rows_pass) {
+        m->pass += 1;
+        m->pos = 0;
+    }
+}
+
+static int launch_step(em_model* m, const StepPlan& p) {
+    const int64_t rows = p.rows;
     const double rd = (double)rows, dd = (double)m->d, kd = (double)m->k;
     int sp = span_begin(m, EM_PHASE_GATHER);
-    k_gather<<<grid_for(rows, 256, m->sms), 256, 0, m->stream>>>(m->X, m->n, m->ld, m->seed, m->pass, m->pos,
-                                                                 (int)rows, 0, m->Xb.p, m->xn.p, m->ids.p,
-                                                                 m->keys.p, m->err.p);
+    k_gather<<<grid_for(rows, 256, m->sms), 256, 0, m->stream>>>(m->X, m->n, m->ld, m->seed, p.pass, p.pos,
+                                                                 (int)rows, 0, m->Xb.p, m->xn.p, m->ids.p, m->err.p);
     CK(cudaGetLastError());
     EM_LAUNCHED(m, 1);
     span_end(m, sp, 0.0, 4.0 * rd * dd);
@@ -508,28 +558,101 @@ static int run_step(em_model* m) {
     span_end(m, sp, 2.0 * rd * kd * dd, 0.0);
     sp = span_begin(m, EM_PHASE_UPDATE);
     const int nbl = (int)((rows + 255) / 256);
-    const int capture = (m->capture && last_pass) ? 1 : 0;
-    k_labels<<<nbl, 256, 0, m->stream>>>(m->keys.p, m->xn.p, (int)rows, (int)m->k, m->ids.p, m->labels.p,
-                                         m->dists.p, m->cnt.p, m->rank.p, m->block_err.p, m->labels_last.p, capture,
-                                         m->err.p);
+    const int capture = (m->capture && p.last_pass) ? 1 : 0;
+    k_labels<<<nbl, 256, 0, m->stream>>>(m->keys.p, m->last_split, m->xn.p, (int)rows, (int)m->k, m->Xb.p, m->ld,
+                                         m->cq.p, m->ids.p, m->labels.p, m->dists.p, m->cnt.p, m->rank.p,
+                                         m->block_err.p, m->labels_last.p, capture, m->err.p);
     CK(cudaGetLastError());
     EM_LAUNCHED(m, 1);
-    CKR(launch_reduce(m, m->Xb.p, rows, nbl, alpha, m->finalize ? last_pass : 0, m->step_err.p + m->t));
+    CKR(launch_reduce(m, m->Xb.p, rows, nbl, p.alpha, m->finalize ? p.last_pass : 0, m->step_err.p + p.t));
     span_end(m, sp, 0.0, 2.0 * rd * dd + 16.0 * rd + 14.0 * kd * dd);
-    if (m->auto_revive && (m->t + 1) % kReviveEvery == 0) {
+    if (p.revive) {
         sp = span_begin(m, EM_PHASE_REVIVE);
-        CKR(launch_revive(m, m->t, rows));
+        CKR(launch_revive(m, p.t, rows));
         span_end(m, sp);
     }
-    m->last_rows = rows;
-    m->last_alpha = alpha;
-    m->rows_assigned += rows;
-    m->t += 1;
-    m->pos += rows;
-    if (m->pos >= rows_pass) {
-        m->pass += 1;
-        m->pos = 0;
+    return EM_OK;
+}
+
+static int run_step(em_model* m) {
+    const StepPlan p = plan_step(m);
+    CKR(launch_step(m, p));
+    advance_step(m, p);
+    return EM_OK;
+}
+
+// Everything a captured step range bakes in: buffer addresses, sizes, options.
+static std::vector<uint64_t> graph_signature(const em_model* m) {
+    const void* ptrs[] = {m->X, m->Xb.p, m->xn.p, m->dists.p, m->ids.p, m->labels.p, m->cnt.p, m->rank.p,
+                          m->N_prev.p, m->cnp.p,
+                          m->off.p, m->perm.p, m->poff.p, m->items.p, m->keys.p, m->block_err.p, m->part.p,
+                          m->step_err.p, m->labels_last.p, m->N.p, m->S.p, m->c.p, m->cn.p, m->cq.p,
+                          m->close_sum.p, m->close_cnt.p, m->err.p, m->rv_dead.p, m->rv_donor.p, m->rv_order.p,
+                          m->rv_times.p, m->rv_ndead.p, m->rv_tree.p, m->rv_target.p, m->rv_splits.p};
+    std::vector<uint64_t> sig;
+    for (const void* q : ptrs) sig.push_back((uint64_t)(uintptr_t)q);
+    const int64_t ints[] = {m->n, m->d, m->k, m->ld, m->kc, m->R, m->sms, m->rec.batch_size, m->rec.total_steps,
+                            m->rec.passes, m->rec.rows_last_pass, (int64_t)m->seed, m->revival, m->finalize,
+                            m->capture, m->auto_revive, m->assign_kernel, m->wait_cycles, m->exact_ties};
+    for (int64_t v : ints) sig.push_back((uint64_t)v);
+    double dbl[] = {m->rec.alpha0, m->tau};
+    for (double v : dbl) {
+        uint64_t u;
+        memcpy(&u, &v, 8);
+        sig.push_back(u);
     }
+    return sig;
+}
+
+// Runs `count` steps from the current position as one CUDA graph (captured on a
+// private stream the first time this exact range is asked for, then replayed).
+static int run_steps_graph(em_model* m, int64_t count) {
+    const std::vector<uint64_t> sig = graph_signature(m);
+    const int64_t t0 = m->t;
+    for (auto& g : m->graph_cache) {
+        if (g.t0 == t0 && g.count == count && g.sig == sig) {
+            CK(cudaGraphLaunch(g.exec, m->stream));
+            for (int64_t i = 0; i < count; ++i) advance_step(m, plan_step(m));
+            EM_LAUNCHED(m, g.launches);
+            return EM_OK;
+        }
+    }
+    if (!m->cap_stream) CK(cudaStreamCreateWithFlags(&m->cap_stream, cudaStreamNonBlocking));
+    const int64_t save_t = m->t, save_pass = m->pass, save_pos = m->pos, save_rows = m->rows_assigned;
+    const int64_t save_last = m->last_rows, save_launches = m->launches;
+    const double save_alpha = m->last_alpha;
+    cudaStream_t user = m->stream;
+    m->stream = m->cap_stream;
+    CK(cudaStreamBeginCapture(m->cap_stream, cudaStreamCaptureModeThreadLocal));
+    int rc = EM_OK;
+    for (int64_t i = 0; i < count && rc == EM_OK; ++i) rc = run_step(m);
+    cudaGraph_t graph = nullptr;
+    const cudaError_t ce = cudaStreamEndCapture(m->cap_stream, &graph);
+    m->stream = user;
+    cudaGraphExec_t exec = nullptr;
+    if (rc == EM_OK && ce == cudaSuccess && graph &&
+        cudaGraphInstantiate(&exec, graph, 0) == cudaSuccess) {
+        cudaGraphDestroy(graph);
+        const int64_t launches = m->launches - save_launches;
+        if (m->graph_cache.size() >= 64) {
+            cudaGraphExecDestroy(m->graph_cache.front().exec);
+            m->graph_cache.erase(m->graph_cache.begin());
+        }
+        m->graph_cache.push_back({sig, t0, count, launches, exec});
+        CK(cudaGraphLaunch(exec, m->stream));
+        return EM_OK;
+    }
+    // capture did not work: undo the bookkeeping and launch the steps directly
+    if (graph) cudaGraphDestroy(graph);
+    cudaGetLastError();
+    m->t = save_t;
+    m->pass = save_pass;
+    m->pos = save_pos;
+    m->rows_assigned = save_rows;
+    m->last_rows = save_last;
+    m->last_alpha = save_alpha;
+    m->launches = save_launches;
+    for (int64_t i = 0; i < count; ++i) CKR(run_step(m));
     return EM_OK;
 }
 
@@ -609,7 +732,8 @@ em_model* em_create(int64_t d, int64_t k, uint64_t seed) {
         return bail(EM_E_CUDA, "cudaStreamCreate failed");
     m->own_stream = true;
     const size_t kd = (size_t)k * m->ld;
-    if (m->N.ensure(k) || m->S.ensure(kd) || m->c.ensure(kd) || m->cn.ensure(k) || m->cq.ensure(kd) ||
+    if (m->N.ensure(k) || m->N_prev.ensure(k) || m->cnp.ensure((size_t)k * ((m->nv + 31) / 32)) ||
+        m->S.ensure(kd) || m->c.ensure(kd) || m->cn.ensure(k) || m->cq.ensure(kd) ||
         m->close_sum.ensure(kd) || m->close_cnt.ensure(k) || m->err.ensure(1) || m->flag.ensure(1) ||
         m->scalar.ensure(4) || m->rv_dead.ensure(k) || m->rv_donor.ensure(k) || m->rv_order.ensure(k) ||
         m->rv_times.ensure(k) || m->rv_ndead.ensure(1) || m->rv_splits.ensure(1) || m->rv_target.ensure(k) ||
@@ -623,9 +747,13 @@ em_model* em_create(int64_t d, int64_t k, uint64_t seed) {
     cudaMemset(m->c.p, 0, kd * sizeof(float));
     cudaMemset(m->cq.p, 0, kd * sizeof(__nv_bfloat16));
     cudaMemset(m->cn.p, 0, k * sizeof(float));
-    if (cudaFuncSetAttribute(tc::k_assign_tc<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(tc::k_assign_tc<64, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              tc::Cfg<64>::kSmemBytes) != cudaSuccess ||
-        cudaFuncSetAttribute(tc::k_assign_tc<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaFuncSetAttribute(tc::k_assign_tc<32, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             tc::Cfg<32>::kSmemBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(tc::k_assign_tc<64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             tc::Cfg<64>::kSmemBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(tc::k_assign_tc<32, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              tc::Cfg<32>::kSmemBytes) != cudaSuccess ||
         cudaFuncSetAttribute(k_revive_select, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kReviveSmemBytes) != cudaSuccess)
@@ -642,12 +770,13 @@ void em_destroy(em_model* m) {
     if (!m) return;
     cudaSetDevice(m->dev);
     if (m->stream) cudaStreamSynchronize(m->stream);
-    m->N.release(); m->S.release(); m->c.release(); m->cn.release(); m->cq.release();
+    m->N.release(); m->N_prev.release(); m->cnp.release(); m->S.release(); m->c.release(); m->cn.release();
+    m->cq.release();
     m->close_sum.release(); m->close_cnt.release(); m->err.release(); m->flag.release();
     m->Xown.release(); m->stage.release(); m->Xb.release(); m->xn.release(); m->dists.release();
     m->ids.release(); m->labels.release(); m->cnt.release(); m->rank.release(); m->off.release();
-    m->perm.release(); m->slab.release(); m->keys.release(); m->block_err.release(); m->pfirst.release();
-    m->plast.release(); m->step_err.release(); m->scalar.release(); m->labels_last.release();
+    m->perm.release(); m->poff.release(); m->items.release(); m->keys.release(); m->block_err.release();
+    m->part.release(); m->step_err.release(); m->scalar.release(); m->labels_last.release();
     m->labels64.release(); m->rv_dead.release(); m->rv_donor.release(); m->rv_order.release();
     m->rv_times.release(); m->rv_ndead.release(); m->rv_tree.release(); m->rv_splits.release();
     m->rv_target.release();
@@ -656,6 +785,8 @@ void em_destroy(em_model* m) {
         cudaEventDestroy(sp.b);
     }
     for (auto ev : m->pool) cudaEventDestroy(ev);
+    for (auto& g : m->graph_cache) cudaGraphExecDestroy(g.exec);
+    if (m->cap_stream) cudaStreamDestroy(m->cap_stream);
     if (m->own_stream && m->stream) cudaStreamDestroy(m->stream);
     delete m;
 }
@@ -705,6 +836,10 @@ int em_set_option(em_model* m, int opt, double v) {
             m->assign_kernel = (int)v;
             break;
         case EM_OPT_PROFILE: m->profile = v != 0; break;
+        case EM_OPT_EXACT_TIES:
+            if (v != -1 && v != 0 && v != 1) return fail(EM_E_INVAL, "exact ties is -1, 0 or 1");
+            m->exact_ties = (int)v;
+            break;
         default: return fail(EM_E_INVAL, "unknown option %d", opt);
     }
     return EM_OK;
@@ -727,6 +862,7 @@ int em_get_option(const em_model* m, int opt, double* v) {
         case EM_OPT_GRAPHS: *v = m->graphs; break;
         case EM_OPT_ASSIGN_KERNEL: *v = m->assign_kernel; break;
         case EM_OPT_PROFILE: *v = m->profile; break;
+        case EM_OPT_EXACT_TIES: *v = m->exact_ties; break;
         default: return fail(EM_E_INVAL, "unknown option %d", opt);
     }
     return EM_OK;
@@ -757,6 +893,12 @@ int em_begin(em_model* m, const void* X, int64_t n, double epochs) {
     const int64_t b = m->rec.batch_size;
     CKR(m->Xb.ensure((size_t)b * m->ld));
     CKR(ensure_batch_buffers(m, b));
+    {  // every batch size the run will see: full batches and the last, partial ones
+        const int64_t sizes[3] = {b, n % b, m->rec.rows_last_pass % b};
+        size_t need = 0;
+        for (int64_t r : sizes) need = std::max(need, keys_needed(m, r));
+        CKR(m->keys.ensure(need));
+    }
     CKR(m->step_err.ensure(m->rec.total_steps));
     CK(cudaMemsetAsync(m->step_err.p, 0, m->rec.total_steps * sizeof(double), m->stream));
     CK(cudaMemsetAsync(m->cnt.p, 0, m->k * sizeof(int32_t), m->stream));
@@ -785,12 +927,13 @@ int em_step(em_model* m, int64_t nsteps, int64_t* done) {
     if (!m) return fail(EM_E_INVAL, "model is NULL");
     if (!m->running) return fail(EM_E_STATE, "no run in progress (call em_begin)");
     CKR(set_device(m));
-    int64_t ran = 0;
-    while (ran < nsteps && m->t < m->rec.total_steps) {
-        CKR(run_step(m));
-        ++ran;
+    const int64_t count = std::max<int64_t>(0, std::min(nsteps, m->rec.total_steps - m->t));
+    if (m->graphs && !m->profile && count >= 2) {
+        CKR(run_steps_graph(m, count));
+    } else {
+        for (int64_t i = 0; i < count; ++i) CKR(run_step(m));
     }
-    if (done) *done = ran;
+    if (done) *done = count;
     return EM_OK;
 }
 
@@ -831,18 +974,20 @@ int em_lloyd(em_model* m, const void* X, int64_t n, int64_t iters) {
     m->n = n;
     CKR(prepare_input(m, X, n, m->Xown, &m->X));
     CKR(ensure_batch_buffers(m, n));
+    CKR(m->keys.ensure(keys_needed(m, n)));
     CK(cudaMemsetAsync(m->cnt.p, 0, m->k * sizeof(int32_t), m->stream));
     CKR(start_centroids(m));
     CUtensorMap tmx;
     CKR(make_tmap(&tmx, m->X, n, (int)m->d, m->ld, tc::BM, m->kc));
     const int nbl = (int)((n + 255) / 256);
     for (int64_t it = 0; it < iters; ++it) {
-        k_rownorm_keys<<<grid_for(n * 32, 256, m->sms), 256, 0, m->stream>>>(m->X, n, m->ld, m->xn.p, m->keys.p);
+        k_rownorm_keys<<<grid_for(n * 32, 256, m->sms), 256, 0, m->stream>>>(m->X, n, m->ld, m->xn.p, nullptr);
         CK(cudaGetLastError());
         EM_LAUNCHED(m, 1);
         CKR(launch_assign(m, tmx, m->X, n));
-        k_labels<<<nbl, 256, 0, m->stream>>>(m->keys.p, m->xn.p, (int)n, (int)m->k, nullptr, m->labels.p,
-                                             m->dists.p, m->cnt.p, m->rank.p, m->block_err.p, nullptr, 0, m->err.p);
+        k_labels<<<nbl, 256, 0, m->stream>>>(m->keys.p, m->last_split, m->xn.p, (int)n, (int)m->k, m->X, m->ld,
+                                             m->cq.p, nullptr, m->labels.p, m->dists.p, m->cnt.p, m->rank.p,
+                                             m->block_err.p, nullptr, 0, m->err.p);
         CK(cudaGetLastError());
         EM_LAUNCHED(m, 1);
         CKR(launch_reduce(m, m->X, n, nbl, 1.0, 0, m->scalar.p));
@@ -857,17 +1002,17 @@ static int assign_pass(em_model* m, const void* X, int64_t n, int64_t* labels_de
     const __nv_bfloat16* A = nullptr;
     CKR(prepare_input(m, X, n, tmp, &A));
     CKR(m->xn.ensure(n));
-    CKR(m->keys.ensure(n));
+    CKR(m->keys.ensure(keys_needed(m, n)));
     CKR(m->block_err.ensure((n + 255) / 256 + 1));
-    k_rownorm_keys<<<grid_for(n * 32, 256, m->sms), 256, 0, m->stream>>>(A, n, m->ld, m->xn.p, m->keys.p);
+    k_rownorm_keys<<<grid_for(n * 32, 256, m->sms), 256, 0, m->stream>>>(A, n, m->ld, m->xn.p, nullptr);
     CK(cudaGetLastError());
     EM_LAUNCHED(m, 1);
     CUtensorMap tmx;
     CKR(make_tmap(&tmx, A, n, (int)m->d, m->ld, tc::BM, m->kc));
     CKR(launch_assign(m, tmx, A, n));
     const int blocks = grid_for(n, 256, m->sms);
-    k_assign_out<<<blocks, 256, 0, m->stream>>>(m->keys.p, m->xn.p, n, (int)m->k, labels_dev, dists_dev, nullptr,
-                                                m->block_err.p, m->err.p);
+    k_assign_out<<<blocks, 256, 0, m->stream>>>(m->keys.p, m->last_split, m->xn.p, n, (int)m->k, A, m->ld, m->cq.p,
+                                                labels_dev, dists_dev, nullptr, m->block_err.p, m->err.p);
     CK(cudaGetLastError());
     k_sum_blocks<<<1, 32, 0, m->stream>>>(m->block_err.p, blocks, sum_dev);
     CK(cudaGetLastError());
@@ -1126,8 +1271,8 @@ constexpr size_t kNaErr = 0;                                                   /
 constexpr size_t kNaCn = 256;                                                  // fp32 [MAX_K]
 constexpr size_t kNaOperand = kNaCn + (size_t)EM_NOALLOC_MAX_K * 4;            // bf16 [MAX_KD]
 constexpr size_t kNaXn = kNaOperand + (size_t)EM_NOALLOC_MAX_KD * 2;           // fp32 [MAX_ROWS]
-constexpr size_t kNaKeys = kNaXn + (size_t)EM_NOALLOC_MAX_ROWS * 4;            // u64 [MAX_ROWS]
-constexpr size_t kNaBlocks = kNaKeys + (size_t)EM_NOALLOC_MAX_ROWS * 8;        // fp64 [kNaMaxBlocks]
+constexpr size_t kNaKeys = kNaXn + (size_t)EM_NOALLOC_MAX_ROWS * 4;            // u64 [2 * MAX_ROWS]
+constexpr size_t kNaBlocks = kNaKeys + (size_t)EM_NOALLOC_MAX_ROWS * 16;       // fp64 [kNaMaxBlocks]
 constexpr int kNaMaxBlocks = 4096;
 constexpr size_t kNaEnd = kNaBlocks + (size_t)kNaMaxBlocks * 8;
 static_assert(kNaEnd <= EM_NOALLOC_SCRATCH_BYTES, "scratch layout exceeds the array");
@@ -1176,9 +1321,13 @@ int noalloc_scratch(int dev, unsigned char** out) {
             cudaGetLastError();
             return fail(EM_E_CUDA, "cudaGetSymbolAddress of the scratch array failed: %s", cudaGetErrorString(e));
         }
-        if (cudaFuncSetAttribute(tc::k_assign_tc<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(tc::k_assign_tc<64, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  tc::Cfg<64>::kSmemBytes) != cudaSuccess ||
-            cudaFuncSetAttribute(tc::k_assign_tc<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            cudaFuncSetAttribute(tc::k_assign_tc<32, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 tc::Cfg<32>::kSmemBytes) != cudaSuccess ||
+            cudaFuncSetAttribute(tc::k_assign_tc<64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 tc::Cfg<64>::kSmemBytes) != cudaSuccess ||
+            cudaFuncSetAttribute(tc::k_assign_tc<32, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  tc::Cfg<32>::kSmemBytes) != cudaSuccess)
             return fail(EM_E_CUDA, "cudaFuncSetAttribute failed");
         g_na_base[dev] = static_cast<unsigned char*>(p);
@@ -1223,21 +1372,33 @@ extern "C" int em_assign_noalloc(const void* X, int64_t n, int64_t d, const floa
     const auto X16 = reinterpret_cast<const __nv_bfloat16*>(X);
     CK(cudaMemsetAsync(err, 0, sizeof(int), stream));  // the previous call's error word is stale
     k_operand_from_centroids<<<grid_for(k * 32, 256, sms), 256, 0, stream>>>(centroids, (int)k, (int)d, cq, cn);
-    k_rownorm_keys<<<grid_for(n * 32, 256, sms), 256, 0, stream>>>(X16, n, (int)d, xn, keys);
+    k_rownorm_keys<<<grid_for(n * 32, 256, sms), 256, 0, stream>>>(X16, n, (int)d, xn, nullptr);
     const int64_t m_tiles = (n + tc::BM - 1) / tc::BM;
     const int64_t n_tiles = (k + tc::BN - 1) / tc::BN;
     const int nkc = (int)((d + kc - 1) / kc);
-    const int split = choose_split(m_tiles, n_tiles, sms);
+    // the key region holds two keys for EM_NOALLOC_MAX_ROWS rows: split * n rows at most
+    const int split = choose_split(m_tiles, n_tiles, sms, (int)std::max<int64_t>(1, EM_NOALLOC_MAX_ROWS / n));
+    const bool top2 = d >= 256;
     const int grid = (int)std::min<int64_t>(m_tiles * split, sms);
     const long long wait_cycles = (long long)(2000.0 * (double)clock_khz);
-    if (kc == 64)
-        tc::k_assign_tc<64><<<grid, tc::kThreads, tc::Cfg<64>::kSmemBytes, stream>>>(
-            tmA, tmB, cn, (int)k, (int)n, nkc, (int)n_tiles, split, keys, wait_cycles, err);
-    else
-        tc::k_assign_tc<32><<<grid, tc::kThreads, tc::Cfg<32>::kSmemBytes, stream>>>(
-            tmA, tmB, cn, (int)k, (int)n, nkc, (int)n_tiles, split, keys, wait_cycles, err);
+#define EM_NA_ASSIGN(KC, T2)                                                                       \
+    tc::k_assign_tc<KC, T2><<<grid, tc::kThreads, tc::Cfg<KC>::kSmemBytes, stream>>>( \
+        tmA, tmB, cn, (int)k, (int)n, nkc, (int)n_tiles, split, keys, wait_cycles, err)
+    if (kc == 64) {
+        if (top2)
+            EM_NA_ASSIGN(64, true);
+        else
+            EM_NA_ASSIGN(64, false);
+    } else {
+        if (top2)
+            EM_NA_ASSIGN(32, true);
+        else
+            EM_NA_ASSIGN(32, false);
+    }
+#undef EM_NA_ASSIGN
     const int oblocks = std::min(grid_for(n, 256, sms), kNaMaxBlocks);
-    k_assign_out<<<oblocks, 256, 0, stream>>>(keys, xn, n, (int)k, labels, dists, nullptr, blocks, err);
+    k_assign_out<<<oblocks, 256, 0, stream>>>(keys, split, xn, n, (int)k, X16, (int)d, cq, labels, dists, nullptr,
+                                             blocks, err);
     CK(cudaGetLastError());
     int h = 0;
     CK(cudaMemcpyAsync(&h, err, sizeof(int), cudaMemcpyDeviceToHost, stream));

@@ -15,8 +15,10 @@
 //   warps 2..5  epilogue: tcgen05.ld of the 128 x 256 fp32 tile (thread = row),
 //               add |c|^2, running argmin; frees the accumulator for the next tile
 // A work unit is (128-row tile, group of 256-wide centroid tiles). When k is
-// split over several units, the per-row results are merged with a 64-bit
-// atomicMin on (order-preserving score, index) keys.
+// split over several units, every group writes its own per-row result
+// ((order-preserving score, index) keys) and the label kernel merges them. With
+// TOP2 the epilogue also keeps the second best candidate, so that near ties can be
+// settled exactly afterwards.
 #pragma once
 
 #include "common.cuh"
@@ -169,7 +171,10 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
 
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
-template <int KC>
+// Output: for every row, the split g of the centroid tiles it covers writes two
+// keys at keys[(g * rows + row) * 2 + {0, 1}]: the best (score, index) and, with
+// TOP2, the second best (without it the second key is empty).
+template <int KC, bool TOP2>
 __global__ void __launch_bounds__(kThreads, 1)
     k_assign_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const float* __restrict__ cn, int k, int rows, int nkc, int n_tiles, int n_split,
@@ -324,7 +329,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int m = u / n_split, g = u - m * n_split;
             const int nt0 = g * tpg, nt1 = min(nt0 + tpg, n_tiles);
             float best = __int_as_float(0x7f800000);  // +inf
-            int bidx = 0;
+            float best2 = best;
+            int bidx = 0, bidx2 = 0;
             for (int nt = nt0; nt < nt1; ++nt) {
                 float* cnb = cn_s + cnbuf * BN;
                 const int j0 = nt * BN;
@@ -342,36 +348,35 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t tbase = tmem_base + lane_base + (uint32_t)(acc * BN);
 #pragma unroll 1
                 for (int ch = 0; ch < BN / 32; ch += 2) {
-                    uint32_t v0[32], v1[32];
-                    tmem_ld32(tbase + ch * 32, v0);
-                    tmem_ld32(tbase + ch * 32 + 32, v1);
+                    uint32_t v[2][32];
+                    tmem_ld32(tbase + ch * 32, v[0]);
+                    tmem_ld32(tbase + ch * 32 + 32, v[1]);
                     tmem_wait_ld();
                     const float4* c4 = reinterpret_cast<const float4*>(cnb + ch * 32);
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const float4 cc = c4[i];
-                        const float s0 = cc.x + __uint_as_float(v0[4 * i + 0]);
-                        const float s1 = cc.y + __uint_as_float(v0[4 * i + 1]);
-                        const float s2 = cc.z + __uint_as_float(v0[4 * i + 2]);
-                        const float s3 = cc.w + __uint_as_float(v0[4 * i + 3]);
-                        const int jb = j0 + ch * 32 + 4 * i;
-                        if (s0 < best) { best = s0; bidx = jb; }
-                        if (s1 < best) { best = s1; bidx = jb + 1; }
-                        if (s2 < best) { best = s2; bidx = jb + 2; }
-                        if (s3 < best) { best = s3; bidx = jb + 3; }
-                    }
+                    for (int h = 0; h < 2; ++h) {
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const float4 cc = c4[8 + i];
-                        const float s0 = cc.x + __uint_as_float(v1[4 * i + 0]);
-                        const float s1 = cc.y + __uint_as_float(v1[4 * i + 1]);
-                        const float s2 = cc.z + __uint_as_float(v1[4 * i + 2]);
-                        const float s3 = cc.w + __uint_as_float(v1[4 * i + 3]);
-                        const int jb = j0 + ch * 32 + 32 + 4 * i;
-                        if (s0 < best) { best = s0; bidx = jb; }
-                        if (s1 < best) { best = s1; bidx = jb + 1; }
-                        if (s2 < best) { best = s2; bidx = jb + 2; }
-                        if (s3 < best) { best = s3; bidx = jb + 3; }
+                        for (int i = 0; i < 8; ++i) {
+                            const float4 cc = c4[8 * h + i];
+                            const float sc[4] = {cc.x + __uint_as_float(v[h][4 * i + 0]),
+                                                 cc.y + __uint_as_float(v[h][4 * i + 1]),
+                                                 cc.z + __uint_as_float(v[h][4 * i + 2]),
+                                                 cc.w + __uint_as_float(v[h][4 * i + 3])};
+                            const int jb = j0 + ch * 32 + 32 * h + 4 * i;
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                if (TOP2) {  // branch-free: a divergent skip test measured slower
+                                    const bool p1 = sc[e] < best, p2 = sc[e] < best2;
+                                    best2 = p1 ? best : (p2 ? sc[e] : best2);
+                                    bidx2 = p1 ? bidx : (p2 ? jb + e : bidx2);
+                                    best = p1 ? sc[e] : best;
+                                    bidx = p1 ? jb + e : bidx;
+                                } else if (sc[e] < best) {
+                                    best = sc[e];
+                                    bidx = jb + e;
+                                }
+                            }
+                        }
                     }
                 }
                 tc_fence_before();
@@ -383,11 +388,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!ok) break;
             const int row = m * BM + 32 * q + lane;
             if (row < rows) {
-                const unsigned long long key = pack_key(best, (uint32_t)bidx);
-                if (n_split > 1)
-                    atomicMin(&keys[row], key);
-                else
-                    keys[row] = key;
+                unsigned long long* out = keys + ((int64_t)g * rows + row) * 2;
+                out[0] = pack_key(best, (uint32_t)bidx);
+                out[1] = TOP2 && best2 < __int_as_float(0x7f800000) ? pack_key(best2, (uint32_t)bidx2) : kEmptyKey;
             }
         }
     }
@@ -423,7 +426,8 @@ __global__ void k_assign_simt(const __nv_bfloat16* __restrict__ A, int ld, int r
             bidx = j;
         }
     }
-    keys[row] = pack_key(best, (uint32_t)bidx);
+    keys[(int64_t)row * 2] = pack_key(best, (uint32_t)bidx);
+    keys[(int64_t)row * 2 + 1] = kEmptyKey;
 }
 
 }  // namespace em

@@ -151,13 +151,12 @@ __global__ void k_init_centroids(const __nv_bfloat16* __restrict__ X, int64_t n,
 }
 
 // Batch gather: row r of the batch is data row pi_pass(base + r); copies it into the
-// contiguous batch buffer, records its id, its squared norm |x|^2 (fp32, from the
-// bf16 values) and resets its search key. Each lane computes one row id; the warp
-// then moves the 32 rows one after another.
+// contiguous batch buffer, records its id and its squared norm |x|^2 (fp32, from the
+// bf16 values). Each lane computes one row id; the warp
+// then moves the 32 rows four at a time (four independent loads in flight per lane).
 __global__ void k_gather(const __nv_bfloat16* __restrict__ X, int64_t n, int ld, uint64_t seed, int64_t pass,
                          int64_t base, int rows, int natural_order, __nv_bfloat16* __restrict__ Xb,
-                         float* __restrict__ xn, int32_t* __restrict__ ids, unsigned long long* __restrict__ keys,
-                         int* err) {
+                         float* __restrict__ xn, int32_t* __restrict__ ids, int* err) {
     const int lane = threadIdx.x & 31;
     const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int nwarps = (gridDim.x * blockDim.x) >> 5;
@@ -175,24 +174,38 @@ __global__ void k_gather(const __nv_bfloat16* __restrict__ X, int64_t n, int ld,
                 id = 0;
             }
             ids[r] = (int32_t)id;
-            keys[r] = kEmptyKey;
         }
         const int cnt = min(32, rows - r0);
-        for (int q = 0; q < cnt; ++q) {
-            const int64_t src = __shfl_sync(0xFFFFFFFFu, id, q);
-            const uint4* s = reinterpret_cast<const uint4*>(X + src * ld);
-            uint4* dstp = reinterpret_cast<uint4*>(Xb + (int64_t)(r0 + q) * ld);
-            float acc = 0.0f;
-            for (int v = lane; v < nv; v += 32) {
-                uint4 u = s[v];
-                dstp[v] = u;
-                float x[8];
-                unpack8_bf16(u, x);
+        for (int q = 0; q < cnt; q += 4) {
+            int64_t src[4];
+            float acc[4];
 #pragma unroll
-                for (int i = 0; i < 8; ++i) acc = fmaf(x[i], x[i], acc);
+            for (int u = 0; u < 4; ++u) {
+                src[u] = __shfl_sync(0xFFFFFFFFu, id, min(q + u, cnt - 1));
+                acc[u] = 0.0f;
             }
-            acc = warp_sum(acc);
-            if (lane == 0) xn[r0 + q] = acc;
+            for (int v = lane; v < nv; v += 32) {
+                uint4 val[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) val[u] = reinterpret_cast<const uint4*>(X + src[u] * ld)[v];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    if (q + u < cnt) {
+                        reinterpret_cast<uint4*>(Xb + (int64_t)(r0 + q + u) * ld)[v] = val[u];
+                        float x[8];
+                        unpack8_bf16(val[u], x);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) acc[u] = fmaf(x[i], x[i], acc[u]);
+                    }
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) acc[u] = warp_sum(acc[u]);
+            if (lane == 0) {
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                    if (q + u < cnt) xn[r0 + q + u] = acc[u];
+            }
         }
     }
 }
@@ -217,7 +230,7 @@ __global__ void k_rownorm_keys(const __nv_bfloat16* __restrict__ X, int64_t rows
         acc = warp_sum(acc);
         if (lane == 0) {
             xn[r] = acc;
-            keys[r] = kEmptyKey;
+            if (keys) keys[r] = kEmptyKey;
         }
     }
 }

@@ -8,14 +8,17 @@
 //   k_labels   decodes each row's search key, counts labels per cluster with
 //              warp-aggregated atomics (__match_any_sync: one atomic per distinct
 //              label per warp) and records each row's rank inside its cluster;
-//   k_offsets  exclusive scan of the counts (segment starts), batch error sum;
-//   k_scatter  writes row ids into label order (perm) with their labels (slab);
-//   k_segsum   walks perm in fixed-size tiles (one warp per tile, so a cluster
-//              with many rows is spread over many warps): a run of equal labels
-//              that lies inside one tile is summed (fp64) and updated at once;
-//              a run cut by a tile edge leaves its partial sum in a per-tile slot;
-//   k_fixup    adds the partial sums of every cut cluster in tile order and
-//              updates it, and decays clusters that received no row.
+//   k_offsets  exclusive scans of the counts (segment starts) and of the chunk
+//              counts (work items), batch error sum;
+//   k_scatter  writes row ids into label order (perm) and one work item per chunk;
+//   k_segsum   one warp per (chunk of at most R rows of one cluster, 256-dim
+//              slice), so a cluster with many rows is spread over many warps and
+//              small clusters never wait on each other: a cluster of one chunk is
+//              summed (fp64) and updated at once; the chunks of a larger cluster
+//              leave partial sums;
+//   k_clusters one warp per cluster: adds the chunk partials of large clusters in
+//              chunk order and updates them, decays clusters that received no row,
+//              and assembles |bf16(c)|^2.
 // Sums are accumulated in fp64 from bf16 values, which makes them independent of
 // the order rows arrive in (the fp64 sum of bf16 values is exact for the data
 // ranges used here), so the update is deterministic.
@@ -25,8 +28,6 @@
 
 namespace em {
 
-constexpr int kMaxVpl = 8;  // 16-byte vectors per lane in one slice: 32 lanes x 8 x 8 = 2048 dims
-
 struct StepParams {
     double alpha;        // step size of this step
     int last_pass;       // accumulate the closing-mean statistics
@@ -35,25 +36,101 @@ struct StepParams {
 
 // ---------------------------------------------------------------- labels + histogram
 
-__global__ void k_labels(const unsigned long long* __restrict__ keys, const float* __restrict__ xn, int rows, int k,
-                         const int32_t* __restrict__ ids, int32_t* __restrict__ labels, float* __restrict__ dists,
-                         int32_t* __restrict__ cnt, int32_t* __restrict__ rank, double* __restrict__ block_err,
-                         int64_t* __restrict__ labels_last, int capture, int* err) {
+// Relative size of a near tie, measured against |x|^2 + |s1| + |s2|: a gap between the
+// two best scores above this can not be reversed by the fp32 accumulation of the
+// search, a smaller one is settled exactly.
+constexpr float kTieRel = 3e-5f;
+
+// Best and second best keys of row r over the splits of the search.
+__device__ __forceinline__ void merge_keys(const unsigned long long* __restrict__ keys, int64_t rows, int nsplit,
+                                           int64_t r, unsigned long long& k1, unsigned long long& k2) {
+    k1 = kEmptyKey;
+    k2 = kEmptyKey;
+    for (int g = 0; g < nsplit; ++g) {
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const unsigned long long c = keys[((int64_t)g * rows + r) * 2 + e];
+            if (c < k1) {
+                k2 = k1;
+                k1 = c;
+            } else if (c < k2) {
+                k2 = c;
+            }
+        }
+    }
+}
+
+// For every lane of the warp whose row is a near tie (flag), the warp recomputes
+// |x - c|^2 of both candidates in fp64 from the bf16 row and the bf16 operands
+// (c = -q / 2, exact) and keeps the smaller (the lower index on an exact tie).
+__device__ __forceinline__ void settle_ties(bool flag, int64_t row, uint32_t& l1, float& s1, uint32_t l2, float s2,
+                                            const __nv_bfloat16* __restrict__ A, int ld,
+                                            const __nv_bfloat16* __restrict__ cq, int lane) {
+    unsigned fm = __ballot_sync(0xFFFFFFFFu, flag);
+    const int nv = ld / 8;
+    while (fm) {
+        const int q = __ffs(fm) - 1;
+        fm &= fm - 1;
+        const int64_t rq = __shfl_sync(0xFFFFFFFFu, row, q);
+        const uint32_t la = __shfl_sync(0xFFFFFFFFu, l1, q), lb = __shfl_sync(0xFFFFFFFFu, l2, q);
+        double da = 0.0, db = 0.0;
+        for (int v = lane; v < nv; v += 32) {
+            float x[8], qa[8], qb[8];
+            unpack8_bf16(reinterpret_cast<const uint4*>(A + rq * ld)[v], x);
+            unpack8_bf16(reinterpret_cast<const uint4*>(cq + (int64_t)la * ld)[v], qa);
+            unpack8_bf16(reinterpret_cast<const uint4*>(cq + (int64_t)lb * ld)[v], qb);
+#pragma unroll
+            for (int t = 0; t < 8; ++t) {
+                const double ea = (double)x[t] + 0.5 * (double)qa[t];
+                const double eb = (double)x[t] + 0.5 * (double)qb[t];
+                da += ea * ea;
+                db += eb * eb;
+            }
+        }
+        da = warp_sum(da);
+        db = warp_sum(db);
+        if (lane == q && (db < da || (db == da && lb < la))) {
+            l1 = lb;
+            s1 = s2;
+        }
+    }
+}
+
+__global__ void k_labels(const unsigned long long* __restrict__ keys, int nsplit, const float* __restrict__ xn,
+                         int rows, int k, const __nv_bfloat16* __restrict__ A, int ld,
+                         const __nv_bfloat16* __restrict__ cq, const int32_t* __restrict__ ids,
+                         int32_t* __restrict__ labels, float* __restrict__ dists, int32_t* __restrict__ cnt,
+                         int32_t* __restrict__ rank, double* __restrict__ block_err, int64_t* __restrict__ labels_last,
+                         int capture, int* err) {
     __shared__ double warp_err[32];
     const int lane = threadIdx.x & 31;
     double e = 0.0;
     const int r = blockIdx.x * blockDim.x + threadIdx.x;
     const bool active = r < rows;
+    uint32_t l1 = 0, l2 = 0;
+    float s1 = 0.0f, s2 = 0.0f, x2 = 0.0f;
+    bool tie = false;
+    if (active) {
+        unsigned long long k1, k2;
+        merge_keys(keys, rows, nsplit, r, k1, k2);
+        l1 = key_label(k1);
+        s1 = key_score(k1);
+        x2 = xn[r];
+        if (l1 >= (uint32_t)k) {  // a row that was never searched, or a corrupted key
+            raise_error(err, EM_E_BOUNDS);
+            l1 = 0;
+        }
+        if (k2 != kEmptyKey) {
+            l2 = key_label(k2);
+            s2 = key_score(k2);
+            tie = l2 < (uint32_t)k && s2 - s1 <= kTieRel * (x2 + fabsf(s1) + fabsf(s2));
+        }
+    }
+    settle_ties(tie, r, l1, s1, l2, s2, A, ld, cq, lane);
     int lab = -1;
     if (active) {
-        const unsigned long long key = keys[r];
-        uint32_t l = key_label(key);
-        if (l >= (uint32_t)k) {  // a row that was never searched, or a corrupted key
-            raise_error(err, EM_E_BOUNDS);
-            l = 0;
-        }
-        lab = (int)l;
-        const float dist = fmaxf(0.0f, xn[r] + key_score(key));
+        lab = (int)l1;
+        const float dist = fmaxf(0.0f, x2 + s1);
         labels[r] = lab;
         dists[r] = dist;
         e = (double)dist;
@@ -79,332 +156,368 @@ __global__ void k_labels(const unsigned long long* __restrict__ keys, const floa
     }
 }
 
-// Exclusive scan of cnt[0..k) into off[0..k]; one CTA of 1024 threads in tiles of
-// 4096 counts. Also adds the per-block error sums in block order.
-__global__ void __launch_bounds__(1024) k_offsets(const int32_t* __restrict__ cnt, int k, int rows,
-                                                  int32_t* __restrict__ off, const double* __restrict__ block_err,
-                                                  int nblocks, double* __restrict__ err_sum_out, int* err) {
-    __shared__ int32_t warp_tot[32];
-    __shared__ int32_t carry_s;
+// Exclusive scans of the counts (segment starts off[0..k]) and of the chunk counts
+// ceil(n_j / R) (first work item of each cluster, poff[0..k]); one CTA of 1024
+// threads in tiles of 4096 clusters. Also adds the per-block error sums in block
+// order and keeps the running counts of before this step (N_prev).
+__global__ void __launch_bounds__(1024) k_offsets(const int32_t* __restrict__ cnt, int k, int rows, int R,
+                                                  int32_t* __restrict__ off, int32_t* __restrict__ poff,
+                                                  const double* __restrict__ block_err, int nblocks,
+                                                  double* __restrict__ err_sum_out, const float* __restrict__ N,
+                                                  float* __restrict__ N_prev, int* err) {
+    __shared__ int2 warp_tot[32];
+    __shared__ int2 carry_s;
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
-    if (tid == 0) carry_s = 0;
+    for (int j = tid; j < k; j += 1024) N_prev[j] = N[j];
+    if (tid == 0) carry_s = make_int2(0, 0);
     __syncthreads();
     for (int base = 0; base < k; base += 4096) {
-        int v[4];
+        int v[4], c[4];
         const int i0 = base + tid * 4;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) v[i] = (i0 + i < k) ? cnt[i0 + i] : 0;
-        const int local = v[0] + v[1] + v[2] + v[3];
-        int incl = local;
+        for (int i = 0; i < 4; ++i) {
+            v[i] = (i0 + i < k) ? cnt[i0 + i] : 0;
+            c[i] = (v[i] + R - 1) / R;
+        }
+        const int local_v = v[0] + v[1] + v[2] + v[3];
+        const int local_c = c[0] + c[1] + c[2] + c[3];
+        int iv = local_v, ic = local_c;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
-            const int t = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-            if (lane >= o) incl += t;
+            const int tv = __shfl_up_sync(0xFFFFFFFFu, iv, o);
+            const int tc = __shfl_up_sync(0xFFFFFFFFu, ic, o);
+            if (lane >= o) {
+                iv += tv;
+                ic += tc;
+            }
         }
-        if (lane == 31) warp_tot[w] = incl;
+        if (lane == 31) warp_tot[w] = make_int2(iv, ic);
         __syncthreads();
         if (w == 0) {
-            int x = warp_tot[lane];
-            int xi = x;
+            const int2 x = warp_tot[lane];
+            int xv = x.x, xc = x.y;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
-                const int t = __shfl_up_sync(0xFFFFFFFFu, xi, o);
-                if (lane >= o) xi += t;
+                const int tv = __shfl_up_sync(0xFFFFFFFFu, xv, o);
+                const int tc = __shfl_up_sync(0xFFFFFFFFu, xc, o);
+                if (lane >= o) {
+                    xv += tv;
+                    xc += tc;
+                }
             }
-            warp_tot[lane] = xi - x;  // exclusive prefix of warp totals
+            warp_tot[lane] = make_int2(xv - x.x, xc - x.y);  // exclusive prefixes of the warp totals
         }
         __syncthreads();
-        const int carry = carry_s;
-        int run = carry + warp_tot[w] + incl - local;
+        const int2 carry = carry_s;
+        int rv = carry.x + warp_tot[w].x + iv - local_v;
+        int rc = carry.y + warp_tot[w].y + ic - local_c;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            if (i0 + i < k) off[i0 + i] = run;
-            run += v[i];
+            if (i0 + i < k) {
+                off[i0 + i] = rv;
+                poff[i0 + i] = rc;
+            }
+            rv += v[i];
+            rc += c[i];
         }
         __syncthreads();
-        if (tid == 1023) carry_s = run;
+        if (tid == 1023) carry_s = make_int2(rv, rc);
         __syncthreads();
     }
-    if (tid == 0) {
-        off[k] = carry_s;
-        if (carry_s != rows) raise_error(err, EM_E_BOUNDS);
+    if (w == 0) {  // batch error: lane-strided partial sums, then a fixed butterfly
         double t = 0.0;
-        for (int b = 0; b < nblocks; ++b) t += block_err[b];
-        *err_sum_out = t;
+        for (int b = lane; b < nblocks; b += 32) t += block_err[b];
+        t = warp_sum(t);
+        if (lane == 0) {
+            off[k] = carry_s.x;
+            poff[k] = carry_s.y;
+            if (carry_s.x != rows) raise_error(err, EM_E_BOUNDS);
+            *err_sum_out = t;
+        }
     }
 }
 
+// perm[pos] is the row the segmented sums read. The first row of every chunk of R
+// rows of a cluster also writes that chunk's work item (cluster, first sorted position).
 __global__ void k_scatter(const int32_t* __restrict__ labels, const int32_t* __restrict__ rank,
-                          const int32_t* __restrict__ off, int rows, int32_t* __restrict__ perm,
-                          int32_t* __restrict__ slab, int* err) {
+                          const int32_t* __restrict__ off, const int32_t* __restrict__ poff, int rows, int R,
+                          int32_t* __restrict__ perm, int2* __restrict__ items, int* err) {
     const int r = blockIdx.x * blockDim.x + threadIdx.x;
     if (r >= rows) return;
     const int lab = labels[r];
-    const int pos = off[lab] + rank[r];
+    const int rk = rank[r];
+    const int pos = off[lab] + rk;
     if (pos < 0 || pos >= rows) {
         raise_error(err, EM_E_BOUNDS);
         return;
     }
     perm[pos] = r;
-    slab[pos] = lab;
+    if (rk % R == 0) items[poff[lab] + rk / R] = make_int2(lab, pos);
 }
 
-// ---------------------------------------------------------------- EMA of one cluster
+// ---------------------------------------------------------------- segmented sums + EMA
 
-// Sums of one slice of dimensions, held by one warp: lane owns vectors
-// v = slice_base + i * 32 + lane (i < VPL) of 8 dims each.
-template <int VPL>
-struct SliceAcc {
-    double a[VPL][8];
-    __device__ __forceinline__ void zero() {
-#pragma unroll
-        for (int i = 0; i < VPL; ++i)
-#pragma unroll
-            for (int t = 0; t < 8; ++t) a[i][t] = 0.0;
-    }
-};
-
-template <int VPL>
-__device__ __forceinline__ void acc_rows(SliceAcc<VPL>& acc, const __nv_bfloat16* __restrict__ src, int ld,
-                                         const int32_t* __restrict__ perm, int s0, int s1, int vbase, int nv,
-                                         int lane) {
-    int s = s0;
-    for (; s + 1 < s1; s += 2) {  // two rows in flight
-        const int64_t r0 = perm[s], r1 = perm[s + 1];
-        const uint4* p0 = reinterpret_cast<const uint4*>(src + r0 * ld);
-        const uint4* p1 = reinterpret_cast<const uint4*>(src + r1 * ld);
-        uint4 u0[VPL], u1[VPL];
-#pragma unroll
-        for (int i = 0; i < VPL; ++i) {
-            const int v = vbase + i * 32 + lane;
-            if (v < nv) {
-                u0[i] = p0[v];
-                u1[i] = p1[v];
-            }
-        }
-#pragma unroll
-        for (int i = 0; i < VPL; ++i) {
-            const int v = vbase + i * 32 + lane;
-            if (v < nv) {
-                float x0[8], x1[8];
-                unpack8_bf16(u0[i], x0);
-                unpack8_bf16(u1[i], x1);
-#pragma unroll
-                for (int t = 0; t < 8; ++t) acc.a[i][t] += (double)x0[t] + (double)x1[t];
-            }
-        }
-    }
-    if (s < s1) {
-        const int64_t r0 = perm[s];
-        const uint4* p0 = reinterpret_cast<const uint4*>(src + r0 * ld);
-#pragma unroll
-        for (int i = 0; i < VPL; ++i) {
-            const int v = vbase + i * 32 + lane;
-            if (v < nv) {
-                float x0[8];
-                unpack8_bf16(p0[v], x0);
-#pragma unroll
-                for (int t = 0; t < 8; ++t) acc.a[i][t] += (double)x0[t];
-            }
-        }
-    }
-}
-
+// State the update kernels read and write. N_prev is the running count before this
+// step (copied by k_offsets), so that every slice of a cluster derives the same new
+// count; cnp[s * k + j] is slice s's part of |bf16(c_j)|^2, added in slice order by
+// k_clusters.
 struct ClusterState {
     float* N;
+    float* N_prev;
     float* S;
     float* c;
     __nv_bfloat16* cq;
     float* cn;
+    float* cnp;
     double* close_sum;
     double* close_cnt;
     int ld;
+    int k;
 };
 
-// EMA update of one slice of cluster j with batch count nj and slice sums acc.
-// Returns this lane's part of |bf16(c_j)|^2 over the slice.
-template <int VPL>
-__device__ __forceinline__ float ema_slice(const ClusterState& st, int j, double nj, double Nnew_d, float Nnew,
-                                           const SliceAcc<VPL>& acc, int vbase, int nv, int lane, double alpha,
-                                           int last_pass) {
-    const double a1 = 1.0 - alpha;
-    float cn_part = 0.0f;
-    float* Srow = st.S + (int64_t)j * st.ld;
-    float* crow = st.c + (int64_t)j * st.ld;
-    __nv_bfloat16* qrow = st.cq + (int64_t)j * st.ld;
+// A slice is 32 16-byte vectors (256 dims) of a row. A warp covers a slice of
+// `rpi` rows at once: lane l handles vector (l % lpr) of row (l / lpr), lpr being
+// the lanes per row (32, or fewer when the row has fewer than 32 vectors).
+struct SliceGeom {
+    int vbase;  // first vector of the slice
+    int nvs;    // vectors in this slice
+    int lpr;    // lanes per row (power of two >= nvs, <= 32)
+    int rpi;    // rows per warp iteration = 32 / lpr
+};
+
+__device__ __forceinline__ SliceGeom slice_geom(int slice, int nv) {
+    SliceGeom g;
+    g.vbase = slice * 32;
+    g.nvs = min(32, nv - g.vbase);
+    int l = 1;
+    while (l < g.nvs) l <<= 1;
+    g.lpr = l;
+    g.rpi = 32 / l;
+    return g;
+}
+
+// Sum over rows perm[s0..s1) of this lane's vector, fp64; the warp's row groups are
+// folded together at the end with a fixed butterfly, so lanes l < lpr hold the
+// slice totals of vector vbase + l.
+__device__ __forceinline__ void sum_rows(double acc[8], const __nv_bfloat16* __restrict__ src, int ld,
+                                         const int32_t* __restrict__ perm, int s0, int s1, const SliceGeom& g,
+                                         int lane) {
 #pragma unroll
-    for (int i = 0; i < VPL; ++i) {
-        const int v = vbase + i * 32 + lane;
-        if (v < nv) {
-            float4* sp = reinterpret_cast<float4*>(Srow) + 2 * v;
-            const float4 s0 = sp[0], s1 = sp[1];
-            const float so[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
-            float sn[8], cv[8];
+    for (int t = 0; t < 8; ++t) acc[t] = 0.0;
+    const int sub = lane / g.lpr, vi = lane % g.lpr;
+    const bool vec_ok = vi < g.nvs;
+    const int v = g.vbase + vi;
+    for (int s = s0; s < s1; s += 4 * g.rpi) {
+        uint4 u[4];
+        bool have[4];
 #pragma unroll
-            for (int t = 0; t < 8; ++t) {
-                sn[t] = (float)(a1 * (double)so[t] + alpha * acc.a[i][t]);
-                cv[t] = Nnew > 0.0f ? (float)((double)sn[t] / (double)Nnew) : 0.0f;
-            }
-            sp[0] = make_float4(sn[0], sn[1], sn[2], sn[3]);
-            sp[1] = make_float4(sn[4], sn[5], sn[6], sn[7]);
-            if (Nnew > 0.0f) store_centroid_vec(crow, qrow, v, cv, cn_part);
-            if (last_pass) {
-                double* cs = st.close_sum + (int64_t)j * st.ld + 8 * v;
+        for (int q = 0; q < 4; ++q) {  // up to four rows in flight per lane
+            const int slot = s + q * g.rpi + sub;
+            have[q] = vec_ok && slot < s1;
+            if (have[q]) u[q] = reinterpret_cast<const uint4*>(src + (int64_t)perm[slot] * ld)[v];
+        }
 #pragma unroll
-                for (int t = 0; t < 8; ++t) cs[t] += acc.a[i][t];
+        for (int q = 0; q < 4; ++q) {
+            if (have[q]) {
+                float x[8];
+                unpack8_bf16(u[q], x);
+#pragma unroll
+                for (int t = 0; t < 8; ++t) acc[t] += (double)x[t];
             }
         }
     }
-    (void)nj;
-    (void)Nnew_d;
+    for (int o = g.lpr; o < 32; o <<= 1)
+#pragma unroll
+        for (int t = 0; t < 8; ++t) acc[t] += __shfl_xor_sync(0xFFFFFFFFu, acc[t], o);
+}
+
+// S row slice of cluster j for lanes l < nvs (vector vbase + l), loaded ahead of use.
+__device__ __forceinline__ void load_s(const ClusterState& st, int j, const SliceGeom& g, int lane, float so[8]) {
+    if (lane < g.nvs) {
+        const float4* sp = reinterpret_cast<const float4*>(st.S + (int64_t)j * st.ld) + 2 * (g.vbase + lane);
+        const float4 s0 = sp[0], s1 = sp[1];
+        so[0] = s0.x; so[1] = s0.y; so[2] = s0.z; so[3] = s0.w;
+        so[4] = s1.x; so[5] = s1.y; so[6] = s1.z; so[7] = s1.w;
+    }
+}
+
+// EMA of one slice of cluster j from its batch sums (lanes l < nvs hold vector
+// vbase + l) and its previous sums so[]: writes S, c, the bf16 operand and the
+// closing-mean sums; slice 0 also writes N and the closing-mean count. Returns
+// the slice's part of |bf16(c_j)|^2 (the same value in every lane).
+__device__ __forceinline__ float ema_slice(const ClusterState& st, int j, double nj, int slice, const SliceGeom& g,
+                                           const double acc[8], const float so[8], int lane, double alpha,
+                                           int last_pass) {
+    const double a1 = 1.0 - alpha;
+    const float Nnew = (float)(a1 * (double)st.N_prev[j] + alpha * nj);
+    float cn_part = 0.0f;
+    if (lane < g.nvs) {
+        const int v = g.vbase + lane;
+        float sn[8], cv[8];
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+            sn[t] = (float)(a1 * (double)so[t] + alpha * acc[t]);
+            cv[t] = (float)((double)sn[t] / (double)Nnew);
+        }
+        float4* sp = reinterpret_cast<float4*>(st.S + (int64_t)j * st.ld) + 2 * v;
+        sp[0] = make_float4(sn[0], sn[1], sn[2], sn[3]);
+        sp[1] = make_float4(sn[4], sn[5], sn[6], sn[7]);
+        store_centroid_vec(st.c + (int64_t)j * st.ld, st.cq + (int64_t)j * st.ld, v, cv, cn_part);
+        if (last_pass) {
+            double* cs = st.close_sum + (int64_t)j * st.ld + 8 * v;
+#pragma unroll
+            for (int t = 0; t < 8; ++t) cs[t] += acc[t];
+        }
+    }
+    cn_part = warp_sum(cn_part);
+    if (lane == 0 && slice == 0) {
+        st.N[j] = Nnew;
+        if (last_pass) st.close_cnt[j] += nj;
+    }
     return cn_part;
 }
 
-// Full EMA of cluster j (all slices) from sums that are already complete in acc
-// (single-slice case) -- used by k_segsum for runs inside one tile.
-template <int VPL>
-__device__ __forceinline__ void ema_cluster_begin(const ClusterState& st, int j, double nj, double alpha,
-                                                  float& Nnew, double& Nnew_d) {
-    const float Nold = st.N[j];
-    Nnew_d = (1.0 - alpha) * (double)Nold + alpha * nj;
-    Nnew = (float)Nnew_d;
-}
-
-template <int VPL>
-__device__ __forceinline__ void ema_cluster_end(const ClusterState& st, int j, double nj, float Nnew, float cn_part,
-                                                int lane, int last_pass) {
-    cn_part = warp_sum(cn_part);
-    if (lane == 0) {
-        st.N[j] = Nnew;
-        if (Nnew > 0.0f) st.cn[j] = cn_part;
-        if (last_pass) st.close_cnt[j] += nj;
-    }
-}
-
-// ---------------------------------------------------------------- segmented sum
-
-template <int VPL>
-__global__ void k_segsum(const __nv_bfloat16* __restrict__ src, const int32_t* __restrict__ perm,
-                         const int32_t* __restrict__ slab, const int32_t* __restrict__ off, int rows, int R,
-                         int nv, ClusterState st, StepParams sp, double* __restrict__ pfirst,
-                         double* __restrict__ plast) {
+// One warp per (work item, slice). A work item is a chunk of at most R label-sorted
+// rows of one cluster. A cluster that fits in one chunk is updated here (its S
+// slice is fetched while the rows load); the chunks of a larger cluster leave
+// their slice sums in part[item] for k_clusters.
+__global__ void __launch_bounds__(256, 3) k_segsum(const __nv_bfloat16* __restrict__ src,
+                                                   const int32_t* __restrict__ perm, const int2* __restrict__ items,
+                                                   const int32_t* __restrict__ off, const int32_t* __restrict__ poff,
+                                                   int R, int nslices, int nv, ClusterState st, StepParams sp,
+                                                   double* __restrict__ part) {
     const int lane = threadIdx.x & 31;
-    const int tile = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    const int t0 = tile * R;
-    if (t0 >= rows) return;
-    const int t1 = min(t0 + R, rows);
-    const int slice_v = 32 * VPL;
-    int slot = t0;
-    while (slot < t1) {
-        const int j = slab[slot];
-        const int js = off[j], je = off[j + 1];
-        const int e = min(je, t1);
-        const bool complete = js >= t0 && je <= t1;
-        const double nj = (double)(je - js);
-        float Nnew = 0.0f;
-        double Nnew_d = 0.0;
-        if (complete) ema_cluster_begin<VPL>(st, j, nj, sp.alpha, Nnew, Nnew_d);
-        float cn_part = 0.0f;
-        for (int vb = 0; vb < nv; vb += slice_v) {
-            SliceAcc<VPL> acc;
-            acc.zero();
-            acc_rows<VPL>(acc, src, st.ld, perm, slot, e, vb, nv, lane);
-            if (complete) {
-                cn_part += ema_slice<VPL>(st, j, nj, Nnew_d, Nnew, acc, vb, nv, lane, sp.alpha, sp.last_pass);
-            } else {
-                double* dst = (js < t0 ? pfirst : plast) + (int64_t)tile * (nv * 8);
+    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int item = warp / nslices, slice = warp - item * nslices;
+    if (item >= poff[st.k]) return;
+    const int2 it = items[item];
+    const int j = it.x, s0 = it.y;
+    const int js = off[j], je = off[j + 1];
+    const int s1 = min(s0 + R, je);
+    const SliceGeom g = slice_geom(slice, nv);
+    const bool single = je - js <= R;
+    float so[8];
+    if (single) load_s(st, j, g, lane, so);
+    double acc[8];
+    sum_rows(acc, src, st.ld, perm, s0, s1, g, lane);
+    if (single) {
+        const float cn_part = ema_slice(st, j, (double)(je - js), slice, g, acc, so, lane, sp.alpha, sp.last_pass);
+        if (lane == 0) st.cnp[(int64_t)slice * st.k + j] = cn_part;
+    } else if (lane < g.nvs) {
+        double* dst = part + (int64_t)item * st.ld + 8 * (g.vbase + lane);
 #pragma unroll
-                for (int i = 0; i < VPL; ++i) {
-                    const int v = vb + i * 32 + lane;
-                    if (v < nv) {
-#pragma unroll
-                        for (int t = 0; t < 8; ++t) dst[8 * v + t] = acc.a[i][t];
-                    }
-                }
-            }
-        }
-        if (complete) ema_cluster_end<VPL>(st, j, nj, Nnew, cn_part, lane, sp.last_pass);
-        slot = e;
+        for (int t = 0; t < 8; ++t) dst[t] = acc[t];
     }
 }
 
-// Clusters cut by tile edges (owned by the tile where their run starts) and
-// clusters that received no row. Also clears the counts for the next step.
-template <int VPL>
-__global__ void k_fixup(const int32_t* __restrict__ slab, const int32_t* __restrict__ off, int32_t* __restrict__ cnt,
-                        int rows, int R, int ntiles, int k, int nv, ClusterState st, StepParams sp,
-                        const double* __restrict__ pfirst, const double* __restrict__ plast) {
+// One warp per cluster, after k_segsum: a cluster without rows decays (S and N by
+// 1 - alpha; its centroid S/N is unchanged); a cluster of one chunk gets
+// |bf16(c)|^2 as the sum of its slice parts in slice order; a cluster of several
+// chunks adds their partial sums in chunk order (four in flight) and is updated
+// here. Clears the counts for the next step.
+__global__ void k_clusters(const int32_t* __restrict__ off, const int32_t* __restrict__ poff,
+                           int32_t* __restrict__ cnt, int R, int nslices, int nv, ClusterState st, StepParams sp,
+                           const double* __restrict__ part) {
     const int lane = threadIdx.x & 31;
     const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int nwarps = (gridDim.x * blockDim.x) >> 5;
-    const int slice_v = 32 * VPL;
-    for (int tile = warp; tile < ntiles; tile += nwarps) {
-        const int t0 = tile * R, t1 = min(t0 + R, rows);
-        if (t1 <= t0) continue;
-        const int j = slab[t1 - 1];
-        const int js = off[j], je = off[j + 1];
-        if (!(js >= t0 && je > t1)) continue;
-        const int last_tile = (je - 1) / R;
-        const double nj = (double)(je - js);
-        float Nnew;
-        double Nnew_d;
-        ema_cluster_begin<VPL>(st, j, nj, sp.alpha, Nnew, Nnew_d);
-        float cn_part = 0.0f;
-        for (int vb = 0; vb < nv; vb += slice_v) {
-            SliceAcc<VPL> acc;
-#pragma unroll
-            for (int i = 0; i < VPL; ++i) {
-                const int v = vb + i * 32 + lane;
-#pragma unroll
-                for (int t = 0; t < 8; ++t) acc.a[i][t] = v < nv ? plast[(int64_t)tile * (nv * 8) + 8 * v + t] : 0.0;
-            }
-            for (int u = tile + 1; u <= last_tile; ++u) {
-#pragma unroll
-                for (int i = 0; i < VPL; ++i) {
-                    const int v = vb + i * 32 + lane;
-                    if (v < nv) {
-#pragma unroll
-                        for (int t = 0; t < 8; ++t) acc.a[i][t] += pfirst[(int64_t)u * (nv * 8) + 8 * v + t];
-                    }
-                }
-            }
-            cn_part += ema_slice<VPL>(st, j, nj, Nnew_d, Nnew, acc, vb, nv, lane, sp.alpha, sp.last_pass);
-        }
-        ema_cluster_end<VPL>(st, j, nj, Nnew, cn_part, lane, sp.last_pass);
-    }
-    // clusters without rows: N and S decay, the centroid S/N is unchanged
-    const float a1 = (float)(1.0 - sp.alpha);
-    for (int j = warp; j < k; j += nwarps) {
-        const bool empty = off[j + 1] == off[j];
+    const double a1 = 1.0 - sp.alpha;
+    for (int j = warp; j < st.k; j += nwarps) {
+        const int nj = off[j + 1] - off[j];
         if (lane == 0) cnt[j] = 0;
-        if (!empty) continue;
-        float* Srow = st.S + (int64_t)j * st.ld;
-        for (int e = lane; e < nv * 8; e += 32) Srow[e] = (float)((double)a1 * 0.0 + (1.0 - sp.alpha) * (double)Srow[e]);
-        if (lane == 0) st.N[j] = (float)((1.0 - sp.alpha) * (double)st.N[j]);
+        if (nj == 0) {
+            float4* row = reinterpret_cast<float4*>(st.S + (int64_t)j * st.ld);
+            for (int v = lane; v < st.ld / 4; v += 32) {
+                const float4 x = row[v];
+                row[v] = make_float4((float)(a1 * (double)x.x), (float)(a1 * (double)x.y), (float)(a1 * (double)x.z),
+                                     (float)(a1 * (double)x.w));
+            }
+            if (lane == 0) st.N[j] = (float)(a1 * (double)st.N_prev[j]);
+        } else if (nj <= R) {
+            if (lane == 0) {
+                float c = 0.0f;
+                for (int s = 0; s < nslices; ++s) c += st.cnp[(int64_t)s * st.k + j];
+                st.cn[j] = c;
+            }
+        } else {
+            const int p0 = poff[j], p1 = poff[j + 1];
+            float cn_total = 0.0f;
+            for (int slice = 0; slice < nslices; ++slice) {
+                const SliceGeom g = slice_geom(slice, nv);
+                float so[8];
+                load_s(st, j, g, lane, so);
+                double acc[8];
+#pragma unroll
+                for (int t = 0; t < 8; ++t) acc[t] = 0.0;
+                if (lane < g.nvs) {
+                    const double* base = part + 8 * (g.vbase + lane);
+                    int p = p0;
+                    for (; p + 3 < p1; p += 4) {
+                        double x[4][8];
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+#pragma unroll
+                            for (int t = 0; t < 8; ++t) x[q][t] = base[(int64_t)(p + q) * st.ld + t];
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+#pragma unroll
+                            for (int t = 0; t < 8; ++t) acc[t] += x[q][t];
+                    }
+                    for (; p < p1; ++p)
+#pragma unroll
+                        for (int t = 0; t < 8; ++t) acc[t] += base[(int64_t)p * st.ld + t];
+                }
+                cn_total += ema_slice(st, j, (double)nj, slice, g, acc, so, lane, sp.alpha, sp.last_pass);
+            }
+            if (lane == 0) st.cn[j] = cn_total;
+        }
     }
 }
 
 // ---------------------------------------------------------------- full assignment pass
 
 // Labels and distances of a full pass (em_assign / em_mse / Lloyd): int64 labels,
-// fp32 squared distances max(0, |x|^2 + score), per-block fp64 sums.
-__global__ void k_assign_out(const unsigned long long* __restrict__ keys, const float* __restrict__ xn, int64_t rows,
-                             int k, int64_t* __restrict__ labels, float* __restrict__ dists,
-                             int32_t* __restrict__ labels32, double* __restrict__ block_err, int* err) {
+// fp32 squared distances max(0, |x|^2 + score), per-block fp64 sums; near ties are
+// settled exactly as in k_labels.
+__global__ void k_assign_out(const unsigned long long* __restrict__ keys, int nsplit, const float* __restrict__ xn,
+                             int64_t rows, int k, const __nv_bfloat16* __restrict__ A, int ld,
+                             const __nv_bfloat16* __restrict__ cq, int64_t* __restrict__ labels,
+                             float* __restrict__ dists, int32_t* __restrict__ labels32, double* __restrict__ block_err,
+                             int* err) {
     __shared__ double warp_err[32];
+    const int lane = threadIdx.x & 31;
     double e = 0.0;
-    for (int64_t r = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; r < rows; r += (int64_t)gridDim.x * blockDim.x) {
-        const unsigned long long key = keys[r];
-        uint32_t l = key_label(key);
-        if (l >= (uint32_t)k) {
-            raise_error(err, EM_E_BOUNDS);
-            l = 0;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t base = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31); base < rows; base += stride) {
+        const int64_t r = base + lane;
+        const bool active = r < rows;
+        uint32_t l1 = 0, l2 = 0;
+        float s1 = 0.0f, s2 = 0.0f, x2 = 0.0f;
+        bool tie = false;
+        if (active) {
+            unsigned long long k1, k2;
+            merge_keys(keys, rows, nsplit, r, k1, k2);
+            l1 = key_label(k1);
+            s1 = key_score(k1);
+            x2 = xn[r];
+            if (l1 >= (uint32_t)k) {
+                raise_error(err, EM_E_BOUNDS);
+                l1 = 0;
+            }
+            if (k2 != kEmptyKey) {
+                l2 = key_label(k2);
+                s2 = key_score(k2);
+                tie = l2 < (uint32_t)k && s2 - s1 <= kTieRel * (x2 + fabsf(s1) + fabsf(s2));
+            }
         }
-        const float dist = fmaxf(0.0f, xn[r] + key_score(key));
-        if (labels) labels[r] = (int64_t)l;
-        if (labels32) labels32[r] = (int32_t)l;
-        if (dists) dists[r] = dist;
-        e += (double)dist;
+        settle_ties(tie, r, l1, s1, l2, s2, A, ld, cq, lane);
+        if (active) {
+            const float dist = fmaxf(0.0f, x2 + s1);
+            if (labels) labels[r] = (int64_t)l1;
+            if (labels32) labels32[r] = (int32_t)l1;
+            if (dists) dists[r] = dist;
+            e += (double)dist;
+        }
     }
     e = warp_sum(e);
     if ((threadIdx.x & 31) == 0) warp_err[threadIdx.x >> 5] = e;

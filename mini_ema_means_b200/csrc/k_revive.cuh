@@ -15,11 +15,12 @@
 //   * resample (the EnCodec-style arm of the ablation): c_j <- a row of the
 //     current batch drawn with Philox(seed, stream 4, t, j), N_j = S_j = 0.
 //
-// The draws are inherently sequential, so one warp makes them on an fp64 tree in
-// shared memory (32 children per node: one load and one ballot per prefix level,
-// one warp scan of the 32 current leaf weights, and a halving updates one suffix
-// of each level with one lane-parallel subtraction); the uniform draws are made
-// in parallel beforehand. The vector work is then done in parallel from the closed form:
+// The draws are inherently sequential, so one warp makes them on an fp64 tree of
+// prefix sums in shared memory (32 children per node: one load and one ballot per
+// level; a halving updates one suffix of each level with one lane-parallel
+// subtraction); the uniform draws are made in parallel beforehand. The donor's
+// current weight is read back as the difference of two prefix values. The vector
+// work is then done in parallel from the closed form:
 // the o-th split taken from donor d (0-based) sees c_d (1 + eps s)^o and N_d / 2^o.
 #pragma once
 
@@ -38,40 +39,47 @@ struct ReviveScratch {
     int64_t* n_splits;  // 1: cumulative number of revived clusters
 };
 
-// Donor tree: level 0 holds the current weight of every cluster (N_j, or 0 for a
-// dead one); level l >= 1 holds, for each group of 32 entries of level l-1, the
-// inclusive prefix of the group totals within its own group of 32.
+// Donor tree, 32 children per node, every level stored as inclusive prefix sums
+// within its groups of 32: level 0 over the current weights of the clusters (N_j,
+// or 0 for a dead one), level l >= 1 over the totals of the groups of level l-1.
+// A search costs one shared-memory load and one ballot per level.
 struct TreeLayout {
     int levels;
-    int size[8];
-    int64_t offset[8];
+    int size[6];
+    int64_t offset[6];
     int64_t total;   // doubles
 };
 
 // Shared memory the selection kernel may use (bytes).
 constexpr int kReviveSmemBytes = 200 * 1024;
 
+constexpr int kMaxLevels = 6;  // 32^6 > 2^30 clusters
+
 EM_HD TreeLayout tree_layout(int k) {
     TreeLayout L{};
     int s = k;
     int64_t off = 0;
     L.levels = 0;
-    while (true) {
-        L.size[L.levels] = s;
-        L.offset[L.levels] = off;
-        off += ((s + 31) / 32) * 32;
-        ++L.levels;
-        if (s <= 32 || L.levels == 8) break;
-        s = (s + 31) / 32;
+    bool done = false;
+#pragma unroll
+    for (int l = 0; l < kMaxLevels; ++l) {
+        if (!done) {
+            L.size[l] = s;
+            L.offset[l] = off;
+            off += ((s + 31) / 32) * 32;
+            L.levels = l + 1;
+            done = s <= 32;
+            s = (s + 31) / 32;
+        }
     }
     L.total = off;
     return L;
 }
 
-// 0: leaves, split counts and upper levels in shared memory; 1: leaves and split
+// 0: every level and the split counts in shared memory; 1: level 0 and the split
 // counts in global memory, upper levels shared; 2: everything in global memory.
 EM_HD int tree_placement(const TreeLayout& L, int k) {
-    const int64_t upper = (L.total - L.offset[L.levels > 1 ? 1 : 0]) * 8;
+    const int64_t upper = (L.levels > 1 ? L.total - L.offset[1] : 0) * 8;
     if (L.total * 8 + (int64_t)k * 4 <= kReviveSmemBytes) return 0;
     if (L.levels > 1 && upper <= kReviveSmemBytes) return 1;
     return 2;
@@ -156,9 +164,11 @@ __global__ void __launch_bounds__(1024) k_revive_select(const float* __restrict_
     extern __shared__ double smem_d[];
     const TreeLayout L = tree_layout(k);
     const int placement = tree_placement(L, k);
-    double* levp[8];
-    int32_t* times;
-    for (int l = 0; l < L.levels; ++l) {
+    // (all loops over levels below have a fixed trip count so that levp[] and
+    // L.size[] are indexed by constants and stay in registers)
+    double* levp[kMaxLevels];
+#pragma unroll
+    for (int l = 0; l < kMaxLevels; ++l) {
         if (placement == 0)
             levp[l] = smem_d + L.offset[l];
         else if (placement == 1 && l > 0)
@@ -166,32 +176,26 @@ __global__ void __launch_bounds__(1024) k_revive_select(const float* __restrict_
         else
             levp[l] = sc.tree + L.offset[l];
     }
-    times = placement == 0 ? reinterpret_cast<int32_t*>(smem_d + L.total) : sc.times;
-    for (int j = tid; j < k; j += 1024) {
-        const float nj = N[j];
-        levp[0][j] = ((double)nj < thr) ? 0.0 : (double)nj;
-        times[j] = 0;
-    }
-    __syncthreads();
-    for (int l = 1; l < L.levels; ++l) {
-        const int sz = L.size[l];
-        const int ngroups = (sz + 31) / 32;
-        for (int gidx = w; gidx < ngroups; gidx += 32) {
-            const int i = gidx * 32 + lane;  // entry of level l = group i of level l-1
-            double v = 0.0;
-            if (i < sz) {
-                if (l == 1) {  // total of 32 leaves
-                    double acc = 0.0;
-                    for (int q = 0; q < 32; ++q) {
-                        const int leaf = i * 32 + q;
-                        if (leaf < L.size[0]) acc += levp[0][leaf];
+    int32_t* times = placement == 0 ? reinterpret_cast<int32_t*>(smem_d + L.total) : sc.times;
+    for (int j = tid; j < k; j += 1024) times[j] = 0;
+#pragma unroll
+    for (int l = 0; l < kMaxLevels; ++l) {
+        if (l < L.levels) {
+            const int sz = L.size[l];
+            const int ngroups = (sz + 31) / 32;
+            for (int gidx = w; gidx < ngroups; gidx += 32) {
+                const int i = gidx * 32 + lane;
+                double v = 0.0;
+                if (i < sz) {
+                    if (l == 0) {
+                        const float nj = N[i];
+                        v = ((double)nj < thr) ? 0.0 : (double)nj;
+                    } else {
+                        v = levp[l > 0 ? l - 1 : 0][i * 32 + 31];  // prefix at the end of child group i
                     }
-                    v = acc;
-                } else {
-                    v = levp[l - 1][i * 32 + 31];  // inclusive prefix at the end of child group i
                 }
+                levp[l][gidx * 32 + lane] = warp_incl_scan(v, lane);
             }
-            levp[l][gidx * 32 + lane] = warp_incl_scan(v, lane);
         }
         __syncthreads();
     }
@@ -199,13 +203,10 @@ __global__ void __launch_bounds__(1024) k_revive_select(const float* __restrict_
     // sequential draws by warp 0
     if (w == 0) {
         const int top = L.levels - 1;
-        double W;
-        if (L.levels == 1) {
-            const double v = lane < L.size[0] ? levp[0][lane] : 0.0;
-            W = __shfl_sync(0xFFFFFFFFu, warp_incl_scan(v, lane), 31);
-        } else {
-            W = levp[top][31];
-        }
+        double W = 0.0;
+#pragma unroll
+        for (int l = 0; l < kMaxLevels; ++l)
+            if (l == top) W = levp[l][31];
         bool exhausted = false;
         for (int i0 = 0; i0 < nd; i0 += 32) {
             const int cnt = min(32, nd - i0);
@@ -219,50 +220,45 @@ __global__ void __launch_bounds__(1024) k_revive_select(const float* __restrict_
                 }
                 double target = __shfl_sync(0xFFFFFFFFu, my_u, q) * W;
                 int node = 0;
-                for (int l = top; l >= 1; --l) {  // prefix levels: one load and one ballot each
-                    const int base = node * 32;
-                    const bool valid = base + lane < L.size[l];
-                    const double P = valid ? levp[l][base + lane] : 0.0;
-                    const double Pprev = __shfl_up_sync(0xFFFFFFFFu, P, 1);
-                    const double prev_incl = lane == 0 ? 0.0 : Pprev;
-                    const unsigned above = __ballot_sync(0xFFFFFFFFu, valid && P > target);
-                    int c;
-                    if (above) {
-                        c = __ffs(above) - 1;
-                    } else {  // target rounded onto the total: the last child with weight
-                        const unsigned pos = __ballot_sync(0xFFFFFFFFu, valid && P > prev_incl);
-                        c = pos ? 31 - __clz(pos) : 0;
+                double wsel = 0.0;  // current weight of the chosen child at the last level
+#pragma unroll
+                for (int l = kMaxLevels - 1; l >= 0; --l) {
+                    if (l <= top) {
+                        const int base = node * 32;
+                        const double* lev = levp[l];
+                        const bool valid = base + lane < L.size[l];
+                        const double P = valid ? lev[base + lane] : 0.0;
+                        const unsigned above = __ballot_sync(0xFFFFFFFFu, valid && P > target);
+                        int c;
+                        if (above) {
+                            c = __ffs(above) - 1;
+                        } else {  // target rounded onto the total: the last child with weight
+                            const double Pp = __shfl_up_sync(0xFFFFFFFFu, P, 1);
+                            const unsigned pos = __ballot_sync(0xFFFFFFFFu, valid && P > (lane ? Pp : 0.0));
+                            c = pos ? 31 - __clz(pos) : 0;
+                        }
+                        const double before = c > 0 ? lev[base + c - 1] : 0.0;  // broadcast load
+                        if (l == 0) wsel = lev[base + c] - before;
+                        target -= before;
+                        node = base + c;
                     }
-                    target -= __shfl_sync(0xFFFFFFFFu, prev_incl, c);
-                    node = base + c;
                 }
-                // leaves: current weights, scanned by the warp
-                const int base = node * 32;
-                const bool valid = base + lane < L.size[0];
-                const double wv = valid ? levp[0][base + lane] : 0.0;
-                const double P = warp_incl_scan(wv, lane);
-                const unsigned above = __ballot_sync(0xFFFFFFFFu, valid && P > target);
-                int c;
-                if (above) {
-                    c = __ffs(above) - 1;
-                } else {
-                    const unsigned pos = __ballot_sync(0xFFFFFFFFu, valid && wv > 0.0);
-                    c = pos ? 31 - __clz(pos) : 0;
-                }
-                const int dn = base + c;
-                const double delta = 0.5 * __shfl_sync(0xFFFFFFFFu, wv, c);  // half its current weight
-                if (lane == c) levp[0][dn] = wv - delta;
+                const int dn = node;
+                const double delta = 0.5 * wsel;  // half of the donor's current weight
                 if (lane == 0) {
                     const int old = times[dn];
                     times[dn] = old + 1;
                     sc.donor[i] = dn;
                     sc.order[i] = old;
                 }
-                int idx = dn >> 5;
-                for (int l = 1; l < L.levels; ++l) {
-                    const int gb = (idx >> 5) << 5;
-                    if (gb + lane >= idx && gb + lane < L.size[l]) levp[l][gb + lane] -= delta;
-                    idx >>= 5;
+                int idx = dn;
+#pragma unroll
+                for (int l = 0; l < kMaxLevels; ++l) {
+                    if (l < L.levels) {
+                        const int gb = (idx >> 5) << 5;
+                        if (gb + lane >= idx && gb + lane < L.size[l]) levp[l][gb + lane] -= delta;
+                        idx >>= 5;
+                    }
                 }
                 W -= delta;
                 __syncwarp();

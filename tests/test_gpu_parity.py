@@ -207,3 +207,52 @@ def test_state_roundtrip_and_errors(em):
     with pytest.raises(em.EmeansError) as e:
         m.train(bad.cuda(), epochs=1.0)
     assert e.value.code == em.EM_E_NONFINITE
+
+
+def test_step_graphs_match_direct_launches(em):
+    """A run replayed from captured step graphs equals the same run launched kernel by
+    kernel, bit for bit, and a second run (graph cache hit) equals the first."""
+    x = synth.hand_shape(6000, 64, 30, seed=12)
+    outs = []
+    for graphs in (0, 1, 1):
+        m = em.Model(64, 50, seed=21, graphs=graphs)
+        m.train(x.cuda(), epochs=3.0)
+        c = torch.empty(50, 64)
+        m.centroids(c)
+        lab = torch.empty(6000, dtype=torch.int64)
+        m.labels(lab)
+        outs.append((c, lab, m.obj(), m.stats()["n_splits"]))
+        if graphs:
+            m.train(x.cuda(), epochs=3.0)  # same run again: replayed from the cache
+            c2 = torch.empty(50, 64)
+            m.centroids(c2)
+            assert torch.equal(c, c2)
+    for c, lab, obj, splits in outs[1:]:
+        assert torch.equal(c, outs[0][0]) and torch.equal(lab, outs[0][1])
+        assert np.array_equal(obj, outs[0][2]) and splits == outs[0][3]
+
+
+@pytest.mark.parametrize("d", [64, 96, 768])
+def test_exact_ties_reproduce_the_fp64_argmin(em, d):
+    """Centroids come in pairs one bf16 step apart, so most rows are near ties of
+    their pair; with exact tie settling the labels equal the fp64 oracle's, and
+    exact duplicates go to the lower index."""
+    n, pairs = 4000, 40
+    g = torch.Generator().manual_seed(d)
+    x = synth.hand_shape(n, d, 10, seed=d)
+    base = x[torch.randint(0, n, (pairs,), generator=g)] + 0.5 * torch.randn(pairs, d, generator=g)
+    base = base.to(torch.bfloat16).float()
+    twin = base.clone()
+    idx = torch.randint(0, d, (pairs,), generator=g)
+    for i in range(pairs):  # move one coordinate of the twin by one bf16 step
+        v = twin[i, idx[i]].to(torch.bfloat16)
+        twin[i, idx[i]] = (v.view(torch.int16) + 1).view(torch.bfloat16).float()
+    c = torch.stack([base, twin], 1).reshape(2 * pairs, d)
+    c[-1] = c[0]  # an exact duplicate: ties go to the lower index
+    m = em.Model(d, 2 * pairs, seed=1, exact_ties=1)
+    m.set_state(c=c)
+    labels = torch.empty(n, dtype=torch.int64, device="cuda")
+    m.assign(x.cuda(), labels=labels)
+    xq = O.search_copy_of_data(x.numpy())
+    ref, _, _ = O.assign(xq, O.search_copy_of_centroids(c.numpy().astype(np.float64)))
+    assert np.array_equal(labels.cpu().numpy(), ref)
