@@ -261,6 +261,9 @@ def run_ours(args, rank, world):
         "peak": peaks["hbm_gbs"], "unit": "GB/s",
         "frac": (prof["update_bytes"] / (u_ms / 1e3) / 1e9) / peaks["hbm_gbs"] if u_ms > 0 else 0.0,
     }
+    # the profiled pass assigns the same rows as the timed one
+    out["assign_only_pts_per_s"] = (rows / (a_ms / 1e3)) if a_ms > 0 else None
+    out["epochs_per_s"] = value / w.n_train
     out["gpu_launches"] = launches
     out["clocks"] = clocks
 
@@ -293,7 +296,7 @@ def lloyd25(m, w, xt, xs, rec):
     # pass replays step graphs instead of capturing them
     for timed in (False, True):
         m.begin(xt, epochs=w.epochs)
-        train_ms, steps, hit = 0.0, 0, None
+        train_ms, steps, hit, eval_s = 0.0, 0, None, 0.0
         history = []
         if timed:
             break
@@ -311,7 +314,9 @@ def lloyd25(m, w, xt, xs, rec):
         torch.cuda.synchronize()
         train_ms += e0.elapsed_time(e1)
         steps = nxt
+        t_eval = time.perf_counter()
         mse = m.mse(xs)
+        eval_s += time.perf_counter() - t_eval
         epochs = steps / full
         history.append((round(epochs, 4), mse))
         if hit is None and mse <= target:
@@ -326,7 +331,7 @@ def lloyd25(m, w, xt, xs, rec):
     if hit is None and final <= target:
         hit = {"seconds": train_ms / 1e3, "epochs": w.epochs, "test_mse": final}
     return {"lloyd25_test_mse": target, "lloyd25_wall_s": lloyd_s, "emeans_final_test_mse": final,
-            "emeans_train_s": train_ms / 1e3, "reached": hit is not None,
+            "emeans_train_s": train_ms / 1e3, "evaluation_s_excluded": eval_s, "reached": hit is not None,
             "time_to_target_s": hit["seconds"] if hit else None, "epochs_to_target": hit["epochs"] if hit else None,
             "final_ratio": final / target, "checkpoints": history}
 
@@ -445,11 +450,42 @@ def run_kernel_case(args):
         rows = args.case_rows if args.case_rows_step else None
         w, xt, _ = datagen.make(args.workload, device="cuda", seed=0, n_train=rows, n_test=1 if rows else None)
         m = em.Model(w.d, w.k, seed=1234)
+        if args.case_batch:
+            m.set_option("batch_size", args.case_batch)
         m.begin(xt, epochs=w.epochs)
         m.step(args.steps)
         m.sync()
     m.close()
     print(json.dumps({"kernel_case": args.kernel_case, "workload": args.workload, "ok": True}))
+
+
+def run_ablation(args):
+    """Revival ablation on one workload: split, resample and none over several
+    seeds. Dead clusters are those that receive no training row in a full
+    assignment pass with the final centroids; test MSE with the same centroids."""
+    import torch
+
+    import datagen
+    import mini_ema_means_b200 as em
+
+    torch.cuda.set_device(0)
+    w, xt, xs = datagen.make(args.workload, device="cuda", seed=0)
+    labels = torch.empty(w.n_train, dtype=torch.int64, device="cuda")
+    out = {"ablation": args.workload, "seeds": args.ablation_seeds, "modes": {}}
+    for mode in ("split", "resample", "none"):
+        rows = []
+        for seed in range(args.ablation_seeds):
+            m = em.Model(w.d, w.k, seed=seed, revival=mode)
+            m.set_option("input_dtype", 1 if w.storage == "bf16" else 0)
+            m.train(xt, epochs=w.epochs)
+            m.assign(xt, labels=labels)
+            dead = int((torch.bincount(labels, minlength=w.k) == 0).sum().item())
+            rows.append({"seed": seed, "dead": dead, "test_mse": m.mse(xs), "splits": m.stats()["n_splits"]})
+            m.close()
+            log(f"[ablation] {mode} seed {seed}: {rows[-1]}")
+        out["modes"][mode] = {"runs": rows, "dead_mean": statistics.mean(r["dead"] for r in rows),
+                              "test_mse_mean": statistics.mean(r["test_mse"] for r in rows)}
+    return out
 
 
 def main():
@@ -469,7 +505,13 @@ def main():
     ap.add_argument("--kernel-case", choices=["assign", "step"], default=None)
     ap.add_argument("--case-rows", type=int, default=262144)
     ap.add_argument("--case-rows-step", action="store_true", help="train the step case on --case-rows rows")
+    ap.add_argument("--case-batch", type=int, default=0, help="batch size of the step case (0: the recipe's)")
+    ap.add_argument("--ablation", action="store_true", help="revival ablation (split / resample / none)")
+    ap.add_argument("--ablation-seeds", type=int, default=5)
     args = ap.parse_args()
+    if args.ablation:
+        print(json.dumps(run_ablation(args)), flush=True)
+        return
     if args.kernel_case:
         run_kernel_case(args)
         return

@@ -357,10 +357,6 @@ static ClusterState cluster_state(em_model* m) {
     return st;
 }
 
-// Rows per work item of the grouped update (a cluster's sorted rows are cut into
-// chunks of at most this many rows).
-constexpr int kChunkRows = 64;
-
 static int ensure_batch_buffers(em_model* m, int64_t cap) {
     m->R = kChunkRows;
     const int64_t max_items = m->k + (cap + m->R - 1) / m->R;
@@ -494,7 +490,7 @@ static int launch_revive(em_model* m, int64_t t, int64_t rows) {
     const ReviveScratch sc = revive_scratch(m);
     const TreeLayout L = tree_layout((int)m->k);
     const int smem = (int)tree_smem_bytes(L, (int)m->k);
-    k_revive_select<<<1, 1024, smem, m->stream>>>(m->N.p, (int)m->k, m->tau, m->seed, t, m->revival, sc, m->err.p);
+    k_revive_select<<<1, kSelectThreads, smem, m->stream>>>(m->N.p, (int)m->k, m->tau, m->seed, t, m->revival, sc, m->err.p);
     CK(cudaGetLastError());
     const ClusterState st = cluster_state(m);
     const int blocks = grid_for(m->k * 32, 256, m->sms);

@@ -6,14 +6,16 @@
 // "Kernels": the distance computation is fused with the selection of the nearest
 // centroid, so no n x k distance matrix is ever written).
 //
-// Structure of one CTA (192 threads, one CTA per SM, persistent over work units):
+// Structure of one CTA (320 threads, one CTA per SM, persistent over work units):
 //   warp 0      TMA producer: 128 x KC tiles of A and 256 x KC tiles of the
 //               centroid operand into a STAGES-deep shared-memory ring
 //   warp 1      allocates 512 TMEM columns; one thread issues tcgen05.mma
 //               (M=128, N=256, K=16, bf16 x bf16 -> fp32) into one of two
 //               TMEM accumulators and commits to mbarriers
-//   warps 2..5  epilogue: tcgen05.ld of the 128 x 256 fp32 tile (thread = row),
-//               add |c|^2, running argmin; frees the accumulator for the next tile
+//   warps 2..9  epilogue: thread = accumulator row; warps w and w + 4 share the
+//               TMEM lane quadrant w % 4 and take the left and right 128 columns
+//               of the tile: tcgen05.ld, free the accumulator, add |c|^2, running
+//               argmin; the two halves of a row are merged once per work unit
 // A work unit is (128-row tile, group of 256-wide centroid tiles). When k is
 // split over several units, every group writes its own per-row result
 // ((order-preserving score, index) keys) and the label kernel merges them. With
@@ -28,8 +30,8 @@ namespace tc {
 
 constexpr int BM = 128;
 constexpr int BN = 256;
-constexpr int kThreads = 192;
-constexpr int kEpiThreads = 128;
+constexpr int kThreads = 320;
+constexpr int kEpiThreads = 256;
 
 template <int KC>
 struct Cfg {
@@ -40,7 +42,8 @@ struct Cfg {
     static constexpr uint64_t kLayout = KC == 64 ? 2ull : 4ull;  // UMMA 128B / 64B swizzle
     static constexpr uint32_t kSBO = 8u * KC * 2u;                // bytes between 8-row groups
     static constexpr int kBarBytes = 256;
-    static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kBarBytes + 2 * BN * 4;
+    // + |c|^2 of two tiles, + the right halves' keys of one row tile
+    static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kBarBytes + 2 * BN * 4 + BM * 2 * 8;
 };
 
 // Instruction descriptor of tcgen05.mma kind::f16: fp32 accumulate (bits 4-5 = 1),
@@ -109,19 +112,22 @@ __device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity, long l
     }
 }
 
-// AND of `ok` over the 128 epilogue threads; doubles as their named barrier 1.
+// AND of `ok` over the 256 epilogue threads; doubles as their named barrier 1.
 __device__ __forceinline__ bool epi_all(bool ok) {
     uint32_t r;
     asm volatile(
         "{\n\t.reg .pred p, q;\n\t"
         "setp.ne.u32 p, %1, 0;\n\t"
-        "bar.red.and.pred q, 1, 128, p;\n\t"
+        "bar.red.and.pred q, 1, 256, p;\n\t"
         "selp.u32 %0, 1, 0, q;\n\t}\n"
         : "=r"(r)
         : "r"((uint32_t)ok)
         : "memory");
     return r != 0;
 }
+
+// Named barrier 2 over the 256 epilogue threads.
+__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 2, 256;" ::: "memory"); }
 
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* tm, int x, int y, uint32_t bar) {
     asm volatile(
@@ -194,6 +200,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 5);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     float* cn_s = reinterpret_cast<float*>(smem + S * C::kStageBytes + C::kBarBytes);
+    unsigned long long* half_keys = reinterpret_cast<unsigned long long*>(cn_s + 2 * BN);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -317,14 +324,23 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
     } else {
-        // ---------------- epilogue: 4 warps, thread = accumulator row
+        // ---------------- epilogue: 8 warps, thread = accumulator row, warp = column half
         const int et = threadIdx.x - 64;
         const int q = warp & 3;
+        const int half = (warp - 2) >> 2;
+        const int rl = 32 * q + lane;  // row within the tile
         const uint32_t lane_base = (uint32_t)(32 * q) << 16;
         int acc = 0;
         uint32_t acc_phase = 0;
         int cnbuf = 0;
         bool ok = true;
+        // |c|^2 of the next tile this CTA handles, loaded one tile ahead
+        auto cn_of = [&](int j) { return j < k ? cn[j] : __int_as_float(0x7f800000); };
+        float cn_next = 0.0f;
+        if (blockIdx.x < units) {
+            const int g0 = blockIdx.x % n_split;
+            cn_next = cn_of(g0 * tpg * BN + et);
+        }
         for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
             const int m = u / n_split, g = u - m * n_split;
             const int nt0 = g * tpg, nt1 = min(nt0 + tpg, n_tiles);
@@ -334,10 +350,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int nt = nt0; nt < nt1; ++nt) {
                 float* cnb = cn_s + cnbuf * BN;
                 const int j0 = nt * BN;
-                cnb[et] = (j0 + et < k) ? cn[j0 + et] : __int_as_float(0x7f800000);
-                cnb[et + 128] = (j0 + et + 128 < k) ? cn[j0 + et + 128] : __int_as_float(0x7f800000);
+                cnb[et] = cn_next;
+                {
+                    int jn = -1;
+                    if (nt + 1 < nt1) {
+                        jn = (nt + 1) * BN;
+                    } else if (u + (int)gridDim.x < units) {
+                        const int gn = (u + (int)gridDim.x) % n_split;
+                        jn = gn * tpg * BN;
+                    }
+                    if (jn >= 0) cn_next = cn_of(jn + et);
+                }
                 const bool got = mbar_wait(smem_u32(&tfull[acc]), acc_phase, wait_limit, err, abort_flag);
-                // one decision for all 128 threads (so none is left at a barrier), and the
+                // one decision for all 256 threads (so none is left at a barrier), and the
                 // barrier that publishes this tile's |c|^2 values
                 if (!epi_all(got)) {
                     ok = false;
@@ -345,52 +370,84 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 tc_fence_after();
                 __syncwarp();
-                const uint32_t tbase = tmem_base + lane_base + (uint32_t)(acc * BN);
+                const uint32_t tbase = tmem_base + lane_base + (uint32_t)(acc * BN + half * 128);
+                const float4* c4 = reinterpret_cast<const float4*>(cnb + half * 128);
+                // two rounds of 64 columns (the register file allows no more per thread
+                // with ten warps: three of them share a sub-partition)
 #pragma unroll 1
-                for (int ch = 0; ch < BN / 32; ch += 2) {
+                for (int r = 0; r < 2; ++r) {
                     uint32_t v[2][32];
-                    tmem_ld32(tbase + ch * 32, v[0]);
-                    tmem_ld32(tbase + ch * 32 + 32, v[1]);
+                    tmem_ld32(tbase + r * 64, v[0]);
+                    tmem_ld32(tbase + r * 64 + 32, v[1]);
                     tmem_wait_ld();
-                    const float4* c4 = reinterpret_cast<const float4*>(cnb + ch * 32);
+                    if (r == 1) {  // the values are in registers: hand the accumulator back
+                        tc_fence_before();
+                        mbar_arrive(smem_u32(&tempty[acc]));
+                    }
 #pragma unroll
-                    for (int h = 0; h < 2; ++h) {
+                    for (int c = 0; c < 2; ++c) {
+                        float sc[32];
 #pragma unroll
                         for (int i = 0; i < 8; ++i) {
-                            const float4 cc = c4[8 * h + i];
-                            const float sc[4] = {cc.x + __uint_as_float(v[h][4 * i + 0]),
-                                                 cc.y + __uint_as_float(v[h][4 * i + 1]),
-                                                 cc.z + __uint_as_float(v[h][4 * i + 2]),
-                                                 cc.w + __uint_as_float(v[h][4 * i + 3])};
-                            const int jb = j0 + ch * 32 + 32 * h + 4 * i;
+                            const float4 cc = c4[16 * r + 8 * c + i];
+                            sc[4 * i + 0] = cc.x + __uint_as_float(v[c][4 * i + 0]);
+                            sc[4 * i + 1] = cc.y + __uint_as_float(v[c][4 * i + 1]);
+                            sc[4 * i + 2] = cc.z + __uint_as_float(v[c][4 * i + 2]);
+                            sc[4 * i + 3] = cc.w + __uint_as_float(v[c][4 * i + 3]);
+                        }
+                        const int jb = j0 + half * 128 + 64 * r + 32 * c;
+                        if (TOP2) {
 #pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                if (TOP2) {  // branch-free: a divergent skip test measured slower
-                                    const bool p1 = sc[e] < best, p2 = sc[e] < best2;
-                                    best2 = p1 ? best : (p2 ? sc[e] : best2);
-                                    bidx2 = p1 ? bidx : (p2 ? jb + e : bidx2);
-                                    best = p1 ? sc[e] : best;
-                                    bidx = p1 ? jb + e : bidx;
-                                } else if (sc[e] < best) {
-                                    best = sc[e];
-                                    bidx = jb + e;
-                                }
+                            for (int e = 0; e < 32; ++e) {  // branch-free: a divergent skip test measured slower
+                                const bool p1 = sc[e] < best, p2 = sc[e] < best2;
+                                best2 = p1 ? best : (p2 ? sc[e] : best2);
+                                bidx2 = p1 ? bidx : (p2 ? jb + e : bidx2);
+                                best = p1 ? sc[e] : best;
+                                bidx = p1 ? jb + e : bidx;
+                            }
+                        } else {
+                            // the chunk minimum first; only a row it improves looks for the
+                            // lowest column that reaches it
+                            float mn = sc[0];
+#pragma unroll
+                            for (int e = 1; e < 32; ++e) mn = fminf(mn, sc[e]);
+                            if (mn < best) {
+                                int first = 31;
+#pragma unroll
+                                for (int e = 30; e >= 0; --e) first = (sc[e] == mn) ? e : first;
+                                best = mn;
+                                bidx = jb + first;
                             }
                         }
                     }
                 }
-                tc_fence_before();
-                mbar_arrive(smem_u32(&tempty[acc]));
                 acc ^= 1;
                 if (acc == 0) acc_phase ^= 1u;
                 cnbuf ^= 1;
             }
             if (!ok) break;
-            const int row = m * BM + 32 * q + lane;
-            if (row < rows) {
+            // merge the two column halves of each row: (score, index) keys order as
+            // the argmin does (lower score, then lower index)
+            const unsigned long long k1 = best < __int_as_float(0x7f800000) ? pack_key(best, (uint32_t)bidx) : kEmptyKey;
+            const unsigned long long k2 =
+                TOP2 && best2 < __int_as_float(0x7f800000) ? pack_key(best2, (uint32_t)bidx2) : kEmptyKey;
+            if (half == 1) {
+                half_keys[2 * rl] = k1;
+                half_keys[2 * rl + 1] = k2;
+            }
+            epi_sync();
+            const int row = m * BM + rl;
+            if (half == 0 && row < rows) {
+                const unsigned long long o1 = half_keys[2 * rl], o2 = half_keys[2 * rl + 1];
                 unsigned long long* out = keys + ((int64_t)g * rows + row) * 2;
-                out[0] = pack_key(best, (uint32_t)bidx);
-                out[1] = TOP2 && best2 < __int_as_float(0x7f800000) ? pack_key(best2, (uint32_t)bidx2) : kEmptyKey;
+                out[0] = k1 < o1 ? k1 : o1;
+                if (TOP2) {
+                    const unsigned long long hi = k1 < o1 ? o1 : k1;
+                    const unsigned long long lo2 = k2 < o2 ? k2 : o2;
+                    out[1] = hi < lo2 ? hi : lo2;
+                } else {
+                    out[1] = kEmptyKey;
+                }
             }
         }
     }

@@ -46,18 +46,42 @@ __device__ __forceinline__ void merge_keys(const unsigned long long* __restrict_
                                            int64_t r, unsigned long long& k1, unsigned long long& k2) {
     k1 = kEmptyKey;
     k2 = kEmptyKey;
-    for (int g = 0; g < nsplit; ++g) {
+    // the first eight splits: all loads issued before the first compare
+    unsigned long long c[8][2];
+#pragma unroll
+    for (int g = 0; g < 8; ++g) {
+        c[g][0] = c[g][1] = kEmptyKey;
+        if (g < nsplit) {
+            const ulonglong2 kk = reinterpret_cast<const ulonglong2*>(keys)[(int64_t)g * rows + r];
+            c[g][0] = kk.x;
+            c[g][1] = kk.y;
+        }
+    }
+    for (int g = 8; g < nsplit; ++g) {  // more splits (small inputs of a full pass)
+        const ulonglong2 kk = reinterpret_cast<const ulonglong2*>(keys)[(int64_t)g * rows + r];
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
-            const unsigned long long c = keys[((int64_t)g * rows + r) * 2 + e];
-            if (c < k1) {
+            const unsigned long long x = e ? kk.y : kk.x;
+            if (x < k1) {
                 k2 = k1;
-                k1 = c;
-            } else if (c < k2) {
-                k2 = c;
+                k1 = x;
+            } else if (x < k2) {
+                k2 = x;
             }
         }
     }
+#pragma unroll
+    for (int g = 0; g < 8; ++g)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const unsigned long long x = c[g][e];
+            if (x < k1) {
+                k2 = k1;
+                k1 = x;
+            } else if (x < k2) {
+                k2 = x;
+            }
+        }
 }
 
 // For every lane of the warp whose row is a near tie (flag), the warp recomputes
@@ -296,28 +320,38 @@ __device__ __forceinline__ SliceGeom slice_geom(int slice, int nv) {
     return g;
 }
 
-// Sum over rows perm[s0..s1) of this lane's vector, fp64; the warp's row groups are
-// folded together at the end with a fixed butterfly, so lanes l < lpr hold the
-// slice totals of vector vbase + l.
+// Rows per work item of the grouped update (one chunk of a cluster).
+constexpr int kChunkRows = 64;
+
+// Sum over rows perm[s0..s1) (at most kChunkRows) of this lane's vector, fp64. The
+// chunk's row ids are loaded once (two per lane) and handed out by shuffles; eight
+// rows are in flight per lane. The warp's row groups are folded together at the
+// end with a fixed butterfly, so lanes l < lpr hold the slice totals of vector
+// vbase + l.
 __device__ __forceinline__ void sum_rows(double acc[8], const __nv_bfloat16* __restrict__ src, int ld,
                                          const int32_t* __restrict__ perm, int s0, int s1, const SliceGeom& g,
                                          int lane) {
 #pragma unroll
     for (int t = 0; t < 8; ++t) acc[t] = 0.0;
+    const int n = s1 - s0;
+    const int pa = lane < n ? perm[s0 + lane] : 0;
+    const int pb = lane + 32 < n ? perm[s0 + 32 + lane] : 0;
     const int sub = lane / g.lpr, vi = lane % g.lpr;
     const bool vec_ok = vi < g.nvs;
     const int v = g.vbase + vi;
-    for (int s = s0; s < s1; s += 4 * g.rpi) {
-        uint4 u[4];
-        bool have[4];
+    for (int s = 0; s < n; s += 8 * g.rpi) {
+        uint4 u[8];
+        bool have[8];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {  // up to four rows in flight per lane
-            const int slot = s + q * g.rpi + sub;
-            have[q] = vec_ok && slot < s1;
-            if (have[q]) u[q] = reinterpret_cast<const uint4*>(src + (int64_t)perm[slot] * ld)[v];
+        for (int q = 0; q < 8; ++q) {
+            const int idx = s + q * g.rpi + sub;
+            const int ra = __shfl_sync(0xFFFFFFFFu, pa, idx & 31);
+            const int rb = __shfl_sync(0xFFFFFFFFu, pb, idx & 31);
+            have[q] = vec_ok && idx < n;
+            if (have[q]) u[q] = reinterpret_cast<const uint4*>(src + (int64_t)(idx < 32 ? ra : rb) * ld)[v];
         }
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
+        for (int q = 0; q < 8; ++q) {
             if (have[q]) {
                 float x[8];
                 unpack8_bf16(u[q], x);
@@ -345,11 +379,11 @@ __device__ __forceinline__ void load_s(const ClusterState& st, int j, const Slic
 // vbase + l) and its previous sums so[]: writes S, c, the bf16 operand and the
 // closing-mean sums; slice 0 also writes N and the closing-mean count. Returns
 // the slice's part of |bf16(c_j)|^2 (the same value in every lane).
-__device__ __forceinline__ float ema_slice(const ClusterState& st, int j, double nj, int slice, const SliceGeom& g,
-                                           const double acc[8], const float so[8], int lane, double alpha,
-                                           int last_pass) {
+__device__ __forceinline__ float ema_slice(const ClusterState& st, int j, double nj, float nprev, int slice,
+                                           const SliceGeom& g, const double acc[8], const float so[8], int lane,
+                                           double alpha, int last_pass) {
     const double a1 = 1.0 - alpha;
-    const float Nnew = (float)(a1 * (double)st.N_prev[j] + alpha * nj);
+    const float Nnew = (float)(a1 * (double)nprev + alpha * nj);
     float cn_part = 0.0f;
     if (lane < g.nvs) {
         const int v = g.vbase + lane;
@@ -381,7 +415,7 @@ __device__ __forceinline__ float ema_slice(const ClusterState& st, int j, double
 // rows of one cluster. A cluster that fits in one chunk is updated here (its S
 // slice is fetched while the rows load); the chunks of a larger cluster leave
 // their slice sums in part[item] for k_clusters.
-__global__ void __launch_bounds__(256, 3) k_segsum(const __nv_bfloat16* __restrict__ src,
+__global__ void __launch_bounds__(256, 2) k_segsum(const __nv_bfloat16* __restrict__ src,
                                                    const int32_t* __restrict__ perm, const int2* __restrict__ items,
                                                    const int32_t* __restrict__ off, const int32_t* __restrict__ poff,
                                                    int R, int nslices, int nv, ClusterState st, StepParams sp,
@@ -397,11 +431,16 @@ __global__ void __launch_bounds__(256, 3) k_segsum(const __nv_bfloat16* __restri
     const SliceGeom g = slice_geom(slice, nv);
     const bool single = je - js <= R;
     float so[8];
-    if (single) load_s(st, j, g, lane, so);
+    float nprev = 0.0f;
+    if (single) {
+        load_s(st, j, g, lane, so);
+        nprev = st.N_prev[j];
+    }
     double acc[8];
     sum_rows(acc, src, st.ld, perm, s0, s1, g, lane);
     if (single) {
-        const float cn_part = ema_slice(st, j, (double)(je - js), slice, g, acc, so, lane, sp.alpha, sp.last_pass);
+        const float cn_part =
+            ema_slice(st, j, (double)(je - js), nprev, slice, g, acc, so, lane, sp.alpha, sp.last_pass);
         if (lane == 0) st.cnp[(int64_t)slice * st.k + j] = cn_part;
     } else if (lane < g.nvs) {
         double* dst = part + (int64_t)item * st.ld + 8 * (g.vbase + lane);
@@ -441,6 +480,7 @@ __global__ void k_clusters(const int32_t* __restrict__ off, const int32_t* __res
             }
         } else {
             const int p0 = poff[j], p1 = poff[j + 1];
+            const float nprev = st.N_prev[j];
             float cn_total = 0.0f;
             for (int slice = 0; slice < nslices; ++slice) {
                 const SliceGeom g = slice_geom(slice, nv);
@@ -467,7 +507,7 @@ __global__ void k_clusters(const int32_t* __restrict__ off, const int32_t* __res
 #pragma unroll
                         for (int t = 0; t < 8; ++t) acc[t] += base[(int64_t)p * st.ld + t];
                 }
-                cn_total += ema_slice(st, j, (double)nj, slice, g, acc, so, lane, sp.alpha, sp.last_pass);
+                cn_total += ema_slice(st, j, (double)nj, nprev, slice, g, acc, so, lane, sp.alpha, sp.last_pass);
             }
             if (lane == 0) st.cn[j] = cn_total;
         }

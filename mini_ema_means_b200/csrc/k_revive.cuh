@@ -16,12 +16,14 @@
 //     current batch drawn with Philox(seed, stream 4, t, j), N_j = S_j = 0.
 //
 // The draws are inherently sequential, so one warp makes them on an fp64 tree of
-// prefix sums in shared memory (32 children per node: one load and one ballot per
-// level; a halving updates one suffix of each level with one lane-parallel
-// subtraction); the uniform draws are made in parallel beforehand. The donor's
-// current weight is read back as the difference of two prefix values. The vector
-// work is then done in parallel from the closed form:
-// the o-th split taken from donor d (0-based) sees c_d (1 + eps s)^o and N_d / 2^o.
+// prefix sums (128 children per node, four per lane: the top group sits in
+// registers, each lower level costs one group load, one ballot and one group
+// store per draw); the uniform draws are made in parallel beforehand. The donor's
+// current weight is read back as the difference of two prefix values, and the
+// number of earlier splits from the same donor is counted per batch of 32 draws
+// with one warp match. The vector work is then done in parallel from the closed
+// form: the o-th split taken from donor d (0-based) sees c_d (1 + eps s)^o and
+// N_d / 2^o.
 #pragma once
 
 #include "k_reduce.cuh"
@@ -39,58 +41,77 @@ struct ReviveScratch {
     int64_t* n_splits;  // 1: cumulative number of revived clusters
 };
 
-// Donor tree, 32 children per node, every level stored as inclusive prefix sums
-// within its groups of 32: level 0 over the current weights of the clusters (N_j,
-// or 0 for a dead one), level l >= 1 over the totals of the groups of level l-1.
-// A search costs one shared-memory load and one ballot per level.
-struct TreeLayout {
-    int levels;
-    int size[6];
-    int64_t offset[6];
-    int64_t total;   // doubles
-};
+// Donor tree, 128 children per node (four per lane of a warp). Level 0 holds, for
+// every group of 128 consecutive clusters, the inclusive prefix sums of their
+// current weights within the group (N_j, or 0 for a dead cluster); level l + 1
+// holds the same over the group totals of level l; the top level (at most 128
+// entries, one group) is kept in the drawing warp's registers. Padding positions
+// of a group repeat its total. Every sum is exact in fp64 (the weights are fp32
+// counts and their halvings), so `offset + within-group prefix` is exactly the
+// cumulative weight up to that cluster and each comparison below is the one a
+// search over the cumulative sums of all k weights would make.
+constexpr int kRadix = 128;
+constexpr int kTreeLevels = 5;  // 128^5 > 2^30 clusters
 
 // Shared memory the selection kernel may use (bytes).
 constexpr int kReviveSmemBytes = 200 * 1024;
 
-constexpr int kMaxLevels = 6;  // 32^6 > 2^30 clusters
+struct TreeLayout {
+    int levels;                   // including the top
+    int size[kTreeLevels];        // entries per level
+    int64_t offset[kTreeLevels];  // doubles; every level padded to a multiple of kRadix
+    int64_t total;                // doubles over all levels
+    int smem_from;                // levels in [smem_from, levels - 1) live in shared memory
+    int64_t smem_base;            // offset[smem_from]: where the shared levels start
+    int64_t smem_end;             // offset[levels - 1]: where they end
+    int times_smem;               // split counters in shared memory too
+    int64_t smem_bytes;           // top staging area + shared levels (+ counters)
+};
 
 EM_HD TreeLayout tree_layout(int k) {
     TreeLayout L{};
     int s = k;
     int64_t off = 0;
-    L.levels = 0;
     bool done = false;
 #pragma unroll
-    for (int l = 0; l < kMaxLevels; ++l) {
+    for (int l = 0; l < kTreeLevels; ++l) {
         if (!done) {
             L.size[l] = s;
             L.offset[l] = off;
-            off += ((s + 31) / 32) * 32;
+            off += ((int64_t)(s + kRadix - 1) / kRadix) * kRadix;
             L.levels = l + 1;
-            done = s <= 32;
-            s = (s + 31) / 32;
+            L.smem_end = L.offset[l];  // the top level's offset, once the loop stops
+            done = s <= kRadix;
+            s = (s + kRadix - 1) / kRadix;
         }
     }
     L.total = off;
+    // shared memory: the top level's staging group, then the levels below the top
+    // from the top down while they fit, then the per-donor counters if they fit
+    int64_t bytes = kRadix * 8;
+    L.smem_from = L.levels - 1;
+    L.smem_base = L.smem_end;
+    bool stop = false;
+#pragma unroll
+    for (int l = kTreeLevels - 2; l >= 0; --l) {
+        if (l <= L.levels - 2 && !stop) {
+            const int64_t lb = ((int64_t)(L.size[l] + kRadix - 1) / kRadix) * kRadix * 8;
+            if (bytes + lb <= kReviveSmemBytes) {
+                bytes += lb;
+                L.smem_from = l;
+                L.smem_base = L.offset[l];
+            } else {
+                stop = true;
+            }
+        }
+    }
+    L.times_smem = (L.smem_from == 0 && bytes + (int64_t)k * 4 <= kReviveSmemBytes) ? 1 : 0;
+    if (L.times_smem) bytes += (int64_t)k * 4;
+    L.smem_bytes = bytes;
     return L;
 }
 
-// 0: every level and the split counts in shared memory; 1: level 0 and the split
-// counts in global memory, upper levels shared; 2: everything in global memory.
-EM_HD int tree_placement(const TreeLayout& L, int k) {
-    const int64_t upper = (L.levels > 1 ? L.total - L.offset[1] : 0) * 8;
-    if (L.total * 8 + (int64_t)k * 4 <= kReviveSmemBytes) return 0;
-    if (L.levels > 1 && upper <= kReviveSmemBytes) return 1;
-    return 2;
-}
-
-EM_HD int64_t tree_smem_bytes(const TreeLayout& L, int k) {
-    const int p = tree_placement(L, k);
-    if (p == 0) return L.total * 8 + (int64_t)k * 4;
-    if (p == 1) return (L.total - L.offset[1]) * 8;
-    return 0;
-}
+EM_HD int64_t tree_smem_bytes(const TreeLayout& L, int) { return L.smem_bytes; }
 
 __device__ __forceinline__ double warp_incl_scan(double v, int lane) {
 #pragma unroll
@@ -101,8 +122,77 @@ __device__ __forceinline__ double warp_incl_scan(double v, int lane) {
     return v;
 }
 
-// One CTA of 1024 threads: dead set, donor tree, sequential donor draws.
-__global__ void __launch_bounds__(1024) k_revive_select(const float* __restrict__ N, int k, double tau, uint64_t seed,
+// Inclusive prefix over one group of 128 values, four consecutive values per lane.
+__device__ __forceinline__ void group_scan(double v[4], int lane) {
+    v[1] += v[0];
+    v[2] += v[1];
+    v[3] += v[2];
+    const double inc = warp_incl_scan(v[3], lane);
+    double ex = __shfl_up_sync(0xFFFFFFFFu, inc, 1);
+    if (lane == 0) ex = 0.0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) v[i] += ex;
+}
+
+__device__ __forceinline__ double pick4(const double v[4], int i) {
+    return i == 0 ? v[0] : (i == 1 ? v[1] : (i == 2 ? v[2] : v[3]));
+}
+
+// Unbiased binary exponent of a positive finite double (subnormals included),
+// from the IEEE 754 encoding.
+__device__ __forceinline__ int exponent_of(double x) {
+    const unsigned long long b = (unsigned long long)__double_as_longlong(x);
+    const int e = (int)((b >> 52) & 0x7FF);
+    if (e) return e - 1023;
+    const unsigned long long mant = b & 0xFFFFFFFFFFFFFull;
+    return -1023 - (__clzll(mant) - 12);
+}
+
+// One step of the descent inside a group whose four prefix values this lane holds.
+// Returns the child position (0..127) and, in *before / *w, the within-group
+// prefix before it and its weight. `last`: the target fell on the total, take the
+// last child with positive weight (the first position that reaches the group total).
+__device__ __forceinline__ int group_select(const double P[4], double base, double t, bool last, int lane,
+                                            double* before, double* w) {
+    const double prev3 = __shfl_up_sync(0xFFFFFFFFu, P[3], 1);
+    const double Pprev = lane ? prev3 : 0.0;
+    unsigned m4 = 0;
+    if (!last) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) m4 |= (base + P[i] > t) ? (1u << i) : 0u;
+    }
+    unsigned bal = __ballot_sync(0xFFFFFFFFu, m4 != 0);
+    if (!bal) {  // target on (or, never in exact arithmetic, past) the total
+        const double tot = __shfl_sync(0xFFFFFFFFu, P[3], 31);
+        m4 = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) m4 |= (P[i] >= tot) ? (1u << i) : 0u;
+        bal = __ballot_sync(0xFFFFFFFFu, m4 != 0);
+    }
+    const int L = __ffs(bal) - 1;
+    const int sub = m4 ? __ffs(m4) - 1 : 0;
+    const double b = sub ? pick4(P, sub - 1) : Pprev;
+    const double wl = pick4(P, sub) - b;
+    const int s = __shfl_sync(0xFFFFFFFFu, sub, L);
+    *before = __shfl_sync(0xFFFFFFFFu, b, L);
+    *w = __shfl_sync(0xFFFFFFFFu, wl, L);
+    return 4 * L + s;
+}
+
+// Subtracts delta from the group positions at or after pos (this lane's four).
+__device__ __forceinline__ bool group_sub(double P[4], int pos, double delta, int lane) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        if (4 * lane + i >= pos) P[i] -= delta;
+    return 4 * lane + 3 >= pos;
+}
+
+// One CTA of kSelectThreads threads: dead set, donor tree, sequential donor draws
+// by warp 0 (which keeps one group per tree level in registers).
+constexpr int kSelectThreads = 512;
+constexpr int kSelectWarps = kSelectThreads / 32;
+
+__global__ void __launch_bounds__(kSelectThreads) k_revive_select(const float* __restrict__ N, int k, double tau, uint64_t seed,
                                                         int64_t t, int mode, ReviveScratch sc, int* err) {
     __shared__ double red[32];
     __shared__ int32_t wcount[32];
@@ -111,12 +201,12 @@ __global__ void __launch_bounds__(1024) k_revive_select(const float* __restrict_
 
     // total count in a fixed order
     double part = 0.0;
-    for (int j = tid; j < k; j += 1024) part += (double)N[j];
+    for (int j = tid; j < k; j += kSelectThreads) part += (double)N[j];
     part = warp_sum(part);
     if (lane == 0) red[w] = part;
     __syncthreads();
     if (w == 0) {
-        double v = warp_sum(red[lane]);
+        double v = warp_sum(lane < kSelectWarps ? red[lane] : 0.0);
         if (lane == 0) red[0] = v;
     }
     __syncthreads();
@@ -127,14 +217,14 @@ __global__ void __launch_bounds__(1024) k_revive_select(const float* __restrict_
     // dead set, compacted in increasing index
     if (tid == 0) base_s = 0;
     __syncthreads();
-    for (int b = 0; b < k; b += 1024) {
+    for (int b = 0; b < k; b += kSelectThreads) {
         const int j = b + tid;
         const bool dead = j < k && (double)N[j] < thr;
         const unsigned m = __ballot_sync(0xFFFFFFFFu, dead);
         if (lane == 0) wcount[w] = __popc(m);
         __syncthreads();
         if (w == 0) {
-            const int c = wcount[lane];
+            const int c = lane < kSelectWarps ? wcount[lane] : 0;
             int incl = c;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
@@ -146,133 +236,172 @@ __global__ void __launch_bounds__(1024) k_revive_select(const float* __restrict_
         __syncthreads();
         if (dead) sc.dead[base_s + wcount[w] + __popc(m & ((1u << lane) - 1u))] = j;
         __syncthreads();
-        if (tid == 1023) base_s += wcount[31] + __popc(m);
+        if (tid == kSelectThreads - 1) base_s += wcount[kSelectWarps - 1] + __popc(m);
         __syncthreads();
     }
     const int nd = base_s;
     if (tid == 0) *sc.ndead = nd;
     if (mode != EM_REVIVE_SPLIT || nd == 0 || !(total > 0.0)) {
-        for (int i = tid; i < nd; i += 1024) sc.donor[i] = -1;
-        for (int j = tid; j < k; j += 1024) sc.times[j] = 0;
+        for (int i = tid; i < nd; i += kSelectThreads) sc.donor[i] = -1;
+        for (int j = tid; j < k; j += kSelectThreads) sc.times[j] = 0;
         return;
     }
 
     // draws of every dead cluster, in parallel (they do not depend on each other)
-    for (int i = tid; i < nd; i += 1024) sc.target[i] = draw_uniform(seed, kStreamRevive, t, sc.dead[i]);
+    for (int i = tid; i < nd; i += kSelectThreads) sc.target[i] = draw_uniform(seed, kStreamRevive, t, sc.dead[i]);
 
-    // donor tree
-    extern __shared__ double smem_d[];
+    // donor tree (loops over levels have a fixed trip count so that the layout
+    // stays in registers)
+    extern __shared__ __align__(16) double smem_d[];
     const TreeLayout L = tree_layout(k);
-    const int placement = tree_placement(L, k);
-    // (all loops over levels below have a fixed trip count so that levp[] and
-    // L.size[] are indexed by constants and stay in registers)
-    double* levp[kMaxLevels];
+    const int top = L.levels - 1;
+    double* level_ptr[kTreeLevels];
 #pragma unroll
-    for (int l = 0; l < kMaxLevels; ++l) {
-        if (placement == 0)
-            levp[l] = smem_d + L.offset[l];
-        else if (placement == 1 && l > 0)
-            levp[l] = smem_d + (L.offset[l] - L.offset[1]);
+    for (int l = 0; l < kTreeLevels; ++l) {
+        if (l == top)
+            level_ptr[l] = smem_d;  // staging group of the top level
+        else if (l >= L.smem_from)
+            level_ptr[l] = smem_d + kRadix + (L.offset[l] - L.smem_base);
         else
-            levp[l] = sc.tree + L.offset[l];
+            level_ptr[l] = sc.tree + L.offset[l];
     }
-    int32_t* times = placement == 0 ? reinterpret_cast<int32_t*>(smem_d + L.total) : sc.times;
-    for (int j = tid; j < k; j += 1024) times[j] = 0;
+    int32_t* times = L.times_smem
+                         ? reinterpret_cast<int32_t*>(smem_d + kRadix + (L.smem_end - L.smem_base))
+                         : sc.times;
+    for (int j = tid; j < k; j += kSelectThreads) times[j] = 0;
 #pragma unroll
-    for (int l = 0; l < kMaxLevels; ++l) {
-        if (l < L.levels) {
+    for (int l = 0; l < kTreeLevels; ++l) {
+        if (l <= top) {
             const int sz = L.size[l];
-            const int ngroups = (sz + 31) / 32;
-            for (int gidx = w; gidx < ngroups; gidx += 32) {
-                const int i = gidx * 32 + lane;
-                double v = 0.0;
-                if (i < sz) {
-                    if (l == 0) {
-                        const float nj = N[i];
-                        v = ((double)nj < thr) ? 0.0 : (double)nj;
-                    } else {
-                        v = levp[l > 0 ? l - 1 : 0][i * 32 + 31];  // prefix at the end of child group i
+            const int ngroups = (sz + kRadix - 1) / kRadix;
+            double* dst = level_ptr[l];
+            const double* below = level_ptr[l > 0 ? l - 1 : 0];
+            for (int g = w; g < ngroups; g += kSelectWarps) {
+                double v[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int j = g * kRadix + 4 * lane + i;
+                    v[i] = 0.0;
+                    if (j < sz) {
+                        if (l == 0) {
+                            const float nj = N[j];
+                            v[i] = ((double)nj < thr) ? 0.0 : (double)nj;
+                        } else {
+                            v[i] = below[(int64_t)j * kRadix + kRadix - 1];  // total of child group j
+                        }
                     }
                 }
-                levp[l][gidx * 32 + lane] = warp_incl_scan(v, lane);
+                group_scan(v, lane);
+                double2* o = reinterpret_cast<double2*>(dst + (int64_t)g * kRadix + 4 * lane);
+                o[0] = make_double2(v[0], v[1]);
+                o[1] = make_double2(v[2], v[3]);
             }
         }
         __syncthreads();
     }
 
-    // sequential draws by warp 0
+    // sequential draws by warp 0: the top group in registers, one group load and
+    // store per lower level per draw
     if (w == 0) {
-        const int top = L.levels - 1;
-        double W = 0.0;
-#pragma unroll
-        for (int l = 0; l < kMaxLevels; ++l)
-            if (l == top) W = levp[l][31];
-        bool exhausted = false;
+        double T[4];
+        {
+            const double2* s = reinterpret_cast<const double2*>(smem_d + 4 * lane);
+            const double2 a = s[0], b = s[1];
+            T[0] = a.x; T[1] = a.y; T[2] = b.x; T[3] = b.y;
+        }
+        double W = __shfl_sync(0xFFFFFFFFu, T[3], 31);
+        int64_t splits = 0;
+        int i_end = nd;  // draws from i_end on get no donor (no weight left)
         for (int i0 = 0; i0 < nd; i0 += 32) {
             const int cnt = min(32, nd - i0);
             const double my_u = lane < cnt ? sc.target[i0 + lane] : 0.0;
+            int my_dn = -1;
             for (int q = 0; q < cnt; ++q) {
-                const int i = i0 + q;
-                if (exhausted || !(W > 0.0)) {
-                    exhausted = true;
-                    if (lane == 0) sc.donor[i] = -1;
-                    continue;
+                if (!(W > 0.0)) {
+                    i_end = i0 + q;
+                    break;
                 }
-                double target = __shfl_sync(0xFFFFFFFFu, my_u, q) * W;
-                int node = 0;
-                double wsel = 0.0;  // current weight of the chosen child at the last level
+                const double tg = __shfl_sync(0xFFFFFFFFu, my_u, q) * W;
+                const bool last = !(tg < W);
+                double before, wsel;
+                int node = group_select(T, 0.0, tg, last, lane, &before, &wsel);
+                double base = before;
+                const int node_top = node;
+                int nodes[kTreeLevels - 1];
+                double P[kTreeLevels - 1][4];
 #pragma unroll
-                for (int l = kMaxLevels - 1; l >= 0; --l) {
-                    if (l <= top) {
-                        const int base = node * 32;
-                        const double* lev = levp[l];
-                        const bool valid = base + lane < L.size[l];
-                        const double P = valid ? lev[base + lane] : 0.0;
-                        const unsigned above = __ballot_sync(0xFFFFFFFFu, valid && P > target);
-                        int c;
-                        if (above) {
-                            c = __ffs(above) - 1;
-                        } else {  // target rounded onto the total: the last child with weight
-                            const double Pp = __shfl_up_sync(0xFFFFFFFFu, P, 1);
-                            const unsigned pos = __ballot_sync(0xFFFFFFFFu, valid && P > (lane ? Pp : 0.0));
-                            c = pos ? 31 - __clz(pos) : 0;
+                for (int l = kTreeLevels - 2; l >= 0; --l) {
+                    if (l < top) {
+                        const int64_t g0 = (int64_t)node * kRadix + 4 * lane;
+                        double2 a, b;
+                        if (l >= L.smem_from) {
+                            const double2* s = reinterpret_cast<const double2*>(
+                                smem_d + kRadix + (L.offset[l] - L.smem_base) + g0);
+                            a = s[0];
+                            b = s[1];
+                        } else {
+                            const double2* s = reinterpret_cast<const double2*>(sc.tree + L.offset[l] + g0);
+                            a = s[0];
+                            b = s[1];
                         }
-                        const double before = c > 0 ? lev[base + c - 1] : 0.0;  // broadcast load
-                        if (l == 0) wsel = lev[base + c] - before;
-                        target -= before;
-                        node = base + c;
+                        P[l][0] = a.x; P[l][1] = a.y; P[l][2] = b.x; P[l][3] = b.y;
+                        const int c = group_select(P[l], base, tg, last, lane, &before, &wsel);
+                        base += before;
+                        node = node * kRadix + c;
+                        nodes[l] = node;
                     }
                 }
-                const int dn = node;
-                const double delta = 0.5 * wsel;  // half of the donor's current weight
-                if (lane == 0) {
-                    const int old = times[dn];
-                    times[dn] = old + 1;
-                    sc.donor[i] = dn;
-                    sc.order[i] = old;
-                }
-                int idx = dn;
+                // the donor keeps the rounded half of its weight (what halving N_d gives);
+                // explicit roundings: a fused multiply-add here would round the half
+                // differently in the subnormal range
+                const double keep = __dmul_rn(0.5, wsel);
+                const double delta = __dsub_rn(wsel, keep);
 #pragma unroll
-                for (int l = 0; l < kMaxLevels; ++l) {
-                    if (l < L.levels) {
-                        const int gb = (idx >> 5) << 5;
-                        if (gb + lane >= idx && gb + lane < L.size[l]) levp[l][gb + lane] -= delta;
-                        idx >>= 5;
+                for (int l = 0; l < kTreeLevels - 1; ++l) {
+                    if (l < top) {
+                        const int g = nodes[l] / kRadix;
+                        const int pos = nodes[l] - g * kRadix;
+                        const bool st = group_sub(P[l], pos, delta, lane);
+                        if (st) {
+                            const int64_t g0 = (int64_t)g * kRadix + 4 * lane;
+                            double2* s = l >= L.smem_from
+                                             ? reinterpret_cast<double2*>(smem_d + kRadix +
+                                                                          (L.offset[l] - L.smem_base) + g0)
+                                             : reinterpret_cast<double2*>(sc.tree + L.offset[l] + g0);
+                            s[0] = make_double2(P[l][0], P[l][1]);
+                            s[1] = make_double2(P[l][2], P[l][3]);
+                        }
                     }
                 }
+                group_sub(T, node_top, delta, lane);
                 W -= delta;
-                __syncwarp();
+                if (lane == q) my_dn = node;
             }
+            // record the batch: donor, and how many earlier splits took the same donor
+            const bool has = lane < cnt && my_dn >= 0;
+            const unsigned peers = __match_any_sync(0xFFFFFFFFu, has ? my_dn : -1);
+            const int leader = __ffs(peers) - 1;
+            int old = 0;
+            if (has && lane == leader) old = times[my_dn];
+            old = __shfl_sync(0xFFFFFFFFu, old, leader);
+            if (has) {
+                const int rk = __popc(peers & ((1u << lane) - 1u));
+                sc.donor[i0 + lane] = my_dn;
+                sc.order[i0 + lane] = old + rk;
+                if (lane == leader) times[my_dn] = old + __popc(peers);
+            } else if (lane < cnt) {
+                sc.donor[i0 + lane] = -1;
+            }
+            splits += __popc(__ballot_sync(0xFFFFFFFFu, has));
+            __syncwarp();  // the counters written above are read by other lanes next batch
+            if (i_end < nd) break;
         }
-        if (lane == 0) {
-            int done = 0;
-            for (int i = 0; i < nd; ++i) done += sc.donor[i] >= 0;
-            *sc.n_splits += done;
-        }
+        for (int i = (i_end / 32 + 1) * 32 + lane; i < nd; i += 32) sc.donor[i] = -1;
+        if (lane == 0) *sc.n_splits += splits;
     }
     __syncthreads();
-    if (placement == 0)
-        for (int j = tid; j < k; j += 1024) sc.times[j] = times[j];
+    if (L.times_smem)
+        for (int j = tid; j < k; j += kSelectThreads) sc.times[j] = times[j];
 }
 
 // Dead clusters take their half of the donor (reads the donors' state before
