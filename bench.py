@@ -139,6 +139,19 @@ def oracle_sample_rate(w, xt_dev, seconds, rows_per_step=None, log_prefix="cpu")
 
 # ---------------------------------------------------------------- our arm
 
+def reduce_over_ranks(ms, rows, device, world):
+    """The job's time is the slowest rank's; its rows are every rank's."""
+    if world <= 1:
+        return ms, rows
+    import torch
+
+    t = torch.tensor([ms], device=device, dtype=torch.float64)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    r = torch.tensor([rows], device=device, dtype=torch.float64)
+    torch.distributed.all_reduce(r)
+    return float(t.item()), int(r.item())
+
+
 def run_ours(args, rank, world):
     import torch
 
@@ -218,15 +231,7 @@ def run_ours(args, rank, world):
     ms_prof, _ = timed_pass(profile=True)
     prof = m.profile(reset=True)
     m.set_option("profile", 0)
-    ms_max = ms
-    rows_all = rows
-    if world > 1:
-        t = torch.tensor([ms], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms_max = float(t.item())
-        r = torch.tensor([rows], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(r)
-        rows_all = int(r.item())
+    ms_max, rows_all = reduce_over_ranks(ms, rows, dev, world)
     value = rows_all / (ms_max / 1e3)
     out = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,

@@ -275,7 +275,7 @@ int em_profile(em_model* m, em_profile_t* out, int reset);
 #define EM_NOALLOC_MAX_ROWS 524288
 #define EM_NOALLOC_MAX_K 65536
 #define EM_NOALLOC_MAX_KD 4194304 /* k * d */
-#define EM_NOALLOC_SCRATCH_BYTES 19922944
+#define EM_NOALLOC_SCRATCH_BYTES 28311552 /* 27 MiB */
 int em_assign_noalloc(const void* X, int64_t n, int64_t d, const float* centroids, int64_t k, int64_t* labels,
                       float* dists, void* stream);
 

@@ -199,13 +199,16 @@ struct em_model {
     DBuf<__nv_bfloat16> Xb;
     DBuf<float> xn, dists;
     DBuf<int32_t> ids, labels, cnt, rank, off, poff, perm;
-    DBuf<int2> items;
+    DBuf<int4> items;
     DBuf<unsigned long long> keys;
     DBuf<double> block_err, part, step_err, scalar;
     DBuf<int64_t> labels_last, labels64;
     // revival scratch
     DBuf<int32_t> rv_dead, rv_donor, rv_order, rv_times, rv_ndead;
     DBuf<double> rv_tree, rv_target;
+    DBuf<int4> ties;          // near-tie rows waiting for k_settle
+    DBuf<int> tie_n;          // their number
+    DBuf<double> tie_corr;    // error-sum change of the rows k_settle relabels
     DBuf<int64_t> rv_splits;
     // run progress
     em_recipe_t rec{};
@@ -367,6 +370,7 @@ static int ensure_batch_buffers(em_model* m, int64_t cap) {
     CKR(m->rank.ensure(cap));
     CKR(m->perm.ensure(cap));
     CKR(m->keys.ensure(cap));
+    CKR(m->ties.ensure(cap));
     CKR(m->cnt.ensure(m->k));
     CKR(m->off.ensure(m->k + 1));
     CKR(m->poff.ensure(m->k + 1));
@@ -405,9 +409,23 @@ static int split_for(const em_model* m, int64_t rows) {
     return choose_split(m_tiles, n_tiles, m->sms);
 }
 
-// Keys the search writes for `rows` rows: two per row per centroid-tile group.
+// Keys the search writes for `rows` rows: two per row per key set, two key sets
+// (column halves) per centroid-tile group.
 static size_t keys_needed(const em_model* m, int64_t rows) {
-    return rows > 0 ? (size_t)split_for(m, rows) * (size_t)rows * 2 : 0;
+    return rows > 0 ? (size_t)split_for(m, rows) * tc::kKeySets * (size_t)rows * 2 : 0;
+}
+
+static TieList tie_list(em_model* m) { return TieList{m->ties.p, m->tie_n.p, m->tie_corr.p}; }
+
+// Settles the near ties the label kernel of `rows` rows queued (a no-op launch when
+// there are none): one warp per row over a fixed grid.
+static int launch_settle(em_model* m, const __nv_bfloat16* A, int32_t* labels32, int64_t* labels64, float* dists,
+                         bool count, const int32_t* ids, int64_t* labels_last, int capture) {
+    k_settle<<<m->sms * 8, 256, 0, m->stream>>>(tie_list(m), m->xn.p, A, m->ld, m->cq.p, labels32, labels64, dists,
+                                                count ? m->cnt.p : nullptr, m->rank.p, ids, labels_last, capture);
+    CK(cudaGetLastError());
+    EM_LAUNCHED(m, 1);
+    return EM_OK;
 }
 
 static int launch_assign(em_model* m, const CUtensorMap& tmA, const __nv_bfloat16* A, int64_t rows) {
@@ -445,7 +463,7 @@ static int launch_assign(em_model* m, const CUtensorMap& tmA, const __nv_bfloat1
 #undef EM_ASSIGN
     CK(cudaGetLastError());
     EM_LAUNCHED(m, 1);
-    m->last_split = split;
+    m->last_split = split * tc::kKeySets;
     return EM_OK;
 }
 
@@ -455,7 +473,7 @@ static int launch_reduce(em_model* m, const __nv_bfloat16* src, int64_t rows, in
                          int last_pass, double* err_sum_out) {
     const StepParams sp{alpha, last_pass, 0};
     k_offsets<<<1, 1024, 0, m->stream>>>(m->cnt.p, (int)m->k, (int)rows, m->R, m->off.p, m->poff.p, m->block_err.p,
-                                         nblocks_labels, err_sum_out, m->N.p, m->N_prev.p, m->err.p);
+                                         nblocks_labels, err_sum_out, m->N.p, m->N_prev.p, tie_list(m), m->err.p);
     CK(cudaGetLastError());
     k_scatter<<<(int)((rows + 255) / 256), 256, 0, m->stream>>>(m->labels.p, m->rank.p, m->off.p, m->poff.p,
                                                                  (int)rows, m->R, m->perm.p, m->items.p, m->err.p);
@@ -463,8 +481,9 @@ static int launch_reduce(em_model* m, const __nv_bfloat16* src, int64_t rows, in
     const int64_t max_items = m->k + (rows + m->R - 1) / m->R;
     const int nslices = (m->nv + 31) / 32;
     const ClusterState st = cluster_state(m);
-    k_segsum<<<(int)((max_items * nslices * 32 + 255) / 256), 256, 0, m->stream>>>(
-        src, m->perm.p, m->items.p, m->off.p, m->poff.p, m->R, nslices, m->nv, st, sp, m->part.p);
+    const int seg_blocks = (int)std::min<int64_t>((max_items * nslices * 32 + 255) / 256, (int64_t)m->sms * 2);
+    k_segsum<<<seg_blocks, 256, 0, m->stream>>>(src, m->perm.p, m->items.p, m->poff.p, nslices, m->nv, st, sp,
+                                                m->part.p);
     k_clusters<<<grid_for(m->k * 32, 256, m->sms), 256, 0, m->stream>>>(m->off.p, m->poff.p, m->cnt.p, m->R, nslices,
                                                                          m->nv, st, sp, m->part.p);
     CK(cudaGetLastError());
@@ -557,9 +576,10 @@ static int launch_step(em_model* m, const StepPlan& p) {
     const int capture = (m->capture && p.last_pass) ? 1 : 0;
     k_labels<<<nbl, 256, 0, m->stream>>>(m->keys.p, m->last_split, m->xn.p, (int)rows, (int)m->k, m->Xb.p, m->ld,
                                          m->cq.p, m->ids.p, m->labels.p, m->dists.p, m->cnt.p, m->rank.p,
-                                         m->block_err.p, m->labels_last.p, capture, m->err.p);
+                                         m->block_err.p, m->labels_last.p, capture, tie_list(m), m->err.p);
     CK(cudaGetLastError());
     EM_LAUNCHED(m, 1);
+    CKR(launch_settle(m, m->Xb.p, m->labels.p, nullptr, m->dists.p, true, m->ids.p, m->labels_last.p, capture));
     CKR(launch_reduce(m, m->Xb.p, rows, nbl, p.alpha, m->finalize ? p.last_pass : 0, m->step_err.p + p.t));
     span_end(m, sp, 0.0, 2.0 * rd * dd + 16.0 * rd + 14.0 * kd * dd);
     if (p.revive) {
@@ -584,7 +604,8 @@ static std::vector<uint64_t> graph_signature(const em_model* m) {
                           m->off.p, m->perm.p, m->poff.p, m->items.p, m->keys.p, m->block_err.p, m->part.p,
                           m->step_err.p, m->labels_last.p, m->N.p, m->S.p, m->c.p, m->cn.p, m->cq.p,
                           m->close_sum.p, m->close_cnt.p, m->err.p, m->rv_dead.p, m->rv_donor.p, m->rv_order.p,
-                          m->rv_times.p, m->rv_ndead.p, m->rv_tree.p, m->rv_target.p, m->rv_splits.p};
+                          m->rv_times.p, m->rv_ndead.p, m->rv_tree.p, m->rv_target.p, m->rv_splits.p,
+                          m->ties.p, m->tie_n.p, m->tie_corr.p};
     std::vector<uint64_t> sig;
     for (const void* q : ptrs) sig.push_back((uint64_t)(uintptr_t)q);
     const int64_t ints[] = {m->n, m->d, m->k, m->ld, m->kc, m->R, m->sms, m->rec.batch_size, m->rec.total_steps,
@@ -733,9 +754,11 @@ em_model* em_create(int64_t d, int64_t k, uint64_t seed) {
         m->close_sum.ensure(kd) || m->close_cnt.ensure(k) || m->err.ensure(1) || m->flag.ensure(1) ||
         m->scalar.ensure(4) || m->rv_dead.ensure(k) || m->rv_donor.ensure(k) || m->rv_order.ensure(k) ||
         m->rv_times.ensure(k) || m->rv_ndead.ensure(1) || m->rv_splits.ensure(1) || m->rv_target.ensure(k) ||
-        m->rv_tree.ensure((size_t)tree_layout((int)k).total))
+        m->rv_tree.ensure((size_t)tree_layout((int)k).total) || m->tie_n.ensure(1) || m->tie_corr.ensure(1))
         return bail(EM_E_NOMEM, "device allocation failed");
     cudaMemset(m->err.p, 0, sizeof(int));
+    cudaMemset(m->tie_n.p, 0, sizeof(int));
+    cudaMemset(m->tie_corr.p, 0, sizeof(double));
     cudaMemset(m->rv_splits.p, 0, sizeof(int64_t));
     cudaMemset(m->rv_ndead.p, 0, sizeof(int32_t));
     cudaMemset(m->N.p, 0, k * sizeof(float));
@@ -775,6 +798,7 @@ void em_destroy(em_model* m) {
     m->part.release(); m->step_err.release(); m->scalar.release(); m->labels_last.release();
     m->labels64.release(); m->rv_dead.release(); m->rv_donor.release(); m->rv_order.release();
     m->rv_times.release(); m->rv_ndead.release(); m->rv_tree.release(); m->rv_splits.release();
+    m->ties.release(); m->tie_n.release(); m->tie_corr.release();
     m->rv_target.release();
     for (auto& sp : m->pending) {
         cudaEventDestroy(sp.a);
@@ -983,9 +1007,10 @@ int em_lloyd(em_model* m, const void* X, int64_t n, int64_t iters) {
         CKR(launch_assign(m, tmx, m->X, n));
         k_labels<<<nbl, 256, 0, m->stream>>>(m->keys.p, m->last_split, m->xn.p, (int)n, (int)m->k, m->X, m->ld,
                                              m->cq.p, nullptr, m->labels.p, m->dists.p, m->cnt.p, m->rank.p,
-                                             m->block_err.p, nullptr, 0, m->err.p);
+                                             m->block_err.p, nullptr, 0, tie_list(m), m->err.p);
         CK(cudaGetLastError());
         EM_LAUNCHED(m, 1);
+        CKR(launch_settle(m, m->X, m->labels.p, nullptr, m->dists.p, true, nullptr, nullptr, 0));
         CKR(launch_reduce(m, m->X, n, nbl, 1.0, 0, m->scalar.p));
     }
     m->have_run = false;
@@ -999,7 +1024,12 @@ static int assign_pass(em_model* m, const void* X, int64_t n, int64_t* labels_de
     CKR(prepare_input(m, X, n, tmp, &A));
     CKR(m->xn.ensure(n));
     CKR(m->keys.ensure(keys_needed(m, n)));
+    CKR(m->ties.ensure(n));
     CKR(m->block_err.ensure((n + 255) / 256 + 1));
+    if (!dists_dev) {  // k_settle needs the provisional distances of relabelled rows
+        CKR(m->dists.ensure(n));
+        dists_dev = m->dists.p;
+    }
     k_rownorm_keys<<<grid_for(n * 32, 256, m->sms), 256, 0, m->stream>>>(A, n, m->ld, m->xn.p, nullptr);
     CK(cudaGetLastError());
     EM_LAUNCHED(m, 1);
@@ -1008,11 +1038,13 @@ static int assign_pass(em_model* m, const void* X, int64_t n, int64_t* labels_de
     CKR(launch_assign(m, tmx, A, n));
     const int blocks = grid_for(n, 256, m->sms);
     k_assign_out<<<blocks, 256, 0, m->stream>>>(m->keys.p, m->last_split, m->xn.p, n, (int)m->k, A, m->ld, m->cq.p,
-                                                labels_dev, dists_dev, nullptr, m->block_err.p, m->err.p);
+                                                labels_dev, dists_dev, nullptr, m->block_err.p, tie_list(m), m->err.p);
     CK(cudaGetLastError());
-    k_sum_blocks<<<1, 32, 0, m->stream>>>(m->block_err.p, blocks, sum_dev);
+    EM_LAUNCHED(m, 1);
+    CKR(launch_settle(m, A, nullptr, labels_dev, dists_dev, false, nullptr, nullptr, 0));
+    k_sum_blocks<<<1, 32, 0, m->stream>>>(m->block_err.p, blocks, sum_dev, tie_list(m));
     CK(cudaGetLastError());
-    EM_LAUNCHED(m, 2);
+    EM_LAUNCHED(m, 1);
     return EM_OK;
 }
 
@@ -1267,8 +1299,8 @@ constexpr size_t kNaErr = 0;                                                   /
 constexpr size_t kNaCn = 256;                                                  // fp32 [MAX_K]
 constexpr size_t kNaOperand = kNaCn + (size_t)EM_NOALLOC_MAX_K * 4;            // bf16 [MAX_KD]
 constexpr size_t kNaXn = kNaOperand + (size_t)EM_NOALLOC_MAX_KD * 2;           // fp32 [MAX_ROWS]
-constexpr size_t kNaKeys = kNaXn + (size_t)EM_NOALLOC_MAX_ROWS * 4;            // u64 [2 * MAX_ROWS]
-constexpr size_t kNaBlocks = kNaKeys + (size_t)EM_NOALLOC_MAX_ROWS * 16;       // fp64 [kNaMaxBlocks]
+constexpr size_t kNaKeys = kNaXn + (size_t)EM_NOALLOC_MAX_ROWS * 4;            // u64 [2 * kKeySets * MAX_ROWS]
+constexpr size_t kNaBlocks = kNaKeys + (size_t)EM_NOALLOC_MAX_ROWS * 16 * tc::kKeySets;  // fp64 [kNaMaxBlocks]
 constexpr int kNaMaxBlocks = 4096;
 constexpr size_t kNaEnd = kNaBlocks + (size_t)kNaMaxBlocks * 8;
 static_assert(kNaEnd <= EM_NOALLOC_SCRATCH_BYTES, "scratch layout exceeds the array");
@@ -1372,8 +1404,10 @@ extern "C" int em_assign_noalloc(const void* X, int64_t n, int64_t d, const floa
     const int64_t m_tiles = (n + tc::BM - 1) / tc::BM;
     const int64_t n_tiles = (k + tc::BN - 1) / tc::BN;
     const int nkc = (int)((d + kc - 1) / kc);
-    // the key region holds two keys for EM_NOALLOC_MAX_ROWS rows: split * n rows at most
-    const int split = choose_split(m_tiles, n_tiles, sms, (int)std::max<int64_t>(1, EM_NOALLOC_MAX_ROWS / n));
+    // the key region holds two keys for EM_NOALLOC_MAX_ROWS rows: split * kKeySets * n
+    // rows at most
+    const int split = choose_split(m_tiles, n_tiles, sms,
+                                   (int)std::max<int64_t>(1, EM_NOALLOC_MAX_ROWS / (tc::kKeySets * n)));
     const bool top2 = d >= 256;
     const int grid = (int)std::min<int64_t>(m_tiles * split, sms);
     const long long wait_cycles = (long long)(2000.0 * (double)clock_khz);
@@ -1393,8 +1427,8 @@ extern "C" int em_assign_noalloc(const void* X, int64_t n, int64_t d, const floa
     }
 #undef EM_NA_ASSIGN
     const int oblocks = std::min(grid_for(n, 256, sms), kNaMaxBlocks);
-    k_assign_out<<<oblocks, 256, 0, stream>>>(keys, split, xn, n, (int)k, X16, (int)d, cq, labels, dists, nullptr,
-                                             blocks, err);
+    k_assign_out<<<oblocks, 256, 0, stream>>>(keys, split * tc::kKeySets, xn, n, (int)k, X16, (int)d, cq, labels,
+                                             dists, nullptr, blocks, TieList{nullptr, nullptr, nullptr}, err);
     CK(cudaGetLastError());
     int h = 0;
     CK(cudaMemcpyAsync(&h, err, sizeof(int), cudaMemcpyDeviceToHost, stream));

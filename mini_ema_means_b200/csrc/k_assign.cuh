@@ -15,10 +15,12 @@
 //   warps 2..9  epilogue: thread = accumulator row; warps w and w + 4 share the
 //               TMEM lane quadrant w % 4 and take the left and right 128 columns
 //               of the tile: tcgen05.ld, free the accumulator, add |c|^2, running
-//               argmin; the two halves of a row are merged once per work unit
-// A work unit is (128-row tile, group of 256-wide centroid tiles). When k is
-// split over several units, every group writes its own per-row result
-// ((order-preserving score, index) keys) and the label kernel merges them. With
+//               argmin. The eight warps never wait for each other: each stages its
+//               own |c|^2 values and writes its own keys (one key set per column
+//               half), and the label kernel merges the key sets
+// A work unit is (128-row tile, group of 256-wide centroid tiles). Every group
+// writes its own per-row results ((order-preserving score, index) keys), two key
+// sets per group, and the label kernel merges them. With
 // TOP2 the epilogue also keeps the second best candidate, so that near ties can be
 // settled exactly afterwards.
 #pragma once
@@ -32,6 +34,8 @@ constexpr int BM = 128;
 constexpr int BN = 256;
 constexpr int kThreads = 320;
 constexpr int kEpiThreads = 256;
+constexpr int kEpiWarps = 8;
+constexpr int kKeySets = 2;  // key sets per centroid-tile group (the two column halves)
 
 template <int KC>
 struct Cfg {
@@ -42,8 +46,8 @@ struct Cfg {
     static constexpr uint64_t kLayout = KC == 64 ? 2ull : 4ull;  // UMMA 128B / 64B swizzle
     static constexpr uint32_t kSBO = 8u * KC * 2u;                // bytes between 8-row groups
     static constexpr int kBarBytes = 256;
-    // + |c|^2 of two tiles, + the right halves' keys of one row tile
-    static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kBarBytes + 2 * BN * 4 + BM * 2 * 8;
+    // + each epilogue warp's |c|^2 values of two tiles (its 128 columns)
+    static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kBarBytes + kEpiWarps * 2 * 128 * 4;
 };
 
 // Instruction descriptor of tcgen05.mma kind::f16: fp32 accumulate (bits 4-5 = 1),
@@ -112,23 +116,6 @@ __device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity, long l
     }
 }
 
-// AND of `ok` over the 256 epilogue threads; doubles as their named barrier 1.
-__device__ __forceinline__ bool epi_all(bool ok) {
-    uint32_t r;
-    asm volatile(
-        "{\n\t.reg .pred p, q;\n\t"
-        "setp.ne.u32 p, %1, 0;\n\t"
-        "bar.red.and.pred q, 1, 256, p;\n\t"
-        "selp.u32 %0, 1, 0, q;\n\t}\n"
-        : "=r"(r)
-        : "r"((uint32_t)ok)
-        : "memory");
-    return r != 0;
-}
-
-// Named barrier 2 over the 256 epilogue threads.
-__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 2, 256;" ::: "memory"); }
-
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* tm, int x, int y, uint32_t bar) {
     asm volatile(
         "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
@@ -177,9 +164,10 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
 
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
-// Output: for every row, the split g of the centroid tiles it covers writes two
-// keys at keys[(g * rows + row) * 2 + {0, 1}]: the best (score, index) and, with
-// TOP2, the second best (without it the second key is empty).
+// Output: for every row, column half h of the split g of the centroid tiles it
+// covers writes two keys at keys[((2 g + h) * rows + row) * 2 + {0, 1}]: the best
+// (score, index) and, with TOP2, the second best (without it the second key is
+// empty).
 template <int KC, bool TOP2>
 __global__ void __launch_bounds__(kThreads, 1)
     k_assign_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -200,7 +188,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 5);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     float* cn_s = reinterpret_cast<float*>(smem + S * C::kStageBytes + C::kBarBytes);
-    unsigned long long* half_keys = reinterpret_cast<unsigned long long*>(cn_s + 2 * BN);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -325,21 +312,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         // ---------------- epilogue: 8 warps, thread = accumulator row, warp = column half
-        const int et = threadIdx.x - 64;
         const int q = warp & 3;
         const int half = (warp - 2) >> 2;
         const int rl = 32 * q + lane;  // row within the tile
         const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+        float* cn_w = cn_s + (warp - 2) * 2 * 128;  // this warp's two |c|^2 buffers
         int acc = 0;
         uint32_t acc_phase = 0;
         int cnbuf = 0;
         bool ok = true;
-        // |c|^2 of the next tile this CTA handles, loaded one tile ahead
-        auto cn_of = [&](int j) { return j < k ? cn[j] : __int_as_float(0x7f800000); };
-        float cn_next = 0.0f;
+        // this lane's four |c|^2 values of the next tile the warp handles, one tile ahead
+        auto cn4_of = [&](int j) {
+            float4 r;
+            r.x = j + 0 < k ? cn[j + 0] : __int_as_float(0x7f800000);
+            r.y = j + 1 < k ? cn[j + 1] : __int_as_float(0x7f800000);
+            r.z = j + 2 < k ? cn[j + 2] : __int_as_float(0x7f800000);
+            r.w = j + 3 < k ? cn[j + 3] : __int_as_float(0x7f800000);
+            return r;
+        };
+        float4 cn_next = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
         if (blockIdx.x < units) {
             const int g0 = blockIdx.x % n_split;
-            cn_next = cn_of(g0 * tpg * BN + et);
+            cn_next = cn4_of(g0 * tpg * BN + half * 128 + 4 * lane);
         }
         for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
             const int m = u / n_split, g = u - m * n_split;
@@ -348,9 +342,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             float best2 = best;
             int bidx = 0, bidx2 = 0;
             for (int nt = nt0; nt < nt1; ++nt) {
-                float* cnb = cn_s + cnbuf * BN;
+                float* cnb = cn_w + cnbuf * 128;
                 const int j0 = nt * BN;
-                cnb[et] = cn_next;
+                reinterpret_cast<float4*>(cnb)[lane] = cn_next;
                 {
                     int jn = -1;
                     if (nt + 1 < nt1) {
@@ -359,19 +353,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const int gn = (u + (int)gridDim.x) % n_split;
                         jn = gn * tpg * BN;
                     }
-                    if (jn >= 0) cn_next = cn_of(jn + et);
+                    if (jn >= 0) cn_next = cn4_of(jn + half * 128 + 4 * lane);
                 }
-                const bool got = mbar_wait(smem_u32(&tfull[acc]), acc_phase, wait_limit, err, abort_flag);
-                // one decision for all 256 threads (so none is left at a barrier), and the
-                // barrier that publishes this tile's |c|^2 values
-                if (!epi_all(got)) {
+                // the whole warp takes one decision (a lane that gave up takes the warp with it)
+                const bool got = __all_sync(0xFFFFFFFFu,
+                                            mbar_wait(smem_u32(&tfull[acc]), acc_phase, wait_limit, err, abort_flag));
+                if (!got) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                __syncwarp();
+                __syncwarp();  // also publishes this warp's |c|^2 values
                 const uint32_t tbase = tmem_base + lane_base + (uint32_t)(acc * BN + half * 128);
-                const float4* c4 = reinterpret_cast<const float4*>(cnb + half * 128);
+                const float4* c4 = reinterpret_cast<const float4*>(cnb);
                 // two rounds of 64 columns (the register file allows no more per thread
                 // with ten warps: three of them share a sub-partition)
 #pragma unroll 1
@@ -426,28 +420,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 cnbuf ^= 1;
             }
             if (!ok) break;
-            // merge the two column halves of each row: (score, index) keys order as
-            // the argmin does (lower score, then lower index)
-            const unsigned long long k1 = best < __int_as_float(0x7f800000) ? pack_key(best, (uint32_t)bidx) : kEmptyKey;
-            const unsigned long long k2 =
-                TOP2 && best2 < __int_as_float(0x7f800000) ? pack_key(best2, (uint32_t)bidx2) : kEmptyKey;
-            if (half == 1) {
-                half_keys[2 * rl] = k1;
-                half_keys[2 * rl + 1] = k2;
-            }
-            epi_sync();
+            // this column half's key set: (score, index) keys order as the argmin does
+            // (lower score, then lower index)
             const int row = m * BM + rl;
-            if (half == 0 && row < rows) {
-                const unsigned long long o1 = half_keys[2 * rl], o2 = half_keys[2 * rl + 1];
-                unsigned long long* out = keys + ((int64_t)g * rows + row) * 2;
-                out[0] = k1 < o1 ? k1 : o1;
-                if (TOP2) {
-                    const unsigned long long hi = k1 < o1 ? o1 : k1;
-                    const unsigned long long lo2 = k2 < o2 ? k2 : o2;
-                    out[1] = hi < lo2 ? hi : lo2;
-                } else {
-                    out[1] = kEmptyKey;
-                }
+            if (row < rows) {
+                unsigned long long* out = keys + ((int64_t)(kKeySets * g + half) * rows + row) * 2;
+                out[0] = best < __int_as_float(0x7f800000) ? pack_key(best, (uint32_t)bidx) : kEmptyKey;
+                out[1] = TOP2 && best2 < __int_as_float(0x7f800000) ? pack_key(best2, (uint32_t)bidx2) : kEmptyKey;
             }
         }
     }

@@ -120,12 +120,32 @@ __device__ __forceinline__ void settle_ties(bool flag, int64_t row, uint32_t& l1
     }
 }
 
+// Near-tie rows are settled after the label kernels, one warp per row and all rows
+// in parallel (k_settle): the label kernels write the provisional best candidate
+// and append the row here.
+struct TieList {
+    int4* e;       // (row, first label, second label, bits of the second score)
+    int* n;        // entries
+    double* corr;  // sum of the distance changes of the rows k_settle relabels
+};
+
+// Appends this warp's flagged rows to the tie list (one atomic per warp).
+__device__ __forceinline__ void push_ties(bool flag, int64_t r, uint32_t l1, uint32_t l2, float s2, const TieList& tl,
+                                          int lane) {
+    const unsigned m = __ballot_sync(0xFFFFFFFFu, flag);
+    if (!m) return;
+    int base = 0;
+    if (lane == 0) base = atomicAdd(tl.n, __popc(m));
+    base = __shfl_sync(0xFFFFFFFFu, base, 0);
+    if (flag) tl.e[base + __popc(m & ((1u << lane) - 1u))] = make_int4((int)r, (int)l1, (int)l2, __float_as_int(s2));
+}
+
 __global__ void k_labels(const unsigned long long* __restrict__ keys, int nsplit, const float* __restrict__ xn,
                          int rows, int k, const __nv_bfloat16* __restrict__ A, int ld,
                          const __nv_bfloat16* __restrict__ cq, const int32_t* __restrict__ ids,
                          int32_t* __restrict__ labels, float* __restrict__ dists, int32_t* __restrict__ cnt,
                          int32_t* __restrict__ rank, double* __restrict__ block_err, int64_t* __restrict__ labels_last,
-                         int capture, int* err) {
+                         int capture, TieList tl, int* err) {
     __shared__ double warp_err[32];
     const int lane = threadIdx.x & 31;
     double e = 0.0;
@@ -150,7 +170,12 @@ __global__ void k_labels(const unsigned long long* __restrict__ keys, int nsplit
             tie = l2 < (uint32_t)k && s2 - s1 <= kTieRel * (x2 + fabsf(s1) + fabsf(s2));
         }
     }
-    settle_ties(tie, r, l1, s1, l2, s2, A, ld, cq, lane);
+    // a near tie is left to k_settle: provisional label and distance now, counted there
+    const bool defer = tie && tl.e != nullptr;
+    if (tl.e)
+        push_ties(defer, r, l1, l2, s2, tl, lane);
+    else
+        settle_ties(tie, r, l1, s1, l2, s2, A, ld, cq, lane);
     int lab = -1;
     if (active) {
         lab = (int)l1;
@@ -158,10 +183,11 @@ __global__ void k_labels(const unsigned long long* __restrict__ keys, int nsplit
         labels[r] = lab;
         dists[r] = dist;
         e = (double)dist;
-        if (capture) labels_last[ids[r]] = lab;
+        if (capture && !defer) labels_last[ids[r]] = lab;
     }
-    const unsigned amask = __ballot_sync(0xFFFFFFFFu, active);
-    if (active) {
+    const bool counted = active && !defer;
+    const unsigned amask = __ballot_sync(0xFFFFFFFFu, counted);
+    if (counted) {
         const unsigned peers = __match_any_sync(amask, lab);
         const int leader = __ffs(peers) - 1;
         const int before = __popc(peers & ((1u << lane) - 1u));
@@ -188,7 +214,7 @@ __global__ void __launch_bounds__(1024) k_offsets(const int32_t* __restrict__ cn
                                                   int32_t* __restrict__ off, int32_t* __restrict__ poff,
                                                   const double* __restrict__ block_err, int nblocks,
                                                   double* __restrict__ err_sum_out, const float* __restrict__ N,
-                                                  float* __restrict__ N_prev, int* err) {
+                                                  float* __restrict__ N_prev, TieList tl, int* err) {
     __shared__ int2 warp_tot[32];
     __shared__ int2 carry_s;
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
@@ -256,6 +282,11 @@ __global__ void __launch_bounds__(1024) k_offsets(const int32_t* __restrict__ cn
             off[k] = carry_s.x;
             poff[k] = carry_s.y;
             if (carry_s.x != rows) raise_error(err, EM_E_BOUNDS);
+            if (tl.n) {  // the relabelled near ties (k_settle ran before), then an empty list
+                t += *tl.corr;
+                *tl.n = 0;
+                *tl.corr = 0.0;
+            }
             *err_sum_out = t;
         }
     }
@@ -265,7 +296,7 @@ __global__ void __launch_bounds__(1024) k_offsets(const int32_t* __restrict__ cn
 // rows of a cluster also writes that chunk's work item (cluster, first sorted position).
 __global__ void k_scatter(const int32_t* __restrict__ labels, const int32_t* __restrict__ rank,
                           const int32_t* __restrict__ off, const int32_t* __restrict__ poff, int rows, int R,
-                          int32_t* __restrict__ perm, int2* __restrict__ items, int* err) {
+                          int32_t* __restrict__ perm, int4* __restrict__ items, int* err) {
     const int r = blockIdx.x * blockDim.x + threadIdx.x;
     if (r >= rows) return;
     const int lab = labels[r];
@@ -276,7 +307,10 @@ __global__ void k_scatter(const int32_t* __restrict__ labels, const int32_t* __r
         return;
     }
     perm[pos] = r;
-    if (rk % R == 0) items[poff[lab] + rk / R] = make_int2(lab, pos);
+    if (rk % R == 0) {  // work item: (cluster, first row, end row, cluster fits in one chunk)
+        const int s0 = off[lab], s1 = off[lab + 1];
+        items[poff[lab] + rk / R] = make_int4(lab, pos, min(pos + R, s1), s1 - s0 <= R ? 1 : 0);
+    }
 }
 
 // ---------------------------------------------------------------- segmented sums + EMA
@@ -323,19 +357,15 @@ __device__ __forceinline__ SliceGeom slice_geom(int slice, int nv) {
 // Rows per work item of the grouped update (one chunk of a cluster).
 constexpr int kChunkRows = 64;
 
-// Sum over rows perm[s0..s1) (at most kChunkRows) of this lane's vector, fp64. The
-// chunk's row ids are loaded once (two per lane) and handed out by shuffles; eight
-// rows are in flight per lane. The warp's row groups are folded together at the
+// Sum over the n (at most kChunkRows) rows of a chunk of this lane's vector, fp64.
+// The chunk's row ids come preloaded, two per lane (pa: rows 0..31, pb: rows
+// 32..63), and are handed out by shuffles; eight rows are in flight per lane. The warp's row groups are folded together at the
 // end with a fixed butterfly, so lanes l < lpr hold the slice totals of vector
 // vbase + l.
-__device__ __forceinline__ void sum_rows(double acc[8], const __nv_bfloat16* __restrict__ src, int ld,
-                                         const int32_t* __restrict__ perm, int s0, int s1, const SliceGeom& g,
-                                         int lane) {
+__device__ __forceinline__ void sum_rows(double acc[8], const __nv_bfloat16* __restrict__ src, int ld, int pa, int pb,
+                                         int n, const SliceGeom& g, int lane) {
 #pragma unroll
     for (int t = 0; t < 8; ++t) acc[t] = 0.0;
-    const int n = s1 - s0;
-    const int pa = lane < n ? perm[s0 + lane] : 0;
-    const int pb = lane + 32 < n ? perm[s0 + 32 + lane] : 0;
     const int sub = lane / g.lpr, vi = lane % g.lpr;
     const bool vec_ok = vi < g.nvs;
     const int v = g.vbase + vi;
@@ -411,41 +441,71 @@ __device__ __forceinline__ float ema_slice(const ClusterState& st, int j, double
     return cn_part;
 }
 
-// One warp per (work item, slice). A work item is a chunk of at most R label-sorted
-// rows of one cluster. A cluster that fits in one chunk is updated here (its S
-// slice is fetched while the rows load); the chunks of a larger cluster leave
-// their slice sums in part[item] for k_clusters.
+// Persistent warps over the (work item, slice) units. A work item is a chunk of
+// at most R label-sorted rows of one cluster. A cluster that fits in one chunk is
+// updated here; the chunks of a larger cluster leave their slice sums in
+// part[item] for k_clusters. Software pipeline: while a unit's rows load and add,
+// the warp already holds the next unit's item and fetches its row ids, S slice and
+// previous count, and the item after that, so that a unit costs about one memory
+// round trip instead of the chain item -> row ids -> rows.
 __global__ void __launch_bounds__(256, 2) k_segsum(const __nv_bfloat16* __restrict__ src,
-                                                   const int32_t* __restrict__ perm, const int2* __restrict__ items,
-                                                   const int32_t* __restrict__ off, const int32_t* __restrict__ poff,
-                                                   int R, int nslices, int nv, ClusterState st, StepParams sp,
-                                                   double* __restrict__ part) {
+                                                   const int32_t* __restrict__ perm, const int4* __restrict__ items,
+                                                   const int32_t* __restrict__ poff, int nslices, int nv,
+                                                   ClusterState st, StepParams sp, double* __restrict__ part) {
     const int lane = threadIdx.x & 31;
-    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    const int item = warp / nslices, slice = warp - item * nslices;
-    if (item >= poff[st.k]) return;
-    const int2 it = items[item];
-    const int j = it.x, s0 = it.y;
-    const int js = off[j], je = off[j + 1];
-    const int s1 = min(s0 + R, je);
-    const SliceGeom g = slice_geom(slice, nv);
-    const bool single = je - js <= R;
-    float so[8];
-    float nprev = 0.0f;
-    if (single) {
-        load_s(st, j, g, lane, so);
-        nprev = st.N_prev[j];
-    }
-    double acc[8];
-    sum_rows(acc, src, st.ld, perm, s0, s1, g, lane);
-    if (single) {
-        const float cn_part =
-            ema_slice(st, j, (double)(je - js), nprev, slice, g, acc, so, lane, sp.alpha, sp.last_pass);
-        if (lane == 0) st.cnp[(int64_t)slice * st.k + j] = cn_part;
-    } else if (lane < g.nvs) {
-        double* dst = part + (int64_t)item * st.ld + 8 * (g.vbase + lane);
+    const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int nw = (gridDim.x * blockDim.x) >> 5;
+    const int nunits = poff[st.k] * nslices;
+    auto item_of = [&](int u) { return u < nunits ? items[u / nslices] : make_int4(0, 0, 0, 0); };
+    auto ids_of = [&](const int4& it, int u, int& pa, int& pb) {
+        const int n = it.z - it.y;
+        pa = (u < nunits && lane < n) ? perm[it.y + lane] : 0;
+        pb = (u < nunits && lane + 32 < n) ? perm[it.y + 32 + lane] : 0;
+    };
+    auto state_of = [&](const int4& it, int u, float so[8], float& np) {
+        np = 0.0f;
+        if (u < nunits && it.w) {
+            load_s(st, it.x, slice_geom(u % nslices, nv), lane, so);
+            np = st.N_prev[it.x];
+        }
+    };
+    int u = gw;
+    int4 it = item_of(u);
+    int pa, pb;
+    ids_of(it, u, pa, pb);
+    float so[8], np;
+    state_of(it, u, so, np);
+    int4 itn = item_of(u + nw);
+    for (; u < nunits; u += nw) {
+        const int un = u + nw;
+        // next unit: row ids, S slice and count (its item arrived during the last unit)
+        int pan, pbn;
+        ids_of(itn, un, pan, pbn);
+        float son[8], npn;
+        state_of(itn, un, son, npn);
+        const int4 itnn = item_of(un + nw);
+        // this unit
+        const int slice = u % nslices;
+        const SliceGeom g = slice_geom(slice, nv);
+        const int j = it.x;
+        double acc[8];
+        sum_rows(acc, src, st.ld, pa, pb, it.z - it.y, g, lane);
+        if (it.w) {
+            const double nj = (double)(it.z - it.y);
+            const float cn_part = ema_slice(st, j, nj, np, slice, g, acc, so, lane, sp.alpha, sp.last_pass);
+            if (lane == 0) st.cnp[(int64_t)slice * st.k + j] = cn_part;
+        } else if (lane < g.nvs) {
+            double* dst = part + (int64_t)(u / nslices) * st.ld + 8 * (g.vbase + lane);
 #pragma unroll
-        for (int t = 0; t < 8; ++t) dst[t] = acc[t];
+            for (int t = 0; t < 8; ++t) dst[t] = acc[t];
+        }
+        it = itn;
+        pa = pan;
+        pb = pbn;
+#pragma unroll
+        for (int t = 0; t < 8; ++t) so[t] = son[t];
+        np = npn;
+        itn = itnn;
     }
 }
 
@@ -523,7 +583,7 @@ __global__ void k_assign_out(const unsigned long long* __restrict__ keys, int ns
                              int64_t rows, int k, const __nv_bfloat16* __restrict__ A, int ld,
                              const __nv_bfloat16* __restrict__ cq, int64_t* __restrict__ labels,
                              float* __restrict__ dists, int32_t* __restrict__ labels32, double* __restrict__ block_err,
-                             int* err) {
+                             TieList tl, int* err) {
     __shared__ double warp_err[32];
     const int lane = threadIdx.x & 31;
     double e = 0.0;
@@ -550,7 +610,10 @@ __global__ void k_assign_out(const unsigned long long* __restrict__ keys, int ns
                 tie = l2 < (uint32_t)k && s2 - s1 <= kTieRel * (x2 + fabsf(s1) + fabsf(s2));
             }
         }
-        settle_ties(tie, r, l1, s1, l2, s2, A, ld, cq, lane);
+        if (tl.e)
+            push_ties(tie, r, l1, l2, s2, tl, lane);
+        else
+            settle_ties(tie, r, l1, s1, l2, s2, A, ld, cq, lane);
         if (active) {
             const float dist = fmaxf(0.0f, x2 + s1);
             if (labels) labels[r] = (int64_t)l1;
@@ -569,11 +632,71 @@ __global__ void k_assign_out(const unsigned long long* __restrict__ keys, int ns
     }
 }
 
-__global__ void k_sum_blocks(const double* __restrict__ block_err, int nblocks, double* __restrict__ out) {
+__global__ void k_sum_blocks(const double* __restrict__ block_err, int nblocks, double* __restrict__ out,
+                             TieList tl) {
     if (blockIdx.x == 0 && threadIdx.x == 0) {
         double t = 0.0;
         for (int b = 0; b < nblocks; ++b) t += block_err[b];
+        if (tl.n) {
+            t += *tl.corr;
+            *tl.n = 0;
+            *tl.corr = 0.0;
+        }
         *out = t;
+    }
+}
+
+// One warp per near-tie row: recomputes |x - c|^2 of both candidates in fp64 from
+// the bf16 row and the bf16 operands (c = -q / 2, exact), keeps the smaller (the
+// lower index on an exact tie), writes the label (int32 and/or int64), and for a
+// relabelled row its distance and the change of the error sum. With cnt, also the
+// row's rank in its cluster (an atomic on the count), and the last-pass label.
+// The distance changes are fp32 differences added in fp64; with few, small terms
+// their sum does not depend on the order the atomics land in.
+__global__ void k_settle(TieList tl, const float* __restrict__ xn, const __nv_bfloat16* __restrict__ A, int ld,
+                         const __nv_bfloat16* __restrict__ cq, int32_t* __restrict__ labels32,
+                         int64_t* __restrict__ labels64, float* __restrict__ dists, int32_t* __restrict__ cnt,
+                         int32_t* __restrict__ rank, const int32_t* __restrict__ ids,
+                         int64_t* __restrict__ labels_last, int capture) {
+    const int lane = threadIdx.x & 31;
+    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int nwarps = (gridDim.x * blockDim.x) >> 5;
+    const int n = *tl.n;
+    const int nv = ld / 8;
+    for (int i = warp; i < n; i += nwarps) {
+        const int4 t = tl.e[i];
+        const int64_t r = t.x;
+        const uint32_t la = (uint32_t)t.y, lb = (uint32_t)t.z;
+        double da = 0.0, db = 0.0;
+        for (int v = lane; v < nv; v += 32) {
+            float x[8], qa[8], qb[8];
+            unpack8_bf16(reinterpret_cast<const uint4*>(A + r * ld)[v], x);
+            unpack8_bf16(reinterpret_cast<const uint4*>(cq + (int64_t)la * ld)[v], qa);
+            unpack8_bf16(reinterpret_cast<const uint4*>(cq + (int64_t)lb * ld)[v], qb);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const double ea = (double)x[u] + 0.5 * (double)qa[u];
+                const double eb = (double)x[u] + 0.5 * (double)qb[u];
+                da += ea * ea;
+                db += eb * eb;
+            }
+        }
+        da = warp_sum(da);
+        db = warp_sum(db);
+        if (lane == 0) {
+            const bool swap = db < da || (db == da && lb < la);
+            const int lab = (int)(swap ? lb : la);
+            if (swap) {
+                const float old = dists[r];
+                const float nd = fmaxf(0.0f, xn[r] + __int_as_float(t.w));
+                dists[r] = nd;
+                atomicAdd(tl.corr, (double)nd - (double)old);
+            }
+            if (labels32) labels32[r] = lab;
+            if (labels64) labels64[r] = (int64_t)lab;
+            if (cnt) rank[r] = atomicAdd(&cnt[lab], 1);
+            if (capture) labels_last[ids[r]] = lab;
+        }
     }
 }
 

@@ -429,13 +429,17 @@ class EmeansOracle:
         b = self.r["batch_size"]
         return self.order[self.pos:min(self.pos + b, rows)]
 
-    def step(self, forced_labels=None, auto_revive=True):
-        """One mini-batch: assign, per-cluster statistics, EMA, then revival if due."""
+    def step(self, forced_labels=None, auto_revive=True, stats=None):
+        """One mini-batch: assign, per-cluster statistics, EMA, then revival if due.
+
+        `stats`, if given, replaces the per-cluster statistics of the batch:
+        stats(rows, labels, k) -> (n_j, s_j). The data-parallel protocol uses it to
+        add the statistics of every rank's share of the batch."""
         ids = self.next_batch_ids()
         xb = self.xq[ids]
         labels, best, second = assign(xb, search_copy_of_centroids(self.c))
         used = labels if forced_labels is None else np.asarray(forced_labels, dtype=np.int64)
-        n_j, s_j = batch_stats(xb, used, self.k)
+        n_j, s_j = (batch_stats if stats is None else stats)(xb, used, self.k)
         alpha = alpha_at(self.t, self.r["total_steps"], self.r["alpha0"])
         self.N, self.S, self.c = ema_update(self.N, self.S, self.c, n_j, s_j, alpha)
         last_pass = self.pass_index == len(self.r["epoch_rows"]) - 1

@@ -1,0 +1,105 @@
+"""Data-parallel e-means on two CPU ranks (gloo), at the level of the oracle.
+
+The method shards by batch rows: every rank assigns its share of each mini-batch,
+computes the per-cluster counts and sums of its rows, the ranks add them with one
+all-reduce of k (d + 1) values, and every rank applies the same EMA update and the
+same revival check (the revival draws are keyed by seed, step and cluster, so no
+further exchange is needed). These tests check that protocol against the
+single-process oracle run, that the ranks stay bit-identical, and the bench's
+aggregation of timings and row counts over ranks.
+"""
+
+import datetime
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+from oracle import emeans_oracle as O
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _data(n=1200, d=12, comps=10, seed=3):
+    rng = np.random.default_rng(seed)
+    mu = rng.normal(0, 4.0, size=(comps, d))
+    x = mu[rng.integers(comps, size=n)] + rng.normal(size=(n, d))
+    return O.search_copy_of_data(x.astype(np.float32))
+
+
+def _init(rank, world, port):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+
+
+def _dp_worker(rank, world, port, out_dir, k, epochs, batch):
+    _init(rank, world, port)
+    try:
+        xq = _data()
+        orc = O.EmeansOracle(xq.shape[1], k, seed=5, batch_size=batch)
+        orc.begin(xq, epochs)
+
+        def shard_stats(rows, labels, kk):
+            # this rank's share of the batch, then one all-reduce of (n_j, s_j)
+            part = np.array_split(np.arange(len(rows)), world)[rank]
+            n_j, s_j = O.batch_stats(rows[part], labels[part], kk)
+            buf = torch.from_numpy(np.concatenate([n_j[:, None], s_j], axis=1))
+            dist.all_reduce(buf)
+            return buf[:, 0].numpy().copy(), buf[:, 1:].numpy().copy()
+
+        while not orc.done:
+            orc.step(stats=shard_stats)
+        c = orc.finalize()
+        np.save(os.path.join(out_dir, f"c{rank}.npy"), c)
+        np.save(os.path.join(out_dir, f"N{rank}.npy"), orc.N)
+        np.save(os.path.join(out_dir, f"splits{rank}.npy"), np.array([orc.n_splits]))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("k,epochs,batch", [(24, 2.0, 128), (40, 1.5, 96)])
+def test_data_parallel_step_matches_single_process(tmp_path, k, epochs, batch):
+    world = 2
+    mp.spawn(_dp_worker, args=(world, _free_port(), str(tmp_path), k, epochs, batch), nprocs=world, join=True)
+    c0, c1 = np.load(tmp_path / "c0.npy"), np.load(tmp_path / "c1.npy")
+    N0, N1 = np.load(tmp_path / "N0.npy"), np.load(tmp_path / "N1.npy")
+    # the ranks hold the same model, bit for bit
+    assert np.array_equal(c0, c1) and np.array_equal(N0, N1)
+    # and it is the single-process run up to the order of the fp64 sums
+    xq = _data()
+    ref = O.EmeansOracle(xq.shape[1], k, seed=5, batch_size=batch)
+    c_ref, _ = ref.train(xq, epochs)
+    np.testing.assert_allclose(c0, c_ref, rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(N0, ref.N, rtol=1e-12, atol=1e-12)
+    assert int(np.load(tmp_path / "splits0.npy")[0]) == ref.n_splits
+
+
+def _agg_worker(rank, world, port, out_dir):
+    _init(rank, world, port)
+    try:
+        import bench
+
+        ms, rows = (12.5, 1000) if rank == 0 else (17.25, 1500)
+        ms_max, rows_all = bench.reduce_over_ranks(ms, rows, torch.device("cpu"), world)
+        np.save(os.path.join(out_dir, f"agg{rank}.npy"), np.array([ms_max, rows_all]))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_bench_aggregates_max_time_and_total_rows(tmp_path):
+    world = 2
+    mp.spawn(_agg_worker, args=(world, _free_port(), str(tmp_path)), nprocs=world, join=True)
+    for r in range(world):
+        ms_max, rows_all = np.load(tmp_path / f"agg{r}.npy")
+        assert ms_max == 17.25 and rows_all == 2500
