@@ -428,6 +428,46 @@ static int launch_settle(em_model* m, const __nv_bfloat16* A, int32_t* labels32,
     return EM_OK;
 }
 
+// Every variant of the search kernel: KC (64 or 32 columns per K chunk), TOP2 (keep
+// the two best), AST (the batch tile stays in shared memory for a whole work unit;
+// rows of at most 128 dims).
+static bool ast_fits(int64_t d, int kc) {
+    const int64_t nkc = (d + kc - 1) / kc;
+    return nkc * tc::BM * kc * 2 <= tc::kAstBufBytes;
+}
+
+static void launch_search(int kc, bool top2, bool ast, int grid, cudaStream_t stream, const CUtensorMap& tmA,
+                          const CUtensorMap& tmB, const float* cn, int k, int rows, int nkc, int n_tiles, int split,
+                          unsigned long long* keys, long long wait, int* err) {
+#define EM_GO(KC, T2, AST)                                                                                       \
+    tc::k_assign_tc<KC, T2, AST><<<grid, tc::kThreads, tc::Cfg<KC, AST>::kSmemBytes, stream>>>(                \
+        tmA, tmB, cn, k, rows, nkc, n_tiles, split, keys, wait, err)
+    if (kc == 64) {
+        if (top2) {
+            if (ast) EM_GO(64, true, true); else EM_GO(64, true, false);
+        } else {
+            if (ast) EM_GO(64, false, true); else EM_GO(64, false, false);
+        }
+    } else {
+        if (top2) {
+            if (ast) EM_GO(32, true, true); else EM_GO(32, true, false);
+        } else {
+            if (ast) EM_GO(32, false, true); else EM_GO(32, false, false);
+        }
+    }
+#undef EM_GO
+}
+
+static bool search_smem_attributes() {
+#define EM_ATTR(KC, T2, AST)                                                                                \
+    (cudaFuncSetAttribute(tc::k_assign_tc<KC, T2, AST>, cudaFuncAttributeMaxDynamicSharedMemorySize,       \
+                          tc::Cfg<KC, AST>::kSmemBytes) == cudaSuccess)
+    return EM_ATTR(64, false, false) && EM_ATTR(64, true, false) && EM_ATTR(32, false, false) &&
+           EM_ATTR(32, true, false) && EM_ATTR(64, false, true) && EM_ATTR(64, true, true) &&
+           EM_ATTR(32, false, true) && EM_ATTR(32, true, true);
+#undef EM_ATTR
+}
+
 static int launch_assign(em_model* m, const CUtensorMap& tmA, const __nv_bfloat16* A, int64_t rows) {
     if (rows <= 0) return EM_OK;
     if (m->keys.cap < keys_needed(m, rows)) return fail(EM_E_STATE, "search key buffer too small");
@@ -446,21 +486,8 @@ static int launch_assign(em_model* m, const CUtensorMap& tmA, const __nv_bfloat1
     const int64_t units = m_tiles * split;
     const int grid = (int)std::min<int64_t>(units, m->sms);
     const bool top2 = use_top2(m);
-#define EM_ASSIGN(KC, T2)                                                                                           \
-    tc::k_assign_tc<KC, T2><<<grid, tc::kThreads, tc::Cfg<KC>::kSmemBytes, m->stream>>>(                           \
-        tmA, m->tm_cq, m->cn.p, (int)m->k, (int)rows, nkc, (int)n_tiles, split, m->keys.p, m->wait_cycles, m->err.p)
-    if (m->kc == 64) {
-        if (top2)
-            EM_ASSIGN(64, true);
-        else
-            EM_ASSIGN(64, false);
-    } else {
-        if (top2)
-            EM_ASSIGN(32, true);
-        else
-            EM_ASSIGN(32, false);
-    }
-#undef EM_ASSIGN
+    launch_search(m->kc, top2, ast_fits(m->d, m->kc), grid, m->stream, tmA, m->tm_cq, m->cn.p, (int)m->k, (int)rows,
+                  nkc, (int)n_tiles, split, m->keys.p, m->wait_cycles, m->err.p);
     CK(cudaGetLastError());
     EM_LAUNCHED(m, 1);
     m->last_split = split * tc::kKeySets;
@@ -478,10 +505,10 @@ static int launch_reduce(em_model* m, const __nv_bfloat16* src, int64_t rows, in
     k_scatter<<<(int)((rows + 255) / 256), 256, 0, m->stream>>>(m->labels.p, m->rank.p, m->off.p, m->poff.p,
                                                                  (int)rows, m->R, m->perm.p, m->items.p, m->err.p);
     CK(cudaGetLastError());
+    const ClusterState st = cluster_state(m);
     const int64_t max_items = m->k + (rows + m->R - 1) / m->R;
     const int nslices = (m->nv + 31) / 32;
-    const ClusterState st = cluster_state(m);
-    const int seg_blocks = (int)std::min<int64_t>((max_items * nslices * 32 + 255) / 256, (int64_t)m->sms * 2);
+    const int seg_blocks = (int)((max_items * nslices * 32 + 255) / 256);
     k_segsum<<<seg_blocks, 256, 0, m->stream>>>(src, m->perm.p, m->items.p, m->poff.p, nslices, m->nv, st, sp,
                                                 m->part.p);
     k_clusters<<<grid_for(m->k * 32, 256, m->sms), 256, 0, m->stream>>>(m->off.p, m->poff.p, m->cnt.p, m->R, nslices,
@@ -766,14 +793,7 @@ em_model* em_create(int64_t d, int64_t k, uint64_t seed) {
     cudaMemset(m->c.p, 0, kd * sizeof(float));
     cudaMemset(m->cq.p, 0, kd * sizeof(__nv_bfloat16));
     cudaMemset(m->cn.p, 0, k * sizeof(float));
-    if (cudaFuncSetAttribute(tc::k_assign_tc<64, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             tc::Cfg<64>::kSmemBytes) != cudaSuccess ||
-        cudaFuncSetAttribute(tc::k_assign_tc<32, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             tc::Cfg<32>::kSmemBytes) != cudaSuccess ||
-        cudaFuncSetAttribute(tc::k_assign_tc<64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             tc::Cfg<64>::kSmemBytes) != cudaSuccess ||
-        cudaFuncSetAttribute(tc::k_assign_tc<32, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             tc::Cfg<32>::kSmemBytes) != cudaSuccess ||
+    if (!search_smem_attributes() ||
         cudaFuncSetAttribute(k_revive_select, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kReviveSmemBytes) != cudaSuccess)
         return bail(EM_E_CUDA, "cudaFuncSetAttribute failed");
@@ -1349,15 +1369,7 @@ int noalloc_scratch(int dev, unsigned char** out) {
             cudaGetLastError();
             return fail(EM_E_CUDA, "cudaGetSymbolAddress of the scratch array failed: %s", cudaGetErrorString(e));
         }
-        if (cudaFuncSetAttribute(tc::k_assign_tc<64, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 tc::Cfg<64>::kSmemBytes) != cudaSuccess ||
-            cudaFuncSetAttribute(tc::k_assign_tc<32, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 tc::Cfg<32>::kSmemBytes) != cudaSuccess ||
-            cudaFuncSetAttribute(tc::k_assign_tc<64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 tc::Cfg<64>::kSmemBytes) != cudaSuccess ||
-            cudaFuncSetAttribute(tc::k_assign_tc<32, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 tc::Cfg<32>::kSmemBytes) != cudaSuccess)
-            return fail(EM_E_CUDA, "cudaFuncSetAttribute failed");
+        if (!search_smem_attributes()) return fail(EM_E_CUDA, "cudaFuncSetAttribute failed");
         g_na_base[dev] = static_cast<unsigned char*>(p);
     }
     *out = g_na_base[dev];
@@ -1411,21 +1423,8 @@ extern "C" int em_assign_noalloc(const void* X, int64_t n, int64_t d, const floa
     const bool top2 = d >= 256;
     const int grid = (int)std::min<int64_t>(m_tiles * split, sms);
     const long long wait_cycles = (long long)(2000.0 * (double)clock_khz);
-#define EM_NA_ASSIGN(KC, T2)                                                                       \
-    tc::k_assign_tc<KC, T2><<<grid, tc::kThreads, tc::Cfg<KC>::kSmemBytes, stream>>>( \
-        tmA, tmB, cn, (int)k, (int)n, nkc, (int)n_tiles, split, keys, wait_cycles, err)
-    if (kc == 64) {
-        if (top2)
-            EM_NA_ASSIGN(64, true);
-        else
-            EM_NA_ASSIGN(64, false);
-    } else {
-        if (top2)
-            EM_NA_ASSIGN(32, true);
-        else
-            EM_NA_ASSIGN(32, false);
-    }
-#undef EM_NA_ASSIGN
+    launch_search(kc, top2, ast_fits(d, kc), grid, static_cast<cudaStream_t>(stream), tmA, tmB, cn, (int)k, (int)n,
+                  nkc, (int)n_tiles, split, keys, wait_cycles, err);
     const int oblocks = std::min(grid_for(n, 256, sms), kNaMaxBlocks);
     k_assign_out<<<oblocks, 256, 0, stream>>>(keys, split * tc::kKeySets, xn, n, (int)k, X16, (int)d, cq, labels,
                                              dists, nullptr, blocks, TieList{nullptr, nullptr, nullptr}, err);

@@ -37,17 +37,25 @@ constexpr int kEpiThreads = 256;
 constexpr int kEpiWarps = 8;
 constexpr int kKeySets = 2;  // key sets per centroid-tile group (the two column halves)
 
-template <int KC>
+// AST ("A stationary", rows of at most 128 dims): the CTA keeps its 128-row tile of
+// the batch in shared memory for the whole work unit (two buffers, so that the
+// next unit's tile loads while this one is used) and streams only centroid tiles
+// through the ring: a third less traffic from L2 per tile.
+constexpr int kAstBufBytes = 32 * 1024;  // one A-stationary buffer: nkc * BM * KC * 2 bytes at most
+
+template <int KC, bool AST = false>
 struct Cfg {
-    static constexpr int kStages = KC == 64 ? 4 : 8;
     static constexpr int kABytes = BM * KC * 2;
     static constexpr int kBBytes = BN * KC * 2;
-    static constexpr int kStageBytes = kABytes + kBBytes;
+    static constexpr int kStageBytes = AST ? kBBytes : kABytes + kBBytes;
+    static constexpr int kStages = AST ? (128 * 1024) / kBBytes : (KC == 64 ? 4 : 8);
+    static constexpr int kAreaBytes = AST ? 2 * kAstBufBytes : 0;  // the A buffers, after the ring
     static constexpr uint64_t kLayout = KC == 64 ? 2ull : 4ull;  // UMMA 128B / 64B swizzle
     static constexpr uint32_t kSBO = 8u * KC * 2u;                // bytes between 8-row groups
     static constexpr int kBarBytes = 256;
     // + each epilogue warp's |c|^2 values of two tiles (its 128 columns)
-    static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kBarBytes + kEpiWarps * 2 * 128 * 4;
+    static constexpr int kSmemBytes =
+        1024 + kStages * kStageBytes + kAreaBytes + kBarBytes + kEpiWarps * 2 * 128 * 4;
 };
 
 // Instruction descriptor of tcgen05.mma kind::f16: fp32 accumulate (bits 4-5 = 1),
@@ -164,30 +172,79 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
 
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
+// One 32-column chunk of a row's scores: adds |c|^2 (c4: the chunk's 32 values) to
+// the raw accumulators v (in place) and updates the running best (TOP2: best two)
+// with the lowest column on ties. Without TOP2 the chunk's minimum is taken as a
+// tree (depth 5, not a chain of 31) and only a row it improves looks for the
+// lowest column that reaches it.
+template <bool TOP2>
+__device__ __forceinline__ void scan_chunk(uint32_t (&v)[32], const float4* c4, int jb, float& best, int& bidx,
+                                           float& best2, int& bidx2) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const float4 cc = c4[i];
+        v[4 * i + 0] = __float_as_uint(cc.x + __uint_as_float(v[4 * i + 0]));
+        v[4 * i + 1] = __float_as_uint(cc.y + __uint_as_float(v[4 * i + 1]));
+        v[4 * i + 2] = __float_as_uint(cc.z + __uint_as_float(v[4 * i + 2]));
+        v[4 * i + 3] = __float_as_uint(cc.w + __uint_as_float(v[4 * i + 3]));
+    }
+    if (TOP2) {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {  // branch-free: a divergent skip test measured slower
+            const float x = __uint_as_float(v[e]);
+            const bool p1 = x < best, p2 = x < best2;
+            best2 = p1 ? best : (p2 ? x : best2);
+            bidx2 = p1 ? bidx : (p2 ? jb + e : bidx2);
+            best = p1 ? x : best;
+            bidx = p1 ? jb + e : bidx;
+        }
+    } else {
+        float m8[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+            m8[e] = fminf(fminf(__uint_as_float(v[e]), __uint_as_float(v[e + 8])),
+                          fminf(__uint_as_float(v[e + 16]), __uint_as_float(v[e + 24])));
+#pragma unroll
+        for (int e = 0; e < 4; ++e) m8[e] = fminf(m8[e], m8[e + 4]);
+        const float mn = fminf(fminf(m8[0], m8[2]), fminf(m8[1], m8[3]));
+        if (mn < best) {
+            unsigned eq = 0;
+#pragma unroll
+            for (int e = 0; e < 32; ++e) eq |= (__uint_as_float(v[e]) == mn) ? (1u << e) : 0u;
+            best = mn;
+            bidx = jb + __ffs(eq) - 1;
+        }
+    }
+}
+
 // Output: for every row, column half h of the split g of the centroid tiles it
 // covers writes two keys at keys[((2 g + h) * rows + row) * 2 + {0, 1}]: the best
 // (score, index) and, with TOP2, the second best (without it the second key is
 // empty).
-template <int KC, bool TOP2>
+template <int KC, bool TOP2, bool AST>
 __global__ void __launch_bounds__(kThreads, 1)
     k_assign_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const float* __restrict__ cn, int k, int rows, int nkc, int n_tiles, int n_split,
                 unsigned long long* __restrict__ keys, long long wait_limit, int* err) {
-    using C = Cfg<KC>;
+    using C = Cfg<KC, AST>;
     constexpr int S = C::kStages;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // ring: (A, B) per stage, or B only with the A buffers after the ring (AST)
     uint8_t* sA = smem;
-    uint8_t* sB = smem + S * C::kABytes;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::kStageBytes);
+    uint8_t* sB = AST ? smem : smem + S * C::kABytes;
+    uint8_t* sArea = smem + S * C::kStageBytes;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::kStageBytes + C::kAreaBytes);
     uint64_t* full = bars;
     uint64_t* empty = bars + S;
     uint64_t* tfull = bars + 2 * S;
     uint64_t* tempty = bars + 2 * S + 2;
     uint64_t* drain = bars + 2 * S + 4;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 5);
+    uint64_t* afull = bars + 2 * S + 5;   // AST: A buffer loaded
+    uint64_t* aempty = bars + 2 * S + 7;  // AST: A buffer no longer read by the MMAs
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 9);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-    float* cn_s = reinterpret_cast<float*>(smem + S * C::kStageBytes + C::kBarBytes);
+    float* cn_s = reinterpret_cast<float*>(smem + S * C::kStageBytes + C::kAreaBytes + C::kBarBytes);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -207,6 +264,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(smem_u32(&tempty[a]), kEpiThreads);
         }
         mbar_init(smem_u32(drain), 1);
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(smem_u32(&afull[a]), 1);
+            mbar_init(smem_u32(&aempty[a]), 1);
+        }
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -233,9 +294,26 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t phase = 0;
             bool ok = true;
             uint32_t armed = 0, armed_parity = 0;  // per-stage bit masks
+            uint32_t aarmed = 0, aarmed_parity = 0;  // the two A buffers (AST)
+            int ua = 0;                              // units started (AST)
             for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
                 const int m = u / n_split, g = u - m * n_split;
                 const int nt0 = g * tpg, nt1 = min(nt0 + tpg, n_tiles);
+                if (AST) {  // the unit's rows, once, into A buffer ua % 2
+                    const int ab = ua & 1;
+                    const uint32_t par = (uint32_t)(ua >> 1) & 1u;
+                    if (!mbar_wait(smem_u32(&aempty[ab]), par ^ 1u, wait_limit, err, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t fb = smem_u32(&afull[ab]);
+                    aarmed |= 1u << ab;
+                    aarmed_parity = (aarmed_parity & ~(1u << ab)) | (par << ab);
+                    mbar_expect_tx(fb, (uint32_t)(nkc * C::kABytes));
+                    for (int kc = 0; kc < nkc; ++kc)
+                        tma_load_2d(smem_u32(sArea + ab * kAstBufBytes + kc * C::kABytes), &tmA, kc * KC, m * BM, fb);
+                    ++ua;
+                }
                 for (int nt = nt0; nt < nt1 && ok; ++nt) {
                     for (int kc = 0; kc < nkc; ++kc) {
                         if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, wait_limit, err, abort_flag)) {
@@ -246,7 +324,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         armed |= 1u << stage;
                         armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
                         mbar_expect_tx(fb, C::kStageBytes);
-                        tma_load_2d(smem_u32(sA + stage * C::kABytes), &tmA, kc * KC, m * BM, fb);
+                        if (!AST) tma_load_2d(smem_u32(sA + stage * C::kABytes), &tmA, kc * KC, m * BM, fb);
                         tma_load_2d(smem_u32(sB + stage * C::kBBytes), &tmB, kc * KC, nt * BN, fb);
                         if (++stage == S) {
                             stage = 0;
@@ -258,6 +336,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!ok) {  // let every copy this thread started land before shared memory is released
                 for (int s2 = 0; s2 < S; ++s2)
                     if (armed & (1u << s2)) mbar_drain(smem_u32(&full[s2]), (armed_parity >> s2) & 1u, drain_limit);
+                for (int a2 = 0; a2 < 2; ++a2)
+                    if (aarmed & (1u << a2)) mbar_drain(smem_u32(&afull[a2]), (aarmed_parity >> a2) & 1u, drain_limit);
             }
         }
     } else if (warp == 1) {
@@ -268,10 +348,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             int acc = 0;
             uint32_t acc_phase = 0;
             bool ok = true;
+            int ua = 0;
             for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
                 const int m = u / n_split, g = u - m * n_split;
                 (void)m;
                 const int nt0 = g * tpg, nt1 = min(nt0 + tpg, n_tiles);
+                const int ab = ua & 1;
+                if (AST) {
+                    if (!mbar_wait(smem_u32(&afull[ab]), (uint32_t)(ua >> 1) & 1u, wait_limit, err, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                }
                 for (int nt = nt0; nt < nt1 && ok; ++nt) {
                     if (!mbar_wait(smem_u32(&tempty[acc]), acc_phase ^ 1u, wait_limit, err, abort_flag)) {
                         ok = false;
@@ -285,7 +374,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                             break;
                         }
                         tc_fence_after();
-                        const uint32_t a0 = smem_u32(sA + stage * C::kABytes);
+                        const uint32_t a0 = AST ? smem_u32(sArea + ab * kAstBufBytes + kc * C::kABytes)
+                                                : smem_u32(sA + stage * C::kABytes);
                         const uint32_t b0 = smem_u32(sB + stage * C::kBBytes);
 #pragma unroll
                         for (int kk = 0; kk < KC / 16; ++kk) {
@@ -303,6 +393,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     umma_commit(smem_u32(&tfull[acc]));
                     acc ^= 1;
                     if (acc == 0) acc_phase ^= 1u;
+                }
+                if (AST && ok) {  // the unit's MMAs are issued: its A buffer frees once they complete
+                    umma_commit(smem_u32(&aempty[ab]));
+                    ++ua;
                 }
             }
             if (!ok) {  // wait for every MMA this thread issued before TMEM is freed
@@ -366,54 +460,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                 __syncwarp();  // also publishes this warp's |c|^2 values
                 const uint32_t tbase = tmem_base + lane_base + (uint32_t)(acc * BN + half * 128);
                 const float4* c4 = reinterpret_cast<const float4*>(cnb);
-                // two rounds of 64 columns (the register file allows no more per thread
-                // with ten warps: three of them share a sub-partition)
+                const int jh = j0 + half * 128;
+                // two rounds of 64 columns; the accumulator goes back once the second
+                // round is in registers (one round of 128 columns needs more registers
+                // than ten warps leave, and its spills made the kernel slower)
 #pragma unroll 1
                 for (int r = 0; r < 2; ++r) {
                     uint32_t v[2][32];
                     tmem_ld32(tbase + r * 64, v[0]);
                     tmem_ld32(tbase + r * 64 + 32, v[1]);
                     tmem_wait_ld();
-                    if (r == 1) {  // the values are in registers: hand the accumulator back
+                    if (r == 1) {
                         tc_fence_before();
                         mbar_arrive(smem_u32(&tempty[acc]));
                     }
 #pragma unroll
-                    for (int c = 0; c < 2; ++c) {
-                        float sc[32];
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            const float4 cc = c4[16 * r + 8 * c + i];
-                            sc[4 * i + 0] = cc.x + __uint_as_float(v[c][4 * i + 0]);
-                            sc[4 * i + 1] = cc.y + __uint_as_float(v[c][4 * i + 1]);
-                            sc[4 * i + 2] = cc.z + __uint_as_float(v[c][4 * i + 2]);
-                            sc[4 * i + 3] = cc.w + __uint_as_float(v[c][4 * i + 3]);
-                        }
-                        const int jb = j0 + half * 128 + 64 * r + 32 * c;
-                        if (TOP2) {
-#pragma unroll
-                            for (int e = 0; e < 32; ++e) {  // branch-free: a divergent skip test measured slower
-                                const bool p1 = sc[e] < best, p2 = sc[e] < best2;
-                                best2 = p1 ? best : (p2 ? sc[e] : best2);
-                                bidx2 = p1 ? bidx : (p2 ? jb + e : bidx2);
-                                best = p1 ? sc[e] : best;
-                                bidx = p1 ? jb + e : bidx;
-                            }
-                        } else {
-                            // the chunk minimum first; only a row it improves looks for the
-                            // lowest column that reaches it
-                            float mn = sc[0];
-#pragma unroll
-                            for (int e = 1; e < 32; ++e) mn = fminf(mn, sc[e]);
-                            if (mn < best) {
-                                int first = 31;
-#pragma unroll
-                                for (int e = 30; e >= 0; --e) first = (sc[e] == mn) ? e : first;
-                                best = mn;
-                                bidx = jb + first;
-                            }
-                        }
-                    }
+                    for (int c = 0; c < 2; ++c)
+                        scan_chunk<TOP2>(v[c], c4 + 16 * r + 8 * c, jh + 64 * r + 32 * c, best, bidx, best2, bidx2);
                 }
                 acc ^= 1;
                 if (acc == 0) acc_phase ^= 1u;

@@ -357,31 +357,31 @@ __device__ __forceinline__ SliceGeom slice_geom(int slice, int nv) {
 // Rows per work item of the grouped update (one chunk of a cluster).
 constexpr int kChunkRows = 64;
 
-// Sum over the n (at most kChunkRows) rows of a chunk of this lane's vector, fp64.
-// The chunk's row ids come preloaded, two per lane (pa: rows 0..31, pb: rows
-// 32..63), and are handed out by shuffles; eight rows are in flight per lane. The warp's row groups are folded together at the
-// end with a fixed butterfly, so lanes l < lpr hold the slice totals of vector
-// vbase + l.
-__device__ __forceinline__ void sum_rows(double acc[8], const __nv_bfloat16* __restrict__ src, int ld, int pa, int pb,
-                                         int n, const SliceGeom& g, int lane) {
+// Sum over rows perm[s0..s1) of this lane's vector, fp64, four rows in flight per
+// lane (each row id is a broadcast load that the first row group brings into L1;
+// preloading the chunk's ids and handing them out by shuffles measured slower).
+// The warp's row groups are folded together at the end with a fixed butterfly, so
+// lanes l < lpr hold the slice totals of vector vbase + l.
+template <int RIF = 4>
+__device__ __forceinline__ void sum_rows(double acc[8], const __nv_bfloat16* __restrict__ src, int ld,
+                                         const int32_t* __restrict__ perm, int s0, int s1, const SliceGeom& g,
+                                         int lane) {
 #pragma unroll
     for (int t = 0; t < 8; ++t) acc[t] = 0.0;
     const int sub = lane / g.lpr, vi = lane % g.lpr;
     const bool vec_ok = vi < g.nvs;
     const int v = g.vbase + vi;
-    for (int s = 0; s < n; s += 8 * g.rpi) {
-        uint4 u[8];
-        bool have[8];
+    for (int s = s0; s < s1; s += RIF * g.rpi) {
+        uint4 u[RIF];
+        bool have[RIF];
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-            const int idx = s + q * g.rpi + sub;
-            const int ra = __shfl_sync(0xFFFFFFFFu, pa, idx & 31);
-            const int rb = __shfl_sync(0xFFFFFFFFu, pb, idx & 31);
-            have[q] = vec_ok && idx < n;
-            if (have[q]) u[q] = reinterpret_cast<const uint4*>(src + (int64_t)(idx < 32 ? ra : rb) * ld)[v];
+        for (int q = 0; q < RIF; ++q) {
+            const int slot = s + q * g.rpi + sub;
+            have[q] = vec_ok && slot < s1;
+            if (have[q]) u[q] = reinterpret_cast<const uint4*>(src + (int64_t)perm[slot] * ld)[v];
         }
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
+        for (int q = 0; q < RIF; ++q) {
             if (have[q]) {
                 float x[8];
                 unpack8_bf16(u[q], x);
@@ -441,71 +441,38 @@ __device__ __forceinline__ float ema_slice(const ClusterState& st, int j, double
     return cn_part;
 }
 
-// Persistent warps over the (work item, slice) units. A work item is a chunk of
-// at most R label-sorted rows of one cluster. A cluster that fits in one chunk is
-// updated here; the chunks of a larger cluster leave their slice sums in
-// part[item] for k_clusters. Software pipeline: while a unit's rows load and add,
-// the warp already holds the next unit's item and fetches its row ids, S slice and
-// previous count, and the item after that, so that a unit costs about one memory
-// round trip instead of the chain item -> row ids -> rows.
-__global__ void __launch_bounds__(256, 2) k_segsum(const __nv_bfloat16* __restrict__ src,
+// One warp per (work item, slice). A work item is a chunk of at most R label-sorted
+// rows of one cluster, and carries (cluster, first row, end row, whether the
+// cluster fits in one chunk), so that the row ids, the S slice and the previous
+// count are all fetched right after the item. A
+// cluster that fits in one chunk is updated here; the chunks of a larger cluster
+// leave their slice sums in part[item] for k_clusters.
+__global__ void __launch_bounds__(256, 3) k_segsum(const __nv_bfloat16* __restrict__ src,
                                                    const int32_t* __restrict__ perm, const int4* __restrict__ items,
                                                    const int32_t* __restrict__ poff, int nslices, int nv,
                                                    ClusterState st, StepParams sp, double* __restrict__ part) {
     const int lane = threadIdx.x & 31;
-    const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    const int nw = (gridDim.x * blockDim.x) >> 5;
-    const int nunits = poff[st.k] * nslices;
-    auto item_of = [&](int u) { return u < nunits ? items[u / nslices] : make_int4(0, 0, 0, 0); };
-    auto ids_of = [&](const int4& it, int u, int& pa, int& pb) {
-        const int n = it.z - it.y;
-        pa = (u < nunits && lane < n) ? perm[it.y + lane] : 0;
-        pb = (u < nunits && lane + 32 < n) ? perm[it.y + 32 + lane] : 0;
-    };
-    auto state_of = [&](const int4& it, int u, float so[8], float& np) {
-        np = 0.0f;
-        if (u < nunits && it.w) {
-            load_s(st, it.x, slice_geom(u % nslices, nv), lane, so);
-            np = st.N_prev[it.x];
-        }
-    };
-    int u = gw;
-    int4 it = item_of(u);
-    int pa, pb;
-    ids_of(it, u, pa, pb);
-    float so[8], np;
-    state_of(it, u, so, np);
-    int4 itn = item_of(u + nw);
-    for (; u < nunits; u += nw) {
-        const int un = u + nw;
-        // next unit: row ids, S slice and count (its item arrived during the last unit)
-        int pan, pbn;
-        ids_of(itn, un, pan, pbn);
-        float son[8], npn;
-        state_of(itn, un, son, npn);
-        const int4 itnn = item_of(un + nw);
-        // this unit
-        const int slice = u % nslices;
-        const SliceGeom g = slice_geom(slice, nv);
-        const int j = it.x;
-        double acc[8];
-        sum_rows(acc, src, st.ld, pa, pb, it.z - it.y, g, lane);
-        if (it.w) {
-            const double nj = (double)(it.z - it.y);
-            const float cn_part = ema_slice(st, j, nj, np, slice, g, acc, so, lane, sp.alpha, sp.last_pass);
-            if (lane == 0) st.cnp[(int64_t)slice * st.k + j] = cn_part;
-        } else if (lane < g.nvs) {
-            double* dst = part + (int64_t)(u / nslices) * st.ld + 8 * (g.vbase + lane);
+    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int item = warp / nslices, slice = warp - item * nslices;
+    if (item >= poff[st.k]) return;
+    const int4 it = items[item];
+    const int j = it.x, n = it.z - it.y;
+    const SliceGeom g = slice_geom(slice, nv);
+    float so[8];
+    float nprev = 0.0f;
+    if (it.w) {
+        load_s(st, j, g, lane, so);
+        nprev = st.N_prev[j];
+    }
+    double acc[8];
+    sum_rows(acc, src, st.ld, perm, it.y, it.z, g, lane);
+    if (it.w) {
+        const float cn_part = ema_slice(st, j, (double)n, nprev, slice, g, acc, so, lane, sp.alpha, sp.last_pass);
+        if (lane == 0) st.cnp[(int64_t)slice * st.k + j] = cn_part;
+    } else if (lane < g.nvs) {
+        double* dst = part + (int64_t)item * st.ld + 8 * (g.vbase + lane);
 #pragma unroll
-            for (int t = 0; t < 8; ++t) dst[t] = acc[t];
-        }
-        it = itn;
-        pa = pan;
-        pb = pbn;
-#pragma unroll
-        for (int t = 0; t < 8; ++t) so[t] = son[t];
-        np = npn;
-        itn = itnn;
+        for (int t = 0; t < 8; ++t) dst[t] = acc[t];
     }
 }
 

@@ -134,10 +134,6 @@ __device__ __forceinline__ void group_scan(double v[4], int lane) {
     for (int i = 0; i < 4; ++i) v[i] += ex;
 }
 
-__device__ __forceinline__ double pick4(const double v[4], int i) {
-    return i == 0 ? v[0] : (i == 1 ? v[1] : (i == 2 ? v[2] : v[3]));
-}
-
 // Unbiased binary exponent of a positive finite double (subnormals included),
 // from the IEEE 754 encoding.
 __device__ __forceinline__ int exponent_of(double x) {
@@ -150,31 +146,75 @@ __device__ __forceinline__ int exponent_of(double x) {
 
 // One step of the descent inside a group whose four prefix values this lane holds.
 // Returns the child position (0..127) and, in *before / *w, the within-group
-// prefix before it and its weight. `last`: the target fell on the total, take the
-// last child with positive weight (the first position that reaches the group total).
+// prefix before it and its weight (*w only when want_w). `last`: the target fell
+// on the total, take the last child with positive weight (the first position that
+// reaches the group total). Written without branches: the fallback mask is formed
+// alongside the normal one and the ballot picks, and lane L (the lane holding the
+// chosen child) selects its values from differences computed before the ballot.
+template <bool want_w>
 __device__ __forceinline__ int group_select(const double P[4], double base, double t, bool last, int lane,
                                             double* before, double* w) {
     const double prev3 = __shfl_up_sync(0xFFFFFFFFu, P[3], 1);
+    const double tot = __shfl_sync(0xFFFFFFFFu, P[3], 31);
     const double Pprev = lane ? prev3 : 0.0;
-    unsigned m4 = 0;
-    if (!last) {
+    unsigned mt = 0, mf = 0;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) m4 |= (base + P[i] > t) ? (1u << i) : 0u;
+    for (int i = 0; i < 4; ++i) {
+        mt |= (base + P[i] > t) ? (1u << i) : 0u;
+        mf |= (P[i] >= tot) ? (1u << i) : 0u;
     }
-    unsigned bal = __ballot_sync(0xFFFFFFFFu, m4 != 0);
-    if (!bal) {  // target on (or, never in exact arithmetic, past) the total
-        const double tot = __shfl_sync(0xFFFFFFFFu, P[3], 31);
-        m4 = 0;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) m4 |= (P[i] >= tot) ? (1u << i) : 0u;
-        bal = __ballot_sync(0xFFFFFFFFu, m4 != 0);
-    }
+    const unsigned bt = __ballot_sync(0xFFFFFFFFu, mt != 0);
+    const unsigned bf = __ballot_sync(0xFFFFFFFFu, mf != 0);
+    // never empty in exact arithmetic unless the target is on the total
+    const bool use_t = !last && bt != 0;
+    const unsigned bal = use_t ? bt : bf;
+    const unsigned m4 = use_t ? mt : mf;
     const int L = __ffs(bal) - 1;
     const int sub = m4 ? __ffs(m4) - 1 : 0;
-    const double b = sub ? pick4(P, sub - 1) : Pprev;
-    const double wl = pick4(P, sub) - b;
+    // prefix before each of the lane's positions, then the one at `sub`
+    const double b = sub == 0 ? Pprev : (sub == 1 ? P[0] : (sub == 2 ? P[1] : P[2]));
     const int s = __shfl_sync(0xFFFFFFFFu, sub, L);
     *before = __shfl_sync(0xFFFFFFFFu, b, L);
+    if (want_w) {
+        const double wl = (sub == 0 ? P[0] : (sub == 1 ? P[1] : (sub == 2 ? P[2] : P[3]))) - b;
+        *w = __shfl_sync(0xFFFFFFFFu, wl, L);
+    }
+    return 4 * L + s;
+}
+
+// The lean select of the two-level draw: the lane masks of `base + P > t`, one
+// ballot, and the chosen lane's values. Returns -1 when no position exceeds the
+// target (the target fell on the total: the caller takes the fallback).
+__device__ __forceinline__ int select_gt(const double P[4], double Pprev, double base, double t, int lane,
+                                         double* before, double* w) {
+    unsigned mt = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) mt |= (base + P[i] > t) ? (1u << i) : 0u;
+    const unsigned bal = __ballot_sync(0xFFFFFFFFu, mt != 0);
+    if (!bal) return -1;
+    const int L = __ffs(bal) - 1;
+    const int sub = mt ? __ffs(mt) - 1 : 0;
+    const double b = sub == 0 ? Pprev : (sub == 1 ? P[0] : (sub == 2 ? P[1] : P[2]));
+    const double wl = (sub == 0 ? P[0] : (sub == 1 ? P[1] : (sub == 2 ? P[2] : P[3]))) - b;
+    const int s = __shfl_sync(0xFFFFFFFFu, sub, L);
+    *before = __shfl_sync(0xFFFFFFFFu, b, L);
+    *w = __shfl_sync(0xFFFFFFFFu, wl, L);
+    return 4 * L + s;
+}
+
+// The last position of a group whose weight is positive (the first position that
+// reaches the group total), with its weight.
+__device__ __forceinline__ int select_last(const double P[4], double Pprev, int lane, double* w) {
+    const double tot = __shfl_sync(0xFFFFFFFFu, P[3], 31);
+    unsigned mf = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) mf |= (P[i] >= tot) ? (1u << i) : 0u;
+    const unsigned bal = __ballot_sync(0xFFFFFFFFu, mf != 0);
+    const int L = __ffs(bal) - 1;
+    const int sub = mf ? __ffs(mf) - 1 : 0;
+    const double b = sub == 0 ? Pprev : (sub == 1 ? P[0] : (sub == 2 ? P[1] : P[2]));
+    const double wl = (sub == 0 ? P[0] : (sub == 1 ? P[1] : (sub == 2 ? P[2] : P[3]))) - b;
+    const int s = __shfl_sync(0xFFFFFFFFu, sub, L);
     *w = __shfl_sync(0xFFFFFFFFu, wl, L);
     return 4 * L + s;
 }
@@ -312,7 +352,77 @@ __global__ void __launch_bounds__(kSelectThreads) k_revive_select(const float* _
         double W = __shfl_sync(0xFFFFFFFFu, T[3], 31);
         int64_t splits = 0;
         int i_end = nd;  // draws from i_end on get no donor (no weight left)
-        for (int i0 = 0; i0 < nd; i0 += 32) {
+        // two levels (k <= 16384): the top group in registers, level 0 in shared memory
+        const bool two_level = top == 1 && L.smem_from == 0;
+        double* lev0 = smem_d + kRadix;
+        double Tprev = __shfl_up_sync(0xFFFFFFFFu, T[3], 1);
+        if (lane == 0) Tprev = 0.0;
+        for (int i0 = 0; two_level && i0 < nd; i0 += 32) {
+            const int cnt = min(32, nd - i0);
+            const double my_u = lane < cnt ? sc.target[i0 + lane] : 0.0;
+            int my_dn = -1;
+            for (int q = 0; q < cnt; ++q) {
+                if (!(W > 0.0)) {
+                    i_end = i0 + q;
+                    break;
+                }
+                const double tg = __shfl_sync(0xFFFFFFFFu, my_u, q) * W;
+                double before, wsel;
+                int g = select_gt(T, Tprev, 0.0, tg, lane, &before, &wsel);
+                double P[4];
+                int pos;
+                if (g >= 0) {
+                    const double2* sp = reinterpret_cast<const double2*>(lev0 + g * kRadix + 4 * lane);
+                    const double2 a = sp[0], b = sp[1];
+                    P[0] = a.x; P[1] = a.y; P[2] = b.x; P[3] = b.y;
+                    double Pprev = __shfl_up_sync(0xFFFFFFFFu, P[3], 1);
+                    if (lane == 0) Pprev = 0.0;
+                    double b0;
+                    pos = select_gt(P, Pprev, before, tg, lane, &b0, &wsel);
+                    if (pos < 0) pos = select_last(P, Pprev, lane, &wsel);  // (exact sums: never)
+                } else {  // the target fell on the total: the last cluster with weight
+                    g = select_last(T, Tprev, lane, &wsel);
+                    const double2* sp = reinterpret_cast<const double2*>(lev0 + g * kRadix + 4 * lane);
+                    const double2 a = sp[0], b = sp[1];
+                    P[0] = a.x; P[1] = a.y; P[2] = b.x; P[3] = b.y;
+                    double Pprev = __shfl_up_sync(0xFFFFFFFFu, P[3], 1);
+                    if (lane == 0) Pprev = 0.0;
+                    pos = select_last(P, Pprev, lane, &wsel);
+                }
+                // the donor keeps the rounded half of its weight (explicit roundings: see below)
+                const double keep = __dmul_rn(0.5, wsel);
+                const double delta = __dsub_rn(wsel, keep);
+                if (group_sub(P, pos, delta, lane)) {
+                    double2* sp = reinterpret_cast<double2*>(lev0 + g * kRadix + 4 * lane);
+                    sp[0] = make_double2(P[0], P[1]);
+                    sp[1] = make_double2(P[2], P[3]);
+                }
+                group_sub(T, g, delta, lane);
+                Tprev = __shfl_up_sync(0xFFFFFFFFu, T[3], 1);
+                if (lane == 0) Tprev = 0.0;
+                W -= delta;
+                if (lane == q) my_dn = g * kRadix + pos;
+            }
+            const bool has = lane < cnt && my_dn >= 0;
+            const unsigned peers = __match_any_sync(0xFFFFFFFFu, has ? my_dn : -1);
+            const int leader = __ffs(peers) - 1;
+            int old = 0;
+            if (has && lane == leader) old = times[my_dn];
+            old = __shfl_sync(0xFFFFFFFFu, old, leader);
+            if (has) {
+                const int rk = __popc(peers & ((1u << lane) - 1u));
+                sc.donor[i0 + lane] = my_dn;
+                sc.order[i0 + lane] = old + rk;
+                if (lane == leader) times[my_dn] = old + __popc(peers);
+            } else if (lane < cnt) {
+                sc.donor[i0 + lane] = -1;
+            }
+            splits += __popc(__ballot_sync(0xFFFFFFFFu, has));
+            __syncwarp();  // the counters written above are read by other lanes next batch
+            if (i_end < nd) break;
+        }
+        // deeper trees or global levels: one group per level, any depth
+        for (int i0 = 0; !two_level && i0 < nd; i0 += 32) {
             const int cnt = min(32, nd - i0);
             const double my_u = lane < cnt ? sc.target[i0 + lane] : 0.0;
             int my_dn = -1;
@@ -323,8 +433,10 @@ __global__ void __launch_bounds__(kSelectThreads) k_revive_select(const float* _
                 }
                 const double tg = __shfl_sync(0xFFFFFFFFu, my_u, q) * W;
                 const bool last = !(tg < W);
-                double before, wsel;
-                int node = group_select(T, 0.0, tg, last, lane, &before, &wsel);
+                double before, wsel = 0.0;
+                // (the weight is needed from the top group only when it is the leaf level)
+                int node = top == 0 ? group_select<true>(T, 0.0, tg, last, lane, &before, &wsel)
+                                    : group_select<false>(T, 0.0, tg, last, lane, &before, &wsel);
                 double base = before;
                 const int node_top = node;
                 int nodes[kTreeLevels - 1];
@@ -345,7 +457,8 @@ __global__ void __launch_bounds__(kSelectThreads) k_revive_select(const float* _
                             b = s[1];
                         }
                         P[l][0] = a.x; P[l][1] = a.y; P[l][2] = b.x; P[l][3] = b.y;
-                        const int c = group_select(P[l], base, tg, last, lane, &before, &wsel);
+                        const int c = l == 0 ? group_select<true>(P[l], base, tg, last, lane, &before, &wsel)
+                                             : group_select<false>(P[l], base, tg, last, lane, &before, &wsel);
                         base += before;
                         node = node * kRadix + c;
                         nodes[l] = node;
