@@ -250,7 +250,8 @@ def run_ours(args, rank, world):
     peak = peaks["bf16_tflops"]
     out["roofline"] = {
         "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-        "frac": achieved / peak, "traffic": args.traffic,
+        "frac": achieved / peak,
+        "traffic": args.traffic if args.traffic is not None else ASSIGN_TRAFFIC.get(args.workload),
         "kernel": "k_assign_tc (tcgen05 bf16 x bf16 -> fp32, fused |c|^2 add + row argmin)",
         "peak_source": f"{peaks['source']} bf16 burst",
         "frac_of_sustained": achieved / peaks["bf16_tflops_sustained"] if peaks.get("bf16_tflops_sustained") else None,
@@ -466,8 +467,9 @@ def run_kernel_case(args):
 
 def run_ablation(args):
     """Revival ablation on one workload: split, resample and none over several
-    seeds. Dead clusters are those that receive no training row in a full
-    assignment pass with the final centroids; test MSE with the same centroids."""
+    seeds. After training, a full assignment pass of the training rows counts each
+    cluster's rows: unused clusters hold fewer than a tenth of the mean count;
+    test MSE with the same centroids."""
     import torch
 
     import datagen
@@ -484,13 +486,26 @@ def run_ablation(args):
             m.set_option("input_dtype", 1 if w.storage == "bf16" else 0)
             m.train(xt, epochs=w.epochs)
             m.assign(xt, labels=labels)
-            dead = int((torch.bincount(labels, minlength=w.k) == 0).sum().item())
-            rows.append({"seed": seed, "dead": dead, "test_mse": m.mse(xs), "splits": m.stats()["n_splits"]})
+            cnt = torch.bincount(labels, minlength=w.k)
+            # unused: fewer rows than a tenth of the mean (the revival criterion);
+            # empty: no row at all (a cluster never revived keeps its starting row,
+            # which it always wins, so this one rarely moves)
+            unused = int((cnt.double() < 0.1 * cnt.double().mean()).sum().item())
+            empty = int((cnt == 0).sum().item())
+            rows.append({"seed": seed, "unused": unused, "empty": empty, "test_mse": m.mse(xs),
+                         "splits": m.stats()["n_splits"]})
             m.close()
             log(f"[ablation] {mode} seed {seed}: {rows[-1]}")
-        out["modes"][mode] = {"runs": rows, "dead_mean": statistics.mean(r["dead"] for r in rows),
+        out["modes"][mode] = {"runs": rows, "unused_mean": statistics.mean(r["unused"] for r in rows),
+                              "empty_mean": statistics.mean(r["empty"] for r in rows),
                               "test_mse_mean": statistics.mean(r["test_mse"] for r in rows)}
     return out
+
+
+# DRAM bytes per assignment launch of the bench's batch, from an ncu capture of the
+# current kernel (profiles/k_assign_tc_emb768_262144rows.md: 262,144 rows, scaled
+# to one 65,536-row batch with the centroid operand counted once).
+ASSIGN_TRAFFIC = {"emb768": 109.7e6}
 
 
 def main():
