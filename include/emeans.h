@@ -53,11 +53,15 @@ enum em_option {
                                     and alpha0 follows equation (3) (README "Manual overrides") */
     EM_OPT_ALPHA0 = 2,           /* 0 (default): from equation (3); else the starting step    */
     EM_OPT_UNUSED_THRESHOLD = 3, /* tau: revive clusters whose running count is below tau x the
-                                    mean count (README `unused_threshold`). Default 0.1; 0 = off */
+                                    mean count (README `unused_threshold`). 0 = off; -1
+                                    (default): 0.1, or 0 for d <= 2 (README "Note on low
+                                    dimension")                                              */
     EM_OPT_REVIVAL = 4,          /* 0 none, 1 split a size-proportional donor (default),
                                     2 resample from the current batch                          */
     EM_OPT_FINALIZE = 5,         /* 1 (default): closing mean at the end of the last pass; 0 off */
-    EM_OPT_LAW = 6,              /* 0 "throughput" law (1), default; 1 "quality" law (2)       */
+    EM_OPT_LAW = 6,              /* 0 "throughput" law (1); 1 "quality" law (2); 2 "auto"
+                                    (default): quality for d <= 16, else throughput (README
+                                    `batch_law`, "Note on low dimension")                      */
     EM_OPT_INPUT_DTYPE = 7,      /* dtype of X: 0 fp32 (default), 1 bf16                       */
     EM_OPT_CHECK_FINITE = 8,     /* 1: scan X for NaN/Inf in em_begin/em_train (EM_E_NONFINITE) */
     EM_OPT_WAIT_LIMIT_MS = 9,    /* limit of every device-side spin wait, ms (default 2000)    */

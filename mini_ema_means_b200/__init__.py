@@ -220,7 +220,7 @@ class Model:
         if name == "revival" and isinstance(value, str):
             value = REVIVAL_MODES[value]
         if name == "law" and isinstance(value, str):
-            value = {"throughput": 0, "quality": 1}[value]
+            value = {"throughput": 0, "quality": 1, "auto": 2}[value]
         if name == "input_dtype" and not isinstance(value, (int, float)):
             value = 1 if "bfloat16" in str(value) or str(value) == "bf16" else 0
         check(em_set_option(self.h, self._OPTS[name], float(value)), f"em_set_option({name})")

@@ -179,8 +179,8 @@ struct em_model {
     uint64_t seed = 1234;
     // options
     int64_t opt_batch = 0;
-    double opt_alpha0 = 0.0, tau = 0.1, wait_ms = 2000.0;
-    int revival = EM_REVIVE_SPLIT, finalize = 1, law = 0, in_dtype = 0, check_finite = 0;
+    double opt_alpha0 = 0.0, tau = -1.0, wait_ms = 2000.0;  // tau < 0: the default for d
+    int revival = EM_REVIVE_SPLIT, finalize = 1, law = 2, in_dtype = 0, check_finite = 0;
     int auto_revive = 1, capture = 1, graphs = 1, assign_kernel = 0, exact_ties = -1;
     int last_split = 1;  // centroid-tile groups of the most recent search (keys per row)
     // state
@@ -531,12 +531,19 @@ static ReviveScratch revive_scratch(em_model* m) {
     return sc;
 }
 
+// The defaults that depend on the dimension (README `batch_law`, `unused_threshold`
+// and "Note on low dimension"): the quality batch law for d <= 16, no revival for
+// d <= 2.
+static int effective_law(const em_model* m) { return m->law == 2 ? (m->d <= 16 ? 1 : 0) : m->law; }
+static double effective_tau(const em_model* m) { return m->tau < 0.0 ? (m->d <= 2 ? 0.0 : 0.1) : m->tau; }
+
 static int launch_revive(em_model* m, int64_t t, int64_t rows) {
-    if (m->revival == EM_REVIVE_NONE || !(m->tau > 0.0)) return EM_OK;
+    if (m->revival == EM_REVIVE_NONE || !(effective_tau(m) > 0.0)) return EM_OK;
     const ReviveScratch sc = revive_scratch(m);
     const TreeLayout L = tree_layout((int)m->k);
     const int smem = (int)tree_smem_bytes(L, (int)m->k);
-    k_revive_select<<<1, kSelectThreads, smem, m->stream>>>(m->N.p, (int)m->k, m->tau, m->seed, t, m->revival, sc, m->err.p);
+    k_revive_select<<<1, kSelectThreads, smem, m->stream>>>(m->N.p, (int)m->k, effective_tau(m), m->seed, t,
+                                                            m->revival, sc, m->err.p);
     CK(cudaGetLastError());
     const ClusterState st = cluster_state(m);
     const int blocks = grid_for(m->k * 32, 256, m->sms);
@@ -843,7 +850,7 @@ int em_set_option(em_model* m, int opt, double v) {
             m->opt_alpha0 = v;
             break;
         case EM_OPT_UNUSED_THRESHOLD:
-            if (!(v >= 0) || v > 1) return fail(EM_E_INVAL, "threshold must be in [0, 1]");
+            if (v != -1 && (!(v >= 0) || v > 1)) return fail(EM_E_INVAL, "threshold must be in [0, 1], or -1");
             m->tau = v;
             break;
         case EM_OPT_REVIVAL:
@@ -852,7 +859,7 @@ int em_set_option(em_model* m, int opt, double v) {
             break;
         case EM_OPT_FINALIZE: m->finalize = v != 0; break;
         case EM_OPT_LAW:
-            if (v != 0 && v != 1) return fail(EM_E_INVAL, "law is 0 or 1");
+            if (v != 0 && v != 1 && v != 2) return fail(EM_E_INVAL, "law is 0, 1 or 2");
             m->law = (int)v;
             break;
         case EM_OPT_INPUT_DTYPE:
@@ -924,7 +931,7 @@ int em_begin(em_model* m, const void* X, int64_t n, double epochs) {
     if (n >= (1ll << 31)) return fail(EM_E_INVAL, "n must be below 2^31");
     if (!(epochs > 0.0)) return fail(EM_E_INVAL, "epochs must be positive");
     CKR(set_device(m));
-    CKR(compute_recipe(n, m->k, m->d, epochs, m->law, m->opt_batch, m->opt_alpha0, &m->rec));
+    CKR(compute_recipe(n, m->k, m->d, epochs, effective_law(m), m->opt_batch, m->opt_alpha0, &m->rec));
     if (m->rec.batch_size > n) return fail(EM_E_INVAL, "batch size larger than n");
     m->running = false;
     m->n = n;

@@ -48,7 +48,8 @@ struct Cfg {
     static constexpr int kABytes = BM * KC * 2;
     static constexpr int kBBytes = BN * KC * 2;
     static constexpr int kStageBytes = AST ? kBBytes : kABytes + kBBytes;
-    static constexpr int kStages = AST ? (128 * 1024) / kBBytes : (KC == 64 ? 4 : 8);
+    // (A stationary: 9 stages of 16 KB or 4 of 32 KB fit beside the two A buffers)
+    static constexpr int kStages = AST ? (KC == 32 ? 9 : 4) : (KC == 64 ? 4 : 8);
     static constexpr int kAreaBytes = AST ? 2 * kAstBufBytes : 0;  // the A buffers, after the ring
     static constexpr uint64_t kLayout = KC == 64 ? 2ull : 4ull;  // UMMA 128B / 64B swizzle
     static constexpr uint32_t kSBO = 8u * KC * 2u;                // bytes between 8-row groups

@@ -302,6 +302,47 @@ def mse(xq: np.ndarray, c64: np.ndarray) -> float:
 
 
 # --------------------------------------------------------------------------
+# Spherical e-means ([README] "Spherical e-means"): centroids rescaled to norm 1
+# before every use, the highest dot product wins, error 2 - 2 x similarity
+# --------------------------------------------------------------------------
+
+def unit_rows(c: np.ndarray) -> np.ndarray:
+    """Each row rescaled to norm 1; a zero row stays zero."""
+    nrm = np.sqrt(np.einsum("ij,ij->i", c, c))
+    out = np.array(c, dtype=np.float64, copy=True)
+    nz = nrm > 0
+    out[nz] = out[nz] / nrm[nz][:, None]
+    return out
+
+
+def assign_dot(xq: np.ndarray, cq: np.ndarray, chunk: int = 4096):
+    """Centroid with the highest dot product with each row (search copies). Returns
+    (labels, best, second): the two highest dot products; ties go to the lowest
+    centroid index."""
+    n = xq.shape[0]
+    labels = np.empty(n, dtype=np.int64)
+    best = np.empty(n)
+    second = np.full(n, -np.inf)
+    for s in range(0, n, chunk):
+        neg = -(xq[s:s + chunk] @ cq.T)
+        lab = np.argmin(neg, axis=1)
+        labels[s:s + chunk] = lab
+        rows = np.arange(neg.shape[0])
+        best[s:s + chunk] = -neg[rows, lab]
+        if cq.shape[0] > 1:
+            neg[rows, lab] = np.inf
+            second[s:s + chunk] = -neg.min(axis=1)
+    return labels, best, second
+
+
+def spherical_error(xq: np.ndarray, c64: np.ndarray) -> float:
+    """Mean of 2 - 2 x (highest similarity) over the rows, with the bf16 search
+    copies of the centroids ([README] "Spherical e-means": the reported error)."""
+    _, best, _ = assign_dot(xq, search_copy_of_centroids(c64))
+    return float((2.0 - 2.0 * best).mean())
+
+
+# --------------------------------------------------------------------------
 # Per-batch statistics and the EMA update ([README] "How the centroid updates work")
 # --------------------------------------------------------------------------
 
@@ -391,9 +432,17 @@ def revive(N, S, c, t, seed, mode="split", tau=DEFAULT_TAU, batch_rows=None):
 class EmeansOracle:
     """e-means in fp64 on the bf16 search copy of the data."""
 
-    def __init__(self, d, k, seed=1234, revival="split", tau=DEFAULT_TAU, closing_mean=True,
-                 law="throughput", batch_size=None, alpha0=None):
+    def __init__(self, d, k, seed=1234, revival="split", tau=None, closing_mean=True,
+                 law="auto", batch_size=None, alpha0=None, spherical=False):
         self.d, self.k, self.seed = int(d), int(k), int(seed)
+        self.spherical = bool(spherical)
+        # defaults that depend on the dimension ([README] `batch_law`, `unused_threshold`
+        # and "Note on low dimension"): the quality batch law for d <= 16, no revival
+        # (threshold 0) for d <= 2
+        if tau is None:
+            tau = 0.0 if self.d <= 2 else DEFAULT_TAU
+        if law == "auto":
+            law = "quality" if self.d <= 16 else "throughput"
         self.revival, self.tau, self.closing = revival, float(tau), bool(closing_mean)
         self.law, self.batch_override, self.alpha_override = law, batch_size, alpha0
         self.n_splits = 0
@@ -408,6 +457,8 @@ class EmeansOracle:
         self.r = recipe(n, self.k, epochs, self.law, self.batch_override, self.alpha_override)
         rows = starting_rows(n, self.k, self.seed) if start_rows is None else np.asarray(start_rows)
         self.c = xq[rows].copy()
+        if self.spherical:
+            self.c = unit_rows(self.c)
         self.N = np.zeros(self.k)
         self.S = np.zeros((self.k, self.d))
         self.t = 0
@@ -437,11 +488,17 @@ class EmeansOracle:
         add the statistics of every rank's share of the batch."""
         ids = self.next_batch_ids()
         xb = self.xq[ids]
-        labels, best, second = assign(xb, search_copy_of_centroids(self.c))
+        if self.spherical:  # highest similarity; the error of a row is 2 - 2 x similarity
+            labels, sim, sim2 = assign_dot(xb, search_copy_of_centroids(self.c))
+            best, second = 2.0 - 2.0 * sim, 2.0 - 2.0 * sim2
+        else:
+            labels, best, second = assign(xb, search_copy_of_centroids(self.c))
         used = labels if forced_labels is None else np.asarray(forced_labels, dtype=np.int64)
         n_j, s_j = (batch_stats if stats is None else stats)(xb, used, self.k)
         alpha = alpha_at(self.t, self.r["total_steps"], self.r["alpha0"])
         self.N, self.S, self.c = ema_update(self.N, self.S, self.c, n_j, s_j, alpha)
+        if self.spherical:
+            self.c = unit_rows(self.c)
         last_pass = self.pass_index == len(self.r["epoch_rows"]) - 1
         if last_pass:
             self.labels_last[ids] = used
@@ -469,6 +526,8 @@ class EmeansOracle:
             return None
         self.N, self.S, self.c, dead, donors = revive(
             self.N, self.S, self.c, t, self.seed, self.revival, self.tau, batch_rows)
+        if self.spherical:
+            self.c = unit_rows(self.c)
         self.n_splits += int(np.count_nonzero(donors >= 0))
         return dead, donors
 
@@ -478,6 +537,8 @@ class EmeansOracle:
         if self.closing:
             hit = self.close_cnt > 0
             self.c[hit] = self.close_sum[hit] / self.close_cnt[hit][:, None]
+        if self.spherical:
+            self.c = unit_rows(self.c)
         return self.c
 
     def train(self, xq: np.ndarray, epochs: float):
@@ -487,15 +548,22 @@ class EmeansOracle:
         return self.finalize(), self.labels_last
 
 
-def lloyd(xq: np.ndarray, c0: np.ndarray, iters: int):
+def lloyd(xq: np.ndarray, c0: np.ndarray, iters: int, spherical: bool = False):
     """Lloyd's k-means as the B = n, alpha = 1 case of the same update ([README]
-    "How the centroid updates work"; [Blog] "Lloyd is a special case")."""
+    "How the centroid updates work"; [Blog] "Lloyd is a special case"); spherical:
+    highest similarity, centroids rescaled to norm 1 ([README] "Spherical e-means")."""
     k = c0.shape[0]
-    N, S, c = np.zeros(k), np.zeros_like(c0), c0.copy()
+    N, S, c = np.zeros(k), np.zeros_like(c0), (unit_rows(c0) if spherical else c0.copy())
     history = []
     for _ in range(iters):
-        labels, best, _ = assign(xq, search_copy_of_centroids(c))
-        history.append(float(best.mean()))
+        if spherical:
+            labels, sim, _ = assign_dot(xq, search_copy_of_centroids(c))
+            history.append(float((2.0 - 2.0 * sim).mean()))
+        else:
+            labels, best, _ = assign(xq, search_copy_of_centroids(c))
+            history.append(float(best.mean()))
         n_j, s_j = batch_stats(xq, labels, k)
         N, S, c = ema_update(N, S, c, n_j, s_j, 1.0)
+        if spherical:
+            c = unit_rows(c)
     return c, history

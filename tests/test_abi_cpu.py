@@ -45,6 +45,12 @@ def test_library_is_the_in_tree_build(em):
     assert os.path.dirname(em.LIB_PATH) == os.path.join(ROOT, "mini_ema_means_b200")
 
 
+def test_host_recipe_needs_an_explicit_law(em):
+    # "auto" (2) depends on d, which the model knows; the host-only recipe refuses it
+    with pytest.raises(em.EmeansError):
+        em.compute_recipe(10_000, 64, 5.0, 2)
+
+
 @pytest.mark.parametrize("n,k,T,law,b,a", [
     (10_000, 64, 5, 0, 0, 0.0), (1_000_000, 4096, 5, 0, 0, 0.0), (1_000_000, 16384, 5, 0, 0, 0.0),
     (10_000_000, 65536, 5, 0, 0, 0.0), (100_000_000, 262144, 3, 0, 0, 0.0), (10_000_000, 65536, 5, 1, 0, 0.0),

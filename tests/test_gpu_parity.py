@@ -69,6 +69,8 @@ def test_tiny_teacher_forced_every_step(em, revival):
     (1000, 8, 1, 1.0, 100, "split"),
     (2600, 264, 257, 1.5, None, "split"),
     (3333, 100, 77, 1.0, 1000, "none"),
+    (3000, 2, 20, 2.0, None, "split"),    # d <= 2: the default threshold turns revival off
+    (4000, 12, 50, 2.0, None, "split"),   # d <= 16: the default batch law is the quality law
 ])
 def test_hand_shapes_teacher_forced(em, n, d, k, epochs, batch, revival):
     x = synth.hand_shape(n, d, max(2, k // 2), seed=n + d)

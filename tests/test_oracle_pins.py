@@ -422,6 +422,27 @@ def test_revival_ablation_ordering_on_stand_in_data():
     assert res["split"][1] < res["none"][1]
 
 
+def test_low_dimension_defaults():
+    """[README] `batch_law` / `unused_threshold` and "Note on low dimension": the
+    default ("auto") batch law is the quality law for d <= 16 and the throughput law
+    above; for d <= 2 the default threshold is 0, so no cluster is ever revived."""
+    n, k, T = 200_000, 256, 5.0
+    for d, law in ((2, "quality"), (16, "quality"), (17, "throughput"), (768, "throughput")):
+        em = O.EmeansOracle(d, k)
+        assert em.law == law
+        assert O.recipe(n, k, T, law)["batch_size"] == O.recipe(n, k, T, em.law)["batch_size"]
+    assert O.EmeansOracle(2, k).tau == 0.0 and O.EmeansOracle(3, k).tau == O.DEFAULT_TAU
+    # the quality batch differs from the throughput batch at these sizes (so the rule shows)
+    assert O.recipe(n, k, T, "quality")["batch_size"] < O.recipe(n, k, T, "throughput")["batch_size"]
+    # d = 2: a revival check with every cluster but one dead revives nothing
+    em = O.EmeansOracle(2, 4, seed=1)
+    em.N = np.array([100.0, 0.0, 0.0, 0.0])
+    em.S = np.zeros((4, 2))
+    em.c = np.arange(8.0).reshape(4, 2)
+    dead, donors = em.maybe_revive(np.zeros((10, 2)), t=4)
+    assert len(dead) == 0 and len(donors) == 0 and np.array_equal(em.N, [100.0, 0.0, 0.0, 0.0])
+
+
 # ---------------------------------------------------------------- whole runs
 
 def test_blog_toy_lloyd_stuck_and_emeans_can_escape():
@@ -476,3 +497,68 @@ def test_closing_mean_is_exact_mean_of_last_pass_assignments():
         m = labels == j
         if m.any():
             assert np.allclose(c[j], x[m].mean(axis=0), rtol=1e-12, atol=1e-12)
+
+
+# ---------------------------------------------------------------- spherical e-means
+
+def _unit(x):
+    return x / np.linalg.norm(x, axis=1, keepdims=True)
+
+
+def test_unit_rows_rescales_and_keeps_zero_rows():
+    c = np.array([[3.0, 4.0], [0.0, 0.0], [-1e-3, 0.0]])
+    u = O.unit_rows(c)
+    assert np.allclose(u[0], [0.6, 0.8]) and np.array_equal(u[1], [0.0, 0.0]) and np.allclose(u[2], [-1.0, 0.0])
+
+
+def test_assign_dot_matches_brute_force_with_lowest_index_ties():
+    g = np.random.default_rng(5)
+    x = O.search_copy_of_data(_unit(g.standard_normal((60, 5))))
+    c = O.search_copy_of_centroids(_unit(g.standard_normal((9, 5))))
+    c[7] = c[2]  # an exact tie: the lower index must win
+    labels, best, second = O.assign_dot(x, c)
+    for i in range(60):
+        dots = [float(np.dot(x[i], c[j])) for j in range(9)]
+        top = max(dots)
+        assert labels[i] == dots.index(top) and best[i] == top
+        assert second[i] == sorted(dots)[-2]
+
+
+def test_similarity_and_distance_agree_on_the_unit_sphere():
+    """[README] "Spherical e-means": on vectors of norm 1 the squared distance is
+    2 - 2 x cosine, so the highest dot product is the nearest centroid."""
+    g = np.random.default_rng(6)
+    x, c = _unit(g.standard_normal((500, 12))), _unit(g.standard_normal((40, 12)))
+    d2 = O.squared_distances(x, c)
+    assert np.allclose(d2, 2.0 - 2.0 * (x @ c.T), atol=1e-12)
+    assert np.array_equal(np.argmin(d2, axis=1), np.argmax(x @ c.T, axis=1))
+
+
+def test_spherical_lloyd_step_is_the_normalised_mean():
+    """B = n and alpha = 1: one spherical update is each cluster's mean rescaled to
+    norm 1 (brute force over the assignment)."""
+    g = np.random.default_rng(7)
+    xq = O.search_copy_of_data(_unit(g.standard_normal((400, 6))))
+    c0 = _unit(g.standard_normal((5, 6)))
+    c1, hist = O.lloyd(xq, c0, 1, spherical=True)
+    cq = O.search_copy_of_centroids(O.unit_rows(c0))
+    for j in range(5):
+        members = [i for i in range(400) if int(np.argmax(xq[i] @ cq.T)) == j]
+        if members:
+            m = xq[members].mean(axis=0)
+            assert np.allclose(c1[j], m / np.linalg.norm(m), atol=1e-12)
+    assert hist[0] == pytest.approx(float(np.mean(2.0 - 2.0 * (xq @ cq.T).max(axis=1))))
+
+
+def test_spherical_run_keeps_unit_centroids_and_error_definition():
+    g = np.random.default_rng(8)
+    xq = O.search_copy_of_data(_unit(g.standard_normal((3000, 8)) + np.repeat(g.standard_normal((6, 8)) * 3, 500, 0)))
+    em = O.EmeansOracle(8, 12, seed=2, spherical=True, law="throughput")
+    c, _ = em.train(xq, 2.0)
+    nrm = np.linalg.norm(c, axis=1)
+    assert np.allclose(nrm[nrm > 0], 1.0, atol=1e-12)
+    err = O.spherical_error(xq, c)
+    _, sim, _ = O.assign_dot(xq, O.search_copy_of_centroids(c))
+    assert err == pytest.approx(float(np.mean(2.0 - 2.0 * sim))) and 0.0 <= err < 2.0
+    # it clusters: far below the error of one random unit centroid per row (about 2)
+    assert err < 1.0
