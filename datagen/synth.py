@@ -107,7 +107,7 @@ def mixture_normalized(n_train, n_test, d, ncomp, zipf_s, seed, device, storage=
             x = mu[comp] + sig[comp, None] * torch.randn(m, d, generator=g, device=device)
             x = x / x.norm(dim=1, keepdim=True).clamp_min(1e-30)
             rows.append(_finish(x, storage))
-        out.append(torch.cat(rows))
+        out.append(torch.cat(rows) if rows else torch.empty(0, d, device=device, dtype=torch.float32))
     return out[0], out[1]
 
 
@@ -133,7 +133,7 @@ def subspace_mixture(n_train, n_test, d, ncomp, spectrum_alpha, seed, device, st
             x = mu[comp] + noise * z
             x = x / x.norm(dim=1, keepdim=True).clamp_min(1e-30)
             rows.append(_finish(x, storage))
-        out.append(torch.cat(rows))
+        out.append(torch.cat(rows) if rows else torch.empty(0, d, device=device, dtype=torch.float32))
     return out[0], out[1]
 
 

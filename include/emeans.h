@@ -73,10 +73,17 @@ enum em_option {
                                     SIMT kernel kept only to localise faults in tests           */
     EM_OPT_PROFILE = 14,         /* 1: bracket every phase of every step with CUDA events on the
                                     model's stream (read with em_profile); 0 (default): off     */
-    EM_OPT_EXACT_TIES = 15       /* 1: the search also keeps each row's second best centroid and
+    EM_OPT_EXACT_TIES = 15,      /* 1: the search also keeps each row's second best centroid and
                                     rows whose two best fp32 scores are within the accumulation
                                     error are settled with exact fp64 distances; 0: plain fp32
                                     argmin; -1 (default): on when d >= 256                       */
+    EM_OPT_SPHERICAL = 16        /* 1: spherical e-means (README "Spherical e-means"): every
+                                    centroid is rescaled to norm 1 before each use (a zero
+                                    centroid stays zero), each row goes to the centroid with the
+                                    highest dot product, the closing mean is rescaled to norm 1,
+                                    and the error of a row is 2 - 2 x its similarity. The rows
+                                    are used as given: normalise them first for cosine
+                                    similarity. 0 (default): k-means. Not changeable during a run */
 };
 
 /* Phases timed by EM_OPT_PROFILE (em_profile_t.ms / spans index). */
@@ -216,11 +223,14 @@ int em_lloyd(em_model* m, const void* X, int64_t n, int64_t iters);
  * `assign` returns each vector's nearest centroid and its squared distance).
  * labels: n int64 (may be NULL); dists: n fp32 squared distances computed with
  * the bf16 search copies and clamped at 0 (may be NULL). Ties go to the lowest
- * centroid index. */
+ * centroid index. With EM_OPT_SPHERICAL, the centroid of highest dot product and
+ * dists = that dot product x . bf16(c) (README "Spherical e-means": higher is
+ * closer). */
 int em_assign(em_model* m, const void* X, int64_t n, int64_t* labels, float* dists);
 
 /* Mean over the rows of X of the squared distance to the nearest centroid
- * (fp64 accumulation), as em_assign measures it. Synchronises. */
+ * (fp64 accumulation), as em_assign measures it; with EM_OPT_SPHERICAL, the mean
+ * of 2 - 2 x the highest similarity. Synchronises. */
 int em_mse(em_model* m, const void* X, int64_t n, double* out);
 
 /* Copies the k x d fp32 centroids into out. */
@@ -235,18 +245,21 @@ int em_stats(const em_model* m, em_stats_t* out);
 
 /* Error of each completed pass, measured while the centroids move (README
  * `obj`): mean squared distance of the pass's rows at the time they were
- * assigned. Writes up to cap values; *count receives the number available. */
+ * assigned (spherical: mean of 2 - 2 x similarity). Writes up to cap values;
+ * *count receives the number available. */
 int em_obj(const em_model* m, double* out, int64_t cap, int64_t* count);
 
 /* Model state: running counts N (k fp32), running sums S (k x d fp32),
  * centroids c (k x d fp32) and the global step counter. Any pointer may be
  * NULL. em_set_state replaces the state of the current run (checkpoint resume,
- * step-by-step comparison); the bf16 search copy is refreshed from c. */
+ * step-by-step comparison); the bf16 search copy is refreshed from c (with
+ * EM_OPT_SPHERICAL, c is first rescaled to norm 1). */
 int em_get_state(const em_model* m, float* N, float* S, float* c, int64_t* step);
 int em_set_state(em_model* m, const float* N, const float* S, const float* c, int64_t step);
 
 /* The most recent training batch: its row ids (int64), labels (int64), squared
- * distances (fp32) and row count. Any pointer may be NULL. */
+ * distances (fp32; spherical: 2 - 2 x similarity) and row count. Any pointer may
+ * be NULL. */
 int em_last_batch(const em_model* m, int64_t* ids, int64_t* labels, float* dists, int64_t* rows);
 
 /* Synchronises the model's stream, adds the pending event spans to the totals and
@@ -255,6 +268,7 @@ int em_profile(em_model* m, em_profile_t* out, int reset);
 
 /* ---- assignment without any allocation ----
  *
+ * (k-means only: squared distances to centroids taken as given.)
  * The paper has no counterpart to this entry point. It serves callers that cannot
  * call cudaMalloc: code whose device memory is owned by another allocator or fixed
  * up front (a serving process that forbids allocation after start-up, a library

@@ -47,6 +47,7 @@ EM_OPT_GRAPHS = 12
 EM_OPT_ASSIGN_KERNEL = 13
 EM_OPT_PROFILE = 14
 EM_OPT_EXACT_TIES = 15
+EM_OPT_SPHERICAL = 16
 
 EM_PHASE_PREPARE = 0
 EM_PHASE_GATHER = 1
@@ -213,7 +214,7 @@ class Model:
         "input_dtype": EM_OPT_INPUT_DTYPE, "check_finite": EM_OPT_CHECK_FINITE,
         "wait_limit_ms": EM_OPT_WAIT_LIMIT_MS, "auto_revive": EM_OPT_AUTO_REVIVE,
         "capture_labels": EM_OPT_CAPTURE_LABELS, "graphs": EM_OPT_GRAPHS, "assign_kernel": EM_OPT_ASSIGN_KERNEL,
-        "profile": EM_OPT_PROFILE, "exact_ties": EM_OPT_EXACT_TIES,
+        "profile": EM_OPT_PROFILE, "exact_ties": EM_OPT_EXACT_TIES, "spherical": EM_OPT_SPHERICAL,
     }
 
     def set_option(self, name, value):

@@ -182,6 +182,7 @@ struct em_model {
     double opt_alpha0 = 0.0, tau = -1.0, wait_ms = 2000.0;  // tau < 0: the default for d
     int revival = EM_REVIVE_SPLIT, finalize = 1, law = 2, in_dtype = 0, check_finite = 0;
     int auto_revive = 1, capture = 1, graphs = 1, assign_kernel = 0, exact_ties = -1;
+    int spherical = 0;  // spherical e-means: unit centroids, highest dot product
     int last_split = 1;  // centroid-tile groups of the most recent search (keys per row)
     // state
     DBuf<float> N, N_prev, S, c, cn, cnp;
@@ -417,12 +418,21 @@ static size_t keys_needed(const em_model* m, int64_t rows) {
 
 static TieList tie_list(em_model* m) { return TieList{m->ties.p, m->tie_n.p, m->tie_corr.p}; }
 
+// Value of a training row (labels kernel): its squared distance, or its spherical error.
+static int training_kind(const em_model* m) { return m->spherical ? kSphericalError : kSquaredDistance; }
+
+// Spherical e-means (README "Spherical e-means"): after every change of the
+// centroids, each is rescaled to norm 1 and the search operand is rebuilt.
+static int normalize_if_spherical(em_model* m);
+
 // Settles the near ties the label kernel of `rows` rows queued (a no-op launch when
 // there are none): one warp per row over a fixed grid.
 static int launch_settle(em_model* m, const __nv_bfloat16* A, int32_t* labels32, int64_t* labels64, float* dists,
                          bool count, const int32_t* ids, int64_t* labels_last, int capture) {
+    const int kind = (count || !m->spherical) ? training_kind(m) : kSimilarity;
     k_settle<<<m->sms * 8, 256, 0, m->stream>>>(tie_list(m), m->xn.p, A, m->ld, m->cq.p, labels32, labels64, dists,
-                                                count ? m->cnt.p : nullptr, m->rank.p, ids, labels_last, capture);
+                                                count ? m->cnt.p : nullptr, m->rank.p, ids, labels_last, capture,
+                                                kind);
     CK(cudaGetLastError());
     EM_LAUNCHED(m, 1);
     return EM_OK;
@@ -515,7 +525,7 @@ static int launch_reduce(em_model* m, const __nv_bfloat16* src, int64_t rows, in
                                                                          m->nv, st, sp, m->part.p);
     CK(cudaGetLastError());
     EM_LAUNCHED(m, 4);
-    return EM_OK;
+    return normalize_if_spherical(m);
 }
 
 static ReviveScratch revive_scratch(em_model* m) {
@@ -556,7 +566,7 @@ static int launch_revive(em_model* m, int64_t t, int64_t rows) {
         EM_LAUNCHED(m, 2);
     }
     CK(cudaGetLastError());
-    return EM_OK;
+    return normalize_if_spherical(m);
 }
 
 // One training step of the current run: what it does (host-side plan), the
@@ -610,7 +620,8 @@ static int launch_step(em_model* m, const StepPlan& p) {
     const int capture = (m->capture && p.last_pass) ? 1 : 0;
     k_labels<<<nbl, 256, 0, m->stream>>>(m->keys.p, m->last_split, m->xn.p, (int)rows, (int)m->k, m->Xb.p, m->ld,
                                          m->cq.p, m->ids.p, m->labels.p, m->dists.p, m->cnt.p, m->rank.p,
-                                         m->block_err.p, m->labels_last.p, capture, tie_list(m), m->err.p);
+                                         m->block_err.p, m->labels_last.p, capture, training_kind(m), tie_list(m),
+                                         m->err.p);
     CK(cudaGetLastError());
     EM_LAUNCHED(m, 1);
     CKR(launch_settle(m, m->Xb.p, m->labels.p, nullptr, m->dists.p, true, m->ids.p, m->labels_last.p, capture));
@@ -644,7 +655,8 @@ static std::vector<uint64_t> graph_signature(const em_model* m) {
     for (const void* q : ptrs) sig.push_back((uint64_t)(uintptr_t)q);
     const int64_t ints[] = {m->n, m->d, m->k, m->ld, m->kc, m->R, m->sms, m->rec.batch_size, m->rec.total_steps,
                             m->rec.passes, m->rec.rows_last_pass, (int64_t)m->seed, m->revival, m->finalize,
-                            m->capture, m->auto_revive, m->assign_kernel, m->wait_cycles, m->exact_ties};
+                            m->capture, m->auto_revive, m->assign_kernel, m->wait_cycles, m->exact_ties,
+                            m->spherical};
     for (int64_t v : ints) sig.push_back((uint64_t)v);
     double dbl[] = {m->rec.alpha0, m->tau};
     for (double v : dbl) {
@@ -707,12 +719,20 @@ static int run_steps_graph(em_model* m, int64_t count) {
     return EM_OK;
 }
 
+static int normalize_if_spherical(em_model* m) {
+    if (!m->spherical) return EM_OK;
+    k_normalize<<<grid_for(m->k * 32, 256, m->sms), 256, 0, m->stream>>>(cluster_state(m), (int)m->k, m->nv);
+    CK(cudaGetLastError());
+    EM_LAUNCHED(m, 1);
+    return EM_OK;
+}
+
 static int start_centroids(em_model* m) {
     k_init_centroids<<<grid_for(m->k * 32, 256, m->sms), 256, 0, m->stream>>>(
         m->X, m->n, m->ld, (int)m->k, m->seed, m->c.p, m->S.p, m->N.p, m->cq.p, m->cn.p, m->err.p);
     CK(cudaGetLastError());
     EM_LAUNCHED(m, 1);
-    return EM_OK;
+    return normalize_if_spherical(m);
 }
 
 // ------------------------------------------------------------------ ABI
@@ -887,6 +907,11 @@ int em_set_option(em_model* m, int opt, double v) {
             if (v != -1 && v != 0 && v != 1) return fail(EM_E_INVAL, "exact ties is -1, 0 or 1");
             m->exact_ties = (int)v;
             break;
+        case EM_OPT_SPHERICAL:
+            if (v != 0 && v != 1) return fail(EM_E_INVAL, "spherical is 0 or 1");
+            if (m->running) return fail(EM_E_STATE, "spherical can not change during a run");
+            m->spherical = (int)v;
+            break;
         default: return fail(EM_E_INVAL, "unknown option %d", opt);
     }
     return EM_OK;
@@ -910,6 +935,7 @@ int em_get_option(const em_model* m, int opt, double* v) {
         case EM_OPT_ASSIGN_KERNEL: *v = m->assign_kernel; break;
         case EM_OPT_PROFILE: *v = m->profile; break;
         case EM_OPT_EXACT_TIES: *v = m->exact_ties; break;
+        case EM_OPT_SPHERICAL: *v = m->spherical; break;
         default: return fail(EM_E_INVAL, "unknown option %d", opt);
     }
     return EM_OK;
@@ -1001,6 +1027,7 @@ int em_finalize(em_model* m) {
                                                                                   m->nv);
         CK(cudaGetLastError());
         EM_LAUNCHED(m, 1);
+        CKR(normalize_if_spherical(m));
         span_end(m, sp);
     }
     m->running = false;
@@ -1034,7 +1061,7 @@ int em_lloyd(em_model* m, const void* X, int64_t n, int64_t iters) {
         CKR(launch_assign(m, tmx, m->X, n));
         k_labels<<<nbl, 256, 0, m->stream>>>(m->keys.p, m->last_split, m->xn.p, (int)n, (int)m->k, m->X, m->ld,
                                              m->cq.p, nullptr, m->labels.p, m->dists.p, m->cnt.p, m->rank.p,
-                                             m->block_err.p, nullptr, 0, tie_list(m), m->err.p);
+                                             m->block_err.p, nullptr, 0, training_kind(m), tie_list(m), m->err.p);
         CK(cudaGetLastError());
         EM_LAUNCHED(m, 1);
         CKR(launch_settle(m, m->X, m->labels.p, nullptr, m->dists.p, true, nullptr, nullptr, 0));
@@ -1065,7 +1092,8 @@ static int assign_pass(em_model* m, const void* X, int64_t n, int64_t* labels_de
     CKR(launch_assign(m, tmx, A, n));
     const int blocks = grid_for(n, 256, m->sms);
     k_assign_out<<<blocks, 256, 0, m->stream>>>(m->keys.p, m->last_split, m->xn.p, n, (int)m->k, A, m->ld, m->cq.p,
-                                                labels_dev, dists_dev, nullptr, m->block_err.p, tie_list(m), m->err.p);
+                                                labels_dev, dists_dev, nullptr, m->block_err.p,
+                                                m->spherical ? kSimilarity : kSquaredDistance, tie_list(m), m->err.p);
     CK(cudaGetLastError());
     EM_LAUNCHED(m, 1);
     CKR(launch_settle(m, A, nullptr, labels_dev, dists_dev, false, nullptr, nullptr, 0));
@@ -1237,6 +1265,7 @@ int em_set_state(em_model* m, const float* N, const float* S, const float* c, in
                              cudaMemcpyDefault, m->stream));
     k_refresh_operand<<<grid_for(m->k * 32, 256, m->sms), 256, 0, m->stream>>>(cluster_state(m), (int)m->k, m->nv);
     CK(cudaGetLastError());
+    CKR(normalize_if_spherical(m));
     if (m->running) {
         // move the run's position to `step` (passes are n rows except a fractional last one)
         m->t = step;
@@ -1434,7 +1463,8 @@ extern "C" int em_assign_noalloc(const void* X, int64_t n, int64_t d, const floa
                   nkc, (int)n_tiles, split, keys, wait_cycles, err);
     const int oblocks = std::min(grid_for(n, 256, sms), kNaMaxBlocks);
     k_assign_out<<<oblocks, 256, 0, stream>>>(keys, split * tc::kKeySets, xn, n, (int)k, X16, (int)d, cq, labels,
-                                             dists, nullptr, blocks, TieList{nullptr, nullptr, nullptr}, err);
+                                             dists, nullptr, blocks, kSquaredDistance, TieList{nullptr, nullptr, nullptr},
+                                             err);
     CK(cudaGetLastError());
     int h = 0;
     CK(cudaMemcpyAsync(&h, err, sizeof(int), cudaMemcpyDeviceToHost, stream));

@@ -84,12 +84,59 @@ __device__ __forceinline__ void merge_keys(const unsigned long long* __restrict_
         }
 }
 
+// What the per-row value written by the label kernels means. The search score of a
+// row is s = |bf16(c)|^2 - 2 x.bf16(c) for k-means and s = -2 x.bf16(c) for spherical
+// e-means (faiss e-means README, "Spherical e-means": unit centroids, highest dot
+// product, error 2 - 2 x similarity).
+enum RowValue : int {
+    kSquaredDistance = 0,  // max(0, |x|^2 + s): the squared distance
+    kSphericalError = 1,   // 2 + s = 2 - 2 x.c: the spherical error of the row
+    kSimilarity = 2,       // -s / 2 = x.c: the similarity (spherical assign)
+};
+
+__device__ __forceinline__ float row_value(int kind, float x2, float s) {
+    if (kind == kSquaredDistance) return fmaxf(0.0f, x2 + s);
+    if (kind == kSphericalError) return 2.0f + s;
+    return -0.5f * s;
+}
+
+// The row's contribution to the error sum: the squared distance, or 2 - 2 x similarity.
+__device__ __forceinline__ float row_error(int kind, float x2, float s) {
+    return kind == kSquaredDistance ? fmaxf(0.0f, x2 + s) : 2.0f + s;
+}
+
+// fp64 comparison value of candidate q for a near tie, from the bf16 row x and the
+// bf16 operand q (= -2 bf16(c), so c = -q / 2 exactly): |x - c|^2 for k-means, the
+// score x.q = -2 x.c for spherical e-means. Lanes add disjoint 8-element vectors.
+__device__ __forceinline__ void tie_terms(bool spherical, const uint4& xv, const uint4& qa_v, const uint4& qb_v,
+                                          double& da, double& db) {
+    float x[8], qa[8], qb[8];
+    unpack8_bf16(xv, x);
+    unpack8_bf16(qa_v, qa);
+    unpack8_bf16(qb_v, qb);
+    if (spherical) {
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+            da += (double)x[t] * (double)qa[t];
+            db += (double)x[t] * (double)qb[t];
+        }
+    } else {
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+            const double ea = (double)x[t] + 0.5 * (double)qa[t];
+            const double eb = (double)x[t] + 0.5 * (double)qb[t];
+            da += ea * ea;
+            db += eb * eb;
+        }
+    }
+}
+
 // For every lane of the warp whose row is a near tie (flag), the warp recomputes
-// |x - c|^2 of both candidates in fp64 from the bf16 row and the bf16 operands
-// (c = -q / 2, exact) and keeps the smaller (the lower index on an exact tie).
+// the comparison value of both candidates in fp64 (tie_terms) and keeps the smaller
+// (the lower index on an exact tie).
 __device__ __forceinline__ void settle_ties(bool flag, int64_t row, uint32_t& l1, float& s1, uint32_t l2, float s2,
                                             const __nv_bfloat16* __restrict__ A, int ld,
-                                            const __nv_bfloat16* __restrict__ cq, int lane) {
+                                            const __nv_bfloat16* __restrict__ cq, bool spherical, int lane) {
     unsigned fm = __ballot_sync(0xFFFFFFFFu, flag);
     const int nv = ld / 8;
     while (fm) {
@@ -98,19 +145,10 @@ __device__ __forceinline__ void settle_ties(bool flag, int64_t row, uint32_t& l1
         const int64_t rq = __shfl_sync(0xFFFFFFFFu, row, q);
         const uint32_t la = __shfl_sync(0xFFFFFFFFu, l1, q), lb = __shfl_sync(0xFFFFFFFFu, l2, q);
         double da = 0.0, db = 0.0;
-        for (int v = lane; v < nv; v += 32) {
-            float x[8], qa[8], qb[8];
-            unpack8_bf16(reinterpret_cast<const uint4*>(A + rq * ld)[v], x);
-            unpack8_bf16(reinterpret_cast<const uint4*>(cq + (int64_t)la * ld)[v], qa);
-            unpack8_bf16(reinterpret_cast<const uint4*>(cq + (int64_t)lb * ld)[v], qb);
-#pragma unroll
-            for (int t = 0; t < 8; ++t) {
-                const double ea = (double)x[t] + 0.5 * (double)qa[t];
-                const double eb = (double)x[t] + 0.5 * (double)qb[t];
-                da += ea * ea;
-                db += eb * eb;
-            }
-        }
+        for (int v = lane; v < nv; v += 32)
+            tie_terms(spherical, reinterpret_cast<const uint4*>(A + rq * ld)[v],
+                      reinterpret_cast<const uint4*>(cq + (int64_t)la * ld)[v],
+                      reinterpret_cast<const uint4*>(cq + (int64_t)lb * ld)[v], da, db);
         da = warp_sum(da);
         db = warp_sum(db);
         if (lane == q && (db < da || (db == da && lb < la))) {
@@ -145,7 +183,7 @@ __global__ void k_labels(const unsigned long long* __restrict__ keys, int nsplit
                          const __nv_bfloat16* __restrict__ cq, const int32_t* __restrict__ ids,
                          int32_t* __restrict__ labels, float* __restrict__ dists, int32_t* __restrict__ cnt,
                          int32_t* __restrict__ rank, double* __restrict__ block_err, int64_t* __restrict__ labels_last,
-                         int capture, TieList tl, int* err) {
+                         int capture, int kind, TieList tl, int* err) {
     __shared__ double warp_err[32];
     const int lane = threadIdx.x & 31;
     double e = 0.0;
@@ -175,14 +213,13 @@ __global__ void k_labels(const unsigned long long* __restrict__ keys, int nsplit
     if (tl.e)
         push_ties(defer, r, l1, l2, s2, tl, lane);
     else
-        settle_ties(tie, r, l1, s1, l2, s2, A, ld, cq, lane);
+        settle_ties(tie, r, l1, s1, l2, s2, A, ld, cq, kind != kSquaredDistance, lane);
     int lab = -1;
     if (active) {
         lab = (int)l1;
-        const float dist = fmaxf(0.0f, x2 + s1);
         labels[r] = lab;
-        dists[r] = dist;
-        e = (double)dist;
+        dists[r] = row_value(kind, x2, s1);
+        e = (double)row_error(kind, x2, s1);
         if (capture && !defer) labels_last[ids[r]] = lab;
     }
     const bool counted = active && !defer;
@@ -543,14 +580,14 @@ __global__ void k_clusters(const int32_t* __restrict__ off, const int32_t* __res
 
 // ---------------------------------------------------------------- full assignment pass
 
-// Labels and distances of a full pass (em_assign / em_mse / Lloyd): int64 labels,
-// fp32 squared distances max(0, |x|^2 + score), per-block fp64 sums; near ties are
-// settled exactly as in k_labels.
+// Labels and row values of a full pass (em_assign / em_mse): int64 labels, fp32
+// values of the given kind (squared distances, or similarities), per-block fp64
+// error sums; near ties are settled exactly as in k_labels.
 __global__ void k_assign_out(const unsigned long long* __restrict__ keys, int nsplit, const float* __restrict__ xn,
                              int64_t rows, int k, const __nv_bfloat16* __restrict__ A, int ld,
                              const __nv_bfloat16* __restrict__ cq, int64_t* __restrict__ labels,
                              float* __restrict__ dists, int32_t* __restrict__ labels32, double* __restrict__ block_err,
-                             TieList tl, int* err) {
+                             int kind, TieList tl, int* err) {
     __shared__ double warp_err[32];
     const int lane = threadIdx.x & 31;
     double e = 0.0;
@@ -580,13 +617,12 @@ __global__ void k_assign_out(const unsigned long long* __restrict__ keys, int ns
         if (tl.e)
             push_ties(tie, r, l1, l2, s2, tl, lane);
         else
-            settle_ties(tie, r, l1, s1, l2, s2, A, ld, cq, lane);
+            settle_ties(tie, r, l1, s1, l2, s2, A, ld, cq, kind != kSquaredDistance, lane);
         if (active) {
-            const float dist = fmaxf(0.0f, x2 + s1);
             if (labels) labels[r] = (int64_t)l1;
             if (labels32) labels32[r] = (int32_t)l1;
-            if (dists) dists[r] = dist;
-            e += (double)dist;
+            if (dists) dists[r] = row_value(kind, x2, s1);
+            e += (double)row_error(kind, x2, s1);
         }
     }
     e = warp_sum(e);
@@ -613,18 +649,18 @@ __global__ void k_sum_blocks(const double* __restrict__ block_err, int nblocks, 
     }
 }
 
-// One warp per near-tie row: recomputes |x - c|^2 of both candidates in fp64 from
-// the bf16 row and the bf16 operands (c = -q / 2, exact), keeps the smaller (the
+// One warp per near-tie row: recomputes the comparison value of both candidates in
+// fp64 from the bf16 row and the bf16 operands (tie_terms), keeps the smaller (the
 // lower index on an exact tie), writes the label (int32 and/or int64), and for a
-// relabelled row its distance and the change of the error sum. With cnt, also the
-// row's rank in its cluster (an atomic on the count), and the last-pass label.
-// The distance changes are fp32 differences added in fp64; with few, small terms
+// relabelled row its value (of the given kind) and the change of the error sum. With
+// cnt, also the row's rank in its cluster (an atomic on the count), and the last-pass
+// label. The error changes are fp32 differences added in fp64; with few, small terms
 // their sum does not depend on the order the atomics land in.
 __global__ void k_settle(TieList tl, const float* __restrict__ xn, const __nv_bfloat16* __restrict__ A, int ld,
                          const __nv_bfloat16* __restrict__ cq, int32_t* __restrict__ labels32,
                          int64_t* __restrict__ labels64, float* __restrict__ dists, int32_t* __restrict__ cnt,
                          int32_t* __restrict__ rank, const int32_t* __restrict__ ids,
-                         int64_t* __restrict__ labels_last, int capture) {
+                         int64_t* __restrict__ labels_last, int capture, int kind) {
     const int lane = threadIdx.x & 31;
     const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int nwarps = (gridDim.x * blockDim.x) >> 5;
@@ -635,19 +671,11 @@ __global__ void k_settle(TieList tl, const float* __restrict__ xn, const __nv_bf
         const int64_t r = t.x;
         const uint32_t la = (uint32_t)t.y, lb = (uint32_t)t.z;
         double da = 0.0, db = 0.0;
-        for (int v = lane; v < nv; v += 32) {
-            float x[8], qa[8], qb[8];
-            unpack8_bf16(reinterpret_cast<const uint4*>(A + r * ld)[v], x);
-            unpack8_bf16(reinterpret_cast<const uint4*>(cq + (int64_t)la * ld)[v], qa);
-            unpack8_bf16(reinterpret_cast<const uint4*>(cq + (int64_t)lb * ld)[v], qb);
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const double ea = (double)x[u] + 0.5 * (double)qa[u];
-                const double eb = (double)x[u] + 0.5 * (double)qb[u];
-                da += ea * ea;
-                db += eb * eb;
-            }
-        }
+        const bool spherical = kind != kSquaredDistance;
+        for (int v = lane; v < nv; v += 32)
+            tie_terms(spherical, reinterpret_cast<const uint4*>(A + r * ld)[v],
+                      reinterpret_cast<const uint4*>(cq + (int64_t)la * ld)[v],
+                      reinterpret_cast<const uint4*>(cq + (int64_t)lb * ld)[v], da, db);
         da = warp_sum(da);
         db = warp_sum(db);
         if (lane == 0) {
@@ -655,9 +683,11 @@ __global__ void k_settle(TieList tl, const float* __restrict__ xn, const __nv_bf
             const int lab = (int)(swap ? lb : la);
             if (swap) {
                 const float old = dists[r];
-                const float nd = fmaxf(0.0f, xn[r] + __int_as_float(t.w));
-                dists[r] = nd;
-                atomicAdd(tl.corr, (double)nd - (double)old);
+                const float nval = row_value(kind, xn[r], __int_as_float(t.w));
+                dists[r] = nval;
+                // a similarity v stands for the error 2 - 2 v
+                const double scale = kind == kSimilarity ? -2.0 : 1.0;
+                atomicAdd(tl.corr, scale * ((double)nval - (double)old));
             }
             if (labels32) labels32[r] = lab;
             if (labels64) labels64[r] = (int64_t)lab;
@@ -704,6 +734,35 @@ __global__ void k_refresh_operand(ClusterState st, int k, int nv) {
         }
         cn_part = warp_sum(cn_part);
         if (lane == 0) st.cn[j] = cn_part;
+    }
+}
+
+// Spherical e-means (faiss e-means README, "Spherical e-means"): before it is used,
+// every centroid is rescaled to norm 1; a zero centroid stays zero. One warp per
+// cluster: the norm of the fp32 centroid in fp64, c <- c / |c| rounded to fp32, the
+// search operand -2 bf16(c), and |c|^2 := 0 since the spherical score has no norm term.
+__global__ void k_normalize(ClusterState st, int k, int nv) {
+    const int lane = threadIdx.x & 31;
+    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int nwarps = (gridDim.x * blockDim.x) >> 5;
+    for (int j = warp; j < k; j += nwarps) {
+        const float4* cr = reinterpret_cast<const float4*>(st.c + (int64_t)j * st.ld);
+        double ss = 0.0;
+        for (int v = lane; v < nv; v += 32) {
+            const float4 a = cr[2 * v], b = cr[2 * v + 1];
+            ss += (double)a.x * a.x + (double)a.y * a.y + (double)a.z * a.z + (double)a.w * a.w;
+            ss += (double)b.x * b.x + (double)b.y * b.y + (double)b.z * b.z + (double)b.w * b.w;
+        }
+        ss = warp_sum(ss);
+        const double nrm = ss > 0.0 ? sqrt(ss) : 1.0;
+        float cn_unused = 0.0f;
+        for (int v = lane; v < nv; v += 32) {
+            const float4 a = cr[2 * v], b = cr[2 * v + 1];
+            const float cv[8] = {(float)(a.x / nrm), (float)(a.y / nrm), (float)(a.z / nrm), (float)(a.w / nrm),
+                                 (float)(b.x / nrm), (float)(b.y / nrm), (float)(b.z / nrm), (float)(b.w / nrm)};
+            store_centroid_vec(st.c + (int64_t)j * st.ld, st.cq + (int64_t)j * st.ld, v, cv, cn_unused);
+        }
+        if (lane == 0) st.cn[j] = 0.0f;
     }
 }
 

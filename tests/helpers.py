@@ -4,7 +4,9 @@ Tolerances (stated once, used by every parity test):
 * labels: bit-exact, except rows whose best-vs-second squared-distance gap is
   below 1e-3 of the best distance (a near tie under the fp32 accumulation of the
   tensor cores vs the fp64 oracle); such rows may hold the other near-tied label
-  and may number at most max(1, 1e-4 x rows compared);
+  and may number at most max(1, 1e-4 x rows compared). Spherical e-means compares
+  errors 2 - 2 x similarity the same way, the gap measured against
+  max(best error, 1e-3 |x|^2) since a row can sit on its centroid;
 * centroids: relative L2 error per centroid <= 1e-3;
 * MSE: relative error <= 1e-3 (0.1 %).
 """
@@ -25,22 +27,34 @@ MSE_REL = 1e-3
 class LabelBook:
     """Accumulates label comparisons over several batches."""
 
-    def __init__(self):
+    def __init__(self, spherical=False):
         self.rows = 0
         self.mismatch = 0
+        self.spherical = spherical
 
     def compare(self, gpu_labels, xq_rows, cq):
         """Checks GPU labels against the oracle's search with search copies cq.
 
-        Returns the accepted labels: the oracle's, except where the GPU picked
-        another label of a near tie (both are correct there)."""
+        Returns the accepted labels (the oracle's, except where the GPU picked
+        another label of a near tie: both are correct there) and the oracle's best
+        value per row (squared distance, or spherical error 2 - 2 x similarity)."""
         gpu_labels = np.asarray(gpu_labels, dtype=np.int64)
-        lab, best, second = O.assign(xq_rows, cq)
+        if self.spherical:
+            lab, sim, sim2 = O.assign_dot(xq_rows, cq)
+            best, second = 2.0 - 2.0 * sim, 2.0 - 2.0 * sim2
+        else:
+            lab, best, second = O.assign(xq_rows, cq)
         diff = np.flatnonzero(gpu_labels != lab)
         if len(diff):
-            d_gpu = ((xq_rows[diff] - cq[gpu_labels[diff]]) ** 2).sum(axis=1)
-            ok = (d_gpu - best[diff]) <= LABEL_GAP_REL * np.maximum(best[diff], 1e-30)
-            ok &= (second[diff] - best[diff]) < LABEL_GAP_REL * np.maximum(best[diff], 1e-30)
+            xr, cg = xq_rows[diff], cq[gpu_labels[diff]]
+            if self.spherical:
+                d_gpu = 2.0 - 2.0 * np.einsum("ij,ij->i", xr, cg)
+                scale = np.maximum(best[diff], 1e-3 * np.einsum("ij,ij->i", xr, xr))
+            else:
+                d_gpu = ((xr - cg) ** 2).sum(axis=1)
+                scale = np.maximum(best[diff], 1e-30)
+            ok = (d_gpu - best[diff]) <= LABEL_GAP_REL * scale
+            ok &= (second[diff] - best[diff]) < LABEL_GAP_REL * scale
             assert ok.all(), f"{(~ok).sum()} labels differ from the oracle outside near ties"
         self.rows += len(lab)
         self.mismatch += len(diff)
@@ -94,8 +108,11 @@ def teacher_forced_run(m, orc, x_dev, xq, epochs, revival, check_every=1, max_st
     assert rec["batch_size"] == r_or["batch_size"] and rec["total_steps"] == r_or["total_steps"]
     assert abs(rec["alpha0"] - r_or["alpha0"]) <= 1e-12 * r_or["alpha0"]
     N, S, c, _ = gpu_state(m, k, d)
-    assert np.array_equal(c, orc.c), "starting centroids differ from the oracle's rows"
-    book = LabelBook()
+    if orc.spherical:  # the starting rows rescaled to norm 1 (fp32 on the GPU, fp64 here)
+        np.testing.assert_allclose(c, orc.c, rtol=1e-6, atol=1e-7)
+    else:
+        assert np.array_equal(c, orc.c), "starting centroids differ from the oracle's rows"
+    book = LabelBook(spherical=orc.spherical)
     worst = {"N": 0.0, "c": 0.0, "dist": 0.0, "revive_c": 0.0}
     total = rec["total_steps"] if max_steps is None else min(max_steps, rec["total_steps"])
     revivals = 0

@@ -41,6 +41,19 @@ def test_every_declared_symbol_is_exported(em):
     assert sorted(em.ABI_FUNCTIONS) == declared
 
 
+def test_binding_constants_match_the_header(em):
+    """Every EM_OPT_*, EM_E_*, EM_PHASE_* and EM_REVIVE_* value of the binding is the
+    header's."""
+    with open(os.path.join(ROOT, "include", "emeans.h")) as f:
+        text = re.sub(r"/\*.*?\*/", "", f.read(), flags=re.S)
+    header = {name: int(val) for name, val in re.findall(r"\b(EM_(?:OPT|E|PHASE|REVIVE)_[A-Z_]+)\s*=\s*(-?\d+)", text)}
+    header.update({name: int(val) for name, val in
+                   re.findall(r"#define\s+(EM_(?:OPT|E|PHASE|REVIVE)_[A-Z_]+)\s+\(?(-?\d+)\)?", text)})
+    assert header["EM_OPT_SPHERICAL"] == 16
+    for name, val in header.items():
+        assert getattr(em, name) == val, name
+
+
 def test_library_is_the_in_tree_build(em):
     assert os.path.dirname(em.LIB_PATH) == os.path.join(ROOT, "mini_ema_means_b200")
 
