@@ -177,7 +177,7 @@ def run_ours(args, rank, world):
     torch.cuda.synchronize()
     log(f"[rank {rank}] data {w.name} ready in {time.time() - t0:.1f} s")
     stream = torch.cuda.current_stream(dev)
-    m = em.Model(w.d, w.k, seed=1234, spherical=int(args.spherical))
+    m = em.Model(w.d, w.k, seed=1234, spherical=int(args.spherical), prefetch=args.prefetch)
     m.set_stream(stream.cuda_stream)
     m.set_option("input_dtype", 1 if w.storage == "bf16" else 0)
     rec = m.begin(xt, epochs=w.epochs)
@@ -252,7 +252,7 @@ def run_ours(args, rank, world):
         "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": workload_desc(w), "method": "spherical e-means" if args.spherical else "e-means",
-                   "batch_size": rec["batch_size"], "alpha0": round(rec["alpha0"], 6),
+                   "batch_size": rec["batch_size"], "alpha0": round(rec["alpha0"], 6), "prefetch": args.prefetch,
                    "steps_per_run": total,
                    "l2": "inputs larger than L2: the fp32 training matrix (%.2f GB) and its bf16 copy are re-read "
                          "in a fresh random order every pass" % (w.n_train * w.d * 4 / 1e9),
@@ -532,6 +532,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=100)
     ap.add_argument("--workload", default="emb768")
     ap.add_argument("--spherical", action="store_true", help="spherical e-means (unit centroids, highest dot product)")
+    ap.add_argument("--prefetch", type=int, default=1, choices=[0, 1],
+                    help="gather the next step's rows on a second stream during the update (default 1)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

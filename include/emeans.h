@@ -77,13 +77,17 @@ enum em_option {
                                     rows whose two best fp32 scores are within the accumulation
                                     error are settled with exact fp64 distances; 0: plain fp32
                                     argmin; -1 (default): on when d >= 256                       */
-    EM_OPT_SPHERICAL = 16        /* 1: spherical e-means (README "Spherical e-means"): every
+    EM_OPT_SPHERICAL = 16,       /* 1: spherical e-means (README "Spherical e-means"): every
                                     centroid is rescaled to norm 1 before each use (a zero
                                     centroid stays zero), each row goes to the centroid with the
                                     highest dot product, the closing mean is rescaled to norm 1,
                                     and the error of a row is 2 - 2 x its similarity. The rows
                                     are used as given: normalise them first for cosine
                                     similarity. 0 (default): k-means. Not changeable during a run */
+    EM_OPT_PREFETCH = 17         /* 1 (default): while a step updates the centroids, the rows of
+                                    the next step are gathered into a second batch buffer on a
+                                    second stream the model owns; 0: each step gathers its own
+                                    rows first. Off while EM_OPT_PROFILE is on                  */
 };
 
 /* Phases timed by EM_OPT_PROFILE (em_profile_t.ms / spans index). */

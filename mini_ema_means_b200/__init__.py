@@ -48,6 +48,7 @@ EM_OPT_ASSIGN_KERNEL = 13
 EM_OPT_PROFILE = 14
 EM_OPT_EXACT_TIES = 15
 EM_OPT_SPHERICAL = 16
+EM_OPT_PREFETCH = 17
 
 EM_PHASE_PREPARE = 0
 EM_PHASE_GATHER = 1
@@ -215,6 +216,7 @@ class Model:
         "wait_limit_ms": EM_OPT_WAIT_LIMIT_MS, "auto_revive": EM_OPT_AUTO_REVIVE,
         "capture_labels": EM_OPT_CAPTURE_LABELS, "graphs": EM_OPT_GRAPHS, "assign_kernel": EM_OPT_ASSIGN_KERNEL,
         "profile": EM_OPT_PROFILE, "exact_ties": EM_OPT_EXACT_TIES, "spherical": EM_OPT_SPHERICAL,
+        "prefetch": EM_OPT_PREFETCH,
     }
 
     def set_option(self, name, value):

@@ -197,9 +197,24 @@ struct em_model {
     // batch buffers
     int64_t bcap = 0;
     int R = 32;
-    DBuf<__nv_bfloat16> Xb;
-    DBuf<float> xn, dists;
-    DBuf<int32_t> ids, labels, cnt, rank, off, poff, perm;
+    // The rows of step t live in slot t & 1. While step t runs its update and
+    // revival on the model's stream, the rows of step t + 1 are gathered into the
+    // other slot on the side stream (EM_OPT_PREFETCH).
+    struct BatchSlot {
+        DBuf<__nv_bfloat16> X;  // the batch rows, bf16
+        DBuf<float> xn;         // their |x|^2
+        DBuf<int32_t> ids;      // their data row ids
+        CUtensorMap tm;         // search operand map over X
+    };
+    BatchSlot slot[2];
+    int prefetch = 1;
+    int64_t ready = -1;        // step whose rows are in slot[ready & 1] (gathered or in flight); -1: none
+    bool ready_synced = true;  // the model's stream is already ordered after that gather
+    bool capturing = false;    // a step range is being captured into a graph
+    cudaStream_t side = nullptr, side_cap = nullptr;
+    cudaEvent_t ev_fork = nullptr, ev_gathered[2] = {nullptr, nullptr};
+    DBuf<float> xn, dists;  // xn: |x|^2 of a full pass (assign, MSE, Lloyd)
+    DBuf<int32_t> labels, cnt, rank, off, poff, perm;
     DBuf<int4> items;
     DBuf<unsigned long long> keys;
     DBuf<double> block_err, part, step_err, scalar;
@@ -218,7 +233,7 @@ struct em_model {
     int64_t last_rows = 0;
     double last_alpha = 0.0;
     int last_was_lloyd = 0;
-    CUtensorMap tm_cq, tm_xb;
+    CUtensorMap tm_cq;
     // profiling (EM_OPT_PROFILE) and launch counting
     int profile = 0;
     int64_t launches = 0;
@@ -274,6 +289,7 @@ static int set_device(const em_model* m) {
 }
 
 static int check_device_errors(em_model* m) {
+    if (m->side) CK(cudaStreamSynchronize(m->side));  // a prefetch gather also reports here
     int h = 0;
     CK(cudaMemcpyAsync(&h, m->err.p, sizeof(int), cudaMemcpyDeviceToHost, m->stream));
     CK(cudaStreamSynchronize(m->stream));
@@ -366,7 +382,6 @@ static int ensure_batch_buffers(em_model* m, int64_t cap) {
     const int64_t max_items = m->k + (cap + m->R - 1) / m->R;
     CKR(m->xn.ensure(cap));
     CKR(m->dists.ensure(cap));
-    CKR(m->ids.ensure(cap));
     CKR(m->labels.ensure(cap));
     CKR(m->rank.ensure(cap));
     CKR(m->perm.ensure(cap));
@@ -427,10 +442,10 @@ static int normalize_if_spherical(em_model* m);
 
 // Settles the near ties the label kernel of `rows` rows queued (a no-op launch when
 // there are none): one warp per row over a fixed grid.
-static int launch_settle(em_model* m, const __nv_bfloat16* A, int32_t* labels32, int64_t* labels64, float* dists,
-                         bool count, const int32_t* ids, int64_t* labels_last, int capture) {
+static int launch_settle(em_model* m, const __nv_bfloat16* A, const float* xn, int32_t* labels32, int64_t* labels64,
+                         float* dists, bool count, const int32_t* ids, int64_t* labels_last, int capture) {
     const int kind = (count || !m->spherical) ? training_kind(m) : kSimilarity;
-    k_settle<<<m->sms * 8, 256, 0, m->stream>>>(tie_list(m), m->xn.p, A, m->ld, m->cq.p, labels32, labels64, dists,
+    k_settle<<<m->sms * 8, 256, 0, m->stream>>>(tie_list(m), xn, A, m->ld, m->cq.p, labels32, labels64, dists,
                                                 count ? m->cnt.p : nullptr, m->rank.p, ids, labels_last, capture,
                                                 kind);
     CK(cudaGetLastError());
@@ -547,11 +562,10 @@ static ReviveScratch revive_scratch(em_model* m) {
 static int effective_law(const em_model* m) { return m->law == 2 ? (m->d <= 16 ? 1 : 0) : m->law; }
 static double effective_tau(const em_model* m) { return m->tau < 0.0 ? (m->d <= 2 ? 0.0 : 0.1) : m->tau; }
 
-static int launch_revive(em_model* m, int64_t t, int64_t rows) {
+static int launch_revive(em_model* m, int64_t t, int64_t rows, const __nv_bfloat16* Xb) {
     if (m->revival == EM_REVIVE_NONE || !(effective_tau(m) > 0.0)) return EM_OK;
     const ReviveScratch sc = revive_scratch(m);
-    const TreeLayout L = tree_layout((int)m->k);
-    const int smem = (int)tree_smem_bytes(L, (int)m->k);
+    const int smem = m->k <= kFastK ? tree32((int)m->k).bytes : (int)tree_smem_bytes(tree_layout((int)m->k), (int)m->k);
     k_revive_select<<<1, kSelectThreads, smem, m->stream>>>(m->N.p, (int)m->k, effective_tau(m), m->seed, t,
                                                             m->revival, sc, m->err.p);
     CK(cudaGetLastError());
@@ -562,7 +576,7 @@ static int launch_revive(em_model* m, int64_t t, int64_t rows) {
         k_revive_donors<<<blocks, 256, 0, m->stream>>>(st, m->nv, sc);
         EM_LAUNCHED(m, 3);
     } else {
-        k_revive_resample<<<blocks, 256, 0, m->stream>>>(st, m->nv, sc, m->Xb.p, (int)rows, m->seed, t);
+        k_revive_resample<<<blocks, 256, 0, m->stream>>>(st, m->nv, sc, Xb, (int)rows, m->seed, t);
         EM_LAUNCHED(m, 2);
     }
     CK(cudaGetLastError());
@@ -577,17 +591,67 @@ struct StepPlan {
     double alpha;
 };
 
-static StepPlan plan_step(const em_model* m) {
+static StepPlan plan_at(const em_model* m, int64_t t, int64_t pass, int64_t pos) {
     StepPlan p;
-    const int64_t rows_pass = (m->pass == m->rec.passes - 1) ? m->rec.rows_last_pass : m->n;
-    p.t = m->t;
-    p.pass = m->pass;
-    p.pos = m->pos;
-    p.rows = std::min<int64_t>(m->rec.batch_size, rows_pass - m->pos);
-    p.last_pass = (m->pass == m->rec.passes - 1) ? 1 : 0;
-    p.alpha = alpha_at(m->t, m->rec.total_steps, m->rec.alpha0);
-    p.revive = (m->auto_revive && (m->t + 1) % kReviveEvery == 0) ? 1 : 0;
+    const int64_t rows_pass = (pass == m->rec.passes - 1) ? m->rec.rows_last_pass : m->n;
+    p.t = t;
+    p.pass = pass;
+    p.pos = pos;
+    p.rows = std::min<int64_t>(m->rec.batch_size, rows_pass - pos);
+    p.last_pass = (pass == m->rec.passes - 1) ? 1 : 0;
+    p.alpha = alpha_at(t, m->rec.total_steps, m->rec.alpha0);
+    p.revive = (m->auto_revive && (t + 1) % kReviveEvery == 0) ? 1 : 0;
     return p;
+}
+
+static StepPlan plan_step(const em_model* m) { return plan_at(m, m->t, m->pass, m->pos); }
+
+// The step after p (same rules as advance_step).
+static StepPlan plan_after(const em_model* m, const StepPlan& p) {
+    const int64_t rows_pass = (p.pass == m->rec.passes - 1) ? m->rec.rows_last_pass : m->n;
+    int64_t pass = p.pass, pos = p.pos + p.rows;
+    if (pos >= rows_pass) {
+        pass += 1;
+        pos = 0;
+    }
+    return plan_at(m, p.t + 1, pass, pos);
+}
+
+// Whether step t gathers the rows of step t + 1 on the side stream.
+static bool prefetches(const em_model* m, int64_t t) {
+    return m->prefetch && !m->profile && t + 1 < m->rec.total_steps;
+}
+
+// Gathers the rows of step p into slot p.t & 1 on `stream`.
+static int launch_gather(em_model* m, const StepPlan& p, cudaStream_t stream) {
+    em_model::BatchSlot& b = m->slot[p.t & 1];
+    k_gather<<<grid_for(p.rows, 128, m->sms), 128, 0, stream>>>(m->X, m->n, m->ld, m->seed, p.pass, p.pos,
+                                                               (int)p.rows, 0, b.X.p, b.xn.p, b.ids.p, m->err.p);
+    CK(cudaGetLastError());
+    EM_LAUNCHED(m, 1);
+    return EM_OK;
+}
+
+// Makes the rows of step p available to the model's stream: gathers them there, or
+// orders the stream after the side-stream gather that a previous step started.
+static int prime_batch(em_model* m, const StepPlan& p) {
+    if (m->ready != p.t) {
+        CKR(launch_gather(m, p, m->stream));
+        m->ready = p.t;
+    } else if (!m->ready_synced) {
+        CK(cudaStreamWaitEvent(m->stream, m->ev_gathered[p.t & 1], 0));
+    }
+    m->ready_synced = true;
+    return EM_OK;
+}
+
+// Orders the model's stream after any side-stream gather still in flight and
+// forgets the prefetched rows (before buffers change or a run is repositioned).
+static int drop_prefetch(em_model* m) {
+    if (m->ready >= 0 && !m->ready_synced) CK(cudaStreamWaitEvent(m->stream, m->ev_gathered[m->ready & 1], 0));
+    m->ready = -1;
+    m->ready_synced = true;
+    return EM_OK;
 }
 
 static void advance_step(em_model* m, const StepPlan& p) {
@@ -606,31 +670,50 @@ static void advance_step(em_model* m, const StepPlan& p) {
 static int launch_step(em_model* m, const StepPlan& p) {
     const int64_t rows = p.rows;
     const double rd = (double)rows, dd = (double)m->d, kd = (double)m->k;
+    em_model::BatchSlot& b = m->slot[p.t & 1];
     int sp = span_begin(m, EM_PHASE_GATHER);
-    k_gather<<<grid_for(rows, 256, m->sms), 256, 0, m->stream>>>(m->X, m->n, m->ld, m->seed, p.pass, p.pos,
-                                                                 (int)rows, 0, m->Xb.p, m->xn.p, m->ids.p, m->err.p);
-    CK(cudaGetLastError());
-    EM_LAUNCHED(m, 1);
-    span_end(m, sp, 0.0, 4.0 * rd * dd);
+    const bool inline_gather = m->ready != p.t;
+    CKR(prime_batch(m, p));
+    span_end(m, sp, 0.0, inline_gather ? 4.0 * rd * dd : 0.0);
+    // The next step's rows are gathered on the side stream while this step searches
+    // and updates: the search holds one CTA per SM with registers and threads to
+    // spare, so the memory-bound gather runs beside the tensor-bound search. Slot
+    // (t + 1) & 1 was last read by step t - 1, whose work is all ordered before the
+    // fork. The gather is submitted after the search (and, in graphs, at a lower
+    // priority) so that the search's CTAs are placed first.
+    const bool pf = prefetches(m, p.t);
+    if (pf) CK(cudaEventRecord(m->ev_fork, m->stream));
     sp = span_begin(m, EM_PHASE_ASSIGN);
-    CKR(launch_assign(m, m->tm_xb, m->Xb.p, rows));
+    CKR(launch_assign(m, b.tm, b.X.p, rows));
     span_end(m, sp, 2.0 * rd * kd * dd, 0.0);
+    if (pf) {
+        cudaStream_t side = m->capturing ? m->side_cap : m->side;
+        const StepPlan q = plan_after(m, p);
+        CK(cudaStreamWaitEvent(side, m->ev_fork, 0));
+        CKR(launch_gather(m, q, side));
+        CK(cudaEventRecord(m->ev_gathered[q.t & 1], side));
+    }
     sp = span_begin(m, EM_PHASE_UPDATE);
     const int nbl = (int)((rows + 255) / 256);
     const int capture = (m->capture && p.last_pass) ? 1 : 0;
-    k_labels<<<nbl, 256, 0, m->stream>>>(m->keys.p, m->last_split, m->xn.p, (int)rows, (int)m->k, m->Xb.p, m->ld,
-                                         m->cq.p, m->ids.p, m->labels.p, m->dists.p, m->cnt.p, m->rank.p,
+    k_labels<<<nbl, 256, 0, m->stream>>>(m->keys.p, m->last_split, b.xn.p, (int)rows, (int)m->k, b.X.p, m->ld,
+                                         m->cq.p, b.ids.p, m->labels.p, m->dists.p, m->cnt.p, m->rank.p,
                                          m->block_err.p, m->labels_last.p, capture, training_kind(m), tie_list(m),
                                          m->err.p);
     CK(cudaGetLastError());
     EM_LAUNCHED(m, 1);
-    CKR(launch_settle(m, m->Xb.p, m->labels.p, nullptr, m->dists.p, true, m->ids.p, m->labels_last.p, capture));
-    CKR(launch_reduce(m, m->Xb.p, rows, nbl, p.alpha, m->finalize ? p.last_pass : 0, m->step_err.p + p.t));
+    CKR(launch_settle(m, b.X.p, b.xn.p, m->labels.p, nullptr, m->dists.p, true, b.ids.p, m->labels_last.p,
+                      capture));
+    CKR(launch_reduce(m, b.X.p, rows, nbl, p.alpha, m->finalize ? p.last_pass : 0, m->step_err.p + p.t));
     span_end(m, sp, 0.0, 2.0 * rd * dd + 16.0 * rd + 14.0 * kd * dd);
     if (p.revive) {
         sp = span_begin(m, EM_PHASE_REVIVE);
-        CKR(launch_revive(m, p.t, rows));
+        CKR(launch_revive(m, p.t, rows, b.X.p));
         span_end(m, sp);
+    }
+    if (pf) {
+        m->ready = p.t + 1;
+        m->ready_synced = false;
     }
     return EM_OK;
 }
@@ -644,7 +727,8 @@ static int run_step(em_model* m) {
 
 // Everything a captured step range bakes in: buffer addresses, sizes, options.
 static std::vector<uint64_t> graph_signature(const em_model* m) {
-    const void* ptrs[] = {m->X, m->Xb.p, m->xn.p, m->dists.p, m->ids.p, m->labels.p, m->cnt.p, m->rank.p,
+    const void* ptrs[] = {m->X, m->slot[0].X.p, m->slot[0].xn.p, m->slot[0].ids.p, m->slot[1].X.p,
+                          m->slot[1].xn.p, m->slot[1].ids.p, m->dists.p, m->labels.p, m->cnt.p, m->rank.p,
                           m->N_prev.p, m->cnp.p,
                           m->off.p, m->perm.p, m->poff.p, m->items.p, m->keys.p, m->block_err.p, m->part.p,
                           m->step_err.p, m->labels_last.p, m->N.p, m->S.p, m->c.p, m->cn.p, m->cq.p,
@@ -656,7 +740,7 @@ static std::vector<uint64_t> graph_signature(const em_model* m) {
     const int64_t ints[] = {m->n, m->d, m->k, m->ld, m->kc, m->R, m->sms, m->rec.batch_size, m->rec.total_steps,
                             m->rec.passes, m->rec.rows_last_pass, (int64_t)m->seed, m->revival, m->finalize,
                             m->capture, m->auto_revive, m->assign_kernel, m->wait_cycles, m->exact_ties,
-                            m->spherical};
+                            m->spherical, m->prefetch};
     for (int64_t v : ints) sig.push_back((uint64_t)v);
     double dbl[] = {m->rec.alpha0, m->tau};
     for (double v : dbl) {
@@ -672,29 +756,46 @@ static std::vector<uint64_t> graph_signature(const em_model* m) {
 static int run_steps_graph(em_model* m, int64_t count) {
     const std::vector<uint64_t> sig = graph_signature(m);
     const int64_t t0 = m->t;
+    // a graph starts from the first step's rows in place and ordered before it
+    CKR(prime_batch(m, plan_step(m)));
     for (auto& g : m->graph_cache) {
         if (g.t0 == t0 && g.count == count && g.sig == sig) {
             CK(cudaGraphLaunch(g.exec, m->stream));
             for (int64_t i = 0; i < count; ++i) advance_step(m, plan_step(m));
+            // the graph ends with the prefetch of the next range's first step joined
+            m->ready = prefetches(m, m->t - 1) ? m->t : -1;
+            m->ready_synced = true;
             EM_LAUNCHED(m, g.launches);
             return EM_OK;
         }
     }
-    if (!m->cap_stream) CK(cudaStreamCreateWithFlags(&m->cap_stream, cudaStreamNonBlocking));
+    if (!m->cap_stream || !m->side_cap) {  // the step kernels above the side-stream gathers
+        int least = 0, greatest = 0;
+        CK(cudaDeviceGetStreamPriorityRange(&least, &greatest));
+        if (!m->cap_stream) CK(cudaStreamCreateWithPriority(&m->cap_stream, cudaStreamNonBlocking, greatest));
+        if (!m->side_cap) CK(cudaStreamCreateWithPriority(&m->side_cap, cudaStreamNonBlocking, least));
+    }
     const int64_t save_t = m->t, save_pass = m->pass, save_pos = m->pos, save_rows = m->rows_assigned;
     const int64_t save_last = m->last_rows, save_launches = m->launches;
     const double save_alpha = m->last_alpha;
     cudaStream_t user = m->stream;
     m->stream = m->cap_stream;
+    m->capturing = true;
     CK(cudaStreamBeginCapture(m->cap_stream, cudaStreamCaptureModeThreadLocal));
     int rc = EM_OK;
     for (int64_t i = 0; i < count && rc == EM_OK; ++i) rc = run_step(m);
+    // join the last step's prefetch so that the graph ends with it
+    if (rc == EM_OK && m->ready >= 0 && !m->ready_synced &&
+        cudaStreamWaitEvent(m->cap_stream, m->ev_gathered[m->ready & 1], 0) != cudaSuccess)
+        rc = EM_E_CUDA;
     cudaGraph_t graph = nullptr;
     const cudaError_t ce = cudaStreamEndCapture(m->cap_stream, &graph);
     m->stream = user;
+    m->capturing = false;
+    m->ready_synced = true;
     cudaGraphExec_t exec = nullptr;
     if (rc == EM_OK && ce == cudaSuccess && graph &&
-        cudaGraphInstantiate(&exec, graph, 0) == cudaSuccess) {
+        cudaGraphInstantiateWithFlags(&exec, graph, cudaGraphInstantiateFlagUseNodePriority) == cudaSuccess) {
         cudaGraphDestroy(graph);
         const int64_t launches = m->launches - save_launches;
         if (m->graph_cache.size() >= 64) {
@@ -715,6 +816,8 @@ static int run_steps_graph(em_model* m, int64_t count) {
     m->last_rows = save_last;
     m->last_alpha = save_alpha;
     m->launches = save_launches;
+    m->ready = t0;  // primed before the capture
+    m->ready_synced = true;
     for (int64_t i = 0; i < count; ++i) CKR(run_step(m));
     return EM_OK;
 }
@@ -802,6 +905,11 @@ em_model* em_create(int64_t d, int64_t k, uint64_t seed) {
     if (cudaStreamCreateWithFlags(&m->stream, cudaStreamNonBlocking) != cudaSuccess)
         return bail(EM_E_CUDA, "cudaStreamCreate failed");
     m->own_stream = true;
+    if (cudaStreamCreateWithFlags(&m->side, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaEventCreateWithFlags(&m->ev_fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&m->ev_gathered[0], cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&m->ev_gathered[1], cudaEventDisableTiming) != cudaSuccess)
+        return bail(EM_E_CUDA, "stream or event creation failed");
     const size_t kd = (size_t)k * m->ld;
     if (m->N.ensure(k) || m->N_prev.ensure(k) || m->cnp.ensure((size_t)k * ((m->nv + 31) / 32)) ||
         m->S.ensure(kd) || m->c.ensure(kd) || m->cn.ensure(k) || m->cq.ensure(kd) ||
@@ -839,8 +947,14 @@ void em_destroy(em_model* m) {
     m->N.release(); m->N_prev.release(); m->cnp.release(); m->S.release(); m->c.release(); m->cn.release();
     m->cq.release();
     m->close_sum.release(); m->close_cnt.release(); m->err.release(); m->flag.release();
-    m->Xown.release(); m->stage.release(); m->Xb.release(); m->xn.release(); m->dists.release();
-    m->ids.release(); m->labels.release(); m->cnt.release(); m->rank.release(); m->off.release();
+    if (m->side) cudaStreamSynchronize(m->side);
+    for (auto& b : m->slot) {
+        b.X.release();
+        b.xn.release();
+        b.ids.release();
+    }
+    m->Xown.release(); m->stage.release(); m->xn.release(); m->dists.release();
+    m->labels.release(); m->cnt.release(); m->rank.release(); m->off.release();
     m->perm.release(); m->poff.release(); m->items.release(); m->keys.release(); m->block_err.release();
     m->part.release(); m->step_err.release(); m->scalar.release(); m->labels_last.release();
     m->labels64.release(); m->rv_dead.release(); m->rv_donor.release(); m->rv_order.release();
@@ -854,6 +968,11 @@ void em_destroy(em_model* m) {
     for (auto ev : m->pool) cudaEventDestroy(ev);
     for (auto& g : m->graph_cache) cudaGraphExecDestroy(g.exec);
     if (m->cap_stream) cudaStreamDestroy(m->cap_stream);
+    if (m->side_cap) cudaStreamDestroy(m->side_cap);
+    if (m->side) cudaStreamDestroy(m->side);
+    if (m->ev_fork) cudaEventDestroy(m->ev_fork);
+    for (auto ev : m->ev_gathered)
+        if (ev) cudaEventDestroy(ev);
     if (m->own_stream && m->stream) cudaStreamDestroy(m->stream);
     delete m;
 }
@@ -907,6 +1026,10 @@ int em_set_option(em_model* m, int opt, double v) {
             if (v != -1 && v != 0 && v != 1) return fail(EM_E_INVAL, "exact ties is -1, 0 or 1");
             m->exact_ties = (int)v;
             break;
+        case EM_OPT_PREFETCH:
+            if (v != 0 && v != 1) return fail(EM_E_INVAL, "prefetch is 0 or 1");
+            m->prefetch = (int)v;
+            break;
         case EM_OPT_SPHERICAL:
             if (v != 0 && v != 1) return fail(EM_E_INVAL, "spherical is 0 or 1");
             if (m->running) return fail(EM_E_STATE, "spherical can not change during a run");
@@ -936,6 +1059,7 @@ int em_get_option(const em_model* m, int opt, double* v) {
         case EM_OPT_PROFILE: *v = m->profile; break;
         case EM_OPT_EXACT_TIES: *v = m->exact_ties; break;
         case EM_OPT_SPHERICAL: *v = m->spherical; break;
+        case EM_OPT_PREFETCH: *v = m->prefetch; break;
         default: return fail(EM_E_INVAL, "unknown option %d", opt);
     }
     return EM_OK;
@@ -964,7 +1088,14 @@ int em_begin(em_model* m, const void* X, int64_t n, double epochs) {
     const int sp = span_begin(m, EM_PHASE_PREPARE);
     CKR(prepare_input(m, X, n, m->Xown, &m->X));
     const int64_t b = m->rec.batch_size;
-    CKR(m->Xb.ensure((size_t)b * m->ld));
+    CKR(drop_prefetch(m));
+    CK(cudaStreamSynchronize(m->stream));  // no gather of a previous run still writes the slots
+    for (auto& bs : m->slot) {
+        CKR(bs.X.ensure((size_t)b * m->ld));
+        CKR(bs.xn.ensure(b));
+        CKR(bs.ids.ensure(b));
+        CKR(make_tmap(&bs.tm, bs.X.p, b, (int)m->d, m->ld, tc::BM, m->kc));
+    }
     CKR(ensure_batch_buffers(m, b));
     {  // every batch size the run will see: full batches and the last, partial ones
         const int64_t sizes[3] = {b, n % b, m->rec.rows_last_pass % b};
@@ -983,7 +1114,6 @@ int em_begin(em_model* m, const void* X, int64_t n, double epochs) {
         CKR(m->labels_last.ensure(n));
         CK(cudaMemsetAsync(m->labels_last.p, 0xFF, n * sizeof(int64_t), m->stream));
     }
-    CKR(make_tmap(&m->tm_xb, m->Xb.p, b, (int)m->d, m->ld, tc::BM, m->kc));
     CKR(start_centroids(m));
     span_end(m, sp);
     m->t = m->pass = m->pos = m->rows_assigned = 0;
@@ -1014,13 +1144,14 @@ int em_revive(em_model* m) {
     if (!m) return fail(EM_E_INVAL, "model is NULL");
     if (!m->running || m->t == 0) return fail(EM_E_STATE, "no step has run");
     CKR(set_device(m));
-    return launch_revive(m, m->t - 1, m->last_rows);
+    return launch_revive(m, m->t - 1, m->last_rows, m->slot[(m->t - 1) & 1].X.p);
 }
 
 int em_finalize(em_model* m) {
     if (!m) return fail(EM_E_INVAL, "model is NULL");
     if (!m->running) return fail(EM_E_STATE, "no run in progress");
     CKR(set_device(m));
+    CKR(drop_prefetch(m));
     if (m->finalize && m->t >= m->rec.total_steps) {
         const int sp = span_begin(m, EM_PHASE_FINALIZE);
         k_closing_mean<<<grid_for(m->k * 32, 256, m->sms), 256, 0, m->stream>>>(cluster_state(m), (int)m->k,
@@ -1044,6 +1175,7 @@ int em_lloyd(em_model* m, const void* X, int64_t n, int64_t iters) {
     if (!m) return fail(EM_E_INVAL, "model is NULL");
     if (n < m->k || n >= (1ll << 31) || iters < 0) return fail(EM_E_INVAL, "bad Lloyd arguments");
     CKR(set_device(m));
+    CKR(drop_prefetch(m));
     m->running = false;
     m->n = n;
     CKR(prepare_input(m, X, n, m->Xown, &m->X));
@@ -1064,7 +1196,7 @@ int em_lloyd(em_model* m, const void* X, int64_t n, int64_t iters) {
                                              m->block_err.p, nullptr, 0, training_kind(m), tie_list(m), m->err.p);
         CK(cudaGetLastError());
         EM_LAUNCHED(m, 1);
-        CKR(launch_settle(m, m->X, m->labels.p, nullptr, m->dists.p, true, nullptr, nullptr, 0));
+        CKR(launch_settle(m, m->X, m->xn.p, m->labels.p, nullptr, m->dists.p, true, nullptr, nullptr, 0));
         CKR(launch_reduce(m, m->X, n, nbl, 1.0, 0, m->scalar.p));
     }
     m->have_run = false;
@@ -1096,7 +1228,7 @@ static int assign_pass(em_model* m, const void* X, int64_t n, int64_t* labels_de
                                                 m->spherical ? kSimilarity : kSquaredDistance, tie_list(m), m->err.p);
     CK(cudaGetLastError());
     EM_LAUNCHED(m, 1);
-    CKR(launch_settle(m, A, nullptr, labels_dev, dists_dev, false, nullptr, nullptr, 0));
+    CKR(launch_settle(m, A, m->xn.p, nullptr, labels_dev, dists_dev, false, nullptr, nullptr, 0));
     k_sum_blocks<<<1, 32, 0, m->stream>>>(m->block_err.p, blocks, sum_dev, tie_list(m));
     CK(cudaGetLastError());
     EM_LAUNCHED(m, 1);
@@ -1256,6 +1388,7 @@ int em_set_state(em_model* m, const float* N, const float* S, const float* c, in
     if (!m) return fail(EM_E_INVAL, "model is NULL");
     if (m->running && (step < 0 || step > m->rec.total_steps)) return fail(EM_E_INVAL, "step out of range");
     CKR(set_device(m));
+    CKR(drop_prefetch(m));
     if (N) CK(cudaMemcpyAsync(m->N.p, N, m->k * sizeof(float), cudaMemcpyDefault, m->stream));
     if (S)
         CK(cudaMemcpy2DAsync(m->S.p, m->ld * sizeof(float), S, m->d * sizeof(float), m->d * sizeof(float), m->k,
@@ -1286,7 +1419,8 @@ int em_last_batch(const em_model* m, int64_t* ids, int64_t* labels, float* dists
     std::vector<int32_t> tmp(r);
     std::vector<int64_t> wide(r);
     if (ids) {
-        CK(cudaMemcpyAsync(tmp.data(), m->ids.p, r * sizeof(int32_t), cudaMemcpyDeviceToHost, m->stream));
+        CK(cudaMemcpyAsync(tmp.data(), m->slot[(m->t - 1) & 1].ids.p, r * sizeof(int32_t), cudaMemcpyDeviceToHost,
+                           m->stream));
         CK(cudaStreamSynchronize(m->stream));
         for (int64_t i = 0; i < r; ++i) wide[i] = tmp[i];
         CK(cudaMemcpy(ids, wide.data(), r * sizeof(int64_t), cudaMemcpyDefault));

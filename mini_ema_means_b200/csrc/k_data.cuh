@@ -152,8 +152,9 @@ __global__ void k_init_centroids(const __nv_bfloat16* __restrict__ X, int64_t n,
 
 // Batch gather: row r of the batch is data row pi_pass(base + r); copies it into the
 // contiguous batch buffer, records its id and its squared norm |x|^2 (fp32, from the
-// bf16 values). Each lane computes one row id; the warp
-// then moves the 32 rows four at a time (four independent loads in flight per lane).
+// bf16 values). Each lane computes one row id; the warp then moves the 32 rows four
+// at a time, with every vector of the four rows (up to 1,024 dims per round) loaded
+// before the first store, so that a warp keeps up to 8 KB of reads in flight.
 __global__ void k_gather(const __nv_bfloat16* __restrict__ X, int64_t n, int ld, uint64_t seed, int64_t pass,
                          int64_t base, int rows, int natural_order, __nv_bfloat16* __restrict__ Xb,
                          float* __restrict__ xn, int32_t* __restrict__ ids, int* err) {
@@ -184,18 +185,30 @@ __global__ void k_gather(const __nv_bfloat16* __restrict__ X, int64_t n, int ld,
                 src[u] = __shfl_sync(0xFFFFFFFFu, id, min(q + u, cnt - 1));
                 acc[u] = 0.0f;
             }
-            for (int v = lane; v < nv; v += 32) {
-                uint4 val[4];
+            // up to 4 x 32 vectors (1,024 dims) of the four rows in flight per round
+            for (int vb = 0; vb < nv; vb += 128) {
+                uint4 val[4][4];
 #pragma unroll
-                for (int u = 0; u < 4; ++u) val[u] = reinterpret_cast<const uint4*>(X + src[u] * ld)[v];
+                for (int u = 0; u < 4; ++u)
+#pragma unroll
+                    for (int it = 0; it < 4; ++it) {
+                        const int v = vb + 32 * it + lane;
+                        if (v < nv) val[u][it] = reinterpret_cast<const uint4*>(X + src[u] * ld)[v];
+                    }
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
                     if (q + u < cnt) {
-                        reinterpret_cast<uint4*>(Xb + (int64_t)(r0 + q + u) * ld)[v] = val[u];
-                        float x[8];
-                        unpack8_bf16(val[u], x);
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) acc[u] = fmaf(x[i], x[i], acc[u]);
+                        for (int it = 0; it < 4; ++it) {
+                            const int v = vb + 32 * it + lane;
+                            if (v < nv) {
+                                reinterpret_cast<uint4*>(Xb + (int64_t)(r0 + q + u) * ld)[v] = val[u][it];
+                                float x[8];
+                                unpack8_bf16(val[u][it], x);
+#pragma unroll
+                                for (int i = 0; i < 8; ++i) acc[u] = fmaf(x[i], x[i], acc[u]);
+                            }
+                        }
                     }
                 }
             }

@@ -16,9 +16,12 @@
 //     current batch drawn with Philox(seed, stream 4, t, j), N_j = S_j = 0.
 //
 // The draws are inherently sequential, so one warp makes them on an fp64 tree of
-// prefix sums (128 children per node, four per lane: the top group sits in
-// registers, each lower level costs one group load, one ballot and one group
-// store per draw); the uniform draws are made in parallel beforehand. The donor's
+// prefix sums, the uniform draws having been made in parallel beforehand. Up to
+// 16,384 clusters the tree has 32 children per node, one per lane, and lives in
+// shared memory with its top level in registers: a draw costs one load, one
+// compare, one ballot and one shuffle per level. Larger k use 128 children per
+// node (four per lane), with the lower levels in global memory when shared memory
+// runs out. The donor's
 // current weight is read back as the difference of two prefix values, and the
 // number of earlier splits from the same donor is counted per batch of 32 draws
 // with one warp match. The vector work is then done in parallel from the closed
@@ -182,49 +185,149 @@ __device__ __forceinline__ int group_select(const double P[4], double base, doub
     return 4 * L + s;
 }
 
-// The lean select of the two-level draw: the lane masks of `base + P > t`, one
-// ballot, and the chosen lane's values. Returns -1 when no position exceeds the
-// target (the target fell on the total: the caller takes the fallback).
-__device__ __forceinline__ int select_gt(const double P[4], double Pprev, double base, double t, int lane,
-                                         double* before, double* w) {
-    unsigned mt = 0;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) mt |= (base + P[i] > t) ? (1u << i) : 0u;
-    const unsigned bal = __ballot_sync(0xFFFFFFFFu, mt != 0);
-    if (!bal) return -1;
-    const int L = __ffs(bal) - 1;
-    const int sub = mt ? __ffs(mt) - 1 : 0;
-    const double b = sub == 0 ? Pprev : (sub == 1 ? P[0] : (sub == 2 ? P[1] : P[2]));
-    const double wl = (sub == 0 ? P[0] : (sub == 1 ? P[1] : (sub == 2 ? P[2] : P[3]))) - b;
-    const int s = __shfl_sync(0xFFFFFFFFu, sub, L);
-    *before = __shfl_sync(0xFFFFFFFFu, b, L);
-    *w = __shfl_sync(0xFFFFFFFFu, wl, L);
-    return 4 * L + s;
-}
-
-// The last position of a group whose weight is positive (the first position that
-// reaches the group total), with its weight.
-__device__ __forceinline__ int select_last(const double P[4], double Pprev, int lane, double* w) {
-    const double tot = __shfl_sync(0xFFFFFFFFu, P[3], 31);
-    unsigned mf = 0;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) mf |= (P[i] >= tot) ? (1u << i) : 0u;
-    const unsigned bal = __ballot_sync(0xFFFFFFFFu, mf != 0);
-    const int L = __ffs(bal) - 1;
-    const int sub = mf ? __ffs(mf) - 1 : 0;
-    const double b = sub == 0 ? Pprev : (sub == 1 ? P[0] : (sub == 2 ? P[1] : P[2]));
-    const double wl = (sub == 0 ? P[0] : (sub == 1 ? P[1] : (sub == 2 ? P[2] : P[3]))) - b;
-    const int s = __shfl_sync(0xFFFFFFFFu, sub, L);
-    *w = __shfl_sync(0xFFFFFFFFu, wl, L);
-    return 4 * L + s;
-}
-
 // Subtracts delta from the group positions at or after pos (this lane's four).
 __device__ __forceinline__ bool group_sub(double P[4], int pos, double delta, int lane) {
 #pragma unroll
     for (int i = 0; i < 4; ++i)
         if (4 * lane + i >= pos) P[i] -= delta;
     return 4 * lane + 3 >= pos;
+}
+
+// ---- radix-32 tree for k <= kFastK: one value per lane at every level
+//
+// Level 0 holds, for each group of 32 consecutive clusters, the inclusive prefix
+// sums of their current weights within the group; level 1 the same over the group
+// totals of level 0; level 2 over those of level 1. The top level (at most 32
+// entries) sits in the drawing warp's registers, one entry per lane, and the levels
+// below it in shared memory. A draw then costs, per level, one load, one compare,
+// one ballot and one shuffle, about a third of the instructions of the radix-128
+// descent; a single warp issuing alone is bound by that count.
+constexpr int kFastK = 16384;
+
+struct Tree32 {
+    int levels;   // 1 (k <= 32), 2 (k <= 1024) or 3
+    int n1;       // entries of level 1 = groups of level 0
+    int n2;       // entries of level 2 = groups of level 1
+    int off1;     // doubles: level 1 (levels == 3), after the top staging group
+    int off0;     // doubles: level 0 (levels >= 2)
+    int times;    // doubles: per-donor split counters (ints), -1 when they do not fit
+    int bytes;    // shared memory
+};
+
+EM_HD Tree32 tree32(int k) {
+    Tree32 T{};
+    T.n1 = (k + 31) / 32;
+    T.n2 = (T.n1 + 31) / 32;
+    T.levels = k <= 32 ? 1 : (k <= 1024 ? 2 : 3);
+    int off = 32;  // top staging group
+    T.off1 = off;
+    if (T.levels == 3) off += T.n2 * 32;  // level 1, padded to whole groups
+    T.off0 = off;
+    if (T.levels >= 2) off += T.n1 * 32;  // level 0, padded to whole groups
+    const int base = off * 8;
+    const int tb = ((k * 4 + 15) / 16) * 16;
+    T.times = base + tb <= kReviveSmemBytes ? off : -1;
+    T.bytes = base + (T.times >= 0 ? tb : 0);
+    return T;
+}
+
+// Inclusive prefix of one value per lane.
+__device__ __forceinline__ double lane_scan(double v, int lane) { return warp_incl_scan(v, lane); }
+
+// First lane whose value passes (ballot, then the lowest set lane); -1 if none.
+__device__ __forceinline__ int first_lane(bool pred) {
+    const unsigned b = __ballot_sync(0xFFFFFFFFu, pred);
+    return b ? __ffs(b) - 1 : -1;
+}
+
+// Sequential donor draws of dead clusters [0, nd) on the radix-32 tree, by one warp.
+// T / Tprev: this lane's inclusive / exclusive prefix of the top level; W: the total.
+// Writes donor, order (earlier splits of the same donor in this check) and the
+// per-donor counters; returns the number of splits.
+template <int LEVELS>
+__device__ __forceinline__ int64_t draw_radix32(double* smem_d, const Tree32& TL, int nd, const ReviveScratch& sc,
+                                                int32_t* times, int lane) {
+    double T = smem_d[lane];
+    double Tprev = lane ? smem_d[lane - 1] : 0.0;
+    double W = __shfl_sync(0xFFFFFFFFu, T, 31);
+    double* L1 = smem_d + TL.off1;
+    double* L0 = smem_d + TL.off0;
+    int64_t splits = 0;
+    int i_end = nd;
+    for (int i0 = 0; i0 < nd; i0 += 32) {
+        const int cnt = min(32, nd - i0);
+        const double my_u = lane < cnt ? sc.target[i0 + lane] : 0.0;
+        int my_dn = -1;
+        for (int q = 0; q < cnt; ++q) {
+            if (!(W > 0.0)) {
+                i_end = i0 + q;
+                break;
+            }
+            const double tg = __shfl_sync(0xFFFFFFFFu, my_u, q) * W;
+            // a target on (or, rounded, past) the total takes the last cluster with
+            // weight: at every level, the first position whose prefix reaches its total
+            const bool on_total = !(tg < W);
+            int g2 = first_lane(on_total ? T >= W : T > tg);
+            if (g2 < 0) g2 = first_lane(T >= W);
+            double before = __shfl_sync(0xFFFFFFFFu, Tprev, g2);
+            int d, l1 = 0, l0 = 0, base1 = 0, base0 = 0;
+            double v1 = 0.0, v0 = 0.0, w;
+            if (LEVELS == 1) {
+                d = g2;
+                w = __shfl_sync(0xFFFFFFFFu, T - Tprev, g2);
+            } else {
+                int g1 = g2;
+                if (LEVELS == 3) {
+                    base1 = g2 * 32;
+                    v1 = L1[base1 + lane];
+                    const double v1p = lane ? L1[base1 + lane - 1] : 0.0;
+                    const double tot1 = __shfl_sync(0xFFFFFFFFu, v1, 31);
+                    l1 = first_lane(on_total ? v1 >= tot1 : before + v1 > tg);
+                    if (l1 < 0) l1 = first_lane(v1 >= tot1);  // (exact sums: never)
+                    before += __shfl_sync(0xFFFFFFFFu, v1p, l1);
+                    g1 = base1 + l1;
+                }
+                base0 = g1 * 32;
+                v0 = L0[base0 + lane];
+                const double v0p = lane ? L0[base0 + lane - 1] : 0.0;
+                const double tot0 = __shfl_sync(0xFFFFFFFFu, v0, 31);
+                l0 = first_lane(on_total ? v0 >= tot0 : before + v0 > tg);
+                if (l0 < 0) l0 = first_lane(v0 >= tot0);  // (exact sums: never)
+                d = base0 + l0;
+                w = __shfl_sync(0xFFFFFFFFu, v0 - v0p, l0);
+            }
+            // the donor keeps the rounded half of its weight; explicit roundings, since
+            // a fused multiply-add would round the half differently in the subnormal range
+            const double keep = __dmul_rn(0.5, w);
+            const double delta = __dsub_rn(w, keep);
+            if (LEVELS >= 2 && lane >= l0) L0[base0 + lane] = v0 - delta;
+            if (LEVELS == 3 && lane >= l1) L1[base1 + lane] = v1 - delta;
+            if (lane >= g2) T -= delta;
+            if (lane > g2) Tprev -= delta;
+            W -= delta;
+            if (lane == q) my_dn = d;
+            __syncwarp();  // the group stored above may be the next draw's
+        }
+        const bool has = lane < cnt && my_dn >= 0;
+        const unsigned peers = __match_any_sync(0xFFFFFFFFu, has ? my_dn : -1);
+        const int leader = __ffs(peers) - 1;
+        int old = 0;
+        if (has && lane == leader) old = times[my_dn];
+        old = __shfl_sync(0xFFFFFFFFu, old, leader);
+        if (has) {
+            const int rk = __popc(peers & ((1u << lane) - 1u));
+            sc.donor[i0 + lane] = my_dn;
+            sc.order[i0 + lane] = old + rk;
+            if (lane == leader) times[my_dn] = old + __popc(peers);
+        } else if (lane < cnt) {
+            sc.donor[i0 + lane] = -1;
+        }
+        splits += __popc(__ballot_sync(0xFFFFFFFFu, has));
+        __syncwarp();  // the counters written above are read by other lanes next batch
+        if (i_end < nd) break;
+    }
+    for (int i = (i_end / 32 + 1) * 32 + lane; i < nd; i += 32) sc.donor[i] = -1;
+    return splits;
 }
 
 // One CTA of kSelectThreads threads: dead set, donor tree, sequential donor draws
@@ -290,9 +393,50 @@ __global__ void __launch_bounds__(kSelectThreads) k_revive_select(const float* _
     // draws of every dead cluster, in parallel (they do not depend on each other)
     for (int i = tid; i < nd; i += kSelectThreads) sc.target[i] = draw_uniform(seed, kStreamRevive, t, sc.dead[i]);
 
-    // donor tree (loops over levels have a fixed trip count so that the layout
-    // stays in registers)
     extern __shared__ __align__(16) double smem_d[];
+    if (k <= kFastK) {  // radix-32 tree in shared memory
+        const Tree32 TL = tree32(k);
+        int32_t* times = TL.times >= 0 ? reinterpret_cast<int32_t*>(smem_d + TL.times) : sc.times;
+        for (int j = tid; j < k; j += kSelectThreads) times[j] = 0;
+        // level 0 (the staging group when it is the top)
+        double* L0 = TL.levels == 1 ? smem_d : smem_d + TL.off0;
+        for (int g = w; g < TL.n1; g += kSelectWarps) {
+            const int j = g * 32 + lane;
+            const float nj = j < k ? N[j] : 0.0f;
+            const double v = (j < k && !((double)nj < thr)) ? (double)nj : 0.0;
+            L0[g * 32 + lane] = lane_scan(v, lane);
+        }
+        __syncthreads();
+        if (TL.levels >= 2) {  // level 1 (staged when it is the top)
+            double* L1 = TL.levels == 2 ? smem_d : smem_d + TL.off1;
+            for (int g = w; g < TL.n2; g += kSelectWarps) {
+                const int i = g * 32 + lane;
+                const double v = i < TL.n1 ? L0[i * 32 + 31] : 0.0;
+                L1[g * 32 + lane] = lane_scan(v, lane);
+            }
+            __syncthreads();
+        }
+        if (TL.levels == 3) {  // level 2, the top
+            if (w == 0) {
+                const double v = lane < TL.n2 ? smem_d[TL.off1 + lane * 32 + 31] : 0.0;
+                smem_d[lane] = lane_scan(v, lane);
+            }
+            __syncthreads();
+        }
+        if (w == 0) {
+            const int64_t splits = TL.levels == 1   ? draw_radix32<1>(smem_d, TL, nd, sc, times, lane)
+                                   : TL.levels == 2 ? draw_radix32<2>(smem_d, TL, nd, sc, times, lane)
+                                                    : draw_radix32<3>(smem_d, TL, nd, sc, times, lane);
+            if (lane == 0) *sc.n_splits += splits;
+        }
+        __syncthreads();
+        if (TL.times >= 0)
+            for (int j = tid; j < k; j += kSelectThreads) sc.times[j] = times[j];
+        return;
+    }
+
+    // donor tree for larger k (loops over levels have a fixed trip count so that
+    // the layout stays in registers)
     const TreeLayout L = tree_layout(k);
     const int top = L.levels - 1;
     double* level_ptr[kTreeLevels];
@@ -352,77 +496,8 @@ __global__ void __launch_bounds__(kSelectThreads) k_revive_select(const float* _
         double W = __shfl_sync(0xFFFFFFFFu, T[3], 31);
         int64_t splits = 0;
         int i_end = nd;  // draws from i_end on get no donor (no weight left)
-        // two levels (k <= 16384): the top group in registers, level 0 in shared memory
-        const bool two_level = top == 1 && L.smem_from == 0;
-        double* lev0 = smem_d + kRadix;
-        double Tprev = __shfl_up_sync(0xFFFFFFFFu, T[3], 1);
-        if (lane == 0) Tprev = 0.0;
-        for (int i0 = 0; two_level && i0 < nd; i0 += 32) {
-            const int cnt = min(32, nd - i0);
-            const double my_u = lane < cnt ? sc.target[i0 + lane] : 0.0;
-            int my_dn = -1;
-            for (int q = 0; q < cnt; ++q) {
-                if (!(W > 0.0)) {
-                    i_end = i0 + q;
-                    break;
-                }
-                const double tg = __shfl_sync(0xFFFFFFFFu, my_u, q) * W;
-                double before, wsel;
-                int g = select_gt(T, Tprev, 0.0, tg, lane, &before, &wsel);
-                double P[4];
-                int pos;
-                if (g >= 0) {
-                    const double2* sp = reinterpret_cast<const double2*>(lev0 + g * kRadix + 4 * lane);
-                    const double2 a = sp[0], b = sp[1];
-                    P[0] = a.x; P[1] = a.y; P[2] = b.x; P[3] = b.y;
-                    double Pprev = __shfl_up_sync(0xFFFFFFFFu, P[3], 1);
-                    if (lane == 0) Pprev = 0.0;
-                    double b0;
-                    pos = select_gt(P, Pprev, before, tg, lane, &b0, &wsel);
-                    if (pos < 0) pos = select_last(P, Pprev, lane, &wsel);  // (exact sums: never)
-                } else {  // the target fell on the total: the last cluster with weight
-                    g = select_last(T, Tprev, lane, &wsel);
-                    const double2* sp = reinterpret_cast<const double2*>(lev0 + g * kRadix + 4 * lane);
-                    const double2 a = sp[0], b = sp[1];
-                    P[0] = a.x; P[1] = a.y; P[2] = b.x; P[3] = b.y;
-                    double Pprev = __shfl_up_sync(0xFFFFFFFFu, P[3], 1);
-                    if (lane == 0) Pprev = 0.0;
-                    pos = select_last(P, Pprev, lane, &wsel);
-                }
-                // the donor keeps the rounded half of its weight (explicit roundings: see below)
-                const double keep = __dmul_rn(0.5, wsel);
-                const double delta = __dsub_rn(wsel, keep);
-                if (group_sub(P, pos, delta, lane)) {
-                    double2* sp = reinterpret_cast<double2*>(lev0 + g * kRadix + 4 * lane);
-                    sp[0] = make_double2(P[0], P[1]);
-                    sp[1] = make_double2(P[2], P[3]);
-                }
-                group_sub(T, g, delta, lane);
-                Tprev = __shfl_up_sync(0xFFFFFFFFu, T[3], 1);
-                if (lane == 0) Tprev = 0.0;
-                W -= delta;
-                if (lane == q) my_dn = g * kRadix + pos;
-            }
-            const bool has = lane < cnt && my_dn >= 0;
-            const unsigned peers = __match_any_sync(0xFFFFFFFFu, has ? my_dn : -1);
-            const int leader = __ffs(peers) - 1;
-            int old = 0;
-            if (has && lane == leader) old = times[my_dn];
-            old = __shfl_sync(0xFFFFFFFFu, old, leader);
-            if (has) {
-                const int rk = __popc(peers & ((1u << lane) - 1u));
-                sc.donor[i0 + lane] = my_dn;
-                sc.order[i0 + lane] = old + rk;
-                if (lane == leader) times[my_dn] = old + __popc(peers);
-            } else if (lane < cnt) {
-                sc.donor[i0 + lane] = -1;
-            }
-            splits += __popc(__ballot_sync(0xFFFFFFFFu, has));
-            __syncwarp();  // the counters written above are read by other lanes next batch
-            if (i_end < nd) break;
-        }
         // deeper trees or global levels: one group per level, any depth
-        for (int i0 = 0; !two_level && i0 < nd; i0 += 32) {
+        for (int i0 = 0; i0 < nd; i0 += 32) {
             const int cnt = min(32, nd - i0);
             const double my_u = lane < cnt ? sc.target[i0 + lane] : 0.0;
             int my_dn = -1;

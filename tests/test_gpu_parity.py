@@ -234,6 +234,38 @@ def test_step_graphs_match_direct_launches(em):
         assert np.array_equal(obj, outs[0][2]) and splits == outs[0][3]
 
 
+@pytest.mark.parametrize("graphs", [0, 1])
+def test_prefetched_batches_match_inline_gathers(em, graphs):
+    """Gathering the next step's rows on the side stream while a step updates gives
+    the same run, bit for bit, as gathering every step's rows in turn: stepped one at
+    a time, in uneven ranges (graphs), across pass ends and a fractional last pass,
+    with a state reset in the middle and the revival's resampling reading the rows."""
+    x = synth.hand_shape(5000, 96, 30, seed=14)
+    outs = []
+    for prefetch in (0, 1):
+        m = em.Model(96, 70, seed=5, graphs=graphs, prefetch=prefetch, revival="resample")
+        m.begin(x.cuda(), epochs=2.5)
+        total = m.recipe()["total_steps"]
+        done = 0
+        for chunk in (1, 3, 2, 7, 1):
+            done += m.step(chunk)
+        N, S, c, step = gpu_state(m, 70, 96)
+        m.set_state(N=torch.from_numpy(N.astype(np.float32)), S=torch.from_numpy(S.astype(np.float32)),
+                    c=torch.from_numpy(c.astype(np.float32)), step=step)
+        while done < total:
+            done += m.step(4)
+        ids = torch.empty(m.recipe()["batch_size"], dtype=torch.int64)
+        r = m.last_batch(ids=ids)
+        m.finalize()
+        cc = torch.empty(70, 96)
+        m.centroids(cc)
+        lab = torch.empty(5000, dtype=torch.int64)
+        m.labels(lab)
+        outs.append((cc, lab, m.obj(), ids[:r].clone()))
+    assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
+    assert np.array_equal(outs[0][2], outs[1][2]) and torch.equal(outs[0][3], outs[1][3])
+
+
 @pytest.mark.parametrize("d", [64, 96, 768])
 def test_exact_ties_reproduce_the_fp64_argmin(em, d):
     """Centroids come in pairs one bf16 step apart, so most rows are near ties of
