@@ -150,6 +150,32 @@ def oracle_sample_rate(w, xt_dev, seconds, rows_per_step=None, log_prefix="cpu",
 
 # ---------------------------------------------------------------- our arm
 
+class stdout_to_stderr:
+    """Sends what native code writes to stdout (NCCL prints its version when a
+    communicator is created) to stderr, so that stdout carries only the JSON line."""
+
+    def __enter__(self):
+        sys.stdout.flush()
+        self.saved = os.dup(1)
+        os.dup2(2, 1)
+        return self
+
+    def __exit__(self, *exc):
+        sys.stdout.flush()
+        os.dup2(self.saved, 1)
+        os.close(self.saved)
+        return False
+
+
+def dp_join(em, m, world):
+    """Data-parallel mode for model m: the torch.distributed group's ranks, or one rank."""
+    with stdout_to_stderr():
+        if world > 1:
+            m.dp_init()
+        else:
+            m.dp_init_id(1, 0, em.dp_unique_id())
+
+
 def reduce_over_ranks(ms, rows, device, world):
     """The job's time is the slowest rank's; its rows are every rank's."""
     if world <= 1:
@@ -173,12 +199,15 @@ def run_ours(args, rank, world):
     torch.cuda.set_device(dev)
     peaks = measured_peaks()
     t0 = time.time()
-    w, xt, xs = datagen.make(args.workload, device=dev, seed=0)
+    # replicas train on the same rows; data-parallel ranks each hold their own
+    w, xt, xs = datagen.make(args.workload, device=dev, seed=rank if args.dp else 0)
     torch.cuda.synchronize()
     log(f"[rank {rank}] data {w.name} ready in {time.time() - t0:.1f} s")
     stream = torch.cuda.current_stream(dev)
     m = em.Model(w.d, w.k, seed=1234, spherical=int(args.spherical), prefetch=args.prefetch)
     m.set_stream(stream.cuda_stream)
+    if args.dp:
+        dp_join(em, m, world)
     m.set_option("input_dtype", 1 if w.storage == "bf16" else 0)
     rec = m.begin(xt, epochs=w.epochs)
     total = rec["total_steps"]
@@ -246,6 +275,8 @@ def run_ours(args, rank, world):
     prof = m.profile(reset=True)
     m.set_option("profile", 0)
     ms_max, rows_all = reduce_over_ranks(ms, rows, dev, world)
+    if args.dp:  # every rank counted the rows of the whole batch
+        rows_all = rows
     value = rows_all / (ms_max / 1e3)
     out = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -256,7 +287,8 @@ def run_ours(args, rank, world):
                    "steps_per_run": total,
                    "l2": "inputs larger than L2: the fp32 training matrix (%.2f GB) and its bf16 copy are re-read "
                          "in a fresh random order every pass" % (w.n_train * w.d * 4 / 1e9),
-                   "parallelism": "replicas" if world > 1 else "single GPU"},
+                   "parallelism": (f"data-parallel dp{world} (NCCL all-reduce of the batch statistics)" if args.dp
+                                   else "replicas" if world > 1 else "single GPU")},
     }
     # roofline of the dominant kernel: the fused assignment (tensor-core bound)
     a_ms = prof["ms"]["assign"]
@@ -291,7 +323,7 @@ def run_ours(args, rank, world):
     if rank == 0 and not args.no_extras:
         out["lloyd25"] = lloyd25(m, w, xt, xs, rec)
     if not args.no_e2e:
-        out["e2e"] = e2e(em, w, xt, stream, world, dev, spherical=args.spherical)
+        out["e2e"] = e2e(em, w, xt, stream, world, dev, spherical=args.spherical, dp=args.dp)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, sample, threads = oracle_sample_rate(w, xt, args.cpu_seconds, spherical=args.spherical)
         out["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample}
@@ -357,7 +389,7 @@ def lloyd25(m, w, xt, xs, rec):
             "final_ratio": final / target, "checkpoints": history}
 
 
-def e2e(em, w, xt, stream, world, dev, spherical=False):
+def e2e(em, w, xt, stream, world, dev, spherical=False, dp=False):
     """em_train through the C ABI with a pinned host matrix: H2D copy, training and
     the centroid read-back inside the timed region."""
     import torch
@@ -365,6 +397,8 @@ def e2e(em, w, xt, stream, world, dev, spherical=False):
     xh = xt.cpu().pin_memory()
     m = em.Model(w.d, w.k, seed=1234, spherical=int(spherical))
     m.set_stream(stream.cuda_stream)
+    if dp:
+        dp_join(em, m, world)
     cent = torch.empty(w.k, w.d).pin_memory()
     m.train(xh, epochs=w.epochs)  # warm-up run
     m.centroids(cent)
@@ -534,6 +568,9 @@ def main():
     ap.add_argument("--spherical", action="store_true", help="spherical e-means (unit centroids, highest dot product)")
     ap.add_argument("--prefetch", type=int, default=1, choices=[0, 1],
                     help="gather the next step's rows on a second stream during the update (default 1)")
+    ap.add_argument("--dp", action="store_true",
+                    help="data-parallel e-means: each rank holds its own rows, the per-batch statistics are added "
+                         "with NCCL (default for several GPUs: independent replicas)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -46,6 +46,7 @@ extern "C" {
 #define EM_E_NONFINITE (-6) /* EM_OPT_CHECK_FINITE found NaN or infinity in the input */
 #define EM_E_STATE (-7)     /* call out of order (e.g. em_step before em_begin)       */
 #define EM_E_NODEVICE (-8)  /* no CUDA device is present                              */
+#define EM_E_COMM (-9)      /* the collective library (NCCL) is missing or a call failed */
 
 /* ---- options (em_set_option / em_get_option; values are doubles) ---- */
 enum em_option {
@@ -304,6 +305,42 @@ int em_assign_noalloc(const void* X, int64_t n, int64_t d, const float* centroid
 /* Waits for the model's stream and reports device-side errors (EM_E_BOUNDS,
  * EM_E_TIMEOUT) raised since the last check. */
 int em_sync(em_model* m);
+
+/* ---- data parallelism (README "Several GPUs": DistributedEmeans) ----
+ *
+ * One process per GPU, each holding its own share of the rows. After em_dp_init,
+ * em_begin / em_train / em_lloyd take this rank's rows (X, n): the recipe is
+ * computed for the rows of all ranks (n x world), every batch is split evenly
+ * across the ranks (each takes its share of a batch from its own per-pass order
+ * of its own rows; rank r's order is keyed by the pass and r), the ranks' per-
+ * cluster statistics (n_j, s_j, fp64, with the batch error) are added with one
+ * NCCL all-reduce per step on the model's stream, and every rank applies the same
+ * EMA update and revival, so all ranks hold the same model. Rank 0's starting
+ * centroids are used (one broadcast at em_begin). Sums of bf16 rows in fp64 are
+ * exact, so the result does not depend on the order the ranks' sums are added
+ * in; with world = 1 a run equals the single-GPU run bit for bit.
+ *
+ * Requirements (README "Several GPUs"): every rank makes the same calls with the
+ * same options and the same n; the batch size and the rows of every pass divide by
+ * world (em_begin returns EM_E_INVAL otherwise); resampling revival needs world = 1.
+ * em_assign / em_mse / em_labels stay local to the rank's rows.
+ *
+ * NCCL is loaded at run time (libnccl.so.2 already in the process, else the first
+ * on the library path); without it these calls return EM_E_COMM. */
+#define EM_NCCL_ID_BYTES 128
+
+/* Writes a fresh communicator id (EM_NCCL_ID_BYTES bytes) to id_out. Rank 0 calls
+ * it and hands the bytes to the other ranks by any means (a torch.distributed
+ * broadcast, a file). Host-only. */
+int em_dp_unique_id(void* id_out);
+
+/* Joins the model to the communicator `id` as `rank` of `world` ranks, on the
+ * model's device (collective: every rank calls it). Replaces an earlier
+ * communicator; not allowed during a run. */
+int em_dp_init(em_model* m, int world, int rank, const void* id);
+
+/* The model's world size and rank (1 and 0 without em_dp_init). */
+int em_dp_world(const em_model* m, int* world, int* rank);
 
 #ifdef __cplusplus
 }

@@ -31,6 +31,7 @@ EM_E_TIMEOUT = -5
 EM_E_NONFINITE = -6
 EM_E_STATE = -7
 EM_E_NODEVICE = -8
+EM_E_COMM = -9
 
 EM_OPT_BATCH_SIZE = 1
 EM_OPT_ALPHA0 = 2
@@ -144,7 +145,19 @@ _SIGS = {
     "em_profile": (ctypes.c_int, [_P, ctypes.POINTER(em_profile_t), ctypes.c_int]),
     "em_assign_noalloc": (ctypes.c_int, [_P, _I64, _I64, _P, _I64, _P, _P, _P]),
     "em_sync": (ctypes.c_int, [_P]),
+    "em_dp_unique_id": (ctypes.c_int, [_P]),
+    "em_dp_init": (ctypes.c_int, [_P, ctypes.c_int, ctypes.c_int, _P]),
+    "em_dp_world": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]),
 }
+
+EM_NCCL_ID_BYTES = 128
+
+
+def dp_unique_id() -> bytes:
+    """A fresh communicator id for em_dp_init (rank 0 makes it, the others receive it)."""
+    buf = ctypes.create_string_buffer(EM_NCCL_ID_BYTES)
+    check(em_dp_unique_id(ctypes.cast(buf, ctypes.c_void_p)), "em_dp_unique_id")
+    return buf.raw
 
 for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(lib, _name)
@@ -197,6 +210,18 @@ def permutation(n, seed, stream, which, idx):
     return out
 
 
+def exchange_dp_id(group=None):
+    """(world, rank, id): rank 0 of a torch.distributed group makes a communicator id
+    and broadcasts it to the group's other ranks."""
+    import torch.distributed as dist
+
+    world, rank = dist.get_world_size(group), dist.get_rank(group)
+    obj = [dp_unique_id() if rank == 0 else None]
+    src = 0 if group is None else dist.get_global_rank(group, 0)
+    dist.broadcast_object_list(obj, src=src, group=group)
+    return world, rank, obj[0]
+
+
 class Model:
     """One e-means model (handle owner). X and outputs are torch tensors or pointers."""
 
@@ -239,6 +264,23 @@ class Model:
 
     def set_stream(self, stream):
         check(em_set_stream(self.h, stream), "em_set_stream")
+
+    def dp_init(self, group=None):
+        """Data-parallel training over the ranks of a torch.distributed group (one
+        process per GPU): rank 0 makes the communicator id and the group broadcasts
+        it; the library then runs its own NCCL communicator."""
+        world, rank, uid = exchange_dp_id(group)
+        self.dp_init_id(world, rank, uid)
+
+    def dp_init_id(self, world, rank, uid: bytes):
+        """em_dp_init with an id already shared by the caller (every rank calls it)."""
+        buf = ctypes.create_string_buffer(bytes(uid), EM_NCCL_ID_BYTES)
+        check(em_dp_init(self.h, int(world), int(rank), ctypes.cast(buf, ctypes.c_void_p)), "em_dp_init")
+
+    def dp_world(self):
+        w, r = ctypes.c_int(), ctypes.c_int()
+        check(em_dp_world(self.h, ctypes.byref(w), ctypes.byref(r)), "em_dp_world")
+        return w.value, r.value
 
     def train(self, X, n=None, epochs=5.0):
         self._dtype_of(X)

@@ -24,6 +24,7 @@ NVCC_FLAGS = [
     "-O3", "-lineinfo", "-std=c++17",
     "-Xcompiler", "-fPIC", "-shared",
     "-Xptxas", "-O3",
+    "-ldl",
 ]
 
 

@@ -13,13 +13,23 @@
 //   k_revive_*      every 5th step: dead-cluster revival
 // No host synchronisation happens inside a run; the step size of step t is
 // computed on the host (cosine schedule) and passed by value.
+//
+// Data-parallel runs (README "Several GPUs": DistributedEmeans, one process per
+// GPU, each with its own share of the rows): every rank searches its share of each
+// batch and k_segsum / k_clusters leave its per-cluster statistics (n_j, s_j, in
+// fp64) instead of updating; one NCCL all-reduce adds them across ranks on the
+// model's stream, and k_apply_stats applies the same EMA on every rank. NCCL is
+// loaded at run time, only when a communicator is created.
 #include <algorithm>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <dlfcn.h>
 #include <mutex>
 #include <vector>
+
+#include <nccl.h>  // types and prototypes only: the library is loaded with dlopen
 
 #include "common.cuh"
 #include "k_assign.cuh"
@@ -105,6 +115,44 @@ static double alpha_at(int64_t t, int64_t total, double alpha0) {
     return amin + (alpha0 - amin) * 0.5 * (1.0 + cos(M_PI * frac));
 }
 
+// ------------------------------------------------------------------ NCCL (loaded on demand)
+
+struct NcclApi {
+    bool ok = false;
+    decltype(&ncclGetUniqueId) get_id = nullptr;
+    decltype(&ncclCommInitRank) init_rank = nullptr;
+    decltype(&ncclAllReduce) all_reduce = nullptr;
+    decltype(&ncclBroadcast) broadcast = nullptr;
+    decltype(&ncclCommDestroy) destroy = nullptr;
+    decltype(&ncclGetErrorString) error_string = nullptr;
+};
+
+// The process's libnccl.so.2 (the one already loaded, if any, else the first on the
+// library path).
+static const NcclApi& nccl() {
+    static NcclApi api;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* h = dlopen("libnccl.so.2", RTLD_NOW | RTLD_GLOBAL);
+        if (!h) h = dlopen("libnccl.so", RTLD_NOW | RTLD_GLOBAL);
+        if (!h) return;
+        api.get_id = reinterpret_cast<decltype(api.get_id)>(dlsym(h, "ncclGetUniqueId"));
+        api.init_rank = reinterpret_cast<decltype(api.init_rank)>(dlsym(h, "ncclCommInitRank"));
+        api.all_reduce = reinterpret_cast<decltype(api.all_reduce)>(dlsym(h, "ncclAllReduce"));
+        api.broadcast = reinterpret_cast<decltype(api.broadcast)>(dlsym(h, "ncclBroadcast"));
+        api.destroy = reinterpret_cast<decltype(api.destroy)>(dlsym(h, "ncclCommDestroy"));
+        api.error_string = reinterpret_cast<decltype(api.error_string)>(dlsym(h, "ncclGetErrorString"));
+        api.ok = api.get_id && api.init_rank && api.all_reduce && api.broadcast && api.destroy && api.error_string;
+    });
+    return api;
+}
+
+#define NCK(call)                                                                                  \
+    do {                                                                                           \
+        const ncclResult_t r_ = (call);                                                            \
+        if (r_ != ncclSuccess) return fail(EM_E_COMM, "%s: %s", #call, nccl().error_string(r_));   \
+    } while (0)
+
 // ------------------------------------------------------------------ tensor maps
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -183,6 +231,11 @@ struct em_model {
     int revival = EM_REVIVE_SPLIT, finalize = 1, law = 2, in_dtype = 0, check_finite = 0;
     int auto_revive = 1, capture = 1, graphs = 1, assign_kernel = 0, exact_ties = -1;
     int spherical = 0;  // spherical e-means: unit centroids, highest dot product
+    // data parallelism (em_dp_init): this rank's share of each batch, statistics
+    // added across ranks with NCCL
+    int dp_world = 1, dp_rank = 0;
+    ncclComm_t comm = nullptr;
+    DBuf<double> stats;  // k x ld sums, k counts, the error sum
     int last_split = 1;  // centroid-tile groups of the most recent search (keys per row)
     // state
     DBuf<float> N, N_prev, S, c, cn, cnp;
@@ -191,7 +244,8 @@ struct em_model {
     DBuf<int> err, flag;
     // data of the current run
     const __nv_bfloat16* X = nullptr;
-    int64_t n = 0;
+    int64_t n = 0;        // rows of a pass over all ranks (the recipe's n)
+    int64_t n_local = 0;  // rows in X (this rank's share in a data-parallel run)
     DBuf<__nv_bfloat16> Xown;
     DBuf<uint8_t> stage;  // host-input staging
     // batch buffers
@@ -523,7 +577,11 @@ static int launch_assign(em_model* m, const CUtensorMap& tmA, const __nv_bfloat1
 // ranks and counts are already in place. `src` holds the rows (batch or data).
 static int launch_reduce(em_model* m, const __nv_bfloat16* src, int64_t rows, int nblocks_labels, double alpha,
                          int last_pass, double* err_sum_out) {
-    const StepParams sp{alpha, last_pass, 0};
+    const bool dp = m->comm != nullptr;
+    double* const stats_err = m->stats.p + (int64_t)m->k * m->ld + m->k;
+    const StepParams sp{alpha, last_pass, 0, dp ? m->stats.p : nullptr};
+    double* const step_err = err_sum_out;
+    if (dp) err_sum_out = stats_err;  // the error sum travels with the statistics
     k_offsets<<<1, 1024, 0, m->stream>>>(m->cnt.p, (int)m->k, (int)rows, m->R, m->off.p, m->poff.p, m->block_err.p,
                                          nblocks_labels, err_sum_out, m->N.p, m->N_prev.p, tie_list(m), m->err.p);
     CK(cudaGetLastError());
@@ -540,6 +598,13 @@ static int launch_reduce(em_model* m, const __nv_bfloat16* src, int64_t rows, in
                                                                          m->nv, st, sp, m->part.p);
     CK(cudaGetLastError());
     EM_LAUNCHED(m, 4);
+    if (dp) {  // add the ranks' statistics, then the same update on every rank
+        NCK(nccl().all_reduce(m->stats.p, m->stats.p, (size_t)m->k * m->ld + m->k + 1, ncclFloat64, ncclSum, m->comm,
+                              m->stream));
+        k_apply_stats<<<grid_for(m->k * 32, 256, m->sms), 256, 0, m->stream>>>(nslices, m->nv, st, sp, step_err);
+        CK(cudaGetLastError());
+        EM_LAUNCHED(m, 1);
+    }
     return normalize_if_spherical(m);
 }
 
@@ -622,11 +687,17 @@ static bool prefetches(const em_model* m, int64_t t) {
     return m->prefetch && !m->profile && t + 1 < m->rec.total_steps;
 }
 
-// Gathers the rows of step p into slot p.t & 1 on `stream`.
+// Gathers this rank's rows of step p into slot p.t & 1 on `stream`. A rank takes
+// the positions [pos / world, (pos + rows) / world) of its own order of its own
+// rows; rank r's order is keyed by the pass plus r * 2^32 (rank 0: the single-GPU
+// order).
 static int launch_gather(em_model* m, const StepPlan& p, cudaStream_t stream) {
     em_model::BatchSlot& b = m->slot[p.t & 1];
-    k_gather<<<grid_for(p.rows, 128, m->sms), 128, 0, stream>>>(m->X, m->n, m->ld, m->seed, p.pass, p.pos,
-                                                               (int)p.rows, 0, b.X.p, b.xn.p, b.ids.p, m->err.p);
+    const int64_t rows = p.rows / m->dp_world;
+    const int64_t key = p.pass + ((int64_t)m->dp_rank << 32);
+    k_gather<<<grid_for(rows, 128, m->sms), 128, 0, stream>>>(m->X, m->n_local, m->ld, m->seed, key,
+                                                             p.pos / m->dp_world, (int)rows, 0, b.X.p, b.xn.p, b.ids.p,
+                                                             m->err.p);
     CK(cudaGetLastError());
     EM_LAUNCHED(m, 1);
     return EM_OK;
@@ -656,7 +727,7 @@ static int drop_prefetch(em_model* m) {
 
 static void advance_step(em_model* m, const StepPlan& p) {
     const int64_t rows_pass = (m->pass == m->rec.passes - 1) ? m->rec.rows_last_pass : m->n;
-    m->last_rows = p.rows;
+    m->last_rows = p.rows / m->dp_world;
     m->last_alpha = p.alpha;
     m->rows_assigned += p.rows;
     m->t += 1;
@@ -668,7 +739,7 @@ static void advance_step(em_model* m, const StepPlan& p) {
 }
 
 static int launch_step(em_model* m, const StepPlan& p) {
-    const int64_t rows = p.rows;
+    const int64_t rows = p.rows / m->dp_world;  // this rank's share
     const double rd = (double)rows, dd = (double)m->d, kd = (double)m->k;
     em_model::BatchSlot& b = m->slot[p.t & 1];
     int sp = span_begin(m, EM_PHASE_GATHER);
@@ -740,7 +811,8 @@ static std::vector<uint64_t> graph_signature(const em_model* m) {
     const int64_t ints[] = {m->n, m->d, m->k, m->ld, m->kc, m->R, m->sms, m->rec.batch_size, m->rec.total_steps,
                             m->rec.passes, m->rec.rows_last_pass, (int64_t)m->seed, m->revival, m->finalize,
                             m->capture, m->auto_revive, m->assign_kernel, m->wait_cycles, m->exact_ties,
-                            m->spherical, m->prefetch};
+                            m->spherical, m->prefetch, m->n_local, m->dp_world, m->dp_rank,
+                            (int64_t)(uintptr_t)m->comm, (int64_t)(uintptr_t)m->stats.p};
     for (int64_t v : ints) sig.push_back((uint64_t)v);
     double dbl[] = {m->rec.alpha0, m->tau};
     for (double v : dbl) {
@@ -832,7 +904,7 @@ static int normalize_if_spherical(em_model* m) {
 
 static int start_centroids(em_model* m) {
     k_init_centroids<<<grid_for(m->k * 32, 256, m->sms), 256, 0, m->stream>>>(
-        m->X, m->n, m->ld, (int)m->k, m->seed, m->c.p, m->S.p, m->N.p, m->cq.p, m->cn.p, m->err.p);
+        m->X, m->n_local, m->ld, (int)m->k, m->seed, m->c.p, m->S.p, m->N.p, m->cq.p, m->cn.p, m->err.p);
     CK(cudaGetLastError());
     EM_LAUNCHED(m, 1);
     return normalize_if_spherical(m);
@@ -959,14 +1031,15 @@ void em_destroy(em_model* m) {
     m->part.release(); m->step_err.release(); m->scalar.release(); m->labels_last.release();
     m->labels64.release(); m->rv_dead.release(); m->rv_donor.release(); m->rv_order.release();
     m->rv_times.release(); m->rv_ndead.release(); m->rv_tree.release(); m->rv_splits.release();
-    m->ties.release(); m->tie_n.release(); m->tie_corr.release();
+    m->ties.release(); m->tie_n.release(); m->tie_corr.release(); m->stats.release();
     m->rv_target.release();
     for (auto& sp : m->pending) {
         cudaEventDestroy(sp.a);
         cudaEventDestroy(sp.b);
     }
     for (auto ev : m->pool) cudaEventDestroy(ev);
-    for (auto& g : m->graph_cache) cudaGraphExecDestroy(g.exec);
+    for (auto& g : m->graph_cache) cudaGraphExecDestroy(g.exec);  // graphs may hold NCCL calls
+    if (m->comm) nccl().destroy(m->comm);
     if (m->cap_stream) cudaStreamDestroy(m->cap_stream);
     if (m->side_cap) cudaStreamDestroy(m->side_cap);
     if (m->side) cudaStreamDestroy(m->side);
@@ -1081,13 +1154,25 @@ int em_begin(em_model* m, const void* X, int64_t n, double epochs) {
     if (n >= (1ll << 31)) return fail(EM_E_INVAL, "n must be below 2^31");
     if (!(epochs > 0.0)) return fail(EM_E_INVAL, "epochs must be positive");
     CKR(set_device(m));
-    CKR(compute_recipe(n, m->k, m->d, epochs, effective_law(m), m->opt_batch, m->opt_alpha0, &m->rec));
-    if (m->rec.batch_size > n) return fail(EM_E_INVAL, "batch size larger than n");
+    // a data-parallel run: n is this rank's share, the recipe is the whole job's
+    const int64_t W = m->dp_world, n_total = n * W;
+    if (n_total >= (1ll << 31)) return fail(EM_E_INVAL, "the rows of all ranks must be below 2^31");
+    CKR(compute_recipe(n_total, m->k, m->d, epochs, effective_law(m), m->opt_batch, m->opt_alpha0, &m->rec));
+    if (m->rec.batch_size > n_total) return fail(EM_E_INVAL, "batch size larger than n");
+    if (W > 1) {  // README "Several GPUs": the batch and the rows of every pass divide by the ranks
+        if (m->rec.batch_size % W || m->rec.rows_last_pass % W)
+            return fail(EM_E_INVAL, "the batch (%lld rows) and the rows of every pass (last: %lld) must divide by "
+                                    "the number of ranks (%lld)",
+                        (long long)m->rec.batch_size, (long long)m->rec.rows_last_pass, (long long)W);
+        if (m->revival == EM_REVIVE_RESAMPLE)
+            return fail(EM_E_INVAL, "resampling draws rows of the whole batch; use it with one rank");
+    }
     m->running = false;
-    m->n = n;
+    m->n = n_total;
+    m->n_local = n;
     const int sp = span_begin(m, EM_PHASE_PREPARE);
     CKR(prepare_input(m, X, n, m->Xown, &m->X));
-    const int64_t b = m->rec.batch_size;
+    const int64_t b = m->rec.batch_size / W;  // this rank's rows of a full batch
     CKR(drop_prefetch(m));
     CK(cudaStreamSynchronize(m->stream));  // no gather of a previous run still writes the slots
     for (auto& bs : m->slot) {
@@ -1098,7 +1183,8 @@ int em_begin(em_model* m, const void* X, int64_t n, double epochs) {
     }
     CKR(ensure_batch_buffers(m, b));
     {  // every batch size the run will see: full batches and the last, partial ones
-        const int64_t sizes[3] = {b, n % b, m->rec.rows_last_pass % b};
+        const int64_t B = m->rec.batch_size;
+        const int64_t sizes[3] = {b, (n_total % B) / W, (m->rec.rows_last_pass % B) / W};
         size_t need = 0;
         for (int64_t r : sizes) need = std::max(need, keys_needed(m, r));
         CKR(m->keys.ensure(need));
@@ -1114,7 +1200,14 @@ int em_begin(em_model* m, const void* X, int64_t n, double epochs) {
         CKR(m->labels_last.ensure(n));
         CK(cudaMemsetAsync(m->labels_last.p, 0xFF, n * sizeof(int64_t), m->stream));
     }
+    if (m->comm) CKR(m->stats.ensure((size_t)m->k * m->ld + m->k + 1));
     CKR(start_centroids(m));
+    if (m->comm && W > 1) {  // README "Several GPUs": rank 0's starting centroids are used
+        const size_t kd = (size_t)m->k * m->ld;
+        NCK(nccl().broadcast(m->c.p, m->c.p, kd, ncclFloat32, 0, m->comm, m->stream));
+        NCK(nccl().broadcast(m->cq.p, m->cq.p, kd * sizeof(__nv_bfloat16), ncclUint8, 0, m->comm, m->stream));
+        NCK(nccl().broadcast(m->cn.p, m->cn.p, (size_t)m->k, ncclFloat32, 0, m->comm, m->stream));
+    }
     span_end(m, sp);
     m->t = m->pass = m->pos = m->rows_assigned = 0;
     m->last_rows = 0;
@@ -1177,12 +1270,20 @@ int em_lloyd(em_model* m, const void* X, int64_t n, int64_t iters) {
     CKR(set_device(m));
     CKR(drop_prefetch(m));
     m->running = false;
-    m->n = n;
+    m->n_local = n;
+    m->n = n * m->dp_world;  // data-parallel: every rank's rows, one summed update per iteration
     CKR(prepare_input(m, X, n, m->Xown, &m->X));
     CKR(ensure_batch_buffers(m, n));
+    if (m->comm) CKR(m->stats.ensure((size_t)m->k * m->ld + m->k + 1));
     CKR(m->keys.ensure(keys_needed(m, n)));
     CK(cudaMemsetAsync(m->cnt.p, 0, m->k * sizeof(int32_t), m->stream));
     CKR(start_centroids(m));
+    if (m->comm && m->dp_world > 1) {  // rank 0's starting rows
+        const size_t kd = (size_t)m->k * m->ld;
+        NCK(nccl().broadcast(m->c.p, m->c.p, kd, ncclFloat32, 0, m->comm, m->stream));
+        NCK(nccl().broadcast(m->cq.p, m->cq.p, kd * sizeof(__nv_bfloat16), ncclUint8, 0, m->comm, m->stream));
+        NCK(nccl().broadcast(m->cn.p, m->cn.p, (size_t)m->k, ncclFloat32, 0, m->comm, m->stream));
+    }
     CUtensorMap tmx;
     CKR(make_tmap(&tmx, m->X, n, (int)m->d, m->ld, tc::BM, m->kc));
     const int nbl = (int)((n + 255) / 256);
@@ -1308,7 +1409,7 @@ int em_labels(const em_model* m, int64_t* out) {
     if (!m || !out) return fail(EM_E_INVAL, "NULL argument");
     if (!m->capture || !m->labels_last.p || m->last_was_lloyd) return fail(EM_E_STATE, "no captured labels");
     CKR(set_device(m));
-    CK(cudaMemcpyAsync(out, m->labels_last.p, m->n * sizeof(int64_t), cudaMemcpyDefault, m->stream));
+    CK(cudaMemcpyAsync(out, m->labels_last.p, m->n_local * sizeof(int64_t), cudaMemcpyDefault, m->stream));
     CK(cudaStreamSynchronize(m->stream));
     return EM_OK;
 }
@@ -1463,6 +1564,43 @@ int em_profile(em_model* m, em_profile_t* out, int reset) {
         m->totals = em_profile_t{};
         m->launches = 0;
     }
+    return EM_OK;
+}
+
+int em_dp_unique_id(void* id_out) {
+    if (!id_out) return fail(EM_E_INVAL, "NULL argument");
+    if (!nccl().ok) return fail(EM_E_COMM, "libnccl.so.2 could not be loaded");
+    NCK(nccl().get_id(reinterpret_cast<ncclUniqueId*>(id_out)));
+    return EM_OK;
+}
+
+int em_dp_init(em_model* m, int world, int rank, const void* id) {
+    if (!m || !id) return fail(EM_E_INVAL, "NULL argument");
+    if (world < 1 || rank < 0 || rank >= world) return fail(EM_E_INVAL, "need 0 <= rank < world");
+    if (m->running) return fail(EM_E_STATE, "a run is in progress");
+    if (!nccl().ok) return fail(EM_E_COMM, "libnccl.so.2 could not be loaded");
+    CKR(set_device(m));
+    CKR(drop_prefetch(m));
+    CK(cudaStreamSynchronize(m->stream));
+    for (auto& g : m->graph_cache) cudaGraphExecDestroy(g.exec);
+    m->graph_cache.clear();
+    if (m->comm) {
+        nccl().destroy(m->comm);
+        m->comm = nullptr;
+    }
+    ncclUniqueId uid;
+    memcpy(&uid, id, sizeof(uid));
+    NCK(nccl().init_rank(&m->comm, world, uid, rank));
+    m->dp_world = world;
+    m->dp_rank = rank;
+    m->have_run = false;
+    return EM_OK;
+}
+
+int em_dp_world(const em_model* m, int* world, int* rank) {
+    if (!m) return fail(EM_E_INVAL, "model is NULL");
+    if (world) *world = m->dp_world;
+    if (rank) *rank = m->dp_rank;
     return EM_OK;
 }
 

@@ -32,6 +32,11 @@ struct StepParams {
     double alpha;        // step size of this step
     int last_pass;       // accumulate the closing-mean statistics
     int capture_labels;  // record the last-pass label of each row
+    // Data-parallel steps: instead of updating the clusters, the sums leave this
+    // rank's batch statistics in stats (k x ld fp64 sums s_j, then k counts n_j,
+    // then the error sum), to be added across ranks before k_apply_stats. nullptr:
+    // the update is applied here.
+    double* stats;
 };
 
 // ---------------------------------------------------------------- labels + histogram
@@ -503,7 +508,14 @@ __global__ void __launch_bounds__(256, 3) k_segsum(const __nv_bfloat16* __restri
     }
     double acc[8];
     sum_rows(acc, src, st.ld, perm, it.y, it.z, g, lane);
-    if (it.w) {
+    if (it.w && sp.stats) {  // this rank's sums of the cluster, for the exchange
+        if (lane < g.nvs) {
+            double* dst = sp.stats + (int64_t)j * st.ld + 8 * (g.vbase + lane);
+#pragma unroll
+            for (int t = 0; t < 8; ++t) dst[t] = acc[t];
+        }
+        if (lane == 0 && slice == 0) sp.stats[(int64_t)st.k * st.ld + j] = (double)n;
+    } else if (it.w) {
         const float cn_part = ema_slice(st, j, (double)n, nprev, slice, g, acc, so, lane, sp.alpha, sp.last_pass);
         if (lane == 0) st.cnp[(int64_t)slice * st.k + j] = cn_part;
     } else if (lane < g.nvs) {
@@ -528,6 +540,33 @@ __global__ void k_clusters(const int32_t* __restrict__ off, const int32_t* __res
     for (int j = warp; j < st.k; j += nwarps) {
         const int nj = off[j + 1] - off[j];
         if (lane == 0) cnt[j] = 0;
+        if (sp.stats) {  // this rank's statistics of cluster j, for the exchange
+            double* row = sp.stats + (int64_t)j * st.ld;
+            if (nj == 0) {
+                for (int v = lane; v < st.ld / 4; v += 32)
+                    reinterpret_cast<double4*>(row)[v] = make_double4(0.0, 0.0, 0.0, 0.0);
+                if (lane == 0) sp.stats[(int64_t)st.k * st.ld + j] = 0.0;
+            } else if (nj > R) {
+                const int p0 = poff[j], p1 = poff[j + 1];
+                for (int slice = 0; slice < nslices; ++slice) {
+                    const SliceGeom g = slice_geom(slice, nv);
+                    if (lane < g.nvs) {
+                        double acc[8];
+#pragma unroll
+                        for (int t = 0; t < 8; ++t) acc[t] = 0.0;
+                        const double* base = part + 8 * (g.vbase + lane);
+                        for (int p = p0; p < p1; ++p)
+#pragma unroll
+                            for (int t = 0; t < 8; ++t) acc[t] += base[(int64_t)p * st.ld + t];
+                        double* dst = row + 8 * (g.vbase + lane);
+#pragma unroll
+                        for (int t = 0; t < 8; ++t) dst[t] = acc[t];
+                    }
+                }
+                if (lane == 0) sp.stats[(int64_t)st.k * st.ld + j] = (double)nj;
+            }
+            continue;
+        }
         if (nj == 0) {
             float4* row = reinterpret_cast<float4*>(st.S + (int64_t)j * st.ld);
             for (int v = lane; v < st.ld / 4; v += 32) {
@@ -575,6 +614,47 @@ __global__ void k_clusters(const int32_t* __restrict__ off, const int32_t* __res
             }
             if (lane == 0) st.cn[j] = cn_total;
         }
+    }
+}
+
+// Data-parallel steps, after the ranks have added their statistics: one warp per
+// cluster applies the EMA from the summed (n_j, s_j), with the same arithmetic as
+// the single-GPU update (a cluster without rows decays; the others go through
+// ema_slice slice by slice), and thread 0 stores the summed error of the step.
+__global__ void k_apply_stats(int nslices, int nv, ClusterState st, StepParams sp, double* __restrict__ err_out) {
+    const int lane = threadIdx.x & 31;
+    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int nwarps = (gridDim.x * blockDim.x) >> 5;
+    const double a1 = 1.0 - sp.alpha;
+    const double* nsum = sp.stats + (int64_t)st.k * st.ld;
+    if (blockIdx.x == 0 && threadIdx.x == 0) *err_out = nsum[st.k];
+    for (int j = warp; j < st.k; j += nwarps) {
+        const double nj = nsum[j];
+        if (nj == 0.0) {
+            float4* row = reinterpret_cast<float4*>(st.S + (int64_t)j * st.ld);
+            for (int v = lane; v < st.ld / 4; v += 32) {
+                const float4 x = row[v];
+                row[v] = make_float4((float)(a1 * (double)x.x), (float)(a1 * (double)x.y), (float)(a1 * (double)x.z),
+                                     (float)(a1 * (double)x.w));
+            }
+            if (lane == 0) st.N[j] = (float)(a1 * (double)st.N_prev[j]);
+            continue;
+        }
+        const float nprev = st.N_prev[j];
+        float cn_total = 0.0f;
+        for (int slice = 0; slice < nslices; ++slice) {
+            const SliceGeom g = slice_geom(slice, nv);
+            float so[8];
+            load_s(st, j, g, lane, so);
+            double acc[8];
+            if (lane < g.nvs) {
+                const double* src = sp.stats + (int64_t)j * st.ld + 8 * (g.vbase + lane);
+#pragma unroll
+                for (int t = 0; t < 8; ++t) acc[t] = src[t];
+            }
+            cn_total += ema_slice(st, j, nj, nprev, slice, g, acc, so, lane, sp.alpha, sp.last_pass);
+        }
+        if (lane == 0) st.cn[j] = cn_total;
     }
 }
 

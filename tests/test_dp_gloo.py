@@ -103,3 +103,54 @@ def test_bench_aggregates_max_time_and_total_rows(tmp_path):
     for r in range(world):
         ms_max, rows_all = np.load(tmp_path / f"agg{r}.npy")
         assert ms_max == 17.25 and rows_all == 2500
+
+
+def _id_worker(rank, world, port, out_dir):
+    _init(rank, world, port)
+    try:
+        import mini_ema_means_b200 as em
+
+        w, r, uid = em.exchange_dp_id()
+        assert (w, r) == (world, rank) and len(uid) == em.EM_NCCL_ID_BYTES
+        with open(os.path.join(out_dir, f"id{rank}.bin"), "wb") as f:
+            f.write(uid)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_communicator_id_reaches_every_rank(tmp_path, em_lib):
+    """Model.dp_init's first half on two gloo ranks: rank 0 makes the NCCL id (host
+    code of the library) and every rank receives the same bytes."""
+    world = 2
+    mp.spawn(_id_worker, args=(world, _free_port(), str(tmp_path)), nprocs=world, join=True)
+    ids = [open(tmp_path / f"id{r}.bin", "rb").read() for r in range(world)]
+    assert ids[0] == ids[1] and len(ids[0]) == 128 and any(ids[0])
+
+
+@pytest.fixture(scope="module")
+def em_lib():
+    import importlib.util
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    spec = importlib.util.spec_from_file_location("_b", os.path.join(root, "mini_ema_means_b200", "build.py"))
+    b = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(b)
+    b.build()
+    import mini_ema_means_b200
+
+    return mini_ema_means_b200
+
+
+def test_rank_orders_are_the_oracles_bijections(em_lib):
+    """A data-parallel rank r walks its own rows in the library's order keyed by
+    pass + r * 2^32 (rank 0: the single-GPU order); the host code of that order is
+    the oracle's bijection for those keys too."""
+    em = em_lib
+    n = 7001
+    idx = np.arange(n, dtype=np.int64)
+    for rank, p in ((0, 0), (1, 0), (3, 2)):
+        which = p + (rank << 32)
+        lib = em.permutation(n, 1234, 2, which, idx)
+        assert np.array_equal(lib, O.pass_order(n, 1234, which))
+        assert np.array_equal(np.sort(lib), idx)
+    assert not np.array_equal(em.permutation(n, 1234, 2, 1 << 32, idx), em.permutation(n, 1234, 2, 0, idx))
