@@ -39,7 +39,11 @@ R9  resample: c_j <- a uniformly drawn row of the current batch, N_j = S_j = 0;
 R10 Lloyd mode: B = n, alpha = 1, natural row order, no revival;
 R11 reported distances and MSE use the bf16 search operands, clamped at 0;
 R12 closing mean: clusters without points in the last pass keep their EMA
-    centroid.
+    centroid;
+R13 FP8 search: the converter's shift is each dimension's midrange and its scale
+    the largest power of two keeping the sample within 448, fitted on the first
+    65,536 rows of the bf16 search copy; rows and centroids are encoded from their
+    bf16 / fp32 values; the running sums stay those of the bf16 rows.
 
 Random draws (starting rows, per-pass order, donor draws, resample rows) come
 from the counter-based generator Philox4x64-10 (Salmon, Moraes, Dror, Shaw,
@@ -108,6 +112,93 @@ def search_copy_of_data(x) -> np.ndarray:
 def search_copy_of_centroids(c64) -> np.ndarray:
     """fp64 centroids -> fp32 (the stored format) -> bf16 (the search format)."""
     return f32_to_bf16(to_f32(c64)).astype(np.float64)
+
+
+# --------------------------------------------------------------------------
+# FP8 search ([README] "Data precision": an FP8 (E4M3) converter calibrated on a
+# sample, with a shift per dimension and one power-of-two scale; values beyond
+# the range clamp to the edge, 448 for FP8; only the search uses the format)
+# --------------------------------------------------------------------------
+
+E4M3_MAX = 448.0
+FP8_CALIBRATION_ROWS = 65536
+
+
+def e4m3_table() -> np.ndarray:
+    """Values of the 127 non-negative finite E4M3 codes 0x00..0x7E, in code order.
+
+    E4M3 (the OCP 8-bit float with 4 exponent bits, bias 7, 3 mantissa bits, no
+    infinities): exponent field 0 holds the subnormals m/8 * 2^-6; fields 1..15
+    hold (1 + m/8) * 2^(e - 7), except that field 15 with mantissa 7 is NaN, so
+    the largest value is 1.75 * 2^8 = 448.
+    """
+    vals = []
+    for code in range(127):
+        e, m = code >> 3, code & 7
+        vals.append(m / 8.0 * 2.0 ** -6 if e == 0 else (1.0 + m / 8.0) * 2.0 ** (e - 7))
+    return np.array(vals)
+
+
+def e4m3_round(v) -> np.ndarray:
+    """Each value rounded to E4M3, nearest with ties to the even code, saturating at
+    +-448 (a finite value beyond it clamps); returned as fp64 values."""
+    v = np.asarray(v, dtype=np.float64)
+    tab = e4m3_table()
+    a = np.minimum(np.abs(v), E4M3_MAX)
+    hi = np.clip(np.searchsorted(tab, a, side="left"), 0, len(tab) - 1)  # first value >= a
+    lo = np.maximum(hi - 1, 0)
+    d_lo, d_hi = a - tab[lo], tab[hi] - a
+    pick_hi = (d_hi < d_lo) | ((d_hi == d_lo) & (hi % 2 == 0))
+    r = np.where(a == tab[hi], tab[hi], np.where(pick_hi, tab[hi], tab[lo]))
+    return np.copysign(r, v)
+
+
+def fp8_calibrate(xq: np.ndarray):
+    """(shift, scale) of the FP8 converter, fitted on the first FP8_CALIBRATION_ROWS
+    rows of the search copy: the shift is each dimension's midrange, computed in
+    fp32 ((min + max) / 2), and the scale the largest power of two that keeps
+    the largest |x - shift| of the sample within 448 (1 when the sample is constant)."""
+    sample = np.asarray(xq[:FP8_CALIBRATION_ROWS], dtype=np.float32)
+    lo, hi = sample.min(axis=0), sample.max(axis=0)
+    shift = ((lo + hi) * np.float32(0.5)).astype(np.float32)
+    half = np.maximum(hi - shift, shift - lo).astype(np.float64)
+    m = float(half.max()) if half.size else 0.0
+    if not m > 0.0:
+        return shift, 1.0
+    e = math.floor(math.log2(E4M3_MAX / m))
+    while m * 2.0 ** e > E4M3_MAX:  # guard the floating-point log
+        e -= 1
+    while m * 2.0 ** (e + 1) <= E4M3_MAX:
+        e += 1
+    return shift, 2.0 ** e
+
+
+def fp8_codes(v, shift, scale) -> np.ndarray:
+    """E4M3 codes of (v - shift) * scale, as fp64 values: the subtraction in fp32
+    (the stored format of the shift), the power-of-two scaling exact, then one
+    rounding to E4M3."""
+    d32 = np.asarray(v, dtype=np.float32) - np.asarray(shift, dtype=np.float32)
+    return e4m3_round(d32.astype(np.float64) * scale)
+
+
+def fp8_search_copy_of_centroids(c64, shift, scale) -> np.ndarray:
+    """fp64 centroids -> fp32 (the stored format) -> FP8 codes."""
+    return fp8_codes(to_f32(c64), shift, scale)
+
+
+def mse_fp8(xq: np.ndarray, c64: np.ndarray, shift, scale) -> float:
+    """Mean squared distance to the nearest centroid with the FP8 search (data units)."""
+    return float(assign_fp8(xq, c64, shift, scale)[1].mean())
+
+
+def assign_fp8(xq: np.ndarray, c64: np.ndarray, shift, scale):
+    """Nearest centroid of each row with the FP8 search: the argmin of |x' - c'|^2
+    over the codes (fp64, ties to the lowest index), reported as squared distances
+    in the data's units, |x' - c'|^2 / scale^2. Returns (labels, best, second)."""
+    xc = fp8_codes(xq, shift, scale)
+    cc = fp8_search_copy_of_centroids(c64, shift, scale)
+    labels, best, second = assign(xc, cc)
+    return labels, best / scale ** 2, second / scale ** 2
 
 
 # --------------------------------------------------------------------------
@@ -433,9 +524,15 @@ class EmeansOracle:
     """e-means in fp64 on the bf16 search copy of the data."""
 
     def __init__(self, d, k, seed=1234, revival="split", tau=None, closing_mean=True,
-                 law="auto", batch_size=None, alpha0=None, spherical=False):
+                 law="auto", batch_size=None, alpha0=None, spherical=False, search="bf16"):
         self.d, self.k, self.seed = int(d), int(k), int(seed)
         self.spherical = bool(spherical)
+        if search not in ("bf16", "fp8"):
+            raise ValueError(search)
+        if search == "fp8" and self.spherical:  # [README] "Spherical e-means": 32- and 16-bit floats only
+            raise ValueError("spherical e-means does not take the FP8 search")
+        self.search = search
+        self.fp8 = None  # (shift, scale) of the FP8 converter, fitted at begin
         # defaults that depend on the dimension ([README] `batch_law`, `unused_threshold`
         # and "Note on low dimension"): the quality batch law for d <= 16, no revival
         # (threshold 0) for d <= 2
@@ -455,6 +552,8 @@ class EmeansOracle:
         self.xq = xq
         self.n = n
         self.r = recipe(n, self.k, epochs, self.law, self.batch_override, self.alpha_override)
+        if self.search == "fp8":
+            self.fp8 = fp8_calibrate(xq)
         rows = starting_rows(n, self.k, self.seed) if start_rows is None else np.asarray(start_rows)
         self.c = xq[rows].copy()
         if self.spherical:
@@ -491,6 +590,8 @@ class EmeansOracle:
         if self.spherical:  # highest similarity; the error of a row is 2 - 2 x similarity
             labels, sim, sim2 = assign_dot(xb, search_copy_of_centroids(self.c))
             best, second = 2.0 - 2.0 * sim, 2.0 - 2.0 * sim2
+        elif self.search == "fp8":
+            labels, best, second = assign_fp8(xb, self.c, *self.fp8)
         else:
             labels, best, second = assign(xb, search_copy_of_centroids(self.c))
         used = labels if forced_labels is None else np.asarray(forced_labels, dtype=np.int64)
@@ -548,7 +649,7 @@ class EmeansOracle:
         return self.finalize(), self.labels_last
 
 
-def lloyd(xq: np.ndarray, c0: np.ndarray, iters: int, spherical: bool = False):
+def lloyd(xq: np.ndarray, c0: np.ndarray, iters: int, spherical: bool = False, fp8=None):
     """Lloyd's k-means as the B = n, alpha = 1 case of the same update ([README]
     "How the centroid updates work"; [Blog] "Lloyd is a special case"); spherical:
     highest similarity, centroids rescaled to norm 1 ([README] "Spherical e-means")."""
@@ -559,6 +660,9 @@ def lloyd(xq: np.ndarray, c0: np.ndarray, iters: int, spherical: bool = False):
         if spherical:
             labels, sim, _ = assign_dot(xq, search_copy_of_centroids(c))
             history.append(float((2.0 - 2.0 * sim).mean()))
+        elif fp8 is not None:  # the FP8 search with the converter (shift, scale)
+            labels, best, _ = assign_fp8(xq, c, *fp8)
+            history.append(float(best.mean()))
         else:
             labels, best, _ = assign(xq, search_copy_of_centroids(c))
             history.append(float(best.mean()))

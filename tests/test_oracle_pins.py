@@ -562,3 +562,101 @@ def test_spherical_run_keeps_unit_centroids_and_error_definition():
     assert err == pytest.approx(float(np.mean(2.0 - 2.0 * sim))) and 0.0 <= err < 2.0
     # it clusters: far below the error of one random unit centroid per row (about 2)
     assert err < 1.0
+
+
+# ---------------------------------------------------------------- FP8 search
+
+def test_e4m3_table_fixed_points():
+    """E4M3 (OCP 8-bit float, 4 exponent bits, bias 7, no infinities): 1.0 is
+    0x38, the largest value 448 is 0x7E, the smallest subnormal 2^-9 is 0x01 and
+    the smallest normal 2^-6 is 0x08; values grow with the code."""
+    t = O.e4m3_table()
+    assert len(t) == 127 and np.all(np.diff(t) > 0)
+    assert t[0x38] == 1.0 and t[0x7E] == 448.0 and t[0x01] == 2.0 ** -9 and t[0x08] == 2.0 ** -6
+    assert t[0x07] == 7.0 / 8.0 * 2.0 ** -6 and t[0x7D] == 416.0
+
+
+def test_e4m3_rounding_matches_torch_and_breaks_ties_to_even():
+    """Nearest rounding against torch's float8_e4m3fn cast (an independent library
+    routine) on in-range values, every exact midpoint between neighbouring codes
+    going to the even code, and saturation of finite values beyond 448."""
+    g = np.random.default_rng(12)
+    x = np.concatenate([g.standard_normal(20000) * 60.0, g.standard_normal(5000) * 1e-2,
+                        g.uniform(-448, 448, 5000)])
+    ref = torch.tensor(x).to(torch.float8_e4m3fn).to(torch.float64).numpy()
+    assert np.array_equal(O.e4m3_round(x), ref)
+    t = O.e4m3_table()
+    mids = (t[:-1] + t[1:]) / 2.0
+    got = O.e4m3_round(mids)
+    codes = np.searchsorted(t, got)
+    assert np.all(codes % 2 == 0) and np.all(t[codes] == got)
+    assert np.array_equal(O.e4m3_round(-mids), -got)
+    assert np.array_equal(O.e4m3_round([449.0, 463.9, 1e6, -5000.0]), [448.0, 448.0, 448.0, -448.0])
+
+
+def test_fp8_calibration_is_midrange_shift_and_largest_power_of_two():
+    g = np.random.default_rng(13)
+    x = O.search_copy_of_data(g.standard_normal((3000, 9)) * np.arange(1, 10) + np.arange(9) * 5.0)
+    shift, scale = O.fp8_calibrate(x)
+    lo, hi = x.min(axis=0), x.max(axis=0)
+    assert np.array_equal(shift, ((lo.astype(np.float32) + hi.astype(np.float32)) * np.float32(0.5)))
+    m = np.maximum(hi - shift, shift - lo).max()
+    assert math.log2(scale) == int(math.log2(scale))
+    assert m * scale <= 448.0 < m * scale * 2.0
+    # only the first rows calibrate; a constant sample keeps scale 1
+    big = np.vstack([x, np.full((1, 9), 1e9)])
+    assert O.fp8_calibrate(big[: len(x)])[1] == scale
+    assert O.fp8_calibrate(np.ones((10, 3)))[1] == 1.0
+
+
+def test_fp8_search_is_the_argmin_over_codes():
+    """Brute force on tiny inputs: the FP8 search picks the centroid whose codes are
+    nearest to the row's codes (ties to the lowest index), and reports that
+    squared distance divided by scale^2."""
+    g = np.random.default_rng(14)
+    x = O.search_copy_of_data(g.standard_normal((40, 5)) * 3.0)
+    c = g.standard_normal((7, 5)) * 3.0
+    shift, scale = O.fp8_calibrate(x)
+    lab, best, _ = O.assign_fp8(x, c, shift, scale)
+    xc, cc = O.fp8_codes(x, shift, scale), O.fp8_codes(O.to_f32(c), shift, scale)
+    for i in range(40):
+        d = [float(((xc[i] - cc[j]) ** 2).sum()) for j in range(7)]
+        assert lab[i] == d.index(min(d)) and best[i] == min(d) / scale ** 2
+
+
+def test_fp8_distances_within_the_quantisation_bound():
+    """Each code is within half an E4M3 step (relative 2^-4, or 2^-10 among the
+    subnormals) of a = (x - shift) * scale. By the triangle inequality the FP8
+    distance |x' - c'| of a row to a centroid is then within |x' - a| + |c' - b| of
+    |a - b|; on separated clusters the FP8 and bf16 searches pick the same labels."""
+    g = np.random.default_rng(15)
+    mu = g.standard_normal((6, 16)) * 20.0
+    x = O.search_copy_of_data(mu[g.integers(6, size=2000)] + g.standard_normal((2000, 16)))
+    shift, scale = O.fp8_calibrate(x)
+    xc = O.fp8_codes(x, shift, scale)
+    a = (x.astype(np.float32) - shift).astype(np.float64) * scale
+    assert np.all(np.abs(xc - a) <= np.maximum(np.abs(a) * 2.0 ** -4, 2.0 ** -10) + 1e-12)
+    lab8, best8, _ = O.assign_fp8(x, mu, shift, scale)
+    lab, _, _ = O.assign(x, O.search_copy_of_centroids(mu))
+    assert np.mean(lab8 == lab) == 1.0
+    cc = O.fp8_codes(O.to_f32(mu), shift, scale)
+    b = (O.to_f32(mu) - shift).astype(np.float64) * scale
+    ex, ec = np.linalg.norm(xc - a, axis=1), np.linalg.norm(cc - b, axis=1)
+    d_exact = np.linalg.norm(a - b[lab8], axis=1)
+    assert np.all(np.abs(np.sqrt(best8) * scale - d_exact) <= ex + ec[lab8] + 1e-9)
+
+
+def test_fp8_training_run_clusters_like_bf16():
+    """An FP8-search run of the oracle on separated clusters ends near the bf16
+    run (same rows, same seed): the search precision is the only change."""
+    g = np.random.default_rng(16)
+    mu = g.standard_normal((12, 8)) * 10.0
+    x = O.search_copy_of_data(mu[g.integers(12, size=6000)] + g.standard_normal((6000, 8)))
+    e8 = O.EmeansOracle(8, 16, seed=3, search="fp8")
+    e16 = O.EmeansOracle(8, 16, seed=3)
+    c8, _ = e8.train(x, 2.0)
+    c16, _ = e16.train(x, 2.0)
+    assert e8.fp8 is not None and e16.fp8 is None
+    assert abs(O.mse(x, c8) - O.mse(x, c16)) <= 0.05 * O.mse(x, c16)
+    with pytest.raises(ValueError):
+        O.EmeansOracle(8, 16, spherical=True, search="fp8")
