@@ -204,7 +204,8 @@ def run_ours(args, rank, world):
     torch.cuda.synchronize()
     log(f"[rank {rank}] data {w.name} ready in {time.time() - t0:.1f} s")
     stream = torch.cuda.current_stream(dev)
-    m = em.Model(w.d, w.k, seed=1234, spherical=int(args.spherical), prefetch=args.prefetch)
+    m = em.Model(w.d, w.k, seed=1234, spherical=int(args.spherical), prefetch=args.prefetch,
+                 search_format=args.search)
     m.set_stream(stream.cuda_stream)
     if args.dp:
         dp_join(em, m, world)
@@ -281,8 +282,9 @@ def run_ours(args, rank, world):
     out = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "vs_baseline": None, "dtype": "e4m3" if args.search == "fp8" else "bf16", "data": "synthetic",
         "config": {"workload": workload_desc(w), "method": "spherical e-means" if args.spherical else "e-means",
+                   "search": args.search,
                    "batch_size": rec["batch_size"], "alpha0": round(rec["alpha0"], 6), "prefetch": args.prefetch,
                    "steps_per_run": total,
                    "l2": "inputs larger than L2: the fp32 training matrix (%.2f GB) and its bf16 copy are re-read "
@@ -294,14 +296,20 @@ def run_ours(args, rank, world):
     a_ms = prof["ms"]["assign"]
     a_n = max(prof["spans"]["assign"], 1)
     achieved = prof["assign_flops"] / (a_ms / 1e3) / 1e12 if a_ms > 0 else 0.0
-    peak = peaks["bf16_tflops"]
+    # an E4M3 contraction takes the measured bf16 peak x the nominal fp8 / bf16 ratio (4.5 / 2.25)
+    ratio = 2.0 if args.search == "fp8" else 1.0
+    peak = peaks["bf16_tflops"] * ratio
     out["roofline"] = {
         "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
         "frac": achieved / peak,
-        "traffic": args.traffic if args.traffic is not None else ASSIGN_TRAFFIC.get(args.workload),
-        "kernel": "k_assign_tc (tcgen05 bf16 x bf16 -> fp32, fused |c|^2 add + row argmin)",
-        "peak_source": f"{peaks['source']} bf16 burst",
-        "frac_of_sustained": achieved / peaks["bf16_tflops_sustained"] if peaks.get("bf16_tflops_sustained") else None,
+        "traffic": (args.traffic if args.traffic is not None
+                    else ASSIGN_TRAFFIC.get(args.workload) if args.search == "bf16" else None),
+        "kernel": ("k_assign_tc (tcgen05 e4m3 x e4m3 -> fp32, fused |c'|^2/2 add + row argmin)" if args.search == "fp8"
+                   else "k_assign_tc (tcgen05 bf16 x bf16 -> fp32, fused |c|^2 add + row argmin)"),
+        "peak_source": (f"{peaks['source']} bf16 burst x 2 (nominal e4m3 / bf16 ratio)" if args.search == "fp8"
+                        else f"{peaks['source']} bf16 burst"),
+        "frac_of_sustained": (achieved / (peaks["bf16_tflops_sustained"] * ratio)
+                              if peaks.get("bf16_tflops_sustained") else None),
         "avg_launch_ms": a_ms / a_n,
         "launches": prof["spans"]["assign"],
         "measured_in": "second timed pass of the same K steps with CUDA events around every launch",
@@ -568,6 +576,8 @@ def main():
     ap.add_argument("--spherical", action="store_true", help="spherical e-means (unit centroids, highest dot product)")
     ap.add_argument("--prefetch", type=int, default=1, choices=[0, 1],
                     help="gather the next step's rows on a second stream during the update (default 1)")
+    ap.add_argument("--search", default="bf16", choices=["bf16", "fp8"],
+                    help="search format: bf16 copies (default) or FP8 E4M3 codes with a fitted converter")
     ap.add_argument("--dp", action="store_true",
                     help="data-parallel e-means: each rank holds its own rows, the per-batch statistics are added "
                          "with NCCL (default for several GPUs: independent replicas)")

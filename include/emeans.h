@@ -85,10 +85,22 @@ enum em_option {
                                     and the error of a row is 2 - 2 x its similarity. The rows
                                     are used as given: normalise them first for cosine
                                     similarity. 0 (default): k-means. Not changeable during a run */
-    EM_OPT_PREFETCH = 17         /* 1 (default): while a step updates the centroids, the rows of
+    EM_OPT_PREFETCH = 17,        /* 1 (default): while a step updates the centroids, the rows of
                                     the next step are gathered into a second batch buffer on a
                                     second stream the model owns; 0: each step gathers its own
                                     rows first. Off while EM_OPT_PROFILE is on                  */
+    EM_OPT_SEARCH_FORMAT = 18    /* 0 (default): the search runs on bf16 copies; 1: on FP8 (E4M3)
+                                    codes (README "Data precision"): a converter fitted on the
+                                    first 65,536 rows of each run's data holds a shift per
+                                    dimension (the midrange) and one power-of-two scale (the
+                                    largest keeping the sample within 448); rows and centroids
+                                    are searched as e4m3((v - shift) * scale), saturating at
+                                    448, on the tensor cores' FP8 path. Counts, sums and
+                                    centroids stay fp32 (sums of the bf16 rows); distances are
+                                    reported in the data's units. Not with spherical e-means or
+                                    the SIMT search; near ties are not settled exactly. Not
+                                    changeable during a run; em_assign on a model without a
+                                    converter fits one on its own rows                          */
 };
 
 /* Phases timed by EM_OPT_PROFILE (em_profile_t.ms / spans index). */
@@ -305,6 +317,12 @@ int em_assign_noalloc(const void* X, int64_t n, int64_t d, const float* centroid
 /* Waits for the model's stream and reports device-side errors (EM_E_BOUNDS,
  * EM_E_TIMEOUT) raised since the last check. */
 int em_sync(em_model* m);
+
+/* The FP8 converter of the model (EM_OPT_SEARCH_FORMAT = 1) fitted by the last
+ * em_begin / em_lloyd (or first em_assign): the shift of each dimension (d fp32
+ * values, host or device pointer, may be NULL) and the power-of-two scale.
+ * EM_E_STATE before any fit. */
+int em_fp8_converter(const em_model* m, float* shift, float* scale);
 
 /* ---- data parallelism (README "Several GPUs": DistributedEmeans) ----
  *

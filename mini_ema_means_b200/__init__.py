@@ -50,6 +50,7 @@ EM_OPT_PROFILE = 14
 EM_OPT_EXACT_TIES = 15
 EM_OPT_SPHERICAL = 16
 EM_OPT_PREFETCH = 17
+EM_OPT_SEARCH_FORMAT = 18
 
 EM_PHASE_PREPARE = 0
 EM_PHASE_GATHER = 1
@@ -145,6 +146,7 @@ _SIGS = {
     "em_profile": (ctypes.c_int, [_P, ctypes.POINTER(em_profile_t), ctypes.c_int]),
     "em_assign_noalloc": (ctypes.c_int, [_P, _I64, _I64, _P, _I64, _P, _P, _P]),
     "em_sync": (ctypes.c_int, [_P]),
+    "em_fp8_converter": (ctypes.c_int, [_P, _P, ctypes.POINTER(ctypes.c_float)]),
     "em_dp_unique_id": (ctypes.c_int, [_P]),
     "em_dp_init": (ctypes.c_int, [_P, ctypes.c_int, ctypes.c_int, _P]),
     "em_dp_world": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]),
@@ -241,12 +243,14 @@ class Model:
         "wait_limit_ms": EM_OPT_WAIT_LIMIT_MS, "auto_revive": EM_OPT_AUTO_REVIVE,
         "capture_labels": EM_OPT_CAPTURE_LABELS, "graphs": EM_OPT_GRAPHS, "assign_kernel": EM_OPT_ASSIGN_KERNEL,
         "profile": EM_OPT_PROFILE, "exact_ties": EM_OPT_EXACT_TIES, "spherical": EM_OPT_SPHERICAL,
-        "prefetch": EM_OPT_PREFETCH,
+        "prefetch": EM_OPT_PREFETCH, "search_format": EM_OPT_SEARCH_FORMAT,
     }
 
     def set_option(self, name, value):
         if name == "revival" and isinstance(value, str):
             value = REVIVAL_MODES[value]
+        if name == "search_format" and isinstance(value, str):
+            value = {"bf16": 0, "fp8": 1, "e4m3": 1}[value]
         if name == "law" and isinstance(value, str):
             value = {"throughput": 0, "quality": 1, "auto": 2}[value]
         if name == "input_dtype" and not isinstance(value, (int, float)):
@@ -276,6 +280,15 @@ class Model:
         """em_dp_init with an id already shared by the caller (every rank calls it)."""
         buf = ctypes.create_string_buffer(bytes(uid), EM_NCCL_ID_BYTES)
         check(em_dp_init(self.h, int(world), int(rank), ctypes.cast(buf, ctypes.c_void_p)), "em_dp_init")
+
+    def fp8_converter(self):
+        """(shift, scale) of the fitted FP8 converter: shift as a float32 ndarray of d."""
+        import numpy as np
+
+        shift = np.empty(self.d, dtype=np.float32)
+        sc = ctypes.c_float()
+        check(em_fp8_converter(self.h, shift.ctypes.data, ctypes.byref(sc)), "em_fp8_converter")
+        return shift, float(sc.value)
 
     def dp_world(self):
         w, r = ctypes.c_int(), ctypes.c_int()

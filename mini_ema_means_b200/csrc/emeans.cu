@@ -36,6 +36,7 @@
 #include "k_data.cuh"
 #include "k_reduce.cuh"
 #include "k_revive.cuh"
+#include "k_fp8.cuh"
 
 using namespace em;
 
@@ -115,6 +116,12 @@ static double alpha_at(int64_t t, int64_t total, double alpha0) {
     return amin + (alpha0 - amin) * 0.5 * (1.0 + cos(M_PI * frac));
 }
 
+static uint32_t __float_as_uint_host(float f) {
+    uint32_t u;
+    memcpy(&u, &f, 4);
+    return u;
+}
+
 // ------------------------------------------------------------------ NCCL (loaded on demand)
 
 struct NcclApi {
@@ -191,6 +198,24 @@ static int make_tmap(CUtensorMap* tm, const void* base, int64_t rows, int d, int
     return EM_OK;
 }
 
+// 2-D tensor map over `rows` rows of d E4M3 codes (row pitch ld8 bytes), boxes of
+// 128 codes (128 bytes, the 128-byte swizzle) x box_rows; columns past d read as 0.
+static int make_tmap8(CUtensorMap* tm, const void* base, int64_t rows, int d, int ld8, int box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return fail(EM_E_CUDA, "cuTensorMapEncodeTiled is not available");
+    if ((reinterpret_cast<uintptr_t>(base) & 15) != 0 || (ld8 & 15) != 0)
+        return fail(EM_E_INVAL, "E4M3 rows must be 16-byte aligned");
+    cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)std::max<int64_t>(rows, 1)};
+    cuuint64_t strides[1] = {(cuuint64_t)ld8};
+    cuuint32_t box[2] = {128u, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(EM_E_CUDA, "cuTensorMapEncodeTiled (E4M3) failed (%d)", (int)r);
+    return EM_OK;
+}
+
 // ------------------------------------------------------------------ model
 
 template <class T>
@@ -231,6 +256,17 @@ struct em_model {
     int revival = EM_REVIVE_SPLIT, finalize = 1, law = 2, in_dtype = 0, check_finite = 0;
     int auto_revive = 1, capture = 1, graphs = 1, assign_kernel = 0, exact_ties = -1;
     int spherical = 0;  // spherical e-means: unit centroids, highest dot product
+    // FP8 search (EM_OPT_SEARCH_FORMAT = 1): the converter fitted at em_begin /
+    // em_lloyd (shift per dimension, power-of-two scale) and the E4M3 operand
+    int fp8 = 0;
+    int ld8 = 0;           // bytes per E4M3 row: d rounded up to 16
+    bool fp8_ready = false;
+    float fp8_scale = 1.0f;
+    DBuf<float> fp8_shift;  // ld values (zero past d)
+    DBuf<float> fp8_lohi, fp8_part;
+    DBuf<uint8_t> cq8, X8full;
+    DBuf<float> cn8, xn8full;
+    CUtensorMap tm_cq8;
     // data parallelism (em_dp_init): this rank's share of each batch, statistics
     // added across ranks with NCCL
     int dp_world = 1, dp_rank = 0;
@@ -259,6 +295,9 @@ struct em_model {
         DBuf<float> xn;         // their |x|^2
         DBuf<int32_t> ids;      // their data row ids
         CUtensorMap tm;         // search operand map over X
+        DBuf<uint8_t> X8;       // FP8 search: the rows' E4M3 codes (pitch ld8 bytes)
+        DBuf<float> xn8;        // and their |x'|^2
+        CUtensorMap tm8;
     };
     BatchSlot slot[2];
     int prefetch = 1;
@@ -470,6 +509,7 @@ static int choose_split(int64_t m_tiles, int64_t n_tiles, int sms, int max_split
 // Nearest-centroid search of `rows` rows described by tmA (row source A for the
 // SIMT path) into m->keys (which the caller has reset to the empty key).
 static bool use_top2(const em_model* m) {
+    if (m->fp8) return false;  // the FP8 search keeps the plain argmin (no exact settling of ties)
     return m->exact_ties == 1 || (m->exact_ties < 0 && m->d >= 256);
 }
 
@@ -490,9 +530,14 @@ static TieList tie_list(em_model* m) { return TieList{m->ties.p, m->tie_n.p, m->
 // Value of a training row (labels kernel): its squared distance, or its spherical error.
 static int training_kind(const em_model* m) { return m->spherical ? kSphericalError : kSquaredDistance; }
 
-// Spherical e-means (README "Spherical e-means"): after every change of the
-// centroids, each is rescaled to norm 1 and the search operand is rebuilt.
-static int normalize_if_spherical(em_model* m);
+// After every change of the centroids: spherical e-means rescales each to norm 1
+// (README "Spherical e-means"), and the FP8 search rebuilds its E4M3 operand.
+static int after_centroid_change(em_model* m);
+
+// How the labels kernels turn a search score into a squared distance.
+static ScoreScale score_scale(const em_model* m) {
+    return m->fp8 ? ScoreScale{2.0f, 1.0f / (m->fp8_scale * m->fp8_scale), -1.0f} : ScoreScale{1.0f, 1.0f, kTieRel};
+}
 
 // Settles the near ties the label kernel of `rows` rows queued (a no-op launch when
 // there are none): one warp per row over a fixed grid.
@@ -517,10 +562,19 @@ static bool ast_fits(int64_t d, int kc) {
 
 static void launch_search(int kc, bool top2, bool ast, int grid, cudaStream_t stream, const CUtensorMap& tmA,
                           const CUtensorMap& tmB, const float* cn, int k, int rows, int nkc, int n_tiles, int split,
-                          unsigned long long* keys, long long wait, int* err) {
+                          unsigned long long* keys, long long wait, int* err, bool f8 = false) {
 #define EM_GO(KC, T2, AST)                                                                                       \
     tc::k_assign_tc<KC, T2, AST><<<grid, tc::kThreads, tc::Cfg<KC, AST>::kSmemBytes, stream>>>(                \
         tmA, tmB, cn, k, rows, nkc, n_tiles, split, keys, wait, err)
+    if (f8) {  // E4M3 rows and operand, 128-code chunks, plain argmin
+        if (ast)
+            tc::k_assign_tc<64, false, true, true><<<grid, tc::kThreads, tc::Cfg<64, true>::kSmemBytes, stream>>>(
+                tmA, tmB, cn, k, rows, nkc, n_tiles, split, keys, wait, err);
+        else
+            tc::k_assign_tc<64, false, false, true><<<grid, tc::kThreads, tc::Cfg<64, false>::kSmemBytes, stream>>>(
+                tmA, tmB, cn, k, rows, nkc, n_tiles, split, keys, wait, err);
+        return;
+    }
     if (kc == 64) {
         if (top2) {
             if (ast) EM_GO(64, true, true); else EM_GO(64, true, false);
@@ -543,7 +597,11 @@ static bool search_smem_attributes() {
                           tc::Cfg<KC, AST>::kSmemBytes) == cudaSuccess)
     return EM_ATTR(64, false, false) && EM_ATTR(64, true, false) && EM_ATTR(32, false, false) &&
            EM_ATTR(32, true, false) && EM_ATTR(64, false, true) && EM_ATTR(64, true, true) &&
-           EM_ATTR(32, false, true) && EM_ATTR(32, true, true);
+           EM_ATTR(32, false, true) && EM_ATTR(32, true, true) &&
+           cudaFuncSetAttribute(tc::k_assign_tc<64, false, false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                tc::Cfg<64, false>::kSmemBytes) == cudaSuccess &&
+           cudaFuncSetAttribute(tc::k_assign_tc<64, false, true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                tc::Cfg<64, true>::kSmemBytes) == cudaSuccess;
 #undef EM_ATTR
 }
 
@@ -560,13 +618,19 @@ static int launch_assign(em_model* m, const CUtensorMap& tmA, const __nv_bfloat1
     }
     const int64_t m_tiles = (rows + tc::BM - 1) / tc::BM;
     const int64_t n_tiles = (m->k + tc::BN - 1) / tc::BN;
-    const int nkc = (int)((m->d + m->kc - 1) / m->kc);
     const int split = split_for(m, rows);
     const int64_t units = m_tiles * split;
     const int grid = (int)std::min<int64_t>(units, m->sms);
-    const bool top2 = use_top2(m);
-    launch_search(m->kc, top2, ast_fits(m->d, m->kc), grid, m->stream, tmA, m->tm_cq, m->cn.p, (int)m->k, (int)rows,
-                  nkc, (int)n_tiles, split, m->keys.p, m->wait_cycles, m->err.p);
+    if (m->fp8) {  // tmA maps E4M3 rows; chunks of 128 codes
+        const int nkc8 = (int)((m->d + 127) / 128);
+        const bool ast8 = (int64_t)nkc8 * tc::BM * 128 <= tc::kAstBufBytes;
+        launch_search(64, false, ast8, grid, m->stream, tmA, m->tm_cq8, m->cn8.p, (int)m->k, (int)rows, nkc8,
+                      (int)n_tiles, split, m->keys.p, m->wait_cycles, m->err.p, true);
+    } else {
+        const int nkc = (int)((m->d + m->kc - 1) / m->kc);
+        launch_search(m->kc, use_top2(m), ast_fits(m->d, m->kc), grid, m->stream, tmA, m->tm_cq, m->cn.p, (int)m->k,
+                      (int)rows, nkc, (int)n_tiles, split, m->keys.p, m->wait_cycles, m->err.p);
+    }
     CK(cudaGetLastError());
     EM_LAUNCHED(m, 1);
     m->last_split = split * tc::kKeySets;
@@ -605,7 +669,7 @@ static int launch_reduce(em_model* m, const __nv_bfloat16* src, int64_t rows, in
         CK(cudaGetLastError());
         EM_LAUNCHED(m, 1);
     }
-    return normalize_if_spherical(m);
+    return after_centroid_change(m);
 }
 
 static ReviveScratch revive_scratch(em_model* m) {
@@ -645,7 +709,7 @@ static int launch_revive(em_model* m, int64_t t, int64_t rows, const __nv_bfloat
         EM_LAUNCHED(m, 2);
     }
     CK(cudaGetLastError());
-    return normalize_if_spherical(m);
+    return after_centroid_change(m);
 }
 
 // One training step of the current run: what it does (host-side plan), the
@@ -695,9 +759,16 @@ static int launch_gather(em_model* m, const StepPlan& p, cudaStream_t stream) {
     em_model::BatchSlot& b = m->slot[p.t & 1];
     const int64_t rows = p.rows / m->dp_world;
     const int64_t key = p.pass + ((int64_t)m->dp_rank << 32);
-    k_gather<<<grid_for(rows, 128, m->sms), 128, 0, stream>>>(m->X, m->n_local, m->ld, m->seed, key,
-                                                             p.pos / m->dp_world, (int)rows, 0, b.X.p, b.xn.p, b.ids.p,
-                                                             m->err.p);
+    if (m->fp8) {
+        const Fp8Out f8{b.X8.p, b.xn8.p, m->fp8_shift.p, m->fp8_scale, m->ld8, (int)m->d};
+        k_gather<true><<<grid_for(rows, 128, m->sms), 128, 0, stream>>>(
+            m->X, m->n_local, m->ld, m->seed, key, p.pos / m->dp_world, (int)rows, 0, b.X.p, b.xn.p, b.ids.p, m->err.p,
+            f8);
+    } else {
+        k_gather<false><<<grid_for(rows, 128, m->sms), 128, 0, stream>>>(
+            m->X, m->n_local, m->ld, m->seed, key, p.pos / m->dp_world, (int)rows, 0, b.X.p, b.xn.p, b.ids.p, m->err.p,
+            Fp8Out{});
+    }
     CK(cudaGetLastError());
     EM_LAUNCHED(m, 1);
     return EM_OK;
@@ -755,7 +826,7 @@ static int launch_step(em_model* m, const StepPlan& p) {
     const bool pf = prefetches(m, p.t);
     if (pf) CK(cudaEventRecord(m->ev_fork, m->stream));
     sp = span_begin(m, EM_PHASE_ASSIGN);
-    CKR(launch_assign(m, b.tm, b.X.p, rows));
+    CKR(launch_assign(m, m->fp8 ? b.tm8 : b.tm, b.X.p, rows));
     span_end(m, sp, 2.0 * rd * kd * dd, 0.0);
     if (pf) {
         cudaStream_t side = m->capturing ? m->side_cap : m->side;
@@ -767,10 +838,10 @@ static int launch_step(em_model* m, const StepPlan& p) {
     sp = span_begin(m, EM_PHASE_UPDATE);
     const int nbl = (int)((rows + 255) / 256);
     const int capture = (m->capture && p.last_pass) ? 1 : 0;
-    k_labels<<<nbl, 256, 0, m->stream>>>(m->keys.p, m->last_split, b.xn.p, (int)rows, (int)m->k, b.X.p, m->ld,
-                                         m->cq.p, b.ids.p, m->labels.p, m->dists.p, m->cnt.p, m->rank.p,
-                                         m->block_err.p, m->labels_last.p, capture, training_kind(m), tie_list(m),
-                                         m->err.p);
+    k_labels<<<nbl, 256, 0, m->stream>>>(m->keys.p, m->last_split, m->fp8 ? b.xn8.p : b.xn.p, (int)rows,
+                                         (int)m->k, b.X.p, m->ld, m->cq.p, b.ids.p, m->labels.p, m->dists.p,
+                                         m->cnt.p, m->rank.p, m->block_err.p, m->labels_last.p, capture,
+                                         training_kind(m), score_scale(m), tie_list(m), m->err.p);
     CK(cudaGetLastError());
     EM_LAUNCHED(m, 1);
     CKR(launch_settle(m, b.X.p, b.xn.p, m->labels.p, nullptr, m->dists.p, true, b.ids.p, m->labels_last.p,
@@ -812,7 +883,10 @@ static std::vector<uint64_t> graph_signature(const em_model* m) {
                             m->rec.passes, m->rec.rows_last_pass, (int64_t)m->seed, m->revival, m->finalize,
                             m->capture, m->auto_revive, m->assign_kernel, m->wait_cycles, m->exact_ties,
                             m->spherical, m->prefetch, m->n_local, m->dp_world, m->dp_rank,
-                            (int64_t)(uintptr_t)m->comm, (int64_t)(uintptr_t)m->stats.p};
+                            (int64_t)(uintptr_t)m->comm, (int64_t)(uintptr_t)m->stats.p, m->fp8,
+                            (int64_t)(uintptr_t)m->slot[0].X8.p, (int64_t)(uintptr_t)m->slot[1].X8.p,
+                            (int64_t)(uintptr_t)m->cq8.p, (int64_t)(uintptr_t)m->fp8_shift.p,
+                            (int64_t)__float_as_uint_host(m->fp8_scale)};
     for (int64_t v : ints) sig.push_back((uint64_t)v);
     double dbl[] = {m->rec.alpha0, m->tau};
     for (double v : dbl) {
@@ -894,12 +968,98 @@ static int run_steps_graph(em_model* m, int64_t count) {
     return EM_OK;
 }
 
-static int normalize_if_spherical(em_model* m) {
-    if (!m->spherical) return EM_OK;
-    k_normalize<<<grid_for(m->k * 32, 256, m->sms), 256, 0, m->stream>>>(cluster_state(m), (int)m->k, m->nv);
+// The E4M3 operand -e4m3((c - shift) * scale) and |c'|^2 / 2 of every centroid.
+static int fp8_operand(em_model* m) {
+    // (without a converter yet, the first search calibrates one and builds the operand)
+    if (!m->fp8 || !m->fp8_ready) return EM_OK;
+    k_fp8_operand<<<grid_for(m->k * 32, 256, m->sms), 256, 0, m->stream>>>(
+        m->c.p, (int)m->k, (int)m->d, m->ld, m->fp8_shift.p, m->fp8_scale, m->cq8.p, m->ld8, m->cn8.p);
     CK(cudaGetLastError());
     EM_LAUNCHED(m, 1);
     return EM_OK;
+}
+
+static int after_centroid_change(em_model* m) {
+    if (m->spherical) {
+        k_normalize<<<grid_for(m->k * 32, 256, m->sms), 256, 0, m->stream>>>(cluster_state(m), (int)m->k, m->nv);
+        CK(cudaGetLastError());
+        EM_LAUNCHED(m, 1);
+    }
+    return fp8_operand(m);
+}
+
+// Fits the FP8 converter on the first rows of X (bf16, n rows; README "Data
+// precision": a shift per dimension and one power-of-two scale, calibrated on a
+// sample): shift = each dimension's midrange in fp32, scale = the largest power of
+// two keeping max |x - shift| within 448. In a data-parallel run the ranks' minima
+// and maxima are combined first, so that every rank holds the same converter.
+static int fp8_calibrate(em_model* m, const __nv_bfloat16* X, int64_t n) {
+    const int64_t rows = std::min<int64_t>(n, kFp8CalibRows);
+    const int d = (int)m->d;
+    const int parts = (int)std::max<int64_t>(1, std::min<int64_t>(rows, 256));
+    CKR(m->fp8_part.ensure((size_t)2 * parts * d));
+    CKR(m->fp8_lohi.ensure((size_t)2 * d));
+    float* lo = m->fp8_lohi.p;
+    float* hi = m->fp8_lohi.p + d;
+    k_fp8_minmax<<<dim3((d + 255) / 256, parts), 256, 0, m->stream>>>(X, rows, d, m->ld, m->fp8_part.p,
+                                                                       m->fp8_part.p + (size_t)parts * d);
+    k_fp8_minmax_reduce<<<(d + 255) / 256, 256, 0, m->stream>>>(m->fp8_part.p, m->fp8_part.p + (size_t)parts * d,
+                                                                 parts, d, lo, hi);
+    CK(cudaGetLastError());
+    EM_LAUNCHED(m, 2);
+    if (m->comm && m->dp_world > 1) {
+        NCK(nccl().all_reduce(lo, lo, (size_t)d, ncclFloat32, ncclMin, m->comm, m->stream));
+        NCK(nccl().all_reduce(hi, hi, (size_t)d, ncclFloat32, ncclMax, m->comm, m->stream));
+    }
+    std::vector<float> h(2 * (size_t)d);
+    CK(cudaMemcpyAsync(h.data(), lo, 2 * (size_t)d * sizeof(float), cudaMemcpyDeviceToHost, m->stream));
+    CK(cudaStreamSynchronize(m->stream));
+    std::vector<float> shift(m->ld, 0.0f);
+    double mx = 0.0;
+    for (int j = 0; j < d; ++j) {
+        const float l = h[j], u = h[d + j];
+        const float sh = (l + u) * 0.5f;
+        shift[j] = sh;
+        mx = std::max(mx, (double)std::max(u - sh, sh - l));
+    }
+    double scale = 1.0;
+    if (mx > 0.0) {
+        int e = (int)std::floor(std::log2((double)kE4M3Max / mx));
+        while (mx * std::ldexp(1.0, e) > (double)kE4M3Max) --e;
+        while (mx * std::ldexp(1.0, e + 1) <= (double)kE4M3Max) ++e;
+        scale = std::ldexp(1.0, e);
+    }
+    if (!(scale >= 0x1p-126 && scale <= 0x1p+126)) return fail(EM_E_INVAL, "the data's range is outside FP8 reach");
+    CKR(m->fp8_shift.ensure(m->ld));
+    CK(cudaMemcpyAsync(m->fp8_shift.p, shift.data(), m->ld * sizeof(float), cudaMemcpyHostToDevice, m->stream));
+    CK(cudaStreamSynchronize(m->stream));
+    m->fp8_scale = (float)scale;
+    m->fp8_ready = true;
+    return EM_OK;
+}
+
+// A run (or Lloyd) on X with the FP8 search: the operand buffers and the converter.
+static int prepare_fp8(em_model* m, const __nv_bfloat16* X, int64_t n) {
+    if (!m->fp8) return EM_OK;
+    if (m->spherical) return fail(EM_E_INVAL, "spherical e-means takes the bf16 search only");
+    if (m->assign_kernel != 0) return fail(EM_E_INVAL, "the FP8 search runs on the tensor-core kernel only");
+    CKR(m->cq8.ensure((size_t)m->k * m->ld8));
+    CKR(m->cn8.ensure(m->k));
+    CKR(make_tmap8(&m->tm_cq8, m->cq8.p, m->k, (int)m->d, m->ld8, tc::BN));
+    return fp8_calibrate(m, X, n);
+}
+
+// E4M3 codes and |x'|^2 of all n rows of A (a full pass) into X8full / xn8full, and
+// the search map over them.
+static int fp8_rows(em_model* m, const __nv_bfloat16* A, int64_t n, CUtensorMap* tm) {
+    CKR(m->X8full.ensure((size_t)n * m->ld8));
+    CKR(m->xn8full.ensure(n));
+    k_fp8_rows<<<grid_for(n * 32, 256, m->sms), 256, 0, m->stream>>>(A, n, (int)m->d, m->ld, m->fp8_shift.p,
+                                                                     m->fp8_scale, m->X8full.p, m->ld8,
+                                                                     m->xn8full.p);
+    CK(cudaGetLastError());
+    EM_LAUNCHED(m, 1);
+    return make_tmap8(tm, m->X8full.p, n, (int)m->d, m->ld8, tc::BM);
 }
 
 static int start_centroids(em_model* m) {
@@ -907,7 +1067,7 @@ static int start_centroids(em_model* m) {
         m->X, m->n_local, m->ld, (int)m->k, m->seed, m->c.p, m->S.p, m->N.p, m->cq.p, m->cn.p, m->err.p);
     CK(cudaGetLastError());
     EM_LAUNCHED(m, 1);
-    return normalize_if_spherical(m);
+    return after_centroid_change(m);
 }
 
 // ------------------------------------------------------------------ ABI
@@ -958,6 +1118,7 @@ em_model* em_create(int64_t d, int64_t k, uint64_t seed) {
     m->k = k;
     m->seed = seed;
     m->ld = (int)((d + 7) / 8 * 8);
+    m->ld8 = (int)((d + 15) / 16 * 16);
     m->nv = m->ld / 8;
     m->kc = (d % 64 == 0) ? 64 : 32;
     auto bail = [&](int code, const char* what) -> em_model* {
@@ -1024,6 +1185,8 @@ void em_destroy(em_model* m) {
         b.X.release();
         b.xn.release();
         b.ids.release();
+        b.X8.release();
+        b.xn8.release();
     }
     m->Xown.release(); m->stage.release(); m->xn.release(); m->dists.release();
     m->labels.release(); m->cnt.release(); m->rank.release(); m->off.release();
@@ -1032,6 +1195,8 @@ void em_destroy(em_model* m) {
     m->labels64.release(); m->rv_dead.release(); m->rv_donor.release(); m->rv_order.release();
     m->rv_times.release(); m->rv_ndead.release(); m->rv_tree.release(); m->rv_splits.release();
     m->ties.release(); m->tie_n.release(); m->tie_corr.release(); m->stats.release();
+    m->fp8_shift.release(); m->fp8_lohi.release(); m->fp8_part.release(); m->cq8.release(); m->X8full.release();
+    m->cn8.release(); m->xn8full.release();
     m->rv_target.release();
     for (auto& sp : m->pending) {
         cudaEventDestroy(sp.a);
@@ -1099,6 +1264,14 @@ int em_set_option(em_model* m, int opt, double v) {
             if (v != -1 && v != 0 && v != 1) return fail(EM_E_INVAL, "exact ties is -1, 0 or 1");
             m->exact_ties = (int)v;
             break;
+        case EM_OPT_SEARCH_FORMAT:
+            if (v != 0 && v != 1) return fail(EM_E_INVAL, "search format is 0 (bf16) or 1 (fp8 e4m3)");
+            if (m->running) return fail(EM_E_STATE, "the search format can not change during a run");
+            if ((int)v != m->fp8) {
+                m->fp8 = (int)v;
+                m->fp8_ready = false;  // a new converter at the next run
+            }
+            break;
         case EM_OPT_PREFETCH:
             if (v != 0 && v != 1) return fail(EM_E_INVAL, "prefetch is 0 or 1");
             m->prefetch = (int)v;
@@ -1133,6 +1306,7 @@ int em_get_option(const em_model* m, int opt, double* v) {
         case EM_OPT_EXACT_TIES: *v = m->exact_ties; break;
         case EM_OPT_SPHERICAL: *v = m->spherical; break;
         case EM_OPT_PREFETCH: *v = m->prefetch; break;
+        case EM_OPT_SEARCH_FORMAT: *v = m->fp8; break;
         default: return fail(EM_E_INVAL, "unknown option %d", opt);
     }
     return EM_OK;
@@ -1172,6 +1346,7 @@ int em_begin(em_model* m, const void* X, int64_t n, double epochs) {
     m->n_local = n;
     const int sp = span_begin(m, EM_PHASE_PREPARE);
     CKR(prepare_input(m, X, n, m->Xown, &m->X));
+    CKR(prepare_fp8(m, m->X, n));
     const int64_t b = m->rec.batch_size / W;  // this rank's rows of a full batch
     CKR(drop_prefetch(m));
     CK(cudaStreamSynchronize(m->stream));  // no gather of a previous run still writes the slots
@@ -1180,6 +1355,11 @@ int em_begin(em_model* m, const void* X, int64_t n, double epochs) {
         CKR(bs.xn.ensure(b));
         CKR(bs.ids.ensure(b));
         CKR(make_tmap(&bs.tm, bs.X.p, b, (int)m->d, m->ld, tc::BM, m->kc));
+        if (m->fp8) {
+            CKR(bs.X8.ensure((size_t)b * m->ld8));
+            CKR(bs.xn8.ensure(b));
+            CKR(make_tmap8(&bs.tm8, bs.X8.p, b, (int)m->d, m->ld8, tc::BM));
+        }
     }
     CKR(ensure_batch_buffers(m, b));
     {  // every batch size the run will see: full batches and the last, partial ones
@@ -1207,6 +1387,7 @@ int em_begin(em_model* m, const void* X, int64_t n, double epochs) {
         NCK(nccl().broadcast(m->c.p, m->c.p, kd, ncclFloat32, 0, m->comm, m->stream));
         NCK(nccl().broadcast(m->cq.p, m->cq.p, kd * sizeof(__nv_bfloat16), ncclUint8, 0, m->comm, m->stream));
         NCK(nccl().broadcast(m->cn.p, m->cn.p, (size_t)m->k, ncclFloat32, 0, m->comm, m->stream));
+        CKR(fp8_operand(m));
     }
     span_end(m, sp);
     m->t = m->pass = m->pos = m->rows_assigned = 0;
@@ -1251,7 +1432,7 @@ int em_finalize(em_model* m) {
                                                                                   m->nv);
         CK(cudaGetLastError());
         EM_LAUNCHED(m, 1);
-        CKR(normalize_if_spherical(m));
+        CKR(after_centroid_change(m));
         span_end(m, sp);
     }
     m->running = false;
@@ -1273,6 +1454,7 @@ int em_lloyd(em_model* m, const void* X, int64_t n, int64_t iters) {
     m->n_local = n;
     m->n = n * m->dp_world;  // data-parallel: every rank's rows, one summed update per iteration
     CKR(prepare_input(m, X, n, m->Xown, &m->X));
+    CKR(prepare_fp8(m, m->X, n));
     CKR(ensure_batch_buffers(m, n));
     if (m->comm) CKR(m->stats.ensure((size_t)m->k * m->ld + m->k + 1));
     CKR(m->keys.ensure(keys_needed(m, n)));
@@ -1283,18 +1465,24 @@ int em_lloyd(em_model* m, const void* X, int64_t n, int64_t iters) {
         NCK(nccl().broadcast(m->c.p, m->c.p, kd, ncclFloat32, 0, m->comm, m->stream));
         NCK(nccl().broadcast(m->cq.p, m->cq.p, kd * sizeof(__nv_bfloat16), ncclUint8, 0, m->comm, m->stream));
         NCK(nccl().broadcast(m->cn.p, m->cn.p, (size_t)m->k, ncclFloat32, 0, m->comm, m->stream));
+        CKR(fp8_operand(m));
     }
     CUtensorMap tmx;
     CKR(make_tmap(&tmx, m->X, n, (int)m->d, m->ld, tc::BM, m->kc));
+    if (m->fp8) CKR(fp8_rows(m, m->X, n, &tmx));  // the rows' codes do not change between iterations
+    const float* x2 = m->fp8 ? m->xn8full.p : m->xn.p;
     const int nbl = (int)((n + 255) / 256);
     for (int64_t it = 0; it < iters; ++it) {
-        k_rownorm_keys<<<grid_for(n * 32, 256, m->sms), 256, 0, m->stream>>>(m->X, n, m->ld, m->xn.p, nullptr);
-        CK(cudaGetLastError());
-        EM_LAUNCHED(m, 1);
+        if (!m->fp8) {
+            k_rownorm_keys<<<grid_for(n * 32, 256, m->sms), 256, 0, m->stream>>>(m->X, n, m->ld, m->xn.p, nullptr);
+            CK(cudaGetLastError());
+            EM_LAUNCHED(m, 1);
+        }
         CKR(launch_assign(m, tmx, m->X, n));
-        k_labels<<<nbl, 256, 0, m->stream>>>(m->keys.p, m->last_split, m->xn.p, (int)n, (int)m->k, m->X, m->ld,
+        k_labels<<<nbl, 256, 0, m->stream>>>(m->keys.p, m->last_split, x2, (int)n, (int)m->k, m->X, m->ld,
                                              m->cq.p, nullptr, m->labels.p, m->dists.p, m->cnt.p, m->rank.p,
-                                             m->block_err.p, nullptr, 0, training_kind(m), tie_list(m), m->err.p);
+                                             m->block_err.p, nullptr, 0, training_kind(m), score_scale(m),
+                                             tie_list(m), m->err.p);
         CK(cudaGetLastError());
         EM_LAUNCHED(m, 1);
         CKR(launch_settle(m, m->X, m->xn.p, m->labels.p, nullptr, m->dists.p, true, nullptr, nullptr, 0));
@@ -1317,16 +1505,25 @@ static int assign_pass(em_model* m, const void* X, int64_t n, int64_t* labels_de
         CKR(m->dists.ensure(n));
         dists_dev = m->dists.p;
     }
-    k_rownorm_keys<<<grid_for(n * 32, 256, m->sms), 256, 0, m->stream>>>(A, n, m->ld, m->xn.p, nullptr);
-    CK(cudaGetLastError());
-    EM_LAUNCHED(m, 1);
     CUtensorMap tmx;
-    CKR(make_tmap(&tmx, A, n, (int)m->d, m->ld, tc::BM, m->kc));
+    if (m->fp8) {  // the model's converter (fitted on this data if the model has none yet)
+        if (!m->fp8_ready) {
+            CKR(prepare_fp8(m, A, n));
+            CKR(fp8_operand(m));
+        }
+        CKR(fp8_rows(m, A, n, &tmx));
+    } else {
+        k_rownorm_keys<<<grid_for(n * 32, 256, m->sms), 256, 0, m->stream>>>(A, n, m->ld, m->xn.p, nullptr);
+        CK(cudaGetLastError());
+        EM_LAUNCHED(m, 1);
+        CKR(make_tmap(&tmx, A, n, (int)m->d, m->ld, tc::BM, m->kc));
+    }
     CKR(launch_assign(m, tmx, A, n));
     const int blocks = grid_for(n, 256, m->sms);
-    k_assign_out<<<blocks, 256, 0, m->stream>>>(m->keys.p, m->last_split, m->xn.p, n, (int)m->k, A, m->ld, m->cq.p,
-                                                labels_dev, dists_dev, nullptr, m->block_err.p,
-                                                m->spherical ? kSimilarity : kSquaredDistance, tie_list(m), m->err.p);
+    k_assign_out<<<blocks, 256, 0, m->stream>>>(m->keys.p, m->last_split, m->fp8 ? m->xn8full.p : m->xn.p, n,
+                                                (int)m->k, A, m->ld, m->cq.p, labels_dev, dists_dev, nullptr,
+                                                m->block_err.p, m->spherical ? kSimilarity : kSquaredDistance,
+                                                score_scale(m), tie_list(m), m->err.p);
     CK(cudaGetLastError());
     EM_LAUNCHED(m, 1);
     CKR(launch_settle(m, A, m->xn.p, nullptr, labels_dev, dists_dev, false, nullptr, nullptr, 0));
@@ -1499,7 +1696,7 @@ int em_set_state(em_model* m, const float* N, const float* S, const float* c, in
                              cudaMemcpyDefault, m->stream));
     k_refresh_operand<<<grid_for(m->k * 32, 256, m->sms), 256, 0, m->stream>>>(cluster_state(m), (int)m->k, m->nv);
     CK(cudaGetLastError());
-    CKR(normalize_if_spherical(m));
+    CKR(after_centroid_change(m));
     if (m->running) {
         // move the run's position to `step` (passes are n rows except a fractional last one)
         m->t = step;
@@ -1564,6 +1761,18 @@ int em_profile(em_model* m, em_profile_t* out, int reset) {
         m->totals = em_profile_t{};
         m->launches = 0;
     }
+    return EM_OK;
+}
+
+int em_fp8_converter(const em_model* m, float* shift, float* scale) {
+    if (!m) return fail(EM_E_INVAL, "model is NULL");
+    if (!m->fp8 || !m->fp8_ready) return fail(EM_E_STATE, "no FP8 converter has been fitted");
+    CKR(set_device(m));
+    if (shift) {
+        CK(cudaMemcpyAsync(shift, m->fp8_shift.p, m->d * sizeof(float), cudaMemcpyDefault, m->stream));
+        CK(cudaStreamSynchronize(m->stream));
+    }
+    if (scale) *scale = m->fp8_scale;
     return EM_OK;
 }
 
@@ -1735,8 +1944,8 @@ extern "C" int em_assign_noalloc(const void* X, int64_t n, int64_t d, const floa
                   nkc, (int)n_tiles, split, keys, wait_cycles, err);
     const int oblocks = std::min(grid_for(n, 256, sms), kNaMaxBlocks);
     k_assign_out<<<oblocks, 256, 0, stream>>>(keys, split * tc::kKeySets, xn, n, (int)k, X16, (int)d, cq, labels,
-                                             dists, nullptr, blocks, kSquaredDistance, TieList{nullptr, nullptr, nullptr},
-                                             err);
+                                             dists, nullptr, blocks, kSquaredDistance, ScoreScale{1.0f, 1.0f, kTieRel},
+                                             TieList{nullptr, nullptr, nullptr}, err);
     CK(cudaGetLastError());
     int h = 0;
     CK(cudaMemcpyAsync(&h, err, sizeof(int), cudaMemcpyDeviceToHost, stream));

@@ -65,6 +65,12 @@ struct Cfg {
 constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
                             ((uint32_t)(BM >> 4) << 24);
 
+// The same for tcgen05.mma kind::f8f6f4 with A and B both E4M3 (format 0 in bits
+// 7-9 and 10-12). A row chunk of 128 E4M3 values is 128 bytes, like a chunk of 64
+// bf16 values, and one MMA consumes K = 32 of them, 32 bytes, like K = 16 bf16: the
+// shared-memory tiles, descriptors and the K loop are byte for byte the bf16 ones.
+constexpr uint32_t kIdescE4M3 = (1u << 4) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return (uint32_t)__cvta_generic_to_shared(p);
 }
@@ -151,6 +157,15 @@ __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a, uint64_t 
         : "memory");
 }
 
+__device__ __forceinline__ void umma_e4m3(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(a), "l"(b), "r"(kIdescE4M3), "r"(accumulate)
+        : "memory");
+}
+
 __device__ __forceinline__ void umma_commit(uint32_t bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
                  : "memory");
@@ -222,13 +237,17 @@ __device__ __forceinline__ void scan_chunk(uint32_t (&v)[32], const float4* c4, 
 // covers writes two keys at keys[((2 g + h) * rows + row) * 2 + {0, 1}]: the best
 // (score, index) and, with TOP2, the second best (without it the second key is
 // empty).
-template <int KC, bool TOP2, bool AST>
+// F8: the batch rows and the centroid operand are E4M3 codes (KC = 64 only: row
+// chunks of 128 bytes = 128 codes).
+template <int KC, bool TOP2, bool AST, bool F8 = false>
 __global__ void __launch_bounds__(kThreads, 1)
     k_assign_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const float* __restrict__ cn, int k, int rows, int nkc, int n_tiles, int n_split,
                 unsigned long long* __restrict__ keys, long long wait_limit, int* err) {
     using C = Cfg<KC, AST>;
     constexpr int S = C::kStages;
+    static_assert(!F8 || KC == 64, "E4M3 rows use 128-byte chunks");
+    constexpr int KX = F8 ? 2 * KC : KC;  // elements per row chunk (the TMA x step)
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     // ring: (A, B) per stage, or B only with the A buffers after the ring (AST)
@@ -312,7 +331,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     aarmed_parity = (aarmed_parity & ~(1u << ab)) | (par << ab);
                     mbar_expect_tx(fb, (uint32_t)(nkc * C::kABytes));
                     for (int kc = 0; kc < nkc; ++kc)
-                        tma_load_2d(smem_u32(sArea + ab * kAstBufBytes + kc * C::kABytes), &tmA, kc * KC, m * BM, fb);
+                        tma_load_2d(smem_u32(sArea + ab * kAstBufBytes + kc * C::kABytes), &tmA, kc * KX, m * BM, fb);
                     ++ua;
                 }
                 for (int nt = nt0; nt < nt1 && ok; ++nt) {
@@ -325,8 +344,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         armed |= 1u << stage;
                         armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
                         mbar_expect_tx(fb, C::kStageBytes);
-                        if (!AST) tma_load_2d(smem_u32(sA + stage * C::kABytes), &tmA, kc * KC, m * BM, fb);
-                        tma_load_2d(smem_u32(sB + stage * C::kBBytes), &tmB, kc * KC, nt * BN, fb);
+                        if (!AST) tma_load_2d(smem_u32(sA + stage * C::kABytes), &tmA, kc * KX, m * BM, fb);
+                        tma_load_2d(smem_u32(sB + stage * C::kBBytes), &tmB, kc * KX, nt * BN, fb);
                         if (++stage == S) {
                             stage = 0;
                             phase ^= 1u;
@@ -382,7 +401,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                         for (int kk = 0; kk < KC / 16; ++kk) {
                             const uint64_t ad = smem_desc(a0 + kk * 32, C::kLayout, C::kSBO);
                             const uint64_t bd = smem_desc(b0 + kk * 32, C::kLayout, C::kSBO);
-                            umma_bf16(d_tmem, ad, bd, (kc | kk) != 0);
+                            if (F8)
+                                umma_e4m3(d_tmem, ad, bd, (kc | kk) != 0);
+                            else
+                                umma_bf16(d_tmem, ad, bd, (kc | kk) != 0);
                         }
                         umma_commit(smem_u32(&empty[stage]));
                         if (++stage == S) {

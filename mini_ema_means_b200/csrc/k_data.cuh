@@ -8,6 +8,7 @@
 #include <cstring>
 
 #include "common.cuh"
+#include "k_fp8_codec.cuh"
 
 namespace em {
 
@@ -155,9 +156,20 @@ __global__ void k_init_centroids(const __nv_bfloat16* __restrict__ X, int64_t n,
 // bf16 values). Each lane computes one row id; the warp then moves the 32 rows four
 // at a time, with every vector of the four rows (up to 1,024 dims per round) loaded
 // before the first store, so that a warp keeps up to 8 KB of reads in flight.
+// With an FP8 search (Fp8Out.X8 set), the rows' E4M3 codes and |x'|^2 are written
+// too (k_fp8.cuh: e4m3((x - shift) * scale), code 0 past the d real columns).
+struct Fp8Out {
+    uint8_t* X8;         // batch codes, pitch ld8 bytes (nullptr: bf16 search)
+    float* xn8;          // |x'|^2 per batch row
+    const float* shift;  // ld values
+    float scale;
+    int ld8, d;
+};
+
+template <bool F8>
 __global__ void k_gather(const __nv_bfloat16* __restrict__ X, int64_t n, int ld, uint64_t seed, int64_t pass,
                          int64_t base, int rows, int natural_order, __nv_bfloat16* __restrict__ Xb,
-                         float* __restrict__ xn, int32_t* __restrict__ ids, int* err) {
+                         float* __restrict__ xn, int32_t* __restrict__ ids, int* err, Fp8Out f8) {
     const int lane = threadIdx.x & 31;
     const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int nwarps = (gridDim.x * blockDim.x) >> 5;
@@ -179,11 +191,12 @@ __global__ void k_gather(const __nv_bfloat16* __restrict__ X, int64_t n, int ld,
         const int cnt = min(32, rows - r0);
         for (int q = 0; q < cnt; q += 4) {
             int64_t src[4];
-            float acc[4];
+            float acc[4], acc8[4];
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
                 src[u] = __shfl_sync(0xFFFFFFFFu, id, min(q + u, cnt - 1));
                 acc[u] = 0.0f;
+                acc8[u] = 0.0f;
             }
             // up to 4 x 32 vectors (1,024 dims) of the four rows in flight per round
             for (int vb = 0; vb < nv; vb += 128) {
@@ -207,6 +220,15 @@ __global__ void k_gather(const __nv_bfloat16* __restrict__ X, int64_t n, int ld,
                                 unpack8_bf16(val[u][it], x);
 #pragma unroll
                                 for (int i = 0; i < 8; ++i) acc[u] = fmaf(x[i], x[i], acc[u]);
+                                if (F8) {
+                                    float sh[8];
+                                    const float4 s0 = reinterpret_cast<const float4*>(f8.shift)[2 * v];
+                                    const float4 s1 = reinterpret_cast<const float4*>(f8.shift)[2 * v + 1];
+                                    sh[0] = s0.x; sh[1] = s0.y; sh[2] = s0.z; sh[3] = s0.w;
+                                    sh[4] = s1.x; sh[5] = s1.y; sh[6] = s1.z; sh[7] = s1.w;
+                                    reinterpret_cast<uint2*>(f8.X8 + (int64_t)(r0 + q + u) * f8.ld8)[v] =
+                                        encode8_e4m3(x, sh, f8.scale, f8.d - 8 * v, acc8[u]);
+                                }
                             }
                         }
                     }
@@ -214,10 +236,17 @@ __global__ void k_gather(const __nv_bfloat16* __restrict__ X, int64_t n, int ld,
             }
 #pragma unroll
             for (int u = 0; u < 4; ++u) acc[u] = warp_sum(acc[u]);
+            if (F8) {
+#pragma unroll
+                for (int u = 0; u < 4; ++u) acc8[u] = warp_sum(acc8[u]);
+            }
             if (lane == 0) {
 #pragma unroll
                 for (int u = 0; u < 4; ++u)
-                    if (q + u < cnt) xn[r0 + q + u] = acc[u];
+                    if (q + u < cnt) {
+                        xn[r0 + q + u] = acc[u];
+                        if (F8) f8.xn8[r0 + q + u] = acc8[u];
+                    }
             }
         }
     }

@@ -99,15 +99,24 @@ enum RowValue : int {
     kSimilarity = 2,       // -s / 2 = x.c: the similarity (spherical assign)
 };
 
-__device__ __forceinline__ float row_value(int kind, float x2, float s) {
-    if (kind == kSquaredDistance) return fmaxf(0.0f, x2 + s);
+// How a squared distance follows from a score: (x2 + mul * score) * dscale. The bf16
+// search has mul = dscale = 1; the FP8 search scores half the squared distance in
+// code units (mul = 2) and reports it in the data's units (dscale = 1 / scale^2).
+// tie_rel: the near-tie window settled in fp64 (kTieRel), or < 0 for none (the
+// FP8 search, whose exact comparison would be on codes the settling does not read).
+struct ScoreScale {
+    float mul, dscale, tie_rel;
+};
+
+__device__ __forceinline__ float row_value(int kind, float x2, float s, ScoreScale sc = {1.0f, 1.0f, kTieRel}) {
+    if (kind == kSquaredDistance) return fmaxf(0.0f, x2 + sc.mul * s) * sc.dscale;
     if (kind == kSphericalError) return 2.0f + s;
     return -0.5f * s;
 }
 
 // The row's contribution to the error sum: the squared distance, or 2 - 2 x similarity.
-__device__ __forceinline__ float row_error(int kind, float x2, float s) {
-    return kind == kSquaredDistance ? fmaxf(0.0f, x2 + s) : 2.0f + s;
+__device__ __forceinline__ float row_error(int kind, float x2, float s, ScoreScale sc = {1.0f, 1.0f, kTieRel}) {
+    return kind == kSquaredDistance ? fmaxf(0.0f, x2 + sc.mul * s) * sc.dscale : 2.0f + s;
 }
 
 // fp64 comparison value of candidate q for a near tie, from the bf16 row x and the
@@ -188,7 +197,7 @@ __global__ void k_labels(const unsigned long long* __restrict__ keys, int nsplit
                          const __nv_bfloat16* __restrict__ cq, const int32_t* __restrict__ ids,
                          int32_t* __restrict__ labels, float* __restrict__ dists, int32_t* __restrict__ cnt,
                          int32_t* __restrict__ rank, double* __restrict__ block_err, int64_t* __restrict__ labels_last,
-                         int capture, int kind, TieList tl, int* err) {
+                         int capture, int kind, ScoreScale sc, TieList tl, int* err) {
     __shared__ double warp_err[32];
     const int lane = threadIdx.x & 31;
     double e = 0.0;
@@ -210,7 +219,7 @@ __global__ void k_labels(const unsigned long long* __restrict__ keys, int nsplit
         if (k2 != kEmptyKey) {
             l2 = key_label(k2);
             s2 = key_score(k2);
-            tie = l2 < (uint32_t)k && s2 - s1 <= kTieRel * (x2 + fabsf(s1) + fabsf(s2));
+            tie = sc.tie_rel >= 0.0f && l2 < (uint32_t)k && s2 - s1 <= sc.tie_rel * (x2 + fabsf(s1) + fabsf(s2));
         }
     }
     // a near tie is left to k_settle: provisional label and distance now, counted there
@@ -223,8 +232,8 @@ __global__ void k_labels(const unsigned long long* __restrict__ keys, int nsplit
     if (active) {
         lab = (int)l1;
         labels[r] = lab;
-        dists[r] = row_value(kind, x2, s1);
-        e = (double)row_error(kind, x2, s1);
+        dists[r] = row_value(kind, x2, s1, sc);
+        e = (double)row_error(kind, x2, s1, sc);
         if (capture && !defer) labels_last[ids[r]] = lab;
     }
     const bool counted = active && !defer;
@@ -667,7 +676,7 @@ __global__ void k_assign_out(const unsigned long long* __restrict__ keys, int ns
                              int64_t rows, int k, const __nv_bfloat16* __restrict__ A, int ld,
                              const __nv_bfloat16* __restrict__ cq, int64_t* __restrict__ labels,
                              float* __restrict__ dists, int32_t* __restrict__ labels32, double* __restrict__ block_err,
-                             int kind, TieList tl, int* err) {
+                             int kind, ScoreScale sc, TieList tl, int* err) {
     __shared__ double warp_err[32];
     const int lane = threadIdx.x & 31;
     double e = 0.0;
@@ -691,7 +700,7 @@ __global__ void k_assign_out(const unsigned long long* __restrict__ keys, int ns
             if (k2 != kEmptyKey) {
                 l2 = key_label(k2);
                 s2 = key_score(k2);
-                tie = l2 < (uint32_t)k && s2 - s1 <= kTieRel * (x2 + fabsf(s1) + fabsf(s2));
+                tie = sc.tie_rel >= 0.0f && l2 < (uint32_t)k && s2 - s1 <= sc.tie_rel * (x2 + fabsf(s1) + fabsf(s2));
             }
         }
         if (tl.e)
@@ -701,8 +710,8 @@ __global__ void k_assign_out(const unsigned long long* __restrict__ keys, int ns
         if (active) {
             if (labels) labels[r] = (int64_t)l1;
             if (labels32) labels32[r] = (int32_t)l1;
-            if (dists) dists[r] = row_value(kind, x2, s1);
-            e += (double)row_error(kind, x2, s1);
+            if (dists) dists[r] = row_value(kind, x2, s1, sc);
+            e += (double)row_error(kind, x2, s1, sc);
         }
     }
     e = warp_sum(e);

@@ -6,7 +6,12 @@ Tolerances (stated once, used by every parity test):
   tensor cores vs the fp64 oracle); such rows may hold the other near-tied label
   and may number at most max(1, 1e-4 x rows compared). Spherical e-means compares
   errors 2 - 2 x similarity the same way, the gap measured against
-  max(best error, 1e-3 |x|^2) since a row can sit on its centroid;
+  max(best error, 1e-3 |x|^2) since a row can sit on its centroid. The FP8
+  search compares E4M3 codes: its tensor cores accumulate the code products in
+  fp32 with some loss (the largest flip measured on this B200: a gap of 1.2e-4 of
+  sum|x'_i c'_i|), and it settles no near tie exactly, so a row may hold another
+  label whose code distance is within FP8_GAP_REL x sum|x'_i c'_i| of the best,
+  with no limit on their number;
 * centroids: relative L2 error per centroid <= 1e-3;
 * MSE: relative error <= 1e-3 (0.1 %).
 """
@@ -19,6 +24,7 @@ import torch
 from oracle import emeans_oracle as O
 
 LABEL_GAP_REL = 1e-3
+FP8_GAP_REL = 2.0 ** -11
 LABEL_MISMATCH_FRACTION = 1e-4
 CENTROID_REL = 1e-3
 MSE_REL = 1e-3
@@ -27,17 +33,20 @@ MSE_REL = 1e-3
 class LabelBook:
     """Accumulates label comparisons over several batches."""
 
-    def __init__(self, spherical=False):
+    def __init__(self, spherical=False, fp8=False):
         self.rows = 0
         self.mismatch = 0
         self.spherical = spherical
+        self.fp8 = fp8
 
-    def compare(self, gpu_labels, xq_rows, cq):
+    def compare(self, gpu_labels, xq_rows, cq, dscale=1.0):
         """Checks GPU labels against the oracle's search with search copies cq.
 
         Returns the accepted labels (the oracle's, except where the GPU picked
         another label of a near tie: both are correct there) and the oracle's best
-        value per row (squared distance, or spherical error 2 - 2 x similarity)."""
+        value per row (squared distance, or spherical error 2 - 2 x similarity).
+        For the FP8 search, xq_rows and cq are the E4M3 codes and dscale = 1 /
+        scale^2 turns their squared distances into the data's units."""
         gpu_labels = np.asarray(gpu_labels, dtype=np.int64)
         if self.spherical:
             lab, sim, sim2 = O.assign_dot(xq_rows, cq)
@@ -50,19 +59,28 @@ class LabelBook:
             if self.spherical:
                 d_gpu = 2.0 - 2.0 * np.einsum("ij,ij->i", xr, cg)
                 scale = np.maximum(best[diff], 1e-3 * np.einsum("ij,ij->i", xr, xr))
+            elif self.fp8:
+                d_gpu = ((xr - cg) ** 2).sum(axis=1)
+                mag = np.abs(xr) @ np.abs(cq).T  # sum |x'_i c'_i| for every centroid
+                scale = None
             else:
                 d_gpu = ((xr - cg) ** 2).sum(axis=1)
                 scale = np.maximum(best[diff], 1e-30)
-            ok = (d_gpu - best[diff]) <= LABEL_GAP_REL * scale
-            ok &= (second[diff] - best[diff]) < LABEL_GAP_REL * scale
+            if self.fp8:
+                ok = (d_gpu - best[diff]) <= FP8_GAP_REL * 2.0 * mag[np.arange(len(diff)), gpu_labels[diff]]
+            else:
+                ok = (d_gpu - best[diff]) <= LABEL_GAP_REL * scale
+                ok &= (second[diff] - best[diff]) < LABEL_GAP_REL * scale
             assert ok.all(), f"{(~ok).sum()} labels differ from the oracle outside near ties"
         self.rows += len(lab)
         self.mismatch += len(diff)
         accepted = lab.copy()
         accepted[diff] = gpu_labels[diff]
-        return accepted, best
+        return accepted, best * dscale
 
     def finish(self):
+        if self.fp8:
+            return  # every mismatch was checked against the FP8 accumulation bound
         allowed = max(1, int(LABEL_MISMATCH_FRACTION * self.rows))
         assert self.mismatch <= allowed, f"{self.mismatch} near-tie label flips in {self.rows} rows (max {allowed})"
 
@@ -112,7 +130,7 @@ def teacher_forced_run(m, orc, x_dev, xq, epochs, revival, check_every=1, max_st
         np.testing.assert_allclose(c, orc.c, rtol=1e-6, atol=1e-7)
     else:
         assert np.array_equal(c, orc.c), "starting centroids differ from the oracle's rows"
-    book = LabelBook(spherical=orc.spherical)
+    book = LabelBook(spherical=orc.spherical, fp8=orc.search == "fp8")
     worst = {"N": 0.0, "c": 0.0, "dist": 0.0, "revive_c": 0.0}
     total = rec["total_steps"] if max_steps is None else min(max_steps, rec["total_steps"])
     revivals = 0
@@ -127,8 +145,18 @@ def teacher_forced_run(m, orc, x_dev, xq, epochs, revival, check_every=1, max_st
         ids, labels, dists = gpu_last_batch(m, rec["batch_size"])
         assert np.array_equal(ids, ids_expected), f"step {t}: batch rows differ from the oracle's order"
         if check:
-            accepted, best = book.compare(labels, xq[ids], O.search_copy_of_centroids(orc.c))
-            tol = 1e-5 * (np.einsum("ij,ij->i", xq[ids], xq[ids]) + best) + 1e-6
+            if orc.search == "fp8":
+                shift, scale = orc.fp8
+                xr = O.fp8_codes(xq[ids], shift, scale)
+                cr = O.fp8_search_copy_of_centroids(orc.c, shift, scale)
+                accepted, best = book.compare(labels, xr, cr, dscale=1.0 / scale ** 2)
+                # the GPU's distance of its label: the code distance up to twice the
+                # accumulation bound on x'.c' (the label may be another near tie)
+                mag = np.einsum("ij,ij->i", np.abs(xr), np.abs(cr[labels]))
+                tol = (2.0 * 2.0 * FP8_GAP_REL * mag) / scale ** 2 + 1e-5 * best + 1e-6
+            else:
+                accepted, best = book.compare(labels, xq[ids], O.search_copy_of_centroids(orc.c))
+                tol = 1e-5 * (np.einsum("ij,ij->i", xq[ids], xq[ids]) + best) + 1e-6
             worst["dist"] = max(worst["dist"], float(np.max(np.abs(dists - best) / tol)))
             assert np.all(np.abs(dists - best) <= tol), f"step {t}: distances differ"
             orc.step(forced_labels=accepted, auto_revive=False)
