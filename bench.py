@@ -499,7 +499,7 @@ def run_kernel_case(args):
     if args.kernel_case == "assign":
         w, xt, _ = datagen.make(args.workload, device="cuda", seed=0, n_train=args.case_rows, n_test=1)
         xb = xt.to(torch.bfloat16).contiguous()
-        m = em.Model(w.d, w.k, seed=1234, input_dtype=1)
+        m = em.Model(w.d, w.k, seed=1234, input_dtype=1, search_format=args.search)
         m.set_state(c=xt[: w.k].float().contiguous())
         lab = torch.empty(w.n_train, dtype=torch.int64, device="cuda")
         for _ in range(2):
@@ -514,7 +514,7 @@ def run_kernel_case(args):
     else:
         rows = args.case_rows if args.case_rows_step else None
         w, xt, _ = datagen.make(args.workload, device="cuda", seed=0, n_train=rows, n_test=1 if rows else None)
-        m = em.Model(w.d, w.k, seed=1234)
+        m = em.Model(w.d, w.k, seed=1234, search_format=args.search)
         if args.case_batch:
             m.set_option("batch_size", args.case_batch)
         m.begin(xt, epochs=w.epochs)

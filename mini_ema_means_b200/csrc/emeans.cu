@@ -109,6 +109,15 @@ static int compute_recipe(int64_t n, int64_t k, int64_t d, double epochs, int la
     return EM_OK;
 }
 
+// Launch shapes of the near-tie settling and the cluster pass (set at build time
+// for sweeps): k_settle blocks per SM, k_clusters threads per block.
+#ifndef EM_SETTLE_BLOCKS_PER_SM
+#define EM_SETTLE_BLOCKS_PER_SM 8
+#endif
+#ifndef EM_CLUSTERS_BLOCK
+#define EM_CLUSTERS_BLOCK 256
+#endif
+
 // cosine step size from alpha0 down to alpha0 / 10 over all steps
 static double alpha_at(int64_t t, int64_t total, double alpha0) {
     const double amin = 0.1 * alpha0;
@@ -544,7 +553,8 @@ static ScoreScale score_scale(const em_model* m) {
 static int launch_settle(em_model* m, const __nv_bfloat16* A, const float* xn, int32_t* labels32, int64_t* labels64,
                          float* dists, bool count, const int32_t* ids, int64_t* labels_last, int capture) {
     const int kind = (count || !m->spherical) ? training_kind(m) : kSimilarity;
-    k_settle<<<m->sms * 8, 256, 0, m->stream>>>(tie_list(m), xn, A, m->ld, m->cq.p, labels32, labels64, dists,
+    k_settle<<<m->sms * EM_SETTLE_BLOCKS_PER_SM, 256, 0, m->stream>>>(tie_list(m), xn, A, m->ld, m->cq.p, labels32,
+                                                                    labels64, dists,
                                                 count ? m->cnt.p : nullptr, m->rank.p, ids, labels_last, capture,
                                                 kind);
     CK(cudaGetLastError());
@@ -658,7 +668,8 @@ static int launch_reduce(em_model* m, const __nv_bfloat16* src, int64_t rows, in
     const int seg_blocks = (int)((max_items * nslices * 32 + 255) / 256);
     k_segsum<<<seg_blocks, 256, 0, m->stream>>>(src, m->perm.p, m->items.p, m->poff.p, nslices, m->nv, st, sp,
                                                 m->part.p);
-    k_clusters<<<grid_for(m->k * 32, 256, m->sms), 256, 0, m->stream>>>(m->off.p, m->poff.p, m->cnt.p, m->R, nslices,
+    k_clusters<<<grid_for(m->k * 32, EM_CLUSTERS_BLOCK, m->sms, 16), EM_CLUSTERS_BLOCK, 0, m->stream>>>(
+        m->off.p, m->poff.p, m->cnt.p, m->R, nslices,
                                                                          m->nv, st, sp, m->part.p);
     CK(cudaGetLastError());
     EM_LAUNCHED(m, 4);

@@ -259,8 +259,12 @@ __global__ void k_labels(const unsigned long long* __restrict__ keys, int nsplit
 
 // Exclusive scans of the counts (segment starts off[0..k]) and of the chunk counts
 // ceil(n_j / R) (first work item of each cluster, poff[0..k]); one CTA of 1024
-// threads in tiles of 4096 clusters. Also adds the per-block error sums in block
-// order and keeps the running counts of before this step (N_prev).
+// threads, 16 consecutive clusters per thread (one pass up to 16,384 clusters).
+// Also adds the per-block error sums in a fixed order (each thread its strided
+// share, then a fixed butterfly and the warps in order) and keeps the running
+// counts of before this step (N_prev); both are issued ahead of the scan.
+constexpr int kOffsetsPer = 16;
+
 __global__ void __launch_bounds__(1024) k_offsets(const int32_t* __restrict__ cnt, int k, int rows, int R,
                                                   int32_t* __restrict__ off, int32_t* __restrict__ poff,
                                                   const double* __restrict__ block_err, int nblocks,
@@ -268,20 +272,36 @@ __global__ void __launch_bounds__(1024) k_offsets(const int32_t* __restrict__ cn
                                                   float* __restrict__ N_prev, TieList tl, int* err) {
     __shared__ int2 warp_tot[32];
     __shared__ int2 carry_s;
+    __shared__ double warp_err[32];
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+    double e = 0.0;
+    for (int b = tid; b < nblocks; b += 1024) e += block_err[b];
     for (int j = tid; j < k; j += 1024) N_prev[j] = N[j];
     if (tid == 0) carry_s = make_int2(0, 0);
+    e = warp_sum(e);
+    if (lane == 0) warp_err[w] = e;
     __syncthreads();
-    for (int base = 0; base < k; base += 4096) {
-        int v[4], c[4];
-        const int i0 = base + tid * 4;
+    const bool vec = (k % 4) == 0;  // 16-byte loads and stores of the counts and offsets
+    for (int base = 0; base < k; base += 1024 * kOffsetsPer) {
+        int v[kOffsetsPer], c[kOffsetsPer];
+        const int i0 = base + tid * kOffsetsPer;
+        if (vec && i0 + kOffsetsPer <= k) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            v[i] = (i0 + i < k) ? cnt[i0 + i] : 0;
-            c[i] = (v[i] + R - 1) / R;
+            for (int q = 0; q < kOffsetsPer / 4; ++q) {
+                const int4 x = reinterpret_cast<const int4*>(cnt + i0)[q];
+                v[4 * q] = x.x; v[4 * q + 1] = x.y; v[4 * q + 2] = x.z; v[4 * q + 3] = x.w;
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < kOffsetsPer; ++i) v[i] = (i0 + i < k) ? cnt[i0 + i] : 0;
         }
-        const int local_v = v[0] + v[1] + v[2] + v[3];
-        const int local_c = c[0] + c[1] + c[2] + c[3];
+        int local_v = 0, local_c = 0;
+#pragma unroll
+        for (int i = 0; i < kOffsetsPer; ++i) {
+            c[i] = (v[i] + R - 1) / R;
+            local_v += v[i];
+            local_c += c[i];
+        }
         int iv = local_v, ic = local_c;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
@@ -312,22 +332,34 @@ __global__ void __launch_bounds__(1024) k_offsets(const int32_t* __restrict__ cn
         const int2 carry = carry_s;
         int rv = carry.x + warp_tot[w].x + iv - local_v;
         int rc = carry.y + warp_tot[w].y + ic - local_c;
+        int ov[kOffsetsPer], oc[kOffsetsPer];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            if (i0 + i < k) {
-                off[i0 + i] = rv;
-                poff[i0 + i] = rc;
-            }
+        for (int i = 0; i < kOffsetsPer; ++i) {
+            ov[i] = rv;
+            oc[i] = rc;
             rv += v[i];
             rc += c[i];
+        }
+        if (vec && i0 + kOffsetsPer <= k) {
+#pragma unroll
+            for (int q = 0; q < kOffsetsPer / 4; ++q) {
+                reinterpret_cast<int4*>(off + i0)[q] = make_int4(ov[4 * q], ov[4 * q + 1], ov[4 * q + 2], ov[4 * q + 3]);
+                reinterpret_cast<int4*>(poff + i0)[q] = make_int4(oc[4 * q], oc[4 * q + 1], oc[4 * q + 2], oc[4 * q + 3]);
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < kOffsetsPer; ++i)
+                if (i0 + i < k) {
+                    off[i0 + i] = ov[i];
+                    poff[i0 + i] = oc[i];
+                }
         }
         __syncthreads();
         if (tid == 1023) carry_s = make_int2(rv, rc);
         __syncthreads();
     }
-    if (w == 0) {  // batch error: lane-strided partial sums, then a fixed butterfly
-        double t = 0.0;
-        for (int b = lane; b < nblocks; b += 32) t += block_err[b];
+    if (w == 0) {  // batch error: the warps' sums in warp order
+        double t = warp_err[lane];
         t = warp_sum(t);
         if (lane == 0) {
             off[k] = carry_s.x;
@@ -406,7 +438,15 @@ __device__ __forceinline__ SliceGeom slice_geom(int slice, int nv) {
 }
 
 // Rows per work item of the grouped update (one chunk of a cluster).
-constexpr int kChunkRows = 64;
+// Launch-shape constants of the grouped update (set at build time for sweeps).
+#ifndef EM_CHUNK_ROWS
+#define EM_CHUNK_ROWS 64
+#endif
+#ifndef EM_SEGSUM_RIF
+#define EM_SEGSUM_RIF 4
+#endif
+constexpr int kChunkRows = EM_CHUNK_ROWS;
+constexpr int kSegsumRif = EM_SEGSUM_RIF;
 
 // Sum over rows perm[s0..s1) of this lane's vector, fp64, four rows in flight per
 // lane (each row id is a broadcast load that the first row group brings into L1;
@@ -516,7 +556,7 @@ __global__ void __launch_bounds__(256, 3) k_segsum(const __nv_bfloat16* __restri
         nprev = st.N_prev[j];
     }
     double acc[8];
-    sum_rows(acc, src, st.ld, perm, it.y, it.z, g, lane);
+    sum_rows<kSegsumRif>(acc, src, st.ld, perm, it.y, it.z, g, lane);
     if (it.w && sp.stats) {  // this rank's sums of the cluster, for the exchange
         if (lane < g.nvs) {
             double* dst = sp.stats + (int64_t)j * st.ld + 8 * (g.vbase + lane);
