@@ -205,7 +205,7 @@ def run_ours(args, rank, world):
     log(f"[rank {rank}] data {w.name} ready in {time.time() - t0:.1f} s")
     stream = torch.cuda.current_stream(dev)
     m = em.Model(w.d, w.k, seed=1234, spherical=int(args.spherical), prefetch=args.prefetch,
-                 search_format=args.search)
+                 search_format=args.search, pdl=args.pdl)
     m.set_stream(stream.cuda_stream)
     if args.dp:
         dp_join(em, m, world)
@@ -286,6 +286,7 @@ def run_ours(args, rank, world):
         "config": {"workload": workload_desc(w), "method": "spherical e-means" if args.spherical else "e-means",
                    "search": args.search,
                    "batch_size": rec["batch_size"], "alpha0": round(rec["alpha0"], 6), "prefetch": args.prefetch,
+                   "pdl": args.pdl,
                    "steps_per_run": total,
                    "l2": "inputs larger than L2: the fp32 training matrix (%.2f GB) and its bf16 copy are re-read "
                          "in a fresh random order every pass" % (w.n_train * w.d * 4 / 1e9),
@@ -576,6 +577,8 @@ def main():
     ap.add_argument("--spherical", action="store_true", help="spherical e-means (unit centroids, highest dot product)")
     ap.add_argument("--prefetch", type=int, default=1, choices=[0, 1],
                     help="gather the next step's rows on a second stream during the update (default 1)")
+    ap.add_argument("--pdl", type=int, default=1, choices=[0, 1],
+                    help="programmatic dependent launch of the step's kernels (default 1)")
     ap.add_argument("--search", default="bf16", choices=["bf16", "fp8"],
                     help="search format: bf16 copies (default) or FP8 E4M3 codes with a fitted converter")
     ap.add_argument("--dp", action="store_true",

@@ -89,7 +89,7 @@ enum em_option {
                                     the next step are gathered into a second batch buffer on a
                                     second stream the model owns; 0: each step gathers its own
                                     rows first. Off while EM_OPT_PROFILE is on                  */
-    EM_OPT_SEARCH_FORMAT = 18    /* 0 (default): the search runs on bf16 copies; 1: on FP8 (E4M3)
+    EM_OPT_SEARCH_FORMAT = 18,   /* 0 (default): the search runs on bf16 copies; 1: on FP8 (E4M3)
                                     codes (README "Data precision"): a converter fitted on the
                                     first 65,536 rows of each run's data holds a shift per
                                     dimension (the midrange) and one power-of-two scale (the
@@ -101,6 +101,9 @@ enum em_option {
                                     the SIMT search; near ties are not settled exactly. Not
                                     changeable during a run; em_assign on a model without a
                                     converter fits one on its own rows                          */
+    EM_OPT_PDL = 19              /* 1 (default): the kernels of a step launch with programmatic
+                                    stream serialization, each starting while its predecessor
+                                    finishes and waiting for it on the device; 0: plain launches */
 };
 
 /* Phases timed by EM_OPT_PROFILE (em_profile_t.ms / spans index). */
@@ -317,6 +320,13 @@ int em_assign_noalloc(const void* X, int64_t n, int64_t d, const float* centroid
 /* Waits for the model's stream and reports device-side errors (EM_E_BOUNDS,
  * EM_E_TIMEOUT) raised since the last check. */
 int em_sync(em_model* m);
+
+/* Exercises the failure path without a fault: which = 0 runs the search kernel's
+ * bounded mbarrier wait on a barrier nothing arrives on, which gives up after
+ * wait_ms and returns EM_E_TIMEOUT; which = 1 raises the index-check error and
+ * returns EM_E_BOUNDS. The error word is cleared when reported, so the model stays
+ * usable. wait_ms in (0, 10000]. */
+int em_selftest(em_model* m, int which, double wait_ms);
 
 /* The FP8 converter of the model (EM_OPT_SEARCH_FORMAT = 1) fitted by the last
  * em_begin / em_lloyd (or first em_assign): the shift of each dimension (d fp32

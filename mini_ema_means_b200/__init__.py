@@ -51,6 +51,7 @@ EM_OPT_EXACT_TIES = 15
 EM_OPT_SPHERICAL = 16
 EM_OPT_PREFETCH = 17
 EM_OPT_SEARCH_FORMAT = 18
+EM_OPT_PDL = 19
 
 EM_PHASE_PREPARE = 0
 EM_PHASE_GATHER = 1
@@ -146,6 +147,7 @@ _SIGS = {
     "em_profile": (ctypes.c_int, [_P, ctypes.POINTER(em_profile_t), ctypes.c_int]),
     "em_assign_noalloc": (ctypes.c_int, [_P, _I64, _I64, _P, _I64, _P, _P, _P]),
     "em_sync": (ctypes.c_int, [_P]),
+    "em_selftest": (ctypes.c_int, [_P, ctypes.c_int, ctypes.c_double]),
     "em_fp8_converter": (ctypes.c_int, [_P, _P, ctypes.POINTER(ctypes.c_float)]),
     "em_dp_unique_id": (ctypes.c_int, [_P]),
     "em_dp_init": (ctypes.c_int, [_P, ctypes.c_int, ctypes.c_int, _P]),
@@ -243,7 +245,7 @@ class Model:
         "wait_limit_ms": EM_OPT_WAIT_LIMIT_MS, "auto_revive": EM_OPT_AUTO_REVIVE,
         "capture_labels": EM_OPT_CAPTURE_LABELS, "graphs": EM_OPT_GRAPHS, "assign_kernel": EM_OPT_ASSIGN_KERNEL,
         "profile": EM_OPT_PROFILE, "exact_ties": EM_OPT_EXACT_TIES, "spherical": EM_OPT_SPHERICAL,
-        "prefetch": EM_OPT_PREFETCH, "search_format": EM_OPT_SEARCH_FORMAT,
+        "prefetch": EM_OPT_PREFETCH, "search_format": EM_OPT_SEARCH_FORMAT, "pdl": EM_OPT_PDL,
     }
 
     def set_option(self, name, value):
@@ -289,6 +291,10 @@ class Model:
         sc = ctypes.c_float()
         check(em_fp8_converter(self.h, shift.ctypes.data, ctypes.byref(sc)), "em_fp8_converter")
         return shift, float(sc.value)
+
+    def selftest(self, which, wait_ms=200.0) -> int:
+        """Status of em_selftest (EM_E_TIMEOUT for which=0, EM_E_BOUNDS for which=1)."""
+        return int(em_selftest(self.h, int(which), float(wait_ms)))
 
     def dp_world(self):
         w, r = ctypes.c_int(), ctypes.c_int()

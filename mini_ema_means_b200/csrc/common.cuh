@@ -19,6 +19,13 @@
 
 namespace em {
 
+// Programmatic dependent launch: every kernel of the library starts by waiting for
+// the grids it depends on (a no-op unless it was launched with programmatic stream
+// serialization), so that the host may let a kernel launch while its predecessor on
+// the stream is still finishing; pdl_release lets the next kernel launch early.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_release() { asm volatile("griddepcontrol.launch_dependents;" :::); }
+
 // ---------------------------------------------------------------- generator
 
 constexpr uint64_t kPhiloxM0 = 0xD2E7470EE14C6C93ull;

@@ -27,6 +27,7 @@
 #include <cstring>
 #include <dlfcn.h>
 #include <mutex>
+#include <utility>
 #include <vector>
 
 #include <nccl.h>  // types and prototypes only: the library is loaded with dlopen
@@ -129,6 +130,26 @@ static uint32_t __float_as_uint_host(float f) {
     uint32_t u;
     memcpy(&u, &f, 4);
     return u;
+}
+
+// Launches `kern` on `stream`, with programmatic stream serialization when `pdl`
+// is set: the kernel may then launch while its predecessor on the stream is still
+// finishing, and waits for it with griddepcontrol.wait (every kernel of the
+// library starts with that wait).
+template <typename... KArgs, typename... Args>
+static cudaError_t launch_k(bool pdl, void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                           Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
 // ------------------------------------------------------------------ NCCL (loaded on demand)
@@ -265,6 +286,7 @@ struct em_model {
     int revival = EM_REVIVE_SPLIT, finalize = 1, law = 2, in_dtype = 0, check_finite = 0;
     int auto_revive = 1, capture = 1, graphs = 1, assign_kernel = 0, exact_ties = -1;
     int spherical = 0;  // spherical e-means: unit centroids, highest dot product
+    int pdl = 1;        // EM_OPT_PDL: programmatic dependent launch of the step's kernels
     // FP8 search (EM_OPT_SEARCH_FORMAT = 1): the converter fitted at em_begin /
     // em_lloyd (shift per dimension, power-of-two scale) and the E4M3 operand
     int fp8 = 0;
@@ -553,7 +575,7 @@ static ScoreScale score_scale(const em_model* m) {
 static int launch_settle(em_model* m, const __nv_bfloat16* A, const float* xn, int32_t* labels32, int64_t* labels64,
                          float* dists, bool count, const int32_t* ids, int64_t* labels_last, int capture) {
     const int kind = (count || !m->spherical) ? training_kind(m) : kSimilarity;
-    k_settle<<<m->sms * EM_SETTLE_BLOCKS_PER_SM, 256, 0, m->stream>>>(tie_list(m), xn, A, m->ld, m->cq.p, labels32,
+    launch_k(m->pdl, k_settle, m->sms * EM_SETTLE_BLOCKS_PER_SM, 256, 0, m->stream, tie_list(m), xn, A, m->ld, m->cq.p, labels32,
                                                                     labels64, dists,
                                                 count ? m->cnt.p : nullptr, m->rank.p, ids, labels_last, capture,
                                                 kind);
@@ -572,17 +594,17 @@ static bool ast_fits(int64_t d, int kc) {
 
 static void launch_search(int kc, bool top2, bool ast, int grid, cudaStream_t stream, const CUtensorMap& tmA,
                           const CUtensorMap& tmB, const float* cn, int k, int rows, int nkc, int n_tiles, int split,
-                          unsigned long long* keys, long long wait, int* err, bool f8 = false) {
-#define EM_GO(KC, T2, AST)                                                                                       \
-    tc::k_assign_tc<KC, T2, AST><<<grid, tc::kThreads, tc::Cfg<KC, AST>::kSmemBytes, stream>>>(                \
-        tmA, tmB, cn, k, rows, nkc, n_tiles, split, keys, wait, err)
+                          unsigned long long* keys, long long wait, int* err, bool f8 = false, bool pdl = false) {
+#define EM_GO(KC, T2, AST)                                                                                 \
+    launch_k(pdl, tc::k_assign_tc<KC, T2, AST>, grid, tc::kThreads, tc::Cfg<KC, AST>::kSmemBytes, stream, tmA, \
+             tmB, cn, k, rows, nkc, n_tiles, split, keys, wait, err)
     if (f8) {  // E4M3 rows and operand, 128-code chunks, plain argmin
         if (ast)
-            tc::k_assign_tc<64, false, true, true><<<grid, tc::kThreads, tc::Cfg<64, true>::kSmemBytes, stream>>>(
-                tmA, tmB, cn, k, rows, nkc, n_tiles, split, keys, wait, err);
+            launch_k(pdl, tc::k_assign_tc<64, false, true, true>, grid, tc::kThreads, tc::Cfg<64, true>::kSmemBytes,
+                     stream, tmA, tmB, cn, k, rows, nkc, n_tiles, split, keys, wait, err);
         else
-            tc::k_assign_tc<64, false, false, true><<<grid, tc::kThreads, tc::Cfg<64, false>::kSmemBytes, stream>>>(
-                tmA, tmB, cn, k, rows, nkc, n_tiles, split, keys, wait, err);
+            launch_k(pdl, tc::k_assign_tc<64, false, false, true>, grid, tc::kThreads, tc::Cfg<64, false>::kSmemBytes,
+                     stream, tmA, tmB, cn, k, rows, nkc, n_tiles, split, keys, wait, err);
         return;
     }
     if (kc == 64) {
@@ -635,11 +657,11 @@ static int launch_assign(em_model* m, const CUtensorMap& tmA, const __nv_bfloat1
         const int nkc8 = (int)((m->d + 127) / 128);
         const bool ast8 = (int64_t)nkc8 * tc::BM * 128 <= tc::kAstBufBytes;
         launch_search(64, false, ast8, grid, m->stream, tmA, m->tm_cq8, m->cn8.p, (int)m->k, (int)rows, nkc8,
-                      (int)n_tiles, split, m->keys.p, m->wait_cycles, m->err.p, true);
+                      (int)n_tiles, split, m->keys.p, m->wait_cycles, m->err.p, true, m->pdl != 0);
     } else {
         const int nkc = (int)((m->d + m->kc - 1) / m->kc);
         launch_search(m->kc, use_top2(m), ast_fits(m->d, m->kc), grid, m->stream, tmA, m->tm_cq, m->cn.p, (int)m->k,
-                      (int)rows, nkc, (int)n_tiles, split, m->keys.p, m->wait_cycles, m->err.p);
+                      (int)rows, nkc, (int)n_tiles, split, m->keys.p, m->wait_cycles, m->err.p, false, m->pdl != 0);
     }
     CK(cudaGetLastError());
     EM_LAUNCHED(m, 1);
@@ -656,19 +678,19 @@ static int launch_reduce(em_model* m, const __nv_bfloat16* src, int64_t rows, in
     const StepParams sp{alpha, last_pass, 0, dp ? m->stats.p : nullptr};
     double* const step_err = err_sum_out;
     if (dp) err_sum_out = stats_err;  // the error sum travels with the statistics
-    k_offsets<<<1, 1024, 0, m->stream>>>(m->cnt.p, (int)m->k, (int)rows, m->R, m->off.p, m->poff.p, m->block_err.p,
+    launch_k(m->pdl, k_offsets, 1, 1024, 0, m->stream, m->cnt.p, (int)m->k, (int)rows, m->R, m->off.p, m->poff.p, m->block_err.p,
                                          nblocks_labels, err_sum_out, m->N.p, m->N_prev.p, tie_list(m), m->err.p);
     CK(cudaGetLastError());
-    k_scatter<<<(int)((rows + 255) / 256), 256, 0, m->stream>>>(m->labels.p, m->rank.p, m->off.p, m->poff.p,
+    launch_k(m->pdl, k_scatter, (int)((rows + 255) / 256), 256, 0, m->stream, m->labels.p, m->rank.p, m->off.p, m->poff.p,
                                                                  (int)rows, m->R, m->perm.p, m->items.p, m->err.p);
     CK(cudaGetLastError());
     const ClusterState st = cluster_state(m);
     const int64_t max_items = m->k + (rows + m->R - 1) / m->R;
     const int nslices = (m->nv + 31) / 32;
     const int seg_blocks = (int)((max_items * nslices * 32 + 255) / 256);
-    k_segsum<<<seg_blocks, 256, 0, m->stream>>>(src, m->perm.p, m->items.p, m->poff.p, nslices, m->nv, st, sp,
+    launch_k(m->pdl, k_segsum, seg_blocks, 256, 0, m->stream, src, m->perm.p, m->items.p, m->poff.p, nslices, m->nv, st, sp,
                                                 m->part.p);
-    k_clusters<<<grid_for(m->k * 32, EM_CLUSTERS_BLOCK, m->sms, 16), EM_CLUSTERS_BLOCK, 0, m->stream>>>(
+    launch_k(m->pdl, k_clusters, grid_for(m->k * 32, EM_CLUSTERS_BLOCK, m->sms, 16), EM_CLUSTERS_BLOCK, 0, m->stream, 
         m->off.p, m->poff.p, m->cnt.p, m->R, nslices,
                                                                          m->nv, st, sp, m->part.p);
     CK(cudaGetLastError());
@@ -676,7 +698,7 @@ static int launch_reduce(em_model* m, const __nv_bfloat16* src, int64_t rows, in
     if (dp) {  // add the ranks' statistics, then the same update on every rank
         NCK(nccl().all_reduce(m->stats.p, m->stats.p, (size_t)m->k * m->ld + m->k + 1, ncclFloat64, ncclSum, m->comm,
                               m->stream));
-        k_apply_stats<<<grid_for(m->k * 32, 256, m->sms), 256, 0, m->stream>>>(nslices, m->nv, st, sp, step_err);
+        launch_k(m->pdl, k_apply_stats, grid_for(m->k * 32, 256, m->sms), 256, 0, m->stream, nslices, m->nv, st, sp, step_err);
         CK(cudaGetLastError());
         EM_LAUNCHED(m, 1);
     }
@@ -706,17 +728,17 @@ static int launch_revive(em_model* m, int64_t t, int64_t rows, const __nv_bfloat
     if (m->revival == EM_REVIVE_NONE || !(effective_tau(m) > 0.0)) return EM_OK;
     const ReviveScratch sc = revive_scratch(m);
     const int smem = m->k <= kFastK ? tree32((int)m->k).bytes : (int)tree_smem_bytes(tree_layout((int)m->k), (int)m->k);
-    k_revive_select<<<1, kSelectThreads, smem, m->stream>>>(m->N.p, (int)m->k, effective_tau(m), m->seed, t,
+    launch_k(m->pdl, k_revive_select, 1, kSelectThreads, smem, m->stream, m->N.p, (int)m->k, effective_tau(m), m->seed, t,
                                                             m->revival, sc, m->err.p);
     CK(cudaGetLastError());
     const ClusterState st = cluster_state(m);
     const int blocks = grid_for(m->k * 32, 256, m->sms);
     if (m->revival == EM_REVIVE_SPLIT) {
-        k_revive_dead<<<blocks, 256, 0, m->stream>>>(st, m->nv, sc);
-        k_revive_donors<<<blocks, 256, 0, m->stream>>>(st, m->nv, sc);
+        launch_k(m->pdl, k_revive_dead, blocks, 256, 0, m->stream, st, m->nv, sc);
+        launch_k(m->pdl, k_revive_donors, blocks, 256, 0, m->stream, st, m->nv, sc);
         EM_LAUNCHED(m, 3);
     } else {
-        k_revive_resample<<<blocks, 256, 0, m->stream>>>(st, m->nv, sc, Xb, (int)rows, m->seed, t);
+        launch_k(m->pdl, k_revive_resample, blocks, 256, 0, m->stream, st, m->nv, sc, Xb, (int)rows, m->seed, t);
         EM_LAUNCHED(m, 2);
     }
     CK(cudaGetLastError());
@@ -772,11 +794,11 @@ static int launch_gather(em_model* m, const StepPlan& p, cudaStream_t stream) {
     const int64_t key = p.pass + ((int64_t)m->dp_rank << 32);
     if (m->fp8) {
         const Fp8Out f8{b.X8.p, b.xn8.p, m->fp8_shift.p, m->fp8_scale, m->ld8, (int)m->d};
-        k_gather<true><<<grid_for(rows, 128, m->sms), 128, 0, stream>>>(
+        launch_k(m->pdl, k_gather<true>, grid_for(rows, 128, m->sms), 128, 0, stream, 
             m->X, m->n_local, m->ld, m->seed, key, p.pos / m->dp_world, (int)rows, 0, b.X.p, b.xn.p, b.ids.p, m->err.p,
             f8);
     } else {
-        k_gather<false><<<grid_for(rows, 128, m->sms), 128, 0, stream>>>(
+        launch_k(m->pdl, k_gather<false>, grid_for(rows, 128, m->sms), 128, 0, stream, 
             m->X, m->n_local, m->ld, m->seed, key, p.pos / m->dp_world, (int)rows, 0, b.X.p, b.xn.p, b.ids.p, m->err.p,
             Fp8Out{});
     }
@@ -849,7 +871,7 @@ static int launch_step(em_model* m, const StepPlan& p) {
     sp = span_begin(m, EM_PHASE_UPDATE);
     const int nbl = (int)((rows + 255) / 256);
     const int capture = (m->capture && p.last_pass) ? 1 : 0;
-    k_labels<<<nbl, 256, 0, m->stream>>>(m->keys.p, m->last_split, m->fp8 ? b.xn8.p : b.xn.p, (int)rows,
+    launch_k(m->pdl, k_labels, nbl, 256, 0, m->stream, m->keys.p, m->last_split, m->fp8 ? b.xn8.p : b.xn.p, (int)rows,
                                          (int)m->k, b.X.p, m->ld, m->cq.p, b.ids.p, m->labels.p, m->dists.p,
                                          m->cnt.p, m->rank.p, m->block_err.p, m->labels_last.p, capture,
                                          training_kind(m), score_scale(m), tie_list(m), m->err.p);
@@ -897,7 +919,7 @@ static std::vector<uint64_t> graph_signature(const em_model* m) {
                             (int64_t)(uintptr_t)m->comm, (int64_t)(uintptr_t)m->stats.p, m->fp8,
                             (int64_t)(uintptr_t)m->slot[0].X8.p, (int64_t)(uintptr_t)m->slot[1].X8.p,
                             (int64_t)(uintptr_t)m->cq8.p, (int64_t)(uintptr_t)m->fp8_shift.p,
-                            (int64_t)__float_as_uint_host(m->fp8_scale)};
+                            (int64_t)__float_as_uint_host(m->fp8_scale), m->pdl};
     for (int64_t v : ints) sig.push_back((uint64_t)v);
     double dbl[] = {m->rec.alpha0, m->tau};
     for (double v : dbl) {
@@ -983,7 +1005,7 @@ static int run_steps_graph(em_model* m, int64_t count) {
 static int fp8_operand(em_model* m) {
     // (without a converter yet, the first search calibrates one and builds the operand)
     if (!m->fp8 || !m->fp8_ready) return EM_OK;
-    k_fp8_operand<<<grid_for(m->k * 32, 256, m->sms), 256, 0, m->stream>>>(
+    launch_k(m->pdl, k_fp8_operand, grid_for(m->k * 32, 256, m->sms), 256, 0, m->stream, 
         m->c.p, (int)m->k, (int)m->d, m->ld, m->fp8_shift.p, m->fp8_scale, m->cq8.p, m->ld8, m->cn8.p);
     CK(cudaGetLastError());
     EM_LAUNCHED(m, 1);
@@ -992,7 +1014,7 @@ static int fp8_operand(em_model* m) {
 
 static int after_centroid_change(em_model* m) {
     if (m->spherical) {
-        k_normalize<<<grid_for(m->k * 32, 256, m->sms), 256, 0, m->stream>>>(cluster_state(m), (int)m->k, m->nv);
+        launch_k(m->pdl, k_normalize, grid_for(m->k * 32, 256, m->sms), 256, 0, m->stream, cluster_state(m), (int)m->k, m->nv);
         CK(cudaGetLastError());
         EM_LAUNCHED(m, 1);
     }
@@ -1275,6 +1297,10 @@ int em_set_option(em_model* m, int opt, double v) {
             if (v != -1 && v != 0 && v != 1) return fail(EM_E_INVAL, "exact ties is -1, 0 or 1");
             m->exact_ties = (int)v;
             break;
+        case EM_OPT_PDL:
+            if (v != 0 && v != 1) return fail(EM_E_INVAL, "pdl is 0 or 1");
+            m->pdl = (int)v;
+            break;
         case EM_OPT_SEARCH_FORMAT:
             if (v != 0 && v != 1) return fail(EM_E_INVAL, "search format is 0 (bf16) or 1 (fp8 e4m3)");
             if (m->running) return fail(EM_E_STATE, "the search format can not change during a run");
@@ -1318,6 +1344,7 @@ int em_get_option(const em_model* m, int opt, double* v) {
         case EM_OPT_SPHERICAL: *v = m->spherical; break;
         case EM_OPT_PREFETCH: *v = m->prefetch; break;
         case EM_OPT_SEARCH_FORMAT: *v = m->fp8; break;
+        case EM_OPT_PDL: *v = m->pdl; break;
         default: return fail(EM_E_INVAL, "unknown option %d", opt);
     }
     return EM_OK;
@@ -1490,7 +1517,7 @@ int em_lloyd(em_model* m, const void* X, int64_t n, int64_t iters) {
             EM_LAUNCHED(m, 1);
         }
         CKR(launch_assign(m, tmx, m->X, n));
-        k_labels<<<nbl, 256, 0, m->stream>>>(m->keys.p, m->last_split, x2, (int)n, (int)m->k, m->X, m->ld,
+        launch_k(m->pdl, k_labels, nbl, 256, 0, m->stream, m->keys.p, m->last_split, x2, (int)n, (int)m->k, m->X, m->ld,
                                              m->cq.p, nullptr, m->labels.p, m->dists.p, m->cnt.p, m->rank.p,
                                              m->block_err.p, nullptr, 0, training_kind(m), score_scale(m),
                                              tie_list(m), m->err.p);
@@ -1829,6 +1856,20 @@ int em_sync(em_model* m) {
     CKR(set_device(m));
     CK(cudaStreamSynchronize(m->stream));
     return check_device_errors(m);
+}
+
+int em_selftest(em_model* m, int which, double wait_ms) {
+    if (!m) return fail(EM_E_INVAL, "model is NULL");
+    if (which != 0 && which != 1) return fail(EM_E_INVAL, "which is 0 (bounded wait) or 1 (index check)");
+    if (!(wait_ms > 0.0 && wait_ms <= 10000.0)) return fail(EM_E_INVAL, "wait_ms must be in (0, 10000]");
+    CKR(set_device(m));
+    CKR(drop_prefetch(m));
+    int clock_khz = 1965000;
+    cudaDeviceGetAttribute(&clock_khz, cudaDevAttrClockRate, m->dev);
+    tc::k_selftest<<<1, 32, 0, m->stream>>>(which, (long long)(wait_ms * (double)clock_khz), m->err.p);
+    CK(cudaGetLastError());
+    EM_LAUNCHED(m, 1);
+    return em_sync(m);
 }
 
 }  // extern "C"

@@ -237,6 +237,24 @@ __device__ __forceinline__ void scan_chunk(uint32_t (&v)[32], const float4* c4, 
 // covers writes two keys at keys[((2 g + h) * rows + row) * 2 + {0, 1}]: the best
 // (score, index) and, with TOP2, the second best (without it the second key is
 // empty).
+// Self-test of the failure path: one thread waits on an mbarrier that nothing
+// arrives on, with the search kernel's bounded wait, so the wait gives up after
+// `wait_limit` cycles and raises EM_E_TIMEOUT in the error word; or (which = 1) the
+// kernel raises EM_E_BOUNDS as a failed index check would. Nothing faults or hangs.
+__global__ void k_selftest(int which, long long wait_limit, int* err) {
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x != 0) return;
+    if (which == 1) {
+        raise_error(err, EM_E_BOUNDS);
+        return;
+    }
+    abort_flag = 0;
+    mbar_init(smem_u32(&bar), 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    mbar_wait(smem_u32(&bar), 0u, wait_limit, err, &abort_flag);  // phase 0 never completes
+}
+
 // F8: the batch rows and the centroid operand are E4M3 codes (KC = 64 only: row
 // chunks of 128 bytes = 128 codes).
 template <int KC, bool TOP2, bool AST, bool F8 = false>
@@ -306,6 +324,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    // the set-up above overlaps the previous kernel; the operands are read after it
+    pdl_wait();
 
     if (warp == 0) {
         // ---------------- TMA producer
@@ -533,6 +553,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 // apart from a fault elsewhere in the step when a parity test fails.
 __global__ void k_assign_simt(const __nv_bfloat16* __restrict__ A, int ld, int rows, const __nv_bfloat16* __restrict__ cq,
                               const float* __restrict__ cn, int k, int d, unsigned long long* __restrict__ keys) {
+    pdl_wait();
     const int row = blockIdx.x * blockDim.x + threadIdx.x;
     if (row >= rows) return;
     const __nv_bfloat16* x = A + (int64_t)row * ld;

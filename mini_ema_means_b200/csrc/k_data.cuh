@@ -38,6 +38,7 @@ __device__ __forceinline__ void unpack8_bf16(uint4 u, float v[8]) {
 // copy of fp32 data; faiss e-means README, "Data precision").
 __global__ void k_cast_f32_bf16(const float* __restrict__ src, int64_t n, int d, int ld,
                                 __nv_bfloat16* __restrict__ dst, int vec_ok) {
+    pdl_wait();
     const int nv = ld / 8;
     const int64_t total = n * nv;
     for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total;
@@ -62,6 +63,7 @@ __global__ void k_cast_f32_bf16(const float* __restrict__ src, int64_t n, int d,
 // bf16 n x d (row stride d) -> bf16 n x ld (padding copy for unaligned rows).
 __global__ void k_pad_bf16(const __nv_bfloat16* __restrict__ src, int64_t n, int d, int ld,
                            __nv_bfloat16* __restrict__ dst) {
+    pdl_wait();
     const int64_t total = n * ld;
     for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total;
          e += (int64_t)gridDim.x * blockDim.x) {
@@ -73,6 +75,7 @@ __global__ void k_pad_bf16(const __nv_bfloat16* __restrict__ src, int64_t n, int
 
 // Sets *flag if any of the first `count` values is NaN or infinite.
 __global__ void k_check_finite(const void* __restrict__ src, int64_t count, int is_bf16, int* flag) {
+    pdl_wait();
     int bad = 0;
     for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < count;
          e += (int64_t)gridDim.x * blockDim.x) {
@@ -118,6 +121,8 @@ __device__ __forceinline__ double warp_sum(double v) {
 __global__ void k_init_centroids(const __nv_bfloat16* __restrict__ X, int64_t n, int ld, int k, uint64_t seed,
                                  float* __restrict__ c, float* __restrict__ S, float* __restrict__ N,
                                  __nv_bfloat16* __restrict__ cq, float* __restrict__ cn, int* err) {
+    pdl_wait();
+    pdl_release();
     const int lane = threadIdx.x & 31;
     const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int nwarps = (gridDim.x * blockDim.x) >> 5;
@@ -170,6 +175,8 @@ template <bool F8>
 __global__ void k_gather(const __nv_bfloat16* __restrict__ X, int64_t n, int ld, uint64_t seed, int64_t pass,
                          int64_t base, int rows, int natural_order, __nv_bfloat16* __restrict__ Xb,
                          float* __restrict__ xn, int32_t* __restrict__ ids, int* err, Fp8Out f8) {
+    pdl_wait();
+    pdl_release();
     const int lane = threadIdx.x & 31;
     const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int nwarps = (gridDim.x * blockDim.x) >> 5;
@@ -256,6 +263,7 @@ __global__ void k_gather(const __nv_bfloat16* __restrict__ X, int64_t n, int ld,
 // of a full assignment pass (em_assign, em_mse, Lloyd iterations).
 __global__ void k_rownorm_keys(const __nv_bfloat16* __restrict__ X, int64_t rows, int ld, float* __restrict__ xn,
                                unsigned long long* __restrict__ keys) {
+    pdl_wait();
     const int lane = threadIdx.x & 31;
     const int64_t warp = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;

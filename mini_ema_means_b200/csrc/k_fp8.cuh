@@ -26,6 +26,7 @@ namespace em {
 // partial per (row block, dimension): part_lo / part_hi[blockIdx.y * d + j].
 __global__ void k_fp8_minmax(const __nv_bfloat16* __restrict__ X, int64_t rows, int d, int ld,
                              float* __restrict__ part_lo, float* __restrict__ part_hi) {
+    pdl_wait();
     const int j = blockIdx.x * blockDim.x + threadIdx.x;
     if (j >= d) return;
     float lo = INFINITY, hi = -INFINITY;
@@ -41,6 +42,7 @@ __global__ void k_fp8_minmax(const __nv_bfloat16* __restrict__ X, int64_t rows, 
 // Calibration, pass 2: the minimum and maximum over the row blocks.
 __global__ void k_fp8_minmax_reduce(const float* __restrict__ part_lo, const float* __restrict__ part_hi, int nparts,
                                     int d, float* __restrict__ lo, float* __restrict__ hi) {
+    pdl_wait();
     const int j = blockIdx.x * blockDim.x + threadIdx.x;
     if (j >= d) return;
     float a = INFINITY, b = -INFINITY;
@@ -57,6 +59,7 @@ __global__ void k_fp8_minmax_reduce(const float* __restrict__ part_lo, const flo
 __global__ void k_fp8_rows(const __nv_bfloat16* __restrict__ X, int64_t rows, int d, int ld,
                            const float* __restrict__ shift, float scale, uint8_t* __restrict__ X8, int ld8,
                            float* __restrict__ xn8) {
+    pdl_wait();
     const int lane = threadIdx.x & 31;
     const int64_t warp = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
@@ -78,6 +81,8 @@ __global__ void k_fp8_rows(const __nv_bfloat16* __restrict__ X, int64_t rows, in
 // |c'|^2 / 2. One warp per cluster.
 __global__ void k_fp8_operand(const float* __restrict__ c, int k, int d, int ld, const float* __restrict__ shift,
                               float scale, uint8_t* __restrict__ cq8, int ld8, float* __restrict__ cn8) {
+    pdl_wait();
+    pdl_release();
     const int lane = threadIdx.x & 31;
     const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int nwarps = (gridDim.x * blockDim.x) >> 5;

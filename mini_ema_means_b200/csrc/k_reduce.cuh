@@ -198,6 +198,8 @@ __global__ void k_labels(const unsigned long long* __restrict__ keys, int nsplit
                          int32_t* __restrict__ labels, float* __restrict__ dists, int32_t* __restrict__ cnt,
                          int32_t* __restrict__ rank, double* __restrict__ block_err, int64_t* __restrict__ labels_last,
                          int capture, int kind, ScoreScale sc, TieList tl, int* err) {
+    pdl_wait();
+    pdl_release();
     __shared__ double warp_err[32];
     const int lane = threadIdx.x & 31;
     double e = 0.0;
@@ -270,6 +272,8 @@ __global__ void __launch_bounds__(1024) k_offsets(const int32_t* __restrict__ cn
                                                   const double* __restrict__ block_err, int nblocks,
                                                   double* __restrict__ err_sum_out, const float* __restrict__ N,
                                                   float* __restrict__ N_prev, TieList tl, int* err) {
+    pdl_wait();
+    pdl_release();
     __shared__ int2 warp_tot[32];
     __shared__ int2 carry_s;
     __shared__ double warp_err[32];
@@ -380,6 +384,8 @@ __global__ void __launch_bounds__(1024) k_offsets(const int32_t* __restrict__ cn
 __global__ void k_scatter(const int32_t* __restrict__ labels, const int32_t* __restrict__ rank,
                           const int32_t* __restrict__ off, const int32_t* __restrict__ poff, int rows, int R,
                           int32_t* __restrict__ perm, int4* __restrict__ items, int* err) {
+    pdl_wait();
+    pdl_release();
     const int r = blockIdx.x * blockDim.x + threadIdx.x;
     if (r >= rows) return;
     const int lab = labels[r];
@@ -538,10 +544,15 @@ __device__ __forceinline__ float ema_slice(const ClusterState& st, int j, double
 // count are all fetched right after the item. A
 // cluster that fits in one chunk is updated here; the chunks of a larger cluster
 // leave their slice sums in part[item] for k_clusters.
-__global__ void __launch_bounds__(256, 3) k_segsum(const __nv_bfloat16* __restrict__ src,
+#ifndef EM_SEGSUM_MIN_BLOCKS
+#define EM_SEGSUM_MIN_BLOCKS 3
+#endif
+__global__ void __launch_bounds__(256, EM_SEGSUM_MIN_BLOCKS) k_segsum(const __nv_bfloat16* __restrict__ src,
                                                    const int32_t* __restrict__ perm, const int4* __restrict__ items,
                                                    const int32_t* __restrict__ poff, int nslices, int nv,
                                                    ClusterState st, StepParams sp, double* __restrict__ part) {
+    pdl_wait();
+    pdl_release();
     const int lane = threadIdx.x & 31;
     const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int item = warp / nslices, slice = warp - item * nslices;
@@ -582,6 +593,8 @@ __global__ void __launch_bounds__(256, 3) k_segsum(const __nv_bfloat16* __restri
 __global__ void k_clusters(const int32_t* __restrict__ off, const int32_t* __restrict__ poff,
                            int32_t* __restrict__ cnt, int R, int nslices, int nv, ClusterState st, StepParams sp,
                            const double* __restrict__ part) {
+    pdl_wait();
+    pdl_release();
     const int lane = threadIdx.x & 31;
     const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int nwarps = (gridDim.x * blockDim.x) >> 5;
@@ -671,6 +684,8 @@ __global__ void k_clusters(const int32_t* __restrict__ off, const int32_t* __res
 // the single-GPU update (a cluster without rows decays; the others go through
 // ema_slice slice by slice), and thread 0 stores the summed error of the step.
 __global__ void k_apply_stats(int nslices, int nv, ClusterState st, StepParams sp, double* __restrict__ err_out) {
+    pdl_wait();
+    pdl_release();
     const int lane = threadIdx.x & 31;
     const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int nwarps = (gridDim.x * blockDim.x) >> 5;
@@ -717,6 +732,7 @@ __global__ void k_assign_out(const unsigned long long* __restrict__ keys, int ns
                              const __nv_bfloat16* __restrict__ cq, int64_t* __restrict__ labels,
                              float* __restrict__ dists, int32_t* __restrict__ labels32, double* __restrict__ block_err,
                              int kind, ScoreScale sc, TieList tl, int* err) {
+    pdl_wait();
     __shared__ double warp_err[32];
     const int lane = threadIdx.x & 31;
     double e = 0.0;
@@ -766,6 +782,7 @@ __global__ void k_assign_out(const unsigned long long* __restrict__ keys, int ns
 
 __global__ void k_sum_blocks(const double* __restrict__ block_err, int nblocks, double* __restrict__ out,
                              TieList tl) {
+    pdl_wait();
     if (blockIdx.x == 0 && threadIdx.x == 0) {
         double t = 0.0;
         for (int b = 0; b < nblocks; ++b) t += block_err[b];
@@ -790,6 +807,8 @@ __global__ void k_settle(TieList tl, const float* __restrict__ xn, const __nv_bf
                          int64_t* __restrict__ labels64, float* __restrict__ dists, int32_t* __restrict__ cnt,
                          int32_t* __restrict__ rank, const int32_t* __restrict__ ids,
                          int64_t* __restrict__ labels_last, int capture, int kind) {
+    pdl_wait();
+    pdl_release();
     const int lane = threadIdx.x & 31;
     const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int nwarps = (gridDim.x * blockDim.x) >> 5;
@@ -829,6 +848,8 @@ __global__ void k_settle(TieList tl, const float* __restrict__ xn, const __nv_bf
 // Closing mean: c_j = exact mean of the rows the last pass assigned to j, for the
 // clusters that received rows (faiss e-means README, "How the centroid updates work").
 __global__ void k_closing_mean(ClusterState st, int k, int nv) {
+    pdl_wait();
+    pdl_release();
     const int lane = threadIdx.x & 31;
     const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int nwarps = (gridDim.x * blockDim.x) >> 5;
@@ -850,6 +871,8 @@ __global__ void k_closing_mean(ClusterState st, int k, int nv) {
 
 // Refreshes the search operand and |bf16(c)|^2 from c (after em_set_state).
 __global__ void k_refresh_operand(ClusterState st, int k, int nv) {
+    pdl_wait();
+    pdl_release();
     const int lane = threadIdx.x & 31;
     const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int nwarps = (gridDim.x * blockDim.x) >> 5;
@@ -871,6 +894,8 @@ __global__ void k_refresh_operand(ClusterState st, int k, int nv) {
 // cluster: the norm of the fp32 centroid in fp64, c <- c / |c| rounded to fp32, the
 // search operand -2 bf16(c), and |c|^2 := 0 since the spherical score has no norm term.
 __global__ void k_normalize(ClusterState st, int k, int nv) {
+    pdl_wait();
+    pdl_release();
     const int lane = threadIdx.x & 31;
     const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int nwarps = (gridDim.x * blockDim.x) >> 5;

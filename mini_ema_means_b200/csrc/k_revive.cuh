@@ -337,6 +337,7 @@ constexpr int kSelectWarps = kSelectThreads / 32;
 
 __global__ void __launch_bounds__(kSelectThreads) k_revive_select(const float* __restrict__ N, int k, double tau, uint64_t seed,
                                                         int64_t t, int mode, ReviveScratch sc, int* err) {
+    pdl_wait();
     __shared__ double red[32];
     __shared__ int32_t wcount[32];
     __shared__ int32_t base_s;
@@ -595,6 +596,8 @@ __global__ void __launch_bounds__(kSelectThreads) k_revive_select(const float* _
 // Dead clusters take their half of the donor (reads the donors' state before
 // k_revive_donors changes it).
 __global__ void k_revive_dead(ClusterState st, int nv, ReviveScratch sc) {
+    pdl_wait();
+    pdl_release();
     const int lane = threadIdx.x & 31;
     const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int nwarps = (gridDim.x * blockDim.x) >> 5;
@@ -635,6 +638,8 @@ __global__ void k_revive_dead(ClusterState st, int nv, ReviveScratch sc) {
 
 // Each donor, once, after all its splits: c_d (1 + eps s)^m, N_d / 2^m, S = N c.
 __global__ void k_revive_donors(ClusterState st, int nv, ReviveScratch sc) {
+    pdl_wait();
+    pdl_release();
     const int lane = threadIdx.x & 31;
     const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int nwarps = (gridDim.x * blockDim.x) >> 5;
@@ -675,6 +680,8 @@ __global__ void k_revive_donors(ClusterState st, int nv, ReviveScratch sc) {
 // Resample arm: each dead cluster restarts from a row of the current batch.
 __global__ void k_revive_resample(ClusterState st, int nv, ReviveScratch sc, const __nv_bfloat16* __restrict__ Xb,
                                   int rows, uint64_t seed, int64_t t) {
+    pdl_wait();
+    pdl_release();
     const int lane = threadIdx.x & 31;
     const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int nwarps = (gridDim.x * blockDim.x) >> 5;

@@ -235,6 +235,29 @@ def test_step_graphs_match_direct_launches(em):
 
 
 @pytest.mark.parametrize("graphs", [0, 1])
+def test_dependent_launches_match_plain_launches(em, graphs):
+    """Letting each kernel of a step launch while its predecessor finishes
+    (programmatic dependent launch, every kernel waiting on the device) gives the
+    same run, bit for bit, as plain stream-ordered launches: with revivals, the
+    FP8 search and spherical e-means too."""
+    x = synth.hand_shape(5000, 96, 30, seed=17)
+    xs = synth.hand_shape(5000, 96, 30, seed=17, normalized=True)
+    for opts, data in ((dict(), x), (dict(search_format="fp8"), x), (dict(spherical=1), xs)):
+        outs = []
+        for pdl in (0, 1):
+            m = em.Model(96, 70, seed=5, graphs=graphs, pdl=pdl, **opts)
+            m.train(data.cuda(), epochs=2.5)
+            c = torch.empty(70, 96)
+            m.centroids(c)
+            lab = torch.empty(5000, dtype=torch.int64)
+            m.labels(lab)
+            outs.append((c, lab, m.obj(), m.stats()["n_splits"]))
+            m.close()
+        assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1]), opts
+        assert np.array_equal(outs[0][2], outs[1][2]) and outs[0][3] == outs[1][3], opts
+
+
+@pytest.mark.parametrize("graphs", [0, 1])
 def test_prefetched_batches_match_inline_gathers(em, graphs):
     """Gathering the next step's rows on the side stream while a step updates gives
     the same run, bit for bit, as gathering every step's rows in turn: stepped one at
@@ -290,3 +313,27 @@ def test_exact_ties_reproduce_the_fp64_argmin(em, d):
     xq = O.search_copy_of_data(x.numpy())
     ref, _, _ = O.assign(xq, O.search_copy_of_centroids(c.numpy().astype(np.float64)))
     assert np.array_equal(labels.cpu().numpy(), ref)
+
+
+def test_failure_path_reports_timeout_and_bounds_and_recovers(em):
+    """Failure detection without a fault: a bounded device-side wait on a barrier
+    nothing arrives on gives up after its limit and the host reads EM_E_TIMEOUT; a
+    failed index check reaches the host as EM_E_BOUNDS; afterwards the same model
+    trains as a fresh one does."""
+    import time
+
+    x = synth.hand_shape(2000, 32, 10, seed=2)
+    m = em.Model(32, 20, seed=4)
+    t0 = time.time()
+    assert m.selftest(0, wait_ms=300.0) == em.EM_E_TIMEOUT
+    assert 0.25 <= time.time() - t0 < 5.0
+    assert m.selftest(1) == em.EM_E_BOUNDS
+    m.train(x.cuda(), epochs=1.0)
+    c = torch.empty(20, 32)
+    m.centroids(c)
+    ref = em.Model(32, 20, seed=4)
+    ref.train(x.cuda(), epochs=1.0)
+    c2 = torch.empty(20, 32)
+    ref.centroids(c2)
+    assert torch.equal(c, c2)
+    assert m.selftest(2) == em.EM_E_INVAL
