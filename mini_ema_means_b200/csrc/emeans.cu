@@ -336,7 +336,7 @@ struct em_model {
     bool ready_synced = true;  // the model's stream is already ordered after that gather
     bool capturing = false;    // a step range is being captured into a graph
     cudaStream_t side = nullptr, side_cap = nullptr;
-    cudaEvent_t ev_fork = nullptr, ev_gathered[2] = {nullptr, nullptr};
+    cudaEvent_t ev_fork = nullptr, ev_sel = nullptr, ev_gathered[2] = {nullptr, nullptr};
     DBuf<float> xn, dists;  // xn: |x|^2 of a full pass (assign, MSE, Lloyd)
     DBuf<int32_t> labels, cnt, rank, off, poff, perm;
     DBuf<int4> items;
@@ -669,10 +669,12 @@ static int launch_assign(em_model* m, const CUtensorMap& tmA, const __nv_bfloat1
     return EM_OK;
 }
 
+static int launch_select(em_model* m, int64_t t, cudaStream_t stream, bool pdl, CountSource src);
+
 // Group rows by label and apply the EMA update (k_offsets .. k_clusters); labels,
 // ranks and counts are already in place. `src` holds the rows (batch or data).
 static int launch_reduce(em_model* m, const __nv_bfloat16* src, int64_t rows, int nblocks_labels, double alpha,
-                         int last_pass, double* err_sum_out) {
+                         int last_pass, double* err_sum_out, int64_t select_t = -1) {
     const bool dp = m->comm != nullptr;
     double* const stats_err = m->stats.p + (int64_t)m->k * m->ld + m->k;
     const StepParams sp{alpha, last_pass, 0, dp ? m->stats.p : nullptr};
@@ -681,6 +683,17 @@ static int launch_reduce(em_model* m, const __nv_bfloat16* src, int64_t rows, in
     launch_k(m->pdl, k_offsets, 1, 1024, 0, m->stream, m->cnt.p, (int)m->k, (int)rows, m->R, m->off.p, m->poff.p, m->block_err.p,
                                          nblocks_labels, err_sum_out, m->N.p, m->N_prev.p, tie_list(m), m->err.p);
     CK(cudaGetLastError());
+    if (select_t >= 0) {
+        // The revival check after this step: its donor selection needs only the new
+        // running counts, which follow from N_prev and the segment sizes k_offsets
+        // has just written, so it runs on the side stream beside the segmented
+        // sums; the model's stream waits for it before the splits (launch_revive).
+        cudaStream_t side = m->capturing ? m->side_cap : m->side;
+        CK(cudaEventRecord(m->ev_fork, m->stream));
+        CK(cudaStreamWaitEvent(side, m->ev_fork, 0));
+        CKR(launch_select(m, select_t, side, false, CountSource{nullptr, m->N_prev.p, m->off.p, alpha}));
+        CK(cudaEventRecord(m->ev_sel, side));
+    }
     launch_k(m->pdl, k_scatter, (int)((rows + 255) / 256), 256, 0, m->stream, m->labels.p, m->rank.p, m->off.p, m->poff.p,
                                                                  (int)rows, m->R, m->perm.p, m->items.p, m->err.p);
     CK(cudaGetLastError());
@@ -724,22 +737,38 @@ static ReviveScratch revive_scratch(em_model* m) {
 static int effective_law(const em_model* m) { return m->law == 2 ? (m->d <= 16 ? 1 : 0) : m->law; }
 static double effective_tau(const em_model* m) { return m->tau < 0.0 ? (m->d <= 2 ? 0.0 : 0.1) : m->tau; }
 
-static int launch_revive(em_model* m, int64_t t, int64_t rows, const __nv_bfloat16* Xb) {
-    if (m->revival == EM_REVIVE_NONE || !(effective_tau(m) > 0.0)) return EM_OK;
+static bool revival_on(const em_model* m) { return m->revival != EM_REVIVE_NONE && effective_tau(m) > 0.0; }
+
+// The donor selection of the revival check after step t, on `stream`, reading the
+// running counts from `src`.
+static int launch_select(em_model* m, int64_t t, cudaStream_t stream, bool pdl, CountSource src) {
     const ReviveScratch sc = revive_scratch(m);
     const int smem = m->k <= kFastK ? tree32((int)m->k).bytes : (int)tree_smem_bytes(tree_layout((int)m->k), (int)m->k);
-    launch_k(m->pdl, k_revive_select, 1, kSelectThreads, smem, m->stream, m->N.p, (int)m->k, effective_tau(m), m->seed, t,
-                                                            m->revival, sc, m->err.p);
+    launch_k(pdl, k_revive_select, 1, kSelectThreads, smem, stream, src, (int)m->k, effective_tau(m), m->seed, t,
+             m->revival, sc, m->err.p);
     CK(cudaGetLastError());
+    EM_LAUNCHED(m, 1);
+    return EM_OK;
+}
+
+// The revival check after step t. `selected`: its donor selection already ran
+// (beside the step's update; launch_reduce), and the model's stream waits for it.
+static int launch_revive(em_model* m, int64_t t, int64_t rows, const __nv_bfloat16* Xb, bool selected = false) {
+    if (!revival_on(m)) return EM_OK;
+    const ReviveScratch sc = revive_scratch(m);
+    if (selected)
+        CK(cudaStreamWaitEvent(m->stream, m->ev_sel, 0));
+    else
+        CKR(launch_select(m, t, m->stream, m->pdl != 0, CountSource{m->N.p, nullptr, nullptr, 0.0}));
     const ClusterState st = cluster_state(m);
     const int blocks = grid_for(m->k * 32, 256, m->sms);
     if (m->revival == EM_REVIVE_SPLIT) {
         launch_k(m->pdl, k_revive_dead, blocks, 256, 0, m->stream, st, m->nv, sc);
         launch_k(m->pdl, k_revive_donors, blocks, 256, 0, m->stream, st, m->nv, sc);
-        EM_LAUNCHED(m, 3);
+        EM_LAUNCHED(m, 2);
     } else {
         launch_k(m->pdl, k_revive_resample, blocks, 256, 0, m->stream, st, m->nv, sc, Xb, (int)rows, m->seed, t);
-        EM_LAUNCHED(m, 2);
+        EM_LAUNCHED(m, 1);
     }
     CK(cudaGetLastError());
     return after_centroid_change(m);
@@ -879,11 +908,16 @@ static int launch_step(em_model* m, const StepPlan& p) {
     EM_LAUNCHED(m, 1);
     CKR(launch_settle(m, b.X.p, b.xn.p, m->labels.p, nullptr, m->dists.p, true, b.ids.p, m->labels_last.p,
                       capture));
-    CKR(launch_reduce(m, b.X.p, rows, nbl, p.alpha, m->finalize ? p.last_pass : 0, m->step_err.p + p.t));
+    // the revival check's donor selection beside the segmented sums (not while
+    // profiling, so that each phase is timed alone; not in data-parallel runs, whose
+    // counts come from the exchange)
+    const bool overlap = p.revive && revival_on(m) && !m->profile && m->comm == nullptr;
+    CKR(launch_reduce(m, b.X.p, rows, nbl, p.alpha, m->finalize ? p.last_pass : 0, m->step_err.p + p.t,
+                      overlap ? p.t : -1));
     span_end(m, sp, 0.0, 2.0 * rd * dd + 16.0 * rd + 14.0 * kd * dd);
     if (p.revive) {
         sp = span_begin(m, EM_PHASE_REVIVE);
-        CKR(launch_revive(m, p.t, rows, b.X.p));
+        CKR(launch_revive(m, p.t, rows, b.X.p, overlap));
         span_end(m, sp);
     }
     if (pf) {
@@ -1173,6 +1207,7 @@ em_model* em_create(int64_t d, int64_t k, uint64_t seed) {
     m->own_stream = true;
     if (cudaStreamCreateWithFlags(&m->side, cudaStreamNonBlocking) != cudaSuccess ||
         cudaEventCreateWithFlags(&m->ev_fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&m->ev_sel, cudaEventDisableTiming) != cudaSuccess ||
         cudaEventCreateWithFlags(&m->ev_gathered[0], cudaEventDisableTiming) != cudaSuccess ||
         cudaEventCreateWithFlags(&m->ev_gathered[1], cudaEventDisableTiming) != cudaSuccess)
         return bail(EM_E_CUDA, "stream or event creation failed");
@@ -1242,6 +1277,7 @@ void em_destroy(em_model* m) {
     if (m->side_cap) cudaStreamDestroy(m->side_cap);
     if (m->side) cudaStreamDestroy(m->side);
     if (m->ev_fork) cudaEventDestroy(m->ev_fork);
+    if (m->ev_sel) cudaEventDestroy(m->ev_sel);
     for (auto ev : m->ev_gathered)
         if (ev) cudaEventDestroy(ev);
     if (m->own_stream && m->stream) cudaStreamDestroy(m->stream);

@@ -502,6 +502,15 @@ __device__ __forceinline__ void load_s(const ClusterState& st, int j, const Slic
     }
 }
 
+// The running count after the step: (1 - a) N_prev + a n_j, with explicit roundings
+// so that every kernel that recomputes it (the revival selection overlaps the
+// segmented sums and derives the counts itself) gets the same fp32 value.
+__device__ __forceinline__ float ema_count(float nprev, double nj, double alpha) {
+    const double a1 = __dsub_rn(1.0, alpha);
+    if (nj == 0.0) return (float)__dmul_rn(a1, (double)nprev);
+    return (float)__dadd_rn(__dmul_rn(a1, (double)nprev), __dmul_rn(alpha, nj));
+}
+
 // EMA of one slice of cluster j from its batch sums (lanes l < nvs hold vector
 // vbase + l) and its previous sums so[]: writes S, c, the bf16 operand and the
 // closing-mean sums; slice 0 also writes N and the closing-mean count. Returns
@@ -510,7 +519,7 @@ __device__ __forceinline__ float ema_slice(const ClusterState& st, int j, double
                                            const SliceGeom& g, const double acc[8], const float so[8], int lane,
                                            double alpha, int last_pass) {
     const double a1 = 1.0 - alpha;
-    const float Nnew = (float)(a1 * (double)nprev + alpha * nj);
+    const float Nnew = ema_count(nprev, nj, alpha);
     float cn_part = 0.0f;
     if (lane < g.nvs) {
         const int v = g.vbase + lane;
@@ -636,7 +645,7 @@ __global__ void k_clusters(const int32_t* __restrict__ off, const int32_t* __res
                 row[v] = make_float4((float)(a1 * (double)x.x), (float)(a1 * (double)x.y), (float)(a1 * (double)x.z),
                                      (float)(a1 * (double)x.w));
             }
-            if (lane == 0) st.N[j] = (float)(a1 * (double)st.N_prev[j]);
+            if (lane == 0) st.N[j] = ema_count(st.N_prev[j], 0.0, sp.alpha);
         } else if (nj <= R) {
             if (lane == 0) {
                 float c = 0.0f;
@@ -701,7 +710,7 @@ __global__ void k_apply_stats(int nslices, int nv, ClusterState st, StepParams s
                 row[v] = make_float4((float)(a1 * (double)x.x), (float)(a1 * (double)x.y), (float)(a1 * (double)x.z),
                                      (float)(a1 * (double)x.w));
             }
-            if (lane == 0) st.N[j] = (float)(a1 * (double)st.N_prev[j]);
+            if (lane == 0) st.N[j] = ema_count(st.N_prev[j], 0.0, sp.alpha);
             continue;
         }
         const float nprev = st.N_prev[j];

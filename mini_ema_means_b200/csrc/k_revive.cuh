@@ -335,7 +335,20 @@ __device__ __forceinline__ int64_t draw_radix32(double* smem_d, const Tree32& TL
 constexpr int kSelectThreads = 512;
 constexpr int kSelectWarps = kSelectThreads / 32;
 
-__global__ void __launch_bounds__(kSelectThreads) k_revive_select(const float* __restrict__ N, int k, double tau, uint64_t seed,
+// Where the selection reads the running counts: N itself, or (off set) the counts
+// this step's update is writing, derived from N_prev and the segment sizes with the
+// update's own arithmetic (ema_count), so that the selection can run beside it.
+struct CountSource {
+    const float* N;
+    const float* N_prev;
+    const int32_t* off;
+    double alpha;
+    __device__ __forceinline__ float operator()(int j) const {
+        return off ? ema_count(N_prev[j], (double)(off[j + 1] - off[j]), alpha) : N[j];
+    }
+};
+
+__global__ void __launch_bounds__(kSelectThreads) k_revive_select(CountSource N, int k, double tau, uint64_t seed,
                                                         int64_t t, int mode, ReviveScratch sc, int* err) {
     pdl_wait();
     __shared__ double red[32];
@@ -345,7 +358,7 @@ __global__ void __launch_bounds__(kSelectThreads) k_revive_select(const float* _
 
     // total count in a fixed order
     double part = 0.0;
-    for (int j = tid; j < k; j += kSelectThreads) part += (double)N[j];
+    for (int j = tid; j < k; j += kSelectThreads) part += (double)N(j);
     part = warp_sum(part);
     if (lane == 0) red[w] = part;
     __syncthreads();
@@ -363,7 +376,7 @@ __global__ void __launch_bounds__(kSelectThreads) k_revive_select(const float* _
     __syncthreads();
     for (int b = 0; b < k; b += kSelectThreads) {
         const int j = b + tid;
-        const bool dead = j < k && (double)N[j] < thr;
+        const bool dead = j < k && (double)N(j) < thr;
         const unsigned m = __ballot_sync(0xFFFFFFFFu, dead);
         if (lane == 0) wcount[w] = __popc(m);
         __syncthreads();
@@ -403,7 +416,7 @@ __global__ void __launch_bounds__(kSelectThreads) k_revive_select(const float* _
         double* L0 = TL.levels == 1 ? smem_d : smem_d + TL.off0;
         for (int g = w; g < TL.n1; g += kSelectWarps) {
             const int j = g * 32 + lane;
-            const float nj = j < k ? N[j] : 0.0f;
+            const float nj = j < k ? N(j) : 0.0f;
             const double v = (j < k && !((double)nj < thr)) ? (double)nj : 0.0;
             L0[g * 32 + lane] = lane_scan(v, lane);
         }
@@ -469,7 +482,7 @@ __global__ void __launch_bounds__(kSelectThreads) k_revive_select(const float* _
                     v[i] = 0.0;
                     if (j < sz) {
                         if (l == 0) {
-                            const float nj = N[j];
+                            const float nj = N(j);
                             v[i] = ((double)nj < thr) ? 0.0 : (double)nj;
                         } else {
                             v[i] = below[(int64_t)j * kRadix + kRadix - 1];  // total of child group j

@@ -337,3 +337,26 @@ def test_failure_path_reports_timeout_and_bounds_and_recovers(em):
     ref.centroids(c2)
     assert torch.equal(c, c2)
     assert m.selftest(2) == em.EM_E_INVAL
+
+
+@pytest.mark.parametrize("k", [70, 3000, 20000])
+def test_overlapped_selection_matches_serial_revival(em, k):
+    """The revival check's donor selection runs beside the segmented sums, deriving
+    the new running counts from N_prev and the segment sizes; with profiling on it
+    runs in line after the update. Both give the same run, bit for bit (dead sets,
+    donors, counts, centroids), on the radix-32 tree (k <= 16,384) and the radix-128
+    one."""
+    x = synth.hand_shape(max(4 * k, 6000), 24, max(8, k // 3), seed=k)
+    outs = []
+    for profile in (0, 1):
+        m = em.Model(24, k, seed=9, profile=profile)
+        m.train(x.cuda(), epochs=2.0)
+        c = torch.empty(k, 24)
+        m.centroids(c)
+        N = torch.empty(k)
+        m.get_state(N=N)
+        outs.append((c, N, m.obj(), m.stats()["n_splits"]))
+        m.close()
+    assert outs[0][3] > 0
+    assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
+    assert np.array_equal(outs[0][2], outs[1][2]) and outs[0][3] == outs[1][3]
