@@ -4,15 +4,22 @@
 // then update, run by `train` internally) is this kernel sequence on the model's
 // stream:
 //   k_gather        batch rows pi_pass(pos..pos+B) -> contiguous bf16 batch, |x|^2
+//                   (and E4M3 codes with the FP8 search); prefetched: the next
+//                   step's rows are gathered on a second stream beside the search
 //   k_assign_tc     nearest centroid of every batch row (tcgen05 + TMA)
 //   k_labels        labels, distances, per-cluster counts and ranks
+//   k_settle        near ties re-decided in fp64
 //   k_offsets       segment starts and work-item starts, batch error sum
 //   k_scatter       rows in label order, one work item per chunk of a cluster
 //   k_segsum        per-chunk sums (fp64) fused with the EMA update of small clusters
 //   k_clusters      large clusters (chunk sums in order), clusters without rows
-//   k_revive_*      every 5th step: dead-cluster revival
-// No host synchronisation happens inside a run; the step size of step t is
-// computed on the host (cosine schedule) and passed by value.
+//   k_normalize / k_fp8_operand   spherical rescaling / the E4M3 operand, if on
+//   k_revive_*      every 5th step: dead-cluster revival (the donor selection runs
+//                   on the second stream beside k_scatter .. k_clusters)
+// The kernels launch with programmatic stream serialization, each waiting on the
+// device for its predecessor. No host synchronisation happens inside a run; the
+// step size of step t is computed on the host (cosine schedule) and passed by
+// value; ranges of steps are captured and replayed as CUDA graphs.
 //
 // Data-parallel runs (README "Several GPUs": DistributedEmeans, one process per
 // GPU, each with its own share of the rows): every rank searches its share of each
