@@ -189,20 +189,37 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 // One 32-column chunk of a row's scores: adds |c|^2 (c4: the chunk's 32 values) to
-// the raw accumulators v (in place) and updates the running best (TOP2: best two)
-// with the lowest column on ties. Without TOP2 the chunk's minimum is taken as a
-// tree (depth 5, not a chain of 31) and only a row it improves looks for the
-// lowest column that reaches it.
+// the raw accumulators v (in place, two lanes per packed add) and updates the
+// running best (TOP2: best two) with the lowest column on ties. Without TOP2 the
+// chunk's minimum is taken as a tree of three-input minima and only a row it
+// improves looks for the lowest column that reaches it.
+// Two fp32 additions in one packed instruction (add.rn.f32x2): each lane rounds as a
+// scalar add does, so the scores are the same bits.
+__device__ __forceinline__ void add2_f32(uint32_t& a0, uint32_t& a1, float b0, float b1) {
+    asm("{\n\t.reg .b64 x, y, z;\n\t"
+        "mov.b64 x, {%0, %1};\n\t"
+        "mov.b64 y, {%2, %3};\n\t"
+        "add.rn.f32x2 z, x, y;\n\t"
+        "mov.b64 {%0, %1}, z;\n\t}"
+        : "+r"(a0), "+r"(a1)
+        : "r"(__float_as_uint(b0)), "r"(__float_as_uint(b1)));
+}
+
+// The minimum of three fp32 values in one instruction (exact).
+__device__ __forceinline__ float min3_f32(float a, float b, float c) {
+    float d;
+    asm("min.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
 template <bool TOP2>
 __device__ __forceinline__ void scan_chunk(uint32_t (&v)[32], const float4* c4, int jb, float& best, int& bidx,
                                            float& best2, int& bidx2) {
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
         const float4 cc = c4[i];
-        v[4 * i + 0] = __float_as_uint(cc.x + __uint_as_float(v[4 * i + 0]));
-        v[4 * i + 1] = __float_as_uint(cc.y + __uint_as_float(v[4 * i + 1]));
-        v[4 * i + 2] = __float_as_uint(cc.z + __uint_as_float(v[4 * i + 2]));
-        v[4 * i + 3] = __float_as_uint(cc.w + __uint_as_float(v[4 * i + 3]));
+        add2_f32(v[4 * i + 0], v[4 * i + 1], cc.x, cc.y);
+        add2_f32(v[4 * i + 2], v[4 * i + 3], cc.z, cc.w);
     }
     if (TOP2) {
 #pragma unroll
@@ -215,14 +232,15 @@ __device__ __forceinline__ void scan_chunk(uint32_t (&v)[32], const float4* c4, 
             bidx = p1 ? jb + e : bidx;
         }
     } else {
-        float m8[8];
+        // the chunk's minimum as a tree of three-input minima (32 -> 11 -> 4 -> 1)
+        float t11[11];
 #pragma unroll
-        for (int e = 0; e < 8; ++e)
-            m8[e] = fminf(fminf(__uint_as_float(v[e]), __uint_as_float(v[e + 8])),
-                          fminf(__uint_as_float(v[e + 16]), __uint_as_float(v[e + 24])));
-#pragma unroll
-        for (int e = 0; e < 4; ++e) m8[e] = fminf(m8[e], m8[e + 4]);
-        const float mn = fminf(fminf(m8[0], m8[2]), fminf(m8[1], m8[3]));
+        for (int e = 0; e < 10; ++e)
+            t11[e] = min3_f32(__uint_as_float(v[3 * e]), __uint_as_float(v[3 * e + 1]), __uint_as_float(v[3 * e + 2]));
+        t11[10] = fminf(__uint_as_float(v[30]), __uint_as_float(v[31]));
+        const float u0 = min3_f32(t11[0], t11[1], t11[2]), u1 = min3_f32(t11[3], t11[4], t11[5]);
+        const float u2 = min3_f32(t11[6], t11[7], t11[8]), u3 = fminf(t11[9], t11[10]);
+        const float mn = min3_f32(u0, u1, fminf(u2, u3));
         if (mn < best) {
             unsigned eq = 0;
 #pragma unroll
