@@ -18,7 +18,7 @@ nearest-centroid search runs on bf16 copies of the data and of the centroids
 oracle rounds both operands exactly as the method does and then computes
 distances in fp64.
 
-Readings taken where the pages are silent (each is listed in the design doc too):
+Readings taken where the pages are silent:
 
 R1  batch size rounds to the nearest power of two in log2, capped at the
     largest power of two <= n/2 ([README] "Scaling laws");
