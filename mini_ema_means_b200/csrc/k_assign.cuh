@@ -14,10 +14,12 @@
 //               TMEM accumulators and commits to mbarriers
 //   warps 2..9  epilogue: thread = accumulator row; warps w and w + 4 share the
 //               TMEM lane quadrant w % 4 and take the left and right 128 columns
-//               of the tile: tcgen05.ld, free the accumulator, add |c|^2, running
-//               argmin. The eight warps never wait for each other: each stages its
-//               own |c|^2 values and writes its own keys (one key set per column
-//               half), and the label kernel merges the key sets
+//               of the tile: tcgen05.ld of 32 columns at a time (the next load in
+//               flight while a chunk is scanned), free the accumulator after the
+//               last, add |c|^2, running argmin. The eight warps never wait for each
+//               other: each stages its own |c|^2 values and writes its own keys
+//               (one key set per column half), and the label kernel merges the key
+//               sets
 // A work unit is (128-row tile, group of 256-wide centroid tiles). Every group
 // writes its own per-row results ((order-preserving score, index) keys), two key
 // sets per group, and the label kernel merges them. With
@@ -32,10 +34,12 @@ namespace tc {
 
 constexpr int BM = 128;
 constexpr int BN = 256;
-constexpr int kThreads = 320;
-constexpr int kEpiThreads = 256;
 constexpr int kEpiWarps = 8;
-constexpr int kKeySets = 2;  // key sets per centroid-tile group (the two column halves)
+constexpr int kEpiThreads = 32 * kEpiWarps;
+constexpr int kThreads = 64 + kEpiThreads;
+constexpr int kKeySets = kEpiWarps / 4;  // key sets per centroid-tile group (the two column halves)
+constexpr int kEpiCols = BN / kKeySets;  // columns of a tile per epilogue warp
+static_assert(kEpiCols % 64 == 0, "the epilogue scans pairs of 32-column chunks");
 
 // AST ("A stationary", rows of at most 128 dims): the CTA keeps its 128-row tile of
 // the batch in shared memory for the whole work unit (two buffers, so that the
@@ -56,7 +60,7 @@ struct Cfg {
     static constexpr int kBarBytes = 256;
     // + each epilogue warp's |c|^2 values of two tiles (its 128 columns)
     static constexpr int kSmemBytes =
-        1024 + kStages * kStageBytes + kAreaBytes + kBarBytes + kEpiWarps * 2 * 128 * 4;
+        1024 + kStages * kStageBytes + kAreaBytes + kBarBytes + kEpiWarps * 2 * kEpiCols * 4;
 };
 
 // Instruction descriptor of tcgen05.mma kind::f16: fp32 accumulate (bits 4-5 = 1),
@@ -186,13 +190,26 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
         : "r"(taddr));
 }
 
-__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+// Waits for this thread's TMEM loads, with the 32 registers of the last one as
+// operands: every use of the loaded values is ordered after the wait.
+__device__ __forceinline__ void tmem_wait_ld32(uint32_t (&r)[32]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                   "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
+                   "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]),
+                   "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]),
+                   "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+                 :
+                 : "memory");
+}
 
 // One 32-column chunk of a row's scores: adds |c|^2 (c4: the chunk's 32 values) to
 // the raw accumulators v (in place, two lanes per packed add) and updates the
 // running best (TOP2: best two) with the lowest column on ties. Without TOP2 the
 // chunk's minimum is taken as a tree of three-input minima and only a row it
-// improves looks for the lowest column that reaches it.
+// improves looks for the lowest column that reaches it: first the triple of the
+// tree's lowest level, then the column within it (a 32-column equality scan here
+// made the search of d = 96 rows 8 % slower).
 // Two fp32 additions in one packed instruction (add.rn.f32x2): each lane rounds as a
 // scalar add does, so the scores are the same bits.
 __device__ __forceinline__ void add2_f32(uint32_t& a0, uint32_t& a1, float b0, float b1) {
@@ -242,11 +259,21 @@ __device__ __forceinline__ void scan_chunk(uint32_t (&v)[32], const float4* c4, 
         const float u2 = min3_f32(t11[6], t11[7], t11[8]), u3 = fminf(t11[9], t11[10]);
         const float mn = min3_f32(u0, u1, fminf(u2, u3));
         if (mn < best) {
-            unsigned eq = 0;
+            // the first triple whose minimum is mn holds the first column that is
+            // (every column of an earlier triple is above mn); then the first of its
+            // two or three columns
+            unsigned tm = 0;
 #pragma unroll
-            for (int e = 0; e < 32; ++e) eq |= (__uint_as_float(v[e]) == mn) ? (1u << e) : 0u;
+            for (int e = 0; e < 11; ++e) tm |= (t11[e] == mn) ? (1u << e) : 0u;
+            const int h = __ffs(tm) - 1;
+            float a = __uint_as_float(v[0]), b = __uint_as_float(v[1]);
+#pragma unroll
+            for (int e = 1; e < 11; ++e) {
+                a = h == e ? __uint_as_float(v[3 * e]) : a;
+                b = h == e ? __uint_as_float(v[3 * e + 1]) : b;
+            }
             best = mn;
-            bidx = jb + __ffs(eq) - 1;
+            bidx = jb + 3 * h + (a == mn ? 0 : (b == mn ? 1 : 2));
         }
     }
 }
@@ -468,27 +495,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
         // ---------------- epilogue: 8 warps, thread = accumulator row, warp = column half
         const int q = warp & 3;
-        const int half = (warp - 2) >> 2;
-        const int rl = 32 * q + lane;  // row within the tile
+        const int half = (warp - 2) >> 2;  // column part of the tile
+        const int rl = 32 * q + lane;      // row within the tile
         const uint32_t lane_base = (uint32_t)(32 * q) << 16;
-        float* cn_w = cn_s + (warp - 2) * 2 * 128;  // this warp's two |c|^2 buffers
+        float* cn_w = cn_s + (warp - 2) * 2 * kEpiCols;  // this warp's two |c|^2 buffers
         int acc = 0;
         uint32_t acc_phase = 0;
         int cnbuf = 0;
         bool ok = true;
-        // this lane's four |c|^2 values of the next tile the warp handles, one tile ahead
-        auto cn4_of = [&](int j) {
-            float4 r;
-            r.x = j + 0 < k ? cn[j + 0] : __int_as_float(0x7f800000);
-            r.y = j + 1 < k ? cn[j + 1] : __int_as_float(0x7f800000);
-            r.z = j + 2 < k ? cn[j + 2] : __int_as_float(0x7f800000);
-            r.w = j + 3 < k ? cn[j + 3] : __int_as_float(0x7f800000);
-            return r;
+        // this lane's |c|^2 values of the next tile the warp handles, one tile ahead
+        constexpr int kPer = kEpiCols / 32;
+        float cn_next[kPer];
+        auto cn_of = [&](int j) {
+#pragma unroll
+            for (int i = 0; i < kPer; ++i) cn_next[i] = j + i < k ? cn[j + i] : __int_as_float(0x7f800000);
         };
-        float4 cn_next = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+#pragma unroll
+        for (int i = 0; i < kPer; ++i) cn_next[i] = 0.0f;
         if (blockIdx.x < units) {
             const int g0 = blockIdx.x % n_split;
-            cn_next = cn4_of(g0 * tpg * BN + half * 128 + 4 * lane);
+            cn_of(g0 * tpg * BN + half * kEpiCols + kPer * lane);
         }
         for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
             const int m = u / n_split, g = u - m * n_split;
@@ -497,9 +523,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             float best2 = best;
             int bidx = 0, bidx2 = 0;
             for (int nt = nt0; nt < nt1; ++nt) {
-                float* cnb = cn_w + cnbuf * 128;
+                float* cnb = cn_w + cnbuf * kEpiCols;
                 const int j0 = nt * BN;
-                reinterpret_cast<float4*>(cnb)[lane] = cn_next;
+#pragma unroll
+                for (int i = 0; i < kPer; ++i) cnb[kPer * lane + i] = cn_next[i];
                 {
                     int jn = -1;
                     if (nt + 1 < nt1) {
@@ -508,7 +535,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const int gn = (u + (int)gridDim.x) % n_split;
                         jn = gn * tpg * BN;
                     }
-                    if (jn >= 0) cn_next = cn4_of(jn + half * 128 + 4 * lane);
+                    if (jn >= 0) cn_of(jn + half * kEpiCols + kPer * lane);
                 }
                 // the whole warp takes one decision (a lane that gave up takes the warp with it)
                 const bool got = __all_sync(0xFFFFFFFFu,
@@ -519,25 +546,30 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 tc_fence_after();
                 __syncwarp();  // also publishes this warp's |c|^2 values
-                const uint32_t tbase = tmem_base + lane_base + (uint32_t)(acc * BN + half * 128);
+                const uint32_t tbase = tmem_base + lane_base + (uint32_t)(acc * BN + half * kEpiCols);
                 const float4* c4 = reinterpret_cast<const float4*>(cnb);
-                const int jh = j0 + half * 128;
-                // two rounds of 64 columns; the accumulator goes back once the second
-                // round is in registers (one round of 128 columns needs more registers
-                // than ten warps leave, and its spills made the kernel slower)
-#pragma unroll 1
-                for (int r = 0; r < 2; ++r) {
-                    uint32_t v[2][32];
-                    tmem_ld32(tbase + r * 64, v[0]);
-                    tmem_ld32(tbase + r * 64 + 32, v[1]);
-                    tmem_wait_ld();
-                    if (r == 1) {
-                        tc_fence_before();
-                        mbar_arrive(smem_u32(&tempty[acc]));
-                    }
+                const int jh = j0 + half * kEpiCols;
+                // chunks of 32 columns, the load of the next in flight while one is
+                // scanned; the accumulator goes back once the last chunk is in registers
+                {
+                    constexpr int kChunks = kEpiCols / 32;
+                    uint32_t va[32], vb[32];
+                    tmem_ld32(tbase, va);
+                    tmem_wait_ld32(va);
 #pragma unroll
-                    for (int c = 0; c < 2; ++c)
-                        scan_chunk<TOP2>(v[c], c4 + 16 * r + 8 * c, jh + 64 * r + 32 * c, best, bidx, best2, bidx2);
+                    for (int c = 0; c < kChunks; c += 2) {
+                        tmem_ld32(tbase + 32 * (c + 1), vb);
+                        scan_chunk<TOP2>(va, c4 + 8 * c, jh + 32 * c, best, bidx, best2, bidx2);
+                        tmem_wait_ld32(vb);
+                        if (c + 2 < kChunks) {
+                            tmem_ld32(tbase + 32 * (c + 2), va);
+                        } else {
+                            tc_fence_before();
+                            mbar_arrive(smem_u32(&tempty[acc]));
+                        }
+                        scan_chunk<TOP2>(vb, c4 + 8 * (c + 1), jh + 32 * (c + 1), best, bidx, best2, bidx2);
+                        if (c + 2 < kChunks) tmem_wait_ld32(va);
+                    }
                 }
                 acc ^= 1;
                 if (acc == 0) acc_phase ^= 1u;
