@@ -528,20 +528,41 @@ static int ensure_batch_buffers(em_model* m, int64_t cap) {
     return EM_OK;
 }
 
-static int choose_split(int64_t m_tiles, int64_t n_tiles, int sms, int max_split = 8) {
-    int best = 1;
-    double best_cost = 1e300;
+// Work units of the search over m_tiles row tiles and n_tiles centroid tiles on
+// `sms` persistent CTAs. A row tile split into s groups is s units, each keeping
+// its own running minimum per row, and the epilogue's cost grows with the new
+// minima it meets; so splitting is used only where it shortens the longest CTA,
+// either for every row tile or, once the row tiles have filled whole waves, only
+// for those of the last wave (the first m_full row tiles stay whole). Candidates
+// are taken in order of split units; a later one wins only if its longest CTA
+// (in centroid tiles) is at least 1.5 % shorter.
+struct Schedule {
+    int split;
+    int m_full;
+};
+
+static Schedule choose_schedule(int64_t m_tiles, int64_t n_tiles, int sms, int max_split = 8) {
+    struct Cand {
+        double cost;
+        int64_t split_units;
+        Schedule s;
+    };
+    Cand c[8];
+    int nc = 0;
+    const int64_t waves = m_tiles / sms, m_full = waves * sms, rest = m_tiles - m_full;
     for (int s = 1; s <= 8; s <<= 1) {
         if (s > n_tiles || s > max_split) break;
-        const int64_t units = m_tiles * s;
-        const int64_t waves = (units + sms - 1) / sms;
-        const double cost = (double)waves * (double)((n_tiles + s - 1) / s);
-        if (cost < best_cost * 0.985) {
-            best_cost = cost;
-            best = s;
-        }
+        const int64_t tpg = (n_tiles + s - 1) / s;
+        c[nc++] = Cand{(double)(((m_tiles * s + sms - 1) / sms) * tpg), s > 1 ? m_tiles * s : 0, Schedule{s, 0}};
+        if (s > 1 && m_full > 0 && rest > 0)
+            c[nc++] = Cand{(double)(waves * n_tiles + ((rest * s + sms - 1) / sms) * tpg), rest * s,
+                           Schedule{s, (int)m_full}};
     }
-    return best;
+    std::stable_sort(c, c + nc, [](const Cand& a, const Cand& b) { return a.split_units < b.split_units; });
+    Cand best = c[0];
+    for (int i = 1; i < nc; ++i)
+        if (c[i].cost < best.cost * 0.985) best = c[i];
+    return best.s;
 }
 
 // Nearest-centroid search of `rows` rows described by tmA (row source A for the
@@ -551,16 +572,16 @@ static bool use_top2(const em_model* m) {
     return m->exact_ties == 1 || (m->exact_ties < 0 && m->d >= 256);
 }
 
-static int split_for(const em_model* m, int64_t rows) {
+static Schedule schedule_for(const em_model* m, int64_t rows) {
     const int64_t m_tiles = (rows + tc::BM - 1) / tc::BM;
     const int64_t n_tiles = (m->k + tc::BN - 1) / tc::BN;
-    return choose_split(m_tiles, n_tiles, m->sms);
+    return choose_schedule(m_tiles, n_tiles, m->sms);
 }
 
 // Keys the search writes for `rows` rows: two per row per key set, two key sets
 // (column halves) per centroid-tile group.
 static size_t keys_needed(const em_model* m, int64_t rows) {
-    return rows > 0 ? (size_t)split_for(m, rows) * tc::kKeySets * (size_t)rows * 2 : 0;
+    return rows > 0 ? (size_t)schedule_for(m, rows).split * tc::kKeySets * (size_t)rows * 2 : 0;
 }
 
 static TieList tie_list(em_model* m) { return TieList{m->ties.p, m->tie_n.p, m->tie_corr.p}; }
@@ -600,18 +621,19 @@ static bool ast_fits(int64_t d, int kc) {
 }
 
 static void launch_search(int kc, bool top2, bool ast, int grid, cudaStream_t stream, const CUtensorMap& tmA,
-                          const CUtensorMap& tmB, const float* cn, int k, int rows, int nkc, int n_tiles, int split,
+                          const CUtensorMap& tmB, const float* cn, int k, int rows, int nkc, int n_tiles, Schedule sc,
                           unsigned long long* keys, long long wait, int* err, bool f8 = false, bool pdl = false) {
+    const int split = sc.split, m_full = sc.m_full;
 #define EM_GO(KC, T2, AST)                                                                                 \
     launch_k(pdl, tc::k_assign_tc<KC, T2, AST>, grid, tc::kThreads, tc::Cfg<KC, AST>::kSmemBytes, stream, tmA, \
-             tmB, cn, k, rows, nkc, n_tiles, split, keys, wait, err)
+             tmB, cn, k, rows, nkc, n_tiles, split, m_full, keys, wait, err)
     if (f8) {  // E4M3 rows and operand, 128-code chunks, plain argmin
         if (ast)
             launch_k(pdl, tc::k_assign_tc<64, false, true, true>, grid, tc::kThreads, tc::Cfg<64, true>::kSmemBytes,
-                     stream, tmA, tmB, cn, k, rows, nkc, n_tiles, split, keys, wait, err);
+                     stream, tmA, tmB, cn, k, rows, nkc, n_tiles, split, m_full, keys, wait, err);
         else
             launch_k(pdl, tc::k_assign_tc<64, false, false, true>, grid, tc::kThreads, tc::Cfg<64, false>::kSmemBytes,
-                     stream, tmA, tmB, cn, k, rows, nkc, n_tiles, split, keys, wait, err);
+                     stream, tmA, tmB, cn, k, rows, nkc, n_tiles, split, m_full, keys, wait, err);
         return;
     }
     if (kc == 64) {
@@ -657,22 +679,22 @@ static int launch_assign(em_model* m, const CUtensorMap& tmA, const __nv_bfloat1
     }
     const int64_t m_tiles = (rows + tc::BM - 1) / tc::BM;
     const int64_t n_tiles = (m->k + tc::BN - 1) / tc::BN;
-    const int split = split_for(m, rows);
-    const int64_t units = m_tiles * split;
+    const Schedule sc = schedule_for(m, rows);
+    const int64_t units = sc.m_full + (m_tiles - sc.m_full) * sc.split;
     const int grid = (int)std::min<int64_t>(units, m->sms);
     if (m->fp8) {  // tmA maps E4M3 rows; chunks of 128 codes
         const int nkc8 = (int)((m->d + 127) / 128);
         const bool ast8 = (int64_t)nkc8 * tc::BM * 128 <= tc::kAstBufBytes;
         launch_search(64, false, ast8, grid, m->stream, tmA, m->tm_cq8, m->cn8.p, (int)m->k, (int)rows, nkc8,
-                      (int)n_tiles, split, m->keys.p, m->wait_cycles, m->err.p, true, m->pdl != 0);
+                      (int)n_tiles, sc, m->keys.p, m->wait_cycles, m->err.p, true, m->pdl != 0);
     } else {
         const int nkc = (int)((m->d + m->kc - 1) / m->kc);
         launch_search(m->kc, use_top2(m), ast_fits(m->d, m->kc), grid, m->stream, tmA, m->tm_cq, m->cn.p, (int)m->k,
-                      (int)rows, nkc, (int)n_tiles, split, m->keys.p, m->wait_cycles, m->err.p, false, m->pdl != 0);
+                      (int)rows, nkc, (int)n_tiles, sc, m->keys.p, m->wait_cycles, m->err.p, false, m->pdl != 0);
     }
     CK(cudaGetLastError());
     EM_LAUNCHED(m, 1);
-    m->last_split = split * tc::kKeySets;
+    m->last_split = sc.split * tc::kKeySets;
     return EM_OK;
 }
 
@@ -2030,15 +2052,15 @@ extern "C" int em_assign_noalloc(const void* X, int64_t n, int64_t d, const floa
     const int nkc = (int)((d + kc - 1) / kc);
     // the key region holds two keys for EM_NOALLOC_MAX_ROWS rows: split * kKeySets * n
     // rows at most
-    const int split = choose_split(m_tiles, n_tiles, sms,
-                                   (int)std::max<int64_t>(1, EM_NOALLOC_MAX_ROWS / (tc::kKeySets * n)));
+    const Schedule sc = choose_schedule(m_tiles, n_tiles, sms,
+                                        (int)std::max<int64_t>(1, EM_NOALLOC_MAX_ROWS / (tc::kKeySets * n)));
     const bool top2 = d >= 256;
-    const int grid = (int)std::min<int64_t>(m_tiles * split, sms);
+    const int grid = (int)std::min<int64_t>(sc.m_full + (m_tiles - sc.m_full) * sc.split, sms);
     const long long wait_cycles = (long long)(2000.0 * (double)clock_khz);
     launch_search(kc, top2, ast_fits(d, kc), grid, static_cast<cudaStream_t>(stream), tmA, tmB, cn, (int)k, (int)n,
-                  nkc, (int)n_tiles, split, keys, wait_cycles, err);
+                  nkc, (int)n_tiles, sc, keys, wait_cycles, err);
     const int oblocks = std::min(grid_for(n, 256, sms), kNaMaxBlocks);
-    k_assign_out<<<oblocks, 256, 0, stream>>>(keys, split * tc::kKeySets, xn, n, (int)k, X16, (int)d, cq, labels,
+    k_assign_out<<<oblocks, 256, 0, stream>>>(keys, sc.split * tc::kKeySets, xn, n, (int)k, X16, (int)d, cq, labels,
                                              dists, nullptr, blocks, kSquaredDistance, ScoreScale{1.0f, 1.0f, kTieRel},
                                              TieList{nullptr, nullptr, nullptr}, err);
     CK(cudaGetLastError());

@@ -22,7 +22,9 @@
 //               sets
 // A work unit is (128-row tile, group of 256-wide centroid tiles). Every group
 // writes its own per-row results ((order-preserving score, index) keys), two key
-// sets per group, and the label kernel merges them. With
+// sets per group, and the label kernel merges them. Row tiles that fill whole
+// waves of CTAs are one group each (and empty the other groups' key sets); only
+// the last wave's row tiles are split, so that it still fills the SMs. With
 // TOP2 the epilogue also keeps the second best candidate, so that near ties can be
 // settled exactly afterwards.
 #pragma once
@@ -300,12 +302,26 @@ __global__ void k_selftest(int which, long long wait_limit, int* err) {
     mbar_wait(smem_u32(&bar), 0u, wait_limit, err, &abort_flag);  // phase 0 never completes
 }
 
+// A work unit: row tile m, centroid-tile group g, centroid tiles [nt0, nt1). The
+// first m_full row tiles are one unit each, over all n_tiles centroid tiles (group
+// 0); every later row tile is n_split units of tpg tiles.
+struct Unit {
+    int m, g, nt0, nt1;
+};
+__device__ __forceinline__ Unit unit_of(int u, int m_full, int n_split, int tpg, int n_tiles) {
+    if (u < m_full) return Unit{u, 0, 0, n_tiles};
+    const int v = u - m_full;
+    const int q = v / n_split;
+    const int g = v - q * n_split;
+    return Unit{m_full + q, g, g * tpg, min(g * tpg + tpg, n_tiles)};
+}
+
 // F8: the batch rows and the centroid operand are E4M3 codes (KC = 64 only: row
 // chunks of 128 bytes = 128 codes).
 template <int KC, bool TOP2, bool AST, bool F8 = false>
 __global__ void __launch_bounds__(kThreads, 1)
     k_assign_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                const float* __restrict__ cn, int k, int rows, int nkc, int n_tiles, int n_split,
+                const float* __restrict__ cn, int k, int rows, int nkc, int n_tiles, int n_split, int m_full,
                 unsigned long long* __restrict__ keys, long long wait_limit, int* err) {
     using C = Cfg<KC, AST>;
     constexpr int S = C::kStages;
@@ -335,7 +351,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const long long drain_limit = wait_limit > 4000000000ll ? wait_limit : 4000000000ll;
     const int m_tiles = (rows + BM - 1) / BM;
     const int tpg = (n_tiles + n_split - 1) / n_split;
-    const int units = m_tiles * n_split;
+    const int units = m_full + (m_tiles - m_full) * n_split;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
@@ -382,8 +398,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t aarmed = 0, aarmed_parity = 0;  // the two A buffers (AST)
             int ua = 0;                              // units started (AST)
             for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
-                const int m = u / n_split, g = u - m * n_split;
-                const int nt0 = g * tpg, nt1 = min(nt0 + tpg, n_tiles);
+                const Unit w = unit_of(u, m_full, n_split, tpg, n_tiles);
+                const int m = w.m, nt0 = w.nt0, nt1 = w.nt1;
                 if (AST) {  // the unit's rows, once, into A buffer ua % 2
                     const int ab = ua & 1;
                     const uint32_t par = (uint32_t)(ua >> 1) & 1u;
@@ -435,9 +451,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             bool ok = true;
             int ua = 0;
             for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
-                const int m = u / n_split, g = u - m * n_split;
-                (void)m;
-                const int nt0 = g * tpg, nt1 = min(nt0 + tpg, n_tiles);
+                const Unit w = unit_of(u, m_full, n_split, tpg, n_tiles);
+                const int nt0 = w.nt0, nt1 = w.nt1;
                 const int ab = ua & 1;
                 if (AST) {
                     if (!mbar_wait(smem_u32(&afull[ab]), (uint32_t)(ua >> 1) & 1u, wait_limit, err, abort_flag)) {
@@ -512,13 +527,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         };
 #pragma unroll
         for (int i = 0; i < kPer; ++i) cn_next[i] = 0.0f;
-        if (blockIdx.x < units) {
-            const int g0 = blockIdx.x % n_split;
-            cn_of(g0 * tpg * BN + half * kEpiCols + kPer * lane);
-        }
+        if (blockIdx.x < units)
+            cn_of(unit_of(blockIdx.x, m_full, n_split, tpg, n_tiles).nt0 * BN + half * kEpiCols + kPer * lane);
         for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
-            const int m = u / n_split, g = u - m * n_split;
-            const int nt0 = g * tpg, nt1 = min(nt0 + tpg, n_tiles);
+            const Unit w = unit_of(u, m_full, n_split, tpg, n_tiles);
+            const int m = w.m, g = w.g, nt0 = w.nt0, nt1 = w.nt1;
             float best = __int_as_float(0x7f800000);  // +inf
             float best2 = best;
             int bidx = 0, bidx2 = 0;
@@ -532,8 +545,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (nt + 1 < nt1) {
                         jn = (nt + 1) * BN;
                     } else if (u + (int)gridDim.x < units) {
-                        const int gn = (u + (int)gridDim.x) % n_split;
-                        jn = gn * tpg * BN;
+                        jn = unit_of(u + (int)gridDim.x, m_full, n_split, tpg, n_tiles).nt0 * BN;
                     }
                     if (jn >= 0) cn_of(jn + half * kEpiCols + kPer * lane);
                 }
@@ -583,6 +595,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 unsigned long long* out = keys + ((int64_t)(kKeySets * g + half) * rows + row) * 2;
                 out[0] = best < __int_as_float(0x7f800000) ? pack_key(best, (uint32_t)bidx) : kEmptyKey;
                 out[1] = TOP2 && best2 < __int_as_float(0x7f800000) ? pack_key(best2, (uint32_t)bidx2) : kEmptyKey;
+                // a whole row tile also empties the other groups' key sets, which the
+                // label kernel reads for every row
+                if (u < m_full)
+                    for (int g2 = 1; g2 < n_split; ++g2)
+                        reinterpret_cast<ulonglong2*>(keys)[(int64_t)(kKeySets * g2 + half) * rows + row] =
+                            make_ulonglong2(kEmptyKey, kEmptyKey);
             }
         }
     }

@@ -107,7 +107,11 @@ def test_host_input_goes_through_the_same_path(em):
 
 
 @pytest.mark.parametrize("n,d,k", [(1, 32, 1), (127, 64, 5), (129, 96, 257), (5000, 768, 4096),
-                                   (3000, 128, 600), (777, 100, 300), (20000, 32, 64), (4100, 256, 2048)])
+                                   (3000, 128, 600), (777, 100, 300), (20000, 32, 64), (4100, 256, 2048),
+                                   # more row tiles than SMs: whole row tiles first, the last
+                                   # wave's split into centroid-tile groups (on 148 SMs: 296
+                                   # whole and 17 split 8 ways; 148 whole and 9 split 2 ways)
+                                   (40000, 32, 2000), (20000, 40, 300), (20000, 256, 512)])
 def test_assign_and_mse_match_oracle(em, n, d, k):
     g = torch.Generator().manual_seed(n * 31 + k)
     x = synth.hand_shape(n, d, 16, seed=n + k)
