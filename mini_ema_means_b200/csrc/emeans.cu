@@ -565,8 +565,8 @@ static Schedule choose_schedule(int64_t m_tiles, int64_t n_tiles, int sms, int m
     return best.s;
 }
 
-// Nearest-centroid search of `rows` rows described by tmA (row source A for the
-// SIMT path) into m->keys (which the caller has reset to the empty key).
+// Whether the search keeps the best two (score, index) keys per key set, so that
+// near ties can be settled exactly afterwards.
 static bool use_top2(const em_model* m) {
     if (m->fp8) return false;  // the FP8 search keeps the plain argmin (no exact settling of ties)
     return m->exact_ties == 1 || (m->exact_ties < 0 && m->d >= 256);
@@ -666,6 +666,8 @@ static bool search_smem_attributes() {
 #undef EM_ATTR
 }
 
+// Nearest-centroid search of `rows` rows described by tmA (row source A for the
+// SIMT path) into m->keys. Every key set the label kernel reads is written.
 static int launch_assign(em_model* m, const CUtensorMap& tmA, const __nv_bfloat16* A, int64_t rows) {
     if (rows <= 0) return EM_OK;
     if (m->keys.cap < keys_needed(m, rows)) return fail(EM_E_STATE, "search key buffer too small");
@@ -1577,7 +1579,7 @@ int em_lloyd(em_model* m, const void* X, int64_t n, int64_t iters) {
     const int nbl = (int)((n + 255) / 256);
     for (int64_t it = 0; it < iters; ++it) {
         if (!m->fp8) {
-            k_rownorm_keys<<<grid_for(n * 32, 256, m->sms), 256, 0, m->stream>>>(m->X, n, m->ld, m->xn.p, nullptr);
+            k_rownorm<<<grid_for(n * 32, 256, m->sms), 256, 0, m->stream>>>(m->X, n, m->ld, m->xn.p);
             CK(cudaGetLastError());
             EM_LAUNCHED(m, 1);
         }
@@ -1616,7 +1618,7 @@ static int assign_pass(em_model* m, const void* X, int64_t n, int64_t* labels_de
         }
         CKR(fp8_rows(m, A, n, &tmx));
     } else {
-        k_rownorm_keys<<<grid_for(n * 32, 256, m->sms), 256, 0, m->stream>>>(A, n, m->ld, m->xn.p, nullptr);
+        k_rownorm<<<grid_for(n * 32, 256, m->sms), 256, 0, m->stream>>>(A, n, m->ld, m->xn.p);
         CK(cudaGetLastError());
         EM_LAUNCHED(m, 1);
         CKR(make_tmap(&tmx, A, n, (int)m->d, m->ld, tc::BM, m->kc));
@@ -2046,7 +2048,7 @@ extern "C" int em_assign_noalloc(const void* X, int64_t n, int64_t d, const floa
     const auto X16 = reinterpret_cast<const __nv_bfloat16*>(X);
     CK(cudaMemsetAsync(err, 0, sizeof(int), stream));  // the previous call's error word is stale
     k_operand_from_centroids<<<grid_for(k * 32, 256, sms), 256, 0, stream>>>(centroids, (int)k, (int)d, cq, cn);
-    k_rownorm_keys<<<grid_for(n * 32, 256, sms), 256, 0, stream>>>(X16, n, (int)d, xn, nullptr);
+    k_rownorm<<<grid_for(n * 32, 256, sms), 256, 0, stream>>>(X16, n, (int)d, xn);
     const int64_t m_tiles = (n + tc::BM - 1) / tc::BM;
     const int64_t n_tiles = (k + tc::BN - 1) / tc::BN;
     const int nkc = (int)((d + kc - 1) / kc);

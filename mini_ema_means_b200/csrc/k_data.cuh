@@ -259,10 +259,9 @@ __global__ void k_gather(const __nv_bfloat16* __restrict__ X, int64_t n, int ld,
     }
 }
 
-// |x|^2 of every row of X in place (no copy) and a reset search key: the prologue
-// of a full assignment pass (em_assign, em_mse, Lloyd iterations).
-__global__ void k_rownorm_keys(const __nv_bfloat16* __restrict__ X, int64_t rows, int ld, float* __restrict__ xn,
-                               unsigned long long* __restrict__ keys) {
+// |x|^2 of every row of X in place (no copy): the prologue of a full assignment
+// pass (em_assign, em_mse, Lloyd iterations).
+__global__ void k_rownorm(const __nv_bfloat16* __restrict__ X, int64_t rows, int ld, float* __restrict__ xn) {
     pdl_wait();
     const int lane = threadIdx.x & 31;
     const int64_t warp = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
@@ -278,10 +277,7 @@ __global__ void k_rownorm_keys(const __nv_bfloat16* __restrict__ X, int64_t rows
             for (int i = 0; i < 8; ++i) acc = fmaf(x[i], x[i], acc);
         }
         acc = warp_sum(acc);
-        if (lane == 0) {
-            xn[r] = acc;
-            if (keys) keys[r] = kEmptyKey;
-        }
+        if (lane == 0) xn[r] = acc;
     }
 }
 
