@@ -22,9 +22,10 @@
 //               sets
 // A work unit is (128-row tile, group of 256-wide centroid tiles). Every group
 // writes its own per-row results ((order-preserving score, index) keys), two key
-// sets per group, and the label kernel merges them. Row tiles that fill whole
-// waves of CTAs are one group each (and empty the other groups' key sets); only
-// the last wave's row tiles are split, so that it still fills the SMs. With
+// sets per group, and the label kernel merges them. The host either splits every
+// row tile into the same number of groups or, when the row tiles fill whole waves
+// of CTAs before a partial one, keeps those whole (one group each, emptying the
+// other groups' key sets) and splits only the last wave's row tiles. With
 // TOP2 the epilogue also keeps the second best candidate, so that near ties can be
 // settled exactly afterwards.
 #pragma once
