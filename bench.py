@@ -132,7 +132,8 @@ def oracle_sample_rate(w, xt_dev, seconds, rows_per_step=None, log_prefix="cpu",
     N = np.zeros(w.k)
     S = np.zeros((w.k, w.d))
     t_total, rows_total, steps = 0.0, 0, 0
-    while t_total < seconds and steps < rec["total_steps"]:
+    # the batches of pass 0 (a full batch each, the last one possibly shorter)
+    while t_total < seconds and steps < rec["total_steps"] and steps * B < w.n_train:
         ids = torch.from_numpy(order[steps * B:(steps + 1) * B]).to(xt_dev.device)
         xb = O.search_copy_of_data(xt_dev.index_select(0, ids).float().cpu().numpy())
         t0 = time.perf_counter()
@@ -142,9 +143,9 @@ def oracle_sample_rate(w, xt_dev, seconds, rows_per_step=None, log_prefix="cpu",
         steps += 1
         log(f"[{log_prefix}] oracle step {steps}: {len(xb)} rows, {t_total:.1f} s so far")
     threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
-    sample = (f"{steps} oracle steps of {B} rows each (search against all {w.k} centroids, per-cluster sums, "
-              f"EMA update{', spherical' if spherical else ''}) from pass 0 of {w.name}; {t_total:.1f} s of host "
-              f"time")
+    sample = (f"{steps} oracle steps, {rows_total} rows in all (batches of up to {B}; search against all {w.k} "
+              f"centroids, per-cluster sums, EMA update{', spherical' if spherical else ''}) from pass 0 of "
+              f"{w.name}; {t_total:.3g} s of host time")
     return rows_total / t_total, sample, threads
 
 
@@ -446,13 +447,14 @@ def run_reference(args):
     # calibrate the rows of one step so that warm-up + timed steps fit the budget
     v0, _, _ = oracle_sample_rate(w, xt, 0.1, rows_per_step=512, log_prefix="ref-calibrate",
                                   spherical=args.spherical)
-    rows = int(max(64, min(65536, v0 * budget / max(args.steps + args.warmup, 1))))
     import numpy as np
     from threadpoolctl import threadpool_info
 
     from oracle import emeans_oracle as O
 
     rec = O.recipe(w.n_train, w.k, w.epochs)
+    # at most one batch of the workload (and never more rows than it has)
+    rows = int(max(1, min(rec["batch_size"], w.n_train, max(64, v0 * budget / max(args.steps + args.warmup, 1)))))
     order = O.pass_order(w.n_train, 1234, 0)
     start = O.starting_rows(w.n_train, w.k, 1234)
     c = O.search_copy_of_data(xt.index_select(0, torch.from_numpy(start).to(xt.device)).float().cpu().numpy())
@@ -462,15 +464,18 @@ def run_reference(args):
 
     def one(t):
         nonlocal N, S, c
-        ids = order[(t * rows) % (w.n_train - rows):][:rows]
+        start = (t * rows) % (w.n_train - rows + 1)
+        ids = order[start:start + rows]
         xb = O.search_copy_of_data(xt.index_select(0, torch.from_numpy(ids).to(xt.device)).float().cpu().numpy())
         t0 = time.perf_counter()
         N, S, c = oracle_step(O, xb, c, N, S, w.k, t, rec, args.spherical)
-        return time.perf_counter() - t0
+        return time.perf_counter() - t0, len(xb)
 
     for t in range(args.warmup):
         one(t)
-    sec = sum(one(args.warmup + t) for t in range(args.steps))
+    timed = [one(args.warmup + t) for t in range(args.steps)]
+    sec = sum(x[0] for x in timed)
+    assert all(x[1] == rows for x in timed)
     threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
     value = args.steps * rows / sec
     sample = (f"{args.steps} oracle steps of {rows} rows each from pass 0 of {w.name} (search against all "
