@@ -289,8 +289,11 @@ def run_ours(args, rank, world):
                    "batch_size": rec["batch_size"], "alpha0": round(rec["alpha0"], 6), "prefetch": args.prefetch,
                    "pdl": args.pdl,
                    "steps_per_run": total,
-                   "l2": "inputs larger than L2: the fp32 training matrix (%.2f GB) and its bf16 copy are re-read "
-                         "in a fresh random order every pass" % (w.n_train * w.d * 4 / 1e9),
+                   "l2": ("inputs larger than L2: the fp32 training matrix (%.2f GB) and its bf16 copy are re-read "
+                          "in a fresh random order every pass" % (w.n_train * w.d * 4 / 1e9)
+                          if w.n_train * w.d * 4 > L2_BYTES else
+                          "inputs fit in L2 (the fp32 training matrix is %.1f MB) and L2 is not flushed between "
+                          "steps" % (w.n_train * w.d * 4 / 1e6)),
                    "parallelism": (f"data-parallel dp{world} (NCCL all-reduce of the batch statistics)" if args.dp
                                    else "replicas" if world > 1 else "single GPU")},
     }
@@ -566,6 +569,8 @@ def run_ablation(args):
                               "test_mse_mean": statistics.mean(r["test_mse"] for r in rows)}
     return out
 
+
+L2_BYTES = 126e6  # the B200's L2 (126 MB)
 
 # DRAM bytes per assignment launch of the bench's batch, from an ncu capture of the
 # current kernel (profiles/k_assign_tc_emb768_262144rows.md: 262,144 rows, scaled
