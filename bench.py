@@ -336,7 +336,7 @@ def run_ours(args, rank, world):
     if rank == 0 and not args.no_extras:
         out["lloyd25"] = lloyd25(m, w, xt, xs, rec)
     if not args.no_e2e:
-        out["e2e"] = e2e(em, w, xt, stream, world, dev, spherical=args.spherical, dp=args.dp)
+        out["e2e"] = e2e(em, w, xt, stream, world, dev, spherical=args.spherical, dp=args.dp, search=args.search)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, sample, threads = oracle_sample_rate(w, xt, args.cpu_seconds, spherical=args.spherical)
         out["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample}
@@ -402,13 +402,14 @@ def lloyd25(m, w, xt, xs, rec):
             "final_ratio": final / target, "checkpoints": history}
 
 
-def e2e(em, w, xt, stream, world, dev, spherical=False, dp=False):
+def e2e(em, w, xt, stream, world, dev, spherical=False, dp=False, search="bf16"):
     """em_train through the C ABI with a pinned host matrix: H2D copy, training and
-    the centroid read-back inside the timed region."""
+    the centroid read-back inside the timed region, with the timed arm's method and
+    search format."""
     import torch
 
     xh = xt.cpu().pin_memory()
-    m = em.Model(w.d, w.k, seed=1234, spherical=int(spherical))
+    m = em.Model(w.d, w.k, seed=1234, spherical=int(spherical), search_format=search)
     m.set_stream(stream.cuda_stream)
     if dp:
         dp_join(em, m, world)
@@ -433,8 +434,9 @@ def e2e(em, w, xt, stream, world, dev, spherical=False, dp=False):
     return {"value": rows / sec, "unit": UNIT,
             "h2d_bytes_per_step": xh.numel() * xh.element_size() / steps,
             "d2h_bytes_per_step": (w.k * w.d * 4) / steps,
-            "what": "em_train on a pinned host fp32 matrix (copied to the device inside the call) + centroid "
-                    "read-back, one whole 5-epoch run, host wall clock"}
+            "what": f"em_train on a pinned host {'fp32' if xh.dtype == torch.float32 else 'bf16'} matrix (copied to "
+                    f"the device inside the call) + centroid read-back, one whole {w.epochs:g}-epoch run, "
+                    f"{search} search, host wall clock"}
 
 
 # ---------------------------------------------------------------- reference arm (the oracle)
