@@ -123,6 +123,8 @@ _SIGS = {
     "em_compute_recipe": (ctypes.c_int, [_I64, _I64, ctypes.c_double, ctypes.c_int, _I64, ctypes.c_double,
                                          ctypes.POINTER(em_recipe_t)]),
     "em_permutation": (ctypes.c_int, [_I64, ctypes.c_uint64, ctypes.c_int, _I64, _P, _I64, _P]),
+    "em_search_schedule": (ctypes.c_int, [_I64, _I64, ctypes.c_int, ctypes.POINTER(ctypes.c_int),
+                                          ctypes.POINTER(ctypes.c_int)]),
     "em_create": (_P, [_I64, _I64, ctypes.c_uint64]),
     "em_destroy": (None, [_P]),
     "em_set_option": (ctypes.c_int, [_P, ctypes.c_int, ctypes.c_double]),
@@ -202,6 +204,15 @@ def compute_recipe(n, k, epochs, law=0, batch_size=0, alpha0=0.0) -> dict:
     check(em_compute_recipe(n, k, float(epochs), int(law), int(batch_size), float(alpha0), ctypes.byref(r)),
           "em_compute_recipe")
     return r.as_dict()
+
+
+def search_schedule(rows, k, sms):
+    """(split, m_full) of the nearest-centroid search for `rows` rows and k
+    centroids on `sms` SMs (host code)."""
+    split, m_full = ctypes.c_int(), ctypes.c_int()
+    check(em_search_schedule(int(rows), int(k), int(sms), ctypes.byref(split), ctypes.byref(m_full)),
+          "em_search_schedule")
+    return split.value, m_full.value
 
 
 def permutation(n, seed, stream, which, idx):

@@ -1202,6 +1202,14 @@ int em_permutation(int64_t n, uint64_t seed, int stream, int64_t which, const in
     return EM_OK;
 }
 
+int em_search_schedule(int64_t rows, int64_t k, int sms, int* split, int* m_full) {
+    if (rows < 1 || k < 1 || sms < 1 || !split || !m_full) return fail(EM_E_INVAL, "bad search schedule arguments");
+    const Schedule sc = choose_schedule((rows + tc::BM - 1) / tc::BM, (k + tc::BN - 1) / tc::BN, sms);
+    *split = sc.split;
+    *m_full = sc.m_full;
+    return EM_OK;
+}
+
 em_model* em_create(int64_t d, int64_t k, uint64_t seed) {
     if (d < 1 || d > 8192 || k < 1 || k > (1ll << 30)) {
         fail(EM_E_INVAL, "need 1 <= d <= 8192 and 1 <= k <= 2^30");

@@ -1,6 +1,7 @@
 """CPU checks of the C ABI library: it loads, exports every declared entry point,
-and its host-side code (recipe, per-pass order) agrees with the oracle. No GPU
-compute is called here."""
+and its host-side code agrees with the oracle (recipe, per-pass order) and with the
+search's documented work units (the search schedule). No GPU compute is called
+here."""
 
 import os
 import re
@@ -115,3 +116,64 @@ def test_create_without_gpu_fails_loudly(em):
     with pytest.raises(em.EmeansError) as e:
         em.Model(32, 64)
     assert e.value.code == em.EM_E_NODEVICE
+
+
+# The search's work units, as the search kernel takes them: the first m_full 128-row
+# tiles are one unit each over all ceil(k / 256) centroid tiles; every later row
+# tile is `split` units, group g covering centroid tiles [g * tpg, (g + 1) * tpg)
+# with tpg = ceil(n_tiles / split); min(units, sms) persistent CTAs take the units
+# round-robin.
+def _units(m_tiles, n_tiles, split, m_full):
+    tpg = -(-n_tiles // split)
+    units = m_full + (m_tiles - m_full) * split
+    u = np.arange(units)
+    whole = u < m_full
+    v = u - m_full
+    m = np.where(whole, u, m_full + v // split)
+    g = np.where(whole, 0, v % split)
+    nt0 = np.where(whole, 0, g * tpg)
+    nt1 = np.where(whole, n_tiles, np.minimum(nt0 + tpg, n_tiles))
+    return u, m, g, np.maximum(nt1 - nt0, 0)
+
+
+@pytest.mark.parametrize("rows,k,expect", [
+    (65536, 16384, (2, 444)),   # deep96 batch: 512 row tiles, only the last wave's 68 split
+    (65536, 4096, (2, 444)),    # emb768 batch
+    (1048576, 65536, (1, 0)),   # sift128 batch: 8192 row tiles fill the waves nearly evenly
+    (40000, 2000, (8, 296)),
+    (20000, 300, (2, 148)),
+    (3000, 40, (1, 0)),         # one centroid tile: never split
+    (1, 1, (1, 0)),
+])
+def test_search_schedule_choices(em, rows, k, expect):
+    assert em.search_schedule(rows, k, 148) == expect
+
+
+def test_search_schedule_covers_every_tile_once_and_keeps_the_longest_cta(em):
+    for sms in (148, 132, 7):
+        for rows in (1, 127, 128, 5000, 18944, 20000, 40000, 65536, 131072, 1048576):
+            for k in (1, 256, 300, 2000, 4096, 16384, 65536):
+                split, m_full = em.search_schedule(rows, k, sms)
+                m_tiles, n_tiles = -(-rows // 128), -(-k // 256)
+                assert split in (1, 2, 4, 8) and (split == 1 or split <= n_tiles)
+                assert m_full == 0 or m_full < m_tiles
+                assert m_full % sms == 0 and (m_full == 0 or split > 1)
+                u, m, g, length = _units(m_tiles, n_tiles, split, m_full)
+                # every row tile: all of its centroid tiles, in one unit or in `split`
+                assert np.array_equal(np.bincount(m, weights=length, minlength=m_tiles), np.full(m_tiles, n_tiles))
+                per_row = np.bincount(m, minlength=m_tiles)
+                assert np.all(per_row[:m_full] == 1) and np.all(per_row[m_full:] == split)
+                # the longest CTA is within 1.5 % of the best schedule that splits every
+                # row tile the same number of ways
+                grid = min(len(u), sms)
+                longest = np.bincount(u % grid, weights=length).max()
+                best_uniform = min(-(-(m_tiles * s) // sms) * -(-n_tiles // s) for s in (1, 2, 4, 8)
+                                   if s == 1 or s <= n_tiles)
+                assert longest <= best_uniform / 0.985, (sms, rows, k, split, m_full, longest, best_uniform)
+
+
+def test_search_schedule_argument_errors(em):
+    for args in ((0, 10, 148), (10, 0, 148), (10, 10, 0)):
+        with pytest.raises(em.EmeansError) as e:
+            em.search_schedule(*args)
+        assert e.value.code == em.EM_E_INVAL
