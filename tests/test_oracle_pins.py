@@ -316,6 +316,12 @@ def test_dead_set_uses_strict_threshold_on_mean_count():
     assert dead.tolist() == [1]
     N2 = np.array([10.0, 1.0, 1.0, 1.0, 1.0, 1.0])  # mean 2.5, threshold 0.25 -> none dead
     assert len(O.revive(N2, N2[:, None] * c, c, 4, 1)[3]) == 0
+    # a count exactly at the threshold is not below it: mean 1.25, and 0.1 x 1.25
+    # rounds to 0.125 exactly in fp64
+    N3 = np.array([0.125, 1.875, 1.5, 1.5])
+    assert 0.1 * (N3.sum() / 4) == 0.125
+    assert len(O.revive(N3, N3[:, None] * c[:4], c[:4], 4, 1, tau=0.1)[3]) == 0
+    assert O.revive(N3 * [0.999, 1, 1, 1], N3[:, None] * c[:4], c[:4], 4, 1, tau=0.1)[3].tolist() == [0]
 
 
 def test_split_halves_count_and_keeps_sums_consistent():
