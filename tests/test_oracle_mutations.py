@@ -15,7 +15,7 @@ from tests import test_oracle_pins as P
 _orig = {name: getattr(O, name) for name in (
     "ema_update", "alpha_at", "squared_distances", "assign", "batch_stats", "f32_to_bf16", "revive",
     "split_sign", "philox4x64_10", "pass_order", "batch_size_law", "alpha0_law", "unit_rows", "e4m3_round",
-    "fp8_calibrate", "assign_dot", "round_batch")}
+    "fp8_calibrate", "assign_dot", "round_batch", "EmeansOracle")}
 
 
 # ---------------------------------------------------------------- the mistakes
@@ -151,6 +151,61 @@ def round_batch_floor(b_raw, n):
     return int(max(1, min(b, cap)))
 
 
+def revive_donor_uniform(N, S, c, t, seed, mode="split", tau=O.DEFAULT_TAU, batch_rows=None):
+    """Donors drawn uniformly among the live clusters instead of in proportion to
+    their counts (the same dead set: every live count replaced by 1)."""
+    k = len(N)
+    live = ~(N < tau * (N.sum() / k))
+    return _orig["revive"](np.where(live, 1.0, 0.0), S, c, t, seed, mode=mode, tau=tau, batch_rows=batch_rows)
+
+
+class ClosingMeanForgotten(O.EmeansOracle):
+    """finalize keeps the running centroids: the closing mean of the last pass is
+    never taken."""
+
+    def finalize(self):
+        self.closing = False
+        return super().finalize()
+
+
+def alpha_off_by_one(t, total_steps, alpha0):
+    """Step t takes the step size of step t + 1."""
+    return _orig["alpha_at"](t + 1, total_steps, alpha0)
+
+
+def ema_centroid_before_update(N, S, c, n_j, s_j, alpha):
+    """c = S / N taken from the statistics before the update."""
+    N2, S2, _ = _orig["ema_update"](N, S, c, n_j, s_j, alpha)
+    c = c.copy()
+    live = N > 0
+    c[live] = S[live] / N[live][:, None]
+    return N2, S2, c
+
+
+def bf16_round_half_up(x32):
+    """bf16 rounding with halfway cases rounded up (in magnitude) instead of to even."""
+    x32 = np.ascontiguousarray(x32, dtype=np.float32)
+    u = x32.view(np.uint32).astype(np.uint64)
+    r = ((u + np.uint64(0x8000)) >> np.uint64(16)) << np.uint64(16)
+    return (r & np.uint64(0xFFFFFFFF)).astype(np.uint32).view(np.float32)
+
+
+def e4m3_no_saturation(v):
+    """Values beyond 448 are not clamped to the largest finite code."""
+    v = np.asarray(v, dtype=np.float64)
+    r = _orig["e4m3_round"](v)
+    return np.where(np.abs(v) > O.E4M3_MAX, np.nan, r)
+
+
+def fp8_scale_not_a_power_of_two(xq):
+    """The scale maps the largest |x - shift| exactly onto 448."""
+    shift, _ = _orig["fp8_calibrate"](xq)
+    sample = np.asarray(xq[:O.FP8_CALIBRATION_ROWS], dtype=np.float32)
+    half = np.maximum(sample.max(axis=0) - shift, shift - sample.min(axis=0)).astype(np.float64)
+    m = float(half.max()) if half.size else 0.0
+    return shift, (O.E4M3_MAX / m if m > 0 else 1.0)
+
+
 MUTATIONS = [
     ("ema_update", ema_without_decay, [P.test_constant_step_single_cluster_is_exponentially_weighted_mean]),
     ("ema_update", ema_weights_swapped, [P.test_full_batch_unit_step_is_one_lloyd_iteration,
@@ -177,6 +232,15 @@ MUTATIONS = [
     ("e4m3_round", e4m3_ties_away_from_zero, [P.test_e4m3_rounding_matches_torch_and_breaks_ties_to_even]),
     ("fp8_calibrate", fp8_shift_is_the_mean, [P.test_fp8_calibration_is_midrange_shift_and_largest_power_of_two]),
     ("assign_dot", assign_dot_lowest_similarity, [P.test_assign_dot_matches_brute_force_with_lowest_index_ties]),
+    ("revive", revive_donor_uniform, [P.test_donor_frequency_proportional_to_size]),
+    ("EmeansOracle", ClosingMeanForgotten, [P.test_closing_mean_is_exact_mean_of_last_pass_assignments]),
+    ("alpha_at", alpha_off_by_one, [P.test_cosine_schedule_endpoints_and_shape]),
+    ("ema_update", ema_centroid_before_update, [P.test_full_batch_unit_step_is_one_lloyd_iteration,
+                                                P.test_constant_step_single_cluster_is_exponentially_weighted_mean]),
+    ("f32_to_bf16", bf16_round_half_up, [P.test_bf16_rounding_matches_torch_cast]),
+    ("e4m3_round", e4m3_no_saturation, [P.test_e4m3_rounding_matches_torch_and_breaks_ties_to_even]),
+    ("fp8_calibrate", fp8_scale_not_a_power_of_two,
+     [P.test_fp8_calibration_is_midrange_shift_and_largest_power_of_two]),
 ]
 
 
