@@ -15,7 +15,7 @@ from tests import test_oracle_pins as P
 _orig = {name: getattr(O, name) for name in (
     "ema_update", "alpha_at", "squared_distances", "assign", "batch_stats", "f32_to_bf16", "revive",
     "split_sign", "philox4x64_10", "pass_order", "batch_size_law", "alpha0_law", "unit_rows", "e4m3_round",
-    "fp8_calibrate", "assign_dot", "round_batch", "EmeansOracle")}
+    "fp8_calibrate", "assign_dot", "round_batch", "EmeansOracle", "draw_uniform")}
 
 
 # ---------------------------------------------------------------- the mistakes
@@ -206,6 +206,28 @@ def fp8_scale_not_a_power_of_two(xq):
     return shift, (O.E4M3_MAX / m if m > 0 else 1.0)
 
 
+def rows_per_pass_floor(n, epochs):
+    """A fractional last pass is dropped (the epochs rounded down)."""
+    import math
+    return [n] * int(math.floor(epochs)) or [n]
+
+
+def draw_uniform_ignores_step(seed, stream, t, j):
+    """The step is left out of the counter: every revival check draws the same."""
+    return _orig["draw_uniform"](seed, stream, 0, j)
+
+
+def spherical_error_one_minus(xq, c64):
+    """1 - similarity instead of 2 - 2 x similarity."""
+    return float((1.0 - O.assign_dot(xq, O.search_copy_of_centroids(c64))[1]).mean())
+
+
+def fp8_codes_scale_before_shift(v, shift, scale):
+    """v x scale - shift: the shift is applied after the scaling."""
+    d32 = (np.asarray(v, dtype=np.float64) * scale).astype(np.float32) - np.asarray(shift, dtype=np.float32)
+    return O.e4m3_round(d32.astype(np.float64))
+
+
 MUTATIONS = [
     ("ema_update", ema_without_decay, [P.test_constant_step_single_cluster_is_exponentially_weighted_mean]),
     ("ema_update", ema_weights_swapped, [P.test_full_batch_unit_step_is_one_lloyd_iteration,
@@ -241,10 +263,18 @@ MUTATIONS = [
     ("e4m3_round", e4m3_no_saturation, [P.test_e4m3_rounding_matches_torch_and_breaks_ties_to_even]),
     ("fp8_calibrate", fp8_scale_not_a_power_of_two,
      [P.test_fp8_calibration_is_midrange_shift_and_largest_power_of_two]),
+    ("REVIVE_EVERY", 4, [P.test_revival_happens_every_fifth_step_only]),
+    ("rows_per_pass", rows_per_pass_floor, [P.test_every_row_once_per_pass_and_fractional_last_pass,
+                                            P.test_recipe_invariants]),
+    ("draw_uniform", draw_uniform_ignores_step, [P.test_donor_frequency_proportional_to_size]),
+    ("spherical_error", spherical_error_one_minus, [P.test_spherical_run_keeps_unit_centroids_and_error_definition]),
+    ("fp8_codes", fp8_codes_scale_before_shift, [P.test_fp8_search_is_the_argmin_over_codes,
+                                                 P.test_fp8_distances_within_the_quantisation_bound]),
 ]
 
 
-@pytest.mark.parametrize("name,mutant,pins", MUTATIONS, ids=[m[1].__name__ for m in MUTATIONS])
+@pytest.mark.parametrize("name,mutant,pins", MUTATIONS,
+                         ids=[getattr(m[1], "__name__", f"{m[0]}={m[1]}") for m in MUTATIONS])
 def test_planted_mistake_fails_a_pin(monkeypatch, name, mutant, pins):
     # the pins hold for the oracle as it stands
     for pin in pins:
