@@ -228,6 +228,20 @@ def fp8_codes_scale_before_shift(v, shift, scale):
     return O.e4m3_round(d32.astype(np.float64))
 
 
+def lloyd_half_step(xq, c0, iters, spherical=False, fp8=None):
+    """Lloyd's update with alpha = 0.5 instead of 1: each centroid only half-way to
+    its rows' mean after the first iteration."""
+    k = c0.shape[0]
+    N, S, c = np.zeros(k), np.zeros_like(c0), c0.copy()
+    history = []
+    for _ in range(iters):
+        labels, best, _ = O.assign(xq, O.search_copy_of_centroids(c))
+        history.append(float(best.mean()))
+        n_j, s_j = O.batch_stats(xq, labels, k)
+        N, S, c = O.ema_update(N, S, c, n_j, s_j, 0.5)
+    return c, history
+
+
 MUTATIONS = [
     ("ema_update", ema_without_decay, [P.test_constant_step_single_cluster_is_exponentially_weighted_mean]),
     ("ema_update", ema_weights_swapped, [P.test_full_batch_unit_step_is_one_lloyd_iteration,
@@ -270,6 +284,7 @@ MUTATIONS = [
     ("spherical_error", spherical_error_one_minus, [P.test_spherical_run_keeps_unit_centroids_and_error_definition]),
     ("fp8_codes", fp8_codes_scale_before_shift, [P.test_fp8_search_is_the_argmin_over_codes,
                                                  P.test_fp8_distances_within_the_quantisation_bound]),
+    ("lloyd", lloyd_half_step, [P.test_lloyd_iterations_match_a_hand_written_lloyd]),
 ]
 
 

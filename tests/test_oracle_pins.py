@@ -296,6 +296,35 @@ def test_lloyd_loss_does_not_increase():
     assert np.all(np.diff(h16) <= 1e-3 * h16[0])
 
 
+def test_lloyd_iterations_match_a_hand_written_lloyd():
+    """[Blog] "Still Lloyd's 1957 algorithm": assign every row to its nearest
+    centroid, then move each centroid to the mean of its rows (a centroid with no
+    rows stays). Written out with loops; the search uses the bf16 copy of the
+    centroids (fp64 -> fp32 -> bf16, by torch's cast), the means are fp64."""
+    g = np.random.default_rng(11)
+    x = O.search_copy_of_data(g.standard_normal((120, 3)).astype(np.float32))
+    c0 = np.vstack([x[:5], [[40.0, 40.0, 40.0]]])  # the last centroid never wins a row
+    c = c0.copy()
+    hist = []
+    for _ in range(3):
+        cb = torch.tensor(c, dtype=torch.float32).to(torch.bfloat16).to(torch.float64).numpy()
+        labels = []
+        for i in range(len(x)):
+            d = [sum((x[i, t] - cb[j, t]) ** 2 for t in range(3)) for j in range(len(c))]
+            labels.append(min(range(len(c)), key=lambda q: (d[q], q)))
+        hist.append(np.mean([sum((x[i, t] - cb[labels[i], t]) ** 2 for t in range(3)) for i in range(len(x))]))
+        new = c.copy()
+        for j in range(len(c)):
+            rows = [x[i] for i in range(len(x)) if labels[i] == j]
+            if rows:
+                new[j] = np.sum(rows, axis=0) / len(rows)
+        c = new
+    c_or, h_or = O.lloyd(x, c0, 3)
+    assert np.allclose(c_or, c, rtol=1e-13, atol=1e-13)
+    assert np.array_equal(c_or[5], c0[5])
+    assert np.allclose(h_or, hist, rtol=1e-12, atol=1e-12)
+
+
 def test_batch_stats_against_loops():
     g = np.random.default_rng(7)
     rows = g.standard_normal((200, 3))
