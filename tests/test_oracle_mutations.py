@@ -15,7 +15,7 @@ from tests import test_oracle_pins as P
 _orig = {name: getattr(O, name) for name in (
     "ema_update", "alpha_at", "squared_distances", "assign", "batch_stats", "f32_to_bf16", "revive",
     "split_sign", "philox4x64_10", "pass_order", "batch_size_law", "alpha0_law", "unit_rows", "e4m3_round",
-    "fp8_calibrate", "assign_dot", "round_batch", "EmeansOracle", "draw_uniform")}
+    "fp8_calibrate", "assign_dot", "round_batch", "EmeansOracle", "draw_uniform", "lloyd", "assign_fp8")}
 
 
 # ---------------------------------------------------------------- the mistakes
@@ -242,6 +242,28 @@ def lloyd_half_step(xq, c0, iters, spherical=False, fp8=None):
     return c, history
 
 
+def spherical_lloyd_not_rescaled(xq, c0, iters, spherical=False, fp8=None):
+    """Spherical Lloyd whose centroids are left at the rows' mean, not rescaled to
+    norm 1 after the update."""
+    if not spherical:
+        return _orig["lloyd"](xq, c0, iters, spherical, fp8)
+    k = c0.shape[0]
+    N, S, c = np.zeros(k), np.zeros_like(c0), O.unit_rows(c0)
+    history = []
+    for _ in range(iters):
+        labels, sim, _ = O.assign_dot(xq, O.search_copy_of_centroids(c))
+        history.append(float((2.0 - 2.0 * sim).mean()))
+        n_j, s_j = O.batch_stats(xq, labels, k)
+        N, S, c = O.ema_update(N, S, c, n_j, s_j, 1.0)
+    return c, history
+
+
+def assign_fp8_in_code_units(xq, c64, shift, scale):
+    """FP8 distances reported in code units (not divided by scale^2)."""
+    labels, best, second = _orig["assign_fp8"](xq, c64, shift, scale)
+    return labels, best * scale ** 2, second * scale ** 2
+
+
 MUTATIONS = [
     ("ema_update", ema_without_decay, [P.test_constant_step_single_cluster_is_exponentially_weighted_mean]),
     ("ema_update", ema_weights_swapped, [P.test_full_batch_unit_step_is_one_lloyd_iteration,
@@ -285,6 +307,8 @@ MUTATIONS = [
     ("fp8_codes", fp8_codes_scale_before_shift, [P.test_fp8_search_is_the_argmin_over_codes,
                                                  P.test_fp8_distances_within_the_quantisation_bound]),
     ("lloyd", lloyd_half_step, [P.test_lloyd_iterations_match_a_hand_written_lloyd]),
+    ("lloyd", spherical_lloyd_not_rescaled, [P.test_spherical_lloyd_step_is_the_normalised_mean]),
+    ("assign_fp8", assign_fp8_in_code_units, [P.test_fp8_distances_within_the_quantisation_bound]),
 ]
 
 
