@@ -180,12 +180,13 @@ int em_compute_recipe(int64_t n, int64_t k, double epochs, int law, int64_t batc
 int em_permutation(int64_t n, uint64_t seed, int stream, int64_t which, const int64_t* idx,
                    int64_t count, int64_t* out);
 
-/* The work split of the nearest-centroid search that em_train, em_step, em_assign
- * and em_mse use for `rows` rows and k centroids on a device with `sms` SMs (host
- * code, no device work). The search's units are 128-row tiles times groups of
- * 256-wide centroid tiles: the first *m_full row tiles are one unit each, over all
- * of k, and every later row tile is *split units (1, 2, 4 or 8). EM_E_INVAL for
- * rows, k or sms below 1 or a NULL output. */
+/* The work split of the nearest-centroid search that em_train, em_step, em_lloyd,
+ * em_assign and em_mse use for `rows` rows and k centroids on a device with `sms`
+ * SMs (host code, no device work; em_assign_noalloc may split less, to fit its
+ * fixed key region). The search's units are 128-row tiles times groups of 256-wide
+ * centroid tiles: the first *m_full row tiles are one unit each, over all of k,
+ * and every later row tile is *split units (1, 2, 4 or 8). EM_E_INVAL for rows, k
+ * or sms below 1 or a NULL output. */
 int em_search_schedule(int64_t rows, int64_t k, int sms, int* split, int* m_full);
 
 /* ---- model ---- */
