@@ -43,7 +43,10 @@ def _init(rank, world, port):
     dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
 
 
-def _dp_worker(rank, world, port, out_dir, k, epochs, batch):
+def _dp_worker(rank, world, port, out_dir, k, epochs, batch, plant=None):
+    """One rank of the protocol. `plant` breaks the exchange on purpose (the checks
+    must then fail): "no_reduce" skips the all-reduce, "sums_not_reduced" adds the
+    counts but keeps each rank's own sums."""
     _init(rank, world, port)
     try:
         xq = _data()
@@ -55,7 +58,12 @@ def _dp_worker(rank, world, port, out_dir, k, epochs, batch):
             part = np.array_split(np.arange(len(rows)), world)[rank]
             n_j, s_j = O.batch_stats(rows[part], labels[part], kk)
             buf = torch.from_numpy(np.concatenate([n_j[:, None], s_j], axis=1))
-            dist.all_reduce(buf)
+            if plant == "sums_not_reduced":
+                counts = buf[:, :1].contiguous()
+                dist.all_reduce(counts)
+                buf[:, :1] = counts
+            elif plant != "no_reduce":
+                dist.all_reduce(buf)
             return buf[:, 0].numpy().copy(), buf[:, 1:].numpy().copy()
 
         while not orc.done:
@@ -68,10 +76,7 @@ def _dp_worker(rank, world, port, out_dir, k, epochs, batch):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("k,epochs,batch", [(24, 2.0, 128), (40, 1.5, 96)])
-def test_data_parallel_step_matches_single_process(tmp_path, k, epochs, batch):
-    world = 2
-    mp.spawn(_dp_worker, args=(world, _free_port(), str(tmp_path), k, epochs, batch), nprocs=world, join=True)
+def _check_against_single_process(tmp_path, k, epochs, batch):
     c0, c1 = np.load(tmp_path / "c0.npy"), np.load(tmp_path / "c1.npy")
     N0, N1 = np.load(tmp_path / "N0.npy"), np.load(tmp_path / "N1.npy")
     # the ranks hold the same model, bit for bit
@@ -83,6 +88,22 @@ def test_data_parallel_step_matches_single_process(tmp_path, k, epochs, batch):
     np.testing.assert_allclose(c0, c_ref, rtol=1e-10, atol=1e-12)
     np.testing.assert_allclose(N0, ref.N, rtol=1e-12, atol=1e-12)
     assert int(np.load(tmp_path / "splits0.npy")[0]) == ref.n_splits
+
+
+@pytest.mark.parametrize("k,epochs,batch", [(24, 2.0, 128), (40, 1.5, 96)])
+def test_data_parallel_step_matches_single_process(tmp_path, k, epochs, batch):
+    world = 2
+    mp.spawn(_dp_worker, args=(world, _free_port(), str(tmp_path), k, epochs, batch), nprocs=world, join=True)
+    _check_against_single_process(tmp_path, k, epochs, batch)
+
+
+@pytest.mark.parametrize("plant", ["no_reduce", "sums_not_reduced"])
+def test_checks_catch_a_broken_exchange(tmp_path, plant):
+    world, k, epochs, batch = 2, 24, 2.0, 128
+    mp.spawn(_dp_worker, args=(world, _free_port(), str(tmp_path), k, epochs, batch, plant), nprocs=world,
+             join=True)
+    with pytest.raises(AssertionError):
+        _check_against_single_process(tmp_path, k, epochs, batch)
 
 
 def _agg_worker(rank, world, port, out_dir):
