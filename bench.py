@@ -190,6 +190,15 @@ def reduce_over_ranks(ms, rows, device, world):
     return float(t.item()), int(r.item())
 
 
+def step_rows(rec, n_train, s):
+    """Rows that step s of a run (0-based, over all passes) processes: a full batch,
+    or what is left of its pass for a pass's last step."""
+    B, full = rec["batch_size"], rec["steps_full_pass"]
+    p = s // full
+    rows_pass = rec["rows_last_pass"] if p == rec["passes"] - 1 else n_train
+    return min(B, rows_pass - (s - p * full) * B)
+
+
 def run_ours(args, rank, world):
     import torch
 
@@ -220,17 +229,12 @@ def run_ours(args, rank, world):
     def steps_loop(K):
         done = 0
         rows = 0
-        B = rec["batch_size"]
-        full = rec["steps_full_pass"]
         while done < K:
             left = total - state["in_run"]
             take = min(left, K - done)
             m.step(take)
             for s in range(state["in_run"], state["in_run"] + take):
-                p = s // full
-                in_pass = s - p * full
-                rows_pass = rec["rows_last_pass"] if p == rec["passes"] - 1 else w.n_train
-                rows += min(B, rows_pass - in_pass * B)
+                rows += step_rows(rec, w.n_train, s)
             state["in_run"] += take
             done += take
             if state["in_run"] >= total:
