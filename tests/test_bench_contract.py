@@ -7,12 +7,15 @@ import os
 import subprocess
 import sys
 
+import pytest
+
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
-def test_reference_arm_line_on_the_tiny_workload():
+@pytest.mark.parametrize("extra", [[], ["--spherical"]])
+def test_reference_arm_line_on_the_tiny_workload(extra):
     out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload", "tiny",
-                          "--steps", "2", "--warmup", "3", "--ref-seconds", "5"],
+                          "--steps", "2", "--warmup", "3", "--ref-seconds", "5"] + extra,
                          cwd=ROOT, capture_output=True, text=True, timeout=300)
     assert out.returncode == 0, out.stderr[-2000:]
     lines = [ln for ln in out.stdout.splitlines() if ln.strip()]
@@ -24,6 +27,7 @@ def test_reference_arm_line_on_the_tiny_workload():
     assert d["impl"] == "reference" and d["steps"] == 2 and d["warmup"] == 3 and d["n_gpus"] == 1
     assert d["value"] > 0 and d["higher_is_better"] is True and d["vs_baseline"] is None
     assert d["config"]["workload"].startswith("tiny")
+    assert d["config"]["method"] == ("spherical e-means" if extra else "e-means")
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["value"] == d["value"] and cb["cores"] >= 1 and cb["unit"] == d["unit"]
     assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
