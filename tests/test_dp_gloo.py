@@ -175,3 +175,32 @@ def test_rank_orders_are_the_oracles_bijections(em_lib):
         assert np.array_equal(lib, O.pass_order(n, 1234, which))
         assert np.array_equal(np.sort(lib), idx)
     assert not np.array_equal(em.permutation(n, 1234, 2, 1 << 32, idx), em.permutation(n, 1234, 2, 0, idx))
+
+
+def _fp8_worker(rank, world, port, out_dir):
+    """One rank of the FP8 converter fit: the minimum and maximum of each dimension
+    over this rank's first rows, combined over the ranks, then the converter of
+    that range."""
+    _init(rank, world, port)
+    try:
+        xq = _data(n=700 + 300 * rank, d=9, seed=20 + rank) * (1.0 + rank)
+        first = np.asarray(xq[:O.FP8_CALIBRATION_ROWS], dtype=np.float32)
+        lo, hi = torch.from_numpy(first.min(axis=0)), torch.from_numpy(first.max(axis=0))
+        dist.all_reduce(lo, op=dist.ReduceOp.MIN)
+        dist.all_reduce(hi, op=dist.ReduceOp.MAX)
+        shift, scale = O.fp8_calibrate(np.vstack([lo.numpy(), hi.numpy()]))
+        np.save(os.path.join(out_dir, f"fp8_{rank}.npy"), np.concatenate([shift.astype(np.float64), [scale]]))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_fp8_converter_over_ranks_is_the_fit_on_all_ranks_first_rows(tmp_path):
+    """The FP8 converter reading for several ranks: fitted on each rank's first
+    rows together (the ranks' minima and maxima combined)."""
+    world = 2
+    mp.spawn(_fp8_worker, args=(world, _free_port(), str(tmp_path)), nprocs=world, join=True)
+    r0, r1 = np.load(tmp_path / "fp8_0.npy"), np.load(tmp_path / "fp8_1.npy")
+    assert np.array_equal(r0, r1)
+    rows = [_data(n=700 + 300 * r, d=9, seed=20 + r) * (1.0 + r) for r in range(world)]
+    shift, scale = O.fp8_calibrate(np.vstack([x[:O.FP8_CALIBRATION_ROWS] for x in rows]))
+    assert np.array_equal(r0[:-1], shift.astype(np.float64)) and r0[-1] == scale
