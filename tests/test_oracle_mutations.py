@@ -264,6 +264,11 @@ def assign_fp8_in_code_units(xq, c64, shift, scale):
     return labels, best * scale ** 2, second * scale ** 2
 
 
+def starting_rows_first_k(n, k, seed):
+    """The first k training rows instead of a keyed random choice."""
+    return np.arange(k, dtype=np.int64)
+
+
 MUTATIONS = [
     ("ema_update", ema_without_decay, [P.test_constant_step_single_cluster_is_exponentially_weighted_mean]),
     ("ema_update", ema_weights_swapped, [P.test_full_batch_unit_step_is_one_lloyd_iteration,
@@ -309,6 +314,7 @@ MUTATIONS = [
     ("lloyd", lloyd_half_step, [P.test_lloyd_iterations_match_a_hand_written_lloyd]),
     ("lloyd", spherical_lloyd_not_rescaled, [P.test_spherical_lloyd_step_is_the_normalised_mean]),
     ("assign_fp8", assign_fp8_in_code_units, [P.test_fp8_distances_within_the_quantisation_bound]),
+    ("starting_rows", starting_rows_first_k, [P.test_starting_rows_are_distinct_training_rows]),
 ]
 
 

@@ -98,6 +98,11 @@ def test_pass_orders_differ_between_passes_and_seeds():
 def test_starting_rows_are_distinct_training_rows():
     rows = O.starting_rows(10000, 64, 1234)
     assert len(set(rows.tolist())) == 64 and rows.min() >= 0 and rows.max() < 10000
+    # a random choice over the whole training set, not a block of it: 64 uniform
+    # draws from [0, 10000) span more than half the range and have a mean near the
+    # middle (both fail with probability far below 1e-6)
+    assert rows.max() - rows.min() > 5000 and abs(rows.mean() - 5000) < 2000
+    assert not np.array_equal(rows, O.starting_rows(10000, 64, 99))
 
 
 def test_every_row_once_per_pass_and_fractional_last_pass():
