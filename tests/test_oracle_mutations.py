@@ -45,7 +45,20 @@ def alpha_to_zero(t, total_steps, alpha0):
 def alpha_linear(t, total_steps, alpha0):
     """A linear decay between the right endpoints instead of the cosine."""
     frac = 0.0 if total_steps <= 1 else t / (total_steps - 1)
+    return alpha0 - 0.9 * alpha0 * frac
+
+
+def alpha_power(t, total_steps, alpha0):
+    """A power-law decay between the right endpoints (not symmetric about the middle)."""
+    frac = 0.0 if total_steps <= 1 else t / (total_steps - 1)
     return alpha0 - 0.9 * alpha0 * frac ** 1.5
+
+
+def alpha_smoothstep(t, total_steps, alpha0):
+    """A smoothstep decay 1 - (3f^2 - 2f^3): right endpoints, decreasing and symmetric
+    about the middle like the cosine, but a different curve."""
+    frac = 0.0 if total_steps <= 1 else t / (total_steps - 1)
+    return 0.1 * alpha0 + 0.9 * alpha0 * (1.0 - (3.0 * frac ** 2 - 2.0 * frac ** 3))
 
 
 def distances_without_centroid_norm(xq, cq):
@@ -275,6 +288,8 @@ MUTATIONS = [
                                          P.test_constant_step_single_cluster_is_exponentially_weighted_mean]),
     ("alpha_at", alpha_to_zero, [P.test_cosine_schedule_endpoints_and_shape]),
     ("alpha_at", alpha_linear, [P.test_cosine_schedule_endpoints_and_shape]),
+    ("alpha_at", alpha_power, [P.test_cosine_schedule_endpoints_and_shape]),
+    ("alpha_at", alpha_smoothstep, [P.test_cosine_schedule_endpoints_and_shape]),
     ("squared_distances", distances_without_centroid_norm, [P.test_assign_matches_brute_force_definition]),
     ("squared_distances", distances_with_plus_cross_term, [P.test_assign_matches_brute_force_definition]),
     ("assign", assign_ties_to_highest, [P.test_assign_ties_go_to_lowest_index]),

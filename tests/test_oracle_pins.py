@@ -179,6 +179,14 @@ def test_cosine_schedule_endpoints_and_shape():
     # cosine: symmetric around the midpoint value (a0 + a0/10) / 2
     assert np.allclose(a + a[::-1], 1.1 * a0, rtol=0, atol=1e-12)
     assert O.alpha_at(0, 1, 0.3) == pytest.approx(0.3, rel=1e-15)
+    # interior points where the cosine has a closed form: with 13 steps, t = 3, 4, 6, 8
+    # are a quarter, a third, a half and two thirds of the way; cos(pi/4) = sqrt(2)/2,
+    # cos(pi/3) = 1/2, cos(pi/2) = 0, cos(2 pi/3) = -1/2.  A linear, power-law or other
+    # symmetric decay with the same endpoints misses at least one of them.
+    a_min = 0.1 * a0
+    span = a0 - a_min
+    for t, half_one_plus_cos in ((3, (1.0 + np.sqrt(2.0) / 2.0) / 2.0), (4, 0.75), (6, 0.5), (8, 0.25)):
+        assert O.alpha_at(t, 13, a0) == pytest.approx(a_min + span * half_one_plus_cos, rel=1e-14), t
 
 
 # ---------------------------------------------------------------- assignment
