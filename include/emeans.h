@@ -180,6 +180,22 @@ int em_compute_recipe(int64_t n, int64_t k, double epochs, int law, int64_t batc
 int em_permutation(int64_t n, uint64_t seed, int stream, int64_t which, const int64_t* idx,
                    int64_t count, int64_t* out);
 
+/* The rows that rank `rank` of `world` takes at each of the first `count` steps of a
+ * data-parallel run over n_local rows per rank (README "Several GPUs": the recipe
+ * is that of all ranks' rows, n_local x world, and each batch is split evenly; the
+ * pages' loop has every rank take positions [start / world, (start + B) / world)
+ * of its own fresh random order of its own rows each pass). Host code only: the
+ * same functions that plan em_step's batches and gathers. For step t: pass[t] is
+ * the pass, first[t] and rows[t] the positions [first, first + rows) of the
+ * rank's order that it takes, key[t] the key of that order (em_permutation with
+ * stream 2 and which = key[t]: the pass plus rank x 2^32). law, batch_override and
+ * alpha_override as in em_compute_recipe. EM_E_INVAL for bad sizes, a rank
+ * outside [0, world), count beyond the run's steps, NULL outputs, or a batch or
+ * last pass that does not divide by world (em_begin's check). */
+int em_dp_schedule(int64_t n_local, int64_t k, double epochs, int law, int64_t batch_override,
+                   double alpha_override, int64_t world, int64_t rank, int64_t count, int64_t* pass,
+                   int64_t* first, int64_t* rows, int64_t* key);
+
 /* The work split of the nearest-centroid search that em_train, em_step, em_lloyd,
  * em_assign and em_mse use for `rows` rows and k centroids on a device with `sms`
  * SMs (host code, no device work; em_assign_noalloc may split less, to fit its

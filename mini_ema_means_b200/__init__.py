@@ -123,6 +123,8 @@ _SIGS = {
     "em_compute_recipe": (ctypes.c_int, [_I64, _I64, ctypes.c_double, ctypes.c_int, _I64, ctypes.c_double,
                                          ctypes.POINTER(em_recipe_t)]),
     "em_permutation": (ctypes.c_int, [_I64, ctypes.c_uint64, ctypes.c_int, _I64, _P, _I64, _P]),
+    "em_dp_schedule": (ctypes.c_int, [_I64, _I64, ctypes.c_double, ctypes.c_int, _I64, ctypes.c_double, _I64, _I64,
+                                      _I64, _P, _P, _P, _P]),
     "em_search_schedule": (ctypes.c_int, [_I64, _I64, ctypes.c_int, ctypes.POINTER(ctypes.c_int),
                                           ctypes.POINTER(ctypes.c_int)]),
     "em_create": (_P, [_I64, _I64, ctypes.c_uint64]),
@@ -223,6 +225,17 @@ def permutation(n, seed, stream, which, idx):
     out = np.empty_like(idx)
     check(em_permutation(n, seed, stream, which, idx.ctypes.data, len(idx), out.ctypes.data), "em_permutation")
     return out
+
+
+def dp_schedule(n_local, k, epochs, world, rank, count, law=0, batch_size=0, alpha0=0.0):
+    """The rows rank `rank` of `world` takes at each of the first `count` steps of a
+    data-parallel run (host code): arrays pass, first, rows, key (int64)."""
+    import numpy as np
+
+    out = [np.empty(count, dtype=np.int64) for _ in range(4)]
+    check(em_dp_schedule(n_local, k, epochs, law, batch_size, alpha0, world, rank, count,
+                         *(o.ctypes.data for o in out)), "em_dp_schedule")
+    return tuple(out)
 
 
 def exchange_dp_id(group=None):

@@ -813,30 +813,64 @@ struct StepPlan {
     double alpha;
 };
 
-static StepPlan plan_at(const em_model* m, int64_t t, int64_t pass, int64_t pos) {
+// Step t of a run whose recipe is `rec` over n rows (all ranks' rows in a data-
+// parallel run), at row `pos` of pass `pass`. Host code only: em_dp_schedule runs
+// it without a model.
+static StepPlan plan_rows(const em_recipe_t& rec, int64_t n, bool auto_revive, int64_t t, int64_t pass,
+                          int64_t pos) {
     StepPlan p;
-    const int64_t rows_pass = (pass == m->rec.passes - 1) ? m->rec.rows_last_pass : m->n;
+    const int64_t rows_pass = (pass == rec.passes - 1) ? rec.rows_last_pass : n;
     p.t = t;
     p.pass = pass;
     p.pos = pos;
-    p.rows = std::min<int64_t>(m->rec.batch_size, rows_pass - pos);
-    p.last_pass = (pass == m->rec.passes - 1) ? 1 : 0;
-    p.alpha = alpha_at(t, m->rec.total_steps, m->rec.alpha0);
-    p.revive = (m->auto_revive && (t + 1) % kReviveEvery == 0) ? 1 : 0;
+    p.rows = std::min<int64_t>(rec.batch_size, rows_pass - pos);
+    p.last_pass = (pass == rec.passes - 1) ? 1 : 0;
+    p.alpha = alpha_at(t, rec.total_steps, rec.alpha0);
+    p.revive = (auto_revive && (t + 1) % kReviveEvery == 0) ? 1 : 0;
     return p;
+}
+
+// The step after p: the next batch of the pass, or the first of the next pass.
+static StepPlan plan_next(const em_recipe_t& rec, int64_t n, bool auto_revive, const StepPlan& p) {
+    const int64_t rows_pass = (p.pass == rec.passes - 1) ? rec.rows_last_pass : n;
+    int64_t pass = p.pass, pos = p.pos + p.rows;
+    if (pos >= rows_pass) {
+        pass += 1;
+        pos = 0;
+    }
+    return plan_rows(rec, n, auto_revive, p.t + 1, pass, pos);
+}
+
+static StepPlan plan_at(const em_model* m, int64_t t, int64_t pass, int64_t pos) {
+    return plan_rows(m->rec, m->n, m->auto_revive != 0, t, pass, pos);
 }
 
 static StepPlan plan_step(const em_model* m) { return plan_at(m, m->t, m->pass, m->pos); }
 
 // The step after p (same rules as advance_step).
 static StepPlan plan_after(const em_model* m, const StepPlan& p) {
-    const int64_t rows_pass = (p.pass == m->rec.passes - 1) ? m->rec.rows_last_pass : m->n;
-    int64_t pass = p.pass, pos = p.pos + p.rows;
-    if (pos >= rows_pass) {
-        pass += 1;
-        pos = 0;
-    }
-    return plan_at(m, p.t + 1, pass, pos);
+    return plan_next(m->rec, m->n, m->auto_revive != 0, p);
+}
+
+// A rank's share of step p's batch (README "Several GPUs": every rank walks its own
+// rows in its own per-pass order and takes an even share of each batch): positions
+// [pos / world, (pos + rows) / world) of its order, whose key is the pass plus
+// rank * 2^32 (rank 0: the single-GPU order).
+struct RankShare {
+    int64_t first, rows, key;
+};
+
+static RankShare rank_share(const StepPlan& p, int64_t world, int64_t rank) {
+    return RankShare{p.pos / world, p.rows / world, p.pass + (rank << 32)};
+}
+
+// README "Several GPUs": the batch and the rows of every pass divide by the ranks.
+static int check_dp_recipe(const em_recipe_t& rec, int64_t world) {
+    if (world > 1 && (rec.batch_size % world || rec.rows_last_pass % world))
+        return fail(EM_E_INVAL, "the batch (%lld rows) and the rows of every pass (last: %lld) must divide by "
+                                "the number of ranks (%lld)",
+                    (long long)rec.batch_size, (long long)rec.rows_last_pass, (long long)world);
+    return EM_OK;
 }
 
 // Whether step t gathers the rows of step t + 1 on the side stream.
@@ -850,16 +884,16 @@ static bool prefetches(const em_model* m, int64_t t) {
 // order).
 static int launch_gather(em_model* m, const StepPlan& p, cudaStream_t stream) {
     em_model::BatchSlot& b = m->slot[p.t & 1];
-    const int64_t rows = p.rows / m->dp_world;
-    const int64_t key = p.pass + ((int64_t)m->dp_rank << 32);
+    const RankShare sh = rank_share(p, m->dp_world, m->dp_rank);
+    const int64_t rows = sh.rows;
+    const int64_t key = sh.key;
     if (m->fp8) {
         const Fp8Out f8{b.X8.p, b.xn8.p, m->fp8_shift.p, m->fp8_scale, m->ld8, (int)m->d};
         launch_k(m->pdl, k_gather<true>, grid_for(rows, 128, m->sms), 128, 0, stream, 
-            m->X, m->n_local, m->ld, m->seed, key, p.pos / m->dp_world, (int)rows, 0, b.X.p, b.xn.p, b.ids.p, m->err.p,
-            f8);
+            m->X, m->n_local, m->ld, m->seed, key, sh.first, (int)rows, 0, b.X.p, b.xn.p, b.ids.p, m->err.p, f8);
     } else {
         launch_k(m->pdl, k_gather<false>, grid_for(rows, 128, m->sms), 128, 0, stream, 
-            m->X, m->n_local, m->ld, m->seed, key, p.pos / m->dp_world, (int)rows, 0, b.X.p, b.xn.p, b.ids.p, m->err.p,
+            m->X, m->n_local, m->ld, m->seed, key, sh.first, (int)rows, 0, b.X.p, b.xn.p, b.ids.p, m->err.p,
             Fp8Out{});
     }
     CK(cudaGetLastError());
@@ -891,7 +925,7 @@ static int drop_prefetch(em_model* m) {
 
 static void advance_step(em_model* m, const StepPlan& p) {
     const int64_t rows_pass = (m->pass == m->rec.passes - 1) ? m->rec.rows_last_pass : m->n;
-    m->last_rows = p.rows / m->dp_world;
+    m->last_rows = rank_share(p, m->dp_world, m->dp_rank).rows;
     m->last_alpha = p.alpha;
     m->rows_assigned += p.rows;
     m->t += 1;
@@ -903,7 +937,7 @@ static void advance_step(em_model* m, const StepPlan& p) {
 }
 
 static int launch_step(em_model* m, const StepPlan& p) {
-    const int64_t rows = p.rows / m->dp_world;  // this rank's share
+    const int64_t rows = rank_share(p, m->dp_world, m->dp_rank).rows;  // this rank's share
     const double rd = (double)rows, dd = (double)m->d, kd = (double)m->k;
     em_model::BatchSlot& b = m->slot[p.t & 1];
     int sp = span_begin(m, EM_PHASE_GATHER);
@@ -1202,6 +1236,30 @@ int em_permutation(int64_t n, uint64_t seed, int stream, int64_t which, const in
     return EM_OK;
 }
 
+int em_dp_schedule(int64_t n_local, int64_t k, double epochs, int law, int64_t batch_override,
+                   double alpha_override, int64_t world, int64_t rank, int64_t count, int64_t* pass, int64_t* first,
+                   int64_t* rows, int64_t* key) {
+    if (n_local < 1 || world < 1 || rank < 0 || rank >= world || count < 0)
+        return fail(EM_E_INVAL, "bad data-parallel schedule arguments");
+    if (count > 0 && (!pass || !first || !rows || !key)) return fail(EM_E_INVAL, "an output is NULL");
+    em_recipe_t rec;
+    CKR(compute_recipe(n_local * world, k, 0, epochs, law, batch_override, alpha_override, &rec));
+    if (rec.batch_size > rec.n) return fail(EM_E_INVAL, "batch size larger than n");
+    CKR(check_dp_recipe(rec, world));
+    if (count > rec.total_steps) return fail(EM_E_INVAL, "count is beyond the run's %lld steps",
+                                             (long long)rec.total_steps);
+    StepPlan p = plan_rows(rec, rec.n, false, 0, 0, 0);
+    for (int64_t t = 0; t < count; ++t) {
+        if (t) p = plan_next(rec, rec.n, false, p);
+        const RankShare sh = rank_share(p, world, rank);
+        pass[t] = p.pass;
+        first[t] = sh.first;
+        rows[t] = sh.rows;
+        key[t] = sh.key;
+    }
+    return EM_OK;
+}
+
 int em_search_schedule(int64_t rows, int64_t k, int sms, int* split, int* m_full) {
     if (rows < 1 || k < 1 || sms < 1 || !split || !m_full) return fail(EM_E_INVAL, "bad search schedule arguments");
     const Schedule sc = choose_schedule((rows + tc::BM - 1) / tc::BM, (k + tc::BN - 1) / tc::BN, sms);
@@ -1446,11 +1504,8 @@ int em_begin(em_model* m, const void* X, int64_t n, double epochs) {
     if (n_total >= (1ll << 31)) return fail(EM_E_INVAL, "the rows of all ranks must be below 2^31");
     CKR(compute_recipe(n_total, m->k, m->d, epochs, effective_law(m), m->opt_batch, m->opt_alpha0, &m->rec));
     if (m->rec.batch_size > n_total) return fail(EM_E_INVAL, "batch size larger than n");
-    if (W > 1) {  // README "Several GPUs": the batch and the rows of every pass divide by the ranks
-        if (m->rec.batch_size % W || m->rec.rows_last_pass % W)
-            return fail(EM_E_INVAL, "the batch (%lld rows) and the rows of every pass (last: %lld) must divide by "
-                                    "the number of ranks (%lld)",
-                        (long long)m->rec.batch_size, (long long)m->rec.rows_last_pass, (long long)W);
+    if (W > 1) {
+        CKR(check_dp_recipe(m->rec, W));
         if (m->revival == EM_REVIVE_RESAMPLE)
             return fail(EM_E_INVAL, "resampling draws rows of the whole batch; use it with one rank");
     }

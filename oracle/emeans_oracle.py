@@ -44,6 +44,13 @@ R13 FP8 search: the converter's shift is each dimension's midrange and its scale
     the largest power of two keeping the sample within 448, fitted on the first
     65,536 rows of the bf16 search copy; rows and centroids are encoded from their
     bf16 / fp32 values; the running sums stay those of the bf16 rows.
+R14 data parallelism ([README] "Several GPUs", the DistributedEmeans loop): each
+    of W ranks holds its own n_local rows; the recipe is that of n_local x W rows;
+    at the step covering positions [pos, pos + rows) of a pass, a rank takes the
+    positions [pos // W, (pos + rows) // W) of its own per-pass order of its own
+    rows, the order keyed by pass + rank x 2^32 (rank 0: the one-rank order); the
+    per-cluster counts and sums (and the batch error) are added over the ranks,
+    and every rank applies the same update; rank 0's starting rows are used.
 
 Random draws (starting rows, per-pass order, donor draws, resample rows) come
 from the counter-based generator Philox4x64-10 (Salmon, Moraes, Dror, Shaw,
@@ -293,6 +300,14 @@ def pass_order(n: int, seed: int, pass_index: int) -> np.ndarray:
     return permute(np.arange(n, dtype=np.uint64), n, seed, STREAM_PASS, pass_index)
 
 
+def dp_share(pos: int, rows: int, world: int):
+    """The positions [lo, hi) of a rank's own per-pass order that it takes when the
+    whole job's batch covers positions [pos, pos + rows) of the pass ([README]
+    "Several GPUs": with the batch summed over all GPUs, every rank takes an even
+    share; the pages' loop slices [start // world, (start + B) // world))."""
+    return pos // world, (pos + rows) // world
+
+
 def starting_rows(n: int, k: int, seed: int) -> np.ndarray:
     """k distinct training rows: the first k images of the start permutation."""
     return permute(np.arange(k, dtype=np.uint64), n, seed, STREAM_INIT, 0)
@@ -524,8 +539,13 @@ class EmeansOracle:
     """e-means in fp64 on the bf16 search copy of the data."""
 
     def __init__(self, d, k, seed=1234, revival="split", tau=None, closing_mean=True,
-                 law="auto", batch_size=None, alpha0=None, spherical=False, search="bf16"):
+                 law="auto", batch_size=None, alpha0=None, spherical=False, search="bf16",
+                 world=1, rank=0, all_reduce=None):
         self.d, self.k, self.seed = int(d), int(k), int(seed)
+        # data parallelism (R14): `all_reduce` adds a float64 vector over the ranks
+        self.world, self.rank, self.all_reduce = int(world), int(rank), all_reduce
+        if not 0 <= self.rank < self.world:
+            raise ValueError("rank outside [0, world)")
         self.spherical = bool(spherical)
         if search not in ("bf16", "fp8"):
             raise ValueError(search)
@@ -545,24 +565,38 @@ class EmeansOracle:
         self.n_splits = 0
 
     # begin: recipe, starting centroids, zero statistics
-    def begin(self, xq: np.ndarray, epochs: float, start_rows=None):
+    def begin(self, xq: np.ndarray, epochs: float, start_rows=None, start_centroids=None):
+        """Recipe, starting centroids, zero statistics. With several ranks (R14), xq is
+        this rank's rows and start_centroids rank 0's starting rows (ranks other
+        than 0 must pass them)."""
         n = xq.shape[0]
         if n < self.k:
             raise ValueError("need at least k rows")
         self.xq = xq
         self.n = n
-        self.r = recipe(n, self.k, epochs, self.law, self.batch_override, self.alpha_override)
+        W = self.world
+        self.r = recipe(n * W, self.k, epochs, self.law, self.batch_override, self.alpha_override)
+        if W > 1:
+            if self.r["batch_size"] % W or self.r["epoch_rows"][-1] % W:
+                raise ValueError("the batch and the rows of every pass must divide by the number of ranks")
+            if self.revival == "resample" or self.search == "fp8":
+                raise ValueError("several ranks: resampling and the FP8 search are not modelled")
         if self.search == "fp8":
             self.fp8 = fp8_calibrate(xq)
-        rows = starting_rows(n, self.k, self.seed) if start_rows is None else np.asarray(start_rows)
-        self.c = xq[rows].copy()
+        if start_centroids is not None:
+            self.c = np.array(start_centroids, dtype=np.float64)
+        else:
+            if self.rank != 0:
+                raise ValueError("ranks other than 0 start from rank 0's rows")
+            rows = starting_rows(n, self.k, self.seed) if start_rows is None else np.asarray(start_rows)
+            self.c = xq[rows].copy()
         if self.spherical:
             self.c = unit_rows(self.c)
         self.N = np.zeros(self.k)
         self.S = np.zeros((self.k, self.d))
         self.t = 0
         self.pass_index, self.pos = 0, 0
-        self.order = pass_order(n, self.seed, 0)
+        self.order = pass_order(n, self.seed, self.order_key(0))
         self.labels_last = np.full(n, -1, dtype=np.int64)
         self.close_sum = np.zeros((self.k, self.d))
         self.close_cnt = np.zeros(self.k)
@@ -574,10 +608,22 @@ class EmeansOracle:
     def done(self):
         return self.pass_index >= len(self.r["epoch_rows"])
 
+    def order_key(self, pass_index):
+        """Key of this rank's order in a pass (R14): the pass plus rank x 2^32."""
+        return pass_index + (self.rank << 32)
+
+    def batch_rows(self):
+        """Rows of the whole job's current batch: positions [pos, pos + rows) of the pass."""
+        return min(self.r["batch_size"], self.r["epoch_rows"][self.pass_index] - self.pos)
+
+    def batch_positions(self):
+        """This rank's positions of its own order in the current batch (R14; one rank:
+        the batch's own positions)."""
+        return dp_share(self.pos, self.batch_rows(), self.world)
+
     def next_batch_ids(self):
-        rows = self.r["epoch_rows"][self.pass_index]
-        b = self.r["batch_size"]
-        return self.order[self.pos:min(self.pos + b, rows)]
+        lo, hi = self.batch_positions()
+        return self.order[lo:hi]
 
     def step(self, forced_labels=None, auto_revive=True, stats=None):
         """One mini-batch: assign, per-cluster statistics, EMA, then revival if due.
@@ -596,6 +642,10 @@ class EmeansOracle:
             labels, best, second = assign(xb, search_copy_of_centroids(self.c))
         used = labels if forced_labels is None else np.asarray(forced_labels, dtype=np.int64)
         n_j, s_j = (batch_stats if stats is None else stats)(xb, used, self.k)
+        err = float(best.sum())
+        if self.world > 1:  # R14: the counts, sums and batch error added over the ranks
+            buf = self.all_reduce(np.concatenate([n_j, s_j.ravel(), [err]]))
+            n_j, s_j, err = buf[:self.k], buf[self.k:-1].reshape(self.k, self.d), float(buf[-1])
         alpha = alpha_at(self.t, self.r["total_steps"], self.r["alpha0"])
         self.N, self.S, self.c = ema_update(self.N, self.S, self.c, n_j, s_j, alpha)
         if self.spherical:
@@ -605,20 +655,20 @@ class EmeansOracle:
             self.labels_last[ids] = used
             self.close_sum += s_j
             self.close_cnt += n_j
-        self._pass_err += float(best.sum())
+        self._pass_err += err
         info = dict(t=self.t, ids=ids, labels=labels, best=best, second=second, alpha=alpha,
                     n_j=n_j, s_j=s_j, revived=None)
         if auto_revive:
             info["revived"] = self.maybe_revive(xb)
         self.t += 1
-        self.pos += len(ids)
+        self.pos += self.batch_rows()
         if self.pos >= self.r["epoch_rows"][self.pass_index]:
             self.obj.append(self._pass_err / self.r["epoch_rows"][self.pass_index])
             self._pass_err = 0.0
             self.pass_index += 1
             self.pos = 0
             if not self.done:
-                self.order = pass_order(self.n, self.seed, self.pass_index)
+                self.order = pass_order(self.n, self.seed, self.order_key(self.pass_index))
         return info
 
     def maybe_revive(self, batch_rows, t=None):

@@ -182,3 +182,27 @@ def teacher_forced_run(m, orc, x_dev, xq, epochs, revival, check_every=1, max_st
             assert st["last_dead"] == (0 if res is None else len(res[0]))
     book.finish()
     return dict(worst=worst, mismatches=book.mismatch, rows=book.rows, revived=revivals)
+
+
+def threaded_assign(assign, workers=None, rows_per_task=2048):
+    """The oracle's search, split into row blocks that run on a thread pool.
+
+    Each row's label and two best distances depend on that row alone, so the
+    result is the oracle's, row for row; numpy releases the GIL inside the matmul
+    and the element-wise passes, so the blocks run in parallel. Used only to make
+    whole oracle runs at full size affordable inside a test."""
+    import os
+    from concurrent.futures import ThreadPoolExecutor
+
+    workers = workers or max(1, min(16, os.cpu_count() or 1))
+
+    def run(xq, cq, chunk=4096):
+        n = xq.shape[0]
+        if n <= rows_per_task:
+            return assign(xq, cq, chunk)
+        starts = range(0, n, rows_per_task)
+        with ThreadPoolExecutor(workers) as ex:
+            parts = list(ex.map(lambda s: assign(xq[s:s + rows_per_task], cq, chunk), starts))
+        return tuple(np.concatenate([p[i] for p in parts]) for i in range(3))
+
+    return run

@@ -1,12 +1,19 @@
-"""Data-parallel e-means on two CPU ranks (gloo), at the level of the oracle.
+"""Data-parallel e-means on CPU ranks (gloo), at the level of the oracle.
 
-The method shards by batch rows: every rank assigns its share of each mini-batch,
-computes the per-cluster counts and sums of its rows, the ranks add them with one
-all-reduce of k (d + 1) values, and every rank applies the same EMA update and the
-same revival check (the revival draws are keyed by seed, step and cluster, so no
-further exchange is needed). These tests check that protocol against the
-single-process oracle run, that the ranks stay bit-identical, and the bench's
-aggregation of timings and row counts over ranks.
+The pages' DistributedEmeans loop ([README] "Several GPUs"): every rank holds its
+own rows and walks them in its own fresh order each pass; the recipe is that of
+all ranks' rows; at each step every rank takes an even share of the batch
+(positions [pos // W, (pos + B) // W) of its order), computes the per-cluster
+counts and sums of its share, the ranks add them (with the batch error) in one
+all-reduce, and every rank applies the same EMA update and the same revival check
+(its draws are keyed by seed, step and cluster, so no further exchange is
+needed). These tests check:
+* a run on 2 and 3 gloo ranks against one process that replays every rank's share
+  of every batch with no collective (and planted broken exchanges fail that);
+* the library's host plan of each rank's batches (em_dp_schedule) against the
+  oracle's protocol, step by step;
+* the bench's aggregation of timings and row counts over ranks, the communicator
+  id exchange and the FP8 converter over ranks.
 """
 
 import datetime
@@ -43,67 +50,139 @@ def _init(rank, world, port):
     dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
 
 
+def _rank_rows(rank, n_local=600, d=12, comps=10):
+    """Rank `rank`'s own rows: every rank holds a different share of one mixture."""
+    return _data(n=n_local, d=d, comps=comps, seed=3 + 100 * rank)
+
+
 def _dp_worker(rank, world, port, out_dir, k, epochs, batch, plant=None):
-    """One rank of the protocol. `plant` breaks the exchange on purpose (the checks
-    must then fail): "no_reduce" skips the all-reduce, "sums_not_reduced" adds the
-    counts but keeps each rank's own sums."""
+    """One rank of the pages' data-parallel loop ([README] "Several GPUs"), as the
+    oracle runs it: own rows, own per-pass order, an even share of each batch, one
+    all-reduce of (n_j, s_j, batch error) per step, rank 0's starting rows.
+    `plant` breaks the protocol on purpose (the checks must then fail):
+    "no_reduce" skips the all-reduce, "sums_not_reduced" adds the counts but keeps
+    each rank's own sums, "rank_blind_order" gives every rank rank 0's order key."""
     _init(rank, world, port)
     try:
-        xq = _data()
-        orc = O.EmeansOracle(xq.shape[1], k, seed=5, batch_size=batch)
-        orc.begin(xq, epochs)
+        xq = _rank_rows(rank)
 
-        def shard_stats(rows, labels, kk):
-            # this rank's share of the batch, then one all-reduce of (n_j, s_j)
-            part = np.array_split(np.arange(len(rows)), world)[rank]
-            n_j, s_j = O.batch_stats(rows[part], labels[part], kk)
-            buf = torch.from_numpy(np.concatenate([n_j[:, None], s_j], axis=1))
+        def all_reduce(v):
+            buf = torch.from_numpy(np.array(v, dtype=np.float64))
             if plant == "sums_not_reduced":
-                counts = buf[:, :1].contiguous()
-                dist.all_reduce(counts)
-                buf[:, :1] = counts
+                head = buf[:k].contiguous()
+                dist.all_reduce(head)
+                buf[:k] = head
             elif plant != "no_reduce":
                 dist.all_reduce(buf)
-            return buf[:, 0].numpy().copy(), buf[:, 1:].numpy().copy()
+            return buf.numpy().copy()
 
+        orc = O.EmeansOracle(xq.shape[1], k, seed=5, batch_size=batch, world=world, rank=rank,
+                             all_reduce=all_reduce)
+        if plant == "rank_blind_order":
+            orc.order_key = lambda p: p
+        c0 = torch.from_numpy(xq[O.starting_rows(len(xq), k, 5)].copy())
+        dist.broadcast(c0, src=0)  # rank 0's starting rows
+        orc.begin(xq, epochs, start_centroids=c0.numpy())
         while not orc.done:
-            orc.step(stats=shard_stats)
+            orc.step()
         c = orc.finalize()
         np.save(os.path.join(out_dir, f"c{rank}.npy"), c)
         np.save(os.path.join(out_dir, f"N{rank}.npy"), orc.N)
+        np.save(os.path.join(out_dir, f"obj{rank}.npy"), np.array(orc.obj))
         np.save(os.path.join(out_dir, f"splits{rank}.npy"), np.array([orc.n_splits]))
     finally:
         dist.destroy_process_group()
 
 
-def _check_against_single_process(tmp_path, k, epochs, batch):
-    c0, c1 = np.load(tmp_path / "c0.npy"), np.load(tmp_path / "c1.npy")
-    N0, N1 = np.load(tmp_path / "N0.npy"), np.load(tmp_path / "N1.npy")
+def _replay_all_ranks(world, k, epochs, batch):
+    """One process replays every rank's share of every batch: rank r's rows are
+    positions [pos // W, (pos + B) // W) of the order keyed by pass + r x 2^32 of
+    its own rows; the batch's labels, counts and sums are computed over the union
+    of the ranks' shares, with no collective at all."""
+    xs = [_rank_rows(r) for r in range(world)]
+    err = {}
+
+    orc = O.EmeansOracle(xs[0].shape[1], k, seed=5, batch_size=batch, world=world, rank=0,
+                         all_reduce=lambda v: np.concatenate([v[:-1], [err["total"]]]))
+
+    def union_stats(_rows, _labels, kk):
+        lo, hi = orc.batch_positions()
+        parts = [x[O.pass_order(len(x), 5, orc.pass_index + (r << 32))[lo:hi]] for r, x in enumerate(xs)]
+        rows = np.concatenate(parts)
+        labels, best, _ = O.assign(rows, O.search_copy_of_centroids(orc.c))
+        err["total"] = float(best.sum())
+        return O.batch_stats(rows, labels, kk)
+
+    orc.begin(xs[0], epochs)
+    while not orc.done:
+        orc.step(stats=union_stats)
+    return orc.finalize(), orc
+
+
+def _check_against_single_process(tmp_path, world, k, epochs, batch):
+    c = [np.load(tmp_path / f"c{r}.npy") for r in range(world)]
+    N = [np.load(tmp_path / f"N{r}.npy") for r in range(world)]
     # the ranks hold the same model, bit for bit
-    assert np.array_equal(c0, c1) and np.array_equal(N0, N1)
-    # and it is the single-process run up to the order of the fp64 sums
-    xq = _data()
-    ref = O.EmeansOracle(xq.shape[1], k, seed=5, batch_size=batch)
-    c_ref, _ = ref.train(xq, epochs)
-    np.testing.assert_allclose(c0, c_ref, rtol=1e-10, atol=1e-12)
-    np.testing.assert_allclose(N0, ref.N, rtol=1e-12, atol=1e-12)
+    assert all(np.array_equal(c[0], x) for x in c) and all(np.array_equal(N[0], x) for x in N)
+    # and it is the one-process replay of every rank's rows, up to the order of the fp64 sums
+    c_ref, ref = _replay_all_ranks(world, k, epochs, batch)
+    np.testing.assert_allclose(c[0], c_ref, rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(N[0], ref.N, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(np.load(tmp_path / "obj0.npy"), ref.obj, rtol=1e-12)
     assert int(np.load(tmp_path / "splits0.npy")[0]) == ref.n_splits
 
 
-@pytest.mark.parametrize("k,epochs,batch", [(24, 2.0, 128), (40, 1.5, 96)])
-def test_data_parallel_step_matches_single_process(tmp_path, k, epochs, batch):
-    world = 2
+@pytest.mark.parametrize("world,k,epochs,batch", [(2, 24, 2.0, 128), (2, 40, 1.5, 96), (3, 16, 2.5, 96)])
+def test_data_parallel_run_matches_one_process_replay(tmp_path, world, k, epochs, batch):
     mp.spawn(_dp_worker, args=(world, _free_port(), str(tmp_path), k, epochs, batch), nprocs=world, join=True)
-    _check_against_single_process(tmp_path, k, epochs, batch)
+    _check_against_single_process(tmp_path, world, k, epochs, batch)
 
 
-@pytest.mark.parametrize("plant", ["no_reduce", "sums_not_reduced"])
+@pytest.mark.parametrize("plant", ["no_reduce", "sums_not_reduced", "rank_blind_order"])
 def test_checks_catch_a_broken_exchange(tmp_path, plant):
     world, k, epochs, batch = 2, 24, 2.0, 128
     mp.spawn(_dp_worker, args=(world, _free_port(), str(tmp_path), k, epochs, batch, plant), nprocs=world,
              join=True)
     with pytest.raises(AssertionError):
-        _check_against_single_process(tmp_path, k, epochs, batch)
+        _check_against_single_process(tmp_path, world, k, epochs, batch)
+
+
+@pytest.mark.parametrize("n_local,world,k,epochs,batch", [
+    (600, 2, 24, 2.0, 128), (600, 2, 40, 1.5, 96), (600, 3, 16, 2.5, 96), (4096, 4, 64, 3.0, 0),
+    (1000, 8, 10, 1.25, 64)])
+def test_library_rank_schedule_is_the_oracles(em_lib, n_local, world, k, epochs, batch):
+    """The library's host plan of a rank's batches (em_dp_schedule: the code em_step
+    and the gather use) against the oracle's protocol, step by step: the pass, the
+    positions of the rank's own order and that order's key."""
+    em = em_lib
+    for rank in range(world):
+        orc = O.EmeansOracle(1, k, seed=5, batch_size=batch or None, law="throughput", world=world, rank=rank,
+                             all_reduce=lambda v: v)
+        xq = O.search_copy_of_data(np.random.default_rng(rank).standard_normal((n_local, 1)).astype(np.float32))
+        orc.begin(xq, epochs, start_centroids=np.zeros((k, 1)))
+        want = []
+        while not orc.done:
+            lo, hi = orc.batch_positions()
+            want.append((orc.pass_index, lo, hi - lo, orc.order_key(orc.pass_index)))
+            orc.step(auto_revive=False)
+        got = em.dp_schedule(n_local, k, epochs, world, rank, len(want), law=0, batch_size=batch)
+        assert [tuple(int(a[t]) for a in got) for t in range(len(want))] == want
+        # each pass, the rank's positions cover its own rows exactly once (a fractional
+        # last pass: its first rows)
+        for p in set(w[0] for w in want):
+            spans = sorted((w[1], w[1] + w[2]) for w in want if w[0] == p)
+            assert spans[0][0] == 0 and all(a[1] == b[0] for a, b in zip(spans, spans[1:]))
+            assert spans[-1][1] == (n_local if p < orc.r["epoch_rows"].__len__() - 1 else
+                                    orc.r["epoch_rows"][-1] // world)
+
+
+def test_library_rejects_a_batch_that_does_not_divide(em_lib):
+    em = em_lib
+    with pytest.raises(em.EmeansError) as e:
+        em.dp_schedule(600, 24, 2.0, 3, 0, 1, batch_size=128)
+    assert e.value.code == em.EM_E_INVAL
+    with pytest.raises(em.EmeansError):
+        em.dp_schedule(600, 24, 2.0, 2, 2, 1, batch_size=128)  # rank outside [0, world)
 
 
 def _agg_worker(rank, world, port, out_dir):
