@@ -579,8 +579,8 @@ def run_ablation(args):
 L2_BYTES = 126e6  # the B200's L2 (126 MB)
 
 # DRAM bytes per assignment launch of the bench's batch, from an ncu capture of the
-# current kernel (profiles/k_assign_tc_emb768_262144rows.md: 262,144 rows, scaled
-# to one 65,536-row batch with the centroid operand counted once).
+# current kernel (262,144 rows, scaled to one 65,536-row batch with the centroid
+# operand counted once).
 ASSIGN_TRAFFIC = {"emb768": 109.6e6}
 
 

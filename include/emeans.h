@@ -164,6 +164,22 @@ typedef struct em_profile_t {
 /* Message of the last failing call on this thread ("" if none). Never NULL. */
 const char* em_last_error(void);
 
+/* EM_E_* code of the last failing call on this thread (0 if none): what a call
+ * that returns a pointer (em_create: NULL) failed with. */
+int em_last_error_code(void);
+
+/* Allocation-failure injection, for testing the out-of-memory paths without
+ * running out of memory (host code, no device work).
+ * After em_fail_allocation(nth), nth >= 1, the nth device allocation the library
+ * attempts (in any thread, counting from 1) fails as a failed cudaMalloc does,
+ * without calling it: the call that made it returns EM_E_NOMEM (em_create:
+ * NULL). The allocations after it run normally. nth <= 0 switches injection off.
+ * Returns the number of device allocations the library attempted since the
+ * previous em_fail_allocation call, so a test can count a sequence of calls'
+ * allocations and then fail each in turn. A model whose call failed this way can
+ * be destroyed, or used again (em_begin / em_train re-acquire what they need). */
+int64_t em_fail_allocation(int64_t nth);
+
 /* Number of CUDA devices visible to the library (0 without a GPU). Host-only. */
 int em_device_count(void);
 

@@ -120,6 +120,8 @@ _I64 = ctypes.c_int64
 _SIGS = {
     "em_last_error": (ctypes.c_char_p, []),
     "em_device_count": (ctypes.c_int, []),
+    "em_last_error_code": (ctypes.c_int, []),
+    "em_fail_allocation": (_I64, [_I64]),
     "em_compute_recipe": (ctypes.c_int, [_I64, _I64, ctypes.c_double, ctypes.c_int, _I64, ctypes.c_double,
                                          ctypes.POINTER(em_recipe_t)]),
     "em_permutation": (ctypes.c_int, [_I64, ctypes.c_uint64, ctypes.c_int, _I64, _P, _I64, _P]),
@@ -227,6 +229,13 @@ def permutation(n, seed, stream, which, idx):
     return out
 
 
+def fail_allocation(nth: int) -> int:
+    """Makes the library's nth device allocation from now on fail as a failed
+    cudaMalloc does (nth <= 0: off); returns the allocations attempted since the
+    previous call (host code)."""
+    return int(em_fail_allocation(int(nth)))
+
+
 def dp_schedule(n_local, k, epochs, world, rank, count, law=0, batch_size=0, alpha0=0.0):
     """The rows rank `rank` of `world` takes at each of the first `count` steps of a
     data-parallel run (host code): arrays pass, first, rows, key (int64)."""
@@ -256,7 +265,7 @@ class Model:
     def __init__(self, d: int, k: int, seed: int = 1234, **options):
         h = em_create(int(d), int(k), int(seed))
         if not h:
-            raise EmeansError(EM_E_NODEVICE if em_device_count() == 0 else EM_E_INVAL, "em_create")
+            raise EmeansError(em_last_error_code() or EM_E_INVAL, "em_create")
         self.h = h
         self.d, self.k, self.seed = int(d), int(k), int(seed)
         for name, value in options.items():

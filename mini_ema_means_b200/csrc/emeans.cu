@@ -33,6 +33,7 @@
 #include <cstdio>
 #include <cstring>
 #include <dlfcn.h>
+#include <atomic>
 #include <mutex>
 #include <utility>
 #include <vector>
@@ -51,12 +52,14 @@ using namespace em;
 // ------------------------------------------------------------------ errors
 
 static thread_local char g_err[1024] = "";
+static thread_local int g_err_code = 0;
 
 static int fail(int code, const char* fmt, ...) {
     va_list ap;
     va_start(ap, fmt);
     vsnprintf(g_err, sizeof(g_err), fmt, ap);
     va_end(ap);
+    g_err_code = code;
     return code;
 }
 
@@ -255,6 +258,21 @@ static int make_tmap8(CUtensorMap* tm, const void* base, int64_t rows, int d, in
 
 // ------------------------------------------------------------------ model
 
+// Allocation-failure injection (em_fail_allocation): the countdown to the device
+// allocation that fails, and the number of allocations attempted.
+static std::atomic<int64_t> g_alloc_fail_at{0};
+static std::atomic<int64_t> g_alloc_attempts{0};
+
+// Whether this allocation attempt is the one em_fail_allocation asked to fail.
+static bool injected_alloc_failure() {
+    g_alloc_attempts.fetch_add(1, std::memory_order_relaxed);
+    int64_t left = g_alloc_fail_at.load(std::memory_order_relaxed);
+    while (left > 0) {
+        if (g_alloc_fail_at.compare_exchange_weak(left, left - 1, std::memory_order_relaxed)) return left == 1;
+    }
+    return false;
+}
+
 template <class T>
 struct DBuf {
     T* p = nullptr;
@@ -264,6 +282,9 @@ struct DBuf {
         if (p) cudaFree(p);
         p = nullptr;
         cap = 0;
+        if (injected_alloc_failure())
+            return fail(EM_E_NOMEM, "cudaMalloc of %zu bytes failed (injected by em_fail_allocation)",
+                        count * sizeof(T));
         if (cudaMalloc(&p, std::max<size_t>(count, 1) * sizeof(T)) != cudaSuccess) {
             cudaGetLastError();
             p = nullptr;
@@ -1175,6 +1196,7 @@ static int prepare_fp8(em_model* m, const __nv_bfloat16* X, int64_t n) {
     if (!m->fp8) return EM_OK;
     if (m->spherical) return fail(EM_E_INVAL, "spherical e-means takes the bf16 search only");
     if (m->assign_kernel != 0) return fail(EM_E_INVAL, "the FP8 search runs on the tensor-core kernel only");
+    m->fp8_ready = false;  // until the operand buffers and the new converter are in place
     CKR(m->cq8.ensure((size_t)m->k * m->ld8));
     CKR(m->cn8.ensure(m->k));
     CKR(make_tmap8(&m->tm_cq8, m->cq8.p, m->k, (int)m->d, m->ld8, tc::BN));
@@ -1207,6 +1229,14 @@ static int start_centroids(em_model* m) {
 extern "C" {
 
 const char* em_last_error(void) { return g_err; }
+
+int em_last_error_code(void) { return g_err_code; }
+
+int64_t em_fail_allocation(int64_t nth) {
+    const int64_t attempts = g_alloc_attempts.exchange(0);
+    g_alloc_fail_at.store(nth > 0 ? nth : 0);
+    return attempts;
+}
 
 int em_device_count(void) {
     int n = 0;
@@ -2115,10 +2145,11 @@ extern "C" int em_assign_noalloc(const void* X, int64_t n, int64_t d, const floa
     const int64_t m_tiles = (n + tc::BM - 1) / tc::BM;
     const int64_t n_tiles = (k + tc::BN - 1) / tc::BN;
     const int nkc = (int)((d + kc - 1) / kc);
-    // the key region holds two keys for EM_NOALLOC_MAX_ROWS rows: split * kKeySets * n
-    // rows at most
+    // the key region holds 2 keys per key set for each of EM_NOALLOC_MAX_ROWS rows, and
+    // the search writes 2 keys per key set for each of its n rows in each of its split
+    // centroid-tile groups: split * n <= EM_NOALLOC_MAX_ROWS
     const Schedule sc = choose_schedule(m_tiles, n_tiles, sms,
-                                        (int)std::max<int64_t>(1, EM_NOALLOC_MAX_ROWS / (tc::kKeySets * n)));
+                                        (int)std::max<int64_t>(1, EM_NOALLOC_MAX_ROWS / n));
     const bool top2 = d >= 256;
     const int grid = (int)std::min<int64_t>(sc.m_full + (m_tiles - sc.m_full) * sc.split, sms);
     const long long wait_cycles = (long long)(2000.0 * (double)clock_khz);
