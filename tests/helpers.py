@@ -10,8 +10,8 @@ Tolerances (stated once, used by every parity test):
   search compares E4M3 codes: its tensor cores accumulate the code products in
   fp32 with some loss (the largest flip measured on this B200: a gap of 1.2e-4 of
   sum|x'_i c'_i|), and it settles no near tie exactly, so a row may hold another
-  label whose code distance is within FP8_GAP_REL x sum|x'_i c'_i| of the best,
-  with no limit on their number;
+  label whose code distance is within FP8_GAP_REL x sum|x'_i c'_i| of the best;
+  such flips may number at most max(1, 1e-4 x rows), as for the bf16 search;
 * centroids: relative L2 error per centroid <= 1e-3;
 * MSE: relative error <= 1e-3 (0.1 %).
 """
@@ -79,9 +79,14 @@ class LabelBook:
         return accepted, best * dscale
 
     def finish(self):
-        if self.fp8:
-            return  # every mismatch was checked against the FP8 accumulation bound
         allowed = max(1, int(LABEL_MISMATCH_FRACTION * self.rows))
+        if self.fp8:
+            # every mismatch was checked against the FP8 accumulation bound above; their
+            # number is held to the same budget as the bf16 search's (none was measured
+            # on a B200 in any FP8 test)
+            print(f"[labels] FP8 search: {self.mismatch} near-tie flips in {self.rows} rows")
+            assert self.mismatch <= allowed, f"{self.mismatch} FP8 near-tie flips in {self.rows} rows (max {allowed})"
+            return
         assert self.mismatch <= allowed, f"{self.mismatch} near-tie label flips in {self.rows} rows (max {allowed})"
 
 

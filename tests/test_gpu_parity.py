@@ -71,6 +71,13 @@ def test_tiny_teacher_forced_every_step(em, revival):
     (3333, 100, 77, 1.0, 1000, "none"),
     (3000, 2, 20, 2.0, None, "split"),    # d <= 2: the default threshold turns revival off
     (4000, 12, 50, 2.0, None, "split"),   # d <= 16: the default batch law is the quality law
+    # the streamed sums' row geometries: 32 lanes of one vector (d = 200), four
+    # vectors per lane (d = 1000), two column slices (d = 1100), and many more rows
+    # than one range per warp holds (8,192-row batches cut into 64-row ranges)
+    (1200, 200, 90, 1.5, 256, "split"),
+    (1100, 1000, 40, 1.0, 256, "split"),
+    (1000, 1100, 33, 1.0, 200, "none"),
+    (60000, 24, 700, 1.0, 8192, "split"),
 ])
 def test_hand_shapes_teacher_forced(em, n, d, k, epochs, batch, revival):
     x = synth.hand_shape(n, d, max(2, k // 2), seed=n + d)
