@@ -753,7 +753,7 @@ static int launch_reduce(em_model* m, const __nv_bfloat16* src, int64_t rows, in
     const int64_t max_items = m->k + (rows + m->R - 1) / m->R;
     const int nslices = (m->nv + 31) / 32;
     const int seg_blocks = (int)((max_items * nslices * 32 + 255) / 256);
-    launch_k(m->pdl, k_segsum, seg_blocks, 256, 0, m->stream, src, m->perm.p, m->items.p, m->poff.p, nslices, m->nv, st, sp,
+    launch_k(m->pdl, k_segsum, seg_blocks, 256, 8 * kSegsumDepth * 32 * 16, m->stream, src, m->perm.p, m->items.p, m->poff.p, nslices, m->nv, st, sp,
                                                 m->part.p);
     launch_k(m->pdl, k_clusters, grid_for(m->k * 32, EM_CLUSTERS_BLOCK, m->sms, 16), EM_CLUSTERS_BLOCK, 0, m->stream, 
         m->off.p, m->poff.p, m->cnt.p, m->R, nslices,

@@ -448,45 +448,66 @@ __device__ __forceinline__ SliceGeom slice_geom(int slice, int nv) {
 #ifndef EM_CHUNK_ROWS
 #define EM_CHUNK_ROWS 64
 #endif
-#ifndef EM_SEGSUM_RIF
-#define EM_SEGSUM_RIF 4
-#endif
 constexpr int kChunkRows = EM_CHUNK_ROWS;
-constexpr int kSegsumRif = EM_SEGSUM_RIF;
 
-// Sum over rows perm[s0..s1) of this lane's vector, fp64, four rows in flight per
-// lane (each row id is a broadcast load that the first row group brings into L1;
-// preloading the chunk's ids and handing them out by shuffles measured slower).
-// The warp's row groups are folded together at the end with a fixed butterfly, so
-// lanes l < lpr hold the slice totals of vector vbase + l.
-template <int RIF = 4>
-__device__ __forceinline__ void sum_rows(double acc[8], const __nv_bfloat16* __restrict__ src, int ld,
-                                         const int32_t* __restrict__ perm, int s0, int s1, const SliceGeom& g,
-                                         int lane) {
+// Row groups of a work item in flight per warp in k_segsum (a group is the `rpi`
+// rows a warp covers at once), staged through a ring in shared memory.
+constexpr int kSegsumDepth = 12;
+static_assert(kChunkRows <= 64, "an item's row ids are preloaded two per lane");
+
+__device__ __forceinline__ void seg_cp_async16(uint32_t dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void seg_cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void seg_cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// sum_rows with the rows staged through shared memory: the item's row ids are
+// loaded at once (two per lane, coalesced) and handed out by shuffles, and every
+// lane copies its own 16-byte vector of each row with cp.async, kSegsumDepth row
+// groups ahead of the adds. Each lane reads back only the vectors it copied
+// itself, so the lanes need no barrier. The sums are the same fp64 sums as
+// sum_rows (exact, so the order of the rows does not matter).
+__device__ __forceinline__ void sum_rows_staged(double acc[8], const __nv_bfloat16* __restrict__ src, int ld,
+                                                const int32_t* __restrict__ perm, int s0, int s1,
+                                                const SliceGeom& g, int lane, uint4* ring) {
+    constexpr int D = kSegsumDepth;
 #pragma unroll
     for (int t = 0; t < 8; ++t) acc[t] = 0.0;
+    const int n = s1 - s0;
     const int sub = lane / g.lpr, vi = lane % g.lpr;
     const bool vec_ok = vi < g.nvs;
     const int v = g.vbase + vi;
-    for (int s = s0; s < s1; s += RIF * g.rpi) {
-        uint4 u[RIF];
-        bool have[RIF];
+    const int id0 = lane < n ? perm[s0 + lane] : 0;
+    const int id1 = 32 + lane < n ? perm[s0 + 32 + lane] : 0;
+    const int ngroups = (n + g.rpi - 1) / g.rpi;
+    const uint32_t ring_s = (uint32_t)__cvta_generic_to_shared(ring);
+    auto issue = [&](int grp) {
+        const int p = grp * g.rpi + sub;  // row of the item (only p < 64 is ever used)
+        const int a = __shfl_sync(0xFFFFFFFFu, id0, p & 31);
+        const int b = __shfl_sync(0xFFFFFFFFu, id1, p & 31);
+        if (grp < ngroups && vec_ok && p < n)
+            seg_cp_async16(ring_s + (uint32_t)(((grp % D) * 32 + lane) * 16),
+                           src + (int64_t)(p < 32 ? a : b) * ld + 8 * v);
+        seg_cp_async_commit();  // (an empty group past the end keeps the count)
+    };
+#pragma unroll 1
+    for (int grp = 0; grp < D; ++grp) issue(grp);
+#pragma unroll 1
+    for (int grp = 0; grp < ngroups; ++grp) {
+        seg_cp_async_wait<D - 1>();  // this lane's copy of group grp has landed
+        const int p = grp * g.rpi + sub;
+        if (vec_ok && p < n) {
+            float x[8];
+            unpack8_bf16(ring[(grp % D) * 32 + lane], x);
 #pragma unroll
-        for (int q = 0; q < RIF; ++q) {
-            const int slot = s + q * g.rpi + sub;
-            have[q] = vec_ok && slot < s1;
-            if (have[q]) u[q] = reinterpret_cast<const uint4*>(src + (int64_t)perm[slot] * ld)[v];
+            for (int t = 0; t < 8; ++t) acc[t] += (double)x[t];
         }
-#pragma unroll
-        for (int q = 0; q < RIF; ++q) {
-            if (have[q]) {
-                float x[8];
-                unpack8_bf16(u[q], x);
-#pragma unroll
-                for (int t = 0; t < 8; ++t) acc[t] += (double)x[t];
-            }
-        }
+        issue(grp + D);
     }
+    seg_cp_async_wait<0>();
     for (int o = g.lpr; o < 32; o <<= 1)
 #pragma unroll
         for (int t = 0; t < 8; ++t) acc[t] += __shfl_xor_sync(0xFFFFFFFFu, acc[t], o);
@@ -550,7 +571,8 @@ __device__ __forceinline__ float ema_slice(const ClusterState& st, int j, double
 // One warp per (work item, slice). A work item is a chunk of at most R label-sorted
 // rows of one cluster, and carries (cluster, first row, end row, whether the
 // cluster fits in one chunk), so that the row ids, the S slice and the previous
-// count are all fetched right after the item. A
+// count are all fetched right after the item; the rows stream through the warp's
+// ring in shared memory (sum_rows_staged). A
 // cluster that fits in one chunk is updated here; the chunks of a larger cluster
 // leave their slice sums in part[item] for k_clusters.
 #ifndef EM_SEGSUM_MIN_BLOCKS
@@ -562,6 +584,7 @@ __global__ void __launch_bounds__(256, EM_SEGSUM_MIN_BLOCKS) k_segsum(const __nv
                                                    ClusterState st, StepParams sp, double* __restrict__ part) {
     pdl_wait();
     pdl_release();
+    extern __shared__ __align__(16) uint4 seg_ring[];  // kSegsumDepth x 32 vectors per warp
     const int lane = threadIdx.x & 31;
     const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int item = warp / nslices, slice = warp - item * nslices;
@@ -576,7 +599,8 @@ __global__ void __launch_bounds__(256, EM_SEGSUM_MIN_BLOCKS) k_segsum(const __nv
         nprev = st.N_prev[j];
     }
     double acc[8];
-    sum_rows<kSegsumRif>(acc, src, st.ld, perm, it.y, it.z, g, lane);
+    sum_rows_staged(acc, src, st.ld, perm, it.y, it.z, g, lane,
+                    seg_ring + (size_t)(threadIdx.x >> 5) * kSegsumDepth * 32);
     if (it.w && sp.stats) {  // this rank's sums of the cluster, for the exchange
         if (lane < g.nvs) {
             double* dst = sp.stats + (int64_t)j * st.ld + 8 * (g.vbase + lane);

@@ -88,3 +88,25 @@ def test_data_parallel_argument_errors(em):
         m.dp_init_id(1, 0, uid)  # not during a run
     m.finalize()
     m.close()
+
+
+@pytest.mark.parametrize("d,k,epochs,batch", [(64, 50, 2.0, 512), (264, 120, 1.5, None)])
+def test_one_rank_statistics_path_against_the_oracle(em, d, k, epochs, batch):
+    """The data-parallel statistics path (this rank's sums and counts into the
+    exchange buffer, the all-reduce, the update from the buffer) checked against
+    the fp64 oracle itself, step by step under teacher forcing, not only against the
+    single-GPU run: batch order, labels, N, S and c after every step, revivals."""
+    from oracle import emeans_oracle as O
+    from tests.helpers import teacher_forced_run
+
+    x = synth.hand_shape(3000, d, max(2, k // 2), seed=d + k + 1)
+    xq = O.search_copy_of_data(x.numpy())
+    opts = dict(auto_revive=0, revival="split")
+    if batch:
+        opts["batch_size"] = batch
+    m = em.Model(d, k, seed=13, **opts)
+    _one_rank(em, m)
+    orc = O.EmeansOracle(d, k, seed=13, revival="split", batch_size=batch)
+    res = teacher_forced_run(m, orc, x.cuda(), xq, epochs, "split")
+    assert res["rows"] == int(round(epochs * 3000))
+    m.close()
