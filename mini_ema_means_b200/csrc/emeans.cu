@@ -733,7 +733,7 @@ static int launch_reduce(em_model* m, const __nv_bfloat16* src, int64_t rows, in
     double* const step_err = err_sum_out;
     if (dp) err_sum_out = stats_err;  // the error sum travels with the statistics
     launch_k(m->pdl, k_offsets, 1, 1024, 0, m->stream, m->cnt.p, (int)m->k, (int)rows, m->R, m->off.p, m->poff.p, m->block_err.p,
-                                         nblocks_labels, err_sum_out, m->N.p, m->N_prev.p, tie_list(m), m->err.p);
+                                         nblocks_labels, err_sum_out, tie_list(m), m->err.p);
     CK(cudaGetLastError());
     if (select_t >= 0) {
         // The revival check after this step: its donor selection needs only the new
@@ -989,7 +989,8 @@ static int launch_step(em_model* m, const StepPlan& p) {
     launch_k(m->pdl, k_labels, nbl, 256, 0, m->stream, m->keys.p, m->last_split, m->fp8 ? b.xn8.p : b.xn.p, (int)rows,
                                          (int)m->k, b.X.p, m->ld, m->cq.p, b.ids.p, m->labels.p, m->dists.p,
                                          m->cnt.p, m->rank.p, m->block_err.p, m->labels_last.p, capture,
-                                         training_kind(m), score_scale(m), tie_list(m), m->err.p);
+                                         training_kind(m), score_scale(m), tie_list(m), m->N.p, m->N_prev.p,
+                                         m->err.p);
     CK(cudaGetLastError());
     EM_LAUNCHED(m, 1);
     CKR(launch_settle(m, b.X.p, b.xn.p, m->labels.p, nullptr, m->dists.p, true, b.ids.p, m->labels_last.p,
@@ -1680,7 +1681,7 @@ int em_lloyd(em_model* m, const void* X, int64_t n, int64_t iters) {
         launch_k(m->pdl, k_labels, nbl, 256, 0, m->stream, m->keys.p, m->last_split, x2, (int)n, (int)m->k, m->X, m->ld,
                                              m->cq.p, nullptr, m->labels.p, m->dists.p, m->cnt.p, m->rank.p,
                                              m->block_err.p, nullptr, 0, training_kind(m), score_scale(m),
-                                             tie_list(m), m->err.p);
+                                             tie_list(m), m->N.p, m->N_prev.p, m->err.p);
         CK(cudaGetLastError());
         EM_LAUNCHED(m, 1);
         CKR(launch_settle(m, m->X, m->xn.p, m->labels.p, nullptr, m->dists.p, true, nullptr, nullptr, 0));

@@ -197,7 +197,8 @@ __global__ void k_labels(const unsigned long long* __restrict__ keys, int nsplit
                          const __nv_bfloat16* __restrict__ cq, const int32_t* __restrict__ ids,
                          int32_t* __restrict__ labels, float* __restrict__ dists, int32_t* __restrict__ cnt,
                          int32_t* __restrict__ rank, double* __restrict__ block_err, int64_t* __restrict__ labels_last,
-                         int capture, int kind, ScoreScale sc, TieList tl, int* err) {
+                         int capture, int kind, ScoreScale sc, TieList tl, const float* __restrict__ N,
+                         float* __restrict__ N_prev, int* err) {
     pdl_wait();
     pdl_release();
     __shared__ double warp_err[32];
@@ -205,6 +206,9 @@ __global__ void k_labels(const unsigned long long* __restrict__ keys, int nsplit
     double e = 0.0;
     const int r = blockIdx.x * blockDim.x + threadIdx.x;
     const bool active = r < rows;
+    // the running counts of before this step (N_prev), which the update and the
+    // revival selection derive the new counts from: one per thread across the grid
+    for (int j = r; j < k; j += gridDim.x * blockDim.x) N_prev[j] = N[j];
     uint32_t l1 = 0, l2 = 0;
     float s1 = 0.0f, s2 = 0.0f, x2 = 0.0f;
     bool tie = false;
@@ -263,15 +267,13 @@ __global__ void k_labels(const unsigned long long* __restrict__ keys, int nsplit
 // ceil(n_j / R) (first work item of each cluster, poff[0..k]); one CTA of 1024
 // threads, 16 consecutive clusters per thread (one pass up to 16,384 clusters).
 // Also adds the per-block error sums in a fixed order (each thread its strided
-// share, then a fixed butterfly and the warps in order) and keeps the running
-// counts of before this step (N_prev); both are issued ahead of the scan.
+// share, then a fixed butterfly and the warps in order), issued ahead of the scan.
 constexpr int kOffsetsPer = 16;
 
 __global__ void __launch_bounds__(1024) k_offsets(const int32_t* __restrict__ cnt, int k, int rows, int R,
                                                   int32_t* __restrict__ off, int32_t* __restrict__ poff,
                                                   const double* __restrict__ block_err, int nblocks,
-                                                  double* __restrict__ err_sum_out, const float* __restrict__ N,
-                                                  float* __restrict__ N_prev, TieList tl, int* err) {
+                                                  double* __restrict__ err_sum_out, TieList tl, int* err) {
     pdl_wait();
     pdl_release();
     __shared__ int2 warp_tot[32];
@@ -280,7 +282,6 @@ __global__ void __launch_bounds__(1024) k_offsets(const int32_t* __restrict__ cn
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
     double e = 0.0;
     for (int b = tid; b < nblocks; b += 1024) e += block_err[b];
-    for (int j = tid; j < k; j += 1024) N_prev[j] = N[j];
     if (tid == 0) carry_s = make_int2(0, 0);
     e = warp_sum(e);
     if (lane == 0) warp_err[w] = e;
