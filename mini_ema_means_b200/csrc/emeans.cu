@@ -791,13 +791,43 @@ static double effective_tau(const em_model* m) { return m->tau < 0.0 ? (m->d <= 
 
 static bool revival_on(const em_model* m) { return m->revival != EM_REVIVE_NONE && effective_tau(m) > 0.0; }
 
+// Shared memory the donor selection kernels may take (the tree and the split counters).
+static bool select_smem_attributes() {
+    const int b = kReviveSmemBytes;
+    const cudaFuncAttribute a = cudaFuncAttributeMaxDynamicSharedMemorySize;
+    return cudaFuncSetAttribute(k_revive_select, a, b) == cudaSuccess &&
+           cudaFuncSetAttribute(k_revive_select_flat<1, 1>, a, b) == cudaSuccess &&
+           cudaFuncSetAttribute(k_revive_select_flat<1, 2>, a, b) == cudaSuccess &&
+           cudaFuncSetAttribute(k_revive_select_flat<1, 4>, a, b) == cudaSuccess &&
+           cudaFuncSetAttribute(k_revive_select_flat<2, 4>, a, b) == cudaSuccess &&
+           cudaFuncSetAttribute(k_revive_select_flat<4, 4>, a, b) == cudaSuccess;
+}
+
 // The donor selection of the revival check after step t, on `stream`, reading the
 // running counts from `src`.
 static int launch_select(em_model* m, int64_t t, cudaStream_t stream, bool pdl, CountSource src) {
     const ReviveScratch sc = revive_scratch(m);
-    const int smem = m->k <= kFastK ? tree32((int)m->k).bytes : (int)tree_smem_bytes(tree_layout((int)m->k), (int)m->k);
-    launch_k(pdl, k_revive_select, 1, kSelectThreads, smem, stream, src, (int)m->k, effective_tau(m), m->seed, t,
-             m->revival, sc, m->err.p);
+    const int k = (int)m->k;
+    const double tau = effective_tau(m);
+    // two-level trees (group size 32 S0, root of at most 32 SR entries) up to kFastK
+    if (k <= 1024)
+        launch_k(pdl, k_revive_select_flat<1, 1>, 1, kSelectThreads, flat_smem_bytes<1>(k), stream, src, k, tau,
+                 m->seed, t, m->revival, sc);
+    else if (k <= 2048)
+        launch_k(pdl, k_revive_select_flat<1, 2>, 1, kSelectThreads, flat_smem_bytes<1>(k), stream, src, k, tau,
+                 m->seed, t, m->revival, sc);
+    else if (k <= 4096)
+        launch_k(pdl, k_revive_select_flat<1, 4>, 1, kSelectThreads, flat_smem_bytes<1>(k), stream, src, k, tau,
+                 m->seed, t, m->revival, sc);
+    else if (k <= 8192)
+        launch_k(pdl, k_revive_select_flat<2, 4>, 1, kSelectThreads, flat_smem_bytes<2>(k), stream, src, k, tau,
+                 m->seed, t, m->revival, sc);
+    else if (k <= kFastK)
+        launch_k(pdl, k_revive_select_flat<4, 4>, 1, kSelectThreads, flat_smem_bytes<4>(k), stream, src, k, tau,
+                 m->seed, t, m->revival, sc);
+    else
+        launch_k(pdl, k_revive_select, 1, kSelectThreads, (int)tree_smem_bytes(tree_layout(k), k), stream, src, k,
+                 tau, m->seed, t, m->revival, sc, m->err.p);
     CK(cudaGetLastError());
     EM_LAUNCHED(m, 1);
     return EM_OK;
@@ -1357,9 +1387,7 @@ em_model* em_create(int64_t d, int64_t k, uint64_t seed) {
     cudaMemset(m->c.p, 0, kd * sizeof(float));
     cudaMemset(m->cq.p, 0, kd * sizeof(__nv_bfloat16));
     cudaMemset(m->cn.p, 0, k * sizeof(float));
-    if (!search_smem_attributes() ||
-        cudaFuncSetAttribute(k_revive_select, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kReviveSmemBytes) != cudaSuccess)
+    if (!search_smem_attributes() || !select_smem_attributes())
         return bail(EM_E_CUDA, "cudaFuncSetAttribute failed");
     if (make_tmap(&m->tm_cq, m->cq.p, k, (int)d, m->ld, tc::BN, m->kc) != EM_OK) {
         em_destroy(m);

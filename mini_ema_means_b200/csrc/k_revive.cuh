@@ -17,16 +17,15 @@
 //
 // The draws are inherently sequential, so one warp makes them on an fp64 tree of
 // prefix sums, the uniform draws having been made in parallel beforehand. Up to
-// 16,384 clusters the tree has 32 children per node, one per lane, and lives in
-// shared memory with its top level in registers: a draw costs one load, one
-// compare, one ballot and one shuffle per level. Larger k use 128 children per
-// node (four per lane), with the lower levels in global memory when shared memory
-// runs out. The donor's
-// current weight is read back as the difference of two prefix values, and the
-// number of earlier splits from the same donor is counted per batch of 32 draws
-// with one warp match. The vector work is then done in parallel from the closed
-// form: the o-th split taken from donor d (0-based) sees c_d (1 + eps s)^o and
-// N_d / 2^o.
+// 16,384 clusters the tree has two levels: groups of 32, 64 or 128 clusters in
+// shared memory and a root of at most 128 group totals in the drawing warp's
+// registers, each lane holding every 32nd position; a level costs a few compares,
+// ballots and population counts. Larger k use 128 children per node (four per
+// lane) on as many levels as needed, the lower ones in global memory when shared
+// memory runs out. The number of earlier splits from the same donor is counted
+// per batch of 32 draws with one warp match. The vector work is then done in
+// parallel from the closed form: the o-th split taken from donor d (0-based) sees
+// c_d (1 + eps s)^o and N_d / 2^o.
 #pragma once
 
 #include "k_reduce.cuh"
@@ -193,143 +192,6 @@ __device__ __forceinline__ bool group_sub(double P[4], int pos, double delta, in
     return 4 * lane + 3 >= pos;
 }
 
-// ---- radix-32 tree for k <= kFastK: one value per lane at every level
-//
-// Level 0 holds, for each group of 32 consecutive clusters, the inclusive prefix
-// sums of their current weights within the group; level 1 the same over the group
-// totals of level 0; level 2 over those of level 1. The top level (at most 32
-// entries) sits in the drawing warp's registers, one entry per lane, and the levels
-// below it in shared memory. A draw then costs, per level, one load, one compare,
-// one ballot and one shuffle, about a third of the instructions of the radix-128
-// descent; a single warp issuing alone is bound by that count.
-constexpr int kFastK = 16384;
-
-struct Tree32 {
-    int levels;   // 1 (k <= 32), 2 (k <= 1024) or 3
-    int n1;       // entries of level 1 = groups of level 0
-    int n2;       // entries of level 2 = groups of level 1
-    int off1;     // doubles: level 1 (levels == 3), after the top staging group
-    int off0;     // doubles: level 0 (levels >= 2)
-    int times;    // doubles: per-donor split counters (ints), -1 when they do not fit
-    int bytes;    // shared memory
-};
-
-EM_HD Tree32 tree32(int k) {
-    Tree32 T{};
-    T.n1 = (k + 31) / 32;
-    T.n2 = (T.n1 + 31) / 32;
-    T.levels = k <= 32 ? 1 : (k <= 1024 ? 2 : 3);
-    int off = 32;  // top staging group
-    T.off1 = off;
-    if (T.levels == 3) off += T.n2 * 32;  // level 1, padded to whole groups
-    T.off0 = off;
-    if (T.levels >= 2) off += T.n1 * 32;  // level 0, padded to whole groups
-    const int base = off * 8;
-    const int tb = ((k * 4 + 15) / 16) * 16;
-    T.times = base + tb <= kReviveSmemBytes ? off : -1;
-    T.bytes = base + (T.times >= 0 ? tb : 0);
-    return T;
-}
-
-// Inclusive prefix of one value per lane.
-__device__ __forceinline__ double lane_scan(double v, int lane) { return warp_incl_scan(v, lane); }
-
-// First lane whose value passes (ballot, then the lowest set lane); -1 if none.
-__device__ __forceinline__ int first_lane(bool pred) {
-    const unsigned b = __ballot_sync(0xFFFFFFFFu, pred);
-    return b ? __ffs(b) - 1 : -1;
-}
-
-// Sequential donor draws of dead clusters [0, nd) on the radix-32 tree, by one warp.
-// T / Tprev: this lane's inclusive / exclusive prefix of the top level; W: the total.
-// Writes donor, order (earlier splits of the same donor in this check) and the
-// per-donor counters; returns the number of splits.
-template <int LEVELS>
-__device__ __forceinline__ int64_t draw_radix32(double* smem_d, const Tree32& TL, int nd, const ReviveScratch& sc,
-                                                int32_t* times, int lane) {
-    double T = smem_d[lane];
-    double Tprev = lane ? smem_d[lane - 1] : 0.0;
-    double W = __shfl_sync(0xFFFFFFFFu, T, 31);
-    double* L1 = smem_d + TL.off1;
-    double* L0 = smem_d + TL.off0;
-    int64_t splits = 0;
-    int i_end = nd;
-    for (int i0 = 0; i0 < nd; i0 += 32) {
-        const int cnt = min(32, nd - i0);
-        const double my_u = lane < cnt ? sc.target[i0 + lane] : 0.0;
-        int my_dn = -1;
-        for (int q = 0; q < cnt; ++q) {
-            if (!(W > 0.0)) {
-                i_end = i0 + q;
-                break;
-            }
-            const double tg = __shfl_sync(0xFFFFFFFFu, my_u, q) * W;
-            // a target on (or, rounded, past) the total takes the last cluster with
-            // weight: at every level, the first position whose prefix reaches its total
-            const bool on_total = !(tg < W);
-            int g2 = first_lane(on_total ? T >= W : T > tg);
-            if (g2 < 0) g2 = first_lane(T >= W);
-            double before = __shfl_sync(0xFFFFFFFFu, Tprev, g2);
-            int d, l1 = 0, l0 = 0, base1 = 0, base0 = 0;
-            double v1 = 0.0, v0 = 0.0, w;
-            if (LEVELS == 1) {
-                d = g2;
-                w = __shfl_sync(0xFFFFFFFFu, T - Tprev, g2);
-            } else {
-                int g1 = g2;
-                if (LEVELS == 3) {
-                    base1 = g2 * 32;
-                    v1 = L1[base1 + lane];
-                    const double v1p = lane ? L1[base1 + lane - 1] : 0.0;
-                    const double tot1 = __shfl_sync(0xFFFFFFFFu, v1, 31);
-                    l1 = first_lane(on_total ? v1 >= tot1 : before + v1 > tg);
-                    if (l1 < 0) l1 = first_lane(v1 >= tot1);  // (exact sums: never)
-                    before += __shfl_sync(0xFFFFFFFFu, v1p, l1);
-                    g1 = base1 + l1;
-                }
-                base0 = g1 * 32;
-                v0 = L0[base0 + lane];
-                const double v0p = lane ? L0[base0 + lane - 1] : 0.0;
-                const double tot0 = __shfl_sync(0xFFFFFFFFu, v0, 31);
-                l0 = first_lane(on_total ? v0 >= tot0 : before + v0 > tg);
-                if (l0 < 0) l0 = first_lane(v0 >= tot0);  // (exact sums: never)
-                d = base0 + l0;
-                w = __shfl_sync(0xFFFFFFFFu, v0 - v0p, l0);
-            }
-            // the donor keeps the rounded half of its weight; explicit roundings, since
-            // a fused multiply-add would round the half differently in the subnormal range
-            const double keep = __dmul_rn(0.5, w);
-            const double delta = __dsub_rn(w, keep);
-            if (LEVELS >= 2 && lane >= l0) L0[base0 + lane] = v0 - delta;
-            if (LEVELS == 3 && lane >= l1) L1[base1 + lane] = v1 - delta;
-            if (lane >= g2) T -= delta;
-            if (lane > g2) Tprev -= delta;
-            W -= delta;
-            if (lane == q) my_dn = d;
-            __syncwarp();  // the group stored above may be the next draw's
-        }
-        const bool has = lane < cnt && my_dn >= 0;
-        const unsigned peers = __match_any_sync(0xFFFFFFFFu, has ? my_dn : -1);
-        const int leader = __ffs(peers) - 1;
-        int old = 0;
-        if (has && lane == leader) old = times[my_dn];
-        old = __shfl_sync(0xFFFFFFFFu, old, leader);
-        if (has) {
-            const int rk = __popc(peers & ((1u << lane) - 1u));
-            sc.donor[i0 + lane] = my_dn;
-            sc.order[i0 + lane] = old + rk;
-            if (lane == leader) times[my_dn] = old + __popc(peers);
-        } else if (lane < cnt) {
-            sc.donor[i0 + lane] = -1;
-        }
-        splits += __popc(__ballot_sync(0xFFFFFFFFu, has));
-        __syncwarp();  // the counters written above are read by other lanes next batch
-        if (i_end < nd) break;
-    }
-    for (int i = (i_end / 32 + 1) * 32 + lane; i < nd; i += 32) sc.donor[i] = -1;
-    return splits;
-}
-
 // One CTA of kSelectThreads threads: dead set, donor tree, sequential donor draws
 // by warp 0 (which keeps one group per tree level in registers).
 constexpr int kSelectThreads = 512;
@@ -408,47 +270,6 @@ __global__ void __launch_bounds__(kSelectThreads) k_revive_select(CountSource N,
     for (int i = tid; i < nd; i += kSelectThreads) sc.target[i] = draw_uniform(seed, kStreamRevive, t, sc.dead[i]);
 
     extern __shared__ __align__(16) double smem_d[];
-    if (k <= kFastK) {  // radix-32 tree in shared memory
-        const Tree32 TL = tree32(k);
-        int32_t* times = TL.times >= 0 ? reinterpret_cast<int32_t*>(smem_d + TL.times) : sc.times;
-        for (int j = tid; j < k; j += kSelectThreads) times[j] = 0;
-        // level 0 (the staging group when it is the top)
-        double* L0 = TL.levels == 1 ? smem_d : smem_d + TL.off0;
-        for (int g = w; g < TL.n1; g += kSelectWarps) {
-            const int j = g * 32 + lane;
-            const float nj = j < k ? N(j) : 0.0f;
-            const double v = (j < k && !((double)nj < thr)) ? (double)nj : 0.0;
-            L0[g * 32 + lane] = lane_scan(v, lane);
-        }
-        __syncthreads();
-        if (TL.levels >= 2) {  // level 1 (staged when it is the top)
-            double* L1 = TL.levels == 2 ? smem_d : smem_d + TL.off1;
-            for (int g = w; g < TL.n2; g += kSelectWarps) {
-                const int i = g * 32 + lane;
-                const double v = i < TL.n1 ? L0[i * 32 + 31] : 0.0;
-                L1[g * 32 + lane] = lane_scan(v, lane);
-            }
-            __syncthreads();
-        }
-        if (TL.levels == 3) {  // level 2, the top
-            if (w == 0) {
-                const double v = lane < TL.n2 ? smem_d[TL.off1 + lane * 32 + 31] : 0.0;
-                smem_d[lane] = lane_scan(v, lane);
-            }
-            __syncthreads();
-        }
-        if (w == 0) {
-            const int64_t splits = TL.levels == 1   ? draw_radix32<1>(smem_d, TL, nd, sc, times, lane)
-                                   : TL.levels == 2 ? draw_radix32<2>(smem_d, TL, nd, sc, times, lane)
-                                                    : draw_radix32<3>(smem_d, TL, nd, sc, times, lane);
-            if (lane == 0) *sc.n_splits += splits;
-        }
-        __syncthreads();
-        if (TL.times >= 0)
-            for (int j = tid; j < k; j += kSelectThreads) sc.times[j] = times[j];
-        return;
-    }
-
     // donor tree for larger k (loops over levels have a fixed trip count so that
     // the layout stays in registers)
     const TreeLayout L = tree_layout(k);
@@ -604,6 +425,257 @@ __global__ void __launch_bounds__(kSelectThreads) k_revive_select(CountSource N,
     __syncthreads();
     if (L.times_smem)
         for (int j = tid; j < k; j += kSelectThreads) sc.times[j] = times[j];
+}
+
+// ---- two-level tree for k <= kFastK, drawn without a shared-memory round trip
+//
+// Level 0 holds, for every group of G0 = 32 S0 consecutive clusters, the inclusive
+// prefix sums of their current weights within the group (dead clusters and the
+// padding past k weigh 0, so padding repeats the group total). The root holds the
+// inclusive prefix of the group totals, at most 32 SR entries, in the drawing
+// warp's registers. Lane l holds position 32 s + l of a group (or of the root) in
+// its slot s, so each lane only ever reads and writes its own positions and the
+// descent needs no warp barrier.
+//
+// A draw counts the positions whose cumulative weight is at most the target: the
+// first position past the target is the donor, as in a search of the cumulative
+// sums of all k weights. Each level costs S (slots) compares, S ballots and S
+// population counts, with no find-first-set and no select over fp64 values. The
+// compares are made on the IEEE 754 encodings: for non-negative doubles the order
+// of the bit patterns as signed 64-bit integers is the order of the values. A
+// target on (or rounded past) the total becomes the largest double below the
+// total, so that the first position reaching the total (the last cluster with
+// weight) is taken, without a branch.
+constexpr int kFastK = 16384;
+
+template <int S0>
+EM_HD int flat_groups(int k) { return (k + 32 * S0 - 1) / (32 * S0); }
+
+template <int S0>
+EM_HD int flat_smem_bytes(int k) {
+    return flat_groups<S0>(k) * 32 * S0 * 8 + ((k * 4 + 15) / 16) * 16;
+}
+
+__device__ __forceinline__ long long dbits(double x) { return __double_as_longlong(x); }
+
+// Slot `s` of a lane's N values (N = 1, 2 or 4; any slot when s is out of range),
+// by selects on the bits of s: an index into a register array would move the
+// array to local memory.
+template <int N>
+__device__ __forceinline__ double pick(const double (&x)[N], int s) {
+    if (N == 1) return x[0];
+    const double lo = (s & 1) ? x[1 % N] : x[0];
+    if (N == 2) return lo;
+    const double hi = (s & 1) ? x[3 % N] : x[2 % N];
+    return (s & 2) ? hi : lo;
+}
+
+template <int S0, int SR>
+__global__ void __launch_bounds__(kSelectThreads) k_revive_select_flat(CountSource N, int k, double tau, uint64_t seed,
+                                                             int64_t t, int mode, ReviveScratch sc) {
+    pdl_wait();
+    constexpr int G0 = 32 * S0;
+    constexpr int RMAX = kFastK / kSelectThreads;  // rows of kSelectThreads clusters
+    __shared__ double red[kSelectWarps];
+    __shared__ double ctot[RMAX * kSelectWarps];    // per (row, warp) chunk totals
+    __shared__ int32_t rcnt[RMAX * kSelectWarps];   // per (row, warp) dead counts, then offsets
+    __shared__ int32_t wsum[kSelectWarps];
+    __shared__ double gtot[32 * SR];                // group totals (the root's entries)
+    extern __shared__ __align__(16) double smem_d[];
+    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+    const int R = (k + kSelectThreads - 1) / kSelectThreads;
+    const int ngroups = flat_groups<S0>(k);
+    double* L0 = smem_d;
+    int32_t* times = reinterpret_cast<int32_t*>(smem_d + (int64_t)ngroups * G0);
+
+    // running counts of cluster tid + kSelectThreads r, loaded once; total in the
+    // order of the other selection kernel (r, then lanes, then warps)
+    float nv[RMAX];
+    double part = 0.0;
+#pragma unroll
+    for (int r = 0; r < RMAX; ++r) {
+        const int j = tid + kSelectThreads * r;
+        nv[r] = (r < R && j < k) ? N(j) : 0.0f;
+        if (r < R && j < k) part += (double)nv[r];
+    }
+    part = warp_sum(part);
+    if (lane == 0) red[w] = part;
+    for (int j = tid; j < k; j += kSelectThreads) times[j] = 0;
+    __syncthreads();
+    const double total = warp_sum(lane < kSelectWarps ? red[lane] : 0.0);
+    const double thr = tau * (total / (double)k);
+
+    // dead set in increasing index: counts per (row, warp), their exclusive scan in
+    // row-major order, then each dead cluster's place
+    unsigned dmask = 0;
+    int my_rc = 0;
+#pragma unroll
+    for (int r = 0; r < RMAX; ++r) {
+        if (r < R) {
+            const int j = tid + kSelectThreads * r;
+            const bool dead = j < k && (double)nv[r] < thr;
+            dmask |= dead ? (1u << r) : 0u;
+            const int c = __popc(__ballot_sync(0xFFFFFFFFu, dead));
+            if (lane == r) my_rc = c;
+        }
+    }
+    if (lane < R) rcnt[lane * kSelectWarps + w] = my_rc;
+    __syncthreads();
+    const int c_in = tid < R * kSelectWarps ? rcnt[tid] : 0;
+    int incl = c_in;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+        if (lane >= o) incl += v;
+    }
+    if (lane == 31) wsum[w] = incl;
+    __syncthreads();
+    const int wv = lane < kSelectWarps ? wsum[lane] : 0;
+    int before_w = lane < w ? wv : 0;
+    int nd = wv;
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+        before_w += __shfl_xor_sync(0xFFFFFFFFu, before_w, o);
+        nd += __shfl_xor_sync(0xFFFFFFFFu, nd, o);
+    }
+    if (tid < R * kSelectWarps) rcnt[tid] = before_w + incl - c_in;
+    __syncthreads();
+#pragma unroll
+    for (int r = 0; r < RMAX; ++r) {
+        if (r < R) {
+            const bool dead = (dmask >> r) & 1u;
+            const unsigned b = __ballot_sync(0xFFFFFFFFu, dead);
+            if (dead) sc.dead[rcnt[r * kSelectWarps + w] + __popc(b & ((1u << lane) - 1u))] = tid + kSelectThreads * r;
+        }
+    }
+    if (tid == 0) *sc.ndead = nd;
+    if (mode != EM_REVIVE_SPLIT || nd == 0 || !(total > 0.0)) {
+        for (int i = tid; i < nd; i += kSelectThreads) sc.donor[i] = -1;
+        for (int j = tid; j < k; j += kSelectThreads) sc.times[j] = 0;
+        return;
+    }
+
+    // level 0 from the loaded counts: warp w's row r is 32 consecutive positions of
+    // group (kSelectThreads r + 32 w) / G0, scanned here; the S0 chunks of a group
+    // are then joined in order (every sum is exact, see above)
+#pragma unroll
+    for (int r = 0; r < RMAX; ++r) {
+        if (r < R) {
+            const int j = tid + kSelectThreads * r;
+            const double v = ((dmask >> r) & 1u) || j >= k ? 0.0 : (double)nv[r];
+            const double x = warp_incl_scan(v, lane);
+            if (j < ngroups * G0) L0[j] = x;
+            if (S0 == 1 && lane == 31 && j < ngroups * G0) gtot[j / G0] = x;
+            if (S0 > 1 && lane == 31) ctot[r * kSelectWarps + w] = x;
+        }
+    }
+    __syncthreads();  // (also publishes the dead list written above)
+    if (S0 > 1) {
+#pragma unroll
+        for (int r = 0; r < RMAX; ++r) {
+            const int j = tid + kSelectThreads * r;
+            if (r < R && j < ngroups * G0) {
+                const int first = w - (w % S0);
+                if (w != first) {
+                    double off = 0.0;
+                    for (int q = first; q < w; ++q) off += ctot[r * kSelectWarps + q];
+                    const double x = L0[j] + off;
+                    L0[j] = x;
+                    if (lane == 31 && w - first == S0 - 1) gtot[j / G0] = x;
+                }
+            }
+        }
+    }
+    // draws of every dead cluster, in parallel (they do not depend on each other)
+    for (int i = tid; i < nd; i += kSelectThreads) sc.target[i] = draw_uniform(seed, kStreamRevive, t, sc.dead[i]);
+    __syncthreads();
+
+    if (w == 0) {
+        double T[SR];
+        double carry = 0.0;
+#pragma unroll
+        for (int s = 0; s < SR; ++s) {
+            const int pos = 32 * s + lane;
+            const double x = warp_incl_scan(pos < ngroups ? gtot[pos] : 0.0, lane) + carry;
+            carry = __shfl_sync(0xFFFFFFFFu, x, 31);
+            T[s] = pos < ngroups ? x : __longlong_as_double(0x7FF0000000000000ll);  // +inf past the root
+        }
+        double W = carry;
+        int64_t splits = 0;
+        double u_cur = lane < nd ? sc.target[lane] : 0.0;
+        for (int i0 = 0; i0 < nd; i0 += 32) {
+            const int cnt = min(32, nd - i0);
+            const double u_next = i0 + 32 + lane < nd ? sc.target[i0 + 32 + lane] : 0.0;
+            int my_dn = -1;
+            for (int q = 0; q < cnt; ++q) {
+                const bool live = W > 0.0;
+                const double tg = __dmul_rn(__shfl_sync(0xFFFFFFFFu, u_cur, q), W);
+                const long long tb = min(dbits(tg), dbits(W) - 1);
+                int g = 0;
+#pragma unroll
+                for (int s = 0; s < SR; ++s) g += __popc(__ballot_sync(0xFFFFFFFFu, dbits(T[s]) <= tb));
+                g = min(g, ngroups - 1);
+                // cumulative weight of the groups before g: root position g - 1
+                const int gp = g - 1;
+                const double ts = pick<SR>(T, gp >> 5);
+                double before = __shfl_sync(0xFFFFFFFFu, ts, gp & 31);
+                if (g == 0) before = 0.0;
+                double* grp = L0 + (int64_t)g * G0;
+                double v[S0];
+#pragma unroll
+                for (int s = 0; s < S0; ++s) v[s] = grp[32 * s + lane];
+                int p = 0;
+#pragma unroll
+                for (int s = 0; s < S0; ++s)
+                    p += __popc(__ballot_sync(0xFFFFFFFFu, dbits(__dadd_rn(before, v[s])) <= tb));
+                p = min(p, G0 - 1);
+                // the donor's weight: within-group prefix at p minus the one before it
+                const double va = pick<S0>(v, p >> 5);
+                const double vb = pick<S0>(v, (p - 1) >> 5);
+                const double a = __shfl_sync(0xFFFFFFFFu, va, p & 31);
+                double b = __shfl_sync(0xFFFFFFFFu, vb, (p - 1) & 31);
+                if (p == 0) b = 0.0;
+                const double wt = __dsub_rn(a, b);
+                // the donor keeps the rounded half of its weight (what halving N_d gives);
+                // explicit roundings: a fused multiply-add would round the half
+                // differently in the subnormal range
+                const double keep = __dmul_rn(0.5, wt);
+                const double delta = live ? __dsub_rn(wt, keep) : 0.0;
+#pragma unroll
+                for (int s = 0; s < S0; ++s)
+                    if (32 * s + lane >= p) grp[32 * s + lane] = __dsub_rn(v[s], delta);
+#pragma unroll
+                for (int s = 0; s < SR; ++s)
+                    if (32 * s + lane >= g) T[s] = __dsub_rn(T[s], delta);
+                W = __dsub_rn(W, delta);
+                // (a position past k or a drained total can only come from inexact
+                // sums, which the weights' range rules out: no donor then)
+                const int d = g * G0 + p;
+                if (lane == q) my_dn = live && d < k ? d : -1;
+            }
+            // record the batch: donor, and how many earlier splits took the same donor
+            const bool has = lane < cnt && my_dn >= 0;
+            const unsigned peers = __match_any_sync(0xFFFFFFFFu, has ? my_dn : -1);
+            const int leader = __ffs(peers) - 1;
+            int old = 0;
+            if (has && lane == leader) old = times[my_dn];
+            old = __shfl_sync(0xFFFFFFFFu, old, leader);
+            if (has) {
+                const int rk = __popc(peers & ((1u << lane) - 1u));
+                sc.donor[i0 + lane] = my_dn;
+                sc.order[i0 + lane] = old + rk;
+                if (lane == leader) times[my_dn] = old + __popc(peers);
+            } else if (lane < cnt) {
+                sc.donor[i0 + lane] = -1;
+            }
+            splits += __popc(__ballot_sync(0xFFFFFFFFu, has));
+            __syncwarp();  // the counters written above are read by other lanes next batch
+            u_cur = u_next;
+        }
+        if (lane == 0) *sc.n_splits += splits;
+    }
+    __syncthreads();
+    for (int j = tid; j < k; j += kSelectThreads) sc.times[j] = times[j];
 }
 
 // Dead clusters take their half of the donor (reads the donors' state before

@@ -408,13 +408,13 @@ def test_failure_path_reports_timeout_and_bounds_and_recovers(em):
     assert m.selftest(2) == em.EM_E_INVAL
 
 
-@pytest.mark.parametrize("k", [70, 3000, 20000])
+@pytest.mark.parametrize("k", [70, 3000, 6000, 12000, 20000])
 def test_overlapped_selection_matches_serial_revival(em, k):
     """The revival check's donor selection runs beside the segmented sums, deriving
     the new running counts from N_prev and the segment sizes; with profiling on it
     runs in line after the update. Both give the same run, bit for bit (dead sets,
-    donors, counts, centroids), on the radix-32 tree (k <= 16,384) and the radix-128
-    one."""
+    donors, counts, centroids), on the two-level trees of every group size
+    (k <= 16,384) and the radix-128 one."""
     x = synth.hand_shape(max(4 * k, 6000), 24, max(8, k // 3), seed=k)
     outs = []
     for profile in (0, 1):
