@@ -533,6 +533,11 @@ __device__ __forceinline__ float ema_count(float nprev, double nj, double alpha)
     return (float)__dadd_rn(__dmul_rn(a1, (double)nprev), __dmul_rn(alpha, nj));
 }
 
+// The centroid is S / N rounded to fp32, computed as the IEEE fp32 quotient of the
+// fp32 S and N: dividing in fp64 and rounding to fp32 gives the same value, since
+// a 53-bit quotient rounded again to 24 bits is the correctly rounded 24-bit
+// quotient (53 >= 2 x 24 + 2; Figueroa, "When is double rounding innocuous?",
+// 1995), and fp32 operands can neither overflow nor underflow in fp64.
 // EMA of one slice of cluster j from its batch sums (lanes l < nvs hold vector
 // vbase + l) and its previous sums so[]: writes S, c, the bf16 operand and the
 // closing-mean sums; slice 0 also writes N and the closing-mean count. Returns
@@ -549,7 +554,7 @@ __device__ __forceinline__ float ema_slice(const ClusterState& st, int j, double
 #pragma unroll
         for (int t = 0; t < 8; ++t) {
             sn[t] = (float)(a1 * (double)so[t] + alpha * acc[t]);
-            cv[t] = (float)((double)sn[t] / (double)Nnew);
+            cv[t] = __fdiv_rn(sn[t], Nnew);  // = (float)((double)sn / (double)N): see above
         }
         float4* sp = reinterpret_cast<float4*>(st.S + (int64_t)j * st.ld) + 2 * v;
         sp[0] = make_float4(sn[0], sn[1], sn[2], sn[3]);
