@@ -8,7 +8,9 @@
 //
 // Structure of one CTA (320 threads, one CTA per SM, persistent over work units):
 //   warp 0      TMA producer: 128 x KC tiles of A and 256 x KC tiles of the
-//               centroid operand into a STAGES-deep shared-memory ring
+//               centroid operand into a STAGES-deep shared-memory ring (with the
+//               batch tile stationary, a stage holds a whole 256-row centroid tile,
+//               so that a tile costs one barrier round trip, not one per K chunk)
 //   warp 1      allocates 512 TMEM columns; one thread issues tcgen05.mma
 //               (M=128, N=256, K=16, bf16 x bf16 -> fp32) into one of two
 //               TMEM accumulators and commits to mbarriers
@@ -353,6 +355,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int m_tiles = (rows + BM - 1) / BM;
     const int tpg = (n_tiles + n_split - 1) / n_split;
     const int units = m_full + (m_tiles - m_full) * n_split;
+    // ring stages in use: chunk stages, or (A stationary) whole centroid tiles of nkc
+    // chunks each, so that a tile costs one barrier round trip instead of nkc
+    const int st_n = AST ? S / nkc : S;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
@@ -417,7 +422,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ++ua;
                 }
                 for (int nt = nt0; nt < nt1 && ok; ++nt) {
-                    for (int kc = 0; kc < nkc; ++kc) {
+                    if (AST) {  // the whole centroid tile into one stage of nkc chunks, one barrier
                         if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, wait_limit, err, abort_flag)) {
                             ok = false;
                             break;
@@ -425,12 +430,29 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const uint32_t fb = smem_u32(&full[stage]);
                         armed |= 1u << stage;
                         armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
-                        mbar_expect_tx(fb, C::kStageBytes);
-                        if (!AST) tma_load_2d(smem_u32(sA + stage * C::kABytes), &tmA, kc * KX, m * BM, fb);
-                        tma_load_2d(smem_u32(sB + stage * C::kBBytes), &tmB, kc * KX, nt * BN, fb);
-                        if (++stage == S) {
+                        mbar_expect_tx(fb, (uint32_t)(nkc * C::kBBytes));
+                        for (int kc = 0; kc < nkc; ++kc)
+                            tma_load_2d(smem_u32(sB + (stage * nkc + kc) * C::kBBytes), &tmB, kc * KX, nt * BN, fb);
+                        if (++stage == st_n) {
                             stage = 0;
                             phase ^= 1u;
+                        }
+                    } else {
+                        for (int kc = 0; kc < nkc; ++kc) {
+                            if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, wait_limit, err, abort_flag)) {
+                                ok = false;
+                                break;
+                            }
+                            const uint32_t fb = smem_u32(&full[stage]);
+                            armed |= 1u << stage;
+                            armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+                            mbar_expect_tx(fb, C::kStageBytes);
+                            tma_load_2d(smem_u32(sA + stage * C::kABytes), &tmA, kc * KX, m * BM, fb);
+                            tma_load_2d(smem_u32(sB + stage * C::kBBytes), &tmB, kc * KX, nt * BN, fb);
+                            if (++stage == S) {
+                                stage = 0;
+                                phase ^= 1u;
+                            }
                         }
                     }
                 }
@@ -469,31 +491,56 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     tc_fence_after();
                     const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
-                    for (int kc = 0; kc < nkc; ++kc) {
+                    if (AST) {  // one stage holds the tile's nkc chunks
                         if (!mbar_wait(smem_u32(&full[stage]), phase, wait_limit, err, abort_flag)) {
                             ok = false;
                             break;
                         }
                         tc_fence_after();
-                        const uint32_t a0 = AST ? smem_u32(sArea + ab * kAstBufBytes + kc * C::kABytes)
-                                                : smem_u32(sA + stage * C::kABytes);
-                        const uint32_t b0 = smem_u32(sB + stage * C::kBBytes);
+                        for (int kc = 0; kc < nkc; ++kc) {
+                            const uint32_t a0 = smem_u32(sArea + ab * kAstBufBytes + kc * C::kABytes);
+                            const uint32_t b0 = smem_u32(sB + (stage * nkc + kc) * C::kBBytes);
 #pragma unroll
-                        for (int kk = 0; kk < KC / 16; ++kk) {
-                            const uint64_t ad = smem_desc(a0 + kk * 32, C::kLayout, C::kSBO);
-                            const uint64_t bd = smem_desc(b0 + kk * 32, C::kLayout, C::kSBO);
-                            if (F8)
-                                umma_e4m3(d_tmem, ad, bd, (kc | kk) != 0);
-                            else
-                                umma_bf16(d_tmem, ad, bd, (kc | kk) != 0);
+                            for (int kk = 0; kk < KC / 16; ++kk) {
+                                const uint64_t ad = smem_desc(a0 + kk * 32, C::kLayout, C::kSBO);
+                                const uint64_t bd = smem_desc(b0 + kk * 32, C::kLayout, C::kSBO);
+                                if (F8)
+                                    umma_e4m3(d_tmem, ad, bd, (kc | kk) != 0);
+                                else
+                                    umma_bf16(d_tmem, ad, bd, (kc | kk) != 0);
+                            }
                         }
                         umma_commit(smem_u32(&empty[stage]));
-                        if (++stage == S) {
+                        if (++stage == st_n) {
                             stage = 0;
                             phase ^= 1u;
                         }
+                    } else {
+                        for (int kc = 0; kc < nkc; ++kc) {
+                            if (!mbar_wait(smem_u32(&full[stage]), phase, wait_limit, err, abort_flag)) {
+                                ok = false;
+                                break;
+                            }
+                            tc_fence_after();
+                            const uint32_t a0 = smem_u32(sA + stage * C::kABytes);
+                            const uint32_t b0 = smem_u32(sB + stage * C::kBBytes);
+#pragma unroll
+                            for (int kk = 0; kk < KC / 16; ++kk) {
+                                const uint64_t ad = smem_desc(a0 + kk * 32, C::kLayout, C::kSBO);
+                                const uint64_t bd = smem_desc(b0 + kk * 32, C::kLayout, C::kSBO);
+                                if (F8)
+                                    umma_e4m3(d_tmem, ad, bd, (kc | kk) != 0);
+                                else
+                                    umma_bf16(d_tmem, ad, bd, (kc | kk) != 0);
+                            }
+                            umma_commit(smem_u32(&empty[stage]));
+                            if (++stage == S) {
+                                stage = 0;
+                                phase ^= 1u;
+                            }
+                        }
+                        if (!ok) break;
                     }
-                    if (!ok) break;
                     umma_commit(smem_u32(&tfull[acc]));
                     acc ^= 1;
                     if (acc == 0) acc_phase ^= 1u;
@@ -523,6 +570,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         constexpr int kPer = kEpiCols / 32;
         float cn_next[kPer];
         auto cn_of = [&](int j) {
+            if (kPer == 4 && j + 4 <= k) {  // (j is a multiple of 4: one 16-byte load)
+                const float4 v = *reinterpret_cast<const float4*>(cn + j);
+                cn_next[0] = v.x;
+                cn_next[1 % kPer] = v.y;
+                cn_next[2 % kPer] = v.z;
+                cn_next[3 % kPer] = v.w;
+                return;
+            }
 #pragma unroll
             for (int i = 0; i < kPer; ++i) cn_next[i] = j + i < k ? cn[j + i] : __int_as_float(0x7f800000);
         };
