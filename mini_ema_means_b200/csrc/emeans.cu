@@ -238,6 +238,23 @@ static int make_tmap(CUtensorMap* tm, const void* base, int64_t rows, int d, int
     return EM_OK;
 }
 
+// 2-D tensor map over `rows` rows of 16 bf16 values (32-byte rows, the 32-byte
+// swizzle), boxes of box_rows rows: the folded search's norms and ones operands.
+static int make_tmap_ext(CUtensorMap* tm, const void* base, int64_t rows, int box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return fail(EM_E_CUDA, "cuTensorMapEncodeTiled is not available");
+    if ((reinterpret_cast<uintptr_t>(base) & 15) != 0) return fail(EM_E_INVAL, "tensor base not 16-byte aligned");
+    cuuint64_t dims[2] = {(cuuint64_t)tc::kExtK, (cuuint64_t)std::max<int64_t>(rows, 1)};
+    cuuint64_t strides[1] = {(cuuint64_t)tc::kExtK * 2};
+    cuuint32_t box[2] = {(cuuint32_t)tc::kExtK, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(EM_E_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return EM_OK;
+}
+
 // 2-D tensor map over `rows` rows of d E4M3 codes (row pitch ld8 bytes), boxes of
 // 128 codes (128 bytes, the 128-byte swizzle) x box_rows; columns past d read as 0.
 static int make_tmap8(CUtensorMap* tm, const void* base, int64_t rows, int d, int ld8, int box_rows) {
@@ -335,6 +352,7 @@ struct em_model {
     // state
     DBuf<float> N, N_prev, S, c, cn, cnp;
     DBuf<__nv_bfloat16> cq;
+    DBuf<__nv_bfloat16> cn3, ones3;  // the folded search's norms (k x 16) and ones (128 x 16) operands
     DBuf<double> close_sum, close_cnt;
     DBuf<int> err, flag;
     // data of the current run
@@ -386,6 +404,7 @@ struct em_model {
     double last_alpha = 0.0;
     int last_was_lloyd = 0;
     CUtensorMap tm_cq;
+    CUtensorMap tm_cn3, tm_ones3;
     // profiling (EM_OPT_PROFILE) and launch counting
     int profile = 0;
     int64_t launches = 0;
@@ -641,49 +660,69 @@ static bool ast_fits(int64_t d, int kc) {
     return nkc * tc::BM * kc * 2 <= tc::kAstBufBytes;
 }
 
+// Whether the folded-norm search fits: with its norms tile beside the nkc chunks, a
+// centroid tile must still leave two stages in the ring.
+static bool fold_fits(int kc, int nkc) {
+    const int ring = kc == 64 ? tc::Cfg<64, true, 2, true>::kStages * tc::Cfg<64, true, 2, true>::kBBytes
+                              : tc::Cfg<32, true, 2, true>::kStages * tc::Cfg<32, true, 2, true>::kBBytes;
+    const int tile = nkc * tc::BN * kc * 2 + tc::kExtBBytes;
+    return ring / tile >= 2;
+}
+
+// tmN / tmO: the norms and ones operands of the folded search (fold), else unused.
 static void launch_search(int kc, bool top2, bool ast, int grid, cudaStream_t stream, const CUtensorMap& tmA,
                           const CUtensorMap& tmB, const float* cn, int k, int rows, int nkc, int n_tiles, Schedule sc,
-                          unsigned long long* keys, long long wait, int* err, bool f8 = false, bool pdl = false) {
+                          unsigned long long* keys, long long wait, int* err, bool f8 = false, bool pdl = false,
+                          bool fold = false, const CUtensorMap* tmN = nullptr, const CUtensorMap* tmO = nullptr) {
     const int split = sc.split, m_full = sc.m_full;
-#define EM_GO(KC, T2, AST)                                                                                 \
-    launch_k(pdl, tc::k_assign_tc<KC, T2, AST>, grid, tc::kThreads, tc::Cfg<KC, AST>::kSmemBytes, stream, tmA, \
-             tmB, cn, k, rows, nkc, n_tiles, split, m_full, keys, wait, err)
+    const CUtensorMap& tn = tmN ? *tmN : tmB;
+    const CUtensorMap& to = tmO ? *tmO : tmB;
+#define EM_GO(KC, T2, AST, FD)                                                                              \
+    launch_k(pdl, tc::k_assign_tc<KC, T2, AST, false, FD>, grid, tc::threads_for<tc::epi_groups<T2, AST>()>(), \
+             tc::Cfg<KC, AST, tc::epi_groups<T2, AST>(), FD>::kSmemBytes, stream, tmA, tmB, tn, to, cn, k, rows, \
+             nkc, n_tiles, split, m_full, keys, wait, err)
     if (f8) {  // E4M3 rows and operand, 128-code chunks, plain argmin
         if (ast)
-            launch_k(pdl, tc::k_assign_tc<64, false, true, true>, grid, tc::kThreads, tc::Cfg<64, true>::kSmemBytes,
-                     stream, tmA, tmB, cn, k, rows, nkc, n_tiles, split, m_full, keys, wait, err);
+            launch_k(pdl, tc::k_assign_tc<64, false, true, true>, grid, tc::threads_for<tc::epi_groups<false, true>()>(),
+                     tc::Cfg<64, true, tc::epi_groups<false, true>()>::kSmemBytes, stream, tmA, tmB, tn, to, cn, k, rows,
+                     nkc, n_tiles, split, m_full, keys, wait, err);
         else
             launch_k(pdl, tc::k_assign_tc<64, false, false, true>, grid, tc::kThreads, tc::Cfg<64, false>::kSmemBytes,
-                     stream, tmA, tmB, cn, k, rows, nkc, n_tiles, split, m_full, keys, wait, err);
+                     stream, tmA, tmB, tn, to, cn, k, rows, nkc, n_tiles, split, m_full, keys, wait, err);
         return;
     }
     if (kc == 64) {
         if (top2) {
-            if (ast) EM_GO(64, true, true); else EM_GO(64, true, false);
+            if (ast) EM_GO(64, true, true, false); else EM_GO(64, true, false, false);
         } else {
-            if (ast) EM_GO(64, false, true); else EM_GO(64, false, false);
+            if (ast && fold) EM_GO(64, false, true, true);
+            else if (ast) EM_GO(64, false, true, false);
+            else EM_GO(64, false, false, false);
         }
     } else {
         if (top2) {
-            if (ast) EM_GO(32, true, true); else EM_GO(32, true, false);
+            if (ast) EM_GO(32, true, true, false); else EM_GO(32, true, false, false);
         } else {
-            if (ast) EM_GO(32, false, true); else EM_GO(32, false, false);
+            if (ast && fold) EM_GO(32, false, true, true);
+            else if (ast) EM_GO(32, false, true, false);
+            else EM_GO(32, false, false, false);
         }
     }
 #undef EM_GO
 }
 
 static bool search_smem_attributes() {
-#define EM_ATTR(KC, T2, AST)                                                                                \
-    (cudaFuncSetAttribute(tc::k_assign_tc<KC, T2, AST>, cudaFuncAttributeMaxDynamicSharedMemorySize,       \
-                          tc::Cfg<KC, AST>::kSmemBytes) == cudaSuccess)
-    return EM_ATTR(64, false, false) && EM_ATTR(64, true, false) && EM_ATTR(32, false, false) &&
-           EM_ATTR(32, true, false) && EM_ATTR(64, false, true) && EM_ATTR(64, true, true) &&
-           EM_ATTR(32, false, true) && EM_ATTR(32, true, true) &&
+#define EM_ATTR(KC, T2, AST, FD)                                                                            \
+    (cudaFuncSetAttribute(tc::k_assign_tc<KC, T2, AST, false, FD>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                          tc::Cfg<KC, AST, tc::epi_groups<T2, AST>(), FD>::kSmemBytes) == cudaSuccess)
+    return EM_ATTR(64, false, false, false) && EM_ATTR(64, true, false, false) && EM_ATTR(32, false, false, false) &&
+           EM_ATTR(32, true, false, false) && EM_ATTR(64, false, true, false) && EM_ATTR(64, true, true, false) &&
+           EM_ATTR(32, false, true, false) && EM_ATTR(32, true, true, false) && EM_ATTR(64, false, true, true) &&
+           EM_ATTR(32, false, true, true) &&
            cudaFuncSetAttribute(tc::k_assign_tc<64, false, false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 tc::Cfg<64, false>::kSmemBytes) == cudaSuccess &&
            cudaFuncSetAttribute(tc::k_assign_tc<64, false, true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                tc::Cfg<64, true>::kSmemBytes) == cudaSuccess;
+                                tc::Cfg<64, true, tc::epi_groups<false, true>()>::kSmemBytes) == cudaSuccess;
 #undef EM_ATTR
 }
 
@@ -712,8 +751,19 @@ static int launch_assign(em_model* m, const CUtensorMap& tmA, const __nv_bfloat1
                       (int)n_tiles, sc, m->keys.p, m->wait_cycles, m->err.p, true, m->pdl != 0);
     } else {
         const int nkc = (int)((m->d + m->kc - 1) / m->kc);
-        launch_search(m->kc, use_top2(m), ast_fits(m->d, m->kc), grid, m->stream, tmA, m->tm_cq, m->cn.p, (int)m->k,
-                      (int)rows, nkc, (int)n_tiles, sc, m->keys.p, m->wait_cycles, m->err.p, false, m->pdl != 0);
+        const bool top2 = use_top2(m), ast = ast_fits(m->d, m->kc);
+        // the folded search takes |c~|^2 from the MMAs: its norms operand is refreshed first
+        // (one more launch, so only where the tiles are many enough for the epilogue to
+        // matter)
+        const bool fold = ast && !top2 && fold_fits(m->kc, nkc) && n_tiles >= 4 && m_tiles * n_tiles >= 4 * m->sms;
+        if (fold) {
+            launch_k(m->pdl, tc::k_fold_norms, grid_for(n_tiles * tc::BN, 256, m->sms), 256, 0, m->stream, m->cn.p,
+                     (int)m->k, (int)(n_tiles * tc::BN), m->cn3.p);
+            EM_LAUNCHED(m, 1);
+        }
+        launch_search(m->kc, top2, ast, grid, m->stream, tmA, m->tm_cq, m->cn.p, (int)m->k, (int)rows, nkc,
+                      (int)n_tiles, sc, m->keys.p, m->wait_cycles, m->err.p, false, m->pdl != 0, fold, &m->tm_cn3,
+                      &m->tm_ones3);
     }
     CK(cudaGetLastError());
     EM_LAUNCHED(m, 1);
@@ -1393,6 +1443,23 @@ em_model* em_create(int64_t d, int64_t k, uint64_t seed) {
         em_destroy(m);
         return nullptr;
     }
+    {  // the folded search's operands: each batch row's (1, 1, 1, 0, ...), and the norms tiles
+        std::vector<__nv_bfloat16> ones((size_t)tc::BM * tc::kExtK, __float2bfloat16(0.0f));
+        for (int r = 0; r < tc::BM; ++r)
+            for (int e = 0; e < 3; ++e) ones[(size_t)r * tc::kExtK + e] = __float2bfloat16(1.0f);
+        // (the norms operand covers whole centroid tiles: rows past k hold +inf)
+        const int64_t k_pad = (k + tc::BN - 1) / tc::BN * tc::BN;
+        if (m->cn3.ensure((size_t)k_pad * tc::kExtK) || m->ones3.ensure((size_t)tc::BM * tc::kExtK))
+            return bail(EM_E_NOMEM, "device allocation failed");
+        cudaMemset(m->cn3.p, 0, (size_t)k_pad * tc::kExtK * sizeof(__nv_bfloat16));
+        if (cudaMemcpy(m->ones3.p, ones.data(), ones.size() * sizeof(__nv_bfloat16), cudaMemcpyHostToDevice) !=
+                cudaSuccess ||
+            make_tmap_ext(&m->tm_cn3, m->cn3.p, k_pad, tc::BN) != EM_OK ||
+            make_tmap_ext(&m->tm_ones3, m->ones3.p, tc::BM, tc::BM) != EM_OK) {
+            em_destroy(m);
+            return nullptr;
+        }
+    }
     if (cudaDeviceSynchronize() != cudaSuccess) return bail(EM_E_CUDA, "device initialisation failed");
     return m;
 }
@@ -1403,6 +1470,8 @@ void em_destroy(em_model* m) {
     if (m->stream) cudaStreamSynchronize(m->stream);
     m->N.release(); m->N_prev.release(); m->cnp.release(); m->S.release(); m->c.release(); m->cn.release();
     m->cq.release();
+    m->cn3.release();
+    m->ones3.release();
     m->close_sum.release(); m->close_cnt.release(); m->err.release(); m->flag.release();
     if (m->side) cudaStreamSynchronize(m->side);
     for (auto& b : m->slot) {

@@ -42,6 +42,17 @@ constexpr int BN = 256;
 constexpr int kEpiWarps = 8;
 constexpr int kEpiThreads = 32 * kEpiWarps;
 constexpr int kThreads = 64 + kEpiThreads;
+
+// Epilogue groups. With the batch tile stationary and a plain argmin (rows of at
+// most 128 dims) a tile holds little tensor work (six K = 16 MMAs at d = 96), and
+// one group of eight warps scanning every tile would keep the tensor pipe waiting.
+// There two groups take the two accumulators in turn, so that each has the time of
+// two tiles for the epilogue of one; at the end of a unit the second group hands
+// its rows' best to the first through shared memory, and the first writes the keys.
+template <bool TOP2, bool AST>
+__host__ __device__ constexpr int epi_groups() { return (AST && !TOP2) ? 2 : 1; }
+template <int G>
+__host__ __device__ constexpr int threads_for() { return 64 + kEpiThreads * G; }
 constexpr int kKeySets = kEpiWarps / 4;  // key sets per centroid-tile group (the two column halves)
 constexpr int kEpiCols = BN / kKeySets;  // columns of a tile per epilogue warp
 static_assert(kEpiCols % 64 == 0, "the epilogue scans pairs of 32-column chunks");
@@ -52,20 +63,36 @@ static_assert(kEpiCols % 64 == 0, "the epilogue scans pairs of 32-column chunks"
 // through the ring: a third less traffic from L2 per tile.
 constexpr int kAstBufBytes = 32 * 1024;  // one A-stationary buffer: nkc * BM * KC * 2 bytes at most
 
-template <int KC, bool AST = false>
+// FOLD (with the batch tile stationary and a plain argmin): |c~|^2 enters the MMAs
+// as one more K = 16 step, ones(128 x 16) x norms(256 x 16), where each centroid's
+// row of the norms operand is (h, m, l, 0, ...) with h + m + l = |c~|^2 exactly (the
+// fp32 value split into three bf16 parts) and each batch row's is (1, 1, 1, 0, ...).
+// The accumulator then holds the score itself, and the epilogue adds nothing. Both
+// extension tiles are 16 wide (32-byte rows, the 32-byte swizzle).
+constexpr int kExtK = 16;
+constexpr int kExtABytes = BM * kExtK * 2;  // the ones tile, loaded once per CTA
+constexpr int kExtBBytes = BN * kExtK * 2;  // a centroid tile's norms, with its chunks
+constexpr uint64_t kExtLayout = 6ull;       // UMMA 32B swizzle
+constexpr uint32_t kExtSBO = 8u * kExtK * 2u;
+
+template <int KC, bool AST = false, int G = 1, bool FOLD = false>
 struct Cfg {
     static constexpr int kABytes = BM * KC * 2;
     static constexpr int kBBytes = BN * KC * 2;
     static constexpr int kStageBytes = AST ? kBBytes : kABytes + kBBytes;
     // (A stationary: 9 stages of 16 KB or 4 of 32 KB fit beside the two A buffers)
     static constexpr int kStages = AST ? (KC == 32 ? 9 : 4) : (KC == 64 ? 4 : 8);
-    static constexpr int kAreaBytes = AST ? 2 * kAstBufBytes : 0;  // the A buffers, after the ring
+    static constexpr int kAreaBytes = AST ? 2 * kAstBufBytes + (FOLD ? kExtABytes : 0) : 0;  // A buffers
     static constexpr uint64_t kLayout = KC == 64 ? 2ull : 4ull;  // UMMA 128B / 64B swizzle
     static constexpr uint32_t kSBO = 8u * KC * 2u;                // bytes between 8-row groups
     static constexpr int kBarBytes = 256;
-    // + each epilogue warp's |c|^2 values of two tiles (its 128 columns)
+    // two groups: per warp pair and unit parity 32 (best, index) pairs, and a full
+    // and an empty barrier
+    static constexpr int kMergeBytes = G == 2 ? 8 * 2 * 32 * 8 + 8 * 2 * 2 * 8 : 0;
+    // + the epilogue warps' |c|^2 values: two tiles of 128 columns per warp (one
+    // group) or one (two groups), then the merge area
     static constexpr int kSmemBytes =
-        1024 + kStages * kStageBytes + kAreaBytes + kBarBytes + kEpiWarps * 2 * kEpiCols * 4;
+        1024 + kStages * kStageBytes + kAreaBytes + kBarBytes + kEpiWarps * 2 * kEpiCols * 4 + kMergeBytes;
 };
 
 // Instruction descriptor of tcgen05.mma kind::f16: fp32 accumulate (bits 4-5 = 1),
@@ -234,14 +261,16 @@ __device__ __forceinline__ float min3_f32(float a, float b, float c) {
     return d;
 }
 
-template <bool TOP2>
+template <bool TOP2, bool ADD = true>
 __device__ __forceinline__ void scan_chunk(uint32_t (&v)[32], const float4* c4, int jb, float& best, int& bidx,
                                            float& best2, int& bidx2) {
+    if (ADD) {  // (without: the norms are already in the accumulator)
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const float4 cc = c4[i];
-        add2_f32(v[4 * i + 0], v[4 * i + 1], cc.x, cc.y);
-        add2_f32(v[4 * i + 2], v[4 * i + 3], cc.z, cc.w);
+        for (int i = 0; i < 8; ++i) {
+            const float4 cc = c4[i];
+            add2_f32(v[4 * i + 0], v[4 * i + 1], cc.x, cc.y);
+            add2_f32(v[4 * i + 2], v[4 * i + 3], cc.z, cc.w);
+        }
     }
     if (TOP2) {
 #pragma unroll
@@ -321,12 +350,15 @@ __device__ __forceinline__ Unit unit_of(int u, int m_full, int n_split, int tpg,
 
 // F8: the batch rows and the centroid operand are E4M3 codes (KC = 64 only: row
 // chunks of 128 bytes = 128 codes).
-template <int KC, bool TOP2, bool AST, bool F8 = false>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int KC, bool TOP2, bool AST, bool F8 = false, bool FOLD = false>
+__global__ void __launch_bounds__(threads_for<epi_groups<TOP2, AST>()>(), 1)
     k_assign_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                const __grid_constant__ CUtensorMap tmN, const __grid_constant__ CUtensorMap tmO,
                 const float* __restrict__ cn, int k, int rows, int nkc, int n_tiles, int n_split, int m_full,
                 unsigned long long* __restrict__ keys, long long wait_limit, int* err) {
-    using C = Cfg<KC, AST>;
+    constexpr int G = epi_groups<TOP2, AST>();
+    static_assert(!FOLD || (AST && !TOP2 && !F8), "the folded norms need the stationary batch tile and bf16");
+    using C = Cfg<KC, AST, G, FOLD>;
     constexpr int S = C::kStages;
     static_assert(!F8 || KC == 64, "E4M3 rows use 128-byte chunks");
     constexpr int KX = F8 ? 2 * KC : KC;  // elements per row chunk (the TMA x step)
@@ -344,9 +376,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t* drain = bars + 2 * S + 4;
     uint64_t* afull = bars + 2 * S + 5;   // AST: A buffer loaded
     uint64_t* aempty = bars + 2 * S + 7;  // AST: A buffer no longer read by the MMAs
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 9);
+    uint64_t* xbar = bars + 2 * S + 9;    // FOLD: the ones tile loaded
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 10);
+    uint8_t* sOnes = sArea + 2 * kAstBufBytes;  // FOLD: the ones tile (1024-aligned, after the A buffers)
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     float* cn_s = reinterpret_cast<float*>(smem + S * C::kStageBytes + C::kAreaBytes + C::kBarBytes);
+    // (two groups) merge slots [warp pair][unit parity][lane], then their barriers
+    float2* mslot = reinterpret_cast<float2*>(cn_s + kEpiWarps * 2 * kEpiCols);
+    uint64_t* mfull = reinterpret_cast<uint64_t*>(mslot + 8 * 2 * 32);
+    uint64_t* mempty = mfull + 16;
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -357,7 +395,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int units = m_full + (m_tiles - m_full) * n_split;
     // ring stages in use: chunk stages, or (A stationary) whole centroid tiles of nkc
     // chunks each, so that a tile costs one barrier round trip instead of nkc
-    const int st_n = AST ? S / nkc : S;
+    // a tile's bytes in the ring (A stationary: its nkc chunks, and with FOLD its norms)
+    const int tile_bytes = nkc * C::kBBytes + (FOLD ? kExtBBytes : 0);
+    const int st_n = AST ? (S * C::kBBytes) / tile_bytes : S;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
@@ -369,10 +409,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(smem_u32(&tempty[a]), kEpiThreads);
         }
         mbar_init(smem_u32(drain), 1);
+        mbar_init(smem_u32(xbar), 1);
         for (int a = 0; a < 2; ++a) {
             mbar_init(smem_u32(&afull[a]), 1);
             mbar_init(smem_u32(&aempty[a]), 1);
         }
+        if (G == 2)
+            for (int i = 0; i < 16; ++i) {
+                mbar_init(smem_u32(&mfull[i]), 32);
+                mbar_init(smem_u32(&mempty[i]), 32);
+            }
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -403,6 +449,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t armed = 0, armed_parity = 0;  // per-stage bit masks
             uint32_t aarmed = 0, aarmed_parity = 0;  // the two A buffers (AST)
             int ua = 0;                              // units started (AST)
+            if (FOLD && (int)blockIdx.x < units) {  // the ones tile, once
+                mbar_expect_tx(smem_u32(xbar), (uint32_t)kExtABytes);
+                tma_load_2d(smem_u32(sOnes), &tmO, 0, 0, smem_u32(xbar));
+            }
             for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
                 const Unit w = unit_of(u, m_full, n_split, tpg, n_tiles);
                 const int m = w.m, nt0 = w.nt0, nt1 = w.nt1;
@@ -430,9 +480,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const uint32_t fb = smem_u32(&full[stage]);
                         armed |= 1u << stage;
                         armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
-                        mbar_expect_tx(fb, (uint32_t)(nkc * C::kBBytes));
+                        mbar_expect_tx(fb, (uint32_t)tile_bytes);
+                        uint8_t* tb = sB + stage * tile_bytes;
                         for (int kc = 0; kc < nkc; ++kc)
-                            tma_load_2d(smem_u32(sB + (stage * nkc + kc) * C::kBBytes), &tmB, kc * KX, nt * BN, fb);
+                            tma_load_2d(smem_u32(tb + kc * C::kBBytes), &tmB, kc * KX, nt * BN, fb);
+                        if (FOLD) tma_load_2d(smem_u32(tb + nkc * C::kBBytes), &tmN, 0, nt * BN, fb);
                         if (++stage == st_n) {
                             stage = 0;
                             phase ^= 1u;
@@ -462,6 +514,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (armed & (1u << s2)) mbar_drain(smem_u32(&full[s2]), (armed_parity >> s2) & 1u, drain_limit);
                 for (int a2 = 0; a2 < 2; ++a2)
                     if (aarmed & (1u << a2)) mbar_drain(smem_u32(&afull[a2]), (aarmed_parity >> a2) & 1u, drain_limit);
+                if (FOLD && (int)blockIdx.x < units) mbar_drain(smem_u32(xbar), 0u, drain_limit);
             }
         }
     } else if (warp == 1) {
@@ -473,6 +526,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t acc_phase = 0;
             bool ok = true;
             int ua = 0;
+            if (FOLD && (int)blockIdx.x < units) {
+                ok = mbar_wait(smem_u32(xbar), 0u, wait_limit, err, abort_flag);
+                tc_fence_after();
+            }
             for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
                 const Unit w = unit_of(u, m_full, n_split, tpg, n_tiles);
                 const int nt0 = w.nt0, nt1 = w.nt1;
@@ -497,9 +554,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                             break;
                         }
                         tc_fence_after();
+                        uint8_t* tb = sB + stage * tile_bytes;
                         for (int kc = 0; kc < nkc; ++kc) {
                             const uint32_t a0 = smem_u32(sArea + ab * kAstBufBytes + kc * C::kABytes);
-                            const uint32_t b0 = smem_u32(sB + (stage * nkc + kc) * C::kBBytes);
+                            const uint32_t b0 = smem_u32(tb + kc * C::kBBytes);
 #pragma unroll
                             for (int kk = 0; kk < KC / 16; ++kk) {
                                 const uint64_t ad = smem_desc(a0 + kk * 32, C::kLayout, C::kSBO);
@@ -510,6 +568,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                                     umma_bf16(d_tmem, ad, bd, (kc | kk) != 0);
                             }
                         }
+                        if (FOLD)  // + (1, 1, 1) . (h, m, l) = |c~|^2 on every row
+                            umma_bf16(d_tmem, smem_desc(smem_u32(sOnes), kExtLayout, kExtSBO),
+                                      smem_desc(smem_u32(tb + nkc * C::kBBytes), kExtLayout, kExtSBO), 1u);
                         umma_commit(smem_u32(&empty[stage]));
                         if (++stage == st_n) {
                             stage = 0;
@@ -556,15 +617,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
     } else {
-        // ---------------- epilogue: 8 warps, thread = accumulator row, warp = column half
+        // ---------------- epilogue: 8 G warps, thread = accumulator row, warp = column half
+        const int ew = warp - 2;
+        const int grp = G == 2 ? ew >> 3 : 0;  // the accumulator this warp's group takes (G = 2)
+        const int wi = ew & 7;                 // the warp's place in its group
         const int q = warp & 3;
-        const int half = (warp - 2) >> 2;  // column part of the tile
+        const int half = wi >> 2;          // column part of the tile
         const int rl = 32 * q + lane;      // row within the tile
         const uint32_t lane_base = (uint32_t)(32 * q) << 16;
-        float* cn_w = cn_s + (warp - 2) * 2 * kEpiCols;  // this warp's two |c|^2 buffers
+        float* cn_w = cn_s + ew * (2 / G) * kEpiCols;  // this warp's |c|^2 buffers (two, or one)
         int acc = 0;
         uint32_t acc_phase = 0;
         int cnbuf = 0;
+        int uc = 0;  // units done (the merge slots alternate)
         bool ok = true;
         // this lane's |c|^2 values of the next tile the warp handles, one tile ahead
         constexpr int kPer = kEpiCols / 32;
@@ -581,10 +646,23 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int i = 0; i < kPer; ++i) cn_next[i] = j + i < k ? cn[j + i] : __int_as_float(0x7f800000);
         };
+        // the tile after (u2, nt2) in this CTA's sequence (u2 >= units: none)
+        auto step_tile = [&](int& u2, int& nt2) {
+            if (nt2 + 1 < unit_of(u2, m_full, n_split, tpg, n_tiles).nt1) {
+                ++nt2;
+                return;
+            }
+            u2 += gridDim.x;
+            if (u2 < units) nt2 = unit_of(u2, m_full, n_split, tpg, n_tiles).nt0;
+        };
 #pragma unroll
         for (int i = 0; i < kPer; ++i) cn_next[i] = 0.0f;
-        if (blockIdx.x < units)
-            cn_of(unit_of(blockIdx.x, m_full, n_split, tpg, n_tiles).nt0 * BN + half * kEpiCols + kPer * lane);
+        if (!FOLD) {  // the first tile of this warp: the first of the sequence, or of its accumulator
+            int u2 = blockIdx.x, nt2 = 0;
+            if (u2 < units) nt2 = unit_of(u2, m_full, n_split, tpg, n_tiles).nt0;
+            for (int i = 0; i < grp && u2 < units; ++i) step_tile(u2, nt2);
+            if (u2 < units) cn_of(nt2 * BN + half * kEpiCols + kPer * lane);
+        }
         for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
             const Unit w = unit_of(u, m_full, n_split, tpg, n_tiles);
             const int m = w.m, g = w.g, nt0 = w.nt0, nt1 = w.nt1;
@@ -592,58 +670,93 @@ __global__ void __launch_bounds__(kThreads, 1)
             float best2 = best;
             int bidx = 0, bidx2 = 0;
             for (int nt = nt0; nt < nt1; ++nt) {
-                float* cnb = cn_w + cnbuf * kEpiCols;
-                const int j0 = nt * BN;
+                if (G == 1 || acc == grp) {
+                    float* cnb = cn_w + cnbuf * kEpiCols;
+                    const int j0 = nt * BN;
+                    if (!FOLD) {
+                        if (G == 2) __syncwarp();  // (one buffer) every lane is done with the last tile's
 #pragma unroll
-                for (int i = 0; i < kPer; ++i) cnb[kPer * lane + i] = cn_next[i];
-                {
-                    int jn = -1;
-                    if (nt + 1 < nt1) {
-                        jn = (nt + 1) * BN;
-                    } else if (u + (int)gridDim.x < units) {
-                        jn = unit_of(u + (int)gridDim.x, m_full, n_split, tpg, n_tiles).nt0 * BN;
+                        for (int i = 0; i < kPer; ++i) cnb[kPer * lane + i] = cn_next[i];
                     }
-                    if (jn >= 0) cn_of(jn + half * kEpiCols + kPer * lane);
-                }
-                // the whole warp takes one decision (a lane that gave up takes the warp with it)
-                const bool got = __all_sync(0xFFFFFFFFu,
-                                            mbar_wait(smem_u32(&tfull[acc]), acc_phase, wait_limit, err, abort_flag));
-                if (!got) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                __syncwarp();  // also publishes this warp's |c|^2 values
-                const uint32_t tbase = tmem_base + lane_base + (uint32_t)(acc * BN + half * kEpiCols);
-                const float4* c4 = reinterpret_cast<const float4*>(cnb);
-                const int jh = j0 + half * kEpiCols;
-                // chunks of 32 columns, the load of the next in flight while one is
-                // scanned; the accumulator goes back once the last chunk is in registers
-                {
-                    constexpr int kChunks = kEpiCols / 32;
-                    uint32_t va[32], vb[32];
-                    tmem_ld32(tbase, va);
-                    tmem_wait_ld32(va);
-#pragma unroll
-                    for (int c = 0; c < kChunks; c += 2) {
-                        tmem_ld32(tbase + 32 * (c + 1), vb);
-                        scan_chunk<TOP2>(va, c4 + 8 * c, jh + 32 * c, best, bidx, best2, bidx2);
-                        tmem_wait_ld32(vb);
-                        if (c + 2 < kChunks) {
-                            tmem_ld32(tbase + 32 * (c + 2), va);
+                    if (!FOLD) {  // the warp's next tile, G tiles on
+                        int u2 = u, nt2 = nt;
+                        if (nt + G < nt1) {
+                            nt2 = nt + G;
                         } else {
-                            tc_fence_before();
-                            mbar_arrive(smem_u32(&tempty[acc]));
+                            for (int i = 0; i < G && u2 < units; ++i) step_tile(u2, nt2);
                         }
-                        scan_chunk<TOP2>(vb, c4 + 8 * (c + 1), jh + 32 * (c + 1), best, bidx, best2, bidx2);
-                        if (c + 2 < kChunks) tmem_wait_ld32(va);
+                        if (u2 < units) cn_of(nt2 * BN + half * kEpiCols + kPer * lane);
                     }
+                    // the whole warp takes one decision (a lane that gave up takes the warp with it)
+                    const bool got = __all_sync(
+                        0xFFFFFFFFu, mbar_wait(smem_u32(&tfull[acc]), acc_phase, wait_limit, err, abort_flag));
+                    if (!got) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    __syncwarp();  // also publishes this warp's |c|^2 values
+                    const uint32_t tbase = tmem_base + lane_base + (uint32_t)(acc * BN + half * kEpiCols);
+                    const float4* c4 = reinterpret_cast<const float4*>(cnb);
+                    const int jh = j0 + half * kEpiCols;
+                    // chunks of 32 columns, the load of the next in flight while one is
+                    // scanned; the accumulator goes back once the last chunk is in registers
+                    {
+                        constexpr int kChunks = kEpiCols / 32;
+                        uint32_t va[32], vb[32];
+                        tmem_ld32(tbase, va);
+                        tmem_wait_ld32(va);
+#pragma unroll
+                        for (int c = 0; c < kChunks; c += 2) {
+                            tmem_ld32(tbase + 32 * (c + 1), vb);
+                            scan_chunk<TOP2, !FOLD>(va, c4 + 8 * c, jh + 32 * c, best, bidx, best2, bidx2);
+                            tmem_wait_ld32(vb);
+                            if (c + 2 < kChunks) {
+                                tmem_ld32(tbase + 32 * (c + 2), va);
+                            } else {
+                                tc_fence_before();
+                                mbar_arrive(smem_u32(&tempty[acc]));
+                            }
+                            scan_chunk<TOP2, !FOLD>(vb, c4 + 8 * (c + 1), jh + 32 * (c + 1), best, bidx, best2, bidx2);
+                            if (c + 2 < kChunks) tmem_wait_ld32(va);
+                        }
+                    }
+                    if (G == 1) cnbuf ^= 1;
                 }
                 acc ^= 1;
                 if (acc == 0) acc_phase ^= 1u;
-                cnbuf ^= 1;
             }
             if (!ok) break;
+            if (G == 2) {
+                // the second group hands its rows' best of this unit to the first
+                const int slot = wi * 2 + (uc & 1);
+                const uint32_t par = (uint32_t)(uc >> 1) & 1u;
+                ++uc;
+                if (grp == 1) {
+                    const bool free_slot = __all_sync(
+                        0xFFFFFFFFu, mbar_wait(smem_u32(&mempty[slot]), par ^ 1u, wait_limit, err, abort_flag));
+                    if (!free_slot) {
+                        ok = false;
+                        break;
+                    }
+                    mslot[slot * 32 + lane] = make_float2(best, __int_as_float(bidx));
+                    mbar_arrive(smem_u32(&mfull[slot]));
+                    continue;
+                }
+                const bool arrived = __all_sync(
+                    0xFFFFFFFFu, mbar_wait(smem_u32(&mfull[slot]), par, wait_limit, err, abort_flag));
+                if (!arrived) {
+                    ok = false;
+                    break;
+                }
+                const float2 o = mslot[slot * 32 + lane];
+                mbar_arrive(smem_u32(&mempty[slot]));
+                const int oi = __float_as_int(o.y);
+                if (o.x < best || (o.x == best && oi < bidx)) {  // lower score, then lower column
+                    best = o.x;
+                    bidx = oi;
+                }
+            }
             // this column half's key set: (score, index) keys order as the argmin does
             // (lower score, then lower index)
             const int row = m * BM + rl;
@@ -668,6 +781,35 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(512u) : "memory");
     }
+}
+
+// The folded search's norms operand: row j is (h, m, l, 0, ...) in bf16 with
+// h + m + l = |c~_j|^2: h the fp32 value rounded to bf16, m the remainder rounded,
+// l the rest, each remainder exact in fp32 (its operands are within a factor of two
+// of each other), so the three parts carry all 24 bits. A non-finite value goes
+// into h alone. The rows from k to k_pad (the rest of the last centroid tile) hold
+// +inf, so that the tile's missing centroids (zero operand rows) never win.
+__global__ void k_fold_norms(const float* __restrict__ cn, int k, int k_pad, __nv_bfloat16* __restrict__ cn3) {
+    pdl_wait();
+    pdl_release();
+    const int j = blockIdx.x * blockDim.x + threadIdx.x;
+    if (j >= k_pad) return;
+    const float c = j < k ? cn[j] : __int_as_float(0x7f800000);
+    const __nv_bfloat16 h = __float2bfloat16_rn(c);
+    __nv_bfloat16 mid = __float2bfloat16_rn(0.0f), lo = mid;
+    if (isfinite(c)) {
+        const float r1 = c - __bfloat162float(h);
+        mid = __float2bfloat16_rn(r1);
+        lo = __float2bfloat16_rn(r1 - __bfloat162float(mid));
+    }
+    uint4 v0;
+    v0.x = (uint32_t)__bfloat16_as_ushort(h) | ((uint32_t)__bfloat16_as_ushort(mid) << 16);
+    v0.y = (uint32_t)__bfloat16_as_ushort(lo);
+    v0.z = 0u;
+    v0.w = 0u;
+    uint4* row = reinterpret_cast<uint4*>(cn3 + (int64_t)j * kExtK);
+    row[0] = v0;
+    row[1] = make_uint4(0u, 0u, 0u, 0u);
 }
 
 }  // namespace tc

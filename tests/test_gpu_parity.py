@@ -118,7 +118,11 @@ def test_host_input_goes_through_the_same_path(em):
                                    # more row tiles than SMs: whole row tiles first, the last
                                    # wave's split into centroid-tile groups (on 148 SMs: 296
                                    # whole and 17 split 8 ways; 148 whole and 9 split 2 ways)
-                                   (40000, 32, 2000), (20000, 40, 300), (20000, 256, 512)])
+                                   (40000, 32, 2000), (20000, 40, 300), (20000, 256, 512),
+                                   # the folded search (|c~|^2 as one more K = 16 MMA step) at
+                                   # d <= 96 with many tiles: K chunks of 32 (one, two, three)
+                                   # and of 64, the last centroid tile partly empty
+                                   (30000, 96, 1100), (25000, 40, 2100), (30000, 64, 1500)])
 def test_assign_and_mse_match_oracle(em, n, d, k):
     g = torch.Generator().manual_seed(n * 31 + k)
     x = synth.hand_shape(n, d, 16, seed=n + k)
