@@ -607,9 +607,11 @@ __global__ void __launch_bounds__(kSelectThreads) k_revive_select_flat(CountSour
             const int cnt = min(32, nd - i0);
             const double u_next = i0 + 32 + lane < nd ? sc.target[i0 + 32 + lane] : 0.0;
             int my_dn = -1;
+            double u = __shfl_sync(0xFFFFFFFFu, u_cur, 0);  // this draw's uniform, taken one draw ahead
             for (int q = 0; q < cnt; ++q) {
                 const bool live = W > 0.0;
-                const double tg = __dmul_rn(__shfl_sync(0xFFFFFFFFu, u_cur, q), W);
+                const double tg = __dmul_rn(u, W);
+                u = __shfl_sync(0xFFFFFFFFu, u_cur, (q + 1) & 31);
                 const long long tb = min(dbits(tg), dbits(W) - 1);
                 int g = 0;
 #pragma unroll
