@@ -850,7 +850,11 @@ static bool select_smem_attributes() {
            cudaFuncSetAttribute(k_revive_select_flat<1, 2>, a, b) == cudaSuccess &&
            cudaFuncSetAttribute(k_revive_select_flat<1, 4>, a, b) == cudaSuccess &&
            cudaFuncSetAttribute(k_revive_select_flat<2, 4>, a, b) == cudaSuccess &&
-           cudaFuncSetAttribute(k_revive_select_flat<4, 4>, a, b) == cudaSuccess;
+           cudaFuncSetAttribute(k_revive_select_flat<4, 4>, a, b) == cudaSuccess &&
+           cudaFuncSetAttribute(k_revive_select_wide<1>, a, b) == cudaSuccess &&
+           cudaFuncSetAttribute(k_revive_select_wide<2>, a, b) == cudaSuccess &&
+           cudaFuncSetAttribute(k_revive_select_wide<4>, a, b) == cudaSuccess &&
+           cudaFuncSetAttribute(k_revive_select_wide<8>, a, b) == cudaSuccess;
 }
 
 // The donor selection of the revival check after step t, on `stream`, reading the
@@ -875,6 +879,19 @@ static int launch_select(em_model* m, int64_t t, cudaStream_t stream, bool pdl, 
     else if (k <= kFastK)
         launch_k(pdl, k_revive_select_flat<4, 4>, 1, kSelectThreads, flat_smem_bytes<4>(k), stream, src, k, tau,
                  m->seed, t, m->revival, sc);
+    // level 0 in global memory, prefetched ahead of the draws, up to kWideK
+    else if (k <= kWideK && wide_root_slots(k) == 1)
+        launch_k(pdl, k_revive_select_wide<1>, 1, kSelectThreads, wide_smem_bytes(k), stream, src, k, tau, m->seed,
+                 t, m->revival, sc);
+    else if (k <= kWideK && wide_root_slots(k) == 2)
+        launch_k(pdl, k_revive_select_wide<2>, 1, kSelectThreads, wide_smem_bytes(k), stream, src, k, tau, m->seed,
+                 t, m->revival, sc);
+    else if (k <= kWideK && wide_root_slots(k) == 4)
+        launch_k(pdl, k_revive_select_wide<4>, 1, kSelectThreads, wide_smem_bytes(k), stream, src, k, tau, m->seed,
+                 t, m->revival, sc);
+    else if (k <= kWideK)
+        launch_k(pdl, k_revive_select_wide<8>, 1, kSelectThreads, wide_smem_bytes(k), stream, src, k, tau, m->seed,
+                 t, m->revival, sc);
     else
         launch_k(pdl, k_revive_select, 1, kSelectThreads, (int)tree_smem_bytes(tree_layout(k), k), stream, src, k,
                  tau, m->seed, t, m->revival, sc, m->err.p);

@@ -210,9 +210,11 @@ struct CountSource {
     }
 };
 
-__global__ void __launch_bounds__(kSelectThreads) k_revive_select(CountSource N, int k, double tau, uint64_t seed,
-                                                        int64_t t, int mode, ReviveScratch sc, int* err) {
-    pdl_wait();
+// The selection's common start: the total count (in a fixed order), the dead set in
+// increasing index, its count, and the uniform draw of every dead cluster. Returns
+// false (with the donors and counters written) when no donor is drawn.
+__device__ __forceinline__ bool select_prologue(const CountSource& N, int k, double tau, uint64_t seed, int64_t t,
+                                                int mode, const ReviveScratch& sc, int& nd_out, double& thr_out) {
     __shared__ double red[32];
     __shared__ int32_t wcount[32];
     __shared__ int32_t base_s;
@@ -232,6 +234,7 @@ __global__ void __launch_bounds__(kSelectThreads) k_revive_select(CountSource N,
     const double total = red[0];
     const double mean = total / (double)k;
     const double thr = tau * mean;
+    thr_out = thr;
 
     // dead set, compacted in increasing index
     if (tid == 0) base_s = 0;
@@ -259,15 +262,26 @@ __global__ void __launch_bounds__(kSelectThreads) k_revive_select(CountSource N,
         __syncthreads();
     }
     const int nd = base_s;
+    nd_out = nd;
     if (tid == 0) *sc.ndead = nd;
     if (mode != EM_REVIVE_SPLIT || nd == 0 || !(total > 0.0)) {
         for (int i = tid; i < nd; i += kSelectThreads) sc.donor[i] = -1;
         for (int j = tid; j < k; j += kSelectThreads) sc.times[j] = 0;
-        return;
+        return false;
     }
 
     // draws of every dead cluster, in parallel (they do not depend on each other)
     for (int i = tid; i < nd; i += kSelectThreads) sc.target[i] = draw_uniform(seed, kStreamRevive, t, sc.dead[i]);
+    return true;
+}
+
+__global__ void __launch_bounds__(kSelectThreads) k_revive_select(CountSource N, int k, double tau, uint64_t seed,
+                                                        int64_t t, int mode, ReviveScratch sc, int* err) {
+    pdl_wait();
+    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+    int nd = 0;
+    double thr = 0.0;
+    if (!select_prologue(N, k, tau, seed, t, mode, sc, nd, thr)) return;
 
     extern __shared__ __align__(16) double smem_d[];
     // donor tree for larger k (loops over levels have a fixed trip count so that
@@ -458,16 +472,22 @@ EM_HD int flat_smem_bytes(int k) {
 
 __device__ __forceinline__ long long dbits(double x) { return __double_as_longlong(x); }
 
-// Slot `s` of a lane's N values (N = 1, 2 or 4; any slot when s is out of range),
-// by selects on the bits of s: an index into a register array would move the
-// array to local memory.
+// Slot `s` of a lane's N values (N = 1, 2, 4 or 8; any slot when s is out of
+// range), by selects on the bits of s: an index into a register array would move
+// the array to local memory.
 template <int N>
 __device__ __forceinline__ double pick(const double (&x)[N], int s) {
+    static_assert(N == 1 || N == 2 || N == 4 || N == 8, "1, 2, 4 or 8 slots");
     if (N == 1) return x[0];
-    const double lo = (s & 1) ? x[1 % N] : x[0];
-    if (N == 2) return lo;
-    const double hi = (s & 1) ? x[3 % N] : x[2 % N];
-    return (s & 2) ? hi : lo;
+    const double a = (s & 1) ? x[1 % N] : x[0];
+    if (N == 2) return a;
+    const double b = (s & 1) ? x[3 % N] : x[2 % N];
+    const double lo = (s & 2) ? b : a;
+    if (N == 4) return lo;
+    const double c = (s & 1) ? x[5 % N] : x[4 % N];
+    const double e = (s & 1) ? x[7 % N] : x[6 % N];
+    const double hi = (s & 2) ? e : c;
+    return (s & 4) ? hi : lo;
 }
 
 template <int S0, int SR>
@@ -678,6 +698,224 @@ __global__ void __launch_bounds__(kSelectThreads) k_revive_select_flat(CountSour
     }
     __syncthreads();
     for (int j = tid; j < k; j += kSelectThreads) sc.times[j] = times[j];
+}
+
+// ---- wide tree for kFastK < k <= kWideK: level 0 in global memory, prefetched ahead
+//
+// Level 0 (global memory) holds the inclusive prefix of the weights within groups
+// of 128 clusters, lane l holding positions 32 s + l (s = 0..3); level 1 (shared
+// memory) the inclusive prefix of the level-0 group totals within groups of 32;
+// the root (the drawing warp's registers, SR slots) that of the level-1 group
+// totals. A draw descends as on the two-level tree. The level-0 group it needs
+// is a global load, so each draw also makes the descent of the draw kWideAhead
+// places later on the current tree and starts loading the group that one points
+// at. When that draw comes, its exact descent decides: if it ends in the same
+// group (it nearly always does: the target has moved by a few clusters' weight),
+// the copy is used after the updates made since it was loaded, in their order
+// (each subtracts the same delta from the same positions as the stored values
+// received); else the group is loaded again.
+constexpr int kWideG0 = 128;
+constexpr int kWideAhead = 4;
+constexpr int kWideK = 32 * 8 * 32 * kWideG0;  // with a root of 8 slots per lane
+
+EM_HD int wide_groups0(int k) { return (k + kWideG0 - 1) / kWideG0; }
+EM_HD int wide_groups1(int k) { return (wide_groups0(k) + 31) / 32; }
+EM_HD int wide_smem_bytes(int k) { return wide_groups1(k) * 32 * 8; }
+// root slots per lane for k (1, 2, 4 or 8)
+EM_HD int wide_root_slots(int k) {
+    const int r = (wide_groups1(k) + 31) / 32;
+    return r <= 1 ? 1 : (r <= 2 ? 2 : (r <= 4 ? 4 : 8));
+}
+
+template <int SR>
+__global__ void __launch_bounds__(kSelectThreads) k_revive_select_wide(CountSource N, int k, double tau,
+                                                                      uint64_t seed, int64_t t, int mode,
+                                                                      ReviveScratch sc) {
+    pdl_wait();
+    constexpr int D = kWideAhead;
+    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+    int nd = 0;
+    double thr = 0.0;
+    if (!select_prologue(N, k, tau, seed, t, mode, sc, nd, thr)) return;
+    extern __shared__ __align__(16) double smem_d[];
+    double* L1 = smem_d;
+    double* L0 = sc.tree;
+    int32_t* times = sc.times;
+    const int n0 = wide_groups0(k), n1 = wide_groups1(k);
+    // level 0, one group per warp at a time (the four slots' counts loaded first)
+    for (int g0 = w; g0 < n0; g0 += kSelectWarps) {
+        double wv[4];
+#pragma unroll
+        for (int s = 0; s < 4; ++s) {
+            const int j = g0 * kWideG0 + 32 * s + lane;
+            const float nj = j < k ? N(j) : 0.0f;
+            wv[s] = (j < k && !((double)nj < thr)) ? (double)nj : 0.0;
+        }
+        double carry = 0.0;
+#pragma unroll
+        for (int s = 0; s < 4; ++s) {
+            const double x = warp_incl_scan(wv[s], lane) + carry;
+            carry = __shfl_sync(0xFFFFFFFFu, x, 31);
+            L0[(int64_t)g0 * kWideG0 + 32 * s + lane] = x;
+        }
+        if (lane == 0) L1[g0] = carry;  // the group's total, scanned below
+    }
+    for (int i = n0 + tid; i < n1 * 32; i += kSelectThreads) L1[i] = 0.0;
+    for (int j = tid; j < k; j += kSelectThreads) times[j] = 0;
+    __syncthreads();
+    for (int g1 = w; g1 < n1; g1 += kSelectWarps) L1[g1 * 32 + lane] = warp_incl_scan(L1[g1 * 32 + lane], lane);
+    __syncthreads();  // (also publishes level 0 and the counters to warp 0)
+    if (w != 0) return;
+
+    double T[SR];
+    double carry = 0.0;
+#pragma unroll
+    for (int s = 0; s < SR; ++s) {
+        const int pos = 32 * s + lane;
+        const double x = warp_incl_scan(pos < n1 ? L1[pos * 32 + 31] : 0.0, lane) + carry;
+        carry = __shfl_sync(0xFFFFFFFFu, x, 31);
+        T[s] = pos < n1 ? x : __longlong_as_double(0x7FF0000000000000ll);
+    }
+    double W = carry;
+    // the descent above level 0 for target bits tb, on the current root and level 1
+    auto upper = [&](long long tb, int& g1, double& v1, int& c1, int& g0, double& before0) {
+        int gg = 0;
+#pragma unroll
+        for (int s = 0; s < SR; ++s) gg += __popc(__ballot_sync(0xFFFFFFFFu, dbits(T[s]) <= tb));
+        g1 = min(gg, n1 - 1);
+        const int gp = g1 - 1;
+        double b1 = __shfl_sync(0xFFFFFFFFu, pick<SR>(T, gp >> 5), gp & 31);
+        if (g1 == 0) b1 = 0.0;
+        v1 = L1[g1 * 32 + lane];
+        c1 = min(__popc(__ballot_sync(0xFFFFFFFFu, dbits(__dadd_rn(b1, v1)) <= tb)), 31);
+        const double vp = __shfl_sync(0xFFFFFFFFu, v1, (c1 - 1) & 31);
+        before0 = c1 ? __dadd_rn(b1, vp) : b1;
+        g0 = min(g1 * 32 + c1, n0 - 1);
+    };
+    // prefetched groups: slot i is for the draw i + 1 places on, loaded before the
+    // updates of the draws in between; ug/up/ud: those updates (group, position,
+    // delta), oldest first
+    double sv[D][4];
+    int sg[D], ug[D], up[D];
+    double ud[D];
+#pragma unroll
+    for (int i = 0; i < D; ++i) {
+        sg[i] = -1;
+        ug[i] = -1;
+        up[i] = 0;
+        ud[i] = 0.0;
+#pragma unroll
+        for (int s = 0; s < 4; ++s) sv[i][s] = 0.0;
+    }
+    int64_t splits = 0;
+    double u_cur = lane < nd ? sc.target[lane] : 0.0;
+    for (int i0 = 0; i0 < nd; i0 += 32) {
+        const int cnt = min(32, nd - i0);
+        const double u_next = i0 + 32 + lane < nd ? sc.target[i0 + 32 + lane] : 0.0;
+        int my_dn = -1;
+        double u = __shfl_sync(0xFFFFFFFFu, u_cur, 0);
+        for (int q = 0; q < cnt; ++q) {
+            const bool live = W > 0.0;
+            const double tg = __dmul_rn(u, W);
+            const long long tb = min(dbits(tg), dbits(W) - 1);
+            u = __shfl_sync(0xFFFFFFFFu, u_cur, (q + 1) & 31);
+            // the uniform of the draw D places on (this batch or the next)
+            const int qa = q + D;
+            const double ua = qa < 32 ? __shfl_sync(0xFFFFFFFFu, u_cur, qa & 31)
+                                      : __shfl_sync(0xFFFFFFFFu, u_next, (qa - 32) & 31);
+            const bool ahead = i0 + qa < nd;
+            int g1, c1, g0;
+            double v1, before0;
+            upper(tb, g1, v1, c1, g0, before0);
+            // this draw's level-0 group: the copy loaded D draws ago, brought up to date
+            double v0[4];
+            if (sg[0] == g0) {
+#pragma unroll
+                for (int s = 0; s < 4; ++s) v0[s] = sv[0][s];
+#pragma unroll
+                for (int i = 0; i < D; ++i)
+                    if (ug[i] == g0)
+#pragma unroll
+                        for (int s = 0; s < 4; ++s)
+                            if (32 * s + lane >= up[i]) v0[s] = __dsub_rn(v0[s], ud[i]);
+            } else {
+#pragma unroll
+                for (int s = 0; s < 4; ++s) v0[s] = L0[(int64_t)g0 * kWideG0 + 32 * s + lane];
+            }
+            // the descent of the draw D places on, on the tree as it is now, and its load
+            int ag0 = -1;
+            double av[4] = {0.0, 0.0, 0.0, 0.0};
+            if (ahead) {
+                const double tga = __dmul_rn(ua, W);
+                const long long tba = min(dbits(tga), dbits(W) - 1);
+                int a1, ac1;
+                double av1, ab0;
+                upper(tba, a1, av1, ac1, ag0, ab0);
+#pragma unroll
+                for (int s = 0; s < 4; ++s) av[s] = L0[(int64_t)ag0 * kWideG0 + 32 * s + lane];
+            }
+            // level 0 of this draw
+            int p = 0;
+#pragma unroll
+            for (int s = 0; s < 4; ++s)
+                p += __popc(__ballot_sync(0xFFFFFFFFu, dbits(__dadd_rn(before0, v0[s])) <= tb));
+            p = min(p, kWideG0 - 1);
+            const double va = pick<4>(v0, p >> 5);
+            const double vb = pick<4>(v0, (p - 1) >> 5);
+            const double a = __shfl_sync(0xFFFFFFFFu, va, p & 31);
+            double b = __shfl_sync(0xFFFFFFFFu, vb, (p - 1) & 31);
+            if (p == 0) b = 0.0;
+            const double wt = __dsub_rn(a, b);
+            // the donor keeps the rounded half of its weight (explicit roundings, as above)
+            const double keep = __dmul_rn(0.5, wt);
+            const double delta = live ? __dsub_rn(wt, keep) : 0.0;
+#pragma unroll
+            for (int s = 0; s < 4; ++s)
+                if (32 * s + lane >= p) L0[(int64_t)g0 * kWideG0 + 32 * s + lane] = __dsub_rn(v0[s], delta);
+            if (lane >= c1) L1[g1 * 32 + lane] = __dsub_rn(v1, delta);
+#pragma unroll
+            for (int s = 0; s < SR; ++s)
+                if (32 * s + lane >= g1) T[s] = __dsub_rn(T[s], delta);
+            W = __dsub_rn(W, delta);
+            // the rings move on by one draw
+#pragma unroll
+            for (int i = 0; i + 1 < D; ++i) {
+                sg[i] = sg[i + 1];
+                ug[i] = ug[i + 1];
+                up[i] = up[i + 1];
+                ud[i] = ud[i + 1];
+#pragma unroll
+                for (int s = 0; s < 4; ++s) sv[i][s] = sv[i + 1][s];
+            }
+            sg[D - 1] = ag0;
+            ug[D - 1] = g0;
+            up[D - 1] = p;
+            ud[D - 1] = delta;
+#pragma unroll
+            for (int s = 0; s < 4; ++s) sv[D - 1][s] = av[s];
+            const int d = g0 * kWideG0 + p;
+            if (lane == q) my_dn = live && d < k ? d : -1;
+        }
+        // record the batch: donor, and how many earlier splits took the same donor
+        const bool has = lane < cnt && my_dn >= 0;
+        const unsigned peers = __match_any_sync(0xFFFFFFFFu, has ? my_dn : -1);
+        const int leader = __ffs(peers) - 1;
+        int old = 0;
+        if (has && lane == leader) old = times[my_dn];
+        old = __shfl_sync(0xFFFFFFFFu, old, leader);
+        if (has) {
+            const int rk = __popc(peers & ((1u << lane) - 1u));
+            sc.donor[i0 + lane] = my_dn;
+            sc.order[i0 + lane] = old + rk;
+            if (lane == leader) times[my_dn] = old + __popc(peers);
+        } else if (lane < cnt) {
+            sc.donor[i0 + lane] = -1;
+        }
+        splits += __popc(__ballot_sync(0xFFFFFFFFu, has));
+        __syncwarp();  // the counters written above are read by other lanes next batch
+        u_cur = u_next;
+    }
+    if (lane == 0) *sc.n_splits += splits;
 }
 
 // Dead clusters take their half of the donor (reads the donors' state before

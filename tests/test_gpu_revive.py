@@ -2,9 +2,10 @@
 
 The donor search keeps a tree of prefix sums whose shape depends on k (up to
 16,384 clusters a root of group totals in registers over groups of 32, 64 or 128
-clusters in shared memory, the root holding up to 32, 64 or 128 entries; above
-that radix-128 levels in shared or global memory), so k runs over the boundaries
-of those shapes. Each case sets
+clusters in shared memory, the root holding up to 32, 64 or 128 entries; up to
+1,048,576 a root over a shared-memory level over groups of 128 in global memory,
+prefetched ahead of the draws; above that radix-128 levels), so k runs over the
+boundaries of those shapes. Each case sets
 N, S and c, runs one revival check through the C ABI and compares with the
 oracle's revival (split arm: sequential size-proportional donor draws):
 
@@ -67,8 +68,8 @@ def _model_at_step_one(em, k, d):
 
 
 CASES = [(k, "random") for k in (1, 2, 31, 33, 127, 128, 129, 1024, 1025, 2048, 2049, 4096, 4097, 8192,
-                                 8193, 16383, 16384, 16385, 20000, 65536, 300000)]
-CASES += [(4096, "one_live"), (300, "one_live"), (8000, "one_live"), (16000, "one_live")]
+                                 8193, 16383, 16384, 16385, 20000, 65536, 131073, 300000, 600000, 1100000)]
+CASES += [(4096, "one_live"), (300, "one_live"), (8000, "one_live"), (16000, "one_live"), (70000, "one_live")]
 CASES += [(16384, "heavy_few"), (8193, "heavy_few"), (2000, "heavy_few"), (65536, "heavy_few")]
 
 
