@@ -14,9 +14,11 @@ oracle's revival (split arm: sequential size-proportional donor draws):
 * the centroids of every cluster the check touched (per-centroid relative L2);
 * the number of dead clusters and of splits.
 
-Patterns: random counts with a dead fraction; one live cluster serving every
-dead one (its weight halves at each draw until it runs out, so the later dead
-clusters stay unrevived); a few heavy clusters among many light ones.
+Patterns: random counts with a dead fraction (300 dead clusters at the largest
+k, where the oracle recomputes a million-entry cumulative sum per draw); one live
+cluster serving every dead one (its weight halves at each draw until it runs out,
+so the later dead clusters stay unrevived); a few heavy clusters among many light
+ones.
 """
 
 import numpy as np
@@ -48,6 +50,10 @@ def _counts(pattern, k, rng):
     elif pattern == "one_live":
         N = np.zeros(k)
         N[rng.integers(k)] = 1000.0
+    elif pattern == "few_dead":  # (300 dead clusters: keeps the oracle's sequential draws short at large k)
+        N = rng.uniform(20.0, 200.0, size=k)
+        dead = rng.choice(k, size=min(k, 300), replace=False)
+        N[dead] = rng.uniform(0.0, 1.0, size=len(dead))
     elif pattern == "heavy_few":
         N = rng.uniform(0.0, 0.5, size=k)
         heavy = rng.choice(k, size=max(1, k // 50), replace=False)
@@ -68,7 +74,8 @@ def _model_at_step_one(em, k, d):
 
 
 CASES = [(k, "random") for k in (1, 2, 31, 33, 127, 128, 129, 1024, 1025, 2048, 2049, 4096, 4097, 8192,
-                                 8193, 16383, 16384, 16385, 20000, 65536, 131073, 300000, 600000, 1100000)]
+                                 8193, 16383, 16384, 16385, 20000, 65536, 131073, 300000)]
+CASES += [(600000, "few_dead"), (1100000, "few_dead")]
 CASES += [(4096, "one_live"), (300, "one_live"), (8000, "one_live"), (16000, "one_live"), (70000, "one_live")]
 CASES += [(16384, "heavy_few"), (8193, "heavy_few"), (2000, "heavy_few"), (65536, "heavy_few")]
 
