@@ -792,24 +792,24 @@ __global__ void __launch_bounds__(threads_for<epi_groups<TOP2, AST>()>(), 1)
 __global__ void k_fold_norms(const float* __restrict__ cn, int k, int k_pad, __nv_bfloat16* __restrict__ cn3) {
     pdl_wait();
     pdl_release();
-    const int j = blockIdx.x * blockDim.x + threadIdx.x;
-    if (j >= k_pad) return;
-    const float c = j < k ? cn[j] : __int_as_float(0x7f800000);
-    const __nv_bfloat16 h = __float2bfloat16_rn(c);
-    __nv_bfloat16 mid = __float2bfloat16_rn(0.0f), lo = mid;
-    if (isfinite(c)) {
-        const float r1 = c - __bfloat162float(h);
-        mid = __float2bfloat16_rn(r1);
-        lo = __float2bfloat16_rn(r1 - __bfloat162float(mid));
+    for (int j = blockIdx.x * blockDim.x + threadIdx.x; j < k_pad; j += gridDim.x * blockDim.x) {
+        const float c = j < k ? cn[j] : __int_as_float(0x7f800000);
+        const __nv_bfloat16 h = __float2bfloat16_rn(c);
+        __nv_bfloat16 mid = __float2bfloat16_rn(0.0f), lo = mid;
+        if (isfinite(c)) {
+            const float r1 = c - __bfloat162float(h);
+            mid = __float2bfloat16_rn(r1);
+            lo = __float2bfloat16_rn(r1 - __bfloat162float(mid));
+        }
+        uint4 v0;
+        v0.x = (uint32_t)__bfloat16_as_ushort(h) | ((uint32_t)__bfloat16_as_ushort(mid) << 16);
+        v0.y = (uint32_t)__bfloat16_as_ushort(lo);
+        v0.z = 0u;
+        v0.w = 0u;
+        uint4* row = reinterpret_cast<uint4*>(cn3 + (int64_t)j * kExtK);
+        row[0] = v0;
+        row[1] = make_uint4(0u, 0u, 0u, 0u);
     }
-    uint4 v0;
-    v0.x = (uint32_t)__bfloat16_as_ushort(h) | ((uint32_t)__bfloat16_as_ushort(mid) << 16);
-    v0.y = (uint32_t)__bfloat16_as_ushort(lo);
-    v0.z = 0u;
-    v0.w = 0u;
-    uint4* row = reinterpret_cast<uint4*>(cn3 + (int64_t)j * kExtK);
-    row[0] = v0;
-    row[1] = make_uint4(0u, 0u, 0u, 0u);
 }
 
 }  // namespace tc
