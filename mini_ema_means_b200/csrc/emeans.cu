@@ -6,6 +6,7 @@
 //   k_gather        batch rows pi_pass(pos..pos+B) -> contiguous bf16 batch, |x|^2
 //                   (and E4M3 codes with the FP8 search); prefetched: the next
 //                   step's rows are gathered on a second stream beside the search
+//   k_fold_norms    (d < 128 with many tiles) the norms operand the search folds in
 //   k_assign_tc     nearest centroid of every batch row (tcgen05 + TMA)
 //   k_labels        labels, distances, per-cluster counts and ranks
 //   k_settle        near ties re-decided in fp64
