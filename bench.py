@@ -314,7 +314,8 @@ def run_ours(args, rank, world):
         "traffic": (args.traffic if args.traffic is not None
                     else ASSIGN_TRAFFIC.get(args.workload) if args.search == "bf16" else None),
         "kernel": ("k_assign_tc (tcgen05 e4m3 x e4m3 -> fp32, fused |c'|^2/2 add + row argmin)" if args.search == "fp8"
-                   else "k_assign_tc (tcgen05 bf16 x bf16 -> fp32, fused |c|^2 add + row argmin)"),
+                   else "k_assign_tc (tcgen05 bf16 x bf16 -> fp32, fused |c|^2 (added, or folded into the MMAs "
+                        "at d < 128) + row argmin)"),
         "peak_source": (f"{peaks['source']} bf16 burst x 2 (nominal e4m3 / bf16 ratio)" if args.search == "fp8"
                         else f"{peaks['source']} bf16 burst"),
         "frac_of_sustained": (achieved / (peaks["bf16_tflops_sustained"] * ratio)
@@ -586,10 +587,11 @@ def run_ablation(args):
 
 L2_BYTES = 126e6  # the B200's L2 (126 MB)
 
-# DRAM bytes per assignment launch of the bench's batch, from an ncu capture of the
-# current kernel (262,144 rows, scaled to one 65,536-row batch with the centroid
-# operand counted once).
-ASSIGN_TRAFFIC = {"emb768": 109.6e6}
+# DRAM bytes per assignment launch of the bench's batch, from ncu captures of the
+# current kernel (emb768: 262,144 rows; deep96: 1,048,576 rows, 205.8 MB read and
+# 24.4 MB written), scaled to one 65,536-row batch by rows for the batch and the
+# keys, with the centroid operand counted once.
+ASSIGN_TRAFFIC = {"emb768": 109.6e6, "deep96": 18.6e6}
 
 
 def main():
